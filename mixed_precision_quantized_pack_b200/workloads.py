@@ -1,0 +1,173 @@
+"""Workload shapes and seeded synthetic inputs for packed KV-cache decode attention.
+
+This module only draws random numbers; it holds none of the method's arithmetic
+(no quantization, packing, retention or attention).  Both the CUDA path and the
+CPU oracle are fed from here, so that they see the very same fp16 tensors.
+
+Distributions (the workloads of "Quantize What Counts: More for Keys, Less for
+Values", §Méthodologie, are real model caches we do not have; these synthetic
+stand-ins keep the property the pages stress: keys carry per-channel outliers,
+values do not):
+
+* keys   k[b,h,t,c] = N(0,1) * sigma[h,c] + mu[h,c], with sigma log-uniform on
+  [0.5, 8] and mu ~ N(0, variance 2), both drawn per (kv head, channel) and
+  shared by every sequence and token;
+* values and queries ~ N(0, 1);
+* thin keys ("Thin Keys, Full Values", §2): 128-dim keys drawn as above and
+  projected to d_k dims by P with N(0, std 1/sqrt(128)) entries, in fp32.
+
+Everything is drawn in fp32 from one ``torch.Generator`` seeded per workload and
+rounded once to fp16.  The generator lives on the device the tensors are made on,
+so a CPU and a CUDA draw of the same seed differ; each test or benchmark uses
+one of them and copies across as needed.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    d_k: int
+    d_v: int
+    context: int          # tokens written by the prefill
+    k_bits: int
+    v_bits: int
+    group_k: int          # tokens per key group
+    group_v: int          # channels per value group
+    window: int           # R, the fp16 recent window
+    log_retain: int
+    appends: int          # append+decode steps after the prefill (0: one decode only)
+    thin_from: int = 0    # >0: keys are a projection of thin_from-dim keys
+    seed: int = 0
+
+    @property
+    def n_rep(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    @property
+    def max_context(self) -> int:
+        return self.context + max(self.appends, 1) + 64
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+    def kvq_config(self, max_context: Optional[int] = None) -> dict:
+        return dict(batch=self.batch, n_q_heads=self.n_q_heads, n_kv_heads=self.n_kv_heads,
+                    d_k=self.d_k, d_v=self.d_v, k_bits=self.k_bits, v_bits=self.v_bits,
+                    group_k=self.group_k, group_v=self.group_v, window=self.window,
+                    log_retain=self.log_retain,
+                    max_context=max_context if max_context is not None else self.max_context)
+
+
+def _base(**kw) -> Workload:
+    return Workload(**kw)
+
+
+# The five workloads named with the metric.  Shapes, bit widths, group sizes and
+# windows as stated there; seeds are 1000 + index.
+WORKLOADS: Dict[str, Workload] = {
+    "tiny": _base(name="tiny-1h-512", batch=1, n_q_heads=1, n_kv_heads=1, d_k=128, d_v=128,
+                  context=512, k_bits=4, v_bits=2, group_k=32, group_v=32, window=64,
+                  log_retain=0, appends=0, seed=1000),
+    "gqa4k": _base(name="gqa-b8-32/8-4k-k4v2", batch=8, n_q_heads=32, n_kv_heads=8, d_k=128,
+                   d_v=128, context=4096, k_bits=4, v_bits=2, group_k=64, group_v=64,
+                   window=128, log_retain=0, appends=1, seed=1001),
+    "long32k": _base(name="long-b32-32/8-32k-k4v2-logretain", batch=32, n_q_heads=32,
+                     n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=4, v_bits=2,
+                     group_k=64, group_v=64, window=128, log_retain=1, appends=0, seed=1002),
+    "thin16k": _base(name="thin-b16-32/8-dk32-dv128-16k-k4v2", batch=16, n_q_heads=32,
+                     n_kv_heads=8, d_k=32, d_v=128, context=16384, k_bits=4, v_bits=2,
+                     group_k=32, group_v=32, window=64, log_retain=0, appends=0,
+                     thin_from=128, seed=1003),
+}
+
+SWEEP_BATCHES = (1, 8, 32, 64)
+SWEEP_BITS = ((8, 4), (4, 2), (2, 2), (16, 16))
+
+
+def sweep_workload(batch: int, k_bits: int, v_bits: int, appends: int = 256) -> Workload:
+    """Context-131072 sweep point: 32/8 heads, d=128, group 64, window 128."""
+    return _base(name=f"sweep-b{batch}-k{k_bits}v{v_bits}-128k", batch=batch, n_q_heads=32,
+                 n_kv_heads=8, d_k=128, d_v=128, context=131072, k_bits=k_bits, v_bits=v_bits,
+                 group_k=64, group_v=64, window=128, log_retain=0, appends=appends,
+                 seed=1004)
+
+
+def _keys(gen: torch.Generator, device, batch: int, heads: int, tokens: int, d: int,
+          sigma: torch.Tensor, mu: torch.Tensor) -> torch.Tensor:
+    x = torch.randn((batch, heads, tokens, d), generator=gen, device=device, dtype=torch.float32)
+    return x * sigma[None, :, None, :] + mu[None, :, None, :]
+
+
+def key_stats(gen: torch.Generator, device, heads: int, d: int):
+    """Per (kv head, channel) outlier scale (log-uniform [0.5, 8]) and mean (N(0, 2))."""
+    u = torch.rand((heads, d), generator=gen, device=device, dtype=torch.float32)
+    sigma = torch.exp(math.log(0.5) + u * (math.log(8.0) - math.log(0.5)))
+    mu = torch.randn((heads, d), generator=gen, device=device, dtype=torch.float32) * math.sqrt(2.0)
+    return sigma, mu
+
+
+class Inputs:
+    """Seeded fp16 tensors for one workload.
+
+    ``k``, ``v``: [B][Hkv][context][d]; ``q``: list of [B][Hq][d_k] (one per decode
+    step); ``k_app``/``v_app``: list of [B][Hkv][d] (one per append step).
+    """
+
+    def __init__(self, w: Workload, device="cpu", batch_slice: Optional[slice] = None):
+        self.w = w
+        dev = torch.device(device)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(w.seed)
+        d_src = w.thin_from if w.thin_from else w.d_k
+        sigma, mu = key_stats(gen, dev, w.n_kv_heads, d_src)
+        proj = None
+        if w.thin_from:
+            proj = torch.randn((w.thin_from, w.d_k), generator=gen, device=dev,
+                               dtype=torch.float32) / math.sqrt(w.thin_from)
+        self.sigma, self.mu, self.proj = sigma, mu, proj
+
+        def keys(batch, tokens):
+            k = _keys(gen, dev, batch, w.n_kv_heads, tokens, d_src, sigma, mu)
+            if proj is not None:
+                k = k @ proj
+            return k.to(torch.float16)
+
+        def normal(shape):
+            return torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.float16)
+
+        B = w.batch
+        self.k = keys(B, w.context)
+        self.v = normal((B, w.n_kv_heads, w.context, w.d_v))
+        n_dec = max(w.appends, 1)
+        self.q: List[torch.Tensor] = []
+        self.k_app: List[torch.Tensor] = []
+        self.v_app: List[torch.Tensor] = []
+        for _ in range(n_dec):
+            self.q.append(normal((B, w.n_q_heads, w.d_k)))
+            if w.appends:
+                self.k_app.append(keys(B, 1)[:, :, 0, :].contiguous())
+                self.v_app.append(normal((B, w.n_kv_heads, w.d_v)))
+        if batch_slice is not None:
+            self.k = self.k[batch_slice].contiguous()
+            self.v = self.v[batch_slice].contiguous()
+            self.q = [x[batch_slice].contiguous() for x in self.q]
+            self.k_app = [x[batch_slice].contiguous() for x in self.k_app]
+            self.v_app = [x[batch_slice].contiguous() for x in self.v_app]
+
+
+def random_fp16(shape, seed: int, device="cpu", scale: float = 1.0, mean: float = 0.0) -> torch.Tensor:
+    """Plain N(mean, scale^2) fp16 tensor from its own seeded generator (small test cases)."""
+    gen = torch.Generator(device=torch.device(device))
+    gen.manual_seed(seed)
+    x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * scale + mean
+    return x.to(torch.float16)

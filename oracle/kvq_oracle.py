@@ -1,0 +1,325 @@
+"""CPU oracle for decode attention over a packed mixed-precision KV cache.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product imports this module: only the
+tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline / reference arm
+may call it.  It shares no code with the CUDA library; both sides are fed the
+same fp16 tensors by ``mixed_precision_quantized_pack_b200.workloads``.
+
+What it computes, step by step in the order the pages give it:
+
+1. Regions.  A full-precision recent window stays fp16 ("LogQuant: Log-Distributed
+   2-Bit Quantization of KV Cache", §Comment LogQuant Fonctionne / §Méthodologie 2);
+   everything older is quantized, never evicted (same page, §Méthodologie 3).
+   Reading: key groups need whole groups of G_k tokens, so the quantized prefix is
+   Q = floor(max(L-R, 0) / G_k) * G_k and the window [Q, L) holds R..R+G_k-1
+   tokens.  Bit width 16 means "not quantized": Q = 0.
+2. Keys are quantized per channel over groups of G_k tokens (LogQuant, §5
+   "par canal par Clé"; group sizes from "Quantize What Counts", §Sensibilité à
+   la Taille de Groupe), with more bits than values (K4V2 by default; same page,
+   §La Solution).  Values are quantized per token over groups of G_v channels.
+3. The quantizer is asymmetric uniform min-max with an fp16 scale and zero per
+   group (reading: the pages name Quanto/HQQ but print no formula):
+       s16 = fp16(fl32(mx - mn) / fl32(2^b - 1)),  s16 == 0 -> +0
+       z16 = fp16(mn)  (exact; -0 -> +0)
+       code = 0 if s16 == 0 else clamp(rint(fl32(fl32(x - z16) / s16)), 0, 2^b-1)
+   All arithmetic is IEEE binary32 with round-to-nearest-even, one operation at
+   a time (numpy float32 ufuncs), rint is half-to-even.
+4. Packing: within a token row, codes are packed channel by channel, least
+   significant bits first, into little-endian uint32 words (channel c of a b-bit
+   row lives in word c // (32/b) at bit (c % (32/b)) * b).  (scale, zero) pairs
+   are stored as fp16 pairs.
+5. Log-spaced retention (LogQuant §Méthodologie 2, "density halves further
+   back"; the printed text is garbled).  Reading: among the quantized positions
+   p < Q, p is kept in fp16 iff p is a multiple of 2^floor(log2(Q - p)); this
+   keeps exactly one token per age octave [2^l, 2^(l+1)), floor(log2 Q)+1 tokens
+   in all, and as Q grows a token can only leave the set.
+6. Attention (fp64) over every token: fp16 values for window and retained
+   tokens, code*s16 + z16 otherwise; scores q.k/sqrt(d_k) ("Thin Keys, Full
+   Values", §2, where d_k may be smaller than d_v; the score form of "HeadQ",
+   §2.1), softmax with max subtraction, p.V.  Token order is irrelevant
+   (LogQuant §4, A.V = A_P.V_P).  GQA: query head hq reads kv head hq // n_rep.
+
+Buffer formats mirror the CUDA library's so the tests can compare bytes:
+  kcode u32 [B][Hkv][Lcap][d_k*kb/32]        ksz fp16 [B][Hkv][Lcap/Gk][d_k][2]
+  vcode u32 [B][Hkv][Lcap][d_v*vb/32]        vsz fp16 [B][Hkv][Lcap][d_v/Gv][2]
+  win_k/v fp16 [B][Hkv][C][d] with token p in slot p % C,
+          C = R + G_k (quantized caches) or Lcap (bits 16)
+  ret_k/v fp16 [B][Hkv][32][d] in ascending position order, ret_idx int32 list.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional
+
+import numpy as np
+
+MAX_RETAINED = 32
+
+
+# ---------------------------------------------------------------- regions -----
+def quantized_prefix(L: int, window: int, group_k: int, k_bits: int) -> int:
+    """Q: number of leading tokens held quantized (step 1 above)."""
+    if k_bits == 16:
+        return 0
+    return max(L - window, 0) // group_k * group_k
+
+
+def retained_positions(Q: int) -> List[int]:
+    """Ascending list {p < Q : p mod 2^floor(log2(Q-p)) == 0} (step 5 above)."""
+    if Q <= 0:
+        return []
+    p = np.arange(Q, dtype=np.int64)
+    age = (Q - p).astype(np.float64)
+    _, e = np.frexp(age)                 # age = m * 2^e, m in [0.5, 1): floor(log2 age) = e-1
+    octave = (e - 1).astype(np.int64)
+    keep = (p % (np.int64(1) << octave)) == 0
+    return [int(x) for x in p[keep]]
+
+
+# -------------------------------------------------------------- quantizer -----
+def minmax_quantize(x: np.ndarray, bits: int, axis: int):
+    """Asymmetric min-max quantizer of step 3 over groups laid along ``axis``.
+
+    ``x`` holds fp16 values (any float dtype holding them exactly).  Returns
+    (codes uint32 with x's shape, s16 fp16, z16 fp16) where s16/z16 keep a
+    length-1 ``axis``.
+    """
+    x32 = np.asarray(x, dtype=np.float16).astype(np.float32)
+    mn = x32.min(axis=axis, keepdims=True)
+    mx = x32.max(axis=axis, keepdims=True)
+    levels = np.float32(2 ** bits - 1)
+    s32 = (mx - mn) / levels
+    s16 = s32.astype(np.float16)
+    s16 = np.where(s16 == 0, np.float16(0.0), s16).astype(np.float16)   # canonical +0
+    z16 = (mn + np.float32(0.0)).astype(np.float16)                     # exact, -0 -> +0
+    sf = s16.astype(np.float32)
+    zf = z16.astype(np.float32)
+    diff = x32 - zf
+    with np.errstate(divide="ignore", invalid="ignore"):
+        quot = diff / sf
+    code = np.rint(quot)
+    code = np.where(sf == 0, np.float32(0.0), code)
+    code = np.clip(code, 0, levels)
+    return code.astype(np.uint32), s16, z16
+
+
+def dequantize(codes: np.ndarray, s16: np.ndarray, z16: np.ndarray) -> np.ndarray:
+    """code * s + z, exactly, in fp64."""
+    return codes.astype(np.float64) * s16.astype(np.float64) + z16.astype(np.float64)
+
+
+def quantize_keys(k: np.ndarray, group_k: int, bits: int):
+    """Keys [n][d] with n a multiple of group_k -> codes [n][d], sz fp16 [n/group_k][d][2].
+
+    One (scale, zero) per channel per group of group_k consecutive tokens.
+    """
+    n, d = k.shape
+    assert n % group_k == 0
+    g = k.reshape(n // group_k, group_k, d)
+    codes, s, z = minmax_quantize(g, bits, axis=1)          # s, z: [ng][1][d]
+    sz = np.stack([s[:, 0, :], z[:, 0, :]], axis=-1)
+    return codes.reshape(n, d), sz
+
+
+def quantize_values(v: np.ndarray, group_v: int, bits: int):
+    """Values [n][d] -> codes [n][d], sz fp16 [n][d/group_v][2] (groups of channels per token)."""
+    n, d = v.shape
+    assert d % group_v == 0
+    g = v.reshape(n, d // group_v, group_v)
+    codes, s, z = minmax_quantize(g, bits, axis=2)          # s, z: [n][ng][1]
+    sz = np.stack([s[:, :, 0], z[:, :, 0]], axis=-1)
+    return codes.reshape(n, d), sz
+
+
+# ---------------------------------------------------------------- packing -----
+def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
+    """[..., d] codes -> [..., d*bits/32] uint32 words, channels LSB-first (step 4)."""
+    per = 32 // bits
+    d = codes.shape[-1]
+    assert d % per == 0
+    c = codes.astype(np.uint64).reshape(codes.shape[:-1] + (d // per, per))
+    shifts = (np.arange(per, dtype=np.uint64) * np.uint64(bits))
+    words = (c << shifts).sum(axis=-1)
+    return words.astype(np.uint32)
+
+
+def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
+    per = 32 // bits
+    w = words.astype(np.uint64)[..., None]
+    shifts = (np.arange(per, dtype=np.uint64) * np.uint64(bits))
+    mask = np.uint64((1 << bits) - 1)
+    c = (w >> shifts) & mask
+    return c.reshape(words.shape[:-1] + (words.shape[-1] * per,)).astype(np.uint32)
+
+
+# -------------------------------------------------------------- attention -----
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
+    """softmax(q.K^T * scale) V in fp64 for one query vector."""
+    q = np.asarray(q, dtype=np.float64)
+    s = (np.asarray(k, dtype=np.float64) @ q) * scale
+    p = np.exp(s - s.max())
+    return (p @ np.asarray(v, dtype=np.float64)) / p.sum()
+
+
+def buffer_bytes(cfg: dict) -> dict:
+    """Bytes of each cache buffer, as laid out above."""
+    B, H, dk, dv = cfg["batch"], cfg["n_kv_heads"], cfg["d_k"], cfg["d_v"]
+    kb, vb, gk, gv, R = cfg["k_bits"], cfg["v_bits"], cfg["group_k"], cfg["group_v"], cfg["window"]
+    if kb == 16:
+        lcap = cfg["max_context"]
+        cap = lcap
+        return dict(kcode=0, ksz=0, vcode=0, vsz=0, win_k=B * H * cap * dk * 2,
+                    win_v=B * H * cap * dv * 2, ret_k=0, ret_v=0)
+    lcap = -(-cfg["max_context"] // gk) * gk
+    cap = R + gk
+    return dict(kcode=B * H * lcap * dk * kb // 8, ksz=B * H * (lcap // gk) * dk * 4,
+                vcode=B * H * lcap * dv * vb // 8, vsz=B * H * lcap * (dv // gv) * 4,
+                win_k=B * H * cap * dk * 2, win_v=B * H * cap * dv * 2,
+                ret_k=B * H * MAX_RETAINED * dk * 2, ret_v=B * H * MAX_RETAINED * dv * 2)
+
+
+# ------------------------------------------------------------------ cache -----
+class OracleCache:
+    """The whole cache of one layer: prefill, append, decode (see module docstring)."""
+
+    def __init__(self, cfg: dict):
+        self.cfg = dict(cfg)
+        B, H = cfg["batch"], cfg["n_kv_heads"]
+        self.B, self.H, self.Hq = B, H, cfg["n_q_heads"]
+        self.dk, self.dv = cfg["d_k"], cfg["d_v"]
+        self.kb, self.vb = cfg["k_bits"], cfg["v_bits"]
+        self.gk, self.gv, self.R = cfg["group_k"], cfg["group_v"], cfg["window"]
+        self.log_retain = bool(cfg["log_retain"]) and self.kb != 16
+        self.max_context = cfg["max_context"]
+        if self.kb == 16:
+            self.lcap = self.max_context
+            self.cap = self.lcap
+        else:
+            self.lcap = -(-self.max_context // self.gk) * self.gk
+            self.cap = self.R + self.gk
+            self.kcode = np.zeros((B, H, self.lcap, self.dk * self.kb // 32), np.uint32)
+            self.ksz = np.zeros((B, H, self.lcap // self.gk, self.dk, 2), np.float16)
+            self.vcode = np.zeros((B, H, self.lcap, self.dv * self.vb // 32), np.uint32)
+            self.vsz = np.zeros((B, H, self.lcap, self.dv // self.gv, 2), np.float16)
+            self.ret_k = np.zeros((B, H, MAX_RETAINED, self.dk), np.float16)
+            self.ret_v = np.zeros((B, H, MAX_RETAINED, self.dv), np.float16)
+        self.win_k = np.zeros((B, H, self.cap, self.dk), np.float16)
+        self.win_v = np.zeros((B, H, self.cap, self.dv), np.float16)
+        self.ret_idx: List[int] = []
+        self.L = 0
+        self.Q = 0
+
+    # -- write path -----------------------------------------------------------
+    def _quantize_rows(self, b: int, h: int, t0: int, k_rows: np.ndarray, v_rows: np.ndarray):
+        """Quantize tokens [t0, t0+n) (n a multiple of G_k) and store their codes."""
+        n = k_rows.shape[0]
+        kc, ksz = quantize_keys(k_rows, self.gk, self.kb)
+        vc, vsz = quantize_values(v_rows, self.gv, self.vb)
+        self.kcode[b, h, t0:t0 + n] = pack_codes(kc, self.kb)
+        self.ksz[b, h, t0 // self.gk:(t0 + n) // self.gk] = ksz
+        self.vcode[b, h, t0:t0 + n] = pack_codes(vc, self.vb)
+        self.vsz[b, h, t0:t0 + n] = vsz
+
+    def prefill(self, k: np.ndarray, v: np.ndarray):
+        """k [B][Hkv][L][d_k], v [B][Hkv][L][d_v] fp16: the cache's first L tokens."""
+        k = np.asarray(k, np.float16)
+        v = np.asarray(v, np.float16)
+        L = k.shape[2]
+        if L > self.max_context:
+            raise ValueError("context exceeds max_context")
+        Q = quantized_prefix(L, self.R, self.gk, self.kb)
+        for b in range(self.B):
+            for h in range(self.H):
+                if Q:
+                    self._quantize_rows(b, h, 0, k[b, h, :Q], v[b, h, :Q])
+                for p in range(Q, L):
+                    self.win_k[b, h, p % self.cap] = k[b, h, p]
+                    self.win_v[b, h, p % self.cap] = v[b, h, p]
+        self.ret_idx = retained_positions(Q) if self.log_retain else []
+        for j, p in enumerate(self.ret_idx):
+            self.ret_k[:, :, j] = k[:, :, p]
+            self.ret_v[:, :, j] = v[:, :, p]
+        self.L, self.Q = L, Q
+
+    def append(self, k_new: np.ndarray, v_new: np.ndarray):
+        """One token per sequence: k_new [B][Hkv][d_k], v_new [B][Hkv][d_v]."""
+        if self.L + 1 > self.max_context:
+            raise ValueError("append past max_context")
+        p = self.L
+        self.win_k[:, :, p % self.cap] = np.asarray(k_new, np.float16)
+        self.win_v[:, :, p % self.cap] = np.asarray(v_new, np.float16)
+        self.L += 1
+        if self.kb != 16 and self.L - self.Q == self.R + self.gk:
+            Q0, Q1 = self.Q, self.Q + self.gk
+            slots = [t % self.cap for t in range(Q0, Q1)]
+            for b in range(self.B):
+                for h in range(self.H):
+                    self._quantize_rows(b, h, Q0, self.win_k[b, h, slots], self.win_v[b, h, slots])
+            if self.log_retain:
+                new = retained_positions(Q1)
+                old = {pos: j for j, pos in enumerate(self.ret_idx)}
+                rk = np.zeros_like(self.ret_k)
+                rv = np.zeros_like(self.ret_v)
+                for j, pos in enumerate(new):
+                    if pos in old:
+                        rk[:, :, j] = self.ret_k[:, :, old[pos]]
+                        rv[:, :, j] = self.ret_v[:, :, old[pos]]
+                    else:                      # a token of the group being quantized now
+                        assert Q0 <= pos < Q1
+                        rk[:, :, j] = self.win_k[:, :, pos % self.cap]
+                        rv[:, :, j] = self.win_v[:, :, pos % self.cap]
+                n = len(new)
+                self.ret_k[:, :, :n] = rk[:, :, :n]
+                self.ret_v[:, :, :n] = rv[:, :, :n]
+                self.ret_idx = new
+            self.Q = Q1
+
+    # -- read path ------------------------------------------------------------
+    def decoded_kv(self, b: int, h: int):
+        """(K_hat [L][d_k], V_hat [L][d_v]) in fp64, positions 0..L-1 in order."""
+        L, Q = self.L, self.Q
+        kh = np.empty((L, self.dk), np.float64)
+        vh = np.empty((L, self.dv), np.float64)
+        if Q:
+            kc = unpack_codes(self.kcode[b, h, :Q], self.kb)                   # [Q][dk]
+            ksz = self.ksz[b, h, :Q // self.gk]                                 # [ng][dk][2]
+            ks = np.repeat(ksz[:, :, 0], self.gk, axis=0)
+            kz = np.repeat(ksz[:, :, 1], self.gk, axis=0)
+            kh[:Q] = dequantize(kc, ks, kz)
+            vc = unpack_codes(self.vcode[b, h, :Q], self.vb)                   # [Q][dv]
+            vsz = self.vsz[b, h, :Q]                                            # [Q][ngv][2]
+            vs = np.repeat(vsz[:, :, 0], self.gv, axis=1)
+            vz = np.repeat(vsz[:, :, 1], self.gv, axis=1)
+            vh[:Q] = dequantize(vc, vs, vz)
+            for j, pos in enumerate(self.ret_idx):
+                kh[pos] = self.ret_k[b, h, j]
+                vh[pos] = self.ret_v[b, h, j]
+        slots = [p % self.cap for p in range(Q, L)]
+        kh[Q:] = self.win_k[b, h, slots]
+        vh[Q:] = self.win_v[b, h, slots]
+        return kh, vh
+
+    def decode(self, q: np.ndarray, rows: Optional[List[int]] = None) -> np.ndarray:
+        """q [B][Hq][d_k] fp16 -> out [B][Hq][d_v] fp64 (rows: optional subset of b)."""
+        if self.L == 0:
+            raise ValueError("decode before prefill")
+        q = np.asarray(q, np.float16).astype(np.float64)
+        n_rep = self.Hq // self.H
+        out = np.full((self.B, self.Hq, self.dv), np.nan)
+        scale = 1.0 / math.sqrt(self.dk)
+        for b in (rows if rows is not None else range(self.B)):
+            for h in range(self.H):
+                kh, vh = self.decoded_kv(b, h)
+                for r in range(n_rep):
+                    hq = h * n_rep + r
+                    out[b, hq] = attention(q[b, hq], kh, vh, scale)
+        return out
+
+
+def max_rel_error(out: np.ndarray, ref: np.ndarray) -> float:
+    """max over rows of max_c |out - ref| / max_c |ref| (rows = all leading dims)."""
+    o = np.asarray(out, np.float64).reshape(-1, out.shape[-1])
+    r = np.asarray(ref, np.float64).reshape(-1, ref.shape[-1])
+    num = np.abs(o - r).max(axis=1)
+    den = np.maximum(np.abs(r).max(axis=1), 1e-30)
+    return float((num / den).max())

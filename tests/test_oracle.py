@@ -1,0 +1,378 @@
+"""Pins of the CPU oracle against facts fixed by the pages and by mathematics.
+
+Each test checks the oracle against something other than itself: hand-derived
+worked examples (tests/golden), closed forms (exact grids), library routines
+(torch's scaled_dot_product_attention in fp64), invariants the pages state
+(softmax invariance to a shared key translation: "HeadQ", §2.1; token-order
+invariance A.V = A_P.V_P: "LogQuant", §4), brute force on tiny inputs, and byte
+arithmetic ("Quantize What Counts", §Résultats: K4V2 saves 25% over K4V4).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from conftest import read_golden
+from oracle import kvq_oracle as O
+from mixed_precision_quantized_pack_b200 import workloads as W
+
+
+def f16bits(x):
+    return int(np.asarray(x, np.float16).view(np.uint16))
+
+
+# ------------------------------------------------------------ golden files ----
+def test_golden_quantizer_examples():
+    rows = read_golden("quantizer_worked.txt")
+    assert len(rows) >= 6
+    for bits, vals, codes, sbits, zbits in rows:
+        x = np.array([float(v) for v in vals], np.float16)
+        c, s, z = O.minmax_quantize(x, int(bits[0]), axis=0)
+        assert [int(t) for t in c] == [int(t) for t in codes], (vals, c)
+        assert f16bits(s[0]) == int(sbits[0], 16)
+        assert f16bits(z[0]) == int(zbits[0], 16)
+
+
+def test_golden_packing_examples():
+    for bits, codes, words in read_golden("packing_worked.txt"):
+        b = int(bits[0])
+        c = np.array([[int(t) for t in codes]], np.uint32)
+        w = O.pack_codes(c, b)
+        assert [int(t) for t in w[0]] == [int(t, 16) for t in words]
+        assert np.array_equal(O.unpack_codes(w, b), c)
+
+
+def test_golden_retention_examples():
+    for q, pos in read_golden("retention_worked.txt"):
+        assert O.retained_positions(int(q[0])) == [int(p) for p in pos]
+
+
+# --------------------------------------------------------------- quantizer ----
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_grid_inputs_give_exact_codes(bits):
+    rng = np.random.default_rng(bits)
+    for trial in range(50):
+        e = int(rng.integers(-8, 0))
+        step = 2.0 ** e
+        levels = 2 ** bits - 1
+        n = int(rng.integers(2, 70))
+        k = rng.integers(0, levels + 1, size=n)
+        k[rng.integers(0, n)] = 0
+        k[(rng.integers(0, n - 1) + 1 + np.argmin(k)) % n] = levels
+        if k.min() != 0 or k.max() != levels:
+            continue
+        z = float(rng.integers(-64, 64)) * step
+        x = np.array([z + int(t) * step for t in k], np.float64)
+        assert np.array_equal(x.astype(np.float16).astype(np.float64), x)   # exact in fp16
+        c, s, zz = O.minmax_quantize(x.astype(np.float16), bits, axis=0)
+        assert np.array_equal(c, k.astype(np.uint32))
+        assert float(s[0]) == step and float(zz[0]) == z
+        assert int(c[np.argmin(x)]) == 0 and int(c[np.argmax(x)]) == levels
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_reconstruction_error_bound(bits):
+    # |x - (code*s + z)| <= s * (1/2 + 2^(b-22)): half a step, plus the fp32 rounding of
+    # (x - z) and of the quotient (each <= 2^-24 relative on a quotient <= 2^b).
+    x = W.random_fp16((400, 64), seed=7, scale=3.0, mean=1.0).numpy()
+    for axis in (0, 1):
+        c, s, z = O.minmax_quantize(x, bits, axis=axis)
+        deq = O.dequantize(c, s, z)
+        err = np.abs(x.astype(np.float64) - deq)
+        bound = s.astype(np.float64) * (0.5 + 2.0 ** (bits - 22))
+        assert np.all(err <= bound + 0.0)
+        assert np.all(c <= 2 ** bits - 1)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_codes_are_nearest_level_brute_force(bits):
+    x = W.random_fp16((200, 8), seed=11, scale=2.0).numpy()
+    c, s, z = O.minmax_quantize(x, bits, axis=1)
+    levels = np.arange(2 ** bits, dtype=np.float64)
+    for i in range(x.shape[0]):
+        si, zi = float(s[i, 0]), float(z[i, 0])
+        for j in range(x.shape[1]):
+            d = np.abs(float(x[i, j]) - (levels * si + zi))
+            best = np.sort(d)
+            if best[1] - best[0] < 1e-5 * si:       # a near tie: either answer is right
+                continue
+            assert int(c[i, j]) == int(np.argmin(d))
+
+
+def test_key_and_value_grouping_axes():
+    # keys: one (s, z) per channel per group of G_k tokens; values: per token per G_v channels
+    k = W.random_fp16((64, 16), seed=3, scale=2.0).numpy()
+    kc, ksz = O.quantize_keys(k, 32, 4)
+    assert ksz.shape == (2, 16, 2)
+    for g in range(2):
+        for ch in range(16):
+            col = k[32 * g:32 * g + 32, ch].astype(np.float32)
+            assert float(ksz[g, ch, 1]) == float(col.min())
+    v = W.random_fp16((5, 64), seed=4).numpy()
+    vc, vsz = O.quantize_values(v, 32, 2)
+    assert vsz.shape == (5, 2, 2)
+    for t in range(5):
+        for g in range(2):
+            assert float(vsz[t, g, 1]) == float(v[t, 32 * g:32 * g + 32].astype(np.float32).min())
+
+
+def test_pack_unpack_roundtrip():
+    rng = np.random.default_rng(5)
+    for bits in (2, 4, 8):
+        c = rng.integers(0, 2 ** bits, size=(7, 128)).astype(np.uint32)
+        assert np.array_equal(O.unpack_codes(O.pack_codes(c, bits), bits), c)
+
+
+# --------------------------------------------------------------- attention ----
+def sdpa_fp64(q, k, v):
+    """torch's attention in fp64; q [B][Hq][dk], k [B][Hkv][L][dk], v [B][Hkv][L][dv]."""
+    q = torch.as_tensor(np.asarray(q, np.float64))
+    k = torch.as_tensor(np.asarray(k, np.float64))
+    v = torch.as_tensor(np.asarray(v, np.float64))
+    rep = q.shape[1] // k.shape[1]
+    k = k.repeat_interleave(rep, dim=1)
+    v = v.repeat_interleave(rep, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(q[:, :, None, :], k, v)
+    return o[:, :, 0, :].numpy()
+
+
+def cfg_of(B, Hq, Hkv, dk, dv, kb, vb, gk, gv, R, log_retain, max_context):
+    return dict(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, d_k=dk, d_v=dv, k_bits=kb, v_bits=vb,
+                group_k=gk, group_v=gv, window=R, log_retain=log_retain, max_context=max_context)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (32, 128)])
+def test_unquantized_cache_matches_library_attention(dk, dv):
+    B, Hq, Hkv, L = 2, 4, 2, 200
+    k = W.random_fp16((B, Hkv, L, dk), seed=21, scale=2.0).numpy()
+    v = W.random_fp16((B, Hkv, L, dv), seed=22).numpy()
+    q = W.random_fp16((B, Hq, dk), seed=23).numpy()
+    c = O.OracleCache(cfg_of(B, Hq, Hkv, dk, dv, 16, 16, 64, 64, 128, 0, 256))
+    c.prefill(k, v)
+    assert c.Q == 0
+    ref = sdpa_fp64(q, k, v)
+    assert np.allclose(c.decode(q), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_whole_context_in_window_is_exact():
+    B, Hq, Hkv, d, L = 1, 4, 1, 64, 100
+    k = W.random_fp16((B, Hkv, L, d), seed=31, scale=3.0).numpy()
+    v = W.random_fp16((B, Hkv, L, d), seed=32).numpy()
+    q = W.random_fp16((B, Hq, d), seed=33).numpy()
+    c = O.OracleCache(cfg_of(B, Hq, Hkv, d, d, 4, 2, 32, 32, 128, 1, 512))
+    c.prefill(k, v)
+    assert c.Q == 0 and c.ret_idx == []
+    assert np.allclose(c.decode(q), sdpa_fp64(q, k, v), rtol=1e-12, atol=1e-12)
+
+
+def grid_cache_inputs(B, H, L, dk, dv, kb, vb, gk, gv, seed):
+    """fp16 K/V that the quantizer reproduces exactly: each key group-channel and each
+    value token-group lies on z + k*2^e with both end codes present."""
+    rng = np.random.default_rng(seed)
+
+    def grid(shape_groups, n, bits):
+        levels = 2 ** bits - 1
+        codes = rng.integers(0, levels + 1, size=shape_groups + (n,))
+        codes[..., 0] = 0
+        codes[..., 1] = levels
+        perm = np.argsort(rng.random(size=codes.shape), axis=-1)
+        codes = np.take_along_axis(codes, perm, axis=-1)
+        e = rng.integers(-6, -2, size=shape_groups + (1,)).astype(np.float64)
+        step = 2.0 ** e
+        z = rng.integers(-32, 32, size=shape_groups + (1,)) * step
+        return z + codes * step
+
+    ng = -(-L // gk)
+    kg = grid((B, H, ng, dk), gk, kb)                      # [B][H][ng][dk][gk]
+    k = kg.transpose(0, 1, 2, 4, 3).reshape(B, H, ng * gk, dk)[:, :, :L]
+    vg = grid((B, H, L, dv // gv), gv, vb)                  # [B][H][L][ngv][gv]
+    v = vg.reshape(B, H, L, dv)
+    assert np.array_equal(k.astype(np.float16).astype(np.float64), k)
+    assert np.array_equal(v.astype(np.float16).astype(np.float64), v)
+    return k.astype(np.float16), v.astype(np.float16)
+
+
+@pytest.mark.parametrize("kb,vb,gk,gv,dk,dv", [(4, 2, 32, 32, 64, 64), (8, 4, 16, 64, 32, 128),
+                                              (2, 2, 64, 16, 64, 32)])
+def test_lossless_grid_cache_decode_equals_exact_attention(kb, vb, gk, gv, dk, dv):
+    # On grid inputs quantization is lossless, so the decode over codes must equal the
+    # library's exact attention: pins dequantization, scale/zero indexing and packing.
+    B, Hq, Hkv, R = 2, 4, 2, 16
+    L = 6 * gk + R + 3
+    k, v = grid_cache_inputs(B, Hkv, L, dk, dv, kb, vb, gk, gv, seed=kb * 10 + vb)
+    q = W.random_fp16((B, Hq, dk), seed=41).numpy()
+    c = O.OracleCache(cfg_of(B, Hq, Hkv, dk, dv, kb, vb, gk, gv, R, 0, L + 8))
+    c.prefill(k, v)
+    assert c.Q == (L - R) // gk * gk and c.Q > 0
+    assert np.allclose(c.decode(q), sdpa_fp64(q, k, v), rtol=1e-11, atol=1e-12)
+
+
+def test_retained_tokens_are_read_in_fp16():
+    # Grid inputs except the retained positions, which are moved off-grid inside the
+    # group's range: the decode is exact only if those tokens come from the fp16 copy.
+    kb, vb, gk, gv, d, R = 4, 2, 32, 32, 64, 32
+    B, Hq, Hkv = 1, 2, 1
+    L = 10 * gk + R
+    k, v = grid_cache_inputs(B, Hkv, L, d, d, kb, vb, gk, gv, seed=5)
+    Q = O.quantized_prefix(L, R, gk, kb)
+    ret = O.retained_positions(Q)
+    kf = k.astype(np.float64)
+    vf = v.astype(np.float64)
+    rset = set(ret)
+    for p in ret:
+        g0 = p // gk * gk
+        lo = kf[0, 0, g0:g0 + gk].min(axis=0)
+        hi = kf[0, 0, g0:g0 + gk].max(axis=0)
+        kf[0, 0, p] = lo + (hi - lo) * 0.37 + 2.0 ** -9
+        vf[0, 0, p] = vf[0, 0, p] + 2.0 ** -9
+        # keep each channel's group extremes on tokens that are not retained
+        free = [t for t in range(g0, g0 + gk) if t not in rset]
+        kf[0, 0, free[0]] = lo
+        kf[0, 0, free[1]] = hi
+    k2, v2 = kf.astype(np.float16), vf.astype(np.float16)
+    q = W.random_fp16((B, Hq, d), seed=6, scale=2.0).numpy()
+    exact = sdpa_fp64(q, k2, v2)
+    with_ret = O.OracleCache(cfg_of(B, Hq, Hkv, d, d, kb, vb, gk, gv, R, 1, L + 8))
+    with_ret.prefill(k2, v2)
+    assert with_ret.ret_idx == ret
+    assert np.allclose(with_ret.decode(q), exact, rtol=1e-11, atol=1e-12)
+    without = O.OracleCache(cfg_of(B, Hq, Hkv, d, d, kb, vb, gk, gv, R, 0, L + 8))
+    without.prefill(k2, v2)
+    assert not np.allclose(without.decode(q), exact, rtol=1e-9, atol=1e-9)
+
+
+def test_shared_key_translation_is_softmax_null():
+    # "HeadQ", §2.1: adding one vector mu to every key adds q.mu to every score; softmax
+    # ignores it.  Per-channel key quantization commutes with it when fp16 adds are exact.
+    B, Hq, Hkv, d, L, gk, R = 1, 4, 1, 64, 32 * 6 + 40, 32, 32
+    rng = np.random.default_rng(8)
+    k = (rng.integers(-1024, 1024, size=(B, Hkv, L, d)) * 2.0 ** -6).astype(np.float16)
+    mu = rng.integers(-8, 9, size=(d,)).astype(np.float64)
+    k_mu = (k.astype(np.float64) + mu).astype(np.float16)
+    assert np.array_equal(k_mu.astype(np.float64), k.astype(np.float64) + mu)
+    v = W.random_fp16((B, Hkv, L, d), seed=9).numpy()
+    q = W.random_fp16((B, Hq, d), seed=10).numpy()
+    cfg = cfg_of(B, Hq, Hkv, d, d, 4, 2, gk, 32, R, 1, L)
+    a, b = O.OracleCache(cfg), O.OracleCache(cfg)
+    a.prefill(k, v)
+    b.prefill(k_mu, v)
+    assert np.array_equal(a.kcode, b.kcode)
+    assert np.array_equal(a.ksz[..., 0], b.ksz[..., 0])
+    ng = a.Q // gk
+    assert np.array_equal(b.ksz[0, 0, :ng, :, 1].astype(np.float64),
+                          a.ksz[0, 0, :ng, :, 1].astype(np.float64) + mu)
+    assert np.allclose(a.decode(q), b.decode(q), rtol=1e-11, atol=1e-12)
+
+
+def test_token_order_invariance():
+    # "LogQuant", §4: A.V = A_P.V_P for any permutation P of the tokens.
+    rng = np.random.default_rng(12)
+    k = rng.normal(size=(300, 32)) * 3
+    v = rng.normal(size=(300, 48))
+    q = rng.normal(size=32)
+    perm = rng.permutation(300)
+    a = O.attention(q, k, v, 1 / math.sqrt(32))
+    b = O.attention(q, k[perm], v[perm], 1 / math.sqrt(32))
+    assert np.allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+def test_thin_key_scale_is_one_over_sqrt_dk():
+    # "Thin Keys, Full Values", §2: softmax(Q K^T / sqrt(d_select)) V with d_select = d_k.
+    rng = np.random.default_rng(13)
+    k = rng.normal(size=(50, 32))
+    v = rng.normal(size=(50, 128))
+    q = rng.normal(size=32)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q)[None, None], torch.tensor(k)[None], torch.tensor(v)[None])[0, 0].numpy()
+    assert np.allclose(O.attention(q, k, v, 1 / math.sqrt(32)), ref, rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------- retention ----
+def retained_by_octaves(Q):
+    """Independent enumeration: for each octave l the multiple of 2^l among ages [2^l, 2^(l+1))."""
+    out = []
+    l = 0
+    while (1 << l) <= Q:
+        lo = max(Q - (1 << (l + 1)) + 1, 0)
+        hi = Q - (1 << l)
+        cands = [p for p in range(lo, hi + 1) if p % (1 << l) == 0]
+        assert len(cands) == 1
+        out.append(cands[0])
+        l += 1
+    return sorted(out)
+
+
+def test_retention_matches_octave_enumeration_and_count():
+    for Q in list(range(1, 300)) + [32640, 32704, 130944, 131008]:
+        r = O.retained_positions(Q)
+        assert r == retained_by_octaves(Q)
+        assert len(r) == int(math.floor(math.log2(Q))) + 1
+        assert len(r) <= O.MAX_RETAINED
+    assert len(O.retained_positions(32640)) == 15          # ~log2(L) at the 32k workload
+
+
+def test_retention_only_shrinks_as_q_grows():
+    gk = 64
+    for Q in range(gk, 40 * gk, gk):
+        old, new = set(O.retained_positions(Q)), set(O.retained_positions(Q + gk))
+        assert all(p in old or Q <= p < Q + gk for p in new)
+
+
+# ------------------------------------------------------ append vs prefill ----
+@pytest.mark.parametrize("log_retain", [0, 1])
+def test_appends_reach_the_same_state_as_one_prefill(log_retain):
+    B, Hq, Hkv, d, gk, gv, R = 2, 4, 2, 32, 16, 16, 24
+    L0, n_app = 70, 90
+    k = W.random_fp16((B, Hkv, L0 + n_app, d), seed=51, scale=4.0).numpy()
+    v = W.random_fp16((B, Hkv, L0 + n_app, d), seed=52).numpy()
+    cfg = cfg_of(B, Hq, Hkv, d, d, 4, 2, gk, gv, R, log_retain, 256)
+    a = O.OracleCache(cfg)
+    a.prefill(k[:, :, :L0], v[:, :, :L0])
+    events = 0
+    for t in range(L0, L0 + n_app):
+        q_before = a.Q
+        old_ret = set(a.ret_idx)
+        a.append(k[:, :, t], v[:, :, t])
+        assert R <= a.L - a.Q < R + gk
+        if a.Q != q_before:
+            events += 1
+            assert a.Q == q_before + gk
+            assert all(p in old_ret or q_before <= p < a.Q for p in a.ret_idx)
+    assert events >= 4
+    b = O.OracleCache(cfg)
+    b.prefill(k, v)
+    assert (a.L, a.Q, a.ret_idx) == (b.L, b.Q, b.ret_idx)
+    for name in ("kcode", "ksz", "vcode", "vsz", "win_k", "win_v", "ret_k", "ret_v"):
+        x, y = getattr(a, name), getattr(b, name)
+        if name.startswith("win"):
+            slots = [p % a.cap for p in range(a.Q, a.L)]
+            x, y = x[:, :, slots], y[:, :, slots]
+        if name.startswith("ret"):
+            x, y = x[:, :, :len(a.ret_idx)], y[:, :, :len(a.ret_idx)]
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), name
+
+
+def test_window_sizes_of_the_workloads():
+    for key, want in (("tiny", 64), ("gqa4k", 128), ("long32k", 128), ("thin16k", 64)):
+        w = W.WORKLOADS[key]
+        Q = O.quantized_prefix(w.context, w.window, w.group_k, w.k_bits)
+        assert w.context - Q == want
+
+
+# ------------------------------------------------------------------- bytes ----
+def test_k4v2_saves_a_quarter_of_k4v4_code_bytes():
+    # "Quantize What Counts", §Résultats / §Contributions: K4V2 uses 25% less KV memory
+    # than K4V4 (code bytes: 4+2 bits vs 4+4 bits per K/V pair of elements).
+    base = cfg_of(8, 32, 8, 128, 128, 4, 4, 64, 64, 128, 0, 4096)
+    a = O.buffer_bytes(base)
+    b = O.buffer_bytes(dict(base, v_bits=2))
+    assert (b["kcode"] + b["vcode"]) / (a["kcode"] + a["vcode"]) == 0.75
+
+
+def test_algorithmic_bytes_per_token_k4v2_g64():
+    # codes + (scale, zero) per token per kv head at d=128, K4 G64 / V2 G64: 64+8+32+8 = 112 B
+    cfg = cfg_of(1, 1, 1, 128, 128, 4, 2, 64, 64, 128, 0, 64 * 100)
+    bb = O.buffer_bytes(cfg)
+    lcap = 64 * 100
+    assert (bb["kcode"] + bb["ksz"] + bb["vcode"] + bb["vsz"]) / lcap == 112
