@@ -1,0 +1,376 @@
+"""Decode-attention throughput over a packed mixed-precision KV cache on B200.
+
+One step = one generation step of every sequence in the batch: append the new
+token's K/V (window write; every group_k steps the oldest window group is
+quantized and the retained set updated) and decode attention of one query token
+per query head over the whole cache (split-K decode kernel + log-sum-exp combine).
+The default workload is the 32k long-context case: batch 32, 32 query / 8 KV heads,
+d = 128, K4/V2 with groups of 64, fp16 window 128, log-spaced retention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+Prints one JSON line (rank 0).  With N > 1 (torchrun) every rank runs its own
+batch (weak scaling, no collective on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixed_precision_quantized_pack_b200 import kvq as K  # noqa: E402
+from mixed_precision_quantized_pack_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode attn tokens/s and achieved HBM GB/s over packed KV (K4V2, ctx 32k)"
+UNIT = "tokens/s"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_long32k_ncu.md")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def decode_bytes(cfg: dict, L: int) -> int:
+    """Algorithmic bytes one decode reads: packed codes and (scale, zero) of the quantized
+    tokens (retained slots included), fp16 window and retained tokens, and q."""
+    B, H, dk, dv = cfg["batch"], cfg["n_kv_heads"], cfg["d_k"], cfg["d_v"]
+    kb, vb, gk, gv, R = cfg["k_bits"], cfg["v_bits"], cfg["group_k"], cfg["group_v"], cfg["window"]
+    if kb == 16:
+        return B * H * L * (dk + dv) * 2 + B * cfg["n_q_heads"] * dk * 2
+    Q = max(L - R, 0) // gk * gk
+    nret = len(K.kvq_retained_positions(Q)) if cfg["log_retain"] else 0
+    per_tok = dk * kb // 8 + dv * vb // 8 + (dv // gv) * 4
+    quant = Q * per_tok + (Q // gk) * dk * 4
+    fp16 = (L - Q + nret) * (dk + dv) * 2
+    return B * H * (quant + fp16) + B * cfg["n_q_heads"] * dk * 2
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def profile_traffic():
+    """dram bytes per decode launch from the committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"decode_source_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "mixed_precision_quantized_pack_b200", "csrc", "decode_mma.cu")
+    try:
+        cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return float(m.group(1)) if cur.startswith(h.group(1)) else None
+
+
+# ------------------------------------------------------------------ CPU oracle ----
+def oracle_decode_sample(w: W.Workload, budget_s: float, steps: int = 1):
+    """Times the CPU oracle's append+decode on whole sequences of the workload until
+    about budget_s seconds of decode work; returns (tokens/s, seconds, sequences, threads)."""
+    from oracle import kvq_oracle as O
+    import threadpoolctl
+    inp = W.Inputs(w.with_(batch=1, appends=max(steps, 1)), device="cpu")
+    oc = O.OracleCache(dict(w.kvq_config(max_context=w.context + steps + 64), batch=1))
+    oc.prefill(inp.k.numpy(), inp.v.numpy())
+    spent, done = 0.0, 0
+    for i in range(steps):
+        t0 = time.perf_counter()
+        oc.append(inp.k_app[i].numpy(), inp.v_app[i].numpy())
+        oc.decode(inp.q[i].numpy())
+        spent += time.perf_counter() - t0
+        done += 1
+        if spent >= budget_s:
+            break
+    threads = max([x.get("num_threads", 1) for x in threadpoolctl.threadpool_info()] or [1])
+    return done / spent, spent, done, threads
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    import threadpoolctl
+    from oracle import kvq_oracle as O
+    steps = args.steps + args.warmup
+    inp = W.Inputs(w.with_(batch=1, appends=steps), device="cpu")
+    oc = O.OracleCache(dict(w.kvq_config(max_context=w.context + steps + 64), batch=1))
+    oc.prefill(inp.k.numpy(), inp.v.numpy())
+    for i in range(steps):
+        t0 = time.perf_counter()
+        oc.append(inp.k_app[i].numpy(), inp.v_app[i].numpy())
+        oc.decode(inp.q[i].numpy())
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    t = sum(times) / len(times)
+    value = 1.0 / t          # one sequence's token per step, same workload
+    threads = max([x.get("num_threads", 1) for x in threadpoolctl.threadpool_info()] or [1])
+    sample = (f"CPU oracle (numpy, fp64 attention) append+decode of 1 of {w.batch} sequences "
+              f"(all {w.n_kv_heads} kv heads) per step at context {w.context}")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm -------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default="long32k", choices=list(W.WORKLOADS))
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    steps, warm = args.steps, max(args.warmup, 3)
+    wl = w.with_(appends=steps + warm, seed=w.seed + 7919 * rank)
+    cfg = wl.kvq_config(max_context=wl.context + steps + warm + 64)
+    inp = W.Inputs(wl, device=dev)
+    cache = K.KVCache(cfg, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # prefill (timed for information)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    cache.prefill(inp.k, inp.v)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    prefill_ms = e0.elapsed_time(e1)
+    del inp.k, inp.v
+    torch.cuda.empty_cache()
+
+    out = torch.empty((wl.batch, wl.n_q_heads, wl.d_v), dtype=torch.float16, device=dev)
+    n_ev = steps + warm
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    launches = 0
+    bytes_read = []
+
+    def step(i, timed):
+        nonlocal launches
+        _, q0, _ = cache.state()
+        cache.append(inp.k_app[i], inp.v_app[i])
+        L, q1, _ = cache.state()
+        starts[i].record(stream)
+        cache.decode(inp.q[i], out=out)
+        ends[i].record(stream)
+        if timed:
+            launches += 2 + 2          # window writes (K, V) + decode + combine
+            if q1 != q0:
+                launches += 2 + (1 if cfg["log_retain"] else 0)
+            bytes_read.append(decode_bytes(cfg, L))
+
+    for i in range(warm):
+        step(i, False)
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(warm, warm + steps):
+        step(i, True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t0.elapsed_time(t1)
+    dec_ms = [starts[i].elapsed_time(ends[i]) for i in range(warm, warm + steps)]
+    dec_avg = sum(dec_ms) / len(dec_ms)
+    status = cache.status()
+    if dist:
+        t = torch.tensor([total_ms, dec_avg], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, dec_avg = float(t[0]), float(t[1])
+    ms_step = total_ms / steps
+    value = world * wl.batch / (ms_step / 1e3)
+    achieved = (sum(bytes_read) / len(bytes_read)) / (dec_avg / 1e3) / 1e9
+    peak, peak_kind = peaks()
+
+    # end to end through the public API: pinned host inputs in, host output back, per step
+    h_q = [x.cpu().pin_memory() for x in inp.q[:steps]]
+    h_k = [x.cpu().pin_memory() for x in inp.k_app[:steps]]
+    h_v = [x.cpu().pin_memory() for x in inp.v_app[:steps]]
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_q = torch.empty_like(inp.q[0])
+    d_k = torch.empty_like(inp.k_app[0])
+    d_v = torch.empty_like(inp.v_app[0])
+    e2e_cache = K.KVCache(cfg, device=dev)
+    inp2 = W.Inputs(wl.with_(appends=1), device=dev)
+    e2e_cache.prefill(inp2.k, inp2.v)
+    del inp2
+    torch.cuda.empty_cache()
+    for i in range(3):
+        d_q.copy_(h_q[i], non_blocking=True)
+        d_k.copy_(h_k[i], non_blocking=True)
+        d_v.copy_(h_v[i], non_blocking=True)
+        e2e_cache.append(d_k, d_v)
+        e2e_cache.decode(d_q, out=out)
+        h_out.copy_(out, non_blocking=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = min(steps, len(h_q)) - 3
+    a.record(stream)
+    for i in range(3, 3 + n_e2e):
+        d_q.copy_(h_q[i], non_blocking=True)
+        d_k.copy_(h_k[i], non_blocking=True)
+        d_v.copy_(h_v[i], non_blocking=True)
+        e2e_cache.append(d_k, d_v)
+        e2e_cache.decode(d_q, out=out)
+        h_out.copy_(out, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a.elapsed_time(b) / max(n_e2e, 1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
+    d2h = out.numel() * 2
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, spent, seqs, threads = oracle_decode_sample(w, args.cpu_budget, steps=8)
+        cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{seqs} append+decode steps of 1 of {w.batch} sequences "
+                         f"(all {w.n_kv_heads} kv heads, context {w.context}) in {spent:.1f} s"}
+
+    if rank == 0:
+        plan = cache.plan()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; keys N(0,1)*sigma_c+mu_c with log-uniform sigma, values/q N(0,1))",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
+                       "n_kv_heads": wl.n_kv_heads, "d_k": wl.d_k, "d_v": wl.d_v,
+                       "context": wl.context, "k_bits": wl.k_bits, "v_bits": wl.v_bits,
+                       "group_k": wl.group_k, "group_v": wl.group_v, "window": wl.window,
+                       "log_retain": wl.log_retain, "parallelism": f"dp{world} (independent batches)",
+                       "l2": "no flush: each decode reads %.0f MB > 126 MB L2" % (bytes_read[0] / 1e6),
+                       "step": "append 1 token + decode, per sequence",
+                       "plan": plan},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": profile_traffic(),
+                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                         "kernel": "decode (split-K kernel + combine), CUDA events per launch",
+                         "decode_ms": dec_avg, "bytes_per_launch": bytes_read[0]},
+            "decode_tokens_per_s": world * wl.batch / (dec_avg / 1e3),
+            "prefill_ms": prefill_ms,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * wl.batch / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    del cache, e2e_cache
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * kvq.h — decode attention read straight from a packed, mixed-precision,
+ * groupwise-quantized KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (one attention layer of autoregressive decoding):
+ *   - the cache keeps every token ("LogQuant: Log-Distributed 2-Bit Quantization
+ *     of KV Cache", §Méthodologie 3: quantize instead of evicting);
+ *   - the most recent tokens stay fp16 (same page, §Comment LogQuant Fonctionne);
+ *     optionally one older token per age octave stays fp16 too (same page,
+ *     §Méthodologie 2, log-based filtering);
+ *   - older keys are quantized per channel over groups of group_k tokens (same
+ *     page, §5), older values per token over groups of group_v channels, keys
+ *     with more bits than values ("Quantize What Counts: More for Keys, Less for
+ *     Values", §La Solution, K4V2);
+ *   - keys may be thinner than values, d_k < d_v ("Thin Keys, Full Values:
+ *     Reducing KV Cache via Low-Dimensional Attention Selection", §2), and the
+ *     score is q.k / sqrt(d_k);
+ *   - the order in which tokens are visited is free (LogQuant §4, A.V = A_P.V_P).
+ *
+ * Quantizer (bit-exact contract; every step IEEE binary32, round to nearest even):
+ *   s = fp16((max - min) / (2^bits - 1))   (+0 if that is zero)
+ *   z = fp16(min)                          (+0 for a signed zero)
+ *   code = s == 0 ? 0 : clamp(rint((x - z) / s), 0, 2^bits - 1)
+ * Regions: with L tokens, Q = floor(max(L - window, 0) / group_k) * group_k
+ * tokens are quantized and [Q, L) are fp16 (Q = 0 when the bit widths are 16).
+ * Retained set (log_retain = 1): { p < Q : p mod 2^floor(log2(Q - p)) == 0 }.
+ *
+ * Buffer layouts (all caller-owned device memory, 256-byte aligned recommended,
+ * 16-byte aligned required; sizes from kvq_buffer_sizes):
+ *   kcode  u32  [B][Hkv][Lcap][d_k*k_bits/32]   token rows, channel c at word
+ *               c/(32/k_bits), bit (c%(32/k_bits))*k_bits (LSB first)
+ *   ksz    f16  [B][Hkv][Lcap/group_k][d_k][2] (scale, zero) per key group and channel
+ *   vcode  u32  [B][Hkv][Lcap][d_v*v_bits/32]   same packing per token row
+ *   vsz    f16  [B][Hkv][Lcap][d_v/group_v][2] (scale, zero) per token and value group
+ *   win_k  f16  [B][Hkv][C][d_k]  token p in slot p % C, C = window + group_k
+ *   win_v  f16  [B][Hkv][C][d_v]  (bits 16: C = max_context, the whole cache)
+ *   ret_k  f16  [B][Hkv][32][d_k] retained tokens, ascending positions
+ *   ret_v  f16  [B][Hkv][32][d_v]
+ * with Lcap = max_context rounded up to a multiple of group_k.
+ *
+ * Conventions: every call is asynchronous on the caller's CUDA stream (passed as
+ * void*, a cudaStream_t; NULL = legacy default stream); no call synchronizes or
+ * copies device memory back to the host, except kvq_read_status.  The library
+ * allocates no device memory.  A cache handle must not be used from two host
+ * threads or two streams at once.  Inputs must be finite; NaN or Inf in K, V or
+ * q gives undefined (but memory-safe) results.  GQA: query head hq reads kv
+ * head hq / (n_q_heads / n_kv_heads).  Every function returns KVQ_OK (0) or one
+ * of the negative codes below and changes nothing when it fails argument checks.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_OK                 0
+#define KVQ_ERR_INVALID_ARG   -1  /* null pointer, non-positive size, L > max_context */
+#define KVQ_ERR_UNSUPPORTED   -2  /* shape / bit width / group outside the built set */
+#define KVQ_ERR_ALIGN         -3  /* a device pointer is not 16-byte aligned */
+#define KVQ_ERR_CAPACITY      -4  /* an append past max_context */
+#define KVQ_ERR_WORKSPACE     -5  /* workspace smaller than kvq_decode_workspace_size */
+#define KVQ_ERR_STATE         -6  /* decode or append before any prefill */
+#define KVQ_ERR_CUDA          -7  /* a CUDA runtime call or kernel launch failed */
+
+#define KVQ_MAX_RETAINED      32
+
+/* Device status bits, written into the first word of a decode workspace. */
+#define KVQ_STATUS_TIMEOUT    1u  /* a bounded wait in the decode kernel gave up */
+
+typedef struct kvq_config {
+    int batch;          /* B, sequences sharing one length */
+    int n_q_heads;      /* Hq */
+    int n_kv_heads;     /* Hkv; Hq % Hkv == 0 */
+    int d_k;            /* key/query head dim: 32, 64, 128 or 256 */
+    int d_v;            /* value head dim: 32, 64, 128 or 256 */
+    int k_bits;         /* 2, 4, 8, or 16 (= unquantized; then v_bits must be 16) */
+    int v_bits;         /* 2, 4, 8, or 16 */
+    int group_k;        /* tokens per key group: 16, 32, 64 or 128 */
+    int group_v;        /* channels per value group: divides d_v, >= 32/v_bits */
+    int window;         /* R >= 0: fp16 recent tokens kept beside the quantized prefix */
+    int log_retain;     /* 0/1: keep log-spaced older tokens in fp16 (ignored at 16 bits) */
+    int max_context;    /* capacity in tokens, >= 1 */
+} kvq_config;
+
+typedef struct kvq_sizes {
+    size_t kcode, ksz, vcode, vsz, win_k, win_v, ret_k, ret_v;
+    size_t workspace;   /* a decode workspace large enough for any length and split count */
+} kvq_sizes;
+
+typedef struct kvq_buffers {
+    void *kcode, *ksz, *vcode, *vsz, *win_k, *win_v, *ret_k, *ret_v;
+} kvq_buffers;
+
+typedef struct kvq_cache kvq_cache;   /* opaque host-side handle */
+
+/* Split plan of one decode call (see kvq_plan_decode). */
+typedef struct kvq_plan {
+    int splits_quant;   /* CTAs per (b, kv head) over the quantized groups */
+    int splits_fp16;    /* CTAs per (b, kv head) over window + retained tokens */
+    int n_groups;       /* quantized groups, Q / group_k */
+    int n_fp16;         /* fp16 tokens: retained + window */
+    int fast_path;      /* 1: tensor-core kernel; 0: generic CUDA-core kernel */
+} kvq_plan;
+
+/* Bytes of each buffer for a configuration (see the layout above).  Host only.
+ * Buffers a configuration does not use (e.g. kcode at 16 bits) get size 0 and
+ * may be passed as NULL.  Errors: INVALID_ARG, UNSUPPORTED. */
+int kvq_buffer_sizes(const kvq_config* cfg, kvq_sizes* out);
+
+/* Create a handle over caller-owned device buffers (not touched here).  Queries
+ * the current device's SM count.  The handle copies cfg and the pointers; the
+ * buffers must outlive it.  Errors: INVALID_ARG, UNSUPPORTED, ALIGN, CUDA. */
+int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** out);
+
+/* Free the handle (not the buffers).  NULL is a no-op. */
+void kvq_cache_destroy(kvq_cache* cache);
+
+/* Fill an empty cache with L >= 1 tokens: k fp16 [B][Hkv][L][d_k], v fp16
+ * [B][Hkv][L][d_v], contiguous device memory.  Quantizes [0, Q), copies [Q, L)
+ * into the window and the retained tokens into ret_k/ret_v.  Resets any earlier
+ * content.  Errors: INVALID_ARG (L < 1 or L > max_context), ALIGN, CUDA. */
+int kvq_quantize_prefill(kvq_cache* cache, const void* k, const void* v, int L, void* stream);
+
+/* Append one token per sequence: k_new fp16 [B][Hkv][d_k], v_new fp16
+ * [B][Hkv][d_v].  When the window reaches window + group_k tokens, its oldest
+ * group_k tokens are quantized and the retained set is updated.
+ * Errors: STATE (no prefill yet), CAPACITY, INVALID_ARG, ALIGN, CUDA. */
+int kvq_append(kvq_cache* cache, const void* k_new, const void* v_new, void* stream);
+
+/* Workspace bytes kvq_decode_attention needs at the cache's current length for
+ * num_splits (0 = automatic).  Always <= kvq_sizes.workspace. */
+int kvq_decode_workspace_size(const kvq_cache* cache, int num_splits, size_t* bytes);
+
+/* Attention of one query token per sequence over all L cached tokens:
+ * q fp16 [B][Hq][d_k] -> out fp16 [B][Hq][d_v].  Scores q.k/sqrt(d_k), fp32
+ * softmax and accumulation, split over tokens (flash-decoding) and merged by a
+ * log-sum-exp combine.  workspace: device scratch of workspace_bytes; its first
+ * 4 bytes are a status word the kernel ORs KVQ_STATUS_* bits into (never
+ * cleared by this call; see kvq_reset_status).  num_splits: 0 = automatic, else
+ * the number of splits over the quantized groups (or over the fp16 tokens when
+ * nothing is quantized), clamped to the available work.
+ * Errors: STATE, INVALID_ARG, ALIGN, WORKSPACE, CUDA. */
+int kvq_decode_attention(kvq_cache* cache, const void* q, void* out, void* workspace,
+                         size_t workspace_bytes, int num_splits, void* stream);
+
+/* The plan kvq_decode_attention would use now (host only, no launch). */
+int kvq_get_plan(const kvq_cache* cache, int num_splits, kvq_plan* out);
+
+/* Pure host planner behind kvq_get_plan, for a configuration, length L, SM count
+ * and split request.  Errors: INVALID_ARG, UNSUPPORTED. */
+int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, kvq_plan* out);
+
+/* Host-side cache state: length L, quantized prefix Q, retained count and the
+ * ascending retained positions (retained_idx: host int[32], may be NULL). */
+int kvq_get_state(const kvq_cache* cache, int* L, int* Q, int* n_retained, int* retained_idx);
+
+/* The retention rule for a quantized prefix of Q tokens (host only): writes the
+ * ascending positions into out[0..cap) and returns their count (>= 0), or
+ * INVALID_ARG if out is NULL while Q > 0, or if cap is too small. */
+int kvq_retained_positions(int Q, int* out, int cap);
+
+/* Zero the status word of a decode workspace (asynchronous, on stream). */
+int kvq_reset_status(void* workspace, void* stream);
+
+/* Wait for stream, then copy the status word of a decode workspace to *status.
+ * The only call that synchronizes. */
+int kvq_read_status(const void* workspace, unsigned int* status, void* stream);
+
+/* Static description of an error code. */
+const char* kvq_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

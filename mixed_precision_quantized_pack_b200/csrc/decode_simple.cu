@@ -1,0 +1,168 @@
+// Generic decode-attention kernel on CUDA cores (any supported shape).
+//
+// Computes, for one (b, kv head) and one split of its tokens, the flash-decoding
+// partial (m, l, o) of every query head sharing the kv head:
+//   k_hat = code * s + z (key groups per channel, value groups per token), or the
+//           fp16 copy for window and retained tokens ("LogQuant: Log-Distributed
+//           2-Bit Quantization of KV Cache", §Méthodologie 2 and 3);
+//   score = q . k_hat / sqrt(d_k) ("Thin Keys, Full Values", §2), kept in log2 units;
+//   online softmax, o = sum_j 2^(score_j - m) v_hat_j.
+// One warp per token: each lane holds d/32 channels, dot products reduce with
+// warp shuffles.  The tensor-core kernel replaces this one on the shapes it
+// supports; this one is the reference GPU path for everything else.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+constexpr int kMaxRep = 8;
+constexpr int kMaxC = 8;      // d / 32, d <= 256
+constexpr int kWarps = 4;
+
+__global__ void __launch_bounds__(kWarps * 32)
+decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials p) {
+  __shared__ float sm_m[kWarps][kMaxRep];
+  __shared__ float sm_l[kWarps][kMaxRep];
+  __shared__ float sm_o[kWarps][kMaxRep][kMaxC * 32];
+
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * d.Hkv + h;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nrep = d.n_rep, ck = d.dk / 32, cv = d.dv / 32;
+
+  float qr[kMaxRep][kMaxC];
+#pragma unroll
+  for (int r = 0; r < kMaxRep; ++r)
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j)
+      qr[r][j] = (r < nrep && j < ck)
+                     ? __half2float(q[(static_cast<size_t>(b) * d.Hq + h * nrep + r) * d.dk + lane + 32 * j]) * w.score_scale
+                     : 0.0f;
+  float m[kMaxRep], l[kMaxRep], o[kMaxRep][kMaxC];
+#pragma unroll
+  for (int r = 0; r < kMaxRep; ++r) {
+    m[r] = -INFINITY;
+    l[r] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j) o[r][j] = 0.0f;
+  }
+
+  const bool quant = split < w.splits_q;
+  int begin, end;
+  if (quant) {
+    begin = static_cast<int>(static_cast<long long>(split) * w.n_groups / w.splits_q) * d.gk;
+    end = static_cast<int>(static_cast<long long>(split + 1) * w.n_groups / w.splits_q) * d.gk;
+  } else {
+    const int f = split - w.splits_q;
+    begin = static_cast<int>(static_cast<long long>(f) * w.n_fp16 / w.splits_f);
+    end = static_cast<int>(static_cast<long long>(f + 1) * w.n_fp16 / w.splits_f);
+  }
+  const int perk = d.kb == 16 ? 1 : 32 / d.kb, perv = d.vb == 16 ? 1 : 32 / d.vb;
+  const uint32_t maskk = (1u << (d.kb & 15)) - 1u, maskv = (1u << (d.vb & 15)) - 1u;
+
+  for (int i = begin + warp; i < end; i += kWarps) {
+    float kh[kMaxC], vh[kMaxC];
+    if (quant) {
+      bool retained = false;
+      for (int r = 0; r < w.ret.n; ++r) retained |= (w.ret.pos[r] == i);
+      if (retained) continue;                                   // read from the fp16 list
+      const uint32_t* kr = cb.kcode + (static_cast<size_t>(bh) * d.lcap + i) * d.kw;
+      const __half2* ks = cb.ksz + (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * d.dk;
+      const uint32_t* vr = cb.vcode + (static_cast<size_t>(bh) * d.lcap + i) * d.vw;
+      const __half2* vs = cb.vsz + (static_cast<size_t>(bh) * d.lcap + i) * d.nvg;
+#pragma unroll
+      for (int j = 0; j < kMaxC; ++j) {
+        kh[j] = 0.0f;
+        vh[j] = 0.0f;
+        if (j < ck) {
+          const int ch = lane + 32 * j;
+          const uint32_t code = (kr[ch / perk] >> ((ch % perk) * d.kb)) & maskk;
+          const float2 sz = __half22float2(ks[ch]);
+          kh[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
+        }
+        if (j < cv) {
+          const int ch = lane + 32 * j;
+          const uint32_t code = (vr[ch / perv] >> ((ch % perv) * d.vb)) & maskv;
+          const float2 sz = __half22float2(vs[ch / d.gv]);
+          vh[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
+        }
+      }
+    } else {
+      const __half *kp, *vp;
+      if (i < w.ret.n) {
+        const size_t s = static_cast<size_t>(bh) * kMaxRetained + i;
+        kp = cb.ret_k + s * d.dk;
+        vp = cb.ret_v + s * d.dv;
+      } else {
+        const int pos = w.Q + (i - w.ret.n);
+        const size_t s = static_cast<size_t>(bh) * d.cap + pos % d.cap;
+        kp = cb.win_k + s * d.dk;
+        vp = cb.win_v + s * d.dv;
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxC; ++j) {
+        kh[j] = j < ck ? __half2float(kp[lane + 32 * j]) : 0.0f;
+        vh[j] = j < cv ? __half2float(vp[lane + 32 * j]) : 0.0f;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxRep; ++r) {
+      if (r >= nrep) break;
+      float s = 0.0f;
+#pragma unroll
+      for (int j = 0; j < kMaxC; ++j) s = fmaf(qr[r][j], kh[j], s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      const float mn = fmaxf(m[r], s);
+      const float alpha = exp2f(m[r] - mn);
+      const float pe = exp2f(s - mn);
+      l[r] = fmaf(l[r], alpha, pe);
+#pragma unroll
+      for (int j = 0; j < kMaxC; ++j) o[r][j] = fmaf(o[r][j], alpha, pe * vh[j]);
+      m[r] = mn;
+    }
+  }
+
+  // merge the warps of this CTA, then write one partial per query head
+#pragma unroll
+  for (int r = 0; r < kMaxRep; ++r) {
+    if (r < nrep) {
+      if (lane == 0) {
+        sm_m[warp][r] = m[r];
+        sm_l[warp][r] = l[r];
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxC; ++j)
+        if (j < cv) sm_o[warp][r][lane + 32 * j] = o[r][j];
+    }
+  }
+  __syncthreads();
+  for (int r = 0; r < nrep; ++r) {
+    float M = -INFINITY;
+    for (int k = 0; k < kWarps; ++k) M = fmaxf(M, sm_m[k][r]);
+    const size_t part = (static_cast<size_t>(b) * d.Hq + h * nrep + r) * w.splits + split;
+    float wk[kWarps];
+    float Lsum = 0.0f;
+    for (int k = 0; k < kWarps; ++k) {
+      wk[k] = (M == -INFINITY || sm_m[k][r] == -INFINITY) ? 0.0f : exp2f(sm_m[k][r] - M);
+      Lsum = fmaf(wk[k], sm_l[k][r], Lsum);
+    }
+    if (threadIdx.x == 0) p.ml[part] = make_float2(M, Lsum);
+    for (int c = threadIdx.x; c < d.dv; c += blockDim.x) {
+      float acc = 0.0f;
+      for (int k = 0; k < kWarps; ++k) acc = fmaf(wk[k], sm_o[k][r][c], acc);
+      p.o[part * d.dv + c] = acc;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_simple(const Dims& d, const CacheBufs& c, const DecodeWork& w,
+                                 const __half* q, const Partials& p, cudaStream_t s) {
+  dim3 grid(w.splits, d.Hkv, d.B);
+  decode_simple_kernel<<<grid, kWarps * 32, 0, s>>>(d, c, w, q, p);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

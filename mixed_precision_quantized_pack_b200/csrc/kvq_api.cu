@@ -1,0 +1,461 @@
+// C ABI of libkvq: argument checks, buffer sizes, the host-side cache state
+// (length L, quantized prefix Q, retained positions), the split planner and the
+// kernel launches.  All state the kernels need is known on the host from the
+// length alone, so no call ever waits for the device.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <new>
+#include <vector>
+
+#include "../../include/kvq.h"
+#include "kvq_internal.cuh"
+
+struct kvq_cache {
+  kvq::Dims d;
+  kvq_buffers buf;
+  int L;
+  int Q;
+  std::vector<int> ret;   // ascending retained positions
+  int sm_count;
+  bool prefilled;
+};
+
+namespace kvq {
+
+size_t workspace_bytes(const Dims& d, int splits) {
+  const size_t rows = static_cast<size_t>(d.B) * d.Hq * splits;
+  const size_t ml = (rows * sizeof(float2) + 255) / 256 * 256;
+  return 256 + ml + rows * d.dv * sizeof(float);
+}
+
+Partials workspace_views(const Dims& d, int splits, void* ws) {
+  const size_t rows = static_cast<size_t>(d.B) * d.Hq * splits;
+  const size_t ml = (rows * sizeof(float2) + 255) / 256 * 256;
+  char* base = static_cast<char*>(ws);
+  Partials p;
+  p.status = reinterpret_cast<unsigned int*>(base);
+  p.ml = reinterpret_cast<float2*>(base + 256);
+  p.o = reinterpret_cast<float*>(base + 256 + ml);
+  return p;
+}
+
+}  // namespace kvq
+
+namespace {
+
+bool is_pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks a configuration and derives the sizes the kernels use.
+int make_dims(const kvq_config* c, kvq::Dims* d) {
+  if (!c || !d) return KVQ_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1 || c->max_context < 1 ||
+      c->window < 0 || (c->log_retain != 0 && c->log_retain != 1))
+    return KVQ_ERR_INVALID_ARG;
+  if (c->n_q_heads % c->n_kv_heads != 0) return KVQ_ERR_UNSUPPORTED;
+  const int n_rep = c->n_q_heads / c->n_kv_heads;
+  if (n_rep > 8) return KVQ_ERR_UNSUPPORTED;
+  if (!is_pow2_in(c->d_k, 32, 256) || !is_pow2_in(c->d_v, 32, 256)) return KVQ_ERR_UNSUPPORTED;
+  const bool raw = c->k_bits == 16 || c->v_bits == 16;
+  if (raw) {
+    if (c->k_bits != 16 || c->v_bits != 16) return KVQ_ERR_UNSUPPORTED;
+  } else {
+    auto okb = [](int b) { return b == 2 || b == 4 || b == 8; };
+    if (!okb(c->k_bits) || !okb(c->v_bits)) return KVQ_ERR_UNSUPPORTED;
+    if (!is_pow2_in(c->group_k, 16, 128)) return KVQ_ERR_UNSUPPORTED;
+    if (c->group_v < 8 || c->group_v > c->d_v || c->d_v % c->group_v != 0 ||
+        c->group_v % 8 != 0 || (c->group_v * c->v_bits) % 32 != 0)
+      return KVQ_ERR_UNSUPPORTED;
+  }
+  // every element index must fit comfortably in 64 bits and every position in int
+  const long long lcap = raw ? c->max_context
+                             : (static_cast<long long>(c->max_context) + c->group_k - 1) /
+                                   c->group_k * c->group_k;
+  if (lcap > (1LL << 30)) return KVQ_ERR_UNSUPPORTED;
+  kvq::Dims x;
+  x.B = c->batch;
+  x.Hq = c->n_q_heads;
+  x.Hkv = c->n_kv_heads;
+  x.n_rep = n_rep;
+  x.dk = c->d_k;
+  x.dv = c->d_v;
+  x.kb = c->k_bits;
+  x.vb = c->v_bits;
+  x.gk = raw ? 1 : c->group_k;
+  x.gv = raw ? c->d_v : c->group_v;
+  x.R = c->window;
+  x.log_retain = raw ? 0 : c->log_retain;
+  x.max_context = c->max_context;
+  x.lcap = static_cast<int>(lcap);
+  x.cap = raw ? c->max_context : c->window + c->group_k;
+  x.kw = raw ? 0 : c->d_k * c->k_bits / 32;
+  x.vw = raw ? 0 : c->d_v * c->v_bits / 32;
+  x.nvg = raw ? 1 : c->d_v / c->group_v;
+  *d = x;
+  return KVQ_OK;
+}
+
+int quantized_prefix(const kvq::Dims& d, int L) {
+  if (!d.quantized()) return 0;
+  const int over = L - d.R;
+  return over > 0 ? over / d.gk * d.gk : 0;
+}
+
+// {p < Q : p mod 2^floor(log2(Q - p)) == 0}, ascending: one position per age octave.
+std::vector<int> retained_positions(int Q) {
+  std::vector<int> out;
+  for (int l = 0; l < 31 && (1 << l) <= Q; ++l) {
+    // ages a in [2^l, 2^(l+1)) are positions (Q - 2^(l+1), Q - 2^l]; keep the multiple of 2^l
+    const int hi = Q - (1 << l);
+    out.push_back(hi / (1 << l) * (1 << l));
+  }
+  std::sort(out.begin(), out.end());
+  return out;
+}
+
+int split_cap(const kvq::Dims& d) {
+  const int rows = d.B * d.Hkv;
+  return std::min(256, std::max(2, 8192 / rows));
+}
+
+// Occupancy assumed by the planner (CTAs per SM) for each decode kernel.
+int ctas_per_sm(bool fast) { return fast ? 3 : 4; }
+
+// Chooses the split counts: the number of CTAs per (b, kv head) over the quantized
+// groups and over the fp16 tokens, trading wave quantization against per-CTA cost.
+int plan_decode(const kvq::Dims& d, int L, int sm_count, int num_splits, bool fast,
+                kvq_plan* out) {
+  if (L < 1 || L > d.max_context || sm_count < 1 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
+  const int Q = quantized_prefix(d, L);
+  const int nret = d.log_retain ? static_cast<int>(retained_positions(Q).size()) : 0;
+  const int nG = Q / d.gk;
+  const int nF = nret + (L - Q);
+  const int rows = d.B * d.Hkv;
+  const int cap = split_cap(d);
+  const long long slots = static_cast<long long>(sm_count) * ctas_per_sm(fast);
+  // cost model in bytes read: per quantized group, per fp16 token, per CTA
+  const double bq = d.quantized()
+                        ? static_cast<double>(d.gk) * (d.kw * 4 + d.vw * 4 + d.nvg * 4) + d.dk * 4.0
+                        : 0.0;
+  const double bf = 2.0 * (d.dk + d.dv);
+  const double cta_cost = 16384.0;
+  auto best_split = [&](int n_units, double unit_bytes, int forced) {
+    if (n_units <= 0) return 0;
+    const int hi = std::min(n_units, cap);
+    if (forced > 0) return std::min(forced, hi);
+    int best = 1;
+    double best_t = 1e300;
+    for (int s = 1; s <= hi; ++s) {
+      const long long waves = (static_cast<long long>(rows) * s + slots - 1) / slots;
+      const double per_cta = ((n_units + s - 1) / s) * unit_bytes + cta_cost;
+      const double t = waves * per_cta;
+      if (t < best_t * 0.999) {
+        best_t = t;
+        best = s;
+      }
+    }
+    return best;
+  };
+  int sq = 0, sf = 0;
+  if (nG > 0) {
+    sq = best_split(nG, bq, num_splits);
+    // fp16 CTAs get about as many bytes as a quantized CTA
+    const double per_q = ((nG + sq - 1) / sq) * bq;
+    int want = static_cast<int>(ceil(nF * bf / std::max(per_q, 1.0)));
+    sf = std::max(1, std::min(want, std::min(cap, (nF + 15) / 16)));
+  } else {
+    sf = best_split((nF + 15) / 16, 16 * bf, num_splits);
+  }
+  if (nF == 0) sf = 0;
+  out->splits_quant = sq;
+  out->splits_fp16 = sf;
+  out->n_groups = nG;
+  out->n_fp16 = nF;
+  out->fast_path = fast ? 1 : 0;
+  return KVQ_OK;
+}
+
+int check_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
+
+kvq::CacheBufs cache_bufs(const kvq_cache* c) {
+  kvq::CacheBufs b;
+  b.kcode = static_cast<const uint32_t*>(c->buf.kcode);
+  b.ksz = static_cast<const __half2*>(c->buf.ksz);
+  b.vcode = static_cast<const uint32_t*>(c->buf.vcode);
+  b.vsz = static_cast<const __half2*>(c->buf.vsz);
+  b.win_k = static_cast<const __half*>(c->buf.win_k);
+  b.win_v = static_cast<const __half*>(c->buf.win_v);
+  b.ret_k = static_cast<const __half*>(c->buf.ret_k);
+  b.ret_v = static_cast<const __half*>(c->buf.ret_v);
+  return b;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_strerror(int code) {
+  switch (code) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported shape, bit width or group size";
+    case KVQ_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    case KVQ_ERR_CAPACITY: return "cache capacity (max_context) exceeded";
+    case KVQ_ERR_WORKSPACE: return "decode workspace too small";
+    case KVQ_ERR_STATE: return "cache not prefilled";
+    case KVQ_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown error";
+  }
+}
+
+int kvq_buffer_sizes(const kvq_config* cfg, kvq_sizes* out) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  kvq::Dims d;
+  const int rc = make_dims(cfg, &d);
+  if (rc) return rc;
+  const size_t bh = static_cast<size_t>(d.B) * d.Hkv;
+  kvq_sizes s;
+  memset(&s, 0, sizeof(s));
+  if (d.quantized()) {
+    s.kcode = bh * d.lcap * d.kw * 4;
+    s.ksz = bh * (d.lcap / d.gk) * d.dk * 4;
+    s.vcode = bh * d.lcap * d.vw * 4;
+    s.vsz = bh * d.lcap * d.nvg * 4;
+    s.ret_k = bh * kvq::kMaxRetained * d.dk * 2;
+    s.ret_v = bh * kvq::kMaxRetained * d.dv * 2;
+  }
+  s.win_k = bh * d.cap * d.dk * 2;
+  s.win_v = bh * d.cap * d.dv * 2;
+  s.workspace = kvq::workspace_bytes(d, 2 * split_cap(d));
+  *out = s;
+  return KVQ_OK;
+}
+
+int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** out) {
+  if (!cfg || !bufs || !out) return KVQ_ERR_INVALID_ARG;
+  kvq::Dims d;
+  int rc = make_dims(cfg, &d);
+  if (rc) return rc;
+  const void* need[] = {bufs->win_k, bufs->win_v};
+  for (const void* p : need)
+    if (!p) return KVQ_ERR_INVALID_ARG;
+  if (d.quantized()) {
+    const void* q[] = {bufs->kcode, bufs->ksz, bufs->vcode, bufs->vsz, bufs->ret_k, bufs->ret_v};
+    for (const void* p : q)
+      if (!p) return KVQ_ERR_INVALID_ARG;
+  }
+  const void* all[] = {bufs->kcode, bufs->ksz, bufs->vcode, bufs->vsz,
+                       bufs->win_k, bufs->win_v, bufs->ret_k, bufs->ret_v};
+  for (const void* p : all)
+    if (p && !aligned16(p)) return KVQ_ERR_ALIGN;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  kvq_cache* c = new (std::nothrow) kvq_cache;
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  c->d = d;
+  c->buf = *bufs;
+  c->L = 0;
+  c->Q = 0;
+  c->sm_count = sms;
+  c->prefilled = false;
+  *out = c;
+  return KVQ_OK;
+}
+
+void kvq_cache_destroy(kvq_cache* cache) { delete cache; }
+
+int kvq_retained_positions(int Q, int* out, int cap) {
+  if (Q < 0) return KVQ_ERR_INVALID_ARG;
+  const std::vector<int> r = retained_positions(Q);
+  if (r.empty()) return 0;
+  if (!out || cap < static_cast<int>(r.size())) return KVQ_ERR_INVALID_ARG;
+  std::copy(r.begin(), r.end(), out);
+  return static_cast<int>(r.size());
+}
+
+int kvq_quantize_prefill(kvq_cache* c, const void* k, const void* v, int L, void* stream) {
+  if (!c || !k || !v) return KVQ_ERR_INVALID_ARG;
+  const kvq::Dims& d = c->d;
+  if (L < 1 || L > d.max_context) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __half* kh = static_cast<const __half*>(k);
+  const __half* vh = static_cast<const __half*>(v);
+  const int Q = quantized_prefix(d, L);
+  const int nbh = d.B * d.Hkv;
+  int rc = KVQ_OK;
+  if (Q > 0) {
+    rc = check_cuda(kvq::launch_quantize_keys(d, kh, L, 0, Q / d.gk,
+                                              static_cast<uint32_t*>(c->buf.kcode),
+                                              static_cast<__half2*>(c->buf.ksz), s));
+    if (!rc)
+      rc = check_cuda(kvq::launch_quantize_values(d, vh, L, 0, Q,
+                                                  static_cast<uint32_t*>(c->buf.vcode),
+                                                  static_cast<__half2*>(c->buf.vsz), s));
+  }
+  if (!rc)
+    rc = check_cuda(kvq::launch_copy_rows(kh, L, Q, static_cast<__half*>(c->buf.win_k), d.cap, Q,
+                                          L - Q, d.dk, nbh, s));
+  if (!rc)
+    rc = check_cuda(kvq::launch_copy_rows(vh, L, Q, static_cast<__half*>(c->buf.win_v), d.cap, Q,
+                                          L - Q, d.dv, nbh, s));
+  std::vector<int> ret;
+  if (d.log_retain) ret = retained_positions(Q);
+  if (!rc && !ret.empty()) {
+    kvq::RetList rl;
+    rl.n = static_cast<int>(ret.size());
+    for (int i = 0; i < rl.n; ++i) rl.pos[i] = ret[i];
+    rc = check_cuda(kvq::launch_copy_retained(d, kh, vh, L, rl, static_cast<__half*>(c->buf.ret_k),
+                                              static_cast<__half*>(c->buf.ret_v), s));
+  }
+  if (rc) return rc;
+  c->L = L;
+  c->Q = Q;
+  c->ret = ret;
+  c->prefilled = true;
+  return KVQ_OK;
+}
+
+int kvq_append(kvq_cache* c, const void* k_new, const void* v_new, void* stream) {
+  if (!c || !k_new || !v_new) return KVQ_ERR_INVALID_ARG;
+  if (!c->prefilled) return KVQ_ERR_STATE;
+  const kvq::Dims& d = c->d;
+  if (c->L + 1 > d.max_context) return KVQ_ERR_CAPACITY;
+  if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int nbh = d.B * d.Hkv;
+  __half* wk = static_cast<__half*>(c->buf.win_k);
+  __half* wv = static_cast<__half*>(c->buf.win_v);
+  const int slot = c->L % d.cap;
+  int rc = check_cuda(kvq::launch_copy_rows(static_cast<const __half*>(k_new), 1, 0, wk, d.cap,
+                                            slot, 1, d.dk, nbh, s));
+  if (!rc)
+    rc = check_cuda(kvq::launch_copy_rows(static_cast<const __half*>(v_new), 1, 0, wv, d.cap, slot,
+                                          1, d.dv, nbh, s));
+  if (rc) return rc;
+  const int L = c->L + 1;
+  int Q = c->Q;
+  std::vector<int> ret = c->ret;
+  if (d.quantized() && L - Q == d.R + d.gk) {
+    // the oldest group_k window tokens become one key group and group_k value rows
+    rc = check_cuda(kvq::launch_quantize_keys(d, wk, d.cap, Q / d.gk, 1,
+                                              static_cast<uint32_t*>(c->buf.kcode),
+                                              static_cast<__half2*>(c->buf.ksz), s));
+    if (!rc)
+      rc = check_cuda(kvq::launch_quantize_values(d, wv, d.cap, Q, d.gk,
+                                                  static_cast<uint32_t*>(c->buf.vcode),
+                                                  static_cast<__half2*>(c->buf.vsz), s));
+    if (!rc && d.log_retain) {
+      const std::vector<int> nr = retained_positions(Q + d.gk);
+      kvq::RetUpdate up;
+      up.n = static_cast<int>(nr.size());
+      for (int i = 0; i < up.n; ++i) {
+        const auto it = std::lower_bound(c->ret.begin(), c->ret.end(), nr[i]);
+        if (it != c->ret.end() && *it == nr[i]) {
+          up.from_window[i] = 0;
+          up.index[i] = static_cast<int>(it - c->ret.begin());
+        } else {
+          up.from_window[i] = 1;
+          up.index[i] = nr[i] % d.cap;
+        }
+      }
+      rc = check_cuda(kvq::launch_update_retained(d, up, wk, wv, static_cast<__half*>(c->buf.ret_k),
+                                                  static_cast<__half*>(c->buf.ret_v), s));
+      ret = nr;
+    }
+    if (rc) return rc;
+    Q += d.gk;
+  }
+  c->L = L;
+  c->Q = Q;
+  c->ret = ret;
+  return KVQ_OK;
+}
+
+int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, kvq_plan* out) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  kvq::Dims d;
+  const int rc = make_dims(cfg, &d);
+  if (rc) return rc;
+  return plan_decode(d, L, sm_count, num_splits, kvq::decode_mma_supported(d), out);
+}
+
+int kvq_get_plan(const kvq_cache* c, int num_splits, kvq_plan* out) {
+  if (!c || !out) return KVQ_ERR_INVALID_ARG;
+  if (!c->prefilled) return KVQ_ERR_STATE;
+  return plan_decode(c->d, c->L, c->sm_count, num_splits, kvq::decode_mma_supported(c->d), out);
+}
+
+int kvq_decode_workspace_size(const kvq_cache* c, int num_splits, size_t* bytes) {
+  if (!c || !bytes) return KVQ_ERR_INVALID_ARG;
+  kvq_plan p;
+  const int rc = kvq_get_plan(c, num_splits, &p);
+  if (rc) return rc;
+  *bytes = kvq::workspace_bytes(c->d, p.splits_quant + p.splits_fp16);
+  return KVQ_OK;
+}
+
+int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace,
+                         size_t workspace_bytes, int num_splits, void* stream) {
+  if (!c || !q || !out || !workspace || num_splits < 0) return KVQ_ERR_INVALID_ARG;
+  if (!c->prefilled) return KVQ_ERR_STATE;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
+  const kvq::Dims& d = c->d;
+  kvq_plan plan;
+  int rc = plan_decode(d, c->L, c->sm_count, num_splits, kvq::decode_mma_supported(d), &plan);
+  if (rc) return rc;
+  kvq::DecodeWork w;
+  w.L = c->L;
+  w.Q = c->Q;
+  w.n_groups = plan.n_groups;
+  w.n_fp16 = plan.n_fp16;
+  w.splits_q = plan.splits_quant;
+  w.splits_f = plan.splits_fp16;
+  w.splits = plan.splits_quant + plan.splits_fp16;
+  w.score_scale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.dk)));
+  w.ret.n = static_cast<int>(c->ret.size());
+  for (int i = 0; i < w.ret.n; ++i) w.ret.pos[i] = c->ret[i];
+  if (workspace_bytes < kvq::workspace_bytes(d, w.splits)) return KVQ_ERR_WORKSPACE;
+  const kvq::Partials parts = kvq::workspace_views(d, w.splits, workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __half* qh = static_cast<const __half*>(q);
+  const kvq::CacheBufs cb = cache_bufs(c);
+  if (plan.fast_path)
+    rc = check_cuda(kvq::launch_decode_mma(d, cb, w, qh, parts, s));
+  else
+    rc = check_cuda(kvq::launch_decode_simple(d, cb, w, qh, parts, s));
+  if (!rc) rc = check_cuda(kvq::launch_combine(d, w, parts, static_cast<__half*>(out), s));
+  return rc;
+}
+
+int kvq_get_state(const kvq_cache* c, int* L, int* Q, int* n_retained, int* retained_idx) {
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  if (L) *L = c->L;
+  if (Q) *Q = c->Q;
+  if (n_retained) *n_retained = static_cast<int>(c->ret.size());
+  if (retained_idx)
+    for (size_t i = 0; i < c->ret.size(); ++i) retained_idx[i] = c->ret[i];
+  return KVQ_OK;
+}
+
+int kvq_reset_status(void* workspace, void* stream) {
+  if (!workspace) return KVQ_ERR_INVALID_ARG;
+  return check_cuda(cudaMemsetAsync(workspace, 0, sizeof(unsigned int),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int kvq_read_status(const void* workspace, unsigned int* status, void* stream) {
+  if (!workspace || !status) return KVQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KVQ_ERR_CUDA;
+  return check_cuda(cudaMemcpy(status, workspace, sizeof(unsigned int), cudaMemcpyDeviceToHost));
+}
+
+}  // extern "C"

@@ -1,0 +1,89 @@
+// Internal declarations shared by the host API and the kernels of libkvq.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace kvq {
+
+constexpr int kMaxRetained = 32;
+
+// Derived sizes of one cache (see include/kvq.h for the layouts).
+struct Dims {
+  int B, Hq, Hkv, n_rep, dk, dv, kb, vb, gk, gv, R, log_retain, max_context;
+  int lcap;   // quantized rows per (b, kv head): max_context rounded up to group_k
+  int cap;    // window ring slots: R + group_k, or max_context at 16 bits
+  int kw;     // u32 words per key row:   dk * kb / 32
+  int vw;     // u32 words per value row: dv * vb / 32
+  int nvg;    // value groups per token:  dv / gv
+  bool quantized() const { return kb != 16; }
+};
+
+// Positions of the retained tokens, ascending (kernel parameter by value).
+struct RetList {
+  int n;
+  int pos[kMaxRetained];
+};
+
+// Where each entry of the new retained list comes from during an append.
+struct RetUpdate {
+  int n;
+  int from_window[kMaxRetained];   // 1: window slot, 0: old retained slot
+  int index[kMaxRetained];         // the slot
+};
+
+// The tokens one decode call reads, and how they are split over CTAs.
+struct DecodeWork {
+  int L, Q;
+  int n_groups;      // Q / gk quantized groups
+  int n_fp16;        // fp16 list: retained entries, then window positions Q..L-1
+  int splits_q;      // CTAs per (b, kv head) over the groups
+  int splits_f;      // CTAs per (b, kv head) over the fp16 list
+  int splits;        // splits_q + splits_f (partials per (b, query head))
+  float score_scale; // log2(e) / sqrt(d_k)
+  RetList ret;
+};
+
+// Device views of the cache buffers.
+struct CacheBufs {
+  const uint32_t* kcode;
+  const __half2* ksz;
+  const uint32_t* vcode;
+  const __half2* vsz;
+  const __half* win_k;
+  const __half* win_v;
+  const __half* ret_k;
+  const __half* ret_v;
+};
+
+// Workspace layout: [status u32, padded to 256 B][(m, l) float2 per partial][o floats]
+struct Partials {
+  unsigned int* status;
+  float2* ml;    // [B*Hq][splits]
+  float* o;      // [B*Hq][splits][dv]
+};
+
+size_t workspace_bytes(const Dims& d, int splits);
+Partials workspace_views(const Dims& d, int splits, void* ws);
+
+// ---- launchers (return the launch error, cudaSuccess when fine) ----
+cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
+                                 int n_groups, uint32_t* kcode, __half2* ksz, cudaStream_t s);
+cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_rows, int t_begin,
+                                   int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s);
+cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,
+                             int dst_rows, int dst_base, int n, int d, int nbh, cudaStream_t s);
+cudaError_t launch_copy_retained(const Dims& d, const __half* k, const __half* v, int L,
+                                 const RetList& ret, __half* ret_k, __half* ret_v, cudaStream_t s);
+cudaError_t launch_update_retained(const Dims& d, const RetUpdate& up, __half* win_k,
+                                   __half* win_v, __half* ret_k, __half* ret_v, cudaStream_t s);
+cudaError_t launch_decode_simple(const Dims& d, const CacheBufs& c, const DecodeWork& w,
+                                 const __half* q, const Partials& p, cudaStream_t s);
+bool decode_mma_supported(const Dims& d);
+cudaError_t launch_decode_mma(const Dims& d, const CacheBufs& c, const DecodeWork& w,
+                              const __half* q, const Partials& p, cudaStream_t s);
+cudaError_t launch_combine(const Dims& d, const DecodeWork& w, const Partials& p, __half* out,
+                           cudaStream_t s);
+
+}  // namespace kvq

@@ -1,0 +1,256 @@
+// Write path of the cache: groupwise min-max quantize-and-pack, window and
+// retained-token copies.
+//
+// Quantizer (asymmetric uniform min-max with an fp16 scale and zero per group;
+// the form is this library's reading of the groupwise quantizers named in
+// "Quantize What Counts: More for Keys, Less for Values", §Méthodologie, and
+// "LogQuant: Log-Distributed 2-Bit Quantization of KV Cache", §5):
+//   s = fp16(fl32(max - min) / (2^b - 1))  (+0 when zero),  z = fp16(min + 0)
+//   code = s == 0 ? 0 : clamp(rint(fl32(fl32(x - z) / s)), 0, 2^b - 1)
+// Every step is an explicit IEEE round-to-nearest intrinsic so that no FMA
+// contraction or fast-math rewrite can change a code.  Keys: one group per
+// channel over group_k consecutive tokens (LogQuant §5, per-channel keys).
+// Values: one group per token over group_v consecutive channels.
+#include "kvq_internal.cuh"
+
+namespace kvq {
+namespace {
+
+struct GroupParams {
+  float scale;   // fp32 value of the fp16 scale
+  float zero;    // fp32 value of the fp16 zero
+  __half2 sz;    // (scale, zero) as stored
+};
+
+template <int BITS>
+__device__ __forceinline__ GroupParams group_params(float mn, float mx) {
+  const float levels = static_cast<float>((1 << BITS) - 1);
+  const float s32 = __fdiv_rn(__fsub_rn(mx, mn), levels);
+  __half s16 = __float2half_rn(s32);
+  if (__half2float(s16) == 0.0f) s16 = __ushort_as_half(0);          // canonical +0
+  const __half z16 = __float2half_rn(__fadd_rn(mn, 0.0f));            // exact, -0 -> +0
+  GroupParams g;
+  g.scale = __half2float(s16);
+  g.zero = __half2float(z16);
+  g.sz = __halves2half2(s16, z16);
+  return g;
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g) {
+  if (g.scale == 0.0f) return 0u;
+  const float levels = static_cast<float>((1 << BITS) - 1);
+  float c = rintf(__fdiv_rn(__fsub_rn(x, g.zero), g.scale));          // half-to-even
+  c = fminf(fmaxf(c, 0.0f), levels);
+  return static_cast<uint32_t>(c);
+}
+
+// One thread per (key group, channel); blockDim = (dk, groups per block).  The
+// 32/BITS lanes holding the channels of one packed word OR their codes together.
+template <int BITS>
+__global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_rows, int dk,
+                                     int gk, int g_begin, int n_groups, int lcap,
+                                     uint32_t* __restrict__ kcode, __half2* __restrict__ ksz) {
+  const int c = threadIdx.x;
+  const int gi = blockIdx.x * blockDim.y + threadIdx.y;
+  if (gi >= n_groups) return;                       // uniform per warp: dk % 32 == 0
+  const int bh = blockIdx.y;
+  const int g = g_begin + gi;
+  const size_t base = static_cast<size_t>(bh) * src_rows;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int t = 0; t < gk; ++t) {
+    const int row = (g * gk + t) % src_rows;
+    const float x = __half2float(src[(base + row) * dk + c]);
+    mn = fminf(mn, x);
+    mx = fmaxf(mx, x);
+  }
+  const GroupParams gp = group_params<BITS>(mn, mx);
+  ksz[(static_cast<size_t>(bh) * (lcap / gk) + g) * dk + c] = gp.sz;
+  constexpr int per = 32 / BITS;                    // channels per word
+  const int words = dk / per;
+  for (int t = 0; t < gk; ++t) {
+    const int row = (g * gk + t) % src_rows;
+    const float x = __half2float(src[(base + row) * dk + c]);
+    uint32_t part = quant_code<BITS>(x, gp) << ((c % per) * BITS);
+#pragma unroll
+    for (int off = 1; off < per; off <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, off);
+    if (c % per == 0)
+      kcode[(static_cast<size_t>(bh) * lcap + g * gk + t) * words + c / per] = part;
+  }
+}
+
+// One thread per (kv row, token, value group).  gv is a multiple of 8 and of 32/BITS.
+template <int BITS>
+__global__ void quantize_values_kernel(const __half* __restrict__ src, int src_rows, int dv,
+                                       int gv, int t_begin, int n_tokens, int nbh, int lcap,
+                                       uint32_t* __restrict__ vcode, __half2* __restrict__ vsz) {
+  const int nvg = dv / gv;
+  const long long total = static_cast<long long>(nbh) * n_tokens * nvg;
+  constexpr int per = 32 / BITS;
+  const int vw = dv / per;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int gidx = static_cast<int>(idx % nvg);
+    const long long r = idx / nvg;
+    const int t = t_begin + static_cast<int>(r % n_tokens);
+    const int bh = static_cast<int>(r / n_tokens);
+    const int row = t % src_rows;
+    const __half* x = src + (static_cast<size_t>(bh) * src_rows + row) * dv + gidx * gv;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int j = 0; j < gv; j += 8) {
+      const uint4 u = *reinterpret_cast<const uint4*>(x + j);
+      const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        mn = fminf(mn, fminf(f.x, f.y));
+        mx = fmaxf(mx, fmaxf(f.x, f.y));
+      }
+    }
+    const GroupParams gp = group_params<BITS>(mn, mx);
+    vsz[(static_cast<size_t>(bh) * lcap + t) * nvg + gidx] = gp.sz;
+    uint32_t* out = vcode + (static_cast<size_t>(bh) * lcap + t) * vw + gidx * (gv / per);
+    for (int w = 0; w < gv / per; ++w) {
+      uint32_t word = 0;
+      for (int k = 0; k < per; ++k) {
+        const float xv = __half2float(x[w * per + k]);
+        word |= quant_code<BITS>(xv, gp) << (k * BITS);
+      }
+      out[w] = word;
+    }
+  }
+}
+
+// dst[bh][(dst_base + i) % dst_rows] = src[bh][(src_base + i) % src_rows], i < n, 16 B at a time.
+__global__ void copy_rows_kernel(const __half* __restrict__ src, int src_rows, int src_base,
+                                 __half* __restrict__ dst, int dst_rows, int dst_base, int n,
+                                 int d, int nbh) {
+  const int vec = d / 8;
+  const long long total = static_cast<long long>(nbh) * n * vec;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int e = static_cast<int>(idx % vec);
+    const long long r = idx / vec;
+    const int i = static_cast<int>(r % n);
+    const int bh = static_cast<int>(r / n);
+    const int sr = (src_base + i) % src_rows;
+    const int dr = (dst_base + i) % dst_rows;
+    const uint4* s = reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + sr) * d);
+    uint4* t = reinterpret_cast<uint4*>(dst + (static_cast<size_t>(bh) * dst_rows + dr) * d);
+    t[e] = s[e];
+  }
+}
+
+// Prefill: ret[bh][j] = K[bh][pos[j]] for the retained positions (keys and values).
+__global__ void copy_retained_kernel(const __half* __restrict__ k, const __half* __restrict__ v,
+                                     int L, int dk, int dv, RetList ret,
+                                     __half* __restrict__ ret_k, __half* __restrict__ ret_v) {
+  const int bh = blockIdx.x;
+  for (int j = 0; j < ret.n; ++j) {
+    const size_t src = static_cast<size_t>(bh) * L + ret.pos[j];
+    const size_t dst = static_cast<size_t>(bh) * kMaxRetained + j;
+    for (int c = threadIdx.x; c < dk / 8; c += blockDim.x)
+      reinterpret_cast<uint4*>(ret_k + dst * dk)[c] = reinterpret_cast<const uint4*>(k + src * dk)[c];
+    for (int c = threadIdx.x; c < dv / 8; c += blockDim.x)
+      reinterpret_cast<uint4*>(ret_v + dst * dv)[c] = reinterpret_cast<const uint4*>(v + src * dv)[c];
+  }
+}
+
+// Append: rebuild the retained list in place, entry i from an old slot >= i or from
+// a window slot.  Entries are handled in ascending order, so an old slot is read
+// before any later entry overwrites it.
+__global__ void update_retained_kernel(RetUpdate up, int cap, int dk, int dv,
+                                       const __half* __restrict__ win_k,
+                                       const __half* __restrict__ win_v, __half* ret_k,
+                                       __half* ret_v) {
+  const int bh = blockIdx.x;
+  for (int i = 0; i < up.n; ++i) {
+    const size_t dst = static_cast<size_t>(bh) * kMaxRetained + i;
+    const __half* sk;
+    const __half* sv;
+    if (up.from_window[i]) {
+      const size_t s = static_cast<size_t>(bh) * cap + up.index[i];
+      sk = win_k + s * dk;
+      sv = win_v + s * dv;
+    } else {
+      const size_t s = static_cast<size_t>(bh) * kMaxRetained + up.index[i];
+      sk = ret_k + s * dk;
+      sv = ret_v + s * dv;
+    }
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    const bool ka = threadIdx.x < dk / 8, va = threadIdx.x < dv / 8;
+    if (ka) a = reinterpret_cast<const uint4*>(sk)[threadIdx.x];
+    if (va) b = reinterpret_cast<const uint4*>(sv)[threadIdx.x];
+    __syncthreads();
+    if (ka) reinterpret_cast<uint4*>(ret_k + dst * dk)[threadIdx.x] = a;
+    if (va) reinterpret_cast<uint4*>(ret_v + dst * dv)[threadIdx.x] = b;
+    __syncthreads();
+  }
+}
+
+inline int grid_for(long long items, int block) {
+  long long g = (items + block - 1) / block;
+  if (g > 148LL * 32) g = 148LL * 32;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
+                                 int n_groups, uint32_t* kcode, __half2* ksz, cudaStream_t s) {
+  if (n_groups <= 0) return cudaSuccess;
+  const int gpb = d.dk >= 256 ? 1 : 256 / d.dk;
+  dim3 block(d.dk, gpb);
+  dim3 grid((n_groups + gpb - 1) / gpb, d.B * d.Hkv);
+  switch (d.kb) {
+    case 2: quantize_keys_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz); break;
+    case 4: quantize_keys_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz); break;
+    case 8: quantize_keys_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_rows, int t_begin,
+                                   int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s) {
+  if (n_tokens <= 0) return cudaSuccess;
+  const int nbh = d.B * d.Hkv;
+  const long long items = static_cast<long long>(nbh) * n_tokens * d.nvg;
+  const int block = 256;
+  const int grid = grid_for(items, block);
+  switch (d.vb) {
+    case 2: quantize_values_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
+    case 4: quantize_values_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
+    case 8: quantize_values_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,
+                             int dst_rows, int dst_base, int n, int d, int nbh, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const long long items = static_cast<long long>(nbh) * n * (d / 8);
+  const int block = 256;
+  copy_rows_kernel<<<grid_for(items, block), block, 0, s>>>(src, src_rows, src_base, dst, dst_rows,
+                                                            dst_base, n, d, nbh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_copy_retained(const Dims& d, const __half* k, const __half* v, int L,
+                                 const RetList& ret, __half* ret_k, __half* ret_v, cudaStream_t s) {
+  if (ret.n <= 0) return cudaSuccess;
+  copy_retained_kernel<<<d.B * d.Hkv, 64, 0, s>>>(k, v, L, d.dk, d.dv, ret, ret_k, ret_v);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_update_retained(const Dims& d, const RetUpdate& up, __half* win_k,
+                                   __half* win_v, __half* ret_k, __half* ret_v, cudaStream_t s) {
+  if (up.n <= 0) return cudaSuccess;
+  const int threads = ((d.dk > d.dv ? d.dk : d.dv) / 8 + 31) / 32 * 32;
+  update_retained_kernel<<<d.B * d.Hkv, threads, 0, s>>>(up, d.cap, d.dk, d.dv, win_k, win_v,
+                                                          ret_k, ret_v);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

@@ -1,0 +1,297 @@
+"""Python binding of libkvq (ctypes): argument marshalling only.
+
+Every computation runs in the library's CUDA kernels; PyTorch only provides
+device memory (``torch.empty`` buffers) and the current CUDA stream.  The
+functions keep the C names (``kvq_quantize_prefill`` ...); ``KVCache`` bundles
+the buffers and the handle for convenience.  Loading fails loudly when the
+library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+KVQ_OK = 0
+KVQ_ERR_INVALID_ARG = -1
+KVQ_ERR_UNSUPPORTED = -2
+KVQ_ERR_ALIGN = -3
+KVQ_ERR_CAPACITY = -4
+KVQ_ERR_WORKSPACE = -5
+KVQ_ERR_STATE = -6
+KVQ_ERR_CUDA = -7
+KVQ_MAX_RETAINED = 32
+KVQ_STATUS_TIMEOUT = 1
+
+CONFIG_FIELDS = ("batch", "n_q_heads", "n_kv_heads", "d_k", "d_v", "k_bits", "v_bits", "group_k",
+                 "group_v", "window", "log_retain", "max_context")
+BUFFER_FIELDS = ("kcode", "ksz", "vcode", "vsz", "win_k", "win_v", "ret_k", "ret_v")
+
+
+class kvq_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in CONFIG_FIELDS]
+
+
+class kvq_sizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in BUFFER_FIELDS + ("workspace",)]
+
+
+class kvq_buffers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_FIELDS]
+
+
+class kvq_plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("splits_quant", "splits_fp16", "n_groups", "n_fp16",
+                                            "fast_path")]
+
+
+class KVQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {kvq_strerror(code)} ({code})")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+# name -> (restype, argtypes)
+_SIGNATURES = {
+    "kvq_buffer_sizes": (_I, [ctypes.POINTER(kvq_config), ctypes.POINTER(kvq_sizes)]),
+    "kvq_cache_init": (_I, [ctypes.POINTER(kvq_config), ctypes.POINTER(kvq_buffers),
+                            ctypes.POINTER(_P)]),
+    "kvq_cache_destroy": (None, [_P]),
+    "kvq_quantize_prefill": (_I, [_P, _P, _P, _I, _P]),
+    "kvq_append": (_I, [_P, _P, _P, _P]),
+    "kvq_decode_workspace_size": (_I, [_P, _I, ctypes.POINTER(ctypes.c_size_t)]),
+    "kvq_decode_attention": (_I, [_P, _P, _P, _P, ctypes.c_size_t, _I, _P]),
+    "kvq_get_plan": (_I, [_P, _I, ctypes.POINTER(kvq_plan)]),
+    "kvq_plan_decode": (_I, [ctypes.POINTER(kvq_config), _I, _I, _I, ctypes.POINTER(kvq_plan)]),
+    "kvq_get_state": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
+                           ctypes.POINTER(_I)]),
+    "kvq_retained_positions": (_I, [_I, ctypes.POINTER(_I), _I]),
+    "kvq_reset_status": (_I, [_P, _P]),
+    "kvq_read_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint), _P]),
+    "kvq_strerror": (ctypes.c_char_p, [_I]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libkvq.so not found at {LIB_PATH}; build it with "
+                               "`python -m mixed_precision_quantized_pack_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(rc: int, where: str) -> int:
+    if rc < 0:
+        raise KVQError(rc, where)
+    return rc
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_config(cfg: Dict[str, int]) -> kvq_config:
+    return kvq_config(*[int(cfg[n]) for n in CONFIG_FIELDS])
+
+
+# ---- the C entry points, same names -----------------------------------------
+def kvq_strerror(code: int) -> str:
+    return lib().kvq_strerror(int(code)).decode()
+
+
+def kvq_buffer_sizes(cfg: Dict[str, int]) -> Dict[str, int]:
+    out = kvq_sizes()
+    _check(lib().kvq_buffer_sizes(ctypes.byref(make_config(cfg)), ctypes.byref(out)),
+           "kvq_buffer_sizes")
+    return {n: int(getattr(out, n)) for n in BUFFER_FIELDS + ("workspace",)}
+
+
+def kvq_plan_decode(cfg: Dict[str, int], L: int, sm_count: int, num_splits: int = 0) -> Dict[str, int]:
+    out = kvq_plan()
+    _check(lib().kvq_plan_decode(ctypes.byref(make_config(cfg)), int(L), int(sm_count),
+                                 int(num_splits), ctypes.byref(out)), "kvq_plan_decode")
+    return {n: int(getattr(out, n)) for n, _ in kvq_plan._fields_}
+
+
+def kvq_retained_positions(Q: int) -> List[int]:
+    buf = (ctypes.c_int * KVQ_MAX_RETAINED)()
+    n = _check(lib().kvq_retained_positions(int(Q), buf, KVQ_MAX_RETAINED), "kvq_retained_positions")
+    return [int(buf[i]) for i in range(n)]
+
+
+def kvq_cache_init(cfg: Dict[str, int], ptrs: Dict[str, int]) -> int:
+    bufs = kvq_buffers(*[ptrs.get(n) or None for n in BUFFER_FIELDS])
+    h = _P()
+    _check(lib().kvq_cache_init(ctypes.byref(make_config(cfg)), ctypes.byref(bufs), ctypes.byref(h)),
+           "kvq_cache_init")
+    return h.value
+
+
+def kvq_cache_destroy(handle: int) -> None:
+    lib().kvq_cache_destroy(handle)
+
+
+def kvq_quantize_prefill(handle: int, k_ptr: int, v_ptr: int, L: int, stream: int) -> None:
+    _check(lib().kvq_quantize_prefill(handle, k_ptr, v_ptr, int(L), stream), "kvq_quantize_prefill")
+
+
+def kvq_append(handle: int, k_ptr: int, v_ptr: int, stream: int) -> None:
+    _check(lib().kvq_append(handle, k_ptr, v_ptr, stream), "kvq_append")
+
+
+def kvq_decode_workspace_size(handle: int, num_splits: int = 0) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().kvq_decode_workspace_size(handle, int(num_splits), ctypes.byref(n)),
+           "kvq_decode_workspace_size")
+    return int(n.value)
+
+
+def kvq_decode_attention(handle: int, q_ptr: int, out_ptr: int, ws_ptr: int, ws_bytes: int,
+                         num_splits: int, stream: int) -> None:
+    _check(lib().kvq_decode_attention(handle, q_ptr, out_ptr, ws_ptr, int(ws_bytes),
+                                      int(num_splits), stream), "kvq_decode_attention")
+
+
+def kvq_get_plan(handle: int, num_splits: int = 0) -> Dict[str, int]:
+    out = kvq_plan()
+    _check(lib().kvq_get_plan(handle, int(num_splits), ctypes.byref(out)), "kvq_get_plan")
+    return {n: int(getattr(out, n)) for n, _ in kvq_plan._fields_}
+
+
+def kvq_get_state(handle: int) -> Tuple[int, int, List[int]]:
+    L, Q, n = _I(), _I(), _I()
+    idx = (ctypes.c_int * KVQ_MAX_RETAINED)()
+    _check(lib().kvq_get_state(handle, ctypes.byref(L), ctypes.byref(Q), ctypes.byref(n), idx),
+           "kvq_get_state")
+    return L.value, Q.value, [int(idx[i]) for i in range(n.value)]
+
+
+def kvq_reset_status(ws_ptr: int, stream: int) -> None:
+    _check(lib().kvq_reset_status(ws_ptr, stream), "kvq_reset_status")
+
+
+def kvq_read_status(ws_ptr: int, stream: int) -> int:
+    st = ctypes.c_uint()
+    _check(lib().kvq_read_status(ws_ptr, ctypes.byref(st), stream), "kvq_read_status")
+    return int(st.value)
+
+
+# ---- convenience: buffers + handle over torch tensors ------------------------
+def _fp16_cuda(t: torch.Tensor, shape, name: str) -> torch.Tensor:
+    if t.dtype != torch.float16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: need a contiguous CUDA fp16 tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+    return t
+
+
+class KVCache:
+    """One attention layer's packed KV cache in device memory owned by PyTorch."""
+
+    def __init__(self, cfg: Dict[str, int], device=None):
+        self.cfg = dict(cfg)
+        self.device = torch.device(device or "cuda")
+        self.sizes = kvq_buffer_sizes(self.cfg)
+        self.buffers: Dict[str, Optional[torch.Tensor]] = {}
+        for n in BUFFER_FIELDS:
+            sz = self.sizes[n]
+            self.buffers[n] = torch.zeros(sz, dtype=torch.uint8, device=self.device) if sz else None
+        ptrs = {n: (b.data_ptr() if b is not None else 0) for n, b in self.buffers.items()}
+        self.handle = kvq_cache_init(self.cfg, ptrs)
+        self.workspace = torch.empty(self.sizes["workspace"], dtype=torch.uint8, device=self.device)
+        kvq_reset_status(self.workspace.data_ptr(), _stream())
+
+    def close(self):
+        if getattr(self, "handle", None):
+            kvq_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # shapes
+    @property
+    def B(self):
+        return self.cfg["batch"]
+
+    def prefill(self, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+        c = self.cfg
+        L = k.shape[2]
+        _fp16_cuda(k, (c["batch"], c["n_kv_heads"], L, c["d_k"]), "k")
+        _fp16_cuda(v, (c["batch"], c["n_kv_heads"], L, c["d_v"]), "v")
+        kvq_quantize_prefill(self.handle, k.data_ptr(), v.data_ptr(), L, _stream(stream))
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+        c = self.cfg
+        _fp16_cuda(k_new, (c["batch"], c["n_kv_heads"], c["d_k"]), "k_new")
+        _fp16_cuda(v_new, (c["batch"], c["n_kv_heads"], c["d_v"]), "v_new")
+        kvq_append(self.handle, k_new.data_ptr(), v_new.data_ptr(), _stream(stream))
+
+    def decode(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, num_splits: int = 0,
+               stream=None) -> torch.Tensor:
+        c = self.cfg
+        _fp16_cuda(q, (c["batch"], c["n_q_heads"], c["d_k"]), "q")
+        if out is None:
+            out = torch.empty((c["batch"], c["n_q_heads"], c["d_v"]), dtype=torch.float16,
+                              device=q.device)
+        _fp16_cuda(out, (c["batch"], c["n_q_heads"], c["d_v"]), "out")
+        kvq_decode_attention(self.handle, q.data_ptr(), out.data_ptr(), self.workspace.data_ptr(),
+                             self.workspace.numel(), num_splits, _stream(stream))
+        return out
+
+    def status(self, stream=None) -> int:
+        return kvq_read_status(self.workspace.data_ptr(), _stream(stream))
+
+    def state(self) -> Tuple[int, int, List[int]]:
+        return kvq_get_state(self.handle)
+
+    def plan(self, num_splits: int = 0) -> Dict[str, int]:
+        return kvq_get_plan(self.handle, num_splits)
+
+    # typed views of the buffers, in the layouts of include/kvq.h
+    def view(self, name: str) -> torch.Tensor:
+        c = self.cfg
+        B, H, dk, dv = c["batch"], c["n_kv_heads"], c["d_k"], c["d_v"]
+        kb, vb, gk, gv = c["k_bits"], c["v_bits"], c["group_k"], c["group_v"]
+        buf = self.buffers[name]
+        if buf is None:
+            raise ValueError(f"{name} is not used by this configuration")
+        if kb == 16:
+            cap = c["max_context"]
+            lcap = cap
+        else:
+            lcap = -(-c["max_context"] // gk) * gk
+            cap = c["window"] + gk
+        shapes = {
+            "kcode": (torch.int32, (B, H, lcap, dk * kb // 32)),
+            "ksz": (torch.float16, (B, H, lcap // gk, dk, 2)),
+            "vcode": (torch.int32, (B, H, lcap, dv * vb // 32)),
+            "vsz": (torch.float16, (B, H, lcap, dv // gv, 2)),
+            "win_k": (torch.float16, (B, H, cap, dk)),
+            "win_v": (torch.float16, (B, H, cap, dv)),
+            "ret_k": (torch.float16, (B, H, KVQ_MAX_RETAINED, dk)),
+            "ret_v": (torch.float16, (B, H, KVQ_MAX_RETAINED, dv)),
+        }
+        dt, shape = shapes[name]
+        return buf.view(dt).view(shape)

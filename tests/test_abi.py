@@ -1,0 +1,140 @@
+"""Host-side checks of the C ABI: no kernel launches, so these run without a GPU."""
+import os
+import re
+
+import pytest
+
+from oracle import kvq_oracle as O
+from mixed_precision_quantized_pack_b200 import kvq as K
+from mixed_precision_quantized_pack_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(kvq_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_function():
+    lib = K.lib()
+    names = header_functions()
+    assert "kvq_decode_attention" in names and "kvq_quantize_prefill" in names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in K._SIGNATURES, f"binding lacks {n}"
+
+
+def cfg(**kw):
+    base = dict(batch=2, n_q_heads=8, n_kv_heads=2, d_k=128, d_v=128, k_bits=4, v_bits=2,
+                group_k=64, group_v=64, window=128, log_retain=1, max_context=4096)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("w", list(W.WORKLOADS.values()) +
+                         [W.sweep_workload(b, kb, vb) for b in (1, 64) for kb, vb in W.SWEEP_BITS])
+def test_buffer_sizes_match_the_oracle_layout(w):
+    c = w.kvq_config()
+    got = K.kvq_buffer_sizes(c)
+    want = O.buffer_bytes(c)
+    for n in K.BUFFER_FIELDS:
+        assert got[n] == want[n], n
+    assert got["workspace"] > 0
+
+
+def test_retention_rule_matches_the_oracle():
+    for Q in list(range(0, 600)) + [32640, 65536, 131008, (1 << 30) - 64]:
+        assert K.kvq_retained_positions(Q) == O.retained_positions(Q) if Q < 200000 else \
+            len(K.kvq_retained_positions(Q)) == 30
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(n_q_heads=6, n_kv_heads=4), K.KVQ_ERR_UNSUPPORTED),
+    (dict(n_q_heads=32, n_kv_heads=2), K.KVQ_ERR_UNSUPPORTED),       # n_rep 16
+    (dict(d_k=96), K.KVQ_ERR_UNSUPPORTED),
+    (dict(k_bits=3), K.KVQ_ERR_UNSUPPORTED),
+    (dict(k_bits=16, v_bits=2), K.KVQ_ERR_UNSUPPORTED),
+    (dict(group_k=48), K.KVQ_ERR_UNSUPPORTED),
+    (dict(group_v=24), K.KVQ_ERR_UNSUPPORTED),
+    (dict(group_v=8, v_bits=2), K.KVQ_ERR_UNSUPPORTED),              # word spans two groups
+    (dict(batch=0), K.KVQ_ERR_INVALID_ARG),
+    (dict(window=-1), K.KVQ_ERR_INVALID_ARG),
+    (dict(log_retain=2), K.KVQ_ERR_INVALID_ARG),
+    (dict(max_context=0), K.KVQ_ERR_INVALID_ARG),
+])
+def test_invalid_configurations_are_rejected(bad, code):
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_buffer_sizes(cfg(**bad))
+    assert e.value.code == code
+
+
+def test_misaligned_buffers_are_rejected_before_any_device_call():
+    c = cfg()
+    ptrs = {n: 4096 * (i + 1) for i, n in enumerate(K.BUFFER_FIELDS)}
+    ptrs["vsz"] += 8
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_cache_init(c, ptrs)
+    assert e.value.code == K.KVQ_ERR_ALIGN
+    ptrs = {n: 4096 * (i + 1) for i, n in enumerate(K.BUFFER_FIELDS)}
+    ptrs["ret_k"] = 0
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_cache_init(c, ptrs)
+    assert e.value.code == K.KVQ_ERR_INVALID_ARG
+
+
+def test_null_arguments_are_errors_not_crashes():
+    lib = K.lib()
+    assert lib.kvq_quantize_prefill(None, None, None, 1, None) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_append(None, None, None, None) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_decode_attention(None, None, None, None, 0, 0, None) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_get_state(None, None, None, None, None) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_reset_status(None, None) == K.KVQ_ERR_INVALID_ARG
+    lib.kvq_cache_destroy(None)
+
+
+def test_strerror_covers_every_code():
+    codes = [K.KVQ_OK, K.KVQ_ERR_INVALID_ARG, K.KVQ_ERR_UNSUPPORTED, K.KVQ_ERR_ALIGN,
+             K.KVQ_ERR_CAPACITY, K.KVQ_ERR_WORKSPACE, K.KVQ_ERR_STATE, K.KVQ_ERR_CUDA]
+    msgs = [K.kvq_strerror(c) for c in codes]
+    assert len(set(msgs)) == len(msgs) and "unknown" in K.kvq_strerror(-99)
+
+
+@pytest.mark.parametrize("key", list(W.WORKLOADS))
+def test_planner_covers_the_work(key):
+    w = W.WORKLOADS[key]
+    c = w.kvq_config()
+    L = w.context + w.appends
+    Q = O.quantized_prefix(L, w.window, w.group_k, w.k_bits)
+    nret = len(O.retained_positions(Q)) if w.log_retain else 0
+    for sms in (1, 148):
+        for req in (0, 1, 3, 1000):
+            p = K.kvq_plan_decode(c, L, sms, req)
+            assert p["n_groups"] == Q // w.group_k
+            assert p["n_fp16"] == nret + L - Q
+            assert 1 <= p["splits_quant"] <= max(1, p["n_groups"])
+            assert 1 <= p["splits_fp16"] <= p["n_fp16"]
+            if req:
+                assert p["splits_quant"] == min(req, p["n_groups"], p["splits_quant"] if req == 1000 else req)
+            ws = K.kvq_buffer_sizes(c)["workspace"]
+            rows = w.batch * w.n_q_heads * (p["splits_quant"] + p["splits_fp16"])
+            assert ws >= 256 + rows * 8 + rows * w.d_v * 4
+
+
+def test_planner_unquantized_cache_splits_the_fp16_tokens():
+    w = W.sweep_workload(1, 16, 16)
+    p = K.kvq_plan_decode(w.kvq_config(), 131072, 148, 0)
+    assert p["n_groups"] == 0 and p["splits_quant"] == 0
+    assert p["n_fp16"] == 131072 and p["splits_fp16"] > 8
+
+
+def test_planner_rejects_lengths_outside_the_cache():
+    c = cfg(max_context=1000)
+    for L in (0, 1001):
+        with pytest.raises(K.KVQError):
+            K.kvq_plan_decode(c, L, 148, 0)

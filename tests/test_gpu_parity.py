@@ -1,0 +1,236 @@
+"""CUDA path vs the CPU oracle, through the C ABI.
+
+Packed codes, (scale, zero) pairs, window slots, retained tokens and retained
+positions must match the oracle bit for bit; attention outputs must be within
+2e-3 of the oracle's fp64 result, measured per (b, query head) as
+max_c |o - o*| / max_c |o*|.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import kvq_oracle as O
+from mixed_precision_quantized_pack_b200 import kvq as K
+from mixed_precision_quantized_pack_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def np16(t):
+    return t.detach().cpu().numpy()
+
+
+def compare_state(gc: K.KVCache, oc: O.OracleCache, b_rows=None, where=""):
+    """Bit-exact comparison of every valid byte of the cache, rows b in b_rows."""
+    L, Q, ret = gc.state()
+    assert (L, Q, ret) == (oc.L, oc.Q, oc.ret_idx), where
+    rows = list(range(gc.B)) if b_rows is None else list(b_rows)
+    c = gc.cfg
+    if c["k_bits"] != 16 and Q:
+        gk = c["group_k"]
+        pairs = [("kcode", slice(0, Q)), ("ksz", slice(0, Q // gk)), ("vcode", slice(0, Q)),
+                 ("vsz", slice(0, Q))]
+        for name, sl in pairs:
+            g = gc.view(name)[rows][:, :, sl].cpu().numpy()
+            o = getattr(oc, name)[:, :, sl]
+            if b_rows is None:
+                o = o[rows]
+            assert np.array_equal(g.view(np.uint8), np.ascontiguousarray(o).view(np.uint8)), \
+                f"{where}: {name} differs"
+    slots = [p % oc.cap for p in range(Q, L)]
+    for name in ("win_k", "win_v"):
+        g = gc.view(name)[rows][:, :, slots].cpu().numpy()
+        o = getattr(oc, name)[:, :, slots]
+        if b_rows is None:
+            o = o[rows]
+        assert np.array_equal(g.view(np.uint16), o.view(np.uint16)), f"{where}: {name} differs"
+    if ret:
+        n = len(ret)
+        for name in ("ret_k", "ret_v"):
+            g = gc.view(name)[rows][:, :, :n].cpu().numpy()
+            o = getattr(oc, name)[:, :, :n]
+            if b_rows is None:
+                o = o[rows]
+            assert np.array_equal(g.view(np.uint16), o.view(np.uint16)), f"{where}: {name} differs"
+
+
+def run_small(w: W.Workload, num_splits=(0,), steps=None):
+    """Prefill + (appends) + decodes of a workload small enough for the full oracle."""
+    need_gpu()
+    inp = W.Inputs(w, device="cpu")
+    cfg = w.kvq_config()
+    gc = K.KVCache(cfg)
+    oc = O.OracleCache(cfg)
+    gc.prefill(inp.k.cuda(), inp.v.cuda())
+    oc.prefill(np16(inp.k), np16(inp.v))
+    compare_state(gc, oc, where="prefill")
+    worst = 0.0
+    n_dec = len(inp.q)
+    for i in range(n_dec):
+        if w.appends:
+            gc.append(inp.k_app[i].cuda(), inp.v_app[i].cuda())
+            oc.append(np16(inp.k_app[i]), np16(inp.v_app[i]))
+        if steps is not None and i not in steps:
+            continue
+        compare_state(gc, oc, where=f"step {i}")
+        ref = oc.decode(np16(inp.q[i]))
+        for s in num_splits:
+            out = gc.decode(inp.q[i].cuda(), num_splits=s)
+            err = O.max_rel_error(out.float().cpu().numpy(), ref)
+            worst = max(worst, err)
+            assert err <= TOL, f"step {i} splits {s}: max rel error {err:.3e}"
+    assert gc.status() == 0
+    return worst
+
+
+def test_tiny_single_head():
+    run_small(W.WORKLOADS["tiny"], num_splits=(0, 1, 2, 5))
+
+
+def test_gqa_4k_with_append():
+    run_small(W.WORKLOADS["gqa4k"], num_splits=(0, 1, 3))
+
+
+def test_thin_keys_16k():
+    run_small(W.WORKLOADS["thin16k"].with_(batch=2), num_splits=(0, 1))
+
+
+@pytest.mark.parametrize("kb,vb", [(8, 4), (4, 2), (2, 2), (4, 4), (8, 8), (2, 4)])
+def test_bit_widths(kb, vb):
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=1500, k_bits=kb, v_bits=vb, appends=70,
+                                   log_retain=1, seed=77)
+    run_small(w, num_splits=(0, 2), steps={0, 1, 57, 58, 69})
+
+
+def test_unquantized_fp16_cache():
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=3000, k_bits=16, v_bits=16, appends=3,
+                                   seed=78)
+    run_small(w, num_splits=(0, 1, 4))
+
+
+@pytest.mark.parametrize("n_q,n_kv", [(8, 8), (16, 8), (64, 8)])
+def test_gqa_group_sizes(n_q, n_kv):
+    w = W.WORKLOADS["gqa4k"].with_(batch=1, n_q_heads=n_q, n_kv_heads=n_kv, context=777, seed=79)
+    run_small(w, num_splits=(0, 1))
+
+
+@pytest.mark.parametrize("gk,gv,R", [(16, 16, 0), (32, 128, 32), (128, 64, 5), (64, 32, 300)])
+def test_group_sizes_and_windows(gk, gv, R):
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=1111, group_k=gk, group_v=gv, window=R,
+                                   log_retain=1, appends=2 * gk + 3, seed=80 + gk)
+    run_small(w, num_splits=(0, 3), steps={0, gk - 1, gk, 2 * gk + 2})
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64), (256, 256), (32, 32)])
+def test_head_dims(dk, dv):
+    w = W.WORKLOADS["gqa4k"].with_(batch=1, n_q_heads=8, n_kv_heads=2, d_k=dk, d_v=dv,
+                                   context=900, group_v=32, seed=81)
+    run_small(w, num_splits=(0,))
+
+
+@pytest.mark.parametrize("L", [1, 5, 127, 128, 129, 191, 192, 193, 256])
+def test_short_contexts(L):
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=L, appends=0, log_retain=1, seed=90 + L)
+    run_small(w, num_splits=(0, 1))
+
+
+def test_split_invariance():
+    need_gpu()
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=6000, log_retain=1, seed=91)
+    inp = W.Inputs(w)
+    gc = K.KVCache(w.kvq_config())
+    gc.prefill(inp.k.cuda(), inp.v.cuda())
+    q = inp.q[0].cuda()
+    outs = [gc.decode(q, num_splits=s).float() for s in (1, 2, 3, 7, 16, 0)]
+    for o in outs[1:]:
+        assert (o - outs[0]).abs().max().item() <= 2e-3 * outs[0].abs().max().item()
+
+
+def test_error_paths():
+    need_gpu()
+    w = W.WORKLOADS["tiny"].with_(context=100)
+    gc = K.KVCache(w.kvq_config(max_context=101))
+    q = torch.zeros((1, 1, 128), dtype=torch.float16, device="cuda")
+    with pytest.raises(K.KVQError) as e:
+        gc.decode(q)
+    assert e.value.code == K.KVQ_ERR_STATE
+    kv = torch.zeros((1, 1, 128), dtype=torch.float16, device="cuda")
+    with pytest.raises(K.KVQError) as e:
+        gc.append(kv, kv)
+    assert e.value.code == K.KVQ_ERR_STATE
+    inp = W.Inputs(w)
+    gc.prefill(inp.k.cuda(), inp.v.cuda())
+    gc.append(kv, kv)
+    with pytest.raises(K.KVQError) as e:
+        gc.append(kv, kv)
+    assert e.value.code == K.KVQ_ERR_CAPACITY
+    need = K.kvq_decode_workspace_size(gc.handle, 0)
+    out = torch.empty((1, 1, 128), dtype=torch.float16, device="cuda")
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_decode_attention(gc.handle, q.data_ptr(), out.data_ptr(), gc.workspace.data_ptr(),
+                               need - 1, 0, K._stream())
+    assert e.value.code == K.KVQ_ERR_WORKSPACE
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_decode_attention(gc.handle, q.data_ptr() + 2, out.data_ptr(),
+                               gc.workspace.data_ptr(), need, 0, K._stream())
+    assert e.value.code == K.KVQ_ERR_ALIGN
+    with pytest.raises(K.KVQError) as e:
+        gc.prefill(inp.k.cuda()[:, :, :0], inp.v.cuda()[:, :, :0])
+    assert e.value.code == K.KVQ_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------- full sizes ----
+def sampled_full_size(w: W.Workload, rows, steps=(0,)):
+    """Full-size workload on the GPU; the oracle recomputes sampled sequences b."""
+    need_gpu()
+    inp = W.Inputs(w, device="cuda")
+    gc = K.KVCache(w.kvq_config())
+    gc.prefill(inp.k, inp.v)
+    ocs = {}
+    for b in rows:
+        sub = dict(w.kvq_config(), batch=1)
+        oc = O.OracleCache(sub)
+        oc.prefill(np16(inp.k[b:b + 1]), np16(inp.v[b:b + 1]))
+        ocs[b] = oc
+    n_dec = len(inp.q)
+    for i in range(n_dec):
+        if w.appends:
+            gc.append(inp.k_app[i], inp.v_app[i])
+            for b, oc in ocs.items():
+                oc.append(np16(inp.k_app[i][b:b + 1]), np16(inp.v_app[i][b:b + 1]))
+        if i not in steps:
+            continue
+        out = gc.decode(inp.q[i]).float().cpu().numpy()
+        for b, oc in ocs.items():
+            compare_state(gc, oc, b_rows=[b], where=f"b={b} step {i}")
+            ref = oc.decode(np16(inp.q[i][b:b + 1]))
+            err = O.max_rel_error(out[b:b + 1], ref)
+            assert err <= TOL, f"b={b} step {i}: {err:.3e}"
+    assert gc.status() == 0
+    del gc, inp
+    torch.cuda.empty_cache()
+
+
+def test_full_size_long_32k_logretain():
+    w = W.WORKLOADS["long32k"]
+    sampled_full_size(w, rows=(0, 31))
+
+
+def test_full_size_gqa_4k():
+    sampled_full_size(W.WORKLOADS["gqa4k"], rows=(3,))
+
+
+def test_full_size_thin_16k():
+    sampled_full_size(W.WORKLOADS["thin16k"], rows=(0, 15))
+
+
+@pytest.mark.parametrize("kb,vb", [(4, 2), (16, 16)])
+def test_full_size_sweep_point_131k(kb, vb):
+    w = W.sweep_workload(8, kb, vb, appends=66)
+    sampled_full_size(w, rows=(5,), steps=(0, 63, 64, 65))
