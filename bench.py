@@ -129,12 +129,27 @@ def profile_traffic():
     if not m or not h:
         return None
     import hashlib
-    src = os.path.join(ROOT, "mixed_precision_quantized_pack_b200", "csrc", "decode_mma.cu")
+    src = os.path.join(ROOT, "mixed_precision_quantized_pack_b200", "csrc", "decode_mma.cuh")
     try:
         cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
     except OSError:
         return None
     return float(m.group(1)) if cur.startswith(h.group(1)) else None
+
+
+# ------------------------------------------------------------------ ranks ---------
+def rank_workload(w: W.Workload, rank: int, steps: int) -> W.Workload:
+    """The batch a rank decodes: same shapes, its own seed (independent sequences)."""
+    return w.with_(appends=steps, seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (identity without a group)."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
 
 
 # ------------------------------------------------------------------ CPU oracle ----
@@ -200,10 +215,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default="long32k", choices=list(W.WORKLOADS))
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.with_(batch=args.batch)
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -219,7 +237,7 @@ def main():
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     steps, warm = args.steps, max(args.warmup, 3)
-    wl = w.with_(appends=steps + warm, seed=w.seed + 7919 * rank)
+    wl = rank_workload(w, rank, steps + warm)
     cfg = wl.kvq_config(max_context=wl.context + steps + warm + 64)
     inp = W.Inputs(wl, device=dev)
     cache = K.KVCache(cfg, device=dev)
@@ -277,10 +295,7 @@ def main():
     dec_ms = [starts[i].elapsed_time(ends[i]) for i in range(warm, warm + steps)]
     dec_avg = sum(dec_ms) / len(dec_ms)
     status = cache.status()
-    if dist:
-        t = torch.tensor([total_ms, dec_avg], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, dec_avg = float(t[0]), float(t[1])
+    total_ms, dec_avg = max_over_ranks([total_ms, dec_avg], dist, dev)
     ms_step = total_ms / steps
     value = world * wl.batch / (ms_step / 1e3)
     achieved = (sum(bytes_read) / len(bytes_read)) / (dec_avg / 1e3) / 1e9
@@ -322,10 +337,7 @@ def main():
     b.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = a.elapsed_time(b) / max(n_e2e, 1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
+    (e2e_ms,) = max_over_ranks([e2e_ms], dist, dev)
     h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
     d2h = out.numel() * 2
 

@@ -146,6 +146,14 @@ int kvq_decode_workspace_size(const kvq_cache* cache, int num_splits, size_t* by
 int kvq_decode_attention(kvq_cache* cache, const void* q, void* out, void* workspace,
                          size_t workspace_bytes, int num_splits, void* stream);
 
+/* Decode kernel selection for a cache (default KVQ_KERNEL_AUTO: the tensor-core
+ * kernel where it is built for the shape, else the generic CUDA-core kernel).
+ * KVQ_KERNEL_TENSOR fails with UNSUPPORTED on shapes it is not built for. */
+#define KVQ_KERNEL_AUTO     0
+#define KVQ_KERNEL_GENERIC  1
+#define KVQ_KERNEL_TENSOR   2
+int kvq_set_decode_kernel(kvq_cache* cache, int kernel);
+
 /* The plan kvq_decode_attention would use now (host only, no launch). */
 int kvq_get_plan(const kvq_cache* cache, int num_splits, kvq_plan* out);
 

@@ -1,13 +1,52 @@
-// Tensor-core decode kernel (placeholder until the fragment-level kernel lands).
-#include "kvq_internal.cuh"
+// Dispatch of the tensor-core decode kernel: a table of the built instances.
+#include "decode_mma.cuh"
+#include "decode_mma_instances.h"
 
 namespace kvq {
+namespace mma {
+#define KVQ_DECL_Q(KB, VB, DK, NREP, GV)                                                     \
+  extern template cudaError_t launch<KB, VB, DK, NREP, GV, 2, true>(                        \
+      const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
+      cudaStream_t);
+#define KVQ_DECL_F(DK, NREP)                                                                 \
+  extern template cudaError_t launch<4, 2, DK, NREP, 64, 2, false>(                         \
+      const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
+      cudaStream_t);
+KVQ_MMA_QUANT_INSTANCES(KVQ_DECL_Q)
+KVQ_MMA_FP16_INSTANCES(KVQ_DECL_F)
+}  // namespace mma
 
-bool decode_mma_supported(const Dims&) { return false; }
+namespace {
 
-cudaError_t launch_decode_mma(const Dims&, const CacheBufs&, const DecodeWork&, const __half*,
-                              const Partials&, cudaStream_t) {
-  return cudaErrorNotSupported;
+using LaunchFn = cudaError_t (*)(const Dims&, const CacheBufs&, const DecodeWork&, const __half*,
+                                 const Partials&, cudaStream_t);
+struct Entry {
+  int kb, vb, dk, nrep, gv;
+  LaunchFn fn;
+};
+
+#define KVQ_ENTRY_Q(KB, VB, DK, NREP, GV) {KB, VB, DK, NREP, GV, &mma::launch<KB, VB, DK, NREP, GV, 2, true>},
+#define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, &mma::launch<4, 2, DK, NREP, 64, 2, false>},
+const Entry kTable[] = {KVQ_MMA_QUANT_INSTANCES(KVQ_ENTRY_Q) KVQ_MMA_FP16_INSTANCES(KVQ_ENTRY_F)};
+
+LaunchFn find(const Dims& d) {
+  if (d.dv != 128) return nullptr;
+  const int gv = d.quantized() ? d.gv : 0;
+  if (d.quantized() && (d.gk < 16 || d.gk > 128 || d.gk % 16 != 0)) return nullptr;
+  for (const Entry& e : kTable)
+    if (e.kb == d.kb && e.vb == d.vb && e.dk == d.dk && e.nrep == d.n_rep && e.gv == gv) return e.fn;
+  return nullptr;
+}
+
+}  // namespace
+
+bool decode_mma_supported(const Dims& d) { return find(d) != nullptr; }
+
+cudaError_t launch_decode_mma(const Dims& d, const CacheBufs& c, const DecodeWork& w,
+                              const __half* q, const Partials& p, cudaStream_t s) {
+  LaunchFn fn = find(d);
+  if (!fn) return cudaErrorNotSupported;
+  return fn(d, c, w, q, p, s);
 }
 
 }  // namespace kvq

@@ -1,0 +1,705 @@
+// Fused dequant + split-K flash-decoding kernel on the tensor cores (sm_100a).
+//
+// One CTA = 4 warps = one split of one (b, kv head).  Splits [0, splits_q) cover
+// whole key groups of the quantized prefix; splits [splits_q, splits) cover the
+// fp16 list (retained tokens, then the window).  Token order is free
+// ("LogQuant: Log-Distributed 2-Bit Quantization of KV Cache", §4), so the two
+// kinds of tokens are visited separately and merged by the log-sum-exp combine.
+//
+// Each warp streams its own units (a key group, or 16 fp16 rows) through a ring
+// of NS shared-memory stages filled by 1-D bulk copies (cp.async.bulk) that
+// complete on a per-stage mbarrier.  Waits are bounded (1 s of globaltimer); on
+// timeout the warp sets KVQ_STATUS_TIMEOUT in the workspace status word, drains
+// its copies (again bounded) and contributes nothing.
+//
+// Scores ("HeadQ", §2.1: s_j = q.k_j/sqrt(d); "Thin Keys, Full Values", §2: d = d_k)
+// use mma.m16n8k16 with the tokens of a 16-token tile on M and, on N, the GQA
+// query heads sharing the kv head, each twice: column 2h holds hi(q'_h), column
+// 2h+1 holds lo(q'_h), where q'_c = q_c * s_{g,c} folds the per-channel key scale
+// into the query once per group and hi/lo are the two fp16 halves of the exact
+// fp32 product (hi + lo == q'_c).  The key codes enter the MMA unconverted: a
+// b-bit field masked in place inside a 16-bit lane is an fp16 subnormal of value
+// code * 2^(p-24), p its bit offset (p + b <= 8 after at most one byte shift), so
+// unpacking is one AND per two codes; the factor 2^-p goes into q' and the common
+// 2^-24 into the softmax scale.  The zero points add sum_c q_c z_{g,c} per group,
+// computed by one more MMA per k-step with z in A and q in B.
+//
+// p.V uses the transposed orientation: channels on M, the 16 tokens on K, and on
+// N again (hi, lo) pairs, now of p_j * s_{j,g} (per-token value scale), moved from
+// the score accumulator layout to the B layout with movmatrix.  Value codes are
+// masked as subnormals too; their 2^(p-24) factors are per output channel and are
+// removed once at the end, where sum_j p_j z_{j,g} is added.
+#pragma once
+
+#include "../../include/kvq.h"
+#include "kvq_internal.cuh"
+#include "ptx.cuh"
+
+namespace kvq {
+namespace mma {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr int kDV = 128;
+
+// ---------------------------------------------------------------- geometry ----
+template <int KB, int VB, int DK, int GV>
+struct Quant {
+  static constexpr int KW = DK * KB / 32;            // u32 words per key row
+  static constexpr int VW = kDV * VB / 32;           // u32 words per value row
+  static constexpr int WPT = KW / 4;                 // key words per thread (a quad shares a row)
+  static constexpr int KSTEPS = DK / 16;
+  static constexpr int RPW = 16 / KB;                // A registers per key word
+  static constexpr int KSPW = RPW / 2;               // k-steps per key word
+  static constexpr int CPW = 32 / KB;                // channels per key word
+  static constexpr int NVG = kDV / GV;               // value groups per token
+  static constexpr int MPG = GV / 16;                // value m-tiles per value group
+  static constexpr int CPG = GV / 8;                 // channels a thread owns per value group
+  static constexpr int RUN = CPG * VB;               // bits of that run in a value row
+  static constexpr int KBYTES_ROW = DK * KB / 8;
+  static constexpr int VBYTES_ROW = kDV * VB / 8;
+  static_assert(WPT >= 1 && KSTEPS == WPT * KSPW, "key row too short for the fragment mapping");
+  static_assert(RUN == 8 || RUN == 16 || RUN == 32, "value run must be 8, 16 or 32 bits");
+  static_assert(MPG >= 1, "value group below 16 channels");
+};
+
+template <int DK>
+struct Raw {
+  static constexpr int KST = DK * 2 + 16;            // padded row strides in shared memory
+  static constexpr int VST = kDV * 2 + 16;
+  static constexpr int BYTES = 16 * (KST + VST);
+  static constexpr int KSTEPS = DK / 16;
+};
+
+// fp16 mantissa-field masks: the `bits`-wide field at bit `pos` of both 16-bit halves.
+template <int BITS, int POS>
+struct Mask {
+  static constexpr uint32_t v = (((1u << BITS) - 1u) << POS) * 0x00010001u;
+};
+
+// Register rho of a key word: the pair (channel c, channel c + 16/KB) as subnormals
+// with factor 2^(p-24), p = (KB * rho) mod 8.
+template <int KB>
+__device__ __forceinline__ void unpack_key_word(uint32_t w, uint32_t (&r)[16 / KB]) {
+  if constexpr (KB == 4) {
+    const uint32_t u = w >> 8;
+    r[0] = w & Mask<4, 0>::v;
+    r[1] = w & Mask<4, 4>::v;
+    r[2] = u & Mask<4, 0>::v;
+    r[3] = u & Mask<4, 4>::v;
+  } else if constexpr (KB == 2) {
+    const uint32_t u = w >> 8;
+    r[0] = w & Mask<2, 0>::v;
+    r[1] = w & Mask<2, 2>::v;
+    r[2] = w & Mask<2, 4>::v;
+    r[3] = w & Mask<2, 6>::v;
+    r[4] = u & Mask<2, 0>::v;
+    r[5] = u & Mask<2, 2>::v;
+    r[6] = u & Mask<2, 4>::v;
+    r[7] = u & Mask<2, 6>::v;
+  } else {
+    r[0] = w & Mask<8, 0>::v;
+    r[1] = (w >> 8) & Mask<8, 0>::v;
+  }
+}
+
+template <int KB>
+__host__ __device__ constexpr int key_reg_shift(int rho) { return (KB * rho) % 8; }
+
+// The codes of one 16-bit piece (token a in the low half, token b in the high
+// half), as subnormal pairs; code e' sits at bit VB*e' of the piece.
+template <int VB>
+__device__ __forceinline__ void unpack_value_piece16(uint32_t x, uint32_t* r) {
+  const uint32_t u = x >> 8;
+  if constexpr (VB == 2) {
+    r[0] = x & Mask<2, 0>::v;
+    r[1] = x & Mask<2, 2>::v;
+    r[2] = x & Mask<2, 4>::v;
+    r[3] = x & Mask<2, 6>::v;
+    r[4] = u & Mask<2, 0>::v;
+    r[5] = u & Mask<2, 2>::v;
+    r[6] = u & Mask<2, 4>::v;
+    r[7] = u & Mask<2, 6>::v;
+  } else if constexpr (VB == 4) {
+    r[0] = x & Mask<4, 0>::v;
+    r[1] = x & Mask<4, 4>::v;
+    r[2] = u & Mask<4, 0>::v;
+    r[3] = u & Mask<4, 4>::v;
+  } else {
+    r[0] = x & Mask<8, 0>::v;
+    r[1] = u & Mask<8, 0>::v;
+  }
+}
+
+template <int VB>
+__device__ __forceinline__ void unpack_value_piece8(uint32_t x, uint32_t* r) {
+  static_assert(VB == 2 || VB == 4 || VB == 8, "");
+  if constexpr (VB == 2) {
+    r[0] = x & Mask<2, 0>::v;
+    r[1] = x & Mask<2, 2>::v;
+    r[2] = x & Mask<2, 4>::v;
+    r[3] = x & Mask<2, 6>::v;
+  } else if constexpr (VB == 4) {
+    r[0] = x & Mask<4, 0>::v;
+    r[1] = x & Mask<4, 4>::v;
+  } else {
+    r[0] = x & Mask<8, 0>::v;
+  }
+}
+
+// Bit offset (within its fp16 lane) of code e of a thread's value run.
+template <int VB, int RUN>
+__host__ __device__ constexpr int value_code_shift(int e) {
+  return RUN == 8 ? (VB * e) % 8 : (VB * (e % (16 / VB))) % 8;
+}
+
+// N consecutive u32 from shared memory at an address aligned to min(4N, 16) bytes.
+template <int N>
+__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* out) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p + i);
+      out[i] = v.x;
+      out[i + 1] = v.y;
+      out[i + 2] = v.z;
+      out[i + 3] = v.w;
+    }
+  } else if constexpr (N == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    out[0] = v.x;
+    out[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) out[i] = p[i];
+  }
+}
+
+// --------------------------------------------------------------- the kernel ----
+struct Smem {
+  // per-CTA header, then per-warp stage rings
+  static constexpr int kQb = 0;                         // u32 [2*KSTEPS (<= 32)][32 lanes]
+  static constexpr int kBars = kQb + 32 * 32 * 4;       // u64 [kWarps][NS]
+  static constexpr int kStages = kBars + kWarps * 4 * 8;
+};
+
+struct StageLayout {
+  int k_off, kmeta_off, v_off, vmeta_off, bytes;
+};
+
+__host__ __device__ inline StageLayout quant_stage_layout(int gk, int dk, int kb, int vb, int nvg) {
+  StageLayout s;
+  s.k_off = 0;
+  s.kmeta_off = gk * dk * kb / 8;
+  s.v_off = s.kmeta_off + dk * 4;
+  s.vmeta_off = s.v_off + gk * kDV * vb / 8;
+  s.bytes = s.vmeta_off + gk * nvg * 4;
+  return s;
+}
+
+template <int KB, int VB, int DK, int NREP, int GV, int NS, bool QUANT>
+__global__ void __launch_bounds__(kThreads, 3)
+decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part,
+                  int stage_bytes) {
+  using G = Quant<(QUANT ? KB : 4), (QUANT ? VB : 2), (QUANT ? DK : 128), (QUANT ? GV : 64)>;
+  using R = Raw<DK>;
+  constexpr int KSTEPS = DK / 16;
+  extern __shared__ __align__(128) unsigned char smem[];
+
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * d.Hkv + h;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qi = lane & 3;          // quad index: C columns 2qi, 2qi+1 = head qi (hi, lo)
+  const int qr = lane >> 2;         // row group: A rows qr, qr+8; B column qr
+  const int bhead = qr >> 1;        // head of this thread's B column
+  const bool blo = (qr & 1) != 0;   // B column holds the lo half
+  const bool bvalid = bhead < NREP;
+  const bool cvalid = qi < NREP;
+  const bool quant = QUANT && split < w.splits_q;
+
+  uint32_t* sm_qb = reinterpret_cast<uint32_t*>(smem + Smem::kQb);
+  const uint32_t bar0 = ptx::smem_addr(smem + Smem::kBars) + warp * NS * 8;
+  unsigned char* my_stages = smem + Smem::kStages + warp * NS * stage_bytes;
+  const uint32_t my_stages_s = ptx::smem_addr(my_stages);
+
+  if (lane == 0) {
+    for (int s = 0; s < NS; ++s) ptx::mbar_init(bar0 + 8 * s, 1);
+    ptx::fence_barrier_init();
+  }
+  const __half* qrow = q + (static_cast<size_t>(b) * d.Hq + h * NREP + (bvalid ? bhead : 0)) * DK;
+
+  // ---------------- work list of this warp ----------------
+  int unit_begin, unit_end;      // quantized: groups; fp16: tiles of 16 list entries
+  int list_begin = 0, list_end = 0;
+  if (quant) {
+    unit_begin = static_cast<int>(static_cast<long long>(split) * w.n_groups / w.splits_q);
+    unit_end = static_cast<int>(static_cast<long long>(split + 1) * w.n_groups / w.splits_q);
+  } else {
+    const int f = split - (QUANT ? w.splits_q : 0);
+    list_begin = static_cast<int>(static_cast<long long>(f) * w.n_fp16 / w.splits_f);
+    list_end = static_cast<int>(static_cast<long long>(f + 1) * w.n_fp16 / w.splits_f);
+    unit_begin = 0;
+    unit_end = (list_end - list_begin + 15) / 16;
+  }
+  const int n_my = unit_end - unit_begin > warp ? (unit_end - unit_begin - warp + kWarps - 1) / kWarps : 0;
+
+  // running softmax state of head qi over this warp's tokens
+  float m_run = -INFINITY, l_run = 0.0f;
+  float zsum[G::NVG];
+#pragma unroll
+  for (int g = 0; g < G::NVG; ++g) zsum[g] = 0.0f;
+  float co[8][4];
+#pragma unroll
+  for (int mv = 0; mv < 8; ++mv)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) co[mv][e] = 0.0f;
+  bool failed = false;
+
+  const float alpha = w.score_scale;                       // log2(e) / sqrt(d_k)
+  const float alpha24 = w.score_scale * 16777216.0f;       // undoes the 2^-24 of subnormal codes
+
+  if (quant) {
+    if constexpr (QUANT) {
+      // B operands: q (scaled by 2^-p per k-slot) in registers, plain q in shared memory
+      uint32_t qf[KSTEPS][2];
+#pragma unroll
+      for (int s = 0; s < KSTEPS; ++s)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int omega = qi * G::WPT + s / G::KSPW;
+          const int rho = 2 * (s % G::KSPW) + j;
+          const int c_lo = G::CPW * omega + rho;
+          const int c_hi = c_lo + 16 / KB;
+          const __half2 pair = bvalid ? __halves2half2(qrow[c_lo], qrow[c_hi]) : __float2half2_rn(0.0f);
+          const float f = 1.0f / static_cast<float>(1 << key_reg_shift<KB>(rho));
+          qf[s][j] = ptx::h2_as_u32(__hmul2(pair, __float2half2_rn(f)));
+          if (warp == 0) sm_qb[(2 * s + j) * 32 + lane] = ptx::h2_as_u32(pair);
+        }
+      __syncthreads();
+
+      // retained positions, one per lane (ascending), for masking the quantized tiles
+      const int ret_pos = lane < w.ret.n ? w.ret.pos[lane] : -1;
+      const StageLayout L = quant_stage_layout(d.gk, DK, KB, VB, G::NVG);
+      const int gk = d.gk;
+      const int mtiles = gk / 16;
+      // per-lane shuffle selectors for the bank-conflict-free value-row loads
+      const bool swap = qi >= 2;
+      const uint32_t sel_lo = swap ? 0x1054u : 0x5410u;
+      const uint32_t sel_hi = swap ? 0x3276u : 0x7632u;
+
+      auto issue = [&](int k) {
+        const int g = unit_begin + warp + kWarps * k;
+        const int st = k % NS;
+        const uint32_t bar = bar0 + 8 * st;
+        const uint32_t dst = my_stages_s + st * stage_bytes;
+        ptx::mbar_arrive_expect_tx(bar, L.bytes);
+        const size_t tok = static_cast<size_t>(bh) * d.lcap + static_cast<size_t>(g) * gk;
+        ptx::bulk_g2s(dst + L.k_off, cb.kcode + tok * G::KW, gk * G::KBYTES_ROW, bar);
+        ptx::bulk_g2s(dst + L.kmeta_off, cb.ksz + (static_cast<size_t>(bh) * (d.lcap / gk) + g) * DK,
+                      DK * 4, bar);
+        ptx::bulk_g2s(dst + L.v_off, cb.vcode + tok * G::VW, gk * G::VBYTES_ROW, bar);
+        ptx::bulk_g2s(dst + L.vmeta_off, cb.vsz + tok * G::NVG, gk * G::NVG * 4, bar);
+      };
+
+      __syncwarp();
+      if (lane == 0)
+        for (int k = 0; k < NS && k < n_my; ++k) issue(k);
+
+      int k = 0;
+      for (; k < n_my; ++k) {
+        const int g = unit_begin + warp + kWarps * k;
+        const int st = k % NS;
+        const bool ok = ptx::mbar_wait_bounded(bar0 + 8 * st, (k / NS) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) {
+          failed = true;
+          break;
+        }
+        const unsigned char* S = my_stages + st * stage_bytes;
+        const uint32_t* skc = reinterpret_cast<const uint32_t*>(S + L.k_off);
+        const uint32_t* skm = reinterpret_cast<const uint32_t*>(S + L.kmeta_off);
+        const uint32_t* svc = reinterpret_cast<const uint32_t*>(S + L.v_off);
+        const uint32_t* svm = reinterpret_cast<const uint32_t*>(S + L.vmeta_off);
+
+        // ---- group prologue: B = hi or lo of q*s, and the zero-point bias ----
+        uint32_t bq[KSTEPS][2];
+        float cbias[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int u = 0; u < G::WPT; ++u) {
+          const int omega = qi * G::WPT + u;
+          uint32_t meta[G::CPW];
+#pragma unroll
+          for (int c4 = 0; c4 < G::CPW; c4 += 4) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(skm + G::CPW * omega + c4);
+            meta[c4] = v4.x;
+            meta[c4 + 1] = v4.y;
+            meta[c4 + 2] = v4.z;
+            meta[c4 + 3] = v4.w;
+          }
+          uint32_t qbx[2 * G::KSPW];
+#pragma unroll
+          for (int e = 0; e < 2 * G::KSPW; ++e) qbx[e] = sm_qb[(2 * u * G::KSPW + e) * 32 + lane];
+#pragma unroll
+          for (int ls = 0; ls < G::KSPW; ++ls) {
+            const int s = u * G::KSPW + ls;
+            uint32_t za[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int rho = 2 * ls + j;
+              const uint32_t mlo = meta[rho], mhi = meta[rho + 16 / KB];
+              const uint32_t s2 = ptx::prmt(mlo, mhi, 0x5410u);   // (s_lo, s_hi)
+              za[j] = ptx::prmt(mlo, mhi, 0x7632u);               // (z_lo, z_hi)
+              const __half2 qs = ptx::u32_as_h2(qf[s][j]);
+              const __half2 sc = ptx::u32_as_h2(s2);
+              const __half2 hi = __hmul2(qs, sc);
+              bq[s][j] = blo ? ptx::h2_as_u32(__hfma2(qs, sc, __hneg2(hi))) : ptx::h2_as_u32(hi);
+            }
+            ptx::mma_16816(cbias, za[0], za[0], za[1], za[1], qbx[2 * ls], qbx[2 * ls + 1]);
+          }
+        }
+        const float beta = cbias[0] * alpha;
+
+        // retained tokens of this group are read from the fp16 list: mask them here
+        const int g0 = g * gk;
+        const unsigned hits = __ballot_sync(0xffffffffu, ret_pos >= g0 && ret_pos < g0 + gk);
+
+        // ---- scores of the whole group ----
+        float sc[8][2];
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          if (mt < mtiles) {
+            float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const int t0 = 16 * mt + qr;
+            uint32_t w0[G::WPT], w1[G::WPT];
+            load_words<G::WPT>(skc + t0 * G::KW + qi * G::WPT, w0);
+            load_words<G::WPT>(skc + (t0 + 8) * G::KW + qi * G::WPT, w1);
+#pragma unroll
+            for (int u = 0; u < G::WPT; ++u) {
+              uint32_t r0[G::RPW], r1[G::RPW];
+              unpack_key_word<KB>(w0[u], r0);
+              unpack_key_word<KB>(w1[u], r1);
+#pragma unroll
+              for (int ls = 0; ls < G::KSPW; ++ls) {
+                const int s = u * G::KSPW + ls;
+                ptx::mma_16816(cs, r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1], bq[s][0],
+                               bq[s][1]);
+              }
+            }
+            sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
+            sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
+            if (hits) {
+              unsigned hb = hits;
+              while (hb) {
+                const int src = __ffs(hb) - 1;
+                hb &= hb - 1;
+                const int off = __shfl_sync(0xffffffffu, ret_pos, src) - g0;
+                if (off == t0) sc[mt][0] = -INFINITY;
+                if (off == t0 + 8) sc[mt][1] = -INFINITY;
+              }
+            }
+          }
+        }
+        // ---- online softmax update for the group ----
+        float gmax = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+          if (mt < mtiles) gmax = fmaxf(gmax, fmaxf(sc[mt][0], sc[mt][1]));
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 4));
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
+        const float m_new = fmaxf(m_run, gmax);
+        if (__any_sync(0xffffffffu, m_new > m_run)) {
+          const float a = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
+          l_run *= a;
+#pragma unroll
+          for (int gg = 0; gg < G::NVG; ++gg) zsum[gg] *= a;
+#pragma unroll
+          for (int mv = 0; mv < 8; ++mv)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) co[mv][e] *= a;
+        }
+        m_run = m_new;
+
+        // ---- p.V over the group ----
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          if (mt < mtiles) {
+            const int t0 = 16 * mt + qr;
+            const float p0 = cvalid && m_new != -INFINITY ? exp2f(sc[mt][0] - m_new) : 0.0f;
+            const float p1 = cvalid && m_new != -INFINITY ? exp2f(sc[mt][1] - m_new) : 0.0f;
+            l_run += p0 + p1;
+            // value (scale, zero) of the two tokens this thread weights
+            uint32_t vm0[G::NVG], vm1[G::NVG];
+            load_words<G::NVG>(svm + t0 * G::NVG, vm0);
+            load_words<G::NVG>(svm + (t0 + 8) * G::NVG, vm1);
+            // value words: tokens 2qi, 2qi+1, 2qi+8, 2qi+9 of the tile, swapped for qi >= 2
+            const int ta = 16 * mt + 2 * qi + (swap ? 1 : 0);
+            const int tb = 16 * mt + 2 * qi + (swap ? 0 : 1);
+#pragma unroll
+            for (int gg = 0; gg < G::NVG; ++gg) {
+              const float2 f0 = __half22float2(ptx::u32_as_h2(vm0[gg]));
+              const float2 f1 = __half22float2(ptx::u32_as_h2(vm1[gg]));
+              zsum[gg] = fmaf(p0, f0.y, fmaf(p1, f1.y, zsum[gg]));
+              const uint32_t x0 = ptx::split_hi_lo(p0 * f0.x);
+              const uint32_t x1 = ptx::split_hi_lo(p1 * f1.x);
+              const uint32_t bp0 = ptx::movmatrix_trans(x0);
+              const uint32_t bp1 = ptx::movmatrix_trans(x1);
+
+              const int bit0 = (gg * GV + qr * G::CPG) * VB;
+              const int wv = bit0 >> 5;
+              const int ob = bit0 & 31;
+              const uint32_t wa0 = svc[ta * G::VW + wv], wb0 = svc[tb * G::VW + wv];
+              const uint32_t wa1 = svc[(ta + 8) * G::VW + wv], wb1 = svc[(tb + 8) * G::VW + wv];
+              uint32_t ra[G::CPG], rb[G::CPG];   // codes of tokens (2qi, 2qi+1) and (2qi+8, 2qi+9)
+              if constexpr (G::RUN == 8) {
+                const uint32_t bsel = static_cast<uint32_t>(ob >> 3);
+                const uint32_t s8 = swap ? ((4 + bsel) | ((4 + bsel) << 4) | (bsel << 8) | (bsel << 12))
+                                         : (bsel | (bsel << 4) | ((4 + bsel) << 8) | ((4 + bsel) << 12));
+                unpack_value_piece8<VB>(ptx::prmt(wa0, wb0, s8), ra);
+                unpack_value_piece8<VB>(ptx::prmt(wa1, wb1, s8), rb);
+              } else if constexpr (G::RUN == 16) {
+                const uint32_t s16 = ob ? sel_hi : sel_lo;
+                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, s16), ra);
+                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, s16), rb);
+              } else {
+                constexpr int n16 = 16 / VB;
+                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_lo), ra);
+                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_hi), ra + n16);
+                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_lo), rb);
+                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_hi), rb + n16);
+              }
+#pragma unroll
+              for (int ml = 0; ml < G::MPG; ++ml)
+                ptx::mma_16816(co[gg * G::MPG + ml], ra[ml], ra[ml + G::MPG], rb[ml], rb[ml + G::MPG],
+                               bp0, bp1);
+            }
+          }
+        }
+
+        // ---- release the stage and refill it ----
+        __syncwarp();
+        if (lane == 0 && k + NS < n_my) {
+          ptx::fence_proxy_async_smem();
+          issue(k + NS);
+        }
+      }
+      if (failed) {
+        // wait (bounded) for every copy this warp still has in flight, then give up
+        if (lane == 0) atomicOr(part.status, KVQ_STATUS_TIMEOUT);
+        const int issued = n_my < k + NS ? n_my : k + NS;
+        for (int kk = k; kk < issued; ++kk)
+          ptx::mbar_wait_bounded(bar0 + 8 * (kk % NS), (kk / NS) & 1, kWaitLimitNs);
+      }
+    }
+  } else {
+    // ---------------- fp16 rows: retained tokens, then the window ----------------
+    uint32_t qn[KSTEPS][2];
+#pragma unroll
+    for (int s = 0; s < KSTEPS; ++s)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int c = 16 * s + 2 * qi + 8 * j;
+        qn[s][j] = (bvalid && !blo) ? ptx::h2_as_u32(__halves2half2(qrow[c], qrow[c + 1])) : 0u;
+      }
+    // stale shared memory must hold finite values: masked rows multiply p = 0
+    for (int i = lane; i < NS * stage_bytes / 16; i += 32)
+      reinterpret_cast<uint4*>(my_stages)[i] = make_uint4(0, 0, 0, 0);
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+
+    auto issue = [&](int k) {
+      const int t = warp + kWarps * k;
+      const int st = k % NS;
+      const uint32_t bar = bar0 + 8 * st;
+      const uint32_t dst = my_stages_s + st * stage_bytes;
+      const int e0 = list_begin + 16 * t;
+      const int nvalid = min(16, list_end - e0);
+      if (lane == 0) ptx::mbar_arrive_expect_tx(bar, nvalid * (DK + kDV) * 2);
+      __syncwarp();
+      const int row = lane & 15;
+      if (row < nvalid) {
+        const int e = e0 + row;
+        size_t slot;
+        const __half* base_k;
+        const __half* base_v;
+        if (e < w.ret.n) {
+          slot = static_cast<size_t>(bh) * kMaxRetained + e;
+          base_k = cb.ret_k;
+          base_v = cb.ret_v;
+        } else {
+          const int pos = w.Q + (e - w.ret.n);
+          slot = static_cast<size_t>(bh) * d.cap + pos % d.cap;
+          base_k = cb.win_k;
+          base_v = cb.win_v;
+        }
+        if (lane < 16)
+          ptx::bulk_g2s(dst + row * R::KST, base_k + slot * DK, DK * 2, bar);
+        else
+          ptx::bulk_g2s(dst + 16 * R::KST + row * R::VST, base_v + slot * kDV, kDV * 2, bar);
+      }
+    };
+
+    for (int k = 0; k < NS && k < n_my; ++k) issue(k);
+    int k = 0;
+    for (; k < n_my; ++k) {
+      const int t = warp + kWarps * k;
+      const int st = k % NS;
+      const bool ok = ptx::mbar_wait_bounded(bar0 + 8 * st, (k / NS) & 1, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) {
+        failed = true;
+        break;
+      }
+      const uint32_t S = my_stages_s + st * stage_bytes;
+      const int nvalid = min(16, list_end - (list_begin + 16 * t));
+      // scores: A = 16 key rows via ldmatrix, B = q (hi columns only)
+      float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const int mi = lane >> 3;                         // which 8x8 matrix this lane addresses
+      const int arow = (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int s = 0; s < KSTEPS; ++s) {
+        uint32_t a0, a1, a2, a3;
+        ptx::ldmatrix_x4(S + arow * R::KST + (16 * s + (mi >> 1) * 8) * 2, a0, a1, a2, a3);
+        ptx::mma_16816(cs, a0, a1, a2, a3, qn[s][0], qn[s][1]);
+      }
+      float s0 = (cs[0] + cs[1]) * alpha;
+      float s1 = (cs[2] + cs[3]) * alpha;
+      if (qr >= nvalid) s0 = -INFINITY;
+      if (qr + 8 >= nvalid) s1 = -INFINITY;
+      float gmax = fmaxf(s0, s1);
+      gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 4));
+      gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
+      gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
+      const float m_new = fmaxf(m_run, gmax);
+      if (__any_sync(0xffffffffu, m_new > m_run)) {
+        const float a = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
+        l_run *= a;
+#pragma unroll
+        for (int mv = 0; mv < 8; ++mv)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) co[mv][e] *= a;
+      }
+      m_run = m_new;
+      const float p0 = cvalid && m_new != -INFINITY ? exp2f(s0 - m_new) : 0.0f;
+      const float p1 = cvalid && m_new != -INFINITY ? exp2f(s1 - m_new) : 0.0f;
+      l_run += p0 + p1;
+      const uint32_t bp0 = ptx::movmatrix_trans(ptx::split_hi_lo(p0));
+      const uint32_t bp1 = ptx::movmatrix_trans(ptx::split_hi_lo(p1));
+      // p.V: A = V^T tiles via ldmatrix.trans (rows = tokens in shared memory)
+      const int vrow = (mi >> 1) * 8 + (lane & 7);
+#pragma unroll
+      for (int mv = 0; mv < 8; ++mv) {
+        uint32_t a0, a1, a2, a3;
+        ptx::ldmatrix_x4_trans(S + 16 * R::KST + vrow * R::VST + (16 * mv + (mi & 1) * 8) * 2, a0, a1,
+                               a2, a3);
+        ptx::mma_16816(co[mv], a0, a1, a2, a3, bp0, bp1);
+      }
+      __syncwarp();
+      if (k + NS < n_my) {
+        if (lane == 0) ptx::fence_proxy_async_smem();
+        issue(k + NS);
+      }
+    }
+    if (failed) {
+      if (lane == 0) atomicOr(part.status, KVQ_STATUS_TIMEOUT);
+      const int issued = n_my < k + NS ? n_my : k + NS;
+      for (int kk = k; kk < issued; ++kk)
+        ptx::mbar_wait_bounded(bar0 + 8 * (kk % NS), (kk / NS) & 1, kWaitLimitNs);
+    }
+  }
+
+  // ---------------- warp totals, then the CTA merge ----------------
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 4);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+#pragma unroll
+  for (int gg = 0; gg < G::NVG; ++gg) {
+    zsum[gg] += __shfl_xor_sync(0xffffffffu, zsum[gg], 4);
+    zsum[gg] += __shfl_xor_sync(0xffffffffu, zsum[gg], 8);
+    zsum[gg] += __shfl_xor_sync(0xffffffffu, zsum[gg], 16);
+  }
+  if (failed) {
+    m_run = -INFINITY;
+    l_run = 0.0f;
+  }
+  __syncthreads();   // every warp is done with its stages: reuse them for the merge
+  float* sm_o = reinterpret_cast<float*>(smem + Smem::kStages);      // [kWarps][NREP][kDV]
+  float* sm_ml = sm_o + kWarps * NREP * kDV;                         // [kWarps][NREP][2]
+  if (cvalid) {
+    float* dst = sm_o + (warp * NREP + qi) * kDV;
+#pragma unroll
+    for (int mv = 0; mv < 8; ++mv) {
+      float o0 = co[mv][0] + co[mv][1];
+      float o1 = co[mv][2] + co[mv][3];
+      int c0, c1;
+      if (quant) {
+        const int gg = mv / G::MPG, ml = mv % G::MPG;
+        c0 = gg * GV + qr * G::CPG + ml;
+        c1 = c0 + G::MPG;
+        o0 = fmaf(o0, static_cast<float>(1 << (24 - value_code_shift<VB, G::RUN>(ml))), zsum[gg]);
+        o1 = fmaf(o1, static_cast<float>(1 << (24 - value_code_shift<VB, G::RUN>(ml + G::MPG))),
+                  zsum[gg]);
+      } else {
+        c0 = 16 * mv + qr;
+        c1 = c0 + 8;
+      }
+      if (failed) o0 = o1 = 0.0f;
+      dst[c0] = o0;
+      dst[c1] = o1;
+    }
+    if (qr == 0) {
+      sm_ml[(warp * NREP + qi) * 2] = m_run;
+      sm_ml[(warp * NREP + qi) * 2 + 1] = l_run;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < NREP * kDV; idx += kThreads) {
+    const int r = idx / kDV, c = idx % kDV;
+    float M = -INFINITY;
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) M = fmaxf(M, sm_ml[(ww * NREP + r) * 2]);
+    float acc = 0.0f, lsum = 0.0f;
+#pragma unroll
+    for (int ww = 0; ww < kWarps; ++ww) {
+      const float mw = sm_ml[(ww * NREP + r) * 2];
+      const float wt = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+      acc = fmaf(wt, sm_o[(ww * NREP + r) * kDV + c], acc);
+      lsum = fmaf(wt, sm_ml[(ww * NREP + r) * 2 + 1], lsum);
+    }
+    const size_t pi = (static_cast<size_t>(b) * d.Hq + h * NREP + r) * w.splits + split;
+    part.o[pi * kDV + c] = acc;
+    if (c == 0) part.ml[pi] = make_float2(M, lsum);
+  }
+}
+
+// Shared memory a launch needs, and the per-warp stage size.
+template <int KB, int VB, int DK, int GV>
+inline int stage_bytes_for(const Dims& d, bool quant) {
+  int s = Raw<DK>::BYTES;
+  if (quant) {
+    const StageLayout L = quant_stage_layout(d.gk, DK, KB, VB, kDV / GV);
+    if (L.bytes > s) s = L.bytes;
+  }
+  return (s + 127) / 128 * 128;
+}
+
+template <int KB, int VB, int DK, int NREP, int GV, int NS, bool QUANT>
+cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
+                   const Partials& p, cudaStream_t s) {
+  const int stage = stage_bytes_for<KB, VB, DK, GV>(d, QUANT);
+  int smem = Smem::kStages + kWarps * NS * stage;
+  const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
+  if (Smem::kStages + merge > smem) smem = Smem::kStages + merge;
+  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, NS, QUANT>;
+  static int configured = 0;
+  if (configured < smem) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  dim3 grid(w.splits, d.Hkv, d.B);
+  kern<<<grid, kThreads, smem, s>>>(d, c, w, q, p, stage);
+  return cudaGetLastError();
+}
+
+}  // namespace mma
+}  // namespace kvq

@@ -20,6 +20,7 @@ struct kvq_cache {
   int Q;
   std::vector<int> ret;   // ascending retained positions
   int sm_count;
+  int kernel;     // KVQ_KERNEL_*
   bool prefilled;
 };
 
@@ -180,6 +181,10 @@ int plan_decode(const kvq::Dims& d, int L, int sm_count, int num_splits, bool fa
 
 int check_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
+bool use_tensor_kernel(const kvq_cache* c) {
+  return c->kernel != KVQ_KERNEL_GENERIC && kvq::decode_mma_supported(c->d);
+}
+
 kvq::CacheBufs cache_bufs(const kvq_cache* c) {
   kvq::CacheBufs b;
   b.kcode = static_cast<const uint32_t*>(c->buf.kcode);
@@ -264,6 +269,7 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
   c->L = 0;
   c->Q = 0;
   c->sm_count = sms;
+  c->kernel = KVQ_KERNEL_AUTO;
   c->prefilled = false;
   *out = c;
   return KVQ_OK;
@@ -390,7 +396,7 @@ int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, 
 int kvq_get_plan(const kvq_cache* c, int num_splits, kvq_plan* out) {
   if (!c || !out) return KVQ_ERR_INVALID_ARG;
   if (!c->prefilled) return KVQ_ERR_STATE;
-  return plan_decode(c->d, c->L, c->sm_count, num_splits, kvq::decode_mma_supported(c->d), out);
+  return plan_decode(c->d, c->L, c->sm_count, num_splits, use_tensor_kernel(c), out);
 }
 
 int kvq_decode_workspace_size(const kvq_cache* c, int num_splits, size_t* bytes) {
@@ -409,7 +415,7 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
   const kvq::Dims& d = c->d;
   kvq_plan plan;
-  int rc = plan_decode(d, c->L, c->sm_count, num_splits, kvq::decode_mma_supported(d), &plan);
+  int rc = plan_decode(d, c->L, c->sm_count, num_splits, use_tensor_kernel(c), &plan);
   if (rc) return rc;
   kvq::DecodeWork w;
   w.L = c->L;
@@ -433,6 +439,13 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
     rc = check_cuda(kvq::launch_decode_simple(d, cb, w, qh, parts, s));
   if (!rc) rc = check_cuda(kvq::launch_combine(d, w, parts, static_cast<__half*>(out), s));
   return rc;
+}
+
+int kvq_set_decode_kernel(kvq_cache* c, int kernel) {
+  if (!c || kernel < KVQ_KERNEL_AUTO || kernel > KVQ_KERNEL_TENSOR) return KVQ_ERR_INVALID_ARG;
+  if (kernel == KVQ_KERNEL_TENSOR && !kvq::decode_mma_supported(c->d)) return KVQ_ERR_UNSUPPORTED;
+  c->kernel = kernel;
+  return KVQ_OK;
 }
 
 int kvq_get_state(const kvq_cache* c, int* L, int* Q, int* n_retained, int* retained_idx) {

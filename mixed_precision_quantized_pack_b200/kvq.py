@@ -26,6 +26,9 @@ KVQ_ERR_WORKSPACE = -5
 KVQ_ERR_STATE = -6
 KVQ_ERR_CUDA = -7
 KVQ_MAX_RETAINED = 32
+KVQ_KERNEL_AUTO = 0
+KVQ_KERNEL_GENERIC = 1
+KVQ_KERNEL_TENSOR = 2
 KVQ_STATUS_TIMEOUT = 1
 
 CONFIG_FIELDS = ("batch", "n_q_heads", "n_kv_heads", "d_k", "d_v", "k_bits", "v_bits", "group_k",
@@ -71,6 +74,7 @@ _SIGNATURES = {
     "kvq_decode_workspace_size": (_I, [_P, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "kvq_decode_attention": (_I, [_P, _P, _P, _P, ctypes.c_size_t, _I, _P]),
     "kvq_get_plan": (_I, [_P, _I, ctypes.POINTER(kvq_plan)]),
+    "kvq_set_decode_kernel": (_I, [_P, _I]),
     "kvq_plan_decode": (_I, [ctypes.POINTER(kvq_config), _I, _I, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_get_state": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                            ctypes.POINTER(_I)]),
@@ -177,6 +181,10 @@ def kvq_get_plan(handle: int, num_splits: int = 0) -> Dict[str, int]:
     return {n: int(getattr(out, n)) for n, _ in kvq_plan._fields_}
 
 
+def kvq_set_decode_kernel(handle: int, kernel: int) -> None:
+    _check(lib().kvq_set_decode_kernel(handle, int(kernel)), "kvq_set_decode_kernel")
+
+
 def kvq_get_state(handle: int) -> Tuple[int, int, List[int]]:
     L, Q, n = _I(), _I(), _I()
     idx = (ctypes.c_int * KVQ_MAX_RETAINED)()
@@ -265,6 +273,9 @@ class KVCache:
 
     def state(self) -> Tuple[int, int, List[int]]:
         return kvq_get_state(self.handle)
+
+    def set_kernel(self, kernel: int) -> None:
+        kvq_set_decode_kernel(self.handle, kernel)
 
     def plan(self, num_splits: int = 0) -> Dict[str, int]:
         return kvq_get_plan(self.handle, num_splits)

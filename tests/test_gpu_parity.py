@@ -15,6 +15,9 @@ from mixed_precision_quantized_pack_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-3
+# AUTO picks the tensor-core kernel wherever it is built for the shape; GENERIC is
+# the CUDA-core kernel.  Both are checked against the oracle.
+KERNELS = (K.KVQ_KERNEL_AUTO, K.KVQ_KERNEL_GENERIC)
 
 
 def need_gpu():
@@ -80,13 +83,28 @@ def run_small(w: W.Workload, num_splits=(0,), steps=None):
             continue
         compare_state(gc, oc, where=f"step {i}")
         ref = oc.decode(np16(inp.q[i]))
-        for s in num_splits:
-            out = gc.decode(inp.q[i].cuda(), num_splits=s)
-            err = O.max_rel_error(out.float().cpu().numpy(), ref)
-            worst = max(worst, err)
-            assert err <= TOL, f"step {i} splits {s}: max rel error {err:.3e}"
+        for kern in KERNELS:
+            gc.set_kernel(kern)
+            for s in num_splits:
+                out = gc.decode(inp.q[i].cuda(), num_splits=s)
+                err = O.max_rel_error(out.float().cpu().numpy(), ref)
+                worst = max(worst, err)
+                assert err <= TOL, f"step {i} kernel {kern} splits {s}: max rel error {err:.3e}"
+        gc.set_kernel(K.KVQ_KERNEL_AUTO)
     assert gc.status() == 0
     return worst
+
+
+def tensor_kernel_built(w: W.Workload) -> bool:
+    return K.kvq_plan_decode(w.kvq_config(), w.context, 148, 0)["fast_path"] == 1
+
+
+@pytest.mark.parametrize("key", list(W.WORKLOADS))
+def test_tensor_kernel_covers_the_named_workloads(key):
+    assert tensor_kernel_built(W.WORKLOADS[key])
+    for b in W.SWEEP_BATCHES:
+        for kb, vb in W.SWEEP_BITS:
+            assert tensor_kernel_built(W.sweep_workload(b, kb, vb))
 
 
 def test_tiny_single_head():
