@@ -154,6 +154,27 @@ int kvq_decode_attention(kvq_cache* cache, const void* q, void* out, void* works
 #define KVQ_KERNEL_TENSOR   2
 int kvq_set_decode_kernel(kvq_cache* cache, int kernel);
 
+/* kvq_decode_attention without a workspace argument, for callers that cannot
+ * allocate device memory: an engine that has reserved the device's memory for
+ * its own pool, a plugin whose host offers no allocator, or a latency-critical
+ * loop that must not pay for cudaMalloc/cudaFree.  (The pages have no
+ * counterpart: this is a property of the library, not of the method.)
+ * The split partials go to a scratch array of KVQ_NOALLOC_SCRATCH_BYTES that
+ * lives in the library; every GPU that loads the library holds it until the
+ * process exits.  Nothing is allocated at call time.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current); make that first call before any stream capture.  The array
+ * is shared by every call and keeps the last call's contents (this call clears
+ * the status word it needs at zero); calls whose executions overlap on the GPU
+ * race on it, so issue them on one stream or otherwise serialize them.
+ * num_splits: 0 = automatic, reduced if needed so that the partials fit in the
+ * array; an explicit split count whose partials do not fit, or a cache so large
+ * that even one split per (b, kv head) does not fit, returns KVQ_ERR_WORKSPACE.
+ * Other errors as for kvq_decode_attention. */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+int kvq_decode_attention_noalloc(kvq_cache* cache, const void* q, void* out, int num_splits,
+                                 void* stream);
+
 /* The plan kvq_decode_attention would use now (host only, no launch). */
 int kvq_get_plan(const kvq_cache* cache, int num_splits, kvq_plan* out);
 

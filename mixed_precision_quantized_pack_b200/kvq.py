@@ -30,6 +30,7 @@ KVQ_KERNEL_AUTO = 0
 KVQ_KERNEL_GENERIC = 1
 KVQ_KERNEL_TENSOR = 2
 KVQ_STATUS_TIMEOUT = 1
+KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 CONFIG_FIELDS = ("batch", "n_q_heads", "n_kv_heads", "d_k", "d_v", "k_bits", "v_bits", "group_k",
                  "group_v", "window", "log_retain", "max_context")
@@ -73,6 +74,7 @@ _SIGNATURES = {
     "kvq_append": (_I, [_P, _P, _P, _P]),
     "kvq_decode_workspace_size": (_I, [_P, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "kvq_decode_attention": (_I, [_P, _P, _P, _P, ctypes.c_size_t, _I, _P]),
+    "kvq_decode_attention_noalloc": (_I, [_P, _P, _P, _I, _P]),
     "kvq_get_plan": (_I, [_P, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_set_decode_kernel": (_I, [_P, _I]),
     "kvq_plan_decode": (_I, [ctypes.POINTER(kvq_config), _I, _I, _I, ctypes.POINTER(kvq_plan)]),
@@ -173,6 +175,13 @@ def kvq_decode_attention(handle: int, q_ptr: int, out_ptr: int, ws_ptr: int, ws_
                          num_splits: int, stream: int) -> None:
     _check(lib().kvq_decode_attention(handle, q_ptr, out_ptr, ws_ptr, int(ws_bytes),
                                       int(num_splits), stream), "kvq_decode_attention")
+
+
+def kvq_decode_attention_noalloc(handle: int, q_ptr: int, out_ptr: int, num_splits: int,
+                                 stream: int) -> None:
+    """Decode without a workspace: the partials go to the library's own scratch array."""
+    _check(lib().kvq_decode_attention_noalloc(handle, q_ptr, out_ptr, int(num_splits), stream),
+           "kvq_decode_attention_noalloc")
 
 
 def kvq_get_plan(handle: int, num_splits: int = 0) -> Dict[str, int]:

@@ -1,0 +1,73 @@
+"""The allocation-free decode entry point, called through the C ABI.
+
+kvq_decode_attention_noalloc serves callers that cannot allocate device memory
+(an engine that owns the device's memory pool, a plugin without an allocator, a
+latency-critical loop that must not call cudaMalloc): instead of a caller
+workspace it writes the split partials to a fixed scratch array inside the
+library.  Its output must match kvq_decode_attention on the same cache, on two
+calls in a row (the array keeps the previous call's contents).  This file is
+collected last and also runs on its own in a fresh process.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixed_precision_quantized_pack_b200 import kvq as K
+from mixed_precision_quantized_pack_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3        # the tolerance of the parity tests: max_c|o - o*| / max_c|o*| per row
+
+
+def rel_err(out: torch.Tensor, ref: torch.Tensor) -> float:
+    o = out.float().reshape(-1, out.shape[-1])
+    r = ref.float().reshape(-1, ref.shape[-1])
+    return float(((o - r).abs().amax(1) / r.abs().amax(1).clamp_min(1e-30)).max())
+
+
+def noalloc(cache: K.KVCache, q: torch.Tensor, num_splits: int = 0) -> torch.Tensor:
+    out = torch.empty((cache.cfg["batch"], cache.cfg["n_q_heads"], cache.cfg["d_v"]),
+                      dtype=torch.float16, device=q.device)
+    K.kvq_decode_attention_noalloc(cache.handle, q.data_ptr(), out.data_ptr(), num_splits,
+                                   K._stream())
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("w", [
+    W.WORKLOADS["gqa4k"].with_(batch=4, appends=2, log_retain=1, seed=301),
+    W.WORKLOADS["long32k"].with_(batch=4, appends=1, seed=302),
+    W.WORKLOADS["thin16k"].with_(batch=2, appends=1, seed=303),
+    W.WORKLOADS["gqa4k"].with_(batch=2, k_bits=16, v_bits=16, appends=1, seed=304),
+], ids=["gqa4k", "long32k", "thin16k", "fp16"])
+def test_noalloc_matches_the_workspace_entry_point_on_two_calls(w):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    inp = W.Inputs(w, device="cuda")
+    cache = K.KVCache(w.kvq_config())
+    cache.prefill(inp.k, inp.v)
+    for step in range(len(inp.q)):
+        cache.append(inp.k_app[step], inp.v_app[step])
+        ref = cache.decode(inp.q[step])
+        torch.cuda.synchronize()
+        first = noalloc(cache, inp.q[step])
+        second = noalloc(cache, inp.q[step])
+        assert rel_err(first, ref) <= TOL
+        assert rel_err(second, ref) <= TOL
+        assert torch.isfinite(second.float()).all()
+
+
+def test_noalloc_rejects_a_split_count_beyond_its_scratch():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = W.WORKLOADS["gqa4k"].with_(batch=8, context=8192, seed=305)
+    inp = W.Inputs(w, device="cuda")
+    cache = K.KVCache(w.kvq_config())
+    cache.prefill(inp.k, inp.v)
+    splits = 100                     # 8 x 32 x 101 partials of 130 floats > 8 MiB
+    assert K.kvq_decode_workspace_size(cache.handle, splits) > K.KVQ_NOALLOC_SCRATCH_BYTES
+    with pytest.raises(K.KVQError) as e:
+        noalloc(cache, inp.q[0], num_splits=splits)
+    assert e.value.code == K.KVQ_ERR_WORKSPACE
+    ref = cache.decode(inp.q[0], num_splits=splits)
+    assert rel_err(noalloc(cache, inp.q[0]), ref) <= TOL
