@@ -4,12 +4,12 @@
 
 namespace kvq {
 namespace mma {
-#define KVQ_DECL_Q(KB, VB, DK, NREP, GV)                                                     \
-  extern template cudaError_t launch<KB, VB, DK, NREP, GV, 2, true>(                        \
+#define KVQ_DECL_Q(KB, VB, DK, NREP, GV, GK)                                                 \
+  extern template cudaError_t launch<KB, VB, DK, NREP, GV, GK, 2, true>(                    \
       const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
       cudaStream_t);
 #define KVQ_DECL_F(DK, NREP)                                                                 \
-  extern template cudaError_t launch<4, 2, DK, NREP, 64, 2, false>(                         \
+  extern template cudaError_t launch<4, 2, DK, NREP, 64, 64, 2, false>(                     \
       const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
       cudaStream_t);
 KVQ_MMA_QUANT_INSTANCES(KVQ_DECL_Q)
@@ -21,20 +21,23 @@ namespace {
 using LaunchFn = cudaError_t (*)(const Dims&, const CacheBufs&, const DecodeWork&, const __half*,
                                  const Partials&, cudaStream_t);
 struct Entry {
-  int kb, vb, dk, nrep, gv;
+  int kb, vb, dk, nrep, gv, gk;
   LaunchFn fn;
 };
 
-#define KVQ_ENTRY_Q(KB, VB, DK, NREP, GV) {KB, VB, DK, NREP, GV, &mma::launch<KB, VB, DK, NREP, GV, 2, true>},
-#define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, &mma::launch<4, 2, DK, NREP, 64, 2, false>},
+#define KVQ_ENTRY_Q(KB, VB, DK, NREP, GV, GK) \
+  {KB, VB, DK, NREP, GV, GK, &mma::launch<KB, VB, DK, NREP, GV, GK, 2, true>},
+#define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, 0, &mma::launch<4, 2, DK, NREP, 64, 64, 2, false>},
 const Entry kTable[] = {KVQ_MMA_QUANT_INSTANCES(KVQ_ENTRY_Q) KVQ_MMA_FP16_INSTANCES(KVQ_ENTRY_F)};
 
 LaunchFn find(const Dims& d) {
   if (d.dv != 128) return nullptr;
   const int gv = d.quantized() ? d.gv : 0;
-  if (d.quantized() && (d.gk < 16 || d.gk > 128 || d.gk % 16 != 0)) return nullptr;
+  const int gk = d.quantized() ? d.gk : 0;
   for (const Entry& e : kTable)
-    if (e.kb == d.kb && e.vb == d.vb && e.dk == d.dk && e.nrep == d.n_rep && e.gv == gv) return e.fn;
+    if (e.kb == d.kb && e.vb == d.vb && e.dk == d.dk && e.nrep == d.n_rep && e.gv == gv &&
+        e.gk == gk)
+      return e.fn;
   return nullptr;
 }
 

@@ -198,7 +198,7 @@ __host__ __device__ inline StageLayout quant_stage_layout(int gk, int dk, int kb
   return s;
 }
 
-template <int KB, int VB, int DK, int NREP, int GV, int NS, bool QUANT>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, int NS, bool QUANT>
 __global__ void __launch_bounds__(kThreads, 3)
 decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part,
                   int stage_bytes) {
@@ -215,7 +215,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   const int bhead = qr >> 1;        // head of this thread's B column
   const bool blo = (qr & 1) != 0;   // B column holds the lo half
   const bool bvalid = bhead < NREP;
-  const bool cvalid = qi < NREP;
+  const bool cvalid = qi < NREP;   // lanes of padding columns compute values nobody reads
   const bool quant = QUANT && split < w.splits_q;
 
   uint32_t* sm_qb = reinterpret_cast<uint32_t*>(smem + Smem::kQb);
@@ -280,9 +280,9 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
 
       // retained positions, one per lane (ascending), for masking the quantized tiles
       const int ret_pos = lane < w.ret.n ? w.ret.pos[lane] : -1;
-      const StageLayout L = quant_stage_layout(d.gk, DK, KB, VB, G::NVG);
-      const int gk = d.gk;
-      const int mtiles = gk / 16;
+      const StageLayout L = quant_stage_layout(GK, DK, KB, VB, G::NVG);
+      constexpr int gk = GK;
+      constexpr int MT = GK / 16;     // 16-token m-tiles per key group
       // per-lane shuffle selectors for the bank-conflict-free value-row loads
       const bool swap = qi >= 2;
       const uint32_t sel_lo = swap ? 0x1054u : 0x5410u;
@@ -359,57 +359,53 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         }
         const float beta = cbias[0] * alpha;
 
+        // ---- scores of the whole group ----
+        float sc[MT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          const int t0 = 16 * mt + qr;
+          uint32_t w0[G::WPT], w1[G::WPT];
+          load_words<G::WPT>(skc + t0 * G::KW + qi * G::WPT, w0);
+          load_words<G::WPT>(skc + (t0 + 8) * G::KW + qi * G::WPT, w1);
+#pragma unroll
+          for (int u = 0; u < G::WPT; ++u) {
+            uint32_t r0[G::RPW], r1[G::RPW];
+            unpack_key_word<KB>(w0[u], r0);
+            unpack_key_word<KB>(w1[u], r1);
+#pragma unroll
+            for (int ls = 0; ls < G::KSPW; ++ls) {
+              const int s = u * G::KSPW + ls;
+              ptx::mma_16816(cs, r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1], bq[s][0],
+                             bq[s][1]);
+            }
+          }
+          sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
+          sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
+        }
         // retained tokens of this group are read from the fp16 list: mask them here
         const int g0 = g * gk;
-        const unsigned hits = __ballot_sync(0xffffffffu, ret_pos >= g0 && ret_pos < g0 + gk);
-
-        // ---- scores of the whole group ----
-        float sc[8][2];
+        unsigned hits = __ballot_sync(0xffffffffu, ret_pos >= g0 && ret_pos < g0 + gk);
+        while (hits) {
+          const int src = __ffs(hits) - 1;
+          hits &= hits - 1;
+          const int off = __shfl_sync(0xffffffffu, ret_pos, src) - g0;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          if (mt < mtiles) {
-            float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            const int t0 = 16 * mt + qr;
-            uint32_t w0[G::WPT], w1[G::WPT];
-            load_words<G::WPT>(skc + t0 * G::KW + qi * G::WPT, w0);
-            load_words<G::WPT>(skc + (t0 + 8) * G::KW + qi * G::WPT, w1);
-#pragma unroll
-            for (int u = 0; u < G::WPT; ++u) {
-              uint32_t r0[G::RPW], r1[G::RPW];
-              unpack_key_word<KB>(w0[u], r0);
-              unpack_key_word<KB>(w1[u], r1);
-#pragma unroll
-              for (int ls = 0; ls < G::KSPW; ++ls) {
-                const int s = u * G::KSPW + ls;
-                ptx::mma_16816(cs, r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1], bq[s][0],
-                               bq[s][1]);
-              }
-            }
-            sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
-            sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
-            if (hits) {
-              unsigned hb = hits;
-              while (hb) {
-                const int src = __ffs(hb) - 1;
-                hb &= hb - 1;
-                const int off = __shfl_sync(0xffffffffu, ret_pos, src) - g0;
-                if (off == t0) sc[mt][0] = -INFINITY;
-                if (off == t0 + 8) sc[mt][1] = -INFINITY;
-              }
-            }
+          for (int mt = 0; mt < MT; ++mt) {
+            if (off == 16 * mt + qr) sc[mt][0] = -INFINITY;
+            if (off == 16 * mt + qr + 8) sc[mt][1] = -INFINITY;
           }
         }
         // ---- online softmax update for the group ----
         float gmax = -INFINITY;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-          if (mt < mtiles) gmax = fmaxf(gmax, fmaxf(sc[mt][0], sc[mt][1]));
+        for (int mt = 0; mt < MT; ++mt) gmax = fmaxf(gmax, fmaxf(sc[mt][0], sc[mt][1]));
         gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 4));
         gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
         gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
         const float m_new = fmaxf(m_run, gmax);
         if (__any_sync(0xffffffffu, m_new > m_run)) {
-          const float a = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
+          const float a = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m_run - m_new);
           l_run *= a;
 #pragma unroll
           for (int gg = 0; gg < G::NVG; ++gg) zsum[gg] *= a;
@@ -419,14 +415,15 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
             for (int e = 0; e < 4; ++e) co[mv][e] *= a;
         }
         m_run = m_new;
+        const float m_use = m_new == -INFINITY ? 0.0f : m_new;   // all masked: every p is 0
 
         // ---- p.V over the group ----
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          if (mt < mtiles) {
+        for (int mt = 0; mt < MT; ++mt) {
+          {
             const int t0 = 16 * mt + qr;
-            const float p0 = cvalid && m_new != -INFINITY ? exp2f(sc[mt][0] - m_new) : 0.0f;
-            const float p1 = cvalid && m_new != -INFINITY ? exp2f(sc[mt][1] - m_new) : 0.0f;
+            const float p0 = ptx::ex2(sc[mt][0] - m_use);
+            const float p1 = ptx::ex2(sc[mt][1] - m_use);
             l_run += p0 + p1;
             // value (scale, zero) of the two tokens this thread weights
             uint32_t vm0[G::NVG], vm1[G::NVG];
@@ -440,8 +437,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
               const float2 f0 = __half22float2(ptx::u32_as_h2(vm0[gg]));
               const float2 f1 = __half22float2(ptx::u32_as_h2(vm1[gg]));
               zsum[gg] = fmaf(p0, f0.y, fmaf(p1, f1.y, zsum[gg]));
-              const uint32_t x0 = ptx::split_hi_lo(p0 * f0.x);
-              const uint32_t x1 = ptx::split_hi_lo(p1 * f1.x);
+              uint32_t x0, x1;
+              ptx::split_hi_lo_pair(p0 * f0.x, p1 * f1.x, x0, x1);
               const uint32_t bp0 = ptx::movmatrix_trans(x0);
               const uint32_t bp1 = ptx::movmatrix_trans(x1);
 
@@ -571,7 +568,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
       const float m_new = fmaxf(m_run, gmax);
       if (__any_sync(0xffffffffu, m_new > m_run)) {
-        const float a = (m_new == -INFINITY) ? 1.0f : exp2f(m_run - m_new);
+        const float a = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m_run - m_new);
         l_run *= a;
 #pragma unroll
         for (int mv = 0; mv < 8; ++mv)
@@ -579,11 +576,14 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
           for (int e = 0; e < 4; ++e) co[mv][e] *= a;
       }
       m_run = m_new;
-      const float p0 = cvalid && m_new != -INFINITY ? exp2f(s0 - m_new) : 0.0f;
-      const float p1 = cvalid && m_new != -INFINITY ? exp2f(s1 - m_new) : 0.0f;
+      const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+      const float p0 = ptx::ex2(s0 - m_use);
+      const float p1 = ptx::ex2(s1 - m_use);
       l_run += p0 + p1;
-      const uint32_t bp0 = ptx::movmatrix_trans(ptx::split_hi_lo(p0));
-      const uint32_t bp1 = ptx::movmatrix_trans(ptx::split_hi_lo(p1));
+      uint32_t x0, x1;
+      ptx::split_hi_lo_pair(p0, p1, x0, x1);
+      const uint32_t bp0 = ptx::movmatrix_trans(x0);
+      const uint32_t bp1 = ptx::movmatrix_trans(x1);
       // p.V: A = V^T tiles via ldmatrix.trans (rows = tokens in shared memory)
       const int vrow = (mi >> 1) * 8 + (lane & 7);
 #pragma unroll
@@ -672,24 +672,24 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
 }
 
 // Shared memory a launch needs, and the per-warp stage size.
-template <int KB, int VB, int DK, int GV>
-inline int stage_bytes_for(const Dims& d, bool quant) {
+template <int KB, int VB, int DK, int GV, int GK>
+inline int stage_bytes_for(bool quant) {
   int s = Raw<DK>::BYTES;
   if (quant) {
-    const StageLayout L = quant_stage_layout(d.gk, DK, KB, VB, kDV / GV);
+    const StageLayout L = quant_stage_layout(GK, DK, KB, VB, kDV / GV);
     if (L.bytes > s) s = L.bytes;
   }
   return (s + 127) / 128 * 128;
 }
 
-template <int KB, int VB, int DK, int NREP, int GV, int NS, bool QUANT>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, int NS, bool QUANT>
 cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
                    const Partials& p, cudaStream_t s) {
-  const int stage = stage_bytes_for<KB, VB, DK, GV>(d, QUANT);
+  const int stage = stage_bytes_for<KB, VB, DK, GV, GK>(QUANT);
   int smem = Smem::kStages + kWarps * NS * stage;
   const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
   if (Smem::kStages + merge > smem) smem = Smem::kStages + merge;
-  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, NS, QUANT>;
+  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, NS, QUANT>;
   static int configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

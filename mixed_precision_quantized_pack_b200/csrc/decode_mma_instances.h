@@ -1,16 +1,17 @@
 // The tensor-core decode instances this library is built with, as an X-macro:
-//   Q(KB, VB, DK, NREP, GV)  quantized caches (value head dim 128)
-//   F(DK, NREP)              unquantized fp16 caches (value head dim 128)
+//   Q(KB, VB, DK, NREP, GV, GK)  quantized caches (value head dim 128)
+//   F(DK, NREP)                  unquantized fp16 caches (value head dim 128)
 // decode_mma.cu builds its dispatch table from the same list; each
-// decode_mma_inst_*.cu file instantiates the entries whose KB it owns.
+// decode_mma_inst_*.cu file instantiates the entries whose KB it owns.  Shapes
+// not listed here run on the generic CUDA-core kernel.
 #pragma once
 
-#define KVQ_MMA_QUANT_INSTANCES(Q)                                                  \
-  Q(4, 2, 128, 4, 64) Q(4, 2, 128, 1, 64) Q(4, 2, 128, 4, 32) Q(4, 2, 128, 1, 32) \
-  Q(4, 2, 32, 4, 32) Q(4, 2, 32, 1, 32) Q(4, 2, 32, 4, 64) Q(4, 2, 32, 1, 64)     \
-  Q(4, 4, 128, 4, 64) Q(4, 4, 128, 1, 64) Q(4, 4, 32, 4, 64) Q(4, 4, 32, 1, 64)   \
-  Q(8, 4, 128, 4, 64) Q(8, 4, 128, 1, 64) Q(8, 4, 128, 4, 32) Q(8, 4, 128, 1, 32) \
-  Q(8, 4, 32, 4, 64) Q(8, 4, 32, 1, 64)                                             \
-  Q(2, 2, 128, 4, 64) Q(2, 2, 128, 1, 64) Q(2, 2, 128, 4, 32) Q(2, 2, 128, 1, 32)
+#define KVQ_MMA_QUANT_INSTANCES(Q)                                                              \
+  Q(4, 2, 128, 4, 64, 64) Q(4, 2, 128, 1, 64, 64) Q(4, 2, 128, 4, 32, 32) Q(4, 2, 128, 1, 32, 32) \
+  Q(4, 2, 32, 4, 32, 32) Q(4, 2, 32, 1, 32, 32) Q(4, 2, 32, 4, 64, 64) Q(4, 2, 32, 1, 64, 64)     \
+  Q(4, 4, 128, 4, 64, 64) Q(4, 4, 128, 1, 64, 64) Q(4, 4, 32, 4, 64, 64) Q(4, 4, 32, 1, 64, 64)   \
+  Q(8, 4, 128, 4, 64, 64) Q(8, 4, 128, 1, 64, 64) Q(8, 4, 128, 4, 32, 32) Q(8, 4, 128, 1, 32, 32) \
+  Q(8, 4, 32, 4, 64, 64) Q(8, 4, 32, 1, 64, 64)                                                 \
+  Q(2, 2, 128, 4, 64, 64) Q(2, 2, 128, 1, 64, 64) Q(2, 2, 128, 4, 32, 32) Q(2, 2, 128, 1, 32, 32)
 
 #define KVQ_MMA_FP16_INSTANCES(F) F(128, 4) F(128, 1) F(32, 4) F(32, 1)

@@ -107,6 +107,23 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
+// 2^x (hardware approximation, relative error about 2^-22; results below 2^-126 flush to 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// (hi, lo) fp16 pairs of two values: hi = fp16(x), lo = fp16(x - hi), so hi + lo == x to
+// about 22 bits.  x0 -> (hi0, lo0) in r0, x1 -> (hi1, lo1) in r1.
+__device__ __forceinline__ void split_hi_lo_pair(float x0, float x1, uint32_t& r0, uint32_t& r1) {
+  const __half2 hi = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(hi);
+  const __half2 lo = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+  r0 = prmt(h2_as_u32(hi), h2_as_u32(lo), 0x5410u);
+  r1 = prmt(h2_as_u32(hi), h2_as_u32(lo), 0x7632u);
+}
+
 // (hi, lo) fp16 pair with hi + lo == x to about 22 bits: hi = fp16(x), lo = fp16(x - hi).
 __device__ __forceinline__ uint32_t split_hi_lo(float x) {
   const __half hi = __float2half_rn(x);
