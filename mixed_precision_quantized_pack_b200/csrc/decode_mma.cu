@@ -5,11 +5,11 @@
 namespace kvq {
 namespace mma {
 #define KVQ_DECL_Q(KB, VB, DK, NREP, GV, GK)                                                 \
-  extern template cudaError_t launch<KB, VB, DK, NREP, GV, GK, 2, true>(                    \
+  extern template cudaError_t launch<KB, VB, DK, NREP, GV, GK, true>(                    \
       const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
       cudaStream_t);
 #define KVQ_DECL_F(DK, NREP)                                                                 \
-  extern template cudaError_t launch<4, 2, DK, NREP, 64, 64, 2, false>(                     \
+  extern template cudaError_t launch<4, 2, DK, NREP, 64, 64, false>(                     \
       const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
       cudaStream_t);
 KVQ_MMA_QUANT_INSTANCES(KVQ_DECL_Q)
@@ -26,8 +26,8 @@ struct Entry {
 };
 
 #define KVQ_ENTRY_Q(KB, VB, DK, NREP, GV, GK) \
-  {KB, VB, DK, NREP, GV, GK, &mma::launch<KB, VB, DK, NREP, GV, GK, 2, true>},
-#define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, 0, &mma::launch<4, 2, DK, NREP, 64, 64, 2, false>},
+  {KB, VB, DK, NREP, GV, GK, &mma::launch<KB, VB, DK, NREP, GV, GK, true>},
+#define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, 0, &mma::launch<4, 2, DK, NREP, 64, 64, false>},
 const Entry kTable[] = {KVQ_MMA_QUANT_INSTANCES(KVQ_ENTRY_Q) KVQ_MMA_FP16_INSTANCES(KVQ_ENTRY_F)};
 
 LaunchFn find(const Dims& d) {

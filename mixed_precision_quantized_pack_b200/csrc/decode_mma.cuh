@@ -6,11 +6,13 @@
 // ("LogQuant: Log-Distributed 2-Bit Quantization of KV Cache", §4), so the two
 // kinds of tokens are visited separately and merged by the log-sum-exp combine.
 //
-// Each warp streams its own units (a key group, or 16 fp16 rows) through a ring
-// of NS shared-memory stages filled by 1-D bulk copies (cp.async.bulk) that
-// complete on a per-stage mbarrier.  Waits are bounded (1 s of globaltimer); on
-// timeout the warp sets KVQ_STATUS_TIMEOUT in the workspace status word, drains
-// its copies (again bounded) and contributes nothing.
+// A CTA's units (key groups, or tiles of 16 fp16 rows) go round-robin to its warps
+// and flow through a CTA-wide ring of shared-memory stages (as many as keep four
+// CTAs per SM), each filled by 1-D bulk copies (cp.async.bulk) that complete on a
+// per-stage mbarrier; the warp that finishes unit k refills its stage with unit
+// k + ring.  Waits are bounded (1 s of globaltimer); on timeout the CTA sets
+// KVQ_STATUS_TIMEOUT in the workspace status word, waits (again bounded) for its
+// last copies and contributes nothing.
 //
 // Scores ("HeadQ", §2.1: s_j = q.k_j/sqrt(d); "Thin Keys, Full Values", §2: d = d_k)
 // use mma.m16n8k16 with the tokens of a 16-token tile on M and, on N, the GQA
@@ -42,6 +44,8 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr int kDV = 128;
+constexpr int kMaxRing = 8;                  // stages of the CTA-wide copy ring, at most
+constexpr int kSmemPerCta = 57344;           // 228 KB per SM / 4 CTAs, minus 1 KB reserved each
 
 // ---------------------------------------------------------------- geometry ----
 template <int KB, int VB, int DK, int GV>
@@ -177,11 +181,21 @@ __device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* out) {
 }
 
 // --------------------------------------------------------------- the kernel ----
+// Shared memory of one CTA: the query for the zero-point MMA (u32 [2*KSTEPS][32 lanes]),
+// then R mbarriers, R copy counters, R unit tags and a failure flag, then a ring of R
+// stages that the CTA's warps share: unit k (a key group or 16 fp16 rows) lives in stage
+// k % R.  The tag of a stage is the unit whose copy was last issued into it: a warp
+// waits for its unit's tag before it waits on the stage's mbarrier, so that barrier is
+// never more than one phase away from the one the warp's parity names.
+template <int KSTEPS>
 struct Smem {
-  // per-CTA header, then per-warp stage rings
-  static constexpr int kQb = 0;                         // u32 [2*KSTEPS (<= 32)][32 lanes]
-  static constexpr int kBars = kQb + 32 * 32 * 4;       // u64 [kWarps][NS]
-  static constexpr int kStages = kBars + kWarps * 4 * 8;
+  static constexpr int kQb = 0;
+  static constexpr int kBars = kQb + 2 * KSTEPS * 32 * 4;
+  static constexpr int kIssued = kBars + kMaxRing * 8;
+  static constexpr int kTag = kIssued + kMaxRing * 4;
+  static constexpr int kFail = kTag + kMaxRing * 4;
+  static constexpr int kStages = kBars + 256;
+  static_assert(kFail + 4 <= kStages, "header overflow");
 };
 
 struct StageLayout {
@@ -198,13 +212,30 @@ __host__ __device__ inline StageLayout quant_stage_layout(int gk, int dk, int kb
   return s;
 }
 
-template <int KB, int VB, int DK, int NREP, int GV, int GK, int NS, bool QUANT>
-__global__ void __launch_bounds__(kThreads, 3)
-decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part,
-                  int stage_bytes) {
+// Bytes of one stage (the larger of a key group and 16 padded fp16 rows) and the number of
+// stages that keep a CTA within a quarter of the SM's shared memory (4 CTAs per SM).
+template <int KB, int VB, int DK, int GV, int GK, bool QUANT>
+constexpr int stage_bytes() {
+  const int raw = Raw<DK>::BYTES;
+  const int qb = QUANT ? GK * DK * KB / 8 + DK * 4 + GK * kDV * VB / 8 + GK * (kDV / GV) * 4 : 0;
+  return ((raw > qb ? raw : qb) + 127) / 128 * 128;
+}
+
+template <int KB, int VB, int DK, int GV, int GK, bool QUANT>
+constexpr int ring_stages() {
+  const int r = (kSmemPerCta - Smem<DK / 16>::kStages) / stage_bytes<KB, VB, DK, GV, GK, QUANT>();
+  return r < 2 ? 2 : (r > kMaxRing ? kMaxRing : r);
+}
+
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT>
+__global__ void __launch_bounds__(kThreads, 4)
+decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part) {
   using G = Quant<(QUANT ? KB : 4), (QUANT ? VB : 2), (QUANT ? DK : 128), (QUANT ? GV : 64)>;
   using R = Raw<DK>;
   constexpr int KSTEPS = DK / 16;
+  constexpr int STAGE = stage_bytes<KB, VB, DK, GV, GK, QUANT>();
+  constexpr int RING = ring_stages<KB, VB, DK, GV, GK, QUANT>();
+  using SM = Smem<KSTEPS>;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -218,13 +249,21 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   const bool cvalid = qi < NREP;   // lanes of padding columns compute values nobody reads
   const bool quant = QUANT && split < w.splits_q;
 
-  uint32_t* sm_qb = reinterpret_cast<uint32_t*>(smem + Smem::kQb);
-  const uint32_t bar0 = ptx::smem_addr(smem + Smem::kBars) + warp * NS * 8;
-  unsigned char* my_stages = smem + Smem::kStages + warp * NS * stage_bytes;
-  const uint32_t my_stages_s = ptx::smem_addr(my_stages);
+  uint32_t* sm_qb = reinterpret_cast<uint32_t*>(smem + SM::kQb);
+  int* sm_issued = reinterpret_cast<int*>(smem + SM::kIssued);
+  volatile int* sm_tag = reinterpret_cast<volatile int*>(smem + SM::kTag);
+  int* sm_fail = reinterpret_cast<int*>(smem + SM::kFail);
+  const uint32_t bar0 = ptx::smem_addr(smem + SM::kBars);
+  unsigned char* stages = smem + SM::kStages;
+  const uint32_t stages_s = ptx::smem_addr(stages);
 
-  if (lane == 0) {
-    for (int s = 0; s < NS; ++s) ptx::mbar_init(bar0 + 8 * s, 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RING; ++s) {
+      ptx::mbar_init(bar0 + 8 * s, 1);
+      sm_issued[s] = 0;
+      sm_tag[s] = -1;
+    }
+    *sm_fail = 0;
     ptx::fence_barrier_init();
   }
   const __half* qrow = q + (static_cast<size_t>(b) * d.Hq + h * NREP + (bvalid ? bhead : 0)) * DK;
@@ -242,11 +281,12 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
     unit_begin = 0;
     unit_end = (list_end - list_begin + 15) / 16;
   }
-  const int n_my = unit_end - unit_begin > warp ? (unit_end - unit_begin - warp + kWarps - 1) / kWarps : 0;
+  // unit k of this CTA (k < n_units) is processed by warp k % kWarps, in stage k % RING
+  const int n_units = unit_end - unit_begin;
 
   // running softmax state of head qi over this warp's tokens
   float m_run = -INFINITY, l_run = 0.0f;
-  float zsum[G::NVG];
+  float zsum[G::NVG];               // sum_j p_j z_{j,g}, lane-partial
 #pragma unroll
   for (int g = 0; g < G::NVG; ++g) zsum[g] = 0.0f;
   float co[8][4];
@@ -288,11 +328,14 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       const uint32_t sel_lo = swap ? 0x1054u : 0x5410u;
       const uint32_t sel_hi = swap ? 0x3276u : 0x7632u;
 
+      // one lane copies unit k (a whole key group: 4 contiguous runs) into stage k % RING
       auto issue = [&](int k) {
-        const int g = unit_begin + warp + kWarps * k;
-        const int st = k % NS;
+        const int g = unit_begin + k;
+        const int st = k % RING;
         const uint32_t bar = bar0 + 8 * st;
-        const uint32_t dst = my_stages_s + st * stage_bytes;
+        const uint32_t dst = stages_s + st * STAGE;
+        sm_issued[st] += 1;
+        sm_tag[st] = k;
         ptx::mbar_arrive_expect_tx(bar, L.bytes);
         const size_t tok = static_cast<size_t>(bh) * d.lcap + static_cast<size_t>(g) * gk;
         ptx::bulk_g2s(dst + L.k_off, cb.kcode + tok * G::KW, gk * G::KBYTES_ROW, bar);
@@ -302,20 +345,19 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         ptx::bulk_g2s(dst + L.vmeta_off, cb.vsz + tok * G::NVG, gk * G::NVG * 4, bar);
       };
 
-      __syncwarp();
-      if (lane == 0)
-        for (int k = 0; k < NS && k < n_my; ++k) issue(k);
+      if (threadIdx.x == 0)
+        for (int k = 0; k < RING && k < n_units; ++k) issue(k);
 
-      int k = 0;
-      for (; k < n_my; ++k) {
-        const int g = unit_begin + warp + kWarps * k;
-        const int st = k % NS;
-        const bool ok = ptx::mbar_wait_bounded(bar0 + 8 * st, (k / NS) & 1, kWaitLimitNs);
+      for (int k = warp; k < n_units; k += kWarps) {
+        const int g = unit_begin + k;
+        const int st = k % RING;
+        const bool ok = ptx::wait_equal_bounded(sm_tag + st, k, kWaitLimitNs) &&
+                        ptx::mbar_wait_bounded(bar0 + 8 * st, (k / RING) & 1, kWaitLimitNs);
         if (!__all_sync(0xffffffffu, ok)) {
           failed = true;
           break;
         }
-        const unsigned char* S = my_stages + st * stage_bytes;
+        const unsigned char* S = stages + st * STAGE;
         const uint32_t* skc = reinterpret_cast<const uint32_t*>(S + L.k_off);
         const uint32_t* skm = reinterpret_cast<const uint32_t*>(S + L.kmeta_off);
         const uint32_t* svc = reinterpret_cast<const uint32_t*>(S + L.v_off);
@@ -323,7 +365,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
 
         // ---- group prologue: B = hi or lo of q*s, and the zero-point bias ----
         uint32_t bq[KSTEPS][2];
-        float cbias[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        float cbias[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
 #pragma unroll
         for (int u = 0; u < G::WPT; ++u) {
           const int omega = qi * G::WPT + u;
@@ -354,16 +396,17 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
               const __half2 hi = __hmul2(qs, sc);
               bq[s][j] = blo ? ptx::h2_as_u32(__hfma2(qs, sc, __hneg2(hi))) : ptx::h2_as_u32(hi);
             }
-            ptx::mma_16816(cbias, za[0], za[0], za[1], za[1], qbx[2 * ls], qbx[2 * ls + 1]);
+            ptx::mma_16816(cbias[s & 1], za[0], za[0], za[1], za[1], qbx[2 * ls], qbx[2 * ls + 1]);
           }
         }
-        const float beta = cbias[0] * alpha;
+        const float beta = (cbias[0][0] + cbias[1][0]) * alpha;
 
         // ---- scores of the whole group ----
         float sc[MT][2];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          // two accumulators (even / odd k-steps) halve the dependent MMA chain
+          float cs[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
           const int t0 = 16 * mt + qr;
           uint32_t w0[G::WPT], w1[G::WPT];
           load_words<G::WPT>(skc + t0 * G::KW + qi * G::WPT, w0);
@@ -376,12 +419,12 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
 #pragma unroll
             for (int ls = 0; ls < G::KSPW; ++ls) {
               const int s = u * G::KSPW + ls;
-              ptx::mma_16816(cs, r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1], bq[s][0],
-                             bq[s][1]);
+              ptx::mma_16816(cs[s & 1], r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1],
+                             bq[s][0], bq[s][1]);
             }
           }
-          sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
-          sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
+          sc[mt][0] = fmaf((cs[0][0] + cs[1][0]) + (cs[0][1] + cs[1][1]), alpha24, beta);
+          sc[mt][1] = fmaf((cs[0][2] + cs[1][2]) + (cs[0][3] + cs[1][3]), alpha24, beta);
         }
         // retained tokens of this group are read from the fp16 list: mask them here
         const int g0 = g * gk;
@@ -473,19 +516,12 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
           }
         }
 
-        // ---- release the stage and refill it ----
+        // ---- release the stage: refill it with unit k + RING ----
         __syncwarp();
-        if (lane == 0 && k + NS < n_my) {
+        if (lane == 0 && k + RING < n_units) {
           ptx::fence_proxy_async_smem();
-          issue(k + NS);
+          issue(k + RING);
         }
-      }
-      if (failed) {
-        // wait (bounded) for every copy this warp still has in flight, then give up
-        if (lane == 0) atomicOr(part.status, KVQ_STATUS_TIMEOUT);
-        const int issued = n_my < k + NS ? n_my : k + NS;
-        for (int kk = k; kk < issued; ++kk)
-          ptx::mbar_wait_bounded(bar0 + 8 * (kk % NS), (kk / NS) & 1, kWaitLimitNs);
       }
     }
   } else {
@@ -499,19 +535,23 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         qn[s][j] = (bvalid && !blo) ? ptx::h2_as_u32(__halves2half2(qrow[c], qrow[c + 1])) : 0u;
       }
     // stale shared memory must hold finite values: masked rows multiply p = 0
-    for (int i = lane; i < NS * stage_bytes / 16; i += 32)
-      reinterpret_cast<uint4*>(my_stages)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < RING * STAGE / 16; i += kThreads)
+      reinterpret_cast<uint4*>(stages)[i] = make_uint4(0, 0, 0, 0);
     ptx::fence_proxy_async_smem();
-    __syncwarp();
+    __syncthreads();
 
+    // the 32 lanes of one warp copy the up to 16 key and 16 value rows of unit k
     auto issue = [&](int k) {
-      const int t = warp + kWarps * k;
-      const int st = k % NS;
+      const int st = k % RING;
       const uint32_t bar = bar0 + 8 * st;
-      const uint32_t dst = my_stages_s + st * stage_bytes;
-      const int e0 = list_begin + 16 * t;
+      const uint32_t dst = stages_s + st * STAGE;
+      const int e0 = list_begin + 16 * k;
       const int nvalid = min(16, list_end - e0);
-      if (lane == 0) ptx::mbar_arrive_expect_tx(bar, nvalid * (DK + kDV) * 2);
+      if (lane == 0) {
+        sm_issued[st] += 1;
+        sm_tag[st] = k;
+        ptx::mbar_arrive_expect_tx(bar, nvalid * (DK + kDV) * 2);
+      }
       __syncwarp();
       const int row = lane & 15;
       if (row < nvalid) {
@@ -536,18 +576,18 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       }
     };
 
-    for (int k = 0; k < NS && k < n_my; ++k) issue(k);
-    int k = 0;
-    for (; k < n_my; ++k) {
-      const int t = warp + kWarps * k;
-      const int st = k % NS;
-      const bool ok = ptx::mbar_wait_bounded(bar0 + 8 * st, (k / NS) & 1, kWaitLimitNs);
+    if (warp == 0)
+      for (int k = 0; k < RING && k < n_units; ++k) issue(k);
+    for (int k = warp; k < n_units; k += kWarps) {
+      const int st = k % RING;
+      const bool ok = ptx::wait_equal_bounded(sm_tag + st, k, kWaitLimitNs) &&
+                      ptx::mbar_wait_bounded(bar0 + 8 * st, (k / RING) & 1, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, ok)) {
         failed = true;
         break;
       }
-      const uint32_t S = my_stages_s + st * stage_bytes;
-      const int nvalid = min(16, list_end - (list_begin + 16 * t));
+      const uint32_t S = stages_s + st * STAGE;
+      const int nvalid = min(16, list_end - (list_begin + 16 * k));
       // scores: A = 16 key rows via ldmatrix, B = q (hi columns only)
       float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
       const int mi = lane >> 3;                         // which 8x8 matrix this lane addresses
@@ -594,17 +634,24 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         ptx::mma_16816(co[mv], a0, a1, a2, a3, bp0, bp1);
       }
       __syncwarp();
-      if (k + NS < n_my) {
+      if (k + RING < n_units) {
         if (lane == 0) ptx::fence_proxy_async_smem();
-        issue(k + NS);
+        issue(k + RING);
       }
     }
-    if (failed) {
-      if (lane == 0) atomicOr(part.status, KVQ_STATUS_TIMEOUT);
-      const int issued = n_my < k + NS ? n_my : k + NS;
-      for (int kk = k; kk < issued; ++kk)
-        ptx::mbar_wait_bounded(bar0 + 8 * (kk % NS), (kk / NS) & 1, kWaitLimitNs);
-    }
+  }
+
+  // A bounded wait gave up: flag it, then wait (bounded) for the last copy issued into
+  // every stage so that no copy lands in shared memory after the CTA has exited.
+  if (failed && lane == 0) {
+    atomicOr(part.status, KVQ_STATUS_TIMEOUT);
+    atomicOr(sm_fail, 1);
+  }
+  __syncthreads();
+  if (*sm_fail) {
+    if (threadIdx.x < RING && sm_issued[threadIdx.x] > 0)
+      ptx::mbar_wait_bounded(bar0 + 8 * threadIdx.x, (sm_issued[threadIdx.x] - 1) & 1, kWaitLimitNs);
+    failed = true;     // the CTA's partial is dropped as a whole
   }
 
   // ---------------- warp totals, then the CTA merge ----------------
@@ -621,8 +668,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
     m_run = -INFINITY;
     l_run = 0.0f;
   }
-  __syncthreads();   // every warp is done with its stages: reuse them for the merge
-  float* sm_o = reinterpret_cast<float*>(smem + Smem::kStages);      // [kWarps][NREP][kDV]
+  __syncthreads();   // every warp is done with the stages: reuse them for the merge
+  float* sm_o = reinterpret_cast<float*>(smem + SM::kStages);        // [kWarps][NREP][kDV]
   float* sm_ml = sm_o + kWarps * NREP * kDV;                         // [kWarps][NREP][2]
   if (cvalid) {
     float* dst = sm_o + (warp * NREP + qi) * kDV;
@@ -671,25 +718,15 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   }
 }
 
-// Shared memory a launch needs, and the per-warp stage size.
-template <int KB, int VB, int DK, int GV, int GK>
-inline int stage_bytes_for(bool quant) {
-  int s = Raw<DK>::BYTES;
-  if (quant) {
-    const StageLayout L = quant_stage_layout(GK, DK, KB, VB, kDV / GV);
-    if (L.bytes > s) s = L.bytes;
-  }
-  return (s + 127) / 128 * 128;
-}
-
-template <int KB, int VB, int DK, int NREP, int GV, int GK, int NS, bool QUANT>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT>
 cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
                    const Partials& p, cudaStream_t s) {
-  const int stage = stage_bytes_for<KB, VB, DK, GV, GK>(QUANT);
-  int smem = Smem::kStages + kWarps * NS * stage;
+  constexpr int stage = stage_bytes<KB, VB, DK, GV, GK, QUANT>();
+  constexpr int ring = ring_stages<KB, VB, DK, GV, GK, QUANT>();
+  int smem = Smem<DK / 16>::kStages + ring * stage;
   const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
-  if (Smem::kStages + merge > smem) smem = Smem::kStages + merge;
-  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, NS, QUANT>;
+  if (Smem<DK / 16>::kStages + merge > smem) smem = Smem<DK / 16>::kStages + merge;
+  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT>;
   static int configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -697,7 +734,7 @@ cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const
     configured = smem;
   }
   dim3 grid(w.splits, d.Hkv, d.B);
-  kern<<<grid, kThreads, smem, s>>>(d, c, w, q, p, stage);
+  kern<<<grid, kThreads, smem, s>>>(d, c, w, q, p);
   return cudaGetLastError();
 }
 

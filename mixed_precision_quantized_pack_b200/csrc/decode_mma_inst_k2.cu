@@ -6,7 +6,7 @@ namespace kvq {
 namespace mma {
 
 #define KVQ_INST_Q(KB, VB, DK, NREP, GV, GK)                                                     \
-  template cudaError_t launch<KB, VB, DK, NREP, GV, GK, 2, true>(                                \
+  template cudaError_t launch<KB, VB, DK, NREP, GV, GK, true>(                                \
       const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,         \
       cudaStream_t);
 #define KVQ_PICK(KB, VB, DK, NREP, GV, GK) KVQ_PICK_##KB(KB, VB, DK, NREP, GV, GK)

@@ -60,6 +60,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// Waits until the shared-memory word *p equals v, giving up after `limit_ns`.
+__device__ __forceinline__ bool wait_equal_bounded(const volatile int* p, int v, uint64_t limit_ns) {
+  if (*p == v) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (*p == v) return true;
+    if ((it & 255u) == 0 && globaltimer() - t0 > limit_ns) return false;
+  }
+}
+
 // ---- bulk copy (1-D TMA), global -> this CTA's shared memory ------------------
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
