@@ -44,7 +44,9 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr int kDV = 128;
-constexpr int kMaxRing = 8;                  // stages of the CTA-wide copy ring, at most
+constexpr int kMaxRing = 8;
+constexpr int kMinRing = kWarps + 1;         // fewer stages than warps would idle a warp
+constexpr float kLazyRescale = 8.0f;         // see the online-softmax update                  // stages of the CTA-wide copy ring, at most
 constexpr int kSmemPerCta = 57344;           // 228 KB per SM / 4 CTAs, minus 1 KB reserved each
 
 // ---------------------------------------------------------------- geometry ----
@@ -180,8 +182,13 @@ __device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* out) {
   }
 }
 
+// The zero-point MMA's copy of q in shared memory: entry e of lane l, grouped four
+// entries per lane so that a lane reads its consecutive entries with one 128-bit load.
+__device__ __forceinline__ int qb_index(int e, int lane) { return ((e >> 2) * 32 + lane) * 4 + (e & 3); }
+
 // --------------------------------------------------------------- the kernel ----
-// Shared memory of one CTA: the query for the zero-point MMA (u32 [2*KSTEPS][32 lanes]),
+// Shared memory of one CTA: the query for the zero-point MMA and the query scaled for the
+// score MMA (each u32 [2*KSTEPS][32 lanes]),
 // then R mbarriers, R copy counters, R unit tags and a failure flag, then a ring of R
 // stages that the CTA's warps share: unit k (a key group or 16 fp16 rows) lives in stage
 // k % R.  The tag of a stage is the unit whose copy was last issued into it: a warp
@@ -190,7 +197,8 @@ __device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* out) {
 template <int KSTEPS>
 struct Smem {
   static constexpr int kQb = 0;
-  static constexpr int kBars = kQb + 2 * KSTEPS * 32 * 4;
+  static constexpr int kQf = kQb + 2 * KSTEPS * 32 * 4;     // q scaled by 2^-p, same layout
+  static constexpr int kBars = kQf + 2 * KSTEPS * 32 * 4;
   static constexpr int kIssued = kBars + kMaxRing * 8;
   static constexpr int kTag = kIssued + kMaxRing * 4;
   static constexpr int kFail = kTag + kMaxRing * 4;
@@ -224,7 +232,7 @@ constexpr int stage_bytes() {
 template <int KB, int VB, int DK, int GV, int GK, bool QUANT>
 constexpr int ring_stages() {
   const int r = (kSmemPerCta - Smem<DK / 16>::kStages) / stage_bytes<KB, VB, DK, GV, GK, QUANT>();
-  return r < 2 ? 2 : (r > kMaxRing ? kMaxRing : r);
+  return r < kMinRing ? kMinRing : (r > kMaxRing ? kMaxRing : r);
 }
 
 template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT>
@@ -250,6 +258,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   const bool quant = QUANT && split < w.splits_q;
 
   uint32_t* sm_qb = reinterpret_cast<uint32_t*>(smem + SM::kQb);
+  uint32_t* sm_qf = reinterpret_cast<uint32_t*>(smem + SM::kQf);
   int* sm_issued = reinterpret_cast<int*>(smem + SM::kIssued);
   volatile int* sm_tag = reinterpret_cast<volatile int*>(smem + SM::kTag);
   int* sm_fail = reinterpret_cast<int*>(smem + SM::kFail);
@@ -302,7 +311,6 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   if (quant) {
     if constexpr (QUANT) {
       // B operands: q (scaled by 2^-p per k-slot) in registers, plain q in shared memory
-      uint32_t qf[KSTEPS][2];
 #pragma unroll
       for (int s = 0; s < KSTEPS; ++s)
 #pragma unroll
@@ -313,8 +321,10 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
           const int c_hi = c_lo + 16 / KB;
           const __half2 pair = bvalid ? __halves2half2(qrow[c_lo], qrow[c_hi]) : __float2half2_rn(0.0f);
           const float f = 1.0f / static_cast<float>(1 << key_reg_shift<KB>(rho));
-          qf[s][j] = ptx::h2_as_u32(__hmul2(pair, __float2half2_rn(f)));
-          if (warp == 0) sm_qb[(2 * s + j) * 32 + lane] = ptx::h2_as_u32(pair);
+          if (warp == 0) {
+            sm_qf[qb_index(2 * s + j, lane)] = ptx::h2_as_u32(__hmul2(pair, __float2half2_rn(f)));
+            sm_qb[qb_index(2 * s + j, lane)] = ptx::h2_as_u32(pair);
+          }
         }
       __syncthreads();
 
@@ -378,9 +388,17 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
             meta[c4 + 2] = v4.z;
             meta[c4 + 3] = v4.w;
           }
-          uint32_t qbx[2 * G::KSPW];
+          uint32_t qbx[2 * G::KSPW], qfx[2 * G::KSPW];
+          if constexpr (2 * G::KSPW >= 4) {
 #pragma unroll
-          for (int e = 0; e < 2 * G::KSPW; ++e) qbx[e] = sm_qb[(2 * u * G::KSPW + e) * 32 + lane];
+            for (int c4 = 0; c4 < 2 * G::KSPW; c4 += 4) {
+              load_words<4>(sm_qb + qb_index(2 * u * G::KSPW + c4, lane), qbx + c4);
+              load_words<4>(sm_qf + qb_index(2 * u * G::KSPW + c4, lane), qfx + c4);
+            }
+          } else {
+            load_words<2 * G::KSPW>(sm_qb + qb_index(2 * u * G::KSPW, lane), qbx);
+            load_words<2 * G::KSPW>(sm_qf + qb_index(2 * u * G::KSPW, lane), qfx);
+          }
 #pragma unroll
           for (int ls = 0; ls < G::KSPW; ++ls) {
             const int s = u * G::KSPW + ls;
@@ -391,7 +409,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
               const uint32_t mlo = meta[rho], mhi = meta[rho + 16 / KB];
               const uint32_t s2 = ptx::prmt(mlo, mhi, 0x5410u);   // (s_lo, s_hi)
               za[j] = ptx::prmt(mlo, mhi, 0x7632u);               // (z_lo, z_hi)
-              const __half2 qs = ptx::u32_as_h2(qf[s][j]);
+              const __half2 qs = ptx::u32_as_h2(qfx[2 * ls + j]);
               const __half2 sc = ptx::u32_as_h2(s2);
               const __half2 hi = __hmul2(qs, sc);
               bq[s][j] = blo ? ptx::h2_as_u32(__hfma2(qs, sc, __hneg2(hi))) : ptx::h2_as_u32(hi);
@@ -405,8 +423,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         float sc[MT][2];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          // two accumulators (even / odd k-steps) halve the dependent MMA chain
-          float cs[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+          float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
           const int t0 = 16 * mt + qr;
           uint32_t w0[G::WPT], w1[G::WPT];
           load_words<G::WPT>(skc + t0 * G::KW + qi * G::WPT, w0);
@@ -419,12 +436,12 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
 #pragma unroll
             for (int ls = 0; ls < G::KSPW; ++ls) {
               const int s = u * G::KSPW + ls;
-              ptx::mma_16816(cs[s & 1], r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1],
-                             bq[s][0], bq[s][1]);
+              ptx::mma_16816(cs, r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1], bq[s][0],
+                             bq[s][1]);
             }
           }
-          sc[mt][0] = fmaf((cs[0][0] + cs[1][0]) + (cs[0][1] + cs[1][1]), alpha24, beta);
-          sc[mt][1] = fmaf((cs[0][2] + cs[1][2]) + (cs[0][3] + cs[1][3]), alpha24, beta);
+          sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
+          sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
         }
         // retained tokens of this group are read from the fp16 list: mask them here
         const int g0 = g * gk;
@@ -446,8 +463,11 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 4));
         gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
         gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
+        // The reference maximum moves only when a score exceeds it by more than
+        // kLazyRescale (log2 units): weights then stay below 2^kLazyRescale and the
+        // accumulators are rescaled rarely.
         const float m_new = fmaxf(m_run, gmax);
-        if (__any_sync(0xffffffffu, m_new > m_run)) {
+        if (__any_sync(0xffffffffu, m_new > m_run + kLazyRescale)) {
           const float a = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m_run - m_new);
           l_run *= a;
 #pragma unroll
@@ -456,9 +476,9 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
           for (int mv = 0; mv < 8; ++mv)
 #pragma unroll
             for (int e = 0; e < 4; ++e) co[mv][e] *= a;
+          m_run = m_new;
         }
-        m_run = m_new;
-        const float m_use = m_new == -INFINITY ? 0.0f : m_new;   // all masked: every p is 0
+        const float m_use = m_run == -INFINITY ? 0.0f : m_run;   // all masked: every p is 0
 
         // ---- p.V over the group ----
 #pragma unroll
@@ -607,16 +627,16 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
       gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
       const float m_new = fmaxf(m_run, gmax);
-      if (__any_sync(0xffffffffu, m_new > m_run)) {
+      if (__any_sync(0xffffffffu, m_new > m_run + kLazyRescale)) {
         const float a = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m_run - m_new);
         l_run *= a;
 #pragma unroll
         for (int mv = 0; mv < 8; ++mv)
 #pragma unroll
           for (int e = 0; e < 4; ++e) co[mv][e] *= a;
+        m_run = m_new;
       }
-      m_run = m_new;
-      const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+      const float m_use = m_run == -INFINITY ? 0.0f : m_run;
       const float p0 = ptx::ex2(s0 - m_use);
       const float p1 = ptx::ex2(s1 - m_use);
       l_run += p0 + p1;
