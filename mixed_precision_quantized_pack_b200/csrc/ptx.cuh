@@ -84,6 +84,23 @@ __device__ __forceinline__ bool wait_equal_bounded(const volatile int* p, int v,
   }
 }
 
+// Barrier `id` over `count` threads (a multiple of 32) that also returns whether any of
+// them passed pred = true.
+__device__ __forceinline__ bool bar_red_or(int id, int count, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return out != 0;
+}
+// Arrives once on an mbarrier (release semantics for this thread's prior writes).
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 // ---- bulk copy (1-D TMA), global -> this CTA's shared memory ------------------
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -232,6 +249,14 @@ __device__ __forceinline__ void tmem_st_16x256b<8>(uint32_t taddr, const uint32_
 template <int N>
 __device__ __forceinline__ void tmem_load_32x32b(uint32_t taddr, uint32_t* r);
 template <>
+__device__ __forceinline__ void tmem_load_32x32b<4>(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+}
+template <>
 __device__ __forceinline__ void tmem_load_32x32b<8>(uint32_t taddr, uint32_t* r) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
                "tcgen05.wait::ld.sync.aligned;"
@@ -268,6 +293,12 @@ __device__ __forceinline__ void tmem_load_32x32b<32>(uint32_t taddr, uint32_t* r
 // 32 lanes x 32 bits, N columns: thread t writes lane t (relative to taddr), columns 0..N-1.
 template <int N>
 __device__ __forceinline__ void tmem_st_32x32b(uint32_t taddr, const uint32_t* r);
+template <>
+__device__ __forceinline__ void tmem_st_32x32b<4>(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
 template <>
 __device__ __forceinline__ void tmem_st_32x32b<8>(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
