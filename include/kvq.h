@@ -30,9 +30,7 @@
  *   kcode  u32  [B][Hkv][Lcap][d_k*k_bits/32]   token rows, channel c at word
  *               c/(32/k_bits), bit (c%(32/k_bits))*k_bits (LSB first)
  *   ksz    f16  [B][Hkv][Lcap/group_k][d_k][2] (scale, zero) per key group and channel
- *   vcode  u32  [B][Hkv][Lcap/group_k][d_v][group_k*v_bits/32]  channel-major inside
- *               each key group: the row of channel c holds the group's tokens,
- *               token t at word t/(32/v_bits), bit (t%(32/v_bits))*v_bits
+ *   vcode  u32  [B][Hkv][Lcap][d_v*v_bits/32]   same packing per token row
  *   vsz    f16  [B][Hkv][Lcap][d_v/group_v][2] (scale, zero) per token and value group
  *   win_k  f16  [B][Hkv][C][d_k]  token p in slot p % C, C = window + group_k
  *   win_v  f16  [B][Hkv][C][d_v]  (bits 16: C = max_context, the whole cache)

@@ -1,26 +1,36 @@
-// Split-K flash-decoding kernel for the fp16 rows of the cache: the retained
-// tokens, then the recent window (or, for an unquantized cache, every token).
+// Fused dequant + split-K flash-decoding kernel on the tensor cores (sm_100a).
 //
-// One CTA = 4 warps = one split of one (b, kv head) over the fp16 list.  The
-// quantized groups are read by the tcgen05 kernel (decode_tc.cuh); token order is
-// free ("LogQuant: Log-Distributed 2-Bit Quantization of KV Cache", §4), so the
-// two kinds of tokens are visited by separate CTAs and merged by the log-sum-exp
-// combine.  The fp16 list of a quantized cache is short (window R plus at most 32
-// retained tokens), so this path stays on warp-level mma.sync.
+// One CTA = 4 warps = one split of one (b, kv head).  Splits [0, splits_q) cover
+// whole key groups of the quantized prefix; splits [splits_q, splits) cover the
+// fp16 list (retained tokens, then the window).  Token order is free
+// ("LogQuant: Log-Distributed 2-Bit Quantization of KV Cache", §4), so the two
+// kinds of tokens are visited separately and merged by the log-sum-exp combine.
 //
-// Units of 16 list rows go round-robin to the CTA's warps and flow through a
-// CTA-wide ring of shared-memory stages filled by 1-D bulk copies (cp.async.bulk)
-// that complete on a per-stage mbarrier; the warp that finishes unit k refills
-// its stage with unit k + ring.  A per-stage unit tag keeps a waiting warp from
-// confusing two phases of the same mbarrier.  Waits are bounded (1 s of
-// globaltimer); on timeout the CTA sets KVQ_STATUS_TIMEOUT in the workspace
-// status word, waits (again bounded) for its last copies and contributes nothing.
+// A CTA's units (key groups, or tiles of 16 fp16 rows) go round-robin to its warps
+// and flow through a CTA-wide ring of shared-memory stages (as many as keep four
+// CTAs per SM), each filled by 1-D bulk copies (cp.async.bulk) that complete on a
+// per-stage mbarrier; the warp that finishes unit k refills its stage with unit
+// k + ring.  Waits are bounded (1 s of globaltimer); on timeout the CTA sets
+// KVQ_STATUS_TIMEOUT in the workspace status word, waits (again bounded) for its
+// last copies and contributes nothing.
 //
-// Scores ("HeadQ", §2.1: s_j = q.k_j/sqrt(d); "Thin Keys, Full Values", §2:
-// d = d_k) use mma.m16n8k16 with the 16 rows of a unit on M and the GQA query
-// heads sharing the kv head on N (column 2h; column 2h+1 stays zero); p.V uses
-// the transposed orientation (channels on M, the 16 rows on K) with p split into
-// (hi, lo) fp16 halves in columns 2h, 2h+1 so that p keeps about 22 bits.
+// Scores ("HeadQ", §2.1: s_j = q.k_j/sqrt(d); "Thin Keys, Full Values", §2: d = d_k)
+// use mma.m16n8k16 with the tokens of a 16-token tile on M and, on N, the GQA
+// query heads sharing the kv head, each twice: column 2h holds hi(q'_h), column
+// 2h+1 holds lo(q'_h), where q'_c = q_c * s_{g,c} folds the per-channel key scale
+// into the query once per group and hi/lo are the two fp16 halves of the exact
+// fp32 product (hi + lo == q'_c).  The key codes enter the MMA unconverted: a
+// b-bit field masked in place inside a 16-bit lane is an fp16 subnormal of value
+// code * 2^(p-24), p its bit offset (p + b <= 8 after at most one byte shift), so
+// unpacking is one AND per two codes; the factor 2^-p goes into q' and the common
+// 2^-24 into the softmax scale.  The zero points add sum_c q_c z_{g,c} per group,
+// computed by one more MMA per k-step with z in A and q in B.
+//
+// p.V uses the transposed orientation: channels on M, the 16 tokens on K, and on
+// N again (hi, lo) pairs, now of p_j * s_{j,g} (per-token value scale), moved from
+// the score accumulator layout to the B layout with movmatrix.  Value codes are
+// masked as subnormals too; their 2^(p-24) factors are per output channel and are
+// removed once at the end, where sum_j p_j z_{j,g} is added.
 #pragma once
 
 #include "../../include/kvq.h"
@@ -36,8 +46,29 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr int kDV = 128;
 constexpr int kMaxRing = 8;
 constexpr int kMinRing = kWarps + 1;         // fewer stages than warps would idle a warp
-constexpr float kLazyRescale = 8.0f;         // see the online-softmax update
+constexpr float kLazyRescale = 8.0f;         // see the online-softmax update                  // stages of the CTA-wide copy ring, at most
 constexpr int kSmemPerCta = 57344;           // 228 KB per SM / 4 CTAs, minus 1 KB reserved each
+
+// ---------------------------------------------------------------- geometry ----
+template <int KB, int VB, int DK, int GV>
+struct Quant {
+  static constexpr int KW = DK * KB / 32;            // u32 words per key row
+  static constexpr int VW = kDV * VB / 32;           // u32 words per value row
+  static constexpr int WPT = KW / 4;                 // key words per thread (a quad shares a row)
+  static constexpr int KSTEPS = DK / 16;
+  static constexpr int RPW = 16 / KB;                // A registers per key word
+  static constexpr int KSPW = RPW / 2;               // k-steps per key word
+  static constexpr int CPW = 32 / KB;                // channels per key word
+  static constexpr int NVG = kDV / GV;               // value groups per token
+  static constexpr int MPG = GV / 16;                // value m-tiles per value group
+  static constexpr int CPG = GV / 8;                 // channels a thread owns per value group
+  static constexpr int RUN = CPG * VB;               // bits of that run in a value row
+  static constexpr int KBYTES_ROW = DK * KB / 8;
+  static constexpr int VBYTES_ROW = kDV * VB / 8;
+  static_assert(WPT >= 1 && KSTEPS == WPT * KSPW, "key row too short for the fragment mapping");
+  static_assert(RUN == 8 || RUN == 16 || RUN == 32, "value run must be 8, 16 or 32 bits");
+  static_assert(MPG >= 1, "value group below 16 channels");
+};
 
 template <int DK>
 struct Raw {
@@ -47,42 +78,175 @@ struct Raw {
   static constexpr int KSTEPS = DK / 16;
 };
 
-// Shared memory of one CTA: R mbarriers, R copy counters, R unit tags and a failure flag,
-// then a ring of R stages that the CTA's warps share: unit k lives in stage k % R.  The
-// tag of a stage is the unit whose copy was last issued into it: a warp waits for its
-// unit's tag before it waits on the stage's mbarrier, so that barrier is never more than
-// one phase away from the one the warp's parity names.
+// fp16 mantissa-field masks: the `bits`-wide field at bit `pos` of both 16-bit halves.
+template <int BITS, int POS>
+struct Mask {
+  static constexpr uint32_t v = (((1u << BITS) - 1u) << POS) * 0x00010001u;
+};
+
+// Register rho of a key word: the pair (channel c, channel c + 16/KB) as subnormals
+// with factor 2^(p-24), p = (KB * rho) mod 8.
+template <int KB>
+__device__ __forceinline__ void unpack_key_word(uint32_t w, uint32_t (&r)[16 / KB]) {
+  if constexpr (KB == 4) {
+    const uint32_t u = w >> 8;
+    r[0] = w & Mask<4, 0>::v;
+    r[1] = w & Mask<4, 4>::v;
+    r[2] = u & Mask<4, 0>::v;
+    r[3] = u & Mask<4, 4>::v;
+  } else if constexpr (KB == 2) {
+    const uint32_t u = w >> 8;
+    r[0] = w & Mask<2, 0>::v;
+    r[1] = w & Mask<2, 2>::v;
+    r[2] = w & Mask<2, 4>::v;
+    r[3] = w & Mask<2, 6>::v;
+    r[4] = u & Mask<2, 0>::v;
+    r[5] = u & Mask<2, 2>::v;
+    r[6] = u & Mask<2, 4>::v;
+    r[7] = u & Mask<2, 6>::v;
+  } else {
+    r[0] = w & Mask<8, 0>::v;
+    r[1] = (w >> 8) & Mask<8, 0>::v;
+  }
+}
+
+template <int KB>
+__host__ __device__ constexpr int key_reg_shift(int rho) { return (KB * rho) % 8; }
+
+// The codes of one 16-bit piece (token a in the low half, token b in the high
+// half), as subnormal pairs; code e' sits at bit VB*e' of the piece.
+template <int VB>
+__device__ __forceinline__ void unpack_value_piece16(uint32_t x, uint32_t* r) {
+  const uint32_t u = x >> 8;
+  if constexpr (VB == 2) {
+    r[0] = x & Mask<2, 0>::v;
+    r[1] = x & Mask<2, 2>::v;
+    r[2] = x & Mask<2, 4>::v;
+    r[3] = x & Mask<2, 6>::v;
+    r[4] = u & Mask<2, 0>::v;
+    r[5] = u & Mask<2, 2>::v;
+    r[6] = u & Mask<2, 4>::v;
+    r[7] = u & Mask<2, 6>::v;
+  } else if constexpr (VB == 4) {
+    r[0] = x & Mask<4, 0>::v;
+    r[1] = x & Mask<4, 4>::v;
+    r[2] = u & Mask<4, 0>::v;
+    r[3] = u & Mask<4, 4>::v;
+  } else {
+    r[0] = x & Mask<8, 0>::v;
+    r[1] = u & Mask<8, 0>::v;
+  }
+}
+
+template <int VB>
+__device__ __forceinline__ void unpack_value_piece8(uint32_t x, uint32_t* r) {
+  static_assert(VB == 2 || VB == 4 || VB == 8, "");
+  if constexpr (VB == 2) {
+    r[0] = x & Mask<2, 0>::v;
+    r[1] = x & Mask<2, 2>::v;
+    r[2] = x & Mask<2, 4>::v;
+    r[3] = x & Mask<2, 6>::v;
+  } else if constexpr (VB == 4) {
+    r[0] = x & Mask<4, 0>::v;
+    r[1] = x & Mask<4, 4>::v;
+  } else {
+    r[0] = x & Mask<8, 0>::v;
+  }
+}
+
+// Bit offset (within its fp16 lane) of code e of a thread's value run.
+template <int VB, int RUN>
+__host__ __device__ constexpr int value_code_shift(int e) {
+  return RUN == 8 ? (VB * e) % 8 : (VB * (e % (16 / VB))) % 8;
+}
+
+// N consecutive u32 from shared memory at an address aligned to min(4N, 16) bytes.
+template <int N>
+__device__ __forceinline__ void load_words(const uint32_t* p, uint32_t* out) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p + i);
+      out[i] = v.x;
+      out[i + 1] = v.y;
+      out[i + 2] = v.z;
+      out[i + 3] = v.w;
+    }
+  } else if constexpr (N == 2) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    out[0] = v.x;
+    out[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) out[i] = p[i];
+  }
+}
+
+// The zero-point MMA's copy of q in shared memory: entry e of lane l, grouped four
+// entries per lane so that a lane reads its consecutive entries with one 128-bit load.
+__device__ __forceinline__ int qb_index(int e, int lane) { return ((e >> 2) * 32 + lane) * 4 + (e & 3); }
+
+// --------------------------------------------------------------- the kernel ----
+// Shared memory of one CTA: the query for the zero-point MMA and the query scaled for the
+// score MMA (each u32 [2*KSTEPS][32 lanes]),
+// then R mbarriers, R copy counters, R unit tags and a failure flag, then a ring of R
+// stages that the CTA's warps share: unit k (a key group or 16 fp16 rows) lives in stage
+// k % R.  The tag of a stage is the unit whose copy was last issued into it: a warp
+// waits for its unit's tag before it waits on the stage's mbarrier, so that barrier is
+// never more than one phase away from the one the warp's parity names.
+template <int KSTEPS>
 struct Smem {
-  static constexpr int kBars = 0;
+  static constexpr int kQb = 0;
+  static constexpr int kQf = kQb + 2 * KSTEPS * 32 * 4;     // q scaled by 2^-p, same layout
+  static constexpr int kBars = kQf + 2 * KSTEPS * 32 * 4;
   static constexpr int kIssued = kBars + kMaxRing * 8;
   static constexpr int kTag = kIssued + kMaxRing * 4;
   static constexpr int kFail = kTag + kMaxRing * 4;
-  static constexpr int kStages = 256;
+  static constexpr int kStages = kBars + 256;
   static_assert(kFail + 4 <= kStages, "header overflow");
 };
 
-template <int DK>
-constexpr int stage_bytes() {
-  return (Raw<DK>::BYTES + 127) / 128 * 128;
+struct StageLayout {
+  int k_off, kmeta_off, v_off, vmeta_off, bytes;
+};
+
+__host__ __device__ inline StageLayout quant_stage_layout(int gk, int dk, int kb, int vb, int nvg) {
+  StageLayout s;
+  s.k_off = 0;
+  s.kmeta_off = gk * dk * kb / 8;
+  s.v_off = s.kmeta_off + dk * 4;
+  s.vmeta_off = s.v_off + gk * kDV * vb / 8;
+  s.bytes = s.vmeta_off + gk * nvg * 4;
+  return s;
 }
 
-template <int DK>
+// Bytes of one stage (the larger of a key group and 16 padded fp16 rows) and the number of
+// stages that keep a CTA within a quarter of the SM's shared memory (4 CTAs per SM).
+template <int KB, int VB, int DK, int GV, int GK, bool QUANT>
+constexpr int stage_bytes() {
+  const int raw = Raw<DK>::BYTES;
+  const int qb = QUANT ? GK * DK * KB / 8 + DK * 4 + GK * kDV * VB / 8 + GK * (kDV / GV) * 4 : 0;
+  return ((raw > qb ? raw : qb) + 127) / 128 * 128;
+}
+
+template <int KB, int VB, int DK, int GV, int GK, bool QUANT>
 constexpr int ring_stages() {
-  const int r = (kSmemPerCta - Smem::kStages) / stage_bytes<DK>();
+  const int r = (kSmemPerCta - Smem<DK / 16>::kStages) / stage_bytes<KB, VB, DK, GV, GK, QUANT>();
   return r < kMinRing ? kMinRing : (r > kMaxRing ? kMaxRing : r);
 }
 
-template <int DK, int NREP>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT>
 __global__ void __launch_bounds__(kThreads, 4)
-decode_fp16_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part) {
+decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part) {
+  using G = Quant<(QUANT ? KB : 4), (QUANT ? VB : 2), (QUANT ? DK : 128), (QUANT ? GV : 64)>;
   using R = Raw<DK>;
   constexpr int KSTEPS = DK / 16;
-  constexpr int STAGE = stage_bytes<DK>();
-  constexpr int RING = ring_stages<DK>();
+  constexpr int STAGE = stage_bytes<KB, VB, DK, GV, GK, QUANT>();
+  constexpr int RING = ring_stages<KB, VB, DK, GV, GK, QUANT>();
+  using SM = Smem<KSTEPS>;
   extern __shared__ __align__(128) unsigned char smem[];
 
-  // the fp16 CTAs' partials follow those of the quantized groups
-  const int split = w.splits_q + blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int bh = b * d.Hkv + h;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qi = lane & 3;          // quad index: C columns 2qi, 2qi+1 = head qi (hi, lo)
@@ -90,13 +254,16 @@ decode_fp16_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict_
   const int bhead = qr >> 1;        // head of this thread's B column
   const bool blo = (qr & 1) != 0;   // B column holds the lo half
   const bool bvalid = bhead < NREP;
-  const bool cvalid = qi < NREP;    // lanes of padding columns compute values nobody reads
+  const bool cvalid = qi < NREP;   // lanes of padding columns compute values nobody reads
+  const bool quant = QUANT && split < w.splits_q;
 
-  int* sm_issued = reinterpret_cast<int*>(smem + Smem::kIssued);
-  volatile int* sm_tag = reinterpret_cast<volatile int*>(smem + Smem::kTag);
-  int* sm_fail = reinterpret_cast<int*>(smem + Smem::kFail);
-  const uint32_t bar0 = ptx::smem_addr(smem + Smem::kBars);
-  unsigned char* stages = smem + Smem::kStages;
+  uint32_t* sm_qb = reinterpret_cast<uint32_t*>(smem + SM::kQb);
+  uint32_t* sm_qf = reinterpret_cast<uint32_t*>(smem + SM::kQf);
+  int* sm_issued = reinterpret_cast<int*>(smem + SM::kIssued);
+  volatile int* sm_tag = reinterpret_cast<volatile int*>(smem + SM::kTag);
+  int* sm_fail = reinterpret_cast<int*>(smem + SM::kFail);
+  const uint32_t bar0 = ptx::smem_addr(smem + SM::kBars);
+  unsigned char* stages = smem + SM::kStages;
   const uint32_t stages_s = ptx::smem_addr(stages);
 
   if (threadIdx.x == 0) {
@@ -110,136 +277,387 @@ decode_fp16_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict_
   }
   const __half* qrow = q + (static_cast<size_t>(b) * d.Hq + h * NREP + (bvalid ? bhead : 0)) * DK;
 
-  // this CTA's rows of the fp16 list, in units of 16
-  const int f = blockIdx.x;
-  const int list_begin = static_cast<int>(static_cast<long long>(f) * w.n_fp16 / w.splits_f);
-  const int list_end = static_cast<int>(static_cast<long long>(f + 1) * w.n_fp16 / w.splits_f);
-  const int n_units = (list_end - list_begin + 15) / 16;
+  // ---------------- work list of this warp ----------------
+  int unit_begin, unit_end;      // quantized: groups; fp16: tiles of 16 list entries
+  int list_begin = 0, list_end = 0;
+  if (quant) {
+    unit_begin = static_cast<int>(static_cast<long long>(split) * w.n_groups / w.splits_q);
+    unit_end = static_cast<int>(static_cast<long long>(split + 1) * w.n_groups / w.splits_q);
+  } else {
+    const int f = split - (QUANT ? w.splits_q : 0);
+    list_begin = static_cast<int>(static_cast<long long>(f) * w.n_fp16 / w.splits_f);
+    list_end = static_cast<int>(static_cast<long long>(f + 1) * w.n_fp16 / w.splits_f);
+    unit_begin = 0;
+    unit_end = (list_end - list_begin + 15) / 16;
+  }
+  // unit k of this CTA (k < n_units) is processed by warp k % kWarps, in stage k % RING
+  const int n_units = unit_end - unit_begin;
 
-  // running softmax state of head qi over this warp's rows
+  // running softmax state of head qi over this warp's tokens
   float m_run = -INFINITY, l_run = 0.0f;
+  float zsum[G::NVG];               // sum_j p_j z_{j,g}, lane-partial
+#pragma unroll
+  for (int g = 0; g < G::NVG; ++g) zsum[g] = 0.0f;
   float co[8][4];
 #pragma unroll
   for (int mv = 0; mv < 8; ++mv)
 #pragma unroll
     for (int e = 0; e < 4; ++e) co[mv][e] = 0.0f;
   bool failed = false;
+
   const float alpha = w.score_scale;                       // log2(e) / sqrt(d_k)
+  const float alpha24 = w.score_scale * 16777216.0f;       // undoes the 2^-24 of subnormal codes
 
-  uint32_t qn[KSTEPS][2];
+  if (quant) {
+    if constexpr (QUANT) {
+      // B operands: q (scaled by 2^-p per k-slot) in registers, plain q in shared memory
 #pragma unroll
-  for (int s = 0; s < KSTEPS; ++s)
+      for (int s = 0; s < KSTEPS; ++s)
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int c = 16 * s + 2 * qi + 8 * j;
-      qn[s][j] = (bvalid && !blo) ? ptx::h2_as_u32(__halves2half2(qrow[c], qrow[c + 1])) : 0u;
-    }
-  // stale shared memory must hold finite values: masked rows multiply p = 0
-  for (int i = threadIdx.x; i < RING * STAGE / 16; i += kThreads)
-    reinterpret_cast<uint4*>(stages)[i] = make_uint4(0, 0, 0, 0);
-  ptx::fence_proxy_async_smem();
-  __syncthreads();
+        for (int j = 0; j < 2; ++j) {
+          const int omega = qi * G::WPT + s / G::KSPW;
+          const int rho = 2 * (s % G::KSPW) + j;
+          const int c_lo = G::CPW * omega + rho;
+          const int c_hi = c_lo + 16 / KB;
+          const __half2 pair = bvalid ? __halves2half2(qrow[c_lo], qrow[c_hi]) : __float2half2_rn(0.0f);
+          const float f = 1.0f / static_cast<float>(1 << key_reg_shift<KB>(rho));
+          if (warp == 0) {
+            sm_qf[qb_index(2 * s + j, lane)] = ptx::h2_as_u32(__hmul2(pair, __float2half2_rn(f)));
+            sm_qb[qb_index(2 * s + j, lane)] = ptx::h2_as_u32(pair);
+          }
+        }
+      __syncthreads();
 
-  // the 32 lanes of one warp copy the up to 16 key and 16 value rows of unit k
-  auto issue = [&](int k) {
-    const int st = k % RING;
-    const uint32_t bar = bar0 + 8 * st;
-    const uint32_t dst = stages_s + st * STAGE;
-    const int e0 = list_begin + 16 * k;
-    const int nvalid = min(16, list_end - e0);
-    if (lane == 0) {
-      sm_issued[st] += 1;
-      sm_tag[st] = k;
-      ptx::mbar_arrive_expect_tx(bar, nvalid * (DK + kDV) * 2);
-    }
-    __syncwarp();
-    const int row = lane & 15;
-    if (row < nvalid) {
-      const int e = e0 + row;
-      size_t slot;
-      const __half* base_k;
-      const __half* base_v;
-      if (e < w.ret.n) {
-        slot = static_cast<size_t>(bh) * kMaxRetained + e;
-        base_k = cb.ret_k;
-        base_v = cb.ret_v;
-      } else {
-        const int pos = w.Q + (e - w.ret.n);
-        slot = static_cast<size_t>(bh) * d.cap + pos % d.cap;
-        base_k = cb.win_k;
-        base_v = cb.win_v;
+      // retained positions, one per lane (ascending), for masking the quantized tiles
+      const int ret_pos = lane < w.ret.n ? w.ret.pos[lane] : -1;
+      const StageLayout L = quant_stage_layout(GK, DK, KB, VB, G::NVG);
+      constexpr int gk = GK;
+      constexpr int MT = GK / 16;     // 16-token m-tiles per key group
+      // per-lane shuffle selectors for the bank-conflict-free value-row loads
+      const bool swap = qi >= 2;
+      const uint32_t sel_lo = swap ? 0x1054u : 0x5410u;
+      const uint32_t sel_hi = swap ? 0x3276u : 0x7632u;
+
+      // one lane copies unit k (a whole key group: 4 contiguous runs) into stage k % RING
+      auto issue = [&](int k) {
+        const int g = unit_begin + k;
+        const int st = k % RING;
+        const uint32_t bar = bar0 + 8 * st;
+        const uint32_t dst = stages_s + st * STAGE;
+        sm_issued[st] += 1;
+        sm_tag[st] = k;
+        ptx::mbar_arrive_expect_tx(bar, L.bytes);
+        const size_t tok = static_cast<size_t>(bh) * d.lcap + static_cast<size_t>(g) * gk;
+        ptx::bulk_g2s(dst + L.k_off, cb.kcode + tok * G::KW, gk * G::KBYTES_ROW, bar);
+        ptx::bulk_g2s(dst + L.kmeta_off, cb.ksz + (static_cast<size_t>(bh) * (d.lcap / gk) + g) * DK,
+                      DK * 4, bar);
+        ptx::bulk_g2s(dst + L.v_off, cb.vcode + tok * G::VW, gk * G::VBYTES_ROW, bar);
+        ptx::bulk_g2s(dst + L.vmeta_off, cb.vsz + tok * G::NVG, gk * G::NVG * 4, bar);
+      };
+
+      if (threadIdx.x == 0)
+        for (int k = 0; k < RING && k < n_units; ++k) issue(k);
+
+      for (int k = warp; k < n_units; k += kWarps) {
+        const int g = unit_begin + k;
+        const int st = k % RING;
+        const bool ok = ptx::wait_equal_bounded(sm_tag + st, k, kWaitLimitNs) &&
+                        ptx::mbar_wait_bounded(bar0 + 8 * st, (k / RING) & 1, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) {
+          failed = true;
+          break;
+        }
+        const unsigned char* S = stages + st * STAGE;
+        const uint32_t* skc = reinterpret_cast<const uint32_t*>(S + L.k_off);
+        const uint32_t* skm = reinterpret_cast<const uint32_t*>(S + L.kmeta_off);
+        const uint32_t* svc = reinterpret_cast<const uint32_t*>(S + L.v_off);
+        const uint32_t* svm = reinterpret_cast<const uint32_t*>(S + L.vmeta_off);
+
+        // ---- group prologue: B = hi or lo of q*s, and the zero-point bias ----
+        uint32_t bq[KSTEPS][2];
+        float cbias[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+#pragma unroll
+        for (int u = 0; u < G::WPT; ++u) {
+          const int omega = qi * G::WPT + u;
+          uint32_t meta[G::CPW];
+#pragma unroll
+          for (int c4 = 0; c4 < G::CPW; c4 += 4) {
+            const uint4 v4 = *reinterpret_cast<const uint4*>(skm + G::CPW * omega + c4);
+            meta[c4] = v4.x;
+            meta[c4 + 1] = v4.y;
+            meta[c4 + 2] = v4.z;
+            meta[c4 + 3] = v4.w;
+          }
+          uint32_t qbx[2 * G::KSPW], qfx[2 * G::KSPW];
+          if constexpr (2 * G::KSPW >= 4) {
+#pragma unroll
+            for (int c4 = 0; c4 < 2 * G::KSPW; c4 += 4) {
+              load_words<4>(sm_qb + qb_index(2 * u * G::KSPW + c4, lane), qbx + c4);
+              load_words<4>(sm_qf + qb_index(2 * u * G::KSPW + c4, lane), qfx + c4);
+            }
+          } else {
+            load_words<2 * G::KSPW>(sm_qb + qb_index(2 * u * G::KSPW, lane), qbx);
+            load_words<2 * G::KSPW>(sm_qf + qb_index(2 * u * G::KSPW, lane), qfx);
+          }
+#pragma unroll
+          for (int ls = 0; ls < G::KSPW; ++ls) {
+            const int s = u * G::KSPW + ls;
+            uint32_t za[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int rho = 2 * ls + j;
+              const uint32_t mlo = meta[rho], mhi = meta[rho + 16 / KB];
+              const uint32_t s2 = ptx::prmt(mlo, mhi, 0x5410u);   // (s_lo, s_hi)
+              za[j] = ptx::prmt(mlo, mhi, 0x7632u);               // (z_lo, z_hi)
+              const __half2 qs = ptx::u32_as_h2(qfx[2 * ls + j]);
+              const __half2 sc = ptx::u32_as_h2(s2);
+              const __half2 hi = __hmul2(qs, sc);
+              bq[s][j] = blo ? ptx::h2_as_u32(__hfma2(qs, sc, __hneg2(hi))) : ptx::h2_as_u32(hi);
+            }
+            ptx::mma_16816(cbias[s & 1], za[0], za[0], za[1], za[1], qbx[2 * ls], qbx[2 * ls + 1]);
+          }
+        }
+        const float beta = (cbias[0][0] + cbias[1][0]) * alpha;
+
+        // ---- scores of the whole group ----
+        float sc[MT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          const int t0 = 16 * mt + qr;
+          uint32_t w0[G::WPT], w1[G::WPT];
+          load_words<G::WPT>(skc + t0 * G::KW + qi * G::WPT, w0);
+          load_words<G::WPT>(skc + (t0 + 8) * G::KW + qi * G::WPT, w1);
+#pragma unroll
+          for (int u = 0; u < G::WPT; ++u) {
+            uint32_t r0[G::RPW], r1[G::RPW];
+            unpack_key_word<KB>(w0[u], r0);
+            unpack_key_word<KB>(w1[u], r1);
+#pragma unroll
+            for (int ls = 0; ls < G::KSPW; ++ls) {
+              const int s = u * G::KSPW + ls;
+              ptx::mma_16816(cs, r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1], bq[s][0],
+                             bq[s][1]);
+            }
+          }
+          sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
+          sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
+        }
+        // retained tokens of this group are read from the fp16 list: mask them here
+        const int g0 = g * gk;
+        unsigned hits = __ballot_sync(0xffffffffu, ret_pos >= g0 && ret_pos < g0 + gk);
+        while (hits) {
+          const int src = __ffs(hits) - 1;
+          hits &= hits - 1;
+          const int off = __shfl_sync(0xffffffffu, ret_pos, src) - g0;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            if (off == 16 * mt + qr) sc[mt][0] = -INFINITY;
+            if (off == 16 * mt + qr + 8) sc[mt][1] = -INFINITY;
+          }
+        }
+        // ---- online softmax update for the group ----
+        float gmax = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) gmax = fmaxf(gmax, fmaxf(sc[mt][0], sc[mt][1]));
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 4));
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
+        gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
+        // The reference maximum moves only when a score exceeds it by more than
+        // kLazyRescale (log2 units): weights then stay below 2^kLazyRescale and the
+        // accumulators are rescaled rarely.
+        const float m_new = fmaxf(m_run, gmax);
+        if (__any_sync(0xffffffffu, m_new > m_run + kLazyRescale)) {
+          const float a = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m_run - m_new);
+          l_run *= a;
+#pragma unroll
+          for (int gg = 0; gg < G::NVG; ++gg) zsum[gg] *= a;
+#pragma unroll
+          for (int mv = 0; mv < 8; ++mv)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) co[mv][e] *= a;
+          m_run = m_new;
+        }
+        const float m_use = m_run == -INFINITY ? 0.0f : m_run;   // all masked: every p is 0
+
+        // ---- p.V over the group ----
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          {
+            const int t0 = 16 * mt + qr;
+            const float p0 = ptx::ex2(sc[mt][0] - m_use);
+            const float p1 = ptx::ex2(sc[mt][1] - m_use);
+            l_run += p0 + p1;
+            // value (scale, zero) of the two tokens this thread weights
+            uint32_t vm0[G::NVG], vm1[G::NVG];
+            load_words<G::NVG>(svm + t0 * G::NVG, vm0);
+            load_words<G::NVG>(svm + (t0 + 8) * G::NVG, vm1);
+            // value words: tokens 2qi, 2qi+1, 2qi+8, 2qi+9 of the tile, swapped for qi >= 2
+            const int ta = 16 * mt + 2 * qi + (swap ? 1 : 0);
+            const int tb = 16 * mt + 2 * qi + (swap ? 0 : 1);
+#pragma unroll
+            for (int gg = 0; gg < G::NVG; ++gg) {
+              const float2 f0 = __half22float2(ptx::u32_as_h2(vm0[gg]));
+              const float2 f1 = __half22float2(ptx::u32_as_h2(vm1[gg]));
+              zsum[gg] = fmaf(p0, f0.y, fmaf(p1, f1.y, zsum[gg]));
+              uint32_t x0, x1;
+              ptx::split_hi_lo_pair(p0 * f0.x, p1 * f1.x, x0, x1);
+              const uint32_t bp0 = ptx::movmatrix_trans(x0);
+              const uint32_t bp1 = ptx::movmatrix_trans(x1);
+
+              const int bit0 = (gg * GV + qr * G::CPG) * VB;
+              const int wv = bit0 >> 5;
+              const int ob = bit0 & 31;
+              const uint32_t wa0 = svc[ta * G::VW + wv], wb0 = svc[tb * G::VW + wv];
+              const uint32_t wa1 = svc[(ta + 8) * G::VW + wv], wb1 = svc[(tb + 8) * G::VW + wv];
+              uint32_t ra[G::CPG], rb[G::CPG];   // codes of tokens (2qi, 2qi+1) and (2qi+8, 2qi+9)
+              if constexpr (G::RUN == 8) {
+                const uint32_t bsel = static_cast<uint32_t>(ob >> 3);
+                const uint32_t s8 = swap ? ((4 + bsel) | ((4 + bsel) << 4) | (bsel << 8) | (bsel << 12))
+                                         : (bsel | (bsel << 4) | ((4 + bsel) << 8) | ((4 + bsel) << 12));
+                unpack_value_piece8<VB>(ptx::prmt(wa0, wb0, s8), ra);
+                unpack_value_piece8<VB>(ptx::prmt(wa1, wb1, s8), rb);
+              } else if constexpr (G::RUN == 16) {
+                const uint32_t s16 = ob ? sel_hi : sel_lo;
+                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, s16), ra);
+                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, s16), rb);
+              } else {
+                constexpr int n16 = 16 / VB;
+                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_lo), ra);
+                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_hi), ra + n16);
+                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_lo), rb);
+                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_hi), rb + n16);
+              }
+#pragma unroll
+              for (int ml = 0; ml < G::MPG; ++ml)
+                ptx::mma_16816(co[gg * G::MPG + ml], ra[ml], ra[ml + G::MPG], rb[ml], rb[ml + G::MPG],
+                               bp0, bp1);
+            }
+          }
+        }
+
+        // ---- release the stage: refill it with unit k + RING ----
+        __syncwarp();
+        if (lane == 0 && k + RING < n_units) {
+          ptx::fence_proxy_async_smem();
+          issue(k + RING);
+        }
       }
-      if (lane < 16)
-        ptx::bulk_g2s(dst + row * R::KST, base_k + slot * DK, DK * 2, bar);
-      else
-        ptx::bulk_g2s(dst + 16 * R::KST + row * R::VST, base_v + slot * kDV, kDV * 2, bar);
     }
-  };
+  } else {
+    // ---------------- fp16 rows: retained tokens, then the window ----------------
+    uint32_t qn[KSTEPS][2];
+#pragma unroll
+    for (int s = 0; s < KSTEPS; ++s)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int c = 16 * s + 2 * qi + 8 * j;
+        qn[s][j] = (bvalid && !blo) ? ptx::h2_as_u32(__halves2half2(qrow[c], qrow[c + 1])) : 0u;
+      }
+    // stale shared memory must hold finite values: masked rows multiply p = 0
+    for (int i = threadIdx.x; i < RING * STAGE / 16; i += kThreads)
+      reinterpret_cast<uint4*>(stages)[i] = make_uint4(0, 0, 0, 0);
+    ptx::fence_proxy_async_smem();
+    __syncthreads();
 
-  if (warp == 0)
-    for (int k = 0; k < RING && k < n_units; ++k) issue(k);
-  for (int k = warp; k < n_units; k += kWarps) {
-    const int st = k % RING;
-    const bool ok = ptx::wait_equal_bounded(sm_tag + st, k, kWaitLimitNs) &&
-                    ptx::mbar_wait_bounded(bar0 + 8 * st, (k / RING) & 1, kWaitLimitNs);
-    if (!__all_sync(0xffffffffu, ok)) {
-      failed = true;
-      break;
-    }
-    const uint32_t S = stages_s + st * STAGE;
-    const int nvalid = min(16, list_end - (list_begin + 16 * k));
-    // scores: A = 16 key rows via ldmatrix, B = q (hi columns only)
-    float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    const int mi = lane >> 3;                         // which 8x8 matrix this lane addresses
-    const int arow = (mi & 1) * 8 + (lane & 7);
+    // the 32 lanes of one warp copy the up to 16 key and 16 value rows of unit k
+    auto issue = [&](int k) {
+      const int st = k % RING;
+      const uint32_t bar = bar0 + 8 * st;
+      const uint32_t dst = stages_s + st * STAGE;
+      const int e0 = list_begin + 16 * k;
+      const int nvalid = min(16, list_end - e0);
+      if (lane == 0) {
+        sm_issued[st] += 1;
+        sm_tag[st] = k;
+        ptx::mbar_arrive_expect_tx(bar, nvalid * (DK + kDV) * 2);
+      }
+      __syncwarp();
+      const int row = lane & 15;
+      if (row < nvalid) {
+        const int e = e0 + row;
+        size_t slot;
+        const __half* base_k;
+        const __half* base_v;
+        if (e < w.ret.n) {
+          slot = static_cast<size_t>(bh) * kMaxRetained + e;
+          base_k = cb.ret_k;
+          base_v = cb.ret_v;
+        } else {
+          const int pos = w.Q + (e - w.ret.n);
+          slot = static_cast<size_t>(bh) * d.cap + pos % d.cap;
+          base_k = cb.win_k;
+          base_v = cb.win_v;
+        }
+        if (lane < 16)
+          ptx::bulk_g2s(dst + row * R::KST, base_k + slot * DK, DK * 2, bar);
+        else
+          ptx::bulk_g2s(dst + 16 * R::KST + row * R::VST, base_v + slot * kDV, kDV * 2, bar);
+      }
+    };
+
+    if (warp == 0)
+      for (int k = 0; k < RING && k < n_units; ++k) issue(k);
+    for (int k = warp; k < n_units; k += kWarps) {
+      const int st = k % RING;
+      const bool ok = ptx::wait_equal_bounded(sm_tag + st, k, kWaitLimitNs) &&
+                      ptx::mbar_wait_bounded(bar0 + 8 * st, (k / RING) & 1, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, ok)) {
+        failed = true;
+        break;
+      }
+      const uint32_t S = stages_s + st * STAGE;
+      const int nvalid = min(16, list_end - (list_begin + 16 * k));
+      // scores: A = 16 key rows via ldmatrix, B = q (hi columns only)
+      float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      const int mi = lane >> 3;                         // which 8x8 matrix this lane addresses
+      const int arow = (mi & 1) * 8 + (lane & 7);
 #pragma unroll
-    for (int s = 0; s < KSTEPS; ++s) {
-      uint32_t a0, a1, a2, a3;
-      ptx::ldmatrix_x4(S + arow * R::KST + (16 * s + (mi >> 1) * 8) * 2, a0, a1, a2, a3);
-      ptx::mma_16816(cs, a0, a1, a2, a3, qn[s][0], qn[s][1]);
-    }
-    float s0 = (cs[0] + cs[1]) * alpha;
-    float s1 = (cs[2] + cs[3]) * alpha;
-    if (qr >= nvalid) s0 = -INFINITY;
-    if (qr + 8 >= nvalid) s1 = -INFINITY;
-    float gmax = fmaxf(s0, s1);
-    gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 4));
-    gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
-    gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
-    // The reference maximum moves only when a score exceeds it by more than
-    // kLazyRescale (log2 units): weights then stay below 2^kLazyRescale and the
-    // accumulators are rescaled rarely.
-    const float m_new = fmaxf(m_run, gmax);
-    if (__any_sync(0xffffffffu, m_new > m_run + kLazyRescale)) {
-      const float a = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m_run - m_new);
-      l_run *= a;
+      for (int s = 0; s < KSTEPS; ++s) {
+        uint32_t a0, a1, a2, a3;
+        ptx::ldmatrix_x4(S + arow * R::KST + (16 * s + (mi >> 1) * 8) * 2, a0, a1, a2, a3);
+        ptx::mma_16816(cs, a0, a1, a2, a3, qn[s][0], qn[s][1]);
+      }
+      float s0 = (cs[0] + cs[1]) * alpha;
+      float s1 = (cs[2] + cs[3]) * alpha;
+      if (qr >= nvalid) s0 = -INFINITY;
+      if (qr + 8 >= nvalid) s1 = -INFINITY;
+      float gmax = fmaxf(s0, s1);
+      gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 4));
+      gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 8));
+      gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
+      const float m_new = fmaxf(m_run, gmax);
+      if (__any_sync(0xffffffffu, m_new > m_run + kLazyRescale)) {
+        const float a = (m_new == -INFINITY) ? 1.0f : ptx::ex2(m_run - m_new);
+        l_run *= a;
 #pragma unroll
-      for (int mv = 0; mv < 8; ++mv)
+        for (int mv = 0; mv < 8; ++mv)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) co[mv][e] *= a;
-      m_run = m_new;
-    }
-    const float m_use = m_run == -INFINITY ? 0.0f : m_run;
-    const float p0 = ptx::ex2(s0 - m_use);
-    const float p1 = ptx::ex2(s1 - m_use);
-    l_run += p0 + p1;
-    uint32_t x0, x1;
-    ptx::split_hi_lo_pair(p0, p1, x0, x1);
-    const uint32_t bp0 = ptx::movmatrix_trans(x0);
-    const uint32_t bp1 = ptx::movmatrix_trans(x1);
-    // p.V: A = V^T tiles via ldmatrix.trans (rows = tokens in shared memory)
-    const int vrow = (mi >> 1) * 8 + (lane & 7);
+          for (int e = 0; e < 4; ++e) co[mv][e] *= a;
+        m_run = m_new;
+      }
+      const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+      const float p0 = ptx::ex2(s0 - m_use);
+      const float p1 = ptx::ex2(s1 - m_use);
+      l_run += p0 + p1;
+      uint32_t x0, x1;
+      ptx::split_hi_lo_pair(p0, p1, x0, x1);
+      const uint32_t bp0 = ptx::movmatrix_trans(x0);
+      const uint32_t bp1 = ptx::movmatrix_trans(x1);
+      // p.V: A = V^T tiles via ldmatrix.trans (rows = tokens in shared memory)
+      const int vrow = (mi >> 1) * 8 + (lane & 7);
 #pragma unroll
-    for (int mv = 0; mv < 8; ++mv) {
-      uint32_t a0, a1, a2, a3;
-      ptx::ldmatrix_x4_trans(S + 16 * R::KST + vrow * R::VST + (16 * mv + (mi & 1) * 8) * 2, a0, a1,
-                             a2, a3);
-      ptx::mma_16816(co[mv], a0, a1, a2, a3, bp0, bp1);
-    }
-    __syncwarp();
-    if (k + RING < n_units) {
-      if (lane == 0) ptx::fence_proxy_async_smem();
-      issue(k + RING);
+      for (int mv = 0; mv < 8; ++mv) {
+        uint32_t a0, a1, a2, a3;
+        ptx::ldmatrix_x4_trans(S + 16 * R::KST + vrow * R::VST + (16 * mv + (mi & 1) * 8) * 2, a0, a1,
+                               a2, a3);
+        ptx::mma_16816(co[mv], a0, a1, a2, a3, bp0, bp1);
+      }
+      __syncwarp();
+      if (k + RING < n_units) {
+        if (lane == 0) ptx::fence_proxy_async_smem();
+        issue(k + RING);
+      }
     }
   }
 
@@ -260,12 +678,18 @@ decode_fp16_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict_
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 4);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 8);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+#pragma unroll
+  for (int gg = 0; gg < G::NVG; ++gg) {
+    zsum[gg] += __shfl_xor_sync(0xffffffffu, zsum[gg], 4);
+    zsum[gg] += __shfl_xor_sync(0xffffffffu, zsum[gg], 8);
+    zsum[gg] += __shfl_xor_sync(0xffffffffu, zsum[gg], 16);
+  }
   if (failed) {
     m_run = -INFINITY;
     l_run = 0.0f;
   }
   __syncthreads();   // every warp is done with the stages: reuse them for the merge
-  float* sm_o = reinterpret_cast<float*>(smem + Smem::kStages);      // [kWarps][NREP][kDV]
+  float* sm_o = reinterpret_cast<float*>(smem + SM::kStages);        // [kWarps][NREP][kDV]
   float* sm_ml = sm_o + kWarps * NREP * kDV;                         // [kWarps][NREP][2]
   if (cvalid) {
     float* dst = sm_o + (warp * NREP + qi) * kDV;
@@ -273,9 +697,21 @@ decode_fp16_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict_
     for (int mv = 0; mv < 8; ++mv) {
       float o0 = co[mv][0] + co[mv][1];
       float o1 = co[mv][2] + co[mv][3];
+      int c0, c1;
+      if (quant) {
+        const int gg = mv / G::MPG, ml = mv % G::MPG;
+        c0 = gg * GV + qr * G::CPG + ml;
+        c1 = c0 + G::MPG;
+        o0 = fmaf(o0, static_cast<float>(1 << (24 - value_code_shift<VB, G::RUN>(ml))), zsum[gg]);
+        o1 = fmaf(o1, static_cast<float>(1 << (24 - value_code_shift<VB, G::RUN>(ml + G::MPG))),
+                  zsum[gg]);
+      } else {
+        c0 = 16 * mv + qr;
+        c1 = c0 + 8;
+      }
       if (failed) o0 = o1 = 0.0f;
-      dst[16 * mv + qr] = o0;
-      dst[16 * mv + qr + 8] = o1;
+      dst[c0] = o0;
+      dst[c1] = o1;
     }
     if (qr == 0) {
       sm_ml[(warp * NREP + qi) * 2] = m_run;
@@ -302,23 +738,22 @@ decode_fp16_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict_
   }
 }
 
-// Launches the fp16-list CTAs: grid.x = w.splits_f, writing partials splits_q .. splits-1.
-template <int DK, int NREP>
-cudaError_t launch_fp16(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
-                        const Partials& p, cudaStream_t s) {
-  constexpr int stage = stage_bytes<DK>();
-  constexpr int ring = ring_stages<DK>();
-  int smem = Smem::kStages + ring * stage;
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT>
+cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
+                   const Partials& p, cudaStream_t s) {
+  constexpr int stage = stage_bytes<KB, VB, DK, GV, GK, QUANT>();
+  constexpr int ring = ring_stages<KB, VB, DK, GV, GK, QUANT>();
+  int smem = Smem<DK / 16>::kStages + ring * stage;
   const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
-  if (Smem::kStages + merge > smem) smem = Smem::kStages + merge;
-  auto kern = decode_fp16_kernel<DK, NREP>;
+  if (Smem<DK / 16>::kStages + merge > smem) smem = Smem<DK / 16>::kStages + merge;
+  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT>;
   static int configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  dim3 grid(w.splits_f, d.Hkv, d.B);
+  dim3 grid(w.splits, d.Hkv, d.B);
   kern<<<grid, kThreads, smem, s>>>(d, c, w, q, p);
   return cudaGetLastError();
 }

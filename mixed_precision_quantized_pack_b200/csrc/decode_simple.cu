@@ -68,13 +68,7 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
       if (retained) continue;                                   // read from the fp16 list
       const uint32_t* kr = cb.kcode + (static_cast<size_t>(bh) * d.lcap + i) * d.kw;
       const __half2* ks = cb.ksz + (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * d.dk;
-      // value codes: channel-major inside the key group, token i % gk of channel ch at
-      // word (i % gk) / perv of that channel's row
-      const int vrw = d.gk / perv;
-      const uint32_t* vr = cb.vcode +
-                           (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * d.dv * vrw +
-                           (i % d.gk) / perv;
-      const int vshift = ((i % d.gk) % perv) * d.vb;
+      const uint32_t* vr = cb.vcode + (static_cast<size_t>(bh) * d.lcap + i) * d.vw;
       const __half2* vs = cb.vsz + (static_cast<size_t>(bh) * d.lcap + i) * d.nvg;
 #pragma unroll
       for (int j = 0; j < kMaxC; ++j) {
@@ -88,7 +82,7 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
         }
         if (j < cv) {
           const int ch = lane + 32 * j;
-          const uint32_t code = (vr[static_cast<size_t>(ch) * vrw] >> vshift) & maskv;
+          const uint32_t code = (vr[ch / perv] >> ((ch % perv) * d.vb)) & maskv;
           const float2 sz = __half22float2(vs[ch / d.gv]);
           vh[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
         }

@@ -122,10 +122,8 @@ int split_cap(const kvq::Dims& d) {
   return std::min(256, std::max(2, 8192 / rows));
 }
 
-// Occupancy assumed by the planner (CTAs per SM) for the kernel that reads the bulk of the
-// tokens: the tcgen05 kernel runs two CTAs per SM (its tensor memory and shared memory
-// take half an SM each); the fp16 mma.sync kernel and the generic kernel run four.
-int ctas_per_sm(const kvq::Dims& d, bool fast) { return fast && d.quantized() ? 2 : 4; }
+// Occupancy assumed by the planner (CTAs per SM) for each decode kernel.
+int ctas_per_sm(bool fast) { return fast ? 3 : 4; }
 
 // Chooses the split counts: the number of CTAs per (b, kv head) over the quantized
 // groups and over the fp16 tokens, trading wave quantization against per-CTA cost.
@@ -138,7 +136,7 @@ int plan_decode(const kvq::Dims& d, int L, int sm_count, int num_splits, bool fa
   const int nF = nret + (L - Q);
   const int rows = d.B * d.Hkv;
   const int cap = split_cap(d);
-  const long long slots = static_cast<long long>(sm_count) * ctas_per_sm(d, fast);
+  const long long slots = static_cast<long long>(sm_count) * ctas_per_sm(fast);
   // cost model in bytes read: per quantized group, per fp16 token, per CTA
   const double bq = d.quantized()
                         ? static_cast<double>(d.gk) * (d.kw * 4 + d.vw * 4 + d.nvg * 4) + d.dk * 4.0

@@ -10,8 +10,7 @@
 // Every step is an explicit IEEE round-to-nearest intrinsic so that no FMA
 // contraction or fast-math rewrite can change a code.  Keys: one group per
 // channel over group_k consecutive tokens (LogQuant §5, per-channel keys).
-// Values: one group per token over group_v consecutive channels, codes stored
-// channel-major inside each key group.
+// Values: one group per token over group_v consecutive channels.
 #include "kvq_internal.cuh"
 
 namespace kvq {
@@ -80,49 +79,44 @@ __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_row
   }
 }
 
-// One thread per (kv row, token); a warp holds 32 consecutive tokens.  Values are
-// stored channel-major inside each key group: the word of channel c holds 32/BITS
-// consecutive tokens, so the 32/BITS lanes of those tokens OR their codes together.
-// n_tokens and t_begin are multiples of gk, itself a multiple of 32/BITS.
+// One thread per (kv row, token, value group).  gv is a multiple of 8 and of 32/BITS.
 template <int BITS>
 __global__ void quantize_values_kernel(const __half* __restrict__ src, int src_rows, int dv,
-                                       int gv, int gk, int t_begin, int n_tokens, int nbh, int lcap,
+                                       int gv, int t_begin, int n_tokens, int nbh, int lcap,
                                        uint32_t* __restrict__ vcode, __half2* __restrict__ vsz) {
-  constexpr int per = 32 / BITS;                    // tokens per word
-  const int lane = threadIdx.x & 31;
-  const int warps_per_bh = (n_tokens + 31) / 32;
-  const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (gw >= static_cast<long long>(nbh) * warps_per_bh) return;      // uniform per warp
-  const int bh = static_cast<int>(gw / warps_per_bh);
-  const int i = static_cast<int>(gw % warps_per_bh) * 32 + lane;
-  const bool valid = i < n_tokens;
-  const int t = t_begin + (valid ? i : 0);
-  const __half* x = src + (static_cast<size_t>(bh) * src_rows + t % src_rows) * dv;
   const int nvg = dv / gv;
-  const int words_per_row = gk / per;               // words of one channel in one group
-  uint32_t* out = vcode + (static_cast<size_t>(bh) * (lcap / gk) + t / gk) * dv * words_per_row +
-                  (t % gk) / per;
-  const int shift = (t % per) * BITS;
-  for (int vg = 0; vg < nvg; ++vg) {
-    const __half* xg = x + vg * gv;
+  const long long total = static_cast<long long>(nbh) * n_tokens * nvg;
+  constexpr int per = 32 / BITS;
+  const int vw = dv / per;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int gidx = static_cast<int>(idx % nvg);
+    const long long r = idx / nvg;
+    const int t = t_begin + static_cast<int>(r % n_tokens);
+    const int bh = static_cast<int>(r / n_tokens);
+    const int row = t % src_rows;
+    const __half* x = src + (static_cast<size_t>(bh) * src_rows + row) * dv + gidx * gv;
     float mn = INFINITY, mx = -INFINITY;
     for (int j = 0; j < gv; j += 8) {
-      const uint4 u = *reinterpret_cast<const uint4*>(xg + j);
-      const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+      const uint4 u = *reinterpret_cast<const uint4*>(x + j);
+      const __half2* h = reinterpret_cast<const __half2*>(&u);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h2[e]);
+        const float2 f = __half22float2(h[e]);
         mn = fminf(mn, fminf(f.x, f.y));
         mx = fmaxf(mx, fmaxf(f.x, f.y));
       }
     }
     const GroupParams gp = group_params<BITS>(mn, mx);
-    if (valid) vsz[(static_cast<size_t>(bh) * lcap + t) * nvg + vg] = gp.sz;
-    for (int c = 0; c < gv; ++c) {
-      uint32_t part = valid ? quant_code<BITS>(__half2float(xg[c]), gp) << shift : 0u;
-#pragma unroll
-      for (int off = 1; off < per; off <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, off);
-      if (valid && shift == 0) out[static_cast<size_t>(vg * gv + c) * words_per_row] = part;
+    vsz[(static_cast<size_t>(bh) * lcap + t) * nvg + gidx] = gp.sz;
+    uint32_t* out = vcode + (static_cast<size_t>(bh) * lcap + t) * vw + gidx * (gv / per);
+    for (int w = 0; w < gv / per; ++w) {
+      uint32_t word = 0;
+      for (int k = 0; k < per; ++k) {
+        const float xv = __half2float(x[w * per + k]);
+        word |= quant_code<BITS>(xv, gp) << (k * BITS);
+      }
+      out[w] = word;
     }
   }
 }
@@ -221,13 +215,13 @@ cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_row
                                    int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s) {
   if (n_tokens <= 0) return cudaSuccess;
   const int nbh = d.B * d.Hkv;
-  const long long threads = static_cast<long long>(nbh) * ((n_tokens + 31) / 32) * 32;
+  const long long items = static_cast<long long>(nbh) * n_tokens * d.nvg;
   const int block = 256;
-  const int grid = static_cast<int>((threads + block - 1) / block);
+  const int grid = grid_for(items, block);
   switch (d.vb) {
-    case 2: quantize_values_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, d.gk, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
-    case 4: quantize_values_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, d.gk, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
-    case 8: quantize_values_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, d.gk, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
+    case 2: quantize_values_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
+    case 4: quantize_values_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
+    case 8: quantize_values_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

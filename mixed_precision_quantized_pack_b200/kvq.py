@@ -306,7 +306,7 @@ class KVCache:
         shapes = {
             "kcode": (torch.int32, (B, H, lcap, dk * kb // 32)),
             "ksz": (torch.float16, (B, H, lcap // gk, dk, 2)),
-            "vcode": (torch.int32, (B, H, lcap // gk, dv, gk * vb // 32)),
+            "vcode": (torch.int32, (B, H, lcap, dv * vb // 32)),
             "vsz": (torch.float16, (B, H, lcap, dv // gv, 2)),
             "win_k": (torch.float16, (B, H, cap, dk)),
             "win_v": (torch.float16, (B, H, cap, dv)),

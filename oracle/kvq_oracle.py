@@ -24,12 +24,10 @@ What it computes, step by step in the order the pages give it:
        code = 0 if s16 == 0 else clamp(rint(fl32(fl32(x - z16) / s16)), 0, 2^b-1)
    All arithmetic is IEEE binary32 with round-to-nearest-even, one operation at
    a time (numpy float32 ufuncs), rint is half-to-even.
-4. Packing: codes are packed least significant bits first into little-endian
-   uint32 words, element i of a b-bit row in word i // (32/b) at bit
-   (i % (32/b)) * b.  A key row is one token's d_k channels.  A value row is one
-   channel's G_k tokens of one key group (values are stored channel-major inside
-   each key group; the pages fix no memory layout, this is the library's).
-   (scale, zero) pairs are stored as fp16 pairs.
+4. Packing: within a token row, codes are packed channel by channel, least
+   significant bits first, into little-endian uint32 words (channel c of a b-bit
+   row lives in word c // (32/b) at bit (c % (32/b)) * b).  (scale, zero) pairs
+   are stored as fp16 pairs.
 5. Log-spaced retention (LogQuant §Méthodologie 2, "density halves further
    back"; the printed text is garbled).  Reading: among the quantized positions
    p < Q, p is kept in fp16 iff p is a multiple of 2^floor(log2(Q - p)); this
@@ -43,7 +41,7 @@ What it computes, step by step in the order the pages give it:
 
 Buffer formats mirror the CUDA library's so the tests can compare bytes:
   kcode u32 [B][Hkv][Lcap][d_k*kb/32]        ksz fp16 [B][Hkv][Lcap/Gk][d_k][2]
-  vcode u32 [B][Hkv][Lcap/Gk][d_v][Gk*vb/32] vsz fp16 [B][Hkv][Lcap][d_v/Gv][2]
+  vcode u32 [B][Hkv][Lcap][d_v*vb/32]        vsz fp16 [B][Hkv][Lcap][d_v/Gv][2]
   win_k/v fp16 [B][Hkv][C][d] with token p in slot p % C,
           C = R + G_k (quantized caches) or Lcap (bits 16)
   ret_k/v fp16 [B][Hkv][32][d] in ascending position order, ret_idx int32 list.
@@ -135,7 +133,7 @@ def quantize_values(v: np.ndarray, group_v: int, bits: int):
 
 # ---------------------------------------------------------------- packing -----
 def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
-    """[..., d] codes -> [..., d*bits/32] uint32 words, elements LSB-first (step 4)."""
+    """[..., d] codes -> [..., d*bits/32] uint32 words, channels LSB-first (step 4)."""
     per = 32 // bits
     d = codes.shape[-1]
     assert d % per == 0
@@ -201,8 +199,7 @@ class OracleCache:
             self.cap = self.R + self.gk
             self.kcode = np.zeros((B, H, self.lcap, self.dk * self.kb // 32), np.uint32)
             self.ksz = np.zeros((B, H, self.lcap // self.gk, self.dk, 2), np.float16)
-            self.vcode = np.zeros((B, H, self.lcap // self.gk, self.dv, self.gk * self.vb // 32),
-                                  np.uint32)
+            self.vcode = np.zeros((B, H, self.lcap, self.dv * self.vb // 32), np.uint32)
             self.vsz = np.zeros((B, H, self.lcap, self.dv // self.gv, 2), np.float16)
             self.ret_k = np.zeros((B, H, MAX_RETAINED, self.dk), np.float16)
             self.ret_v = np.zeros((B, H, MAX_RETAINED, self.dv), np.float16)
@@ -220,8 +217,7 @@ class OracleCache:
         vc, vsz = quantize_values(v_rows, self.gv, self.vb)
         self.kcode[b, h, t0:t0 + n] = pack_codes(kc, self.kb)
         self.ksz[b, h, t0 // self.gk:(t0 + n) // self.gk] = ksz
-        vc_cm = vc.reshape(n // self.gk, self.gk, self.dv).transpose(0, 2, 1)  # [groups][dv][Gk]
-        self.vcode[b, h, t0 // self.gk:(t0 + n) // self.gk] = pack_codes(vc_cm, self.vb)
+        self.vcode[b, h, t0:t0 + n] = pack_codes(vc, self.vb)
         self.vsz[b, h, t0:t0 + n] = vsz
 
     def prefill(self, k: np.ndarray, v: np.ndarray):
@@ -290,8 +286,7 @@ class OracleCache:
             ks = np.repeat(ksz[:, :, 0], self.gk, axis=0)
             kz = np.repeat(ksz[:, :, 1], self.gk, axis=0)
             kh[:Q] = dequantize(kc, ks, kz)
-            vc = unpack_codes(self.vcode[b, h, :Q // self.gk], self.vb)        # [groups][dv][Gk]
-            vc = vc.transpose(0, 2, 1).reshape(Q, self.dv)                     # [Q][dv]
+            vc = unpack_codes(self.vcode[b, h, :Q], self.vb)                   # [Q][dv]
             vsz = self.vsz[b, h, :Q]                                            # [Q][ngv][2]
             vs = np.repeat(vsz[:, :, 0], self.gv, axis=1)
             vz = np.repeat(vsz[:, :, 1], self.gv, axis=1)

@@ -37,7 +37,7 @@ def compare_state(gc: K.KVCache, oc: O.OracleCache, b_rows=None, where=""):
     c = gc.cfg
     if c["k_bits"] != 16 and Q:
         gk = c["group_k"]
-        pairs = [("kcode", slice(0, Q)), ("ksz", slice(0, Q // gk)), ("vcode", slice(0, Q // gk)),
+        pairs = [("kcode", slice(0, Q)), ("ksz", slice(0, Q // gk)), ("vcode", slice(0, Q)),
                  ("vsz", slice(0, Q))]
         for name, sl in pairs:
             g = gc.view(name)[rows][:, :, sl].cpu().numpy()

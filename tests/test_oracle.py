@@ -34,22 +34,6 @@ def test_golden_quantizer_examples():
         assert f16bits(z[0]) == int(zbits[0], 16)
 
 
-def test_golden_channel_major_value_codes():
-    """Value codes of a key group are stored channel by channel, tokens LSB-first."""
-    cfg = dict(batch=1, n_q_heads=1, n_kv_heads=1, d_k=32, d_v=32, k_bits=4, v_bits=2, group_k=16,
-               group_v=16, window=16, log_retain=0, max_context=48)
-    t = np.arange(32)[:, None]
-    c = np.arange(32)[None, :]
-    v = np.where(c < 16, (t + c) % 4, (3 * t + c) % 4).astype(np.float16)
-    k = np.zeros((32, 32), np.float16)
-    cache = O.OracleCache(cfg)
-    cache.prefill(k[None, None], v[None, None])
-    assert cache.Q == 16
-    assert np.all(cache.vsz[0, 0, :16, :, 0] == 1) and np.all(cache.vsz[0, 0, :16, :, 1] == 0)
-    for ch, word in read_golden("value_layout_worked.txt"):
-        assert int(cache.vcode[0, 0, 0, int(ch[0]), 0]) == int(word[0], 16), ch
-
-
 def test_golden_packing_examples():
     for bits, codes, words in read_golden("packing_worked.txt"):
         b = int(bits[0])
