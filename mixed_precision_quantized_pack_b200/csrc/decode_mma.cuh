@@ -24,7 +24,9 @@
 // code * 2^(p-24), p its bit offset (p + b <= 8 after at most one byte shift), so
 // unpacking is one AND per two codes; the factor 2^-p goes into q' and the common
 // 2^-24 into the softmax scale.  The zero points add sum_c q_c z_{g,c} per group,
-// computed by one more MMA per k-step with z in A and q in B.
+// computed by one more MMA per k-step with z in A and q in B.  A group's key
+// (scale, zero) block lists, per packed word, the channel pairs of its registers,
+// so the B pairs (s_c, s_c+16/b) and the A pairs (z_c, z_c+16/b) are plain loads.
 //
 // p.V uses the transposed orientation: channels on M, the 16 tokens on K, and on
 // N again (hi, lo) pairs, now of p_j * s_{j,g} (per-token value scale), moved from
@@ -406,9 +408,9 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const int rho = 2 * ls + j;
-              const uint32_t mlo = meta[rho], mhi = meta[rho + 16 / KB];
-              const uint32_t s2 = ptx::prmt(mlo, mhi, 0x5410u);   // (s_lo, s_hi)
-              za[j] = ptx::prmt(mlo, mhi, 0x7632u);               // (z_lo, z_hi)
+              // the word's block holds (s_c, s_c+16/KB) for each register, then the zeros
+              const uint32_t s2 = meta[rho];
+              za[j] = meta[G::RPW + rho];
               const __half2 qs = ptx::u32_as_h2(qfx[2 * ls + j]);
               const __half2 sc = ptx::u32_as_h2(s2);
               const __half2 hi = __hmul2(qs, sc);

@@ -67,7 +67,8 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
       for (int r = 0; r < w.ret.n; ++r) retained |= (w.ret.pos[r] == i);
       if (retained) continue;                                   // read from the fp16 list
       const uint32_t* kr = cb.kcode + (static_cast<size_t>(bh) * d.lcap + i) * d.kw;
-      const __half2* ks = cb.ksz + (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * d.dk;
+      const __half* ks = reinterpret_cast<const __half*>(cb.ksz) +
+                         (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * 2 * d.dk;
       const uint32_t* vr = cb.vcode + (static_cast<size_t>(bh) * d.lcap + i) * d.vw;
       const __half2* vs = cb.vsz + (static_cast<size_t>(bh) * d.lcap + i) * d.nvg;
 #pragma unroll
@@ -77,8 +78,9 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
         if (j < ck) {
           const int ch = lane + 32 * j;
           const uint32_t code = (kr[ch / perk] >> ((ch % perk) * d.kb)) & maskk;
-          const float2 sz = __half22float2(ks[ch]);
-          kh[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
+          // (scale, zero) of channel ch in the group's paired block
+          const int slot = (ch / perk) * 2 * perk + (ch % perk % (perk / 2)) * 2 + (ch % perk) / (perk / 2);
+          kh[j] = fmaf(static_cast<float>(code), __half2float(ks[slot]), __half2float(ks[slot + perk]));
         }
         if (j < cv) {
           const int ch = lane + 32 * j;

@@ -9,7 +9,8 @@
 //   code = s == 0 ? 0 : clamp(rint(fl32(fl32(x - z) / s)), 0, 2^b - 1)
 // Every step is an explicit IEEE round-to-nearest intrinsic so that no FMA
 // contraction or fast-math rewrite can change a code.  Keys: one group per
-// channel over group_k consecutive tokens (LogQuant §5, per-channel keys).
+// channel over group_k consecutive tokens (LogQuant §5, per-channel keys); a group's
+// (scale, zero) block is stored in the order the decode kernel pairs channels.
 // Values: one group per token over group_v consecutive channels.
 #include "kvq_internal.cuh"
 
@@ -65,7 +66,16 @@ __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_row
     mx = fmaxf(mx, x);
   }
   const GroupParams gp = group_params<BITS>(mn, mx);
-  ksz[(static_cast<size_t>(bh) * (lcap / gk) + g) * dk + c] = gp.sz;
+  {
+    // the group's block of 2*dk fp16: per packed word w, the scales of channels
+    // (w*per + i, w*per + i + per/2) for i < per/2, then their zeros in the same order
+    constexpr int per_w = 32 / BITS, half_w = 16 / BITS;
+    const int wd = c / per_w, r = c % per_w;
+    const int slot = wd * 2 * per_w + (r % half_w) * 2 + r / half_w;
+    __half* blk = reinterpret_cast<__half*>(ksz) + (static_cast<size_t>(bh) * (lcap / gk) + g) * 2 * dk;
+    blk[slot] = __low2half(gp.sz);
+    blk[slot + per_w] = __high2half(gp.sz);
+  }
   constexpr int per = 32 / BITS;                    // channels per word
   const int words = dk / per;
   for (int t = 0; t < gk; ++t) {

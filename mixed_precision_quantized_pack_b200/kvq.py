@@ -305,7 +305,7 @@ class KVCache:
             cap = c["window"] + gk
         shapes = {
             "kcode": (torch.int32, (B, H, lcap, dk * kb // 32)),
-            "ksz": (torch.float16, (B, H, lcap // gk, dk, 2)),
+            "ksz": (torch.float16, (B, H, lcap // gk, 2 * dk)),
             "vcode": (torch.int32, (B, H, lcap, dv * vb // 32)),
             "vsz": (torch.float16, (B, H, lcap, dv // gv, 2)),
             "win_k": (torch.float16, (B, H, cap, dk)),

@@ -26,8 +26,13 @@ What it computes, step by step in the order the pages give it:
    a time (numpy float32 ufuncs), rint is half-to-even.
 4. Packing: within a token row, codes are packed channel by channel, least
    significant bits first, into little-endian uint32 words (channel c of a b-bit
-   row lives in word c // (32/b) at bit (c % (32/b)) * b).  (scale, zero) pairs
-   are stored as fp16 pairs.
+   row lives in word c // (32/b) at bit (c % (32/b)) * b).  Value (scale, zero)
+   pairs are stored as fp16 pairs.  The key (scale, zero) of one group follow the
+   packed words of a key row: for word w (channels w*P .. w*P+P-1, P = 32/b,
+   H = 16/b) come the P scales in the order (w*P+i, w*P+i+H) for i < H, then the
+   P zeros in the same order (key_meta_order).  The pages fix no memory layout;
+   this one puts the two channels whose codes share a 32-bit word half by half
+   next to each other.
 5. Log-spaced retention (LogQuant §Méthodologie 2, "density halves further
    back"; the printed text is garbled).  Reading: among the quantized positions
    p < Q, p is kept in fp16 iff p is a multiple of 2^floor(log2(Q - p)); this
@@ -40,7 +45,7 @@ What it computes, step by step in the order the pages give it:
    (LogQuant §4, A.V = A_P.V_P).  GQA: query head hq reads kv head hq // n_rep.
 
 Buffer formats mirror the CUDA library's so the tests can compare bytes:
-  kcode u32 [B][Hkv][Lcap][d_k*kb/32]        ksz fp16 [B][Hkv][Lcap/Gk][d_k][2]
+  kcode u32 [B][Hkv][Lcap][d_k*kb/32]        ksz fp16 [B][Hkv][Lcap/Gk][2*d_k] (key_meta_order)
   vcode u32 [B][Hkv][Lcap][d_v*vb/32]        vsz fp16 [B][Hkv][Lcap][d_v/Gv][2]
   win_k/v fp16 [B][Hkv][C][d] with token p in slot p % C,
           C = R + G_k (quantized caches) or Lcap (bits 16)
@@ -143,6 +148,35 @@ def pack_codes(codes: np.ndarray, bits: int) -> np.ndarray:
     return words.astype(np.uint32)
 
 
+def key_meta_order(d_k: int, bits: int):
+    """Slot order of one key group's fp16 (scale, zero) block (step 4): for slot i of
+    the 2*d_k slots, the channel it holds and whether it is the scale (0) or zero (1)."""
+    per, half = 32 // bits, 16 // bits
+    chan, which = [], []
+    for w in range(d_k // per):
+        for part in (0, 1):                          # scales, then zeros
+            for i in range(half):
+                for c in (w * per + i, w * per + i + half):
+                    chan.append(c)
+                    which.append(part)
+    return np.array(chan), np.array(which)
+
+
+def pack_key_meta(sz: np.ndarray, bits: int) -> np.ndarray:
+    """sz fp16 [..., d_k, 2] (scale, zero per channel) -> [..., 2*d_k] in key_meta_order."""
+    chan, which = key_meta_order(sz.shape[-2], bits)
+    return sz[..., chan, which]
+
+
+def unpack_key_meta(block: np.ndarray, bits: int) -> np.ndarray:
+    """Inverse of pack_key_meta: [..., 2*d_k] -> [..., d_k, 2]."""
+    d_k = block.shape[-1] // 2
+    chan, which = key_meta_order(d_k, bits)
+    out = np.empty(block.shape[:-1] + (d_k, 2), block.dtype)
+    out[..., chan, which] = block
+    return out
+
+
 def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
     per = 32 // bits
     w = words.astype(np.uint64)[..., None]
@@ -198,7 +232,7 @@ class OracleCache:
             self.lcap = -(-self.max_context // self.gk) * self.gk
             self.cap = self.R + self.gk
             self.kcode = np.zeros((B, H, self.lcap, self.dk * self.kb // 32), np.uint32)
-            self.ksz = np.zeros((B, H, self.lcap // self.gk, self.dk, 2), np.float16)
+            self.ksz = np.zeros((B, H, self.lcap // self.gk, 2 * self.dk), np.float16)
             self.vcode = np.zeros((B, H, self.lcap, self.dv * self.vb // 32), np.uint32)
             self.vsz = np.zeros((B, H, self.lcap, self.dv // self.gv, 2), np.float16)
             self.ret_k = np.zeros((B, H, MAX_RETAINED, self.dk), np.float16)
@@ -216,7 +250,7 @@ class OracleCache:
         kc, ksz = quantize_keys(k_rows, self.gk, self.kb)
         vc, vsz = quantize_values(v_rows, self.gv, self.vb)
         self.kcode[b, h, t0:t0 + n] = pack_codes(kc, self.kb)
-        self.ksz[b, h, t0 // self.gk:(t0 + n) // self.gk] = ksz
+        self.ksz[b, h, t0 // self.gk:(t0 + n) // self.gk] = pack_key_meta(ksz, self.kb)
         self.vcode[b, h, t0:t0 + n] = pack_codes(vc, self.vb)
         self.vsz[b, h, t0:t0 + n] = vsz
 
@@ -282,7 +316,7 @@ class OracleCache:
         vh = np.empty((L, self.dv), np.float64)
         if Q:
             kc = unpack_codes(self.kcode[b, h, :Q], self.kb)                   # [Q][dk]
-            ksz = self.ksz[b, h, :Q // self.gk]                                 # [ng][dk][2]
+            ksz = unpack_key_meta(self.ksz[b, h, :Q // self.gk], self.kb)       # [ng][dk][2]
             ks = np.repeat(ksz[:, :, 0], self.gk, axis=0)
             kz = np.repeat(ksz[:, :, 1], self.gk, axis=0)
             kh[:Q] = dequantize(kc, ks, kz)

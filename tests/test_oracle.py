@@ -34,6 +34,23 @@ def test_golden_quantizer_examples():
         assert f16bits(z[0]) == int(zbits[0], 16)
 
 
+def test_golden_key_meta_order():
+    """Slot order of a key group's (scale, zero) block, against a hand-written list."""
+    for bits, order in read_golden("key_meta_worked.txt"):
+        b = int(bits[0])
+        d_k = len(order) // 2
+        chan, which = O.key_meta_order(d_k, b)
+        got = [("s" if w == 0 else "z") + str(c) for c, w in zip(chan, which)]
+        assert got == order, (b, got)
+        # pack/unpack are mutually inverse and place channel c's scale where the list says
+        sz = np.arange(2 * d_k, dtype=np.float16).reshape(d_k, 2)
+        blk = O.pack_key_meta(sz, b)
+        for slot, name in enumerate(order):
+            c = int(name[1:])
+            assert blk[slot] == sz[c, 0 if name[0] == "s" else 1]
+        assert np.array_equal(O.unpack_key_meta(blk, b), sz)
+
+
 def test_golden_packing_examples():
     for bits, codes, words in read_golden("packing_worked.txt"):
         b = int(bits[0])
@@ -258,10 +275,11 @@ def test_shared_key_translation_is_softmax_null():
     a.prefill(k, v)
     b.prefill(k_mu, v)
     assert np.array_equal(a.kcode, b.kcode)
-    assert np.array_equal(a.ksz[..., 0], b.ksz[..., 0])
     ng = a.Q // gk
-    assert np.array_equal(b.ksz[0, 0, :ng, :, 1].astype(np.float64),
-                          a.ksz[0, 0, :ng, :, 1].astype(np.float64) + mu)
+    sa = O.unpack_key_meta(a.ksz[0, 0, :ng], 4)          # [ng][d][(scale, zero)]
+    sb = O.unpack_key_meta(b.ksz[0, 0, :ng], 4)
+    assert np.array_equal(sa[..., 0], sb[..., 0])
+    assert np.array_equal(sb[..., 1].astype(np.float64), sa[..., 1].astype(np.float64) + mu)
     assert np.allclose(a.decode(q), b.decode(q), rtol=1e-11, atol=1e-12)
 
 
