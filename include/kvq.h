@@ -31,7 +31,9 @@
  *               c/(32/k_bits), bit (c%(32/k_bits))*k_bits (LSB first)
  *   ksz    f16  [B][Hkv][Lcap/group_k][2*d_k]  (scale, zero) per key group and channel:
  *               for each packed word w of a key row (P = 32/k_bits channels, H = P/2)
- *               the scales of channels (wP+i, wP+i+H), i < H, then their zeros
+ *               the scales of channels (wP+i, wP+i+H), i < H, then their zeros; with
+ *               W = d_k*k_bits/32 words and 4 | W, word w's block is stored at
+ *               position (w % (W/4))*4 + w/(W/4)
  *   vcode  u32  [B][Hkv][Lcap][d_v*v_bits/32]   same packing per token row
  *   vsz    f16  [B][Hkv][Lcap][d_v/group_v][2] (scale, zero) per token and value group
  *   win_k  f16  [B][Hkv][C][d_k]  token p in slot p % C, C = window + group_k

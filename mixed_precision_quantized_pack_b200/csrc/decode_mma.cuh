@@ -26,7 +26,9 @@
 // 2^-24 into the softmax scale.  The zero points add sum_c q_c z_{g,c} per group,
 // computed by one more MMA per k-step with z in A and q in B.  A group's key
 // (scale, zero) block lists, per packed word, the channel pairs of its registers,
-// so the B pairs (s_c, s_c+16/b) and the A pairs (z_c, z_c+16/b) are plain loads.
+// so the B pairs (s_c, s_c+16/b) and the A pairs (z_c, z_c+16/b) are plain loads;
+// the words' blocks are quarter-interleaved so that the four quads of a warp, which
+// read the four quarters of a key row, load neighbouring blocks.
 //
 // p.V uses the transposed orientation: channels on M, the 16 tokens on K, and on
 // N again (hi, lo) pairs, now of p_j * s_{j,g} (per-token value scale), moved from
@@ -384,7 +386,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
           uint32_t meta[G::CPW];
 #pragma unroll
           for (int c4 = 0; c4 < G::CPW; c4 += 4) {
-            const uint4 v4 = *reinterpret_cast<const uint4*>(skm + G::CPW * omega + c4);
+            // word omega = qi * WPT + u: its block is stored at position u * 4 + qi
+            const uint4 v4 = *reinterpret_cast<const uint4*>(skm + G::CPW * (u * 4 + qi) + c4);
             meta[c4] = v4.x;
             meta[c4 + 1] = v4.y;
             meta[c4 + 2] = v4.z;

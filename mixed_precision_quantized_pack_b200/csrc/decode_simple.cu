@@ -78,8 +78,10 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
         if (j < ck) {
           const int ch = lane + 32 * j;
           const uint32_t code = (kr[ch / perk] >> ((ch % perk) * d.kb)) & maskk;
-          // (scale, zero) of channel ch in the group's paired block
-          const int slot = (ch / perk) * 2 * perk + (ch % perk % (perk / 2)) * 2 + (ch % perk) / (perk / 2);
+          // (scale, zero) of channel ch in the group's paired, quarter-interleaved block
+          const int kwords = d.dk / perk, kq = kwords % 4 == 0 ? kwords / 4 : 0;
+          const int kwd = ch / perk, kpos = kq ? (kwd % kq) * 4 + kwd / kq : kwd;
+          const int slot = kpos * 2 * perk + (ch % perk % (perk / 2)) * 2 + (ch % perk) / (perk / 2);
           kh[j] = fmaf(static_cast<float>(code), __half2float(ks[slot]), __half2float(ks[slot + perk]));
         }
         if (j < cv) {

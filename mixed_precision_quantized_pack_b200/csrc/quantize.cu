@@ -68,10 +68,13 @@ __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_row
   const GroupParams gp = group_params<BITS>(mn, mx);
   {
     // the group's block of 2*dk fp16: per packed word w, the scales of channels
-    // (w*per + i, w*per + i + per/2) for i < per/2, then their zeros in the same order
+    // (w*per + i, w*per + i + per/2) for i < per/2, then their zeros in the same order;
+    // the words' blocks quarter-interleaved when 4 divides the words per row
     constexpr int per_w = 32 / BITS, half_w = 16 / BITS;
+    const int words = dk / per_w, quarter = words % 4 == 0 ? words / 4 : 0;
     const int wd = c / per_w, r = c % per_w;
-    const int slot = wd * 2 * per_w + (r % half_w) * 2 + r / half_w;
+    const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
+    const int slot = pos * 2 * per_w + (r % half_w) * 2 + r / half_w;
     __half* blk = reinterpret_cast<__half*>(ksz) + (static_cast<size_t>(bh) * (lcap / gk) + g) * 2 * dk;
     blk[slot] = __low2half(gp.sz);
     blk[slot + per_w] = __high2half(gp.sz);

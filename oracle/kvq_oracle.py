@@ -30,9 +30,12 @@ What it computes, step by step in the order the pages give it:
    pairs are stored as fp16 pairs.  The key (scale, zero) of one group follow the
    packed words of a key row: for word w (channels w*P .. w*P+P-1, P = 32/b,
    H = 16/b) come the P scales in the order (w*P+i, w*P+i+H) for i < H, then the
-   P zeros in the same order (key_meta_order).  The pages fix no memory layout;
-   this one puts the two channels whose codes share a 32-bit word half by half
-   next to each other.
+   P zeros in the same order.  When the row has W >= 4 words and 4 divides W,
+   the blocks of the W words are stored quarter-interleaved: the block of word w
+   sits at position (w mod W/4) * 4 + w div W/4 (key_meta_order).  The pages fix
+   no memory layout; this one puts the two channels whose codes share a 32-bit
+   word half by half next to each other, and the blocks that the four quarters of
+   a key row need at the same time next to each other.
 5. Log-spaced retention (LogQuant §Méthodologie 2, "density halves further
    back"; the printed text is garbled).  Reading: among the quantized positions
    p < Q, p is kept in fp16 iff p is a multiple of 2^floor(log2(Q - p)); this
@@ -152,8 +155,11 @@ def key_meta_order(d_k: int, bits: int):
     """Slot order of one key group's fp16 (scale, zero) block (step 4): for slot i of
     the 2*d_k slots, the channel it holds and whether it is the scale (0) or zero (1)."""
     per, half = 32 // bits, 16 // bits
+    words = d_k // per
+    quarter = words // 4 if words % 4 == 0 else 0
     chan, which = [], []
-    for w in range(d_k // per):
+    for pos in range(words):
+        w = (pos % 4) * quarter + pos // 4 if quarter else pos     # word stored at pos
         for part in (0, 1):                          # scales, then zeros
             for i in range(half):
                 for c in (w * per + i, w * per + i + half):
