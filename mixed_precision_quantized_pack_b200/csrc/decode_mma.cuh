@@ -505,8 +505,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
               const float2 f0 = __half22float2(ptx::u32_as_h2(vm0[gg]));
               const float2 f1 = __half22float2(ptx::u32_as_h2(vm1[gg]));
               zsum[gg] = fmaf(p0, f0.y, fmaf(p1, f1.y, zsum[gg]));
-              uint32_t x0, x1;
-              ptx::split_hi_lo_pair(p0 * f0.x, p1 * f1.x, x0, x1);
+              const uint32_t x0 = ptx::split_hi_lo_trunc(p0 * f0.x);
+              const uint32_t x1 = ptx::split_hi_lo_trunc(p1 * f1.x);
               const uint32_t bp0 = ptx::movmatrix_trans(x0);
               const uint32_t bp1 = ptx::movmatrix_trans(x1);
 
@@ -645,8 +645,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       const float p0 = ptx::ex2(s0 - m_use);
       const float p1 = ptx::ex2(s1 - m_use);
       l_run += p0 + p1;
-      uint32_t x0, x1;
-      ptx::split_hi_lo_pair(p0, p1, x0, x1);
+      const uint32_t x0 = ptx::split_hi_lo_trunc(p0);
+      const uint32_t x1 = ptx::split_hi_lo_trunc(p1);
       const uint32_t bp0 = ptx::movmatrix_trans(x0);
       const uint32_t bp1 = ptx::movmatrix_trans(x1);
       // p.V: A = V^T tiles via ldmatrix.trans (rows = tokens in shared memory)

@@ -340,11 +340,8 @@ int kvq_append(kvq_cache* c, const void* k_new, const void* v_new, void* stream)
   __half* wk = static_cast<__half*>(c->buf.win_k);
   __half* wv = static_cast<__half*>(c->buf.win_v);
   const int slot = c->L % d.cap;
-  int rc = check_cuda(kvq::launch_copy_rows(static_cast<const __half*>(k_new), 1, 0, wk, d.cap,
-                                            slot, 1, d.dk, nbh, s));
-  if (!rc)
-    rc = check_cuda(kvq::launch_copy_rows(static_cast<const __half*>(v_new), 1, 0, wv, d.cap, slot,
-                                          1, d.dv, nbh, s));
+  int rc = check_cuda(kvq::launch_append_token(d, static_cast<const __half*>(k_new),
+                                               static_cast<const __half*>(v_new), wk, wv, slot, s));
   if (rc) return rc;
   const int L = c->L + 1;
   int Q = c->Q;

@@ -74,6 +74,8 @@ cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_row
                                    int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s);
 cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,
                              int dst_rows, int dst_base, int n, int d, int nbh, cudaStream_t s);
+cudaError_t launch_append_token(const Dims& d, const __half* k, const __half* v, __half* win_k,
+                                __half* win_v, int slot, cudaStream_t s);
 cudaError_t launch_copy_retained(const Dims& d, const __half* k, const __half* v, int L,
                                  const RetList& ret, __half* ret_k, __half* ret_v, cudaStream_t s);
 cudaError_t launch_update_retained(const Dims& d, const RetUpdate& up, __half* win_k,

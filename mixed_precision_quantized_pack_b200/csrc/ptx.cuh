@@ -138,22 +138,14 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// (hi, lo) fp16 pairs of two values: hi = fp16(x), lo = fp16(x - hi), so hi + lo == x to
-// about 22 bits.  x0 -> (hi0, lo0) in r0, x1 -> (hi1, lo1) in r1.
-__device__ __forceinline__ void split_hi_lo_pair(float x0, float x1, uint32_t& r0, uint32_t& r1) {
-  const __half2 hi = __floats2half2_rn(x0, x1);
-  const float2 hf = __half22float2(hi);
-  const __half2 lo = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
-  r0 = prmt(h2_as_u32(hi), h2_as_u32(lo), 0x5410u);
-  r1 = prmt(h2_as_u32(hi), h2_as_u32(lo), 0x7632u);
+// (hi, lo) fp16 pair of x in one register (hi in the low half): hi is x truncated to 11
+// significant bits, so it converts to fp16 exactly when |x| >= 2^-14 and x - hi is
+// exact in fp32; hi + lo == x to about 22 bits.
+__device__ __forceinline__ uint32_t split_hi_lo_trunc(float x) {
+  const float hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+  return h2_as_u32(__floats2half2_rn(hi, x - hi));
 }
 
-// (hi, lo) fp16 pair with hi + lo == x to about 22 bits: hi = fp16(x), lo = fp16(x - hi).
-__device__ __forceinline__ uint32_t split_hi_lo(float x) {
-  const __half hi = __float2half_rn(x);
-  const float rest = x - __half2float(hi);
-  return h2_as_u32(__halves2half2(hi, __float2half_rn(rest)));
-}
 
 }  // namespace ptx
 }  // namespace kvq

@@ -154,6 +154,25 @@ __global__ void copy_rows_kernel(const __half* __restrict__ src, int src_rows, i
   }
 }
 
+// Append: the new token's key and value rows of every (b, kv head) into window slot `slot`
+// (one launch for both, 16 B per thread).
+__global__ void append_token_kernel(const __half* __restrict__ k, const __half* __restrict__ v,
+                                    __half* __restrict__ win_k, __half* __restrict__ win_v, int slot,
+                                    int cap, int dk, int dv, int nbh) {
+  const int vk = dk / 8, vv = dv / 8;
+  const int total = nbh * (vk + vv);
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
+    const int bh = idx / (vk + vv), e = idx % (vk + vv);
+    if (e < vk) {
+      reinterpret_cast<uint4*>(win_k + (static_cast<size_t>(bh) * cap + slot) * dk)[e] =
+          reinterpret_cast<const uint4*>(k + static_cast<size_t>(bh) * dk)[e];
+    } else {
+      reinterpret_cast<uint4*>(win_v + (static_cast<size_t>(bh) * cap + slot) * dv)[e - vk] =
+          reinterpret_cast<const uint4*>(v + static_cast<size_t>(bh) * dv)[e - vk];
+    }
+  }
+}
+
 // Prefill: ret[bh][j] = K[bh][pos[j]] for the retained positions (keys and values).
 __global__ void copy_retained_kernel(const __half* __restrict__ k, const __half* __restrict__ v,
                                      int L, int dk, int dv, RetList ret,
@@ -247,6 +266,16 @@ cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __ha
   const int block = 256;
   copy_rows_kernel<<<grid_for(items, block), block, 0, s>>>(src, src_rows, src_base, dst, dst_rows,
                                                             dst_base, n, d, nbh);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_token(const Dims& d, const __half* k, const __half* v, __half* win_k,
+                                __half* win_v, int slot, cudaStream_t s) {
+  const int nbh = d.B * d.Hkv;
+  const int total = nbh * (d.dk + d.dv) / 8;
+  const int block = 256;
+  append_token_kernel<<<(total + block - 1) / block, block, 0, s>>>(k, v, win_k, win_v, slot, d.cap, d.dk,
+                                                                  d.dv, nbh);
   return cudaGetLastError();
 }
 
