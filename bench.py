@@ -296,6 +296,10 @@ def main():
     for i in range(warm, warm + steps):
         step(i, True)
     t1.record(stream)
+    # wait for the GPU without holding the interpreter lock, so that the clock sampler
+    # keeps polling while the timed steps run
+    while not t1.query():
+        time.sleep(0.0002)
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
