@@ -195,6 +195,15 @@ int kvq_get_state(const kvq_cache* cache, int* L, int* Q, int* n_retained, int* 
  * INVALID_ARG if out is NULL while Q > 0, or if cap is too small. */
 int kvq_retained_positions(int Q, int* out, int cap);
 
+/* Test hook for the timeout path (no counterpart on the pages).  Arms the next
+ * kvq_decode_attention on this cache: when it runs the tensor-core kernel, one CTA
+ * asks its first shared-memory copy for 16 bytes more than the copy delivers, so
+ * that CTA's bounded waits give up after their 1 s limit; it then sets
+ * KVQ_STATUS_TIMEOUT in the workspace status word and contributes nothing, and the
+ * call's output is undefined.  Nothing faults or hangs, the context stays usable and
+ * the following calls are normal.  Returns KVQ_OK or KVQ_ERR_INVALID_ARG. */
+int kvq_debug_stall_next_decode(kvq_cache* cache);
+
 /* Zero the status word of a decode workspace (asynchronous, on stream). */
 int kvq_reset_status(void* workspace, void* stream);
 

@@ -350,7 +350,9 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         const uint32_t dst = stages_s + st * STAGE;
         sm_issued[st] += 1;
         sm_tag[st] = k;
-        ptx::mbar_arrive_expect_tx(bar, L.bytes);
+        // (test hook) one stage that never completes: its waits run into their bound
+        const bool stall = w.stall && k == 0 && split == 0 && h == 0 && b == 0;
+        ptx::mbar_arrive_expect_tx(bar, L.bytes + (stall ? 16u : 0u));
         const size_t tok = static_cast<size_t>(bh) * d.lcap + static_cast<size_t>(g) * gk;
         ptx::bulk_g2s(dst + L.k_off, cb.kcode + tok * G::KW, gk * G::KBYTES_ROW, bar);
         ptx::bulk_g2s(dst + L.kmeta_off, cb.ksz + (static_cast<size_t>(bh) * (d.lcap / gk) + g) * DK,
@@ -575,7 +577,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       if (lane == 0) {
         sm_issued[st] += 1;
         sm_tag[st] = k;
-        ptx::mbar_arrive_expect_tx(bar, nvalid * (DK + kDV) * 2);
+        const bool stall = w.stall && k == 0 && split == w.splits_q && h == 0 && b == 0;
+        ptx::mbar_arrive_expect_tx(bar, nvalid * (DK + kDV) * 2 + (stall ? 16 : 0));
       }
       __syncwarp();
       const int row = lane & 15;

@@ -22,6 +22,7 @@ struct kvq_cache {
   int sm_count;
   int kernel;     // KVQ_KERNEL_*
   bool prefilled;
+  bool stall_next;  // test hook armed by kvq_debug_stall_next_decode
 };
 
 namespace kvq {
@@ -271,6 +272,7 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
   c->sm_count = sms;
   c->kernel = KVQ_KERNEL_AUTO;
   c->prefilled = false;
+  c->stall_next = false;
   *out = c;
   return KVQ_OK;
 }
@@ -336,7 +338,6 @@ int kvq_append(kvq_cache* c, const void* k_new, const void* v_new, void* stream)
   if (c->L + 1 > d.max_context) return KVQ_ERR_CAPACITY;
   if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int nbh = d.B * d.Hkv;
   __half* wk = static_cast<__half*>(c->buf.win_k);
   __half* wv = static_cast<__half*>(c->buf.win_v);
   const int slot = c->L % d.cap;
@@ -425,6 +426,8 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
   w.score_scale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.dk)));
   w.ret.n = static_cast<int>(c->ret.size());
   for (int i = 0; i < w.ret.n; ++i) w.ret.pos[i] = c->ret[i];
+  w.stall = c->stall_next && plan.fast_path ? 1 : 0;
+  c->stall_next = false;
   if (workspace_bytes < kvq::workspace_bytes(d, w.splits)) return KVQ_ERR_WORKSPACE;
   const kvq::Partials parts = kvq::workspace_views(d, w.splits, workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -436,6 +439,12 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
     rc = check_cuda(kvq::launch_decode_simple(d, cb, w, qh, parts, s));
   if (!rc) rc = check_cuda(kvq::launch_combine(d, w, parts, static_cast<__half*>(out), s));
   return rc;
+}
+
+int kvq_debug_stall_next_decode(kvq_cache* c) {
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  c->stall_next = true;
+  return KVQ_OK;
 }
 
 int kvq_set_decode_kernel(kvq_cache* c, int kernel) {

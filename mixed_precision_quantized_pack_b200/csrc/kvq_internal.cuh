@@ -42,6 +42,7 @@ struct DecodeWork {
   int splits_f;      // CTAs per (b, kv head) over the fp16 list
   int splits;        // splits_q + splits_f (partials per (b, query head))
   float score_scale; // log2(e) / sqrt(d_k)
+  int stall;         // test hook: CTA (0, 0, 0) asks for 16 bytes more than its first copy delivers
   RetList ret;
 };
 

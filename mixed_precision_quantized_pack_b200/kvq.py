@@ -77,6 +77,7 @@ _SIGNATURES = {
     "kvq_decode_attention_noalloc": (_I, [_P, _P, _P, _I, _P]),
     "kvq_get_plan": (_I, [_P, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_set_decode_kernel": (_I, [_P, _I]),
+    "kvq_debug_stall_next_decode": (_I, [_P]),
     "kvq_plan_decode": (_I, [ctypes.POINTER(kvq_config), _I, _I, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_get_state": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
                            ctypes.POINTER(_I)]),
@@ -194,6 +195,10 @@ def kvq_set_decode_kernel(handle: int, kernel: int) -> None:
     _check(lib().kvq_set_decode_kernel(handle, int(kernel)), "kvq_set_decode_kernel")
 
 
+def kvq_debug_stall_next_decode(handle: int) -> None:
+    _check(lib().kvq_debug_stall_next_decode(handle), "kvq_debug_stall_next_decode")
+
+
 def kvq_get_state(handle: int) -> Tuple[int, int, List[int]]:
     L, Q, n = _I(), _I(), _I()
     idx = (ctypes.c_int * KVQ_MAX_RETAINED)()
@@ -279,6 +284,9 @@ class KVCache:
 
     def status(self, stream=None) -> int:
         return kvq_read_status(self.workspace.data_ptr(), _stream(stream))
+
+    def reset_status(self, stream=None) -> None:
+        kvq_reset_status(self.workspace.data_ptr(), _stream(stream))
 
     def state(self) -> Tuple[int, int, List[int]]:
         return kvq_get_state(self.handle)

@@ -170,6 +170,35 @@ def test_split_invariance():
         assert (o - outs[0]).abs().max().item() <= 2e-3 * outs[0].abs().max().item()
 
 
+def test_a_wait_that_runs_out_sets_the_timeout_status():
+    """The tensor-core kernel's waits are bounded: when one gives up (the test hook makes one
+    copy stage ask for 16 bytes more than it receives) the call sets KVQ_STATUS_TIMEOUT
+    within seconds, and the context and the cache stay usable for the next call."""
+    need_gpu()
+    import time
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=1024, appends=0, seed=91)
+    inp = W.Inputs(w, device="cpu")
+    cfg = w.kvq_config()
+    gc = K.KVCache(cfg)
+    oc = O.OracleCache(cfg)
+    gc.prefill(inp.k.cuda(), inp.v.cuda())
+    oc.prefill(np16(inp.k), np16(inp.v))
+    ref = oc.decode(np16(inp.q[0]))
+    q = inp.q[0].cuda()
+    assert O.max_rel_error(gc.decode(q).float().cpu().numpy(), ref) <= TOL
+    assert gc.status() == 0
+    K.kvq_debug_stall_next_decode(gc.handle)
+    t0 = time.time()
+    gc.decode(q)
+    status = gc.status()
+    assert status & K.KVQ_STATUS_TIMEOUT
+    assert time.time() - t0 < 30
+    gc.reset_status()
+    out = gc.decode(q)
+    assert gc.status() == 0
+    assert O.max_rel_error(out.float().cpu().numpy(), ref) <= TOL
+
+
 def test_error_paths():
     need_gpu()
     w = W.WORKLOADS["tiny"].with_(context=100)
