@@ -46,6 +46,18 @@ What it computes, step by step in the order the pages give it:
    Values", §2, where d_k may be smaller than d_v; the score form of "HeadQ",
    §2.1), softmax with max subtraction, p.V.  Token order is irrelevant
    (LogQuant §4, A.V = A_P.V_P).  GQA: query head hq reads kv head hq // n_rep.
+7. Optional side code ("HeadQ: ... correction dans l'espace des scores", §3,
+   Aperçu de l'algorithme, steps 2 and 3), with a basis U_h of r columns per kv
+   head (fp32 [d_k][r], given by the caller; the pages learn it by PCA over
+   calibration queries).  When a key group is quantized, for each of its tokens:
+       e = fl32(k - fl32(code * s16 + z16))           (the base residual)
+       y_i = sum_c U_h[c, i] * e_c                      (fp32, c ascending from +0,
+                                                         one product and one sum at a time)
+   and the side quantizer Q_q (reading: the step-3 quantizer, per coordinate i
+   over the group's G_k tokens, on the fp32 y; z16 = fp16(min) then rounds)
+   gives side codes and one fp16 (scale, zero) per coordinate.  Decode adds
+   (U_h^T q) . z_hat_j / sqrt(d_k), z_hat = code * s + z, to the score of every
+   quantized token that is not retained; window and retained tokens are exact.
 
 Buffer formats mirror the CUDA library's so the tests can compare bytes:
   kcode u32 [B][Hkv][Lcap][d_k*kb/32]        ksz fp16 [B][Hkv][Lcap/Gk][2*d_k] (key_meta_order)
@@ -53,6 +65,8 @@ Buffer formats mirror the CUDA library's so the tests can compare bytes:
   win_k/v fp16 [B][Hkv][C][d] with token p in slot p % C,
           C = R + G_k (quantized caches) or Lcap (bits 16)
   ret_k/v fp16 [B][Hkv][32][d] in ascending position order, ret_idx int32 list.
+  zcode u8 [B][Hkv][Lcap][r*q/8]: the r side codes of a token, coordinate i at bit
+        i*q of the little-endian row (pack_side); zsz fp16 [B][Hkv][Lcap/Gk][r][2].
 """
 from __future__ import annotations
 
@@ -88,11 +102,15 @@ def retained_positions(Q: int) -> List[int]:
 def minmax_quantize(x: np.ndarray, bits: int, axis: int):
     """Asymmetric min-max quantizer of step 3 over groups laid along ``axis``.
 
-    ``x`` holds fp16 values (any float dtype holding them exactly).  Returns
-    (codes uint32 with x's shape, s16 fp16, z16 fp16) where s16/z16 keep a
+    ``x`` holds fp16 values (any float dtype holding them exactly), or fp32 values
+    (float32 dtype: the side coordinates of step 7, where z16 = fp16(min) rounds).
+    Returns (codes uint32 with x's shape, s16 fp16, z16 fp16) where s16/z16 keep a
     length-1 ``axis``.
     """
-    x32 = np.asarray(x, dtype=np.float16).astype(np.float32)
+    x = np.asarray(x)
+    # fp32 data (the side quantizer's projections) is taken as it is; anything else
+    # holds fp16 values and is read through fp16, which is exact
+    x32 = x if x.dtype == np.float32 else x.astype(np.float16).astype(np.float32)
     mn = x32.min(axis=axis, keepdims=True)
     mx = x32.max(axis=axis, keepdims=True)
     levels = np.float32(2 ** bits - 1)
@@ -114,6 +132,64 @@ def minmax_quantize(x: np.ndarray, bits: int, axis: int):
 def dequantize(codes: np.ndarray, s16: np.ndarray, z16: np.ndarray) -> np.ndarray:
     """code * s + z, exactly, in fp64."""
     return codes.astype(np.float64) * s16.astype(np.float64) + z16.astype(np.float64)
+
+
+def key_residual(k: np.ndarray, codes: np.ndarray, s16: np.ndarray, z16: np.ndarray) -> np.ndarray:
+    """Step 7: e = fl32(k - fl32(code * s16 + z16)), elementwise, fp32 (code*s16 is exact)."""
+    k32 = np.asarray(k, np.float16).astype(np.float32)
+    base = codes.astype(np.float32) * s16.astype(np.float32)
+    base = base + z16.astype(np.float32)
+    return k32 - base
+
+
+def side_project(e: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """Step 7: y[n][i] = sum_c U[c][i] * e[n][c] in fp32, c ascending from +0, one
+    rounded product and one rounded sum at a time.  e fp32 [n][d], U fp32 [d][r]."""
+    e = np.asarray(e, np.float32)
+    U = np.asarray(U, np.float32)
+    y = np.zeros((e.shape[0], U.shape[1]), np.float32)
+    for c in range(e.shape[1]):
+        y = y + e[:, c:c + 1] * U[c][None, :]
+    return y
+
+
+def side_code_group(k: np.ndarray, kcodes: np.ndarray, ksz: np.ndarray, U: np.ndarray,
+                    bits: int, group_k: int):
+    """Side code of keys [n][d] (n a multiple of group_k) whose base codes [n][d] and
+    per-group (scale, zero) ksz fp16 [n/group_k][d][2] are given: returns side codes
+    uint32 [n][r] and side (scale, zero) fp16 [n/group_k][r][2] (step 7)."""
+    n, d = k.shape
+    s = np.repeat(ksz[:, :, 0], group_k, axis=0)
+    z = np.repeat(ksz[:, :, 1], group_k, axis=0)
+    y = side_project(key_residual(k, kcodes, s, z), U)                   # [n][r] fp32
+    r = y.shape[1]
+    codes, ss, sz = minmax_quantize(y.reshape(n // group_k, group_k, r), bits, axis=1)
+    return codes.reshape(n, r), np.stack([ss[:, 0, :], sz[:, 0, :]], axis=-1)
+
+
+def side_query(U: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """U^T q in fp64 (step 7): the query's coordinates in the side basis, U fp32 [d][r]."""
+    return np.asarray(U, np.float64).T @ np.asarray(q, np.float64)
+
+
+def pack_side(codes: np.ndarray, bits: int) -> np.ndarray:
+    """[..., r] side codes -> [..., ceil(r*bits/8)] bytes: coordinate i at bit i*bits of
+    the little-endian row, unused high bits 0."""
+    r = codes.shape[-1]
+    shifts = np.arange(r, dtype=np.uint64) * np.uint64(bits)
+    row = (codes.astype(np.uint64) << shifts).sum(axis=-1)
+    nbytes = -(-r * bits // 8)
+    out = [(row >> np.uint64(8 * j)) & np.uint64(0xFF) for j in range(nbytes)]
+    return np.stack(out, axis=-1).astype(np.uint8)
+
+
+def unpack_side(rows: np.ndarray, bits: int, r: int) -> np.ndarray:
+    """Inverse of pack_side."""
+    acc = np.zeros(rows.shape[:-1], np.uint64)
+    for j in range(rows.shape[-1]):
+        acc |= rows[..., j].astype(np.uint64) << np.uint64(8 * j)
+    shifts = np.arange(r, dtype=np.uint64) * np.uint64(bits)
+    return ((acc[..., None] >> shifts) & np.uint64((1 << bits) - 1)).astype(np.uint32)
 
 
 def quantize_keys(k: np.ndarray, group_k: int, bits: int):
@@ -193,10 +269,15 @@ def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
 
 
 # -------------------------------------------------------------- attention -----
-def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
-    """softmax(q.K^T * scale) V in fp64 for one query vector."""
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+              extra: Optional[np.ndarray] = None) -> np.ndarray:
+    """softmax((q.K^T + extra) * scale) V in fp64 for one query vector; ``extra`` is the
+    per-token additive logit correction of step 7 (before the 1/sqrt(d) scale)."""
     q = np.asarray(q, dtype=np.float64)
-    s = (np.asarray(k, dtype=np.float64) @ q) * scale
+    s = np.asarray(k, dtype=np.float64) @ q
+    if extra is not None:
+        s = s + extra
+    s = s * scale
     p = np.exp(s - s.max())
     return (p @ np.asarray(v, dtype=np.float64)) / p.sum()
 
@@ -209,21 +290,33 @@ def buffer_bytes(cfg: dict) -> dict:
         lcap = cfg["max_context"]
         cap = lcap
         return dict(kcode=0, ksz=0, vcode=0, vsz=0, win_k=B * H * cap * dk * 2,
-                    win_v=B * H * cap * dv * 2, ret_k=0, ret_v=0)
+                    win_v=B * H * cap * dv * 2, ret_k=0, ret_v=0, zcode=0, zsz=0)
     lcap = -(-cfg["max_context"] // gk) * gk
     cap = R + gk
+    sr, sq = cfg.get("side_rank", 0), cfg.get("side_bits", 0)
     return dict(kcode=B * H * lcap * dk * kb // 8, ksz=B * H * (lcap // gk) * dk * 4,
                 vcode=B * H * lcap * dv * vb // 8, vsz=B * H * lcap * (dv // gv) * 4,
                 win_k=B * H * cap * dk * 2, win_v=B * H * cap * dv * 2,
-                ret_k=B * H * MAX_RETAINED * dk * 2, ret_v=B * H * MAX_RETAINED * dv * 2)
+                ret_k=B * H * MAX_RETAINED * dk * 2, ret_v=B * H * MAX_RETAINED * dv * 2,
+                zcode=B * H * lcap * sr * sq // 8, zsz=B * H * (lcap // gk) * sr * 4)
 
 
 # ------------------------------------------------------------------ cache -----
 class OracleCache:
-    """The whole cache of one layer: prefill, append, decode (see module docstring)."""
+    """The whole cache of one layer: prefill, append, decode (see module docstring).
 
-    def __init__(self, cfg: dict):
+    ``side_basis`` fp32 [Hkv][d_k][r] is required when cfg["side_rank"] = r > 0 (step 7).
+    """
+
+    def __init__(self, cfg: dict, side_basis: Optional[np.ndarray] = None):
         self.cfg = dict(cfg)
+        self.sr = int(cfg.get("side_rank", 0))
+        self.sq = int(cfg.get("side_bits", 0))
+        if self.sr:
+            if cfg["k_bits"] == 16 or side_basis is None:
+                raise ValueError("a side code needs quantized keys and a basis")
+            self.U = np.asarray(side_basis, np.float32)
+            assert self.U.shape == (cfg["n_kv_heads"], cfg["d_k"], self.sr)
         B, H = cfg["batch"], cfg["n_kv_heads"]
         self.B, self.H, self.Hq = B, H, cfg["n_q_heads"]
         self.dk, self.dv = cfg["d_k"], cfg["d_v"]
@@ -243,6 +336,9 @@ class OracleCache:
             self.vsz = np.zeros((B, H, self.lcap, self.dv // self.gv, 2), np.float16)
             self.ret_k = np.zeros((B, H, MAX_RETAINED, self.dk), np.float16)
             self.ret_v = np.zeros((B, H, MAX_RETAINED, self.dv), np.float16)
+            if self.sr:
+                self.zcode = np.zeros((B, H, self.lcap, self.sr * self.sq // 8), np.uint8)
+                self.zsz = np.zeros((B, H, self.lcap // self.gk, self.sr, 2), np.float16)
         self.win_k = np.zeros((B, H, self.cap, self.dk), np.float16)
         self.win_v = np.zeros((B, H, self.cap, self.dv), np.float16)
         self.ret_idx: List[int] = []
@@ -259,6 +355,10 @@ class OracleCache:
         self.ksz[b, h, t0 // self.gk:(t0 + n) // self.gk] = pack_key_meta(ksz, self.kb)
         self.vcode[b, h, t0:t0 + n] = pack_codes(vc, self.vb)
         self.vsz[b, h, t0:t0 + n] = vsz
+        if self.sr:
+            zc, zsz = side_code_group(k_rows, kc, ksz, self.U[h], self.sq, self.gk)
+            self.zcode[b, h, t0:t0 + n] = pack_side(zc, self.sq)
+            self.zsz[b, h, t0 // self.gk:(t0 + n) // self.gk] = zsz
 
     def prefill(self, k: np.ndarray, v: np.ndarray):
         """k [B][Hkv][L][d_k], v [B][Hkv][L][d_v] fp16: the cache's first L tokens."""
@@ -339,8 +439,25 @@ class OracleCache:
         vh[Q:] = self.win_v[b, h, slots]
         return kh, vh
 
-    def decode(self, q: np.ndarray, rows: Optional[List[int]] = None) -> np.ndarray:
-        """q [B][Hq][d_k] fp16 -> out [B][Hq][d_v] fp64 (rows: optional subset of b)."""
+    def decoded_side(self, b: int, h: int) -> np.ndarray:
+        """z_hat [L][r] in fp64 (step 7): code*s + z for quantized tokens that are not
+        retained, 0 for retained and window tokens."""
+        Q = self.Q
+        zh = np.zeros((self.L, self.sr), np.float64)
+        if Q:
+            zc = unpack_side(self.zcode[b, h, :Q], self.sq, self.sr)          # [Q][r]
+            zsz = self.zsz[b, h, :Q // self.gk]                                  # [ng][r][2]
+            zs = np.repeat(zsz[:, :, 0], self.gk, axis=0)
+            zz = np.repeat(zsz[:, :, 1], self.gk, axis=0)
+            zh[:Q] = dequantize(zc, zs, zz)
+            for pos in self.ret_idx:
+                zh[pos] = 0.0
+        return zh
+
+    def decode(self, q: np.ndarray, rows: Optional[List[int]] = None,
+               side_sign: float = 1.0) -> np.ndarray:
+        """q [B][Hq][d_k] fp16 -> out [B][Hq][d_v] fp64 (rows: optional subset of b).
+        ``side_sign`` = -1 flips the side correction (the pages' wrong-sign control)."""
         if self.L == 0:
             raise ValueError("decode before prefill")
         q = np.asarray(q, np.float16).astype(np.float64)
@@ -350,9 +467,13 @@ class OracleCache:
         for b in (rows if rows is not None else range(self.B)):
             for h in range(self.H):
                 kh, vh = self.decoded_kv(b, h)
+                zh = self.decoded_side(b, h) if self.sr else None
                 for r in range(n_rep):
                     hq = h * n_rep + r
-                    out[b, hq] = attention(q[b, hq], kh, vh, scale)
+                    extra = None
+                    if zh is not None:
+                        extra = side_sign * (zh @ side_query(self.U[h], q[b, hq]))
+                    out[b, hq] = attention(q[b, hq], kh, vh, scale, extra)
         return out
 
 

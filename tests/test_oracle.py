@@ -394,3 +394,255 @@ def test_algorithmic_bytes_per_token_k4v2_g64():
     bb = O.buffer_bytes(cfg)
     lcap = 64 * 100
     assert (bb["kcode"] + bb["ksz"] + bb["vcode"] + bb["vsz"]) / lcap == 112
+
+
+# ------------------------------------------------------- HeadQ side code ----
+# "HeadQ: Distortion visible par le modele et correction dans l'espace des scores pour la
+# quantification du cache KV", §3 (Apercu de l'algorithme): base key, residual, side code
+# Q_q(U^T e), and the additive logit correction q^T U z_hat / sqrt(d).
+from fractions import Fraction
+
+
+def _golden_headq():
+    rows = {}
+    for fields in read_golden("headq_worked.txt"):
+        name = fields[0][0]
+        rows.setdefault(name, []).append(fields[1:])
+    return rows
+
+
+def test_golden_headq_worked_example():
+    g = _golden_headq()
+    num = lambda xs: [float(x) for x in xs]
+    k = np.array([num(r[1]) for r in sorted(g["K"], key=lambda r: int(r[0][0]))], np.float16)
+    U = np.array([num(r[1]) for r in sorted(g["U"], key=lambda r: int(r[0][0]))], np.float32)
+    gk = k.shape[0]
+    kc, ksz = O.quantize_keys(k, gk, 2)
+    for ch, sz, codes in g["base"]:
+        c = int(ch[0])
+        assert [float(ksz[0, c, 0]), float(ksz[0, c, 1])] == num(sz)
+        assert [int(x) for x in kc[:, c]] == [int(x) for x in codes]
+    s = np.repeat(ksz[:, :, 0], gk, axis=0)
+    z = np.repeat(ksz[:, :, 1], gk, axis=0)
+    e = O.key_residual(k, kc, s, z)
+    for t, vals in g["residual"]:
+        assert list(e[int(t[0])]) == num(vals)
+    y = O.side_project(e, U)
+    for t, vals in g["y"]:
+        assert list(y[int(t[0])]) == num(vals)
+    zc, zsz = O.side_code_group(k, kc, ksz, U, 2, gk)
+    for i, sz, codes in g["side"]:
+        c = int(i[0])
+        assert [float(zsz[0, c, 0]), float(zsz[0, c, 1])] == num(sz)
+        assert [int(x) for x in zc[:, c]] == [int(x) for x in codes]
+    packed = O.pack_side(zc, 2)
+    assert [int(x) for x in packed[:, 0]] == [int(x, 16) for x in g["packed"][0][0]]
+    assert np.array_equal(O.unpack_side(packed, 2, 2), zc)
+    zh = O.dequantize(zc, np.repeat(zsz[:, :, 0], gk, axis=0), np.repeat(zsz[:, :, 1], gk, axis=0))
+    for t, vals in g["zhat"]:
+        assert list(zh[int(t[0])]) == num(vals)
+    q = np.array(num(g["q"][0][0]))
+    qt = O.side_query(U, q)
+    assert list(qt) == num(g["qt"][0][0])
+    assert list(zh @ qt) == num(g["correction"][0][0])
+    kh = O.dequantize(kc, s, z)
+    assert list(kh @ q) == num(g["base_dot"][0][0])
+    assert list(k.astype(np.float64) @ q) == num(g["exact_dot"][0][0])
+
+
+# IEEE binary formats emulated on exact rationals (independent of numpy's float32)
+def _round(x: Fraction, mant: int, emin: int) -> Fraction:
+    """Round-to-nearest-even of x to a binary float with `mant` significant bits and
+    minimum normal exponent `emin` (subnormals below it)."""
+    if x == 0:
+        return Fraction(0)
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, emin)
+    ulp = Fraction(2) ** (e - mant + 1)
+    n = a / ulp
+    m, rem = divmod(n.numerator, n.denominator)
+    if 2 * rem > n.denominator or (2 * rem == n.denominator and m % 2 == 1):
+        m += 1
+    return (m * ulp) if x > 0 else -(m * ulp)
+
+
+def r32(x):
+    return _round(Fraction(x), 24, -126)
+
+
+def r16(x):
+    return _round(Fraction(x), 11, -14)
+
+
+def _rint_even(x: Fraction) -> int:
+    m, rem = divmod(x.numerator, x.denominator)
+    if 2 * rem > x.denominator or (2 * rem == x.denominator and m % 2 == 1):
+        m += 1
+    return m
+
+
+@pytest.mark.parametrize("side_bits", [4, 8])
+def test_side_code_matches_exact_rational_ieee_emulation(side_bits):
+    """Residual, projection and side quantizer against the same steps on exact rationals,
+    each operation rounded by an independent IEEE emulation."""
+    n, d, r, gk, kb = 16, 16, 4, 8, 4
+    k = W.random_fp16((n, d), seed=91, scale=3.0, mean=0.5).numpy()
+    rng = np.random.default_rng(92)
+    U = rng.standard_normal((d, r)).astype(np.float32)
+    kc, ksz = O.quantize_keys(k, gk, kb)
+    zc, zsz = O.side_code_group(k, kc, ksz, U, side_bits, gk)
+    levels = 2 ** side_bits - 1
+    for g in range(n // gk):
+        y = [[None] * r for _ in range(gk)]
+        for t in range(gk):
+            row = g * gk + t
+            e = []
+            for c in range(d):
+                base = r32(Fraction(int(kc[row, c])) * Fraction(float(ksz[g, c, 0])) +
+                           Fraction(float(ksz[g, c, 1])))
+                e.append(r32(Fraction(float(k[row, c])) - base))
+            for i in range(r):
+                acc = Fraction(0)
+                for c in range(d):
+                    acc = r32(acc + r32(Fraction(float(U[c, i])) * e[c]))
+                y[t][i] = acc
+        for i in range(r):
+            col = [y[t][i] for t in range(gk)]
+            mn, mx = min(col), max(col)
+            s16 = r16(r32(r32(mx - mn) / levels))
+            z16 = r16(mn)
+            assert Fraction(float(zsz[g, i, 0])) == s16
+            assert Fraction(float(zsz[g, i, 1])) == z16
+            for t in range(gk):
+                if s16 == 0:
+                    want = 0
+                else:
+                    want = min(max(_rint_even(r32(r32(col[t] - z16) / s16)), 0), levels)
+                assert int(zc[g * gk + t, i]) == want, (g, t, i)
+
+
+def test_side_projection_sums_channels_in_ascending_order():
+    # fp32: (2^24 + 1) rounds to 2^24 (tie to even), so the ascending sum is 0 and the
+    # descending one is 1; the definition fixes the ascending order.
+    ones = np.ones((3, 1), np.float32)
+    up = np.array([[2.0 ** 24, 1.0, -2.0 ** 24]], np.float32)
+    assert float(O.side_project(up, ones)[0, 0]) == 0.0
+    assert float(O.side_project(up[:, ::-1].copy(), ones)[0, 0]) == 1.0
+
+
+def side_cfg(B, Hq, Hkv, d, kb, vb, gk, gv, R, log_retain, max_context, sr, sq):
+    return dict(cfg_of(B, Hq, Hkv, d, d, kb, vb, gk, gv, R, log_retain, max_context),
+                side_rank=sr, side_bits=sq)
+
+
+def test_standard_basis_side_code_is_a_per_channel_residual_correction():
+    """U_h = columns of the identity (channels ch_h): y = e[:, ch_h] exactly, so the decode
+    equals plain attention over keys k_hat + z_hat placed on those channels."""
+    B, Hq, Hkv, d, gk, R, L = 2, 8, 2, 32, 16, 24, 200
+    k = W.random_fp16((B, Hkv, L, d), seed=61, scale=4.0, mean=1.0).numpy()
+    v = W.random_fp16((B, Hkv, L, d), seed=62).numpy()
+    q = W.random_fp16((B, Hq, d), seed=63).numpy()
+    chans = [[3, 17, 0, 30], [9, 1, 22, 14]]
+    U = np.zeros((Hkv, d, 4), np.float32)
+    for h in range(Hkv):
+        for i, c in enumerate(chans[h]):
+            U[h, c, i] = 1.0
+    cfg = side_cfg(B, Hq, Hkv, d, 2, 4, gk, 16, R, 1, 256, 4, 8)
+    oc = O.OracleCache(cfg, side_basis=U)
+    oc.prefill(k, v)
+    assert oc.Q > 0 and oc.ret_idx
+    got = oc.decode(q)
+    keff = np.empty((B, Hkv, L, d))
+    veff = np.empty((B, Hkv, L, d))
+    for b in range(B):
+        for h in range(Hkv):
+            kh, vh = oc.decoded_kv(b, h)
+            veff[b, h] = vh
+            Q = oc.Q
+            kc = O.unpack_codes(oc.kcode[b, h, :Q], 2)
+            ksz = O.unpack_key_meta(oc.ksz[b, h, :Q // gk], 2)
+            e = O.key_residual(k[b, h, :Q], kc, np.repeat(ksz[:, :, 0], gk, 0), np.repeat(ksz[:, :, 1], gk, 0))
+            for i, c in enumerate(chans[h]):
+                col = e[:, c].reshape(Q // gk, gk)
+                codes, s, z = O.minmax_quantize(col, 8, axis=1)
+                zh = O.dequantize(codes, s, z).reshape(Q)
+                zh[oc.ret_idx] = 0.0
+                kh[:Q, c] += zh
+            keff[b, h] = kh
+    want = sdpa_fp64(q.astype(np.float64), keff, veff)
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
+def test_zero_residual_gives_a_null_side_code():
+    """Keys on the base grid: e = 0, y = 0, every side scale and zero 0, output unchanged."""
+    B, Hq, Hkv, d, gk, R, L = 1, 4, 1, 32, 16, 16, 96
+    rng = np.random.default_rng(71)
+    k = rng.integers(0, 16, size=(B, Hkv, L, d)).astype(np.float16)
+    k[:, :, ::gk, :] = 0          # every (group, channel) holds 0 and 15: s = 1, z = 0
+    k[:, :, 1::gk, :] = 15
+    v = W.random_fp16((B, Hkv, L, d), seed=72).numpy()
+    q = W.random_fp16((B, Hq, d), seed=73).numpy()
+    U = np.linalg.qr(rng.standard_normal((d, 4)))[0].astype(np.float32)[None]
+    base = O.OracleCache(cfg_of(B, Hq, Hkv, d, d, 4, 2, gk, 16, R, 0, 128))
+    side = O.OracleCache(side_cfg(B, Hq, Hkv, d, 4, 2, gk, 16, R, 0, 128, 4, 4), side_basis=U)
+    base.prefill(k, v)
+    side.prefill(k, v)
+    assert side.Q > 0
+    assert not side.zsz[:, :, :side.Q // gk].any() and not side.zcode[:, :, :side.Q].any()
+    assert np.array_equal(side.decode(q), base.decode(q))
+
+
+def test_side_correction_recovers_scores_in_the_basis_and_wrong_sign_hurts():
+    """q in span(U_h): the score error of the corrected keys is the side quantizer's own
+    (small) error; flipping the correction's sign (the pages' wrong-sign control) is worse
+    than no correction at all."""
+    B, Hq, Hkv, d, gk, R, L = 1, 4, 2, 64, 32, 32, 600
+    rng = np.random.default_rng(81)
+    k = W.random_fp16((B, Hkv, L, d), seed=82, scale=2.0, mean=0.5).numpy()
+    v = W.random_fp16((B, Hkv, L, d), seed=83).numpy()
+    U = np.stack([np.linalg.qr(rng.standard_normal((d, 4)))[0] for _ in range(Hkv)]).astype(np.float32)
+    a = rng.standard_normal((B, Hq, 4)) * 2.0
+    q = np.einsum("qdr,bqr->bqd", U[np.arange(Hq) // (Hq // Hkv)].astype(np.float64), a)
+    q = q.astype(np.float16)
+    cfg = cfg_of(B, Hq, Hkv, d, d, 2, 8, gk, 16, R, 0, 1024)
+    base = O.OracleCache(cfg)
+    side = O.OracleCache(dict(cfg, side_rank=4, side_bits=8), side_basis=U)
+    base.prefill(k, v)
+    side.prefill(k, v)
+    # exact keys with the same decoded values isolate the score error
+    vd = np.stack([np.stack([side.decoded_kv(b, h)[1] for h in range(Hkv)]) for b in range(B)])
+    ref = sdpa_fp64(q.astype(np.float64), k.astype(np.float64), vd)
+    e_base = O.max_rel_error(base.decode(q), ref)
+    e_side = O.max_rel_error(side.decode(q), ref)
+    e_flip = O.max_rel_error(side.decode(q, side_sign=-1.0), ref)
+    assert e_side < 0.05 * e_base, (e_side, e_base)
+    assert e_flip > e_base, (e_flip, e_base)
+
+
+def test_side_appends_reach_the_same_state_as_one_prefill():
+    B, Hq, Hkv, d, gk, gv, R = 2, 4, 2, 32, 16, 16, 24
+    L0, n_app = 70, 60
+    k = W.random_fp16((B, Hkv, L0 + n_app, d), seed=95, scale=4.0).numpy()
+    v = W.random_fp16((B, Hkv, L0 + n_app, d), seed=96).numpy()
+    U = np.random.default_rng(97).standard_normal((Hkv, d, 8)).astype(np.float32)
+    cfg = side_cfg(B, Hq, Hkv, d, 4, 2, gk, gv, R, 1, 256, 8, 4)
+    a = O.OracleCache(cfg, side_basis=U)
+    a.prefill(k[:, :, :L0], v[:, :, :L0])
+    for t in range(L0, L0 + n_app):
+        a.append(k[:, :, t], v[:, :, t])
+    b = O.OracleCache(cfg, side_basis=U)
+    b.prefill(k, v)
+    assert (a.L, a.Q) == (b.L, b.Q) and a.Q > L0
+    for name in ("zcode", "zsz"):
+        assert np.array_equal(getattr(a, name).view(np.uint8), getattr(b, name).view(np.uint8)), name
+
+
+def test_side_code_bytes_per_token():
+    # r*q/8 code bytes per token and one fp16 (scale, zero) per coordinate per key group
+    for sr, sq, per_tok in ((4, 4, 2 + 16 / 64), (4, 8, 4 + 16 / 64), (8, 4, 4 + 32 / 64)):
+        cfg = dict(cfg_of(1, 1, 1, 128, 128, 2, 2, 64, 64, 128, 0, 64 * 100), side_rank=sr, side_bits=sq)
+        bb = O.buffer_bytes(cfg)
+        assert (bb["zcode"] + bb["zsz"]) / (64 * 100) == per_tok
