@@ -55,8 +55,9 @@ def decode_bytes(cfg: dict, L: int) -> int:
         return B * H * L * (dk + dv) * 2 + B * cfg["n_q_heads"] * dk * 2
     Q = max(L - R, 0) // gk * gk
     nret = len(K.kvq_retained_positions(Q)) if cfg["log_retain"] else 0
-    per_tok = dk * kb // 8 + dv * vb // 8 + (dv // gv) * 4
-    quant = Q * per_tok + (Q // gk) * dk * 4
+    sr, sq = cfg.get("side_rank", 0), cfg.get("side_bits", 0)
+    per_tok = dk * kb // 8 + dv * vb // 8 + (dv // gv) * 4 + sr * sq // 8
+    quant = Q * per_tok + (Q // gk) * (dk * 4 + sr * 4)
     fp16 = (L - Q + nret) * (dk + dv) * 2
     return B * H * (quant + fp16) + B * cfg["n_q_heads"] * dk * 2
 
@@ -168,7 +169,8 @@ def oracle_decode_sample(w: W.Workload, budget_s: float, steps: int = 1):
     from oracle import kvq_oracle as O
     import threadpoolctl
     inp = W.Inputs(w.with_(batch=1, appends=max(steps, 1)), device="cpu")
-    oc = O.OracleCache(dict(w.kvq_config(max_context=w.context + steps + 64), batch=1))
+    oc = O.OracleCache(dict(w.kvq_config(max_context=w.context + steps + 64), batch=1),
+                       side_basis=None if inp.side_basis is None else inp.side_basis.numpy())
     oc.prefill(inp.k.numpy(), inp.v.numpy())
     spent, done = 0.0, 0
     for i in range(steps):
@@ -192,7 +194,8 @@ def run_reference(args, w):
     from oracle import kvq_oracle as O
     steps = args.steps + args.warmup
     inp = W.Inputs(w.with_(batch=1, appends=steps), device="cpu")
-    oc = O.OracleCache(dict(w.kvq_config(max_context=w.context + steps + 64), batch=1))
+    oc = O.OracleCache(dict(w.kvq_config(max_context=w.context + steps + 64), batch=1),
+                       side_basis=None if inp.side_basis is None else inp.side_basis.numpy())
     oc.prefill(inp.k.numpy(), inp.v.numpy())
     for i in range(steps):
         t0 = time.perf_counter()
@@ -249,7 +252,7 @@ def main():
     wl = rank_workload(w, rank, steps + warm)
     cfg = wl.kvq_config(max_context=wl.context + steps + warm + 64)
     inp = W.Inputs(wl, device=dev)
-    cache = K.KVCache(cfg, device=dev)
+    cache = K.KVCache(cfg, device=dev, side_basis=inp.side_basis)
     stream = torch.cuda.current_stream(dev)
 
     # prefill (timed for information)
@@ -322,8 +325,8 @@ def main():
     d_q = torch.empty_like(inp.q[0])
     d_k = torch.empty_like(inp.k_app[0])
     d_v = torch.empty_like(inp.v_app[0])
-    e2e_cache = K.KVCache(cfg, device=dev)
     inp2 = W.Inputs(wl.with_(appends=1), device=dev)
+    e2e_cache = K.KVCache(cfg, device=dev, side_basis=inp2.side_basis)
     e2e_cache.prefill(inp2.k, inp2.v)
     del inp2
     torch.cuda.empty_cache()

@@ -25,6 +25,18 @@
  * tokens are quantized and [Q, L) are fp16 (Q = 0 when the bit widths are 16).
  * Retained set (log_retain = 1): { p < Q : p mod 2^floor(log2(Q - p)) == 0 }.
  *
+ * Optional side code (side_rank r > 0; "HeadQ: Distortion visible par le modele et
+ * correction dans l'espace des scores pour la quantification du cache KV", §3):
+ * with a caller-given basis U_h (fp32 [d_k][r] per kv head), each quantized key
+ * group also stores, per token, the base residual projected on U_h and quantized:
+ *   e = fl32(k - fl32(code * s + z))                  per channel
+ *   y_i = sum_c U_h[c][i] * e_c                        fp32, c ascending from +0,
+ *                                                      one rounded product and sum per c
+ *   side codes: the quantizer above with side_bits, per coordinate i over the
+ *   group's group_k tokens (z = fp16(min y_i) rounds to nearest)
+ * and decode adds (U_h^T q) . z_hat_j / sqrt(d_k), z_hat = code * s + z, to the
+ * score of every quantized token that is not retained.
+ *
  * Buffer layouts (all caller-owned device memory, 256-byte aligned recommended,
  * 16-byte aligned required; sizes from kvq_buffer_sizes):
  *   kcode  u32  [B][Hkv][Lcap][d_k*k_bits/32]   token rows, channel c at word
@@ -40,6 +52,12 @@
  *   win_v  f16  [B][Hkv][C][d_v]  (bits 16: C = max_context, the whole cache)
  *   ret_k  f16  [B][Hkv][32][d_k] retained tokens, ascending positions
  *   ret_v  f16  [B][Hkv][32][d_v]
+ *   zcode  u8   [B][Hkv][Lcap][r*side_bits/8]  side codes of a token, coordinate i
+ *               at bit i*side_bits of the little-endian row   (side_rank r > 0 only)
+ *   zsz    f16  [B][Hkv][Lcap/group_k][r][2]   side (scale, zero) per key group and
+ *               coordinate
+ *   side_u f32  [Hkv][d_k][r]  the basis U_h; written by the caller before the first
+ *               prefill, read by prefill, append and decode, never written here
  * with Lcap = max_context rounded up to a multiple of group_k.
  *
  * Conventions: every call is asynchronous on the caller's CUDA stream (passed as
@@ -87,15 +105,19 @@ typedef struct kvq_config {
     int window;         /* R >= 0: fp16 recent tokens kept beside the quantized prefix */
     int log_retain;     /* 0/1: keep log-spaced older tokens in fp16 (ignored at 16 bits) */
     int max_context;    /* capacity in tokens, >= 1 */
+    int side_rank;      /* r: 0 (no side code), 4 or 8; needs quantized keys */
+    int side_bits;      /* bits per side code: 4 or 8, with side_rank*side_bits 16 or 32 */
 } kvq_config;
 
 typedef struct kvq_sizes {
     size_t kcode, ksz, vcode, vsz, win_k, win_v, ret_k, ret_v;
     size_t workspace;   /* a decode workspace large enough for any length and split count */
+    size_t zcode, zsz, side_u;   /* side code buffers (0 without a side code) */
 } kvq_sizes;
 
 typedef struct kvq_buffers {
     void *kcode, *ksz, *vcode, *vsz, *win_k, *win_v, *ret_k, *ret_v;
+    void *zcode, *zsz, *side_u;  /* side code buffers (NULL without a side code) */
 } kvq_buffers;
 
 typedef struct kvq_cache kvq_cache;   /* opaque host-side handle */

@@ -12,7 +12,12 @@ namespace mma {
   extern template cudaError_t launch<4, 2, DK, NREP, 64, 64, false>(                     \
       const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
       cudaStream_t);
+#define KVQ_DECL_S(KB, VB, DK, NREP, GV, GK, SR, SQ)                                       \
+  extern template cudaError_t launch<KB, VB, DK, NREP, GV, GK, true, SR, SQ>(              \
+      const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
+      cudaStream_t);
 KVQ_MMA_QUANT_INSTANCES(KVQ_DECL_Q)
+KVQ_MMA_SIDE_INSTANCES(KVQ_DECL_S)
 KVQ_MMA_FP16_INSTANCES(KVQ_DECL_F)
 }  // namespace mma
 
@@ -21,14 +26,17 @@ namespace {
 using LaunchFn = cudaError_t (*)(const Dims&, const CacheBufs&, const DecodeWork&, const __half*,
                                  const Partials&, cudaStream_t);
 struct Entry {
-  int kb, vb, dk, nrep, gv, gk;
+  int kb, vb, dk, nrep, gv, gk, sr, sq;
   LaunchFn fn;
 };
 
 #define KVQ_ENTRY_Q(KB, VB, DK, NREP, GV, GK) \
-  {KB, VB, DK, NREP, GV, GK, &mma::launch<KB, VB, DK, NREP, GV, GK, true>},
-#define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, 0, &mma::launch<4, 2, DK, NREP, 64, 64, false>},
-const Entry kTable[] = {KVQ_MMA_QUANT_INSTANCES(KVQ_ENTRY_Q) KVQ_MMA_FP16_INSTANCES(KVQ_ENTRY_F)};
+  {KB, VB, DK, NREP, GV, GK, 0, 0, &mma::launch<KB, VB, DK, NREP, GV, GK, true>},
+#define KVQ_ENTRY_S(KB, VB, DK, NREP, GV, GK, SR, SQ) \
+  {KB, VB, DK, NREP, GV, GK, SR, SQ, &mma::launch<KB, VB, DK, NREP, GV, GK, true, SR, SQ>},
+#define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, 0, 0, 0, &mma::launch<4, 2, DK, NREP, 64, 64, false>},
+const Entry kTable[] = {KVQ_MMA_QUANT_INSTANCES(KVQ_ENTRY_Q) KVQ_MMA_SIDE_INSTANCES(KVQ_ENTRY_S)
+                            KVQ_MMA_FP16_INSTANCES(KVQ_ENTRY_F)};
 
 LaunchFn find(const Dims& d) {
   if (d.dv != 128) return nullptr;
@@ -36,7 +44,7 @@ LaunchFn find(const Dims& d) {
   const int gk = d.quantized() ? d.gk : 0;
   for (const Entry& e : kTable)
     if (e.kb == d.kb && e.vb == d.vb && e.dk == d.dk && e.nrep == d.n_rep && e.gv == gv &&
-        e.gk == gk)
+        e.gk == gk && e.sr == d.sr && (d.sr == 0 || e.sq == d.sq))
       return e.fn;
   return nullptr;
 }

@@ -30,6 +30,13 @@
 // the words' blocks are quarter-interleaved so that the four quads of a warp, which
 // read the four quarters of a key row, load neighbouring blocks.
 //
+// With a side code ("HeadQ: Distortion visible par le modele et correction dans
+// l'espace des scores pour la quantification du cache KV", §3, step 3) each 16-token
+// tile gets one more MMA (m16n8k8) into the same score accumulator: A = the side
+// codes of the tile's tokens (r coordinates on K, masked as subnormals like the key
+// codes), B = (hi, lo) of (U_h^T q)_i * s_i per head, and the side zeros add
+// sum_i (U_h^T q)_i z_i to the group's bias.  U_h^T q is formed once per CTA.
+//
 // p.V uses the transposed orientation: channels on M, the 16 tokens on K, and on
 // N again (hi, lo) pairs, now of p_j * s_{j,g} (per-token value scale), moved from
 // the score accumulator layout to the B layout with movmatrix.  Value codes are
@@ -72,6 +79,26 @@ struct Quant {
   static_assert(WPT >= 1 && KSTEPS == WPT * KSPW, "key row too short for the fragment mapping");
   static_assert(RUN == 8 || RUN == 16 || RUN == 32, "value run must be 8, 16 or 32 bits");
   static_assert(MPG >= 1, "value group below 16 channels");
+};
+
+// Side-code geometry: SR coordinates of SQ bits per token, one row of ZB bytes.  Quad qi
+// (lanes with lane % 4 == qi) holds k-slots (2qi, 2qi+1) of the m16n8k8 side MMA, i.e.
+// coordinates (qi, qi + SR/2) for qi < SR/2; its A register of a row is
+// (row >> shift(qi)) & mask(qi), a pair of subnormals with factor 2^(p(qi)-24).
+template <int SR, int SQ>
+struct Side {
+  static constexpr int ZB = SR * SQ / 8;
+  static constexpr int NQ = SR / 2;            // quads that hold coordinates
+  static_assert(SR == 0 || (SR * SQ == 16 || SR * SQ == 32), "side row of 16 or 32 bits");
+  __host__ __device__ static constexpr int shift(int qi) {
+    return SR == 8 ? 8 * (qi >> 1) : (SQ == 8 ? 8 * qi : 0);
+  }
+  __host__ __device__ static constexpr int pos(int qi) {   // bit offset of the field in its half
+    return SR == 8 ? 4 * (qi & 1) : (SQ == 8 ? 0 : 4 * qi);
+  }
+  __host__ __device__ static constexpr uint32_t mask(int qi) {
+    return qi >= NQ ? 0u : (SQ == 8 ? 0x00FF00FFu : (0x000F000Fu << pos(qi)));
+  }
 };
 
 template <int DK>
@@ -198,7 +225,7 @@ __device__ __forceinline__ int qb_index(int e, int lane) { return ((e >> 2) * 32
 // k % R.  The tag of a stage is the unit whose copy was last issued into it: a warp
 // waits for its unit's tag before it waits on the stage's mbarrier, so that barrier is
 // never more than one phase away from the one the warp's parity names.
-template <int KSTEPS>
+template <int KSTEPS, int SR = 0>
 struct Smem {
   static constexpr int kQb = 0;
   static constexpr int kQf = kQb + 2 * KSTEPS * 32 * 4;     // q scaled by 2^-p, same layout
@@ -206,48 +233,56 @@ struct Smem {
   static constexpr int kIssued = kBars + kMaxRing * 8;
   static constexpr int kTag = kIssued + kMaxRing * 4;
   static constexpr int kFail = kTag + kMaxRing * 4;
-  static constexpr int kStages = kBars + 256;
-  static_assert(kFail + 4 <= kStages, "header overflow");
+  static constexpr int kQt = kFail + 16;                     // U_h^T q: fp32 [4 heads][SR]
+  static constexpr int kStages = kBars + (SR ? 512 : 256);
+  static_assert(kQt + 4 * SR * 4 <= kStages, "header overflow");
 };
 
 struct StageLayout {
-  int k_off, kmeta_off, v_off, vmeta_off, bytes;
+  int k_off, kmeta_off, v_off, vmeta_off, z_off, zmeta_off, bytes;
 };
 
-__host__ __device__ inline StageLayout quant_stage_layout(int gk, int dk, int kb, int vb, int nvg) {
+__host__ __device__ inline StageLayout quant_stage_layout(int gk, int dk, int kb, int vb, int nvg,
+                                                          int zb = 0, int sr = 0) {
   StageLayout s;
   s.k_off = 0;
   s.kmeta_off = gk * dk * kb / 8;
   s.v_off = s.kmeta_off + dk * 4;
   s.vmeta_off = s.v_off + gk * kDV * vb / 8;
-  s.bytes = s.vmeta_off + gk * nvg * 4;
+  s.z_off = s.vmeta_off + gk * nvg * 4;
+  s.zmeta_off = s.z_off + gk * zb;
+  s.bytes = s.zmeta_off + sr * 4;
   return s;
 }
 
 // Bytes of one stage (the larger of a key group and 16 padded fp16 rows) and the number of
 // stages that keep a CTA within a quarter of the SM's shared memory (4 CTAs per SM).
-template <int KB, int VB, int DK, int GV, int GK, bool QUANT>
+template <int KB, int VB, int DK, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
 constexpr int stage_bytes() {
   const int raw = Raw<DK>::BYTES;
-  const int qb = QUANT ? GK * DK * KB / 8 + DK * 4 + GK * kDV * VB / 8 + GK * (kDV / GV) * 4 : 0;
+  const int qb = QUANT ? GK * DK * KB / 8 + DK * 4 + GK * kDV * VB / 8 + GK * (kDV / GV) * 4 +
+                             GK * Side<SR, SQ>::ZB + SR * 4
+                       : 0;
   return ((raw > qb ? raw : qb) + 127) / 128 * 128;
 }
 
-template <int KB, int VB, int DK, int GV, int GK, bool QUANT>
+template <int KB, int VB, int DK, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
 constexpr int ring_stages() {
-  const int r = (kSmemPerCta - Smem<DK / 16>::kStages) / stage_bytes<KB, VB, DK, GV, GK, QUANT>();
+  const int r = (kSmemPerCta - Smem<DK / 16, SR>::kStages) /
+                stage_bytes<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
   return r < kMinRing ? kMinRing : (r > kMaxRing ? kMaxRing : r);
 }
 
-template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
 __global__ void __launch_bounds__(kThreads, 4)
 decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part) {
   using G = Quant<(QUANT ? KB : 4), (QUANT ? VB : 2), (QUANT ? DK : 128), (QUANT ? GV : 64)>;
   using R = Raw<DK>;
+  using Z = Side<SR, SQ>;
   constexpr int KSTEPS = DK / 16;
-  constexpr int STAGE = stage_bytes<KB, VB, DK, GV, GK, QUANT>();
-  constexpr int RING = ring_stages<KB, VB, DK, GV, GK, QUANT>();
-  using SM = Smem<KSTEPS>;
+  constexpr int STAGE = stage_bytes<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
+  constexpr int RING = ring_stages<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
+  using SM = Smem<KSTEPS, SR>;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -330,11 +365,46 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
             sm_qb[qb_index(2 * s + j, lane)] = ptx::h2_as_u32(pair);
           }
         }
+      if constexpr (SR > 0) {
+        // U_h^T q of head `warp`: each lane sums DK/32 channels, then the warp reduces
+        float* sm_qt = reinterpret_cast<float*>(smem + SM::kQt);
+        if (warp < NREP) {
+          const __half* qw = q + (static_cast<size_t>(b) * d.Hq + h * NREP + warp) * DK;
+          const float* uh = cb.side_u + static_cast<size_t>(h) * DK * SR;
+          float acc[SR];
+#pragma unroll
+          for (int i = 0; i < SR; ++i) acc[i] = 0.0f;
+#pragma unroll
+          for (int cc = 0; cc < DK / 32; ++cc) {
+            const int c = lane + 32 * cc;
+            const float qc = __half2float(qw[c]);
+#pragma unroll
+            for (int i4 = 0; i4 < SR; i4 += 4) {
+              const float4 u4 = *reinterpret_cast<const float4*>(uh + c * SR + i4);
+              acc[i4] = fmaf(u4.x, qc, acc[i4]);
+              acc[i4 + 1] = fmaf(u4.y, qc, acc[i4 + 1]);
+              acc[i4 + 2] = fmaf(u4.z, qc, acc[i4 + 2]);
+              acc[i4 + 3] = fmaf(u4.w, qc, acc[i4 + 3]);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < SR; ++i) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+          }
+          if (lane < SR) {
+            float v = acc[0];
+#pragma unroll
+            for (int i = 1; i < SR; ++i) v = lane == i ? acc[i] : v;
+            sm_qt[warp * SR + lane] = v;
+          }
+        }
+      }
       __syncthreads();
 
       // retained positions, one per lane (ascending), for masking the quantized tiles
       const int ret_pos = lane < w.ret.n ? w.ret.pos[lane] : -1;
-      const StageLayout L = quant_stage_layout(GK, DK, KB, VB, G::NVG);
+      const StageLayout L = quant_stage_layout(GK, DK, KB, VB, G::NVG, Z::ZB, SR);
       constexpr int gk = GK;
       constexpr int MT = GK / 16;     // 16-token m-tiles per key group
       // per-lane shuffle selectors for the bank-conflict-free value-row loads
@@ -359,6 +429,11 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
                       DK * 4, bar);
         ptx::bulk_g2s(dst + L.v_off, cb.vcode + tok * G::VW, gk * G::VBYTES_ROW, bar);
         ptx::bulk_g2s(dst + L.vmeta_off, cb.vsz + tok * G::NVG, gk * G::NVG * 4, bar);
+        if constexpr (SR > 0) {
+          ptx::bulk_g2s(dst + L.z_off, cb.zcode + tok * Z::ZB, gk * Z::ZB, bar);
+          ptx::bulk_g2s(dst + L.zmeta_off, cb.zsz + (static_cast<size_t>(bh) * (d.lcap / gk) + g) * SR,
+                        SR * 4, bar);
+        }
       };
 
       if (threadIdx.x == 0)
@@ -424,7 +499,27 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
             ptx::mma_16816(cbias[s & 1], za[0], za[0], za[1], za[1], qbx[2 * ls], qbx[2 * ls + 1]);
           }
         }
-        const float beta = (cbias[0][0] + cbias[1][0]) * alpha;
+        float side_bias = 0.0f;
+        uint32_t bz = 0u;                 // B of the side MMA: (hi or lo) of (U^T q)_i * s_i * 2^-p
+        if constexpr (SR > 0) {
+          const float* sm_qt = reinterpret_cast<const float*>(smem + SM::kQt);
+          const __half2* zm = reinterpret_cast<const __half2*>(S + L.zmeta_off);
+          if (qi < Z::NQ) {
+            const float f = 1.0f / static_cast<float>(1 << Z::pos(qi));
+            const float2 m0 = __half22float2(zm[qi]), m1 = __half22float2(zm[qi + Z::NQ]);
+            const int hb = bvalid ? bhead : 0;
+            const float x0 = sm_qt[hb * SR + qi] * m0.x * f;
+            const float x1 = sm_qt[hb * SR + qi + Z::NQ] * m1.x * f;
+            const __half2 p0 = ptx::u32_as_h2(ptx::split_hi_lo_trunc(x0));
+            const __half2 p1 = ptx::u32_as_h2(ptx::split_hi_lo_trunc(x1));
+            bz = ptx::h2_as_u32(blo ? __highs2half2(p0, p1) : __lows2half2(p0, p1));
+          }
+          const int hc = cvalid ? qi : 0;
+#pragma unroll
+          for (int i = 0; i < SR; ++i)
+            side_bias = fmaf(sm_qt[hc * SR + i], __high2float(zm[i]), side_bias);
+        }
+        const float beta = (cbias[0][0] + cbias[1][0] + side_bias) * alpha;
 
         // ---- scores of the whole group ----
         float sc[MT][2];
@@ -446,6 +541,19 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
               ptx::mma_16816(cs, r0[2 * ls], r1[2 * ls], r0[2 * ls + 1], r1[2 * ls + 1], bq[s][0],
                              bq[s][1]);
             }
+          }
+          if constexpr (SR > 0) {
+            const unsigned char* zr = S + L.z_off;
+            uint32_t x0, x1;
+            if constexpr (Z::ZB == 4) {
+              x0 = *reinterpret_cast<const uint32_t*>(zr + t0 * 4);
+              x1 = *reinterpret_cast<const uint32_t*>(zr + (t0 + 8) * 4);
+            } else {
+              // (c0 c1 | c2 c3) of a 16-bit row -> c0 c1 in the low half, c2 c3 in the high half
+              x0 = ptx::prmt(*reinterpret_cast<const uint16_t*>(zr + t0 * 2), 0u, 0x0100u);
+              x1 = ptx::prmt(*reinterpret_cast<const uint16_t*>(zr + (t0 + 8) * 2), 0u, 0x0100u);
+            }
+            ptx::mma_1688(cs, (x0 >> Z::shift(qi)) & Z::mask(qi), (x1 >> Z::shift(qi)) & Z::mask(qi), bz);
           }
           sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
           sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
@@ -746,15 +854,16 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   }
 }
 
-template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
 cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
                    const Partials& p, cudaStream_t s) {
-  constexpr int stage = stage_bytes<KB, VB, DK, GV, GK, QUANT>();
-  constexpr int ring = ring_stages<KB, VB, DK, GV, GK, QUANT>();
-  int smem = Smem<DK / 16>::kStages + ring * stage;
+  constexpr int stage = stage_bytes<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
+  constexpr int ring = ring_stages<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
+  constexpr int hdr = Smem<DK / 16, SR>::kStages;
+  int smem = hdr + ring * stage;
   const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
-  if (Smem<DK / 16>::kStages + merge > smem) smem = Smem<DK / 16>::kStages + merge;
-  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT>;
+  if (hdr + merge > smem) smem = hdr + merge;
+  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ>;
   static int configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

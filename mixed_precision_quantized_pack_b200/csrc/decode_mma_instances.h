@@ -1,9 +1,11 @@
 // The tensor-core decode instances this library is built with, as an X-macro:
-//   Q(KB, VB, DK, NREP, GV, GK)  quantized caches (value head dim 128)
-//   F(DK, NREP)                  unquantized fp16 caches (value head dim 128)
-// decode_mma.cu builds its dispatch table from the same list; each
-// decode_mma_inst_*.cu file instantiates the entries whose KB it owns.  Shapes
-// not listed here run on the generic CUDA-core kernel.
+//   Q(KB, VB, DK, NREP, GV, GK)          quantized caches (value head dim 128)
+//   S(KB, VB, DK, NREP, GV, GK, SR, SQ)  quantized caches with a rank-SR, SQ-bit side code
+//   F(DK, NREP)                          unquantized fp16 caches (value head dim 128)
+// decode_mma.cu builds its dispatch table from the same lists; each
+// decode_mma_inst_k*.cu file instantiates the Q entries whose KB it owns,
+// decode_mma_inst_side.cu the S entries.  Shapes not listed here run on the
+// generic CUDA-core kernel.
 #pragma once
 
 #define KVQ_MMA_QUANT_INSTANCES(Q)                                                              \
@@ -15,3 +17,7 @@
   Q(2, 2, 128, 4, 64, 64) Q(2, 2, 128, 1, 64, 64) Q(2, 2, 128, 4, 32, 32) Q(2, 2, 128, 1, 32, 32)
 
 #define KVQ_MMA_FP16_INSTANCES(F) F(128, 4) F(128, 1) F(32, 4) F(32, 1)
+
+#define KVQ_MMA_SIDE_INSTANCES(S)                                                               \
+  S(4, 2, 128, 4, 64, 64, 4, 4) S(4, 2, 128, 4, 64, 64, 4, 8) S(4, 2, 128, 4, 64, 64, 8, 4)      \
+  S(2, 2, 128, 4, 64, 64, 4, 4) S(2, 2, 128, 4, 64, 64, 4, 8) S(2, 2, 128, 4, 64, 64, 8, 4)

@@ -5,7 +5,10 @@
 //   k_hat = code * s + z (key groups per channel, value groups per token), or the
 //           fp16 copy for window and retained tokens ("LogQuant: Log-Distributed
 //           2-Bit Quantization of KV Cache", §Méthodologie 2 and 3);
-//   score = q . k_hat / sqrt(d_k) ("Thin Keys, Full Values", §2), kept in log2 units;
+//   score = q . k_hat / sqrt(d_k) ("Thin Keys, Full Values", §2), kept in log2 units,
+//           plus (U_h^T q) . z_hat for quantized tokens when the cache has a side code
+//           ("HeadQ: Distortion visible par le modele et correction dans l'espace des
+//           scores pour la quantification du cache KV", §3, step 3);
 //   online softmax, o = sum_j 2^(score_j - m) v_hat_j.
 // One warp per token: each lane holds d/32 channels, dot products reduce with
 // warp shuffles.  The tensor-core kernel replaces this one on the shapes it
@@ -24,6 +27,7 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
   __shared__ float sm_m[kWarps][kMaxRep];
   __shared__ float sm_l[kWarps][kMaxRep];
   __shared__ float sm_o[kWarps][kMaxRep][kMaxC * 32];
+  __shared__ float sm_qt[kMaxRep][8];     // U_h^T q of each query head, times the score scale
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int bh = b * d.Hkv + h;
@@ -47,6 +51,18 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
     for (int j = 0; j < kMaxC; ++j) o[r][j] = 0.0f;
   }
 
+  if (d.sr) {
+    for (int idx = threadIdx.x; idx < nrep * d.sr; idx += blockDim.x) {
+      const int r = idx / d.sr, i = idx % d.sr;
+      const __half* qh = q + (static_cast<size_t>(b) * d.Hq + h * nrep + r) * d.dk;
+      const float* u = cb.side_u + static_cast<size_t>(h) * d.dk * d.sr + i;
+      float acc = 0.0f;
+      for (int c = 0; c < d.dk; ++c) acc = fmaf(u[c * d.sr], __half2float(qh[c]), acc);
+      sm_qt[r][i] = acc * w.score_scale;
+    }
+    __syncthreads();
+  }
+
   const bool quant = split < w.splits_q;
   int begin, end;
   if (quant) {
@@ -62,10 +78,26 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
 
   for (int i = begin + warp; i < end; i += kWarps) {
     float kh[kMaxC], vh[kMaxC];
+    float zhat[8];                                              // side code, decoded
+#pragma unroll
+    for (int j = 0; j < 8; ++j) zhat[j] = 0.0f;
     if (quant) {
       bool retained = false;
       for (int r = 0; r < w.ret.n; ++r) retained |= (w.ret.pos[r] == i);
       if (retained) continue;                                   // read from the fp16 list
+      if (d.sr) {
+        const uint8_t* zr = cb.zcode + (static_cast<size_t>(bh) * d.lcap + i) * d.zb;
+        const uint32_t row = d.zb == 4 ? *reinterpret_cast<const uint32_t*>(zr)
+                                       : *reinterpret_cast<const uint16_t*>(zr);
+        const __half2* zs = cb.zsz + (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * d.sr;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < d.sr) {
+            const float2 sz = __half22float2(zs[j]);
+            const uint32_t code = (row >> (j * d.sq)) & ((1u << d.sq) - 1u);
+            zhat[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
+          }
+      }
       const uint32_t* kr = cb.kcode + (static_cast<size_t>(bh) * d.lcap + i) * d.kw;
       const __half* ks = reinterpret_cast<const __half*>(cb.ksz) +
                          (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * 2 * d.dk;
@@ -117,6 +149,11 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
       for (int j = 0; j < kMaxC; ++j) s = fmaf(qr[r][j], kh[j], s);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      if (d.sr) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < d.sr) s = fmaf(sm_qt[r][j], zhat[j], s);
+      }
       const float mn = fmaxf(m[r], s);
       const float alpha = exp2f(m[r] - mn);
       const float pe = exp2f(s - mn);

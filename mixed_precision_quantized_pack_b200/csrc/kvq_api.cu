@@ -72,6 +72,14 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
         c->group_v % 8 != 0 || (c->group_v * c->v_bits) % 32 != 0)
       return KVQ_ERR_UNSUPPORTED;
   }
+  // side code: rank 4 or 8, 4 or 8 bits, one 2- or 4-byte row per token, quantized keys
+  if (c->side_rank != 0) {
+    if (raw) return KVQ_ERR_UNSUPPORTED;
+    if (c->side_rank != 4 && c->side_rank != 8) return KVQ_ERR_UNSUPPORTED;
+    if (c->side_bits != 4 && c->side_bits != 8) return KVQ_ERR_UNSUPPORTED;
+    const int row_bits = c->side_rank * c->side_bits;
+    if (row_bits != 16 && row_bits != 32) return KVQ_ERR_UNSUPPORTED;
+  }
   // every element index must fit comfortably in 64 bits and every position in int
   const long long lcap = raw ? c->max_context
                              : (static_cast<long long>(c->max_context) + c->group_k - 1) /
@@ -96,6 +104,9 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
   x.kw = raw ? 0 : c->d_k * c->k_bits / 32;
   x.vw = raw ? 0 : c->d_v * c->v_bits / 32;
   x.nvg = raw ? 1 : c->d_v / c->group_v;
+  x.sr = c->side_rank;
+  x.sq = c->side_rank ? c->side_bits : 0;
+  x.zb = c->side_rank * x.sq / 8;
   *d = x;
   return KVQ_OK;
 }
@@ -123,7 +134,9 @@ int split_cap(const kvq::Dims& d) {
   return std::min(256, std::max(2, 8192 / rows));
 }
 
-// Occupancy assumed by the planner (CTAs per SM) for each decode kernel.
+// CTAs per SM the planner's wave model assumes.  Both kernels are resident 4 per SM; for
+// the tensor-core kernel the model uses 3, which picks the split counts measured fastest
+// on the long-context workloads.
 int ctas_per_sm(bool fast) { return fast ? 3 : 4; }
 
 // Chooses the split counts: the number of CTAs per (b, kv head) over the quantized
@@ -140,7 +153,8 @@ int plan_decode(const kvq::Dims& d, int L, int sm_count, int num_splits, bool fa
   const long long slots = static_cast<long long>(sm_count) * ctas_per_sm(fast);
   // cost model in bytes read: per quantized group, per fp16 token, per CTA
   const double bq = d.quantized()
-                        ? static_cast<double>(d.gk) * (d.kw * 4 + d.vw * 4 + d.nvg * 4) + d.dk * 4.0
+                        ? static_cast<double>(d.gk) * (d.kw * 4 + d.vw * 4 + d.nvg * 4 + d.zb) +
+                              d.dk * 4.0 + d.sr * 4.0
                         : 0.0;
   const double bf = 2.0 * (d.dk + d.dv);
   const double cta_cost = 16384.0;
@@ -196,6 +210,9 @@ kvq::CacheBufs cache_bufs(const kvq_cache* c) {
   b.win_v = static_cast<const __half*>(c->buf.win_v);
   b.ret_k = static_cast<const __half*>(c->buf.ret_k);
   b.ret_v = static_cast<const __half*>(c->buf.ret_v);
+  b.zcode = static_cast<const uint8_t*>(c->buf.zcode);
+  b.zsz = static_cast<const __half2*>(c->buf.zsz);
+  b.side_u = static_cast<const float*>(c->buf.side_u);
   return b;
 }
 
@@ -232,6 +249,11 @@ int kvq_buffer_sizes(const kvq_config* cfg, kvq_sizes* out) {
     s.vsz = bh * d.lcap * d.nvg * 4;
     s.ret_k = bh * kvq::kMaxRetained * d.dk * 2;
     s.ret_v = bh * kvq::kMaxRetained * d.dv * 2;
+    if (d.sr) {
+      s.zcode = bh * d.lcap * d.zb;
+      s.zsz = bh * (d.lcap / d.gk) * d.sr * 4;
+      s.side_u = static_cast<size_t>(d.Hkv) * d.dk * d.sr * 4;
+    }
   }
   s.win_k = bh * d.cap * d.dk * 2;
   s.win_v = bh * d.cap * d.dv * 2;
@@ -253,8 +275,13 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
     for (const void* p : q)
       if (!p) return KVQ_ERR_INVALID_ARG;
   }
-  const void* all[] = {bufs->kcode, bufs->ksz, bufs->vcode, bufs->vsz,
-                       bufs->win_k, bufs->win_v, bufs->ret_k, bufs->ret_v};
+  if (d.sr) {
+    const void* z[] = {bufs->zcode, bufs->zsz, bufs->side_u};
+    for (const void* p : z)
+      if (!p) return KVQ_ERR_INVALID_ARG;
+  }
+  const void* all[] = {bufs->kcode, bufs->ksz, bufs->vcode, bufs->vsz, bufs->win_k, bufs->win_v,
+                       bufs->ret_k, bufs->ret_v, bufs->zcode, bufs->zsz, bufs->side_u};
   for (const void* p : all)
     if (p && !aligned16(p)) return KVQ_ERR_ALIGN;
   int dev = 0, sms = 0;
@@ -304,6 +331,11 @@ int kvq_quantize_prefill(kvq_cache* c, const void* k, const void* v, int L, void
                                               static_cast<uint32_t*>(c->buf.kcode),
                                               static_cast<__half2*>(c->buf.ksz), s));
     if (!rc)
+      rc = check_cuda(kvq::launch_quantize_side(
+          d, kh, L, 0, Q / d.gk, static_cast<const uint32_t*>(c->buf.kcode),
+          static_cast<const __half2*>(c->buf.ksz), static_cast<const float*>(c->buf.side_u),
+          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), s));
+    if (!rc)
       rc = check_cuda(kvq::launch_quantize_values(d, vh, L, 0, Q,
                                                   static_cast<uint32_t*>(c->buf.vcode),
                                                   static_cast<__half2*>(c->buf.vsz), s));
@@ -352,6 +384,11 @@ int kvq_append(kvq_cache* c, const void* k_new, const void* v_new, void* stream)
     rc = check_cuda(kvq::launch_quantize_keys(d, wk, d.cap, Q / d.gk, 1,
                                               static_cast<uint32_t*>(c->buf.kcode),
                                               static_cast<__half2*>(c->buf.ksz), s));
+    if (!rc)
+      rc = check_cuda(kvq::launch_quantize_side(
+          d, wk, d.cap, Q / d.gk, 1, static_cast<const uint32_t*>(c->buf.kcode),
+          static_cast<const __half2*>(c->buf.ksz), static_cast<const float*>(c->buf.side_u),
+          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), s));
     if (!rc)
       rc = check_cuda(kvq::launch_quantize_values(d, wv, d.cap, Q, d.gk,
                                                   static_cast<uint32_t*>(c->buf.vcode),

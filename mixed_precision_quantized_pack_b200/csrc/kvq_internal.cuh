@@ -17,6 +17,9 @@ struct Dims {
   int kw;     // u32 words per key row:   dk * kb / 32
   int vw;     // u32 words per value row: dv * vb / 32
   int nvg;    // value groups per token:  dv / gv
+  int sr;     // side-code rank r (0: no side code)
+  int sq;     // bits per side code
+  int zb;     // bytes per side-code row: sr * sq / 8 (2 or 4)
   bool quantized() const { return kb != 16; }
 };
 
@@ -56,6 +59,9 @@ struct CacheBufs {
   const __half* win_v;
   const __half* ret_k;
   const __half* ret_v;
+  const uint8_t* zcode;   // side codes (null without a side code)
+  const __half2* zsz;     // side (scale, zero) per key group and coordinate
+  const float* side_u;    // basis U_h, fp32 [Hkv][dk][sr]
 };
 
 // Workspace layout: [status u32, padded to 256 B][(m, l) float2 per partial][o floats]
@@ -71,6 +77,11 @@ Partials workspace_views(const Dims& d, int splits, void* ws);
 // ---- launchers (return the launch error, cudaSuccess when fine) ----
 cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
                                  int n_groups, uint32_t* kcode, __half2* ksz, cudaStream_t s);
+// Side codes of key groups [g_begin, g_begin + n_groups) whose base codes and (scale, zero)
+// are already in kcode / ksz (same stream); keys read from src as for launch_quantize_keys.
+cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows, int g_begin,
+                                 int n_groups, const uint32_t* kcode, const __half2* ksz,
+                                 const float* side_u, uint8_t* zcode, __half2* zsz, cudaStream_t s);
 cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_rows, int t_begin,
                                    int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s);
 cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,

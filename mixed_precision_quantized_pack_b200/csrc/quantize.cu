@@ -92,6 +92,96 @@ __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_row
   }
 }
 
+// Side code of key groups ("HeadQ: Distortion visible par le modele et correction dans
+// l'espace des scores pour la quantification du cache KV", §3, Aperçu de l'algorithme,
+// step 2): for every token of the group the base residual e = k - (code*s + z) of each
+// channel, its projection y = U_h^T e on the kv head's basis (fp32, channels summed in
+// ascending order, one rounded product and one rounded sum per channel), then the
+// min-max quantizer above per coordinate over the group's tokens.  The base codes and
+// (scale, zero) are read back from kcode / ksz, so both describe the same key.
+// One CTA per (group, b * kv head).  Shared memory: e [gk][dk + 1] (padded so that the
+// threads of a warp, which read one channel of several tokens, hit distinct banks),
+// U_h [dk][sr] and y [gk][sr].
+template <int SQ>
+__global__ void quantize_side_kernel(const __half* __restrict__ src, int src_rows, int dk, int kb,
+                                     int gk, int g_begin, int lcap, int hkv, int sr, int zb,
+                                     const uint32_t* __restrict__ kcode,
+                                     const __half2* __restrict__ ksz,
+                                     const float* __restrict__ side_u,
+                                     uint8_t* __restrict__ zcode, __half2* __restrict__ zsz) {
+  extern __shared__ float sm_side[];
+  __shared__ float2 params[8];
+  const int es = dk + 1;
+  float* e = sm_side;
+  float* u = e + gk * es;
+  float* y = u + dk * sr;
+  const int g = g_begin + blockIdx.x;
+  const int bh = blockIdx.y;
+  const int h = bh % hkv;
+  const size_t base = static_cast<size_t>(bh) * src_rows;
+  const int per = 32 / kb, half = per / 2, words = dk / per;
+  const int quarter = words % 4 == 0 ? words / 4 : 0;
+  const __half* blk =
+      reinterpret_cast<const __half*>(ksz) + (static_cast<size_t>(bh) * (lcap / gk) + g) * 2 * dk;
+  for (int idx = threadIdx.x; idx < gk * dk; idx += blockDim.x) {
+    const int t = idx / dk, c = idx % dk;
+    const int row = (g * gk + t) % src_rows;
+    const float x = __half2float(src[(base + row) * dk + c]);
+    const uint32_t w = kcode[(static_cast<size_t>(bh) * lcap + g * gk + t) * words + c / per];
+    const uint32_t code = (w >> ((c % per) * kb)) & ((1u << kb) - 1u);
+    // the channel's (scale, zero) slots in the group's paired, quarter-interleaved block
+    const int wd = c / per, r = c % per;
+    const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
+    const int slot = pos * 2 * per + (r % half) * 2 + r / half;
+    const float kh = __fadd_rn(__fmul_rn(static_cast<float>(code), __half2float(blk[slot])),
+                               __half2float(blk[slot + per]));
+    e[t * es + c] = __fsub_rn(x, kh);
+  }
+  for (int idx = threadIdx.x; idx < dk * sr; idx += blockDim.x)
+    u[idx] = side_u[static_cast<size_t>(h) * dk * sr + idx];
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < gk * sr; idx += blockDim.x) {
+    const int t = idx / sr, i = idx % sr;
+    float acc = 0.0f;
+    for (int c = 0; c < dk; ++c) acc = __fadd_rn(acc, __fmul_rn(e[t * es + c], u[c * sr + i]));
+    y[idx] = acc;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int i = warp; i < sr; i += blockDim.x / 32) {
+    float mn = INFINITY, mx = -INFINITY;
+    for (int t = lane; t < gk; t += 32) {
+      mn = fminf(mn, y[t * sr + i]);
+      mx = fmaxf(mx, y[t * sr + i]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    }
+    if (lane == 0) {
+      const GroupParams gp = group_params<SQ>(mn, mx);
+      zsz[(static_cast<size_t>(bh) * (lcap / gk) + g) * sr + i] = gp.sz;
+      params[i] = make_float2(gp.scale, gp.zero);
+    }
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < gk; t += blockDim.x) {
+    uint32_t row = 0;
+    for (int i = 0; i < sr; ++i) {
+      GroupParams gp;
+      gp.scale = params[i].x;
+      gp.zero = params[i].y;
+      row |= quant_code<SQ>(y[t * sr + i], gp) << (i * SQ);
+    }
+    uint8_t* dst = zcode + (static_cast<size_t>(bh) * lcap + g * gk + t) * zb;
+    if (zb == 4)
+      *reinterpret_cast<uint32_t*>(dst) = row;
+    else
+      *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(row);
+  }
+}
+
 // One thread per (kv row, token, value group).  gv is a multiple of 8 and of 32/BITS.
 template <int BITS>
 __global__ void quantize_values_kernel(const __half* __restrict__ src, int src_rows, int dv,
@@ -240,6 +330,24 @@ cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows,
     case 8: quantize_keys_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz); break;
     default: return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows, int g_begin,
+                                 int n_groups, const uint32_t* kcode, const __half2* ksz,
+                                 const float* side_u, uint8_t* zcode, __half2* zsz, cudaStream_t s) {
+  if (n_groups <= 0 || d.sr == 0) return cudaSuccess;
+  const size_t smem = (static_cast<size_t>(d.gk) * (d.dk + 1) + d.dk * d.sr + d.gk * d.sr) * 4;
+  dim3 grid(n_groups, d.B * d.Hkv);
+  auto kern = d.sq == 4 ? quantize_side_kernel<4> : quantize_side_kernel<8>;
+  if (d.sq != 4 && d.sq != 8) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<grid, 256, smem, s>>>(src, src_rows, d.dk, d.kb, d.gk, g_begin, d.lcap, d.Hkv, d.sr, d.zb,
+                               kcode, ksz, side_u, zcode, zsz);
   return cudaGetLastError();
 }
 

@@ -33,8 +33,11 @@ KVQ_STATUS_TIMEOUT = 1
 KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 CONFIG_FIELDS = ("batch", "n_q_heads", "n_kv_heads", "d_k", "d_v", "k_bits", "v_bits", "group_k",
-                 "group_v", "window", "log_retain", "max_context")
+                 "group_v", "window", "log_retain", "max_context", "side_rank", "side_bits")
+OPTIONAL_CONFIG = ("side_rank", "side_bits")          # default 0: no side code
 BUFFER_FIELDS = ("kcode", "ksz", "vcode", "vsz", "win_k", "win_v", "ret_k", "ret_v")
+SIDE_FIELDS = ("zcode", "zsz", "side_u")
+SIZE_FIELDS = BUFFER_FIELDS + ("workspace",) + SIDE_FIELDS
 
 
 class kvq_config(ctypes.Structure):
@@ -42,11 +45,11 @@ class kvq_config(ctypes.Structure):
 
 
 class kvq_sizes(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_size_t) for n in BUFFER_FIELDS + ("workspace",)]
+    _fields_ = [(n, ctypes.c_size_t) for n in SIZE_FIELDS]
 
 
 class kvq_buffers(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_FIELDS]
+    _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_FIELDS + SIDE_FIELDS]
 
 
 class kvq_plan(ctypes.Structure):
@@ -117,7 +120,7 @@ def _stream(stream=None) -> int:
 
 
 def make_config(cfg: Dict[str, int]) -> kvq_config:
-    return kvq_config(*[int(cfg[n]) for n in CONFIG_FIELDS])
+    return kvq_config(*[int(cfg.get(n, 0) if n in OPTIONAL_CONFIG else cfg[n]) for n in CONFIG_FIELDS])
 
 
 # ---- the C entry points, same names -----------------------------------------
@@ -129,7 +132,7 @@ def kvq_buffer_sizes(cfg: Dict[str, int]) -> Dict[str, int]:
     out = kvq_sizes()
     _check(lib().kvq_buffer_sizes(ctypes.byref(make_config(cfg)), ctypes.byref(out)),
            "kvq_buffer_sizes")
-    return {n: int(getattr(out, n)) for n in BUFFER_FIELDS + ("workspace",)}
+    return {n: int(getattr(out, n)) for n in SIZE_FIELDS}
 
 
 def kvq_plan_decode(cfg: Dict[str, int], L: int, sm_count: int, num_splits: int = 0) -> Dict[str, int]:
@@ -146,7 +149,7 @@ def kvq_retained_positions(Q: int) -> List[int]:
 
 
 def kvq_cache_init(cfg: Dict[str, int], ptrs: Dict[str, int]) -> int:
-    bufs = kvq_buffers(*[ptrs.get(n) or None for n in BUFFER_FIELDS])
+    bufs = kvq_buffers(*[ptrs.get(n) or None for n in BUFFER_FIELDS + SIDE_FIELDS])
     h = _P()
     _check(lib().kvq_cache_init(ctypes.byref(make_config(cfg)), ctypes.byref(bufs), ctypes.byref(h)),
            "kvq_cache_init")
@@ -226,16 +229,25 @@ def _fp16_cuda(t: torch.Tensor, shape, name: str) -> torch.Tensor:
 
 
 class KVCache:
-    """One attention layer's packed KV cache in device memory owned by PyTorch."""
+    """One attention layer's packed KV cache in device memory owned by PyTorch.
 
-    def __init__(self, cfg: Dict[str, int], device=None):
+    With cfg["side_rank"] = r > 0 the cache keeps a side code and ``side_basis`` (fp32
+    [Hkv][d_k][r], any device) is copied into the cache's basis buffer."""
+
+    def __init__(self, cfg: Dict[str, int], device=None, side_basis: Optional[torch.Tensor] = None):
         self.cfg = dict(cfg)
         self.device = torch.device(device or "cuda")
         self.sizes = kvq_buffer_sizes(self.cfg)
         self.buffers: Dict[str, Optional[torch.Tensor]] = {}
-        for n in BUFFER_FIELDS:
+        for n in BUFFER_FIELDS + SIDE_FIELDS:
             sz = self.sizes[n]
             self.buffers[n] = torch.zeros(sz, dtype=torch.uint8, device=self.device) if sz else None
+        r = int(self.cfg.get("side_rank", 0))
+        if r:
+            shape = (self.cfg["n_kv_heads"], self.cfg["d_k"], r)
+            if side_basis is None or tuple(side_basis.shape) != shape:
+                raise ValueError(f"side_basis: need an fp32 tensor of shape {shape}")
+            self.view("side_u").copy_(side_basis.to(torch.float32))
         ptrs = {n: (b.data_ptr() if b is not None else 0) for n, b in self.buffers.items()}
         self.handle = kvq_cache_init(self.cfg, ptrs)
         self.workspace = torch.empty(self.sizes["workspace"], dtype=torch.uint8, device=self.device)
@@ -321,5 +333,12 @@ class KVCache:
             "ret_k": (torch.float16, (B, H, KVQ_MAX_RETAINED, dk)),
             "ret_v": (torch.float16, (B, H, KVQ_MAX_RETAINED, dv)),
         }
+        r, sq = int(c.get("side_rank", 0)), int(c.get("side_bits", 0))
+        if r:
+            shapes.update({
+                "zcode": (torch.uint8, (B, H, lcap, r * sq // 8)),
+                "zsz": (torch.float16, (B, H, lcap // gk, r, 2)),
+                "side_u": (torch.float32, (H, dk, r)),
+            })
         dt, shape = shapes[name]
         return buf.view(dt).view(shape)

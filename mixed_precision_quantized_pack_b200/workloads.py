@@ -14,7 +14,12 @@ values do not):
   shared by every sequence and token;
 * values and queries ~ N(0, 1);
 * thin keys ("Thin Keys, Full Values", §2): 128-dim keys drawn as above and
-  projected to d_k dims by P with N(0, std 1/sqrt(128)) entries, in fp32.
+  projected to d_k dims by P with N(0, std 1/sqrt(128)) entries, in fp32;
+* side-code workloads ("HeadQ", §3): per kv head a basis U_h, the orthonormal
+  factor of a Gaussian d_k x r matrix, standing in for the PCA basis of calibration
+  queries; their queries put a fraction f of their energy in span(U_h):
+  q = sqrt(1-f) n + sqrt(f d_k / r) U_h a with n, a ~ N(0, I), so |q|^2 ~ d_k as
+  for plain queries.
 
 Everything is drawn in fp32 from one ``torch.Generator`` seeded per workload and
 rounded once to fp16.  The generator lives on the device the tensors are made on,
@@ -48,6 +53,9 @@ class Workload:
     appends: int          # append+decode steps after the prefill (0: one decode only)
     thin_from: int = 0    # >0: keys are a projection of thin_from-dim keys
     seed: int = 0
+    side_rank: int = 0    # >0: a side code of this rank ...
+    side_bits: int = 0    # ... and bits per code
+    q_in_basis: float = 0.0   # side workloads: fraction of query energy in span(U_h)
 
     @property
     def n_rep(self) -> int:
@@ -65,7 +73,8 @@ class Workload:
                     d_k=self.d_k, d_v=self.d_v, k_bits=self.k_bits, v_bits=self.v_bits,
                     group_k=self.group_k, group_v=self.group_v, window=self.window,
                     log_retain=self.log_retain,
-                    max_context=max_context if max_context is not None else self.max_context)
+                    max_context=max_context if max_context is not None else self.max_context,
+                    side_rank=self.side_rank, side_bits=self.side_bits)
 
 
 def _base(**kw) -> Workload:
@@ -88,6 +97,12 @@ WORKLOADS: Dict[str, Workload] = {
                      n_kv_heads=8, d_k=32, d_v=128, context=16384, k_bits=4, v_bits=2,
                      group_k=32, group_v=32, window=64, log_retain=0, appends=0,
                      thin_from=128, seed=1003),
+    # the 32k case with 2-bit keys and a rank-4, 4-bit side code ("HeadQ", §5: rank 4 on
+    # the 2-bit rows it repairs most)
+    "headq32k": _base(name="headq-b32-32/8-32k-k2v2-r4q4-logretain", batch=32, n_q_heads=32,
+                      n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=2, v_bits=2,
+                      group_k=64, group_v=64, window=128, log_retain=1, appends=0, seed=1005,
+                      side_rank=4, side_bits=4, q_in_basis=0.9),
 }
 
 SWEEP_BATCHES = (1, 8, 32, 64)
@@ -148,12 +163,29 @@ class Inputs:
         B = w.batch
         self.k = keys(B, w.context)
         self.v = normal((B, w.n_kv_heads, w.context, w.d_v))
+        self.side_basis: Optional[torch.Tensor] = None
+        if w.side_rank:
+            g = torch.randn((w.n_kv_heads, w.d_k, w.side_rank), generator=gen, device=dev,
+                            dtype=torch.float32)
+            self.side_basis = torch.linalg.qr(g.cpu().double())[0].float().to(dev)
+
+        def query(batch):
+            n = torch.randn((batch, w.n_q_heads, w.d_k), generator=gen, device=dev, dtype=torch.float32)
+            if not w.side_rank:
+                return n.to(torch.float16)
+            a = torch.randn((batch, w.n_q_heads, w.side_rank), generator=gen, device=dev,
+                            dtype=torch.float32)
+            U = self.side_basis.repeat_interleave(w.n_rep, dim=0)          # [Hq][d_k][r]
+            f = w.q_in_basis
+            q = math.sqrt(1.0 - f) * n + math.sqrt(f * w.d_k / w.side_rank) * torch.einsum("hdr,bhr->bhd", U, a)
+            return q.to(torch.float16)
+
         n_dec = max(w.appends, 1)
         self.q: List[torch.Tensor] = []
         self.k_app: List[torch.Tensor] = []
         self.v_app: List[torch.Tensor] = []
         for _ in range(n_dec):
-            self.q.append(normal((B, w.n_q_heads, w.d_k)))
+            self.q.append(query(B))
             if w.appends:
                 self.k_app.append(keys(B, 1)[:, :, 0, :].contiguous())
                 self.v_app.append(normal((B, w.n_kv_heads, w.d_v)))

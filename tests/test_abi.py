@@ -138,3 +138,40 @@ def test_planner_rejects_lengths_outside_the_cache():
     for L in (0, 1001):
         with pytest.raises(K.KVQError):
             K.kvq_plan_decode(c, L, 148, 0)
+
+
+# ---------------------------------------------------------------- side code ----
+@pytest.mark.parametrize("sr,sq", [(4, 4), (4, 8), (8, 4)])
+def test_side_buffer_sizes_match_the_oracle_layout(sr, sq):
+    for w in (W.WORKLOADS["headq32k"], W.WORKLOADS["long32k"].with_(side_rank=sr, side_bits=sq)):
+        c = dict(w.kvq_config(), side_rank=sr, side_bits=sq)
+        got = K.kvq_buffer_sizes(c)
+        want = O.buffer_bytes(c)
+        for n in K.BUFFER_FIELDS + ("zcode", "zsz"):
+            assert got[n] == want[n], n
+        assert got["side_u"] == c["n_kv_heads"] * c["d_k"] * sr * 4
+
+
+@pytest.mark.parametrize("bad", [
+    dict(side_rank=3, side_bits=4), dict(side_rank=4, side_bits=2), dict(side_rank=8, side_bits=8),
+    dict(side_rank=16, side_bits=2), dict(side_rank=4, side_bits=4, k_bits=16, v_bits=16),
+])
+def test_invalid_side_codes_are_rejected(bad):
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_buffer_sizes(cfg(**bad))
+    assert e.value.code == K.KVQ_ERR_UNSUPPORTED
+
+
+def test_side_code_buffers_are_required_and_aligned():
+    c = cfg(side_rank=4, side_bits=4)
+    fields = K.BUFFER_FIELDS + K.SIDE_FIELDS
+    ptrs = {n: 4096 * (i + 1) for i, n in enumerate(fields)}
+    ptrs["side_u"] = 0
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_cache_init(c, ptrs)
+    assert e.value.code == K.KVQ_ERR_INVALID_ARG
+    ptrs = {n: 4096 * (i + 1) for i, n in enumerate(fields)}
+    ptrs["zsz"] += 4
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_cache_init(c, ptrs)
+    assert e.value.code == K.KVQ_ERR_ALIGN

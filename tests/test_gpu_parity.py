@@ -39,6 +39,8 @@ def compare_state(gc: K.KVCache, oc: O.OracleCache, b_rows=None, where=""):
         gk = c["group_k"]
         pairs = [("kcode", slice(0, Q)), ("ksz", slice(0, Q // gk)), ("vcode", slice(0, Q)),
                  ("vsz", slice(0, Q))]
+        if c.get("side_rank", 0):
+            pairs += [("zcode", slice(0, Q)), ("zsz", slice(0, Q // gk))]
         for name, sl in pairs:
             g = gc.view(name)[rows][:, :, sl].cpu().numpy()
             o = getattr(oc, name)[:, :, sl]
@@ -63,13 +65,21 @@ def compare_state(gc: K.KVCache, oc: O.OracleCache, b_rows=None, where=""):
             assert np.array_equal(g.view(np.uint16), o.view(np.uint16)), f"{where}: {name} differs"
 
 
+def make_caches(cfg, inp, batch=None):
+    """A GPU cache and an oracle cache of one configuration (with the inputs' side basis)."""
+    U = inp.side_basis
+    gc = K.KVCache(cfg, side_basis=U)
+    ocfg = cfg if batch is None else dict(cfg, batch=batch)
+    oc = O.OracleCache(ocfg, side_basis=None if U is None else U.cpu().numpy())
+    return gc, oc
+
+
 def run_small(w: W.Workload, num_splits=(0,), steps=None):
     """Prefill + (appends) + decodes of a workload small enough for the full oracle."""
     need_gpu()
     inp = W.Inputs(w, device="cpu")
     cfg = w.kvq_config()
-    gc = K.KVCache(cfg)
-    oc = O.OracleCache(cfg)
+    gc, oc = make_caches(cfg, inp)
     gc.prefill(inp.k.cuda(), inp.v.cuda())
     oc.prefill(np16(inp.k), np16(inp.v))
     compare_state(gc, oc, where="prefill")
@@ -237,12 +247,13 @@ def sampled_full_size(w: W.Workload, rows, steps=(0,)):
     """Full-size workload on the GPU; the oracle recomputes sampled sequences b."""
     need_gpu()
     inp = W.Inputs(w, device="cuda")
-    gc = K.KVCache(w.kvq_config())
+    gc = K.KVCache(w.kvq_config(), side_basis=inp.side_basis)
     gc.prefill(inp.k, inp.v)
+    U = None if inp.side_basis is None else inp.side_basis.cpu().numpy()
     ocs = {}
     for b in rows:
         sub = dict(w.kvq_config(), batch=1)
-        oc = O.OracleCache(sub)
+        oc = O.OracleCache(sub, side_basis=U)
         oc.prefill(np16(inp.k[b:b + 1]), np16(inp.v[b:b + 1]))
         ocs[b] = oc
     n_dec = len(inp.q)
@@ -281,3 +292,30 @@ def test_full_size_thin_16k():
 def test_full_size_sweep_point_131k(kb, vb):
     w = W.sweep_workload(8, kb, vb, appends=66)
     sampled_full_size(w, rows=(5,), steps=(0, 63, 64, 65))
+
+
+# ------------------------------------------------------- HeadQ side code ----
+@pytest.mark.parametrize("kb", [4, 2])
+@pytest.mark.parametrize("sr,sq", [(4, 4), (4, 8), (8, 4)])
+def test_side_code_tensor_kernel(kb, sr, sq):
+    """Side codes bit-exact after prefill and across appends that quantize new groups;
+    outputs of both kernels within the bound (the tensor-core kernel is built for these)."""
+    w = W.WORKLOADS["headq32k"].with_(batch=2, context=1500, k_bits=kb, side_rank=sr,
+                                      side_bits=sq, appends=70, seed=101 + sr + sq)
+    assert tensor_kernel_built(w)
+    run_small(w, num_splits=(0, 3), steps={0, 1, 57, 58, 69})
+
+
+@pytest.mark.parametrize("shape", [
+    dict(n_q_heads=8, n_kv_heads=8, d_k=128, group_k=64),     # n_rep 1
+    dict(n_q_heads=8, n_kv_heads=2, d_k=64, d_v=64, group_k=32, group_v=32),
+    dict(n_q_heads=8, n_kv_heads=2, d_k=256, d_v=128, group_k=128, k_bits=8, v_bits=4),
+])
+def test_side_code_generic_kernel_shapes(shape):
+    w = W.WORKLOADS["headq32k"].with_(batch=2, context=900, appends=2, seed=111, **shape)
+    assert not tensor_kernel_built(w)
+    run_small(w, num_splits=(0, 2))
+
+
+def test_full_size_headq_32k():
+    sampled_full_size(W.WORKLOADS["headq32k"], rows=(0, 31))
