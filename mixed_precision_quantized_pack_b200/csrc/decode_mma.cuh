@@ -55,10 +55,11 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr int kDV = 128;
-constexpr int kMaxRing = 8;
+constexpr int kMaxRing = 8;                  // stages of a CTA-wide copy ring, at most
 constexpr int kMinRing = kWarps + 1;         // fewer stages than warps would idle a warp
-constexpr float kLazyRescale = 8.0f;         // see the online-softmax update                  // stages of the CTA-wide copy ring, at most
-constexpr int kSmemPerCta = 57344;           // 228 KB per SM / 4 CTAs, minus 1 KB reserved each
+constexpr float kLazyRescale = 8.0f;         // see the online-softmax update
+constexpr int kCtasPerSm = 4;
+constexpr int kSmemPerCta = 233472 / kCtasPerSm - 1024;   // 228 KB per SM, 1 KB reserved per CTA
 
 // ---------------------------------------------------------------- geometry ----
 template <int KB, int VB, int DK, int GV>
@@ -255,33 +256,41 @@ __host__ __device__ inline StageLayout quant_stage_layout(int gk, int dk, int kb
   return s;
 }
 
-// Bytes of one stage (the larger of a key group and 16 padded fp16 rows) and the number of
-// stages that keep a CTA within a quarter of the SM's shared memory (4 CTAs per SM).
-template <int KB, int VB, int DK, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
-constexpr int stage_bytes() {
-  const int raw = Raw<DK>::BYTES;
-  const int qb = QUANT ? GK * DK * KB / 8 + DK * 4 + GK * kDV * VB / 8 + GK * (kDV / GV) * 4 +
-                             GK * Side<SR, SQ>::ZB + SR * 4
-                       : 0;
-  return ((raw > qb ? raw : qb) + 127) / 128 * 128;
+// Bytes of one stage, rounded to 128: a whole key group for the quantized splits, 16 padded
+// fp16 rows for the fp16 splits.  Each kind of split has its own ring over the same shared
+// memory, with as many stages as keep a CTA within its share of the SM (kCtasPerSm CTAs).
+template <int KB, int VB, int DK, int GV, int GK, int SR, int SQ>
+constexpr int quant_stage_bytes() {
+  return (GK * DK * KB / 8 + DK * 4 + GK * kDV * VB / 8 + GK * (kDV / GV) * 4 + GK * Side<SR, SQ>::ZB +
+          SR * 4 + 127) / 128 * 128;
 }
 
-template <int KB, int VB, int DK, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
-constexpr int ring_stages() {
-  const int r = (kSmemPerCta - Smem<DK / 16, SR>::kStages) /
-                stage_bytes<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
-  return r < kMinRing ? kMinRing : (r > kMaxRing ? kMaxRing : r);
+template <int DK>
+constexpr int raw_stage_bytes() { return (Raw<DK>::BYTES + 127) / 128 * 128; }
+
+constexpr int ring_for(int avail, int stage, int lo) {
+  return avail / stage < lo ? lo : (avail / stage > kMaxRing ? kMaxRing : avail / stage);
 }
+
+template <int KB, int VB, int DK, int GV, int GK, bool QUANT, int SR, int SQ>
+struct Rings {
+  static constexpr int HDR = Smem<DK / 16, SR>::kStages;
+  static constexpr int STAGE_Q = QUANT ? quant_stage_bytes<KB, VB, DK, GV, GK, SR, SQ>() : 128;
+  static constexpr int STAGE_F = raw_stage_bytes<DK>();
+  static constexpr int RING_Q = QUANT ? ring_for(kSmemPerCta - HDR, STAGE_Q, kMinRing) : 0;
+  static constexpr int RING_F = ring_for(kSmemPerCta - HDR, STAGE_F, kWarps);
+  static constexpr int BYTES = HDR + (RING_Q * STAGE_Q > RING_F * STAGE_F ? RING_Q * STAGE_Q
+                                                                          : RING_F * STAGE_F);
+};
 
 template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part) {
   using G = Quant<(QUANT ? KB : 4), (QUANT ? VB : 2), (QUANT ? DK : 128), (QUANT ? GV : 64)>;
   using R = Raw<DK>;
   using Z = Side<SR, SQ>;
   constexpr int KSTEPS = DK / 16;
-  constexpr int STAGE = stage_bytes<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
-  constexpr int RING = ring_stages<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
+  using RG = Rings<KB, VB, DK, GV, GK, QUANT, SR, SQ>;
   using SM = Smem<KSTEPS, SR>;
   extern __shared__ __align__(128) unsigned char smem[];
 
@@ -294,7 +303,6 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   const bool blo = (qr & 1) != 0;   // B column holds the lo half
   const bool bvalid = bhead < NREP;
   const bool cvalid = qi < NREP;   // lanes of padding columns compute values nobody reads
-  const bool quant = QUANT && split < w.splits_q;
 
   uint32_t* sm_qb = reinterpret_cast<uint32_t*>(smem + SM::kQb);
   uint32_t* sm_qf = reinterpret_cast<uint32_t*>(smem + SM::kQf);
@@ -305,8 +313,10 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   unsigned char* stages = smem + SM::kStages;
   const uint32_t stages_s = ptx::smem_addr(stages);
 
+  const bool quant = QUANT && split < w.splits_q;
+  const int ring = quant ? RG::RING_Q : RG::RING_F;     // stages of this CTA's ring
   if (threadIdx.x == 0) {
-    for (int s = 0; s < RING; ++s) {
+    for (int s = 0; s < ring; ++s) {
       ptx::mbar_init(bar0 + 8 * s, 1);
       sm_issued[s] = 0;
       sm_tag[s] = -1;
@@ -329,7 +339,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
     unit_begin = 0;
     unit_end = (list_end - list_begin + 15) / 16;
   }
-  // unit k of this CTA (k < n_units) is processed by warp k % kWarps, in stage k % RING
+  // unit k of this CTA (k < n_units) is processed by warp k % kWarps, in stage k % ring
   const int n_units = unit_end - unit_begin;
 
   // running softmax state of head qi over this warp's tokens
@@ -412,6 +422,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       const uint32_t sel_lo = swap ? 0x1054u : 0x5410u;
       const uint32_t sel_hi = swap ? 0x3276u : 0x7632u;
 
+      constexpr int RING = RG::RING_Q, STAGE = RG::STAGE_Q;
       // one lane copies unit k (a whole key group: 4 contiguous runs) into stage k % RING
       auto issue = [&](int k) {
         const int g = unit_begin + k;
@@ -661,6 +672,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
     }
   } else {
     // ---------------- fp16 rows: retained tokens, then the window ----------------
+    constexpr int RING = RG::RING_F, STAGE = RG::STAGE_F;
     uint32_t qn[KSTEPS][2];
 #pragma unroll
     for (int s = 0; s < KSTEPS; ++s)
@@ -785,7 +797,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   }
   __syncthreads();
   if (*sm_fail) {
-    if (threadIdx.x < RING && sm_issued[threadIdx.x] > 0)
+    if (threadIdx.x < ring && sm_issued[threadIdx.x] > 0)
       ptx::mbar_wait_bounded(bar0 + 8 * threadIdx.x, (sm_issued[threadIdx.x] - 1) & 1, kWaitLimitNs);
     failed = true;     // the CTA's partial is dropped as a whole
   }
@@ -857,12 +869,10 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
 template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
 cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
                    const Partials& p, cudaStream_t s) {
-  constexpr int stage = stage_bytes<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
-  constexpr int ring = ring_stages<KB, VB, DK, GV, GK, QUANT, SR, SQ>();
-  constexpr int hdr = Smem<DK / 16, SR>::kStages;
-  int smem = hdr + ring * stage;
+  using RG = Rings<KB, VB, DK, GV, GK, QUANT, SR, SQ>;
+  int smem = RG::BYTES;
   const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
-  if (hdr + merge > smem) smem = hdr + merge;
+  if (RG::HDR + merge > smem) smem = RG::HDR + merge;
   auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ>;
   static int configured = 0;
   if (configured < smem) {
