@@ -58,6 +58,18 @@ What it computes, step by step in the order the pages give it:
    gives side codes and one fp16 (scale, zero) per coordinate.  Decode adds
    (U_h^T q) . z_hat_j / sqrt(d_k), z_hat = code * s + z, to the score of every
    quantized token that is not retained; window and retained tokens are exact.
+8. Optional key-only rotation ("Quantize What Counts", §Contributions Clés and
+   §Résultats, Intégration de la Rotation: rotating the keys alone, as QuaRot
+   does, recovers most of K4V4's accuracy at K4V2).  Reading: a randomized
+   Hadamard rotation R = H_d diag(sigma) / sqrt(d) (Sylvester H_d, signs sigma
+   given by the caller), applied to every key before it is cached (prefill and
+   append) and to the query at decode, so that q'.k' = q.k.  To keep every step
+   exact but the fp16 roundings, keys are scaled by 1/c_k and queries by 1/c_q,
+   powers of two with c_k * c_q = d (c_k = 2^ceil(log2(d)/2)):
+       k' = fp16(FWHT(sigma * k) / c_k),   q' = fp16(FWHT(sigma * q) / c_q)
+   where FWHT is the Walsh-Hadamard transform in fp32 by butterflies of span
+   1, 2, 4, ..., d/2, each (x_i, x_{i+h}) -> (x_i + x_{i+h}, x_i - x_{i+h}).
+   The rotated keys are then cached exactly as unrotated ones would be.
 
 Buffer formats mirror the CUDA library's so the tests can compare bytes:
   kcode u32 [B][Hkv][Lcap][d_k*kb/32]        ksz fp16 [B][Hkv][Lcap/Gk][2*d_k] (key_meta_order)
@@ -192,6 +204,41 @@ def unpack_side(rows: np.ndarray, bits: int, r: int) -> np.ndarray:
     return ((acc[..., None] >> shifts) & np.uint64((1 << bits) - 1)).astype(np.uint32)
 
 
+def fwht32(x: np.ndarray) -> np.ndarray:
+    """Step 8: Walsh-Hadamard transform along the last axis in fp32, butterflies of span
+    1, 2, ..., d/2, each pair (i, i+h) with i & h == 0 -> (x_i + x_{i+h}, x_i - x_{i+h})."""
+    y = np.asarray(x, np.float32).copy()
+    d = y.shape[-1]
+    h = 1
+    while h < d:
+        for i in range(d):
+            if i & h == 0:
+                a = y[..., i].copy()
+                b = y[..., i + h].copy()
+                y[..., i] = a + b
+                y[..., i + h] = a - b
+        h *= 2
+    return y
+
+
+def rotation_scales(d: int):
+    """(c_k, c_q): powers of two with c_k * c_q = d, c_k = 2^ceil(log2(d)/2)."""
+    e = int(math.log2(d))
+    ck = 2 ** ((e + 1) // 2)
+    return ck, d // ck
+
+
+def sign_vector(sign_bits, d: int) -> np.ndarray:
+    """sigma_c = -1 where bit c of the little-endian words sign_bits is set, else +1."""
+    return np.array([-1.0 if (sign_bits[c // 32] >> (c % 32)) & 1 else 1.0 for c in range(d)], np.float32)
+
+
+def rotate_rows(x: np.ndarray, sigma: np.ndarray, c: int) -> np.ndarray:
+    """Step 8: fp16(FWHT(sigma * x) / c) for fp16 rows x [..., d] (sigma*x and /c are exact)."""
+    y = np.asarray(x, np.float16).astype(np.float32) * sigma
+    return (fwht32(y) / np.float32(c)).astype(np.float16)
+
+
 def quantize_keys(k: np.ndarray, group_k: int, bits: int):
     """Keys [n][d] with n a multiple of group_k -> codes [n][d], sz fp16 [n/group_k][d][2].
 
@@ -312,6 +359,10 @@ class OracleCache:
         self.cfg = dict(cfg)
         self.sr = int(cfg.get("side_rank", 0))
         self.sq = int(cfg.get("side_bits", 0))
+        self.rot = bool(cfg.get("rot_keys", 0))
+        if self.rot:
+            self.sigma = sign_vector(cfg["rot_signs"], cfg["d_k"])
+            self.ck, self.cq = rotation_scales(cfg["d_k"])
         if self.sr:
             if cfg["k_bits"] == 16 or side_basis is None:
                 raise ValueError("a side code needs quantized keys and a basis")
@@ -363,6 +414,8 @@ class OracleCache:
     def prefill(self, k: np.ndarray, v: np.ndarray):
         """k [B][Hkv][L][d_k], v [B][Hkv][L][d_v] fp16: the cache's first L tokens."""
         k = np.asarray(k, np.float16)
+        if self.rot:
+            k = rotate_rows(k, self.sigma, self.ck)
         v = np.asarray(v, np.float16)
         L = k.shape[2]
         if L > self.max_context:
@@ -386,7 +439,10 @@ class OracleCache:
         if self.L + 1 > self.max_context:
             raise ValueError("append past max_context")
         p = self.L
-        self.win_k[:, :, p % self.cap] = np.asarray(k_new, np.float16)
+        k_new = np.asarray(k_new, np.float16)
+        if self.rot:
+            k_new = rotate_rows(k_new, self.sigma, self.ck)
+        self.win_k[:, :, p % self.cap] = k_new
         self.win_v[:, :, p % self.cap] = np.asarray(v_new, np.float16)
         self.L += 1
         if self.kb != 16 and self.L - self.Q == self.R + self.gk:
@@ -460,7 +516,10 @@ class OracleCache:
         ``side_sign`` = -1 flips the side correction (the pages' wrong-sign control)."""
         if self.L == 0:
             raise ValueError("decode before prefill")
-        q = np.asarray(q, np.float16).astype(np.float64)
+        q = np.asarray(q, np.float16)
+        if self.rot:
+            q = rotate_rows(q, self.sigma, self.cq)
+        q = q.astype(np.float64)
         n_rep = self.Hq // self.H
         out = np.full((self.B, self.Hq, self.dv), np.nan)
         scale = 1.0 / math.sqrt(self.dk)

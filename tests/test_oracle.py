@@ -646,3 +646,114 @@ def test_side_code_bytes_per_token():
         cfg = dict(cfg_of(1, 1, 1, 128, 128, 2, 2, 64, 64, 128, 0, 64 * 100), side_rank=sr, side_bits=sq)
         bb = O.buffer_bytes(cfg)
         assert (bb["zcode"] + bb["zsz"]) / (64 * 100) == per_tok
+
+
+# ------------------------------------------------------ key-only rotation ----
+# "Quantize What Counts", §Contributions Clés and §Résultats (Intégration de la Rotation).
+def sylvester(d):
+    H = np.array([[1.0]])
+    while H.shape[0] < d:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def test_golden_rotation_examples():
+    for name, bits, d, k, kr, q, qr, dot in read_golden("rotation_worked.txt"):
+        d = int(d[0])
+        sigma = O.sign_vector([int(bits[0], 16)], d)
+        ck, cq = O.rotation_scales(d)
+        assert ck * cq == d
+        got_k = O.rotate_rows(np.array([[float(x) for x in k]], np.float16), sigma, ck)[0]
+        got_q = O.rotate_rows(np.array([[float(x) for x in q]], np.float16), sigma, cq)[0]
+        assert [float(x) for x in got_k] == [float(x) for x in kr], name
+        assert [float(x) for x in got_q] == [float(x) for x in qr], name
+        assert float(got_k.astype(np.float64) @ got_q.astype(np.float64)) == float(dot[0])
+
+
+@pytest.mark.parametrize("d", [2, 4, 8, 16, 32, 64, 128, 256])
+def test_fwht_is_the_sylvester_hadamard_product(d):
+    rng = np.random.default_rng(d)
+    x = rng.integers(-50, 50, size=(5, d)).astype(np.float32)     # sums stay exact in fp32
+    assert np.array_equal(O.fwht32(x).astype(np.float64), x.astype(np.float64) @ sylvester(d).T)
+    ck, cq = O.rotation_scales(d)
+    assert ck * cq == d and ck in (cq, 2 * cq)
+
+
+def test_fwht_rounding_matches_exact_rational_ieee_emulation():
+    """The butterflies on random fp16 data, each add/sub rounded by the independent emulation."""
+    d = 32
+    x = W.random_fp16((6, d), seed=121, scale=100.0).numpy().astype(np.float32)
+    x[0, 0] = 2.0 ** 24                     # force roundings that depend on the order
+    x[0, 1] = 1.0
+    x[0, 3] = -(2.0 ** 24)
+    got = O.fwht32(x)
+    for row in range(x.shape[0]):
+        y = [Fraction(float(v)) for v in x[row]]
+        h = 1
+        while h < d:
+            for i in range(d):
+                if i & h == 0:
+                    a, b = y[i], y[i + h]
+                    y[i], y[i + h] = r32(a + b), r32(a - b)
+            h *= 2
+        assert [Fraction(float(v)) for v in got[row]] == y, row
+
+
+def test_rotation_preserves_scores_up_to_the_fp16_roundings():
+    d = 128
+    k = W.random_fp16((300, d), seed=131, scale=4.0, mean=1.0).numpy()
+    q = W.random_fp16((7, d), seed=132).numpy()
+    for bits in ([0] * 4, [0x9E3779B9, 0x7F4A7C15, 0x12345678, 0xDEADBEEF]):
+        sigma = O.sign_vector(bits, d)
+        ck, cq = O.rotation_scales(d)
+        kr = O.rotate_rows(k, sigma, ck).astype(np.float64)
+        qr = O.rotate_rows(q, sigma, cq).astype(np.float64)
+        exact = q.astype(np.float64) @ k.astype(np.float64).T
+        rot = qr @ kr.T
+        # each rotated coordinate is rounded once to fp16 (2^-11 relative) and |R x| = |x|
+        bound = 2.0 ** -10 * np.linalg.norm(q.astype(np.float64), axis=1)[:, None] * \
+            np.linalg.norm(k.astype(np.float64), axis=1)[None, :] * 1.01
+        assert np.all(np.abs(rot - exact) <= bound)
+        assert np.allclose(np.linalg.norm(kr, axis=1) * ck / math.sqrt(d),
+                           np.linalg.norm(k.astype(np.float64), axis=1), rtol=2e-3)
+
+
+def rot_cfg(B, Hq, Hkv, d, kb, vb, gk, gv, R, log_retain, max_context, bits):
+    return dict(cfg_of(B, Hq, Hkv, d, d, kb, vb, gk, gv, R, log_retain, max_context),
+                rot_keys=1, rot_signs=list(bits))
+
+
+def test_rotated_unquantized_cache_matches_library_attention():
+    B, Hq, Hkv, d, L = 2, 8, 2, 64, 150
+    k = W.random_fp16((B, Hkv, L, d), seed=141, scale=3.0).numpy()
+    v = W.random_fp16((B, Hkv, L, d), seed=142).numpy()
+    q = W.random_fp16((B, Hq, d), seed=143).numpy()
+    bits = [0x0F0F1234, 0x89ABCDEF]
+    oc = O.OracleCache(rot_cfg(B, Hq, Hkv, d, 16, 16, 64, 64, 0, 0, 256, bits))
+    oc.prefill(k, v)
+    got = oc.decode(q)
+    sigma = O.sign_vector(bits, d)
+    ck, cq = O.rotation_scales(d)
+    want = sdpa_fp64(O.rotate_rows(q, sigma, cq), O.rotate_rows(k, sigma, ck), v)
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+    plain = sdpa_fp64(q, k, v)
+    assert O.max_rel_error(got, plain) < 2e-2          # the fp16 roundings of the rotation only
+
+
+def test_rotated_appends_reach_the_same_state_as_one_prefill():
+    B, Hq, Hkv, d, gk, gv, R = 2, 4, 2, 32, 16, 16, 24
+    L0, n_app = 70, 60
+    k = W.random_fp16((B, Hkv, L0 + n_app, d), seed=161, scale=4.0).numpy()
+    v = W.random_fp16((B, Hkv, L0 + n_app, d), seed=162).numpy()
+    cfg = rot_cfg(B, Hq, Hkv, d, 4, 2, gk, gv, R, 1, 256, [0xC0FFEE11])
+    a = O.OracleCache(cfg)
+    a.prefill(k[:, :, :L0], v[:, :, :L0])
+    for t in range(L0, L0 + n_app):
+        a.append(k[:, :, t], v[:, :, t])
+    b = O.OracleCache(cfg)
+    b.prefill(k, v)
+    assert (a.L, a.Q, a.ret_idx) == (b.L, b.Q, b.ret_idx)
+    for name in ("kcode", "ksz", "ret_k"):
+        assert np.array_equal(getattr(a, name).view(np.uint8), getattr(b, name).view(np.uint8)), name
+    q = W.random_fp16((B, Hq, d), seed=163).numpy()
+    assert np.array_equal(a.decode(q), b.decode(q))
