@@ -37,6 +37,16 @@
  * and decode adds (U_h^T q) . z_hat_j / sqrt(d_k), z_hat = code * s + z, to the
  * score of every quantized token that is not retained.
  *
+ * Optional key-only rotation (rot_keys = 1; "Quantize What Counts: More for Keys,
+ * Less for Values", Intégration de la Rotation): every key is rotated before it is
+ * cached and every query before it is used, by the randomized Hadamard transform
+ *   k' = fp16(FWHT(sigma * k) / c_k),   q' = fp16(FWHT(sigma * q) / c_q)
+ * with sigma_c = -1 where bit c of rot_signs is set, c_k = 2^ceil(log2(d_k)/2),
+ * c_q = d_k / c_k (so q'.k' = q.k before the fp16 roundings), and FWHT the fp32
+ * Walsh-Hadamard transform by butterflies of span 1, 2, ..., d_k/2, each
+ * (x_i, x_{i+h}) -> (x_i + x_{i+h}, x_i - x_{i+h}).  The cache then holds k'
+ * everywhere (codes, window, retained copies, side code).
+ *
  * Buffer layouts (all caller-owned device memory, 256-byte aligned recommended,
  * 16-byte aligned required; sizes from kvq_buffer_sizes):
  *   kcode  u32  [B][Hkv][Lcap][d_k*k_bits/32]   token rows, channel c at word
@@ -107,6 +117,8 @@ typedef struct kvq_config {
     int max_context;    /* capacity in tokens, >= 1 */
     int side_rank;      /* r: 0 (no side code), 4 or 8; needs quantized keys */
     int side_bits;      /* bits per side code: 4 or 8, with side_rank*side_bits 16 or 32 */
+    int rot_keys;       /* 0/1: key-only rotation */
+    unsigned int rot_signs[8];  /* rotation signs: bit c (word c/32, bit c%32) set -> -1 */
 } kvq_config;
 
 typedef struct kvq_sizes {

@@ -324,7 +324,23 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
     *sm_fail = 0;
     ptx::fence_barrier_init();
   }
-  const __half* qrow = q + (static_cast<size_t>(b) * d.Hq + h * NREP + (bvalid ? bhead : 0)) * DK;
+  // the query rows of this CTA's heads (head j at qbase + j * DK); with key rotation, their
+  // rotations, written by warp j into the stage area before the ring uses it
+  const __half* qbase = q + (static_cast<size_t>(b) * d.Hq + h * NREP) * DK;
+  if (d.rot) {
+    __half* qr_s = reinterpret_cast<__half*>(stages);
+    if (warp < NREP) {
+      float x[DK / 32];
+#pragma unroll
+      for (int m = 0; m < DK / 32; ++m) x[m] = __half2float(qbase[warp * DK + lane + 32 * m]);
+      rotate_row_warp<DK / 32>(x, DK / 32, d.rot_signs, d.rot_inv_cq, lane);
+#pragma unroll
+      for (int m = 0; m < DK / 32; ++m) qr_s[warp * DK + lane + 32 * m] = __float2half_rn(x[m]);
+    }
+    __syncthreads();
+    qbase = qr_s;
+  }
+  const __half* qrow = qbase + (bvalid ? bhead : 0) * DK;
 
   // ---------------- work list of this warp ----------------
   int unit_begin, unit_end;      // quantized: groups; fp16: tiles of 16 list entries
@@ -379,7 +395,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         // U_h^T q of head `warp`: each lane sums DK/32 channels, then the warp reduces
         float* sm_qt = reinterpret_cast<float*>(smem + SM::kQt);
         if (warp < NREP) {
-          const __half* qw = q + (static_cast<size_t>(b) * d.Hq + h * NREP + warp) * DK;
+          const __half* qw = qbase + warp * DK;
           const float* uh = cb.side_u + static_cast<size_t>(h) * DK * SR;
           float acc[SR];
 #pragma unroll
@@ -447,8 +463,10 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         }
       };
 
-      if (threadIdx.x == 0)
+      if (threadIdx.x == 0) {
+        ptx::fence_proxy_async_smem();     // the rotated query rows were written to the stages
         for (int k = 0; k < RING && k < n_units; ++k) issue(k);
+      }
 
       for (int k = warp; k < n_units; k += kWarps) {
         const int g = unit_begin + k;
@@ -681,6 +699,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         const int c = 16 * s + 2 * qi + 8 * j;
         qn[s][j] = (bvalid && !blo) ? ptx::h2_as_u32(__halves2half2(qrow[c], qrow[c + 1])) : 0u;
       }
+    if (d.rot) __syncthreads();          // every warp has read the rotated query rows
     // stale shared memory must hold finite values: masked rows multiply p = 0
     for (int i = threadIdx.x; i < RING * STAGE / 16; i += kThreads)
       reinterpret_cast<uint4*>(stages)[i] = make_uint4(0, 0, 0, 0);

@@ -34,14 +34,23 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nrep = d.n_rep, ck = d.dk / 32, cv = d.dv / 32;
 
+  // query rows (lane holds channels lane + 32 j), rotated when the keys are, times the scale
   float qr[kMaxRep][kMaxC];
 #pragma unroll
-  for (int r = 0; r < kMaxRep; ++r)
+  for (int r = 0; r < kMaxRep; ++r) {
 #pragma unroll
     for (int j = 0; j < kMaxC; ++j)
       qr[r][j] = (r < nrep && j < ck)
-                     ? __half2float(q[(static_cast<size_t>(b) * d.Hq + h * nrep + r) * d.dk + lane + 32 * j]) * w.score_scale
+                     ? __half2float(q[(static_cast<size_t>(b) * d.Hq + h * nrep + r) * d.dk + lane + 32 * j])
                      : 0.0f;
+    if (d.rot && r < nrep) {
+      rotate_row_warp<kMaxC>(qr[r], ck, d.rot_signs, d.rot_inv_cq, lane);
+#pragma unroll
+      for (int j = 0; j < kMaxC; ++j) qr[r][j] = __half2float(__float2half_rn(qr[r][j]));
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j) qr[r][j] *= w.score_scale;
+  }
   float m[kMaxRep], l[kMaxRep], o[kMaxRep][kMaxC];
 #pragma unroll
   for (int r = 0; r < kMaxRep; ++r) {
@@ -52,13 +61,19 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
   }
 
   if (d.sr) {
-    for (int idx = threadIdx.x; idx < nrep * d.sr; idx += blockDim.x) {
-      const int r = idx / d.sr, i = idx % d.sr;
-      const __half* qh = q + (static_cast<size_t>(b) * d.Hq + h * nrep + r) * d.dk;
-      const float* u = cb.side_u + static_cast<size_t>(h) * d.dk * d.sr + i;
-      float acc = 0.0f;
-      for (int c = 0; c < d.dk; ++c) acc = fmaf(u[c * d.sr], __half2float(qh[c]), acc);
-      sm_qt[r][i] = acc * w.score_scale;
+    // U_h^T q (of the rotated query, when keys are rotated), times the scale: warp 0
+    if (warp == 0) {
+      const float* u = cb.side_u + static_cast<size_t>(h) * d.dk * d.sr;
+      for (int r = 0; r < nrep; ++r)
+        for (int i = 0; i < d.sr; ++i) {
+          float acc = 0.0f;
+#pragma unroll
+          for (int j = 0; j < kMaxC; ++j)
+            if (j < ck) acc = fmaf(u[(lane + 32 * j) * d.sr + i], qr[r][j], acc);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+          if (lane == 0) sm_qt[r][i] = acc;
+        }
     }
     __syncthreads();
   }

@@ -80,6 +80,7 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
     const int row_bits = c->side_rank * c->side_bits;
     if (row_bits != 16 && row_bits != 32) return KVQ_ERR_UNSUPPORTED;
   }
+  if (c->rot_keys != 0 && c->rot_keys != 1) return KVQ_ERR_INVALID_ARG;
   // every element index must fit comfortably in 64 bits and every position in int
   const long long lcap = raw ? c->max_context
                              : (static_cast<long long>(c->max_context) + c->group_k - 1) /
@@ -107,6 +108,14 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
   x.sr = c->side_rank;
   x.sq = c->side_rank ? c->side_bits : 0;
   x.zb = c->side_rank * x.sq / 8;
+  x.rot = c->rot_keys;
+  for (int i = 0; i < 8; ++i) x.rot_signs[i] = c->rot_keys ? c->rot_signs[i] : 0u;
+  // c_k = 2^ceil(log2(d_k)/2), c_q = d_k / c_k: both powers of two, so 1/c is exact
+  int log2d = 0;
+  while ((1 << log2d) < x.dk) ++log2d;
+  const int ck = 1 << ((log2d + 1) / 2);
+  x.rot_inv_ck = 1.0f / static_cast<float>(ck);
+  x.rot_inv_cq = static_cast<float>(ck) / static_cast<float>(x.dk);
   *d = x;
   return KVQ_OK;
 }
@@ -329,20 +338,22 @@ int kvq_quantize_prefill(kvq_cache* c, const void* k, const void* v, int L, void
   if (Q > 0) {
     rc = check_cuda(kvq::launch_quantize_keys(d, kh, L, 0, Q / d.gk,
                                               static_cast<uint32_t*>(c->buf.kcode),
-                                              static_cast<__half2*>(c->buf.ksz), s));
+                                              static_cast<__half2*>(c->buf.ksz), d.rot != 0, s));
     if (!rc)
       rc = check_cuda(kvq::launch_quantize_side(
           d, kh, L, 0, Q / d.gk, static_cast<const uint32_t*>(c->buf.kcode),
           static_cast<const __half2*>(c->buf.ksz), static_cast<const float*>(c->buf.side_u),
-          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), s));
+          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), d.rot != 0, s));
     if (!rc)
       rc = check_cuda(kvq::launch_quantize_values(d, vh, L, 0, Q,
                                                   static_cast<uint32_t*>(c->buf.vcode),
                                                   static_cast<__half2*>(c->buf.vsz), s));
   }
   if (!rc)
-    rc = check_cuda(kvq::launch_copy_rows(kh, L, Q, static_cast<__half*>(c->buf.win_k), d.cap, Q,
-                                          L - Q, d.dk, nbh, s));
+    rc = check_cuda(d.rot ? kvq::launch_rotate_key_rows(d, kh, L, Q, static_cast<__half*>(c->buf.win_k),
+                                                        d.cap, Q, L - Q, nullptr, s)
+                          : kvq::launch_copy_rows(kh, L, Q, static_cast<__half*>(c->buf.win_k), d.cap,
+                                                  Q, L - Q, d.dk, nbh, s));
   if (!rc)
     rc = check_cuda(kvq::launch_copy_rows(vh, L, Q, static_cast<__half*>(c->buf.win_v), d.cap, Q,
                                           L - Q, d.dv, nbh, s));
@@ -352,8 +363,12 @@ int kvq_quantize_prefill(kvq_cache* c, const void* k, const void* v, int L, void
     kvq::RetList rl;
     rl.n = static_cast<int>(ret.size());
     for (int i = 0; i < rl.n; ++i) rl.pos[i] = ret[i];
-    rc = check_cuda(kvq::launch_copy_retained(d, kh, vh, L, rl, static_cast<__half*>(c->buf.ret_k),
+    rc = check_cuda(kvq::launch_copy_retained(d, d.rot ? nullptr : kh, vh, L, rl,
+                                              static_cast<__half*>(c->buf.ret_k),
                                               static_cast<__half*>(c->buf.ret_v), s));
+    if (!rc && d.rot)
+      rc = check_cuda(kvq::launch_rotate_key_rows(d, kh, L, 0, static_cast<__half*>(c->buf.ret_k),
+                                                  kvq::kMaxRetained, 0, rl.n, &rl, s));
   }
   if (rc) return rc;
   c->L = L;
@@ -373,22 +388,25 @@ int kvq_append(kvq_cache* c, const void* k_new, const void* v_new, void* stream)
   __half* wk = static_cast<__half*>(c->buf.win_k);
   __half* wv = static_cast<__half*>(c->buf.win_v);
   const int slot = c->L % d.cap;
-  int rc = check_cuda(kvq::launch_append_token(d, static_cast<const __half*>(k_new),
+  const __half* kn = static_cast<const __half*>(k_new);
+  int rc = check_cuda(kvq::launch_append_token(d, d.rot ? nullptr : kn,
                                                static_cast<const __half*>(v_new), wk, wv, slot, s));
+  if (!rc && d.rot) rc = check_cuda(kvq::launch_rotate_key_rows(d, kn, 1, 0, wk, d.cap, slot, 1, nullptr, s));
   if (rc) return rc;
   const int L = c->L + 1;
   int Q = c->Q;
   std::vector<int> ret = c->ret;
   if (d.quantized() && L - Q == d.R + d.gk) {
     // the oldest group_k window tokens become one key group and group_k value rows
+    // the window already holds the cached (rotated, if so configured) keys
     rc = check_cuda(kvq::launch_quantize_keys(d, wk, d.cap, Q / d.gk, 1,
                                               static_cast<uint32_t*>(c->buf.kcode),
-                                              static_cast<__half2*>(c->buf.ksz), s));
+                                              static_cast<__half2*>(c->buf.ksz), false, s));
     if (!rc)
       rc = check_cuda(kvq::launch_quantize_side(
           d, wk, d.cap, Q / d.gk, 1, static_cast<const uint32_t*>(c->buf.kcode),
           static_cast<const __half2*>(c->buf.ksz), static_cast<const float*>(c->buf.side_u),
-          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), s));
+          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), false, s));
     if (!rc)
       rc = check_cuda(kvq::launch_quantize_values(d, wv, d.cap, Q, d.gk,
                                                   static_cast<uint32_t*>(c->buf.vcode),

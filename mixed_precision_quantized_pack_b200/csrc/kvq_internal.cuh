@@ -20,8 +20,45 @@ struct Dims {
   int sr;     // side-code rank r (0: no side code)
   int sq;     // bits per side code
   int zb;     // bytes per side-code row: sr * sq / 8 (2 or 4)
+  int rot;    // key-only rotation on/off
+  unsigned int rot_signs[8];   // bit c set: sigma_c = -1
+  float rot_inv_ck, rot_inv_cq;   // 1/c_k (keys), 1/c_q (queries): powers of two
   bool quantized() const { return kb != 16; }
 };
+
+// The rotation of one key or query row of d = 32 * M channels by a warp, lane l holding
+// channels l + 32 m in x[m]: x <- FWHT(sigma * x) * inv_c in fp32, butterflies of span
+// 1, 2, ..., d/2 in that order, each (x_i, x_{i+h}) -> (x_i + x_{i+h}, x_i - x_{i+h});
+// spans below 32 pair lanes, longer spans pair registers.  (Randomized Hadamard key-only
+// rotation: "Quantize What Counts: More for Keys, Less for Values", Intégration de la
+// Rotation.)  m_count <= M is the number of valid registers (d / 32).
+template <int M>
+__device__ __forceinline__ void rotate_row_warp(float (&x)[M], int m_count, const unsigned int* signs,
+                                                float inv_c, int lane) {
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+    if (m < m_count && ((signs[m] >> lane) & 1u)) x[m] = -x[m];
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const float y = __shfl_xor_sync(0xffffffffu, x[m], h);
+      x[m] = (lane & h) ? __fsub_rn(y, x[m]) : __fadd_rn(x[m], y);
+    }
+  }
+#pragma unroll
+  for (int hm = 1; hm < M; hm <<= 1) {
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+      if ((m & hm) == 0 && (m | hm) < m_count) {
+        const float a = x[m], b = x[m | hm];
+        x[m] = __fadd_rn(a, b);
+        x[m | hm] = __fsub_rn(a, b);
+      }
+  }
+#pragma unroll
+  for (int m = 0; m < M; ++m) x[m] = __fmul_rn(x[m], inv_c);
+}
 
 // Positions of the retained tokens, ascending (kernel parameter by value).
 struct RetList {
@@ -75,19 +112,31 @@ size_t workspace_bytes(const Dims& d, int splits);
 Partials workspace_views(const Dims& d, int splits, void* ws);
 
 // ---- launchers (return the launch error, cudaSuccess when fine) ----
+// rotate: src holds unrotated keys that are rotated on the fly (prefill); otherwise src
+// already holds the cached (rotated or not) keys (the window, on append)
 cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
-                                 int n_groups, uint32_t* kcode, __half2* ksz, cudaStream_t s);
+                                 int n_groups, uint32_t* kcode, __half2* ksz, bool rotate,
+                                 cudaStream_t s);
 // Side codes of key groups [g_begin, g_begin + n_groups) whose base codes and (scale, zero)
 // are already in kcode / ksz (same stream); keys read from src as for launch_quantize_keys.
 cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows, int g_begin,
                                  int n_groups, const uint32_t* kcode, const __half2* ksz,
-                                 const float* side_u, uint8_t* zcode, __half2* zsz, cudaStream_t s);
+                                 const float* side_u, uint8_t* zcode, __half2* zsz, bool rotate,
+                                 cudaStream_t s);
 cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_rows, int t_begin,
                                    int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s);
 cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,
                              int dst_rows, int dst_base, int n, int d, int nbh, cudaStream_t s);
+// Rotated key rows (one warp per row): dst[bh][dst row i] = rotate(src[bh][src row i]) for
+// i < n, rows (src_base + i) % src_rows -> (dst_base + i) % dst_rows, or, when `list` is
+// given, rows list->pos[i] -> i.
+cudaError_t launch_rotate_key_rows(const Dims& d, const __half* src, int src_rows, int src_base,
+                                   __half* dst, int dst_rows, int dst_base, int n,
+                                   const RetList* list, cudaStream_t s);
+// k may be null: only the value row is copied
 cudaError_t launch_append_token(const Dims& d, const __half* k, const __half* v, __half* win_k,
                                 __half* win_v, int slot, cudaStream_t s);
+// k may be null: only the value rows are copied
 cudaError_t launch_copy_retained(const Dims& d, const __half* k, const __half* v, int L,
                                  const RetList& ret, __half* ret_k, __half* ret_v, cudaStream_t s);
 cudaError_t launch_update_retained(const Dims& d, const RetUpdate& up, __half* win_k,

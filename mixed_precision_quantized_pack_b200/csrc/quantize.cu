@@ -48,20 +48,48 @@ __device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g) {
 
 // One thread per (key group, channel); blockDim = (dk, groups per block).  The
 // 32/BITS lanes holding the channels of one packed word OR their codes together.
-template <int BITS>
+// ROT: the source keys are unrotated; the block's warps first rotate the rows of its
+// groups into shared memory ([groups per block][gk][dk] fp16) and the quantizer reads
+// those.
+template <int BITS, bool ROT>
 __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_rows, int dk,
                                      int gk, int g_begin, int n_groups, int lcap,
-                                     uint32_t* __restrict__ kcode, __half2* __restrict__ ksz) {
+                                     uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
+                                     Dims d) {
+  extern __shared__ __half sm_rot[];
   const int c = threadIdx.x;
   const int gi = blockIdx.x * blockDim.y + threadIdx.y;
-  if (gi >= n_groups) return;                       // uniform per warp: dk % 32 == 0
   const int bh = blockIdx.y;
-  const int g = g_begin + gi;
   const size_t base = static_cast<size_t>(bh) * src_rows;
+  if constexpr (ROT) {
+    const int tid = threadIdx.y * blockDim.x + threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x * blockDim.y / 32;
+    for (int rr = warp; rr < blockDim.y * gk; rr += nwarps) {
+      const int yy = rr / gk, t = rr % gk;
+      const int gg = blockIdx.x * blockDim.y + yy;
+      if (gg >= n_groups) continue;                  // uniform per warp
+      const int row = ((g_begin + gg) * gk + t) % src_rows;
+      float x[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) x[m] = m < dk / 32 ? __half2float(src[(base + row) * dk + lane + 32 * m]) : 0.0f;
+      rotate_row_warp<8>(x, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (m < dk / 32) sm_rot[(static_cast<size_t>(yy) * gk + t) * dk + lane + 32 * m] = __float2half_rn(x[m]);
+    }
+    __syncthreads();
+  }
+  if (gi >= n_groups) return;                       // uniform per warp: dk % 32 == 0
+  const int g = g_begin + gi;
+  // key t of the group, channel c
+  auto key = [&](int t) -> float {
+    if constexpr (ROT) return __half2float(sm_rot[(static_cast<size_t>(threadIdx.y) * gk + t) * dk + c]);
+    const int row = (g * gk + t) % src_rows;
+    return __half2float(src[(base + row) * dk + c]);
+  };
   float mn = INFINITY, mx = -INFINITY;
   for (int t = 0; t < gk; ++t) {
-    const int row = (g * gk + t) % src_rows;
-    const float x = __half2float(src[(base + row) * dk + c]);
+    const float x = key(t);
     mn = fminf(mn, x);
     mx = fmaxf(mx, x);
   }
@@ -82,8 +110,7 @@ __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_row
   constexpr int per = 32 / BITS;                    // channels per word
   const int words = dk / per;
   for (int t = 0; t < gk; ++t) {
-    const int row = (g * gk + t) % src_rows;
-    const float x = __half2float(src[(base + row) * dk + c]);
+    const float x = key(t);
     uint32_t part = quant_code<BITS>(x, gp) << ((c % per) * BITS);
 #pragma unroll
     for (int off = 1; off < per; off <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, off);
@@ -102,13 +129,13 @@ __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_row
 // One CTA per (group, b * kv head).  Shared memory: e [gk][dk + 1] (padded so that the
 // threads of a warp, which read one channel of several tokens, hit distinct banks),
 // U_h [dk][sr] and y [gk][sr].
-template <int SQ>
+template <int SQ, bool ROT>
 __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_rows, int dk, int kb,
                                      int gk, int g_begin, int lcap, int hkv, int sr, int zb,
                                      const uint32_t* __restrict__ kcode,
                                      const __half2* __restrict__ ksz,
                                      const float* __restrict__ side_u,
-                                     uint8_t* __restrict__ zcode, __half2* __restrict__ zsz) {
+                                     uint8_t* __restrict__ zcode, __half2* __restrict__ zsz, Dims d) {
   extern __shared__ float sm_side[];
   __shared__ float2 params[8];
   const int es = dk + 1;
@@ -123,10 +150,31 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
   const int quarter = words % 4 == 0 ? words / 4 : 0;
   const __half* blk =
       reinterpret_cast<const __half*>(ksz) + (static_cast<size_t>(bh) * (lcap / gk) + g) * 2 * dk;
+  // the cached key of token t, channel c: the source key, or its rotation (ROT: rotated
+  // by warps into e, then read back from there)
+  if constexpr (ROT) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x / 32;
+    for (int t = warp; t < gk; t += nwarps) {
+      const int row = (g * gk + t) % src_rows;
+      float x[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) x[m] = m < dk / 32 ? __half2float(src[(base + row) * dk + lane + 32 * m]) : 0.0f;
+      rotate_row_warp<8>(x, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (m < dk / 32) e[t * es + lane + 32 * m] = __half2float(__float2half_rn(x[m]));
+    }
+    __syncthreads();
+  }
   for (int idx = threadIdx.x; idx < gk * dk; idx += blockDim.x) {
     const int t = idx / dk, c = idx % dk;
-    const int row = (g * gk + t) % src_rows;
-    const float x = __half2float(src[(base + row) * dk + c]);
+    float x;
+    if constexpr (ROT) {
+      x = e[t * es + c];
+    } else {
+      const int row = (g * gk + t) % src_rows;
+      x = __half2float(src[(base + row) * dk + c]);
+    }
     const uint32_t w = kcode[(static_cast<size_t>(bh) * lcap + g * gk + t) * words + c / per];
     const uint32_t code = (w >> ((c % per) * kb)) & ((1u << kb) - 1u);
     // the channel's (scale, zero) slots in the group's paired, quarter-interleaved block
@@ -254,12 +302,39 @@ __global__ void append_token_kernel(const __half* __restrict__ k, const __half* 
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
     const int bh = idx / (vk + vv), e = idx % (vk + vv);
     if (e < vk) {
-      reinterpret_cast<uint4*>(win_k + (static_cast<size_t>(bh) * cap + slot) * dk)[e] =
-          reinterpret_cast<const uint4*>(k + static_cast<size_t>(bh) * dk)[e];
+      if (k)
+        reinterpret_cast<uint4*>(win_k + (static_cast<size_t>(bh) * cap + slot) * dk)[e] =
+            reinterpret_cast<const uint4*>(k + static_cast<size_t>(bh) * dk)[e];
     } else {
       reinterpret_cast<uint4*>(win_v + (static_cast<size_t>(bh) * cap + slot) * dv)[e - vk] =
           reinterpret_cast<const uint4*>(v + static_cast<size_t>(bh) * dv)[e - vk];
     }
+  }
+}
+
+// Rotated key rows, one warp per (b * kv head, row i < n): source row (src_base + i) %
+// src_rows, or list->pos[i], into destination row (dst_base + i) % dst_rows.
+__global__ void rotate_key_rows_kernel(const __half* __restrict__ src, int src_rows, int src_base,
+                                       __half* __restrict__ dst, int dst_rows, int dst_base, int n,
+                                       int nbh, RetList list, int use_list, Dims d) {
+  const int lane = threadIdx.x & 31;
+  const long long total = static_cast<long long>(nbh) * n;
+  const int dk = d.dk;
+  for (long long r = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) / 32; r < total;
+       r += static_cast<long long>(gridDim.x) * blockDim.x / 32) {
+    const int i = static_cast<int>(r % n);
+    const int bh = static_cast<int>(r / n);
+    const int sr = use_list ? list.pos[i] : (src_base + i) % src_rows;
+    const int dr = (dst_base + i) % dst_rows;
+    const __half* s = src + (static_cast<size_t>(bh) * src_rows + sr) * dk;
+    __half* t = dst + (static_cast<size_t>(bh) * dst_rows + dr) * dk;
+    float x[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) x[m] = m < dk / 32 ? __half2float(s[lane + 32 * m]) : 0.0f;
+    rotate_row_warp<8>(x, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
+#pragma unroll
+    for (int m = 0; m < 8; ++m)
+      if (m < dk / 32) t[lane + 32 * m] = __float2half_rn(x[m]);
   }
 }
 
@@ -271,8 +346,9 @@ __global__ void copy_retained_kernel(const __half* __restrict__ k, const __half*
   for (int j = 0; j < ret.n; ++j) {
     const size_t src = static_cast<size_t>(bh) * L + ret.pos[j];
     const size_t dst = static_cast<size_t>(bh) * kMaxRetained + j;
-    for (int c = threadIdx.x; c < dk / 8; c += blockDim.x)
-      reinterpret_cast<uint4*>(ret_k + dst * dk)[c] = reinterpret_cast<const uint4*>(k + src * dk)[c];
+    if (k)
+      for (int c = threadIdx.x; c < dk / 8; c += blockDim.x)
+        reinterpret_cast<uint4*>(ret_k + dst * dk)[c] = reinterpret_cast<const uint4*>(k + src * dk)[c];
     for (int c = threadIdx.x; c < dv / 8; c += blockDim.x)
       reinterpret_cast<uint4*>(ret_v + dst * dv)[c] = reinterpret_cast<const uint4*>(v + src * dv)[c];
   }
@@ -318,28 +394,55 @@ inline int grid_for(long long items, int block) {
 
 }  // namespace
 
-cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
-                                 int n_groups, uint32_t* kcode, __half2* ksz, cudaStream_t s) {
-  if (n_groups <= 0) return cudaSuccess;
+template <bool ROT>
+cudaError_t launch_quantize_keys_t(const Dims& d, const __half* src, int src_rows, int g_begin,
+                                   int n_groups, uint32_t* kcode, __half2* ksz, cudaStream_t s) {
   const int gpb = d.dk >= 256 ? 1 : 256 / d.dk;
   dim3 block(d.dk, gpb);
   dim3 grid((n_groups + gpb - 1) / gpb, d.B * d.Hkv);
-  switch (d.kb) {
-    case 2: quantize_keys_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz); break;
-    case 4: quantize_keys_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz); break;
-    case 8: quantize_keys_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz); break;
-    default: return cudaErrorInvalidValue;
+  const size_t smem = ROT ? static_cast<size_t>(gpb) * d.gk * d.dk * 2 : 0;
+  auto kern = d.kb == 2 ? quantize_keys_kernel<2, ROT>
+            : d.kb == 4 ? quantize_keys_kernel<4, ROT> : quantize_keys_kernel<8, ROT>;
+  if (d.kb != 2 && d.kb != 4 && d.kb != 8) return cudaErrorInvalidValue;
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
   }
+  kern<<<grid, block, smem, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
+                                 int n_groups, uint32_t* kcode, __half2* ksz, bool rotate,
+                                 cudaStream_t s) {
+  if (n_groups <= 0) return cudaSuccess;
+  return rotate ? launch_quantize_keys_t<true>(d, src, src_rows, g_begin, n_groups, kcode, ksz, s)
+                : launch_quantize_keys_t<false>(d, src, src_rows, g_begin, n_groups, kcode, ksz, s);
+}
+
+cudaError_t launch_rotate_key_rows(const Dims& d, const __half* src, int src_rows, int src_base,
+                                   __half* dst, int dst_rows, int dst_base, int n,
+                                   const RetList* list, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int nbh = d.B * d.Hkv;
+  const long long warps = static_cast<long long>(nbh) * n;
+  RetList empty;
+  empty.n = 0;
+  rotate_key_rows_kernel<<<grid_for(warps * 32, 256), 256, 0, s>>>(
+      src, src_rows, src_base, dst, dst_rows, dst_base, n, nbh, list ? *list : empty, list ? 1 : 0, d);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows, int g_begin,
                                  int n_groups, const uint32_t* kcode, const __half2* ksz,
-                                 const float* side_u, uint8_t* zcode, __half2* zsz, cudaStream_t s) {
+                                 const float* side_u, uint8_t* zcode, __half2* zsz, bool rotate,
+                                 cudaStream_t s) {
   if (n_groups <= 0 || d.sr == 0) return cudaSuccess;
   const size_t smem = (static_cast<size_t>(d.gk) * (d.dk + 1) + d.dk * d.sr + d.gk * d.sr) * 4;
   dim3 grid(n_groups, d.B * d.Hkv);
-  auto kern = d.sq == 4 ? quantize_side_kernel<4> : quantize_side_kernel<8>;
+  auto kern = d.sq == 4 ? (rotate ? quantize_side_kernel<4, true> : quantize_side_kernel<4, false>)
+                        : (rotate ? quantize_side_kernel<8, true> : quantize_side_kernel<8, false>);
   if (d.sq != 4 && d.sq != 8) return cudaErrorInvalidValue;
   if (smem > 48 * 1024) {
     const cudaError_t e =
@@ -347,7 +450,7 @@ cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows,
     if (e != cudaSuccess) return e;
   }
   kern<<<grid, 256, smem, s>>>(src, src_rows, d.dk, d.kb, d.gk, g_begin, d.lcap, d.Hkv, d.sr, d.zb,
-                               kcode, ksz, side_u, zcode, zsz);
+                               kcode, ksz, side_u, zcode, zsz, d);
   return cudaGetLastError();
 }
 

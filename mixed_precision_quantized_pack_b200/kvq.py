@@ -33,15 +33,16 @@ KVQ_STATUS_TIMEOUT = 1
 KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 CONFIG_FIELDS = ("batch", "n_q_heads", "n_kv_heads", "d_k", "d_v", "k_bits", "v_bits", "group_k",
-                 "group_v", "window", "log_retain", "max_context", "side_rank", "side_bits")
-OPTIONAL_CONFIG = ("side_rank", "side_bits")          # default 0: no side code
+                 "group_v", "window", "log_retain", "max_context", "side_rank", "side_bits",
+                 "rot_keys")
+OPTIONAL_CONFIG = ("side_rank", "side_bits", "rot_keys")   # default 0: no side code, no rotation
 BUFFER_FIELDS = ("kcode", "ksz", "vcode", "vsz", "win_k", "win_v", "ret_k", "ret_v")
 SIDE_FIELDS = ("zcode", "zsz", "side_u")
 SIZE_FIELDS = BUFFER_FIELDS + ("workspace",) + SIDE_FIELDS
 
 
 class kvq_config(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in CONFIG_FIELDS]
+    _fields_ = [(n, ctypes.c_int) for n in CONFIG_FIELDS] + [("rot_signs", ctypes.c_uint * 8)]
 
 
 class kvq_sizes(ctypes.Structure):
@@ -120,7 +121,11 @@ def _stream(stream=None) -> int:
 
 
 def make_config(cfg: Dict[str, int]) -> kvq_config:
-    return kvq_config(*[int(cfg.get(n, 0) if n in OPTIONAL_CONFIG else cfg[n]) for n in CONFIG_FIELDS])
+    """cfg: the kvq_config fields by name; "rot_signs" is a list of up to 8 uint32 words."""
+    c = kvq_config(*[int(cfg.get(n, 0) if n in OPTIONAL_CONFIG else cfg[n]) for n in CONFIG_FIELDS])
+    for i, word in enumerate(list(cfg.get("rot_signs", ()))[:8]):
+        c.rot_signs[i] = int(word) & 0xFFFFFFFF
+    return c
 
 
 # ---- the C entry points, same names -----------------------------------------

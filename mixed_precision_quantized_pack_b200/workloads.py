@@ -56,6 +56,8 @@ class Workload:
     side_rank: int = 0    # >0: a side code of this rank ...
     side_bits: int = 0    # ... and bits per code
     q_in_basis: float = 0.0   # side workloads: fraction of query energy in span(U_h)
+    rot_keys: int = 0     # key-only rotation, with signs drawn from rot_seed
+    rot_seed: int = 0
 
     @property
     def n_rep(self) -> int:
@@ -74,7 +76,15 @@ class Workload:
                     group_k=self.group_k, group_v=self.group_v, window=self.window,
                     log_retain=self.log_retain,
                     max_context=max_context if max_context is not None else self.max_context,
-                    side_rank=self.side_rank, side_bits=self.side_bits)
+                    side_rank=self.side_rank, side_bits=self.side_bits, rot_keys=self.rot_keys,
+                    rot_signs=rotation_signs(self.rot_seed) if self.rot_keys else [0] * 8)
+
+
+def rotation_signs(seed: int) -> List[int]:
+    """Eight random 32-bit words (the rotation's sign bits), from their own seeded generator."""
+    gen = torch.Generator()
+    gen.manual_seed(seed)
+    return [int(x) for x in torch.randint(0, 2 ** 32, (8,), generator=gen, dtype=torch.int64)]
 
 
 def _base(**kw) -> Workload:
@@ -103,6 +113,10 @@ WORKLOADS: Dict[str, Workload] = {
                       n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=2, v_bits=2,
                       group_k=64, group_v=64, window=128, log_retain=1, appends=0, seed=1005,
                       side_rank=4, side_bits=4, q_in_basis=0.9),
+    # the 32k case with the keys rotated ("Quantize What Counts", rotation of the keys only)
+    "rot32k": _base(name="rot-b32-32/8-32k-k4v2-logretain", batch=32, n_q_heads=32, n_kv_heads=8,
+                    d_k=128, d_v=128, context=32768, k_bits=4, v_bits=2, group_k=64, group_v=64,
+                    window=128, log_retain=1, appends=0, seed=1006, rot_keys=1, rot_seed=77),
 }
 
 SWEEP_BATCHES = (1, 8, 32, 64)

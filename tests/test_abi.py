@@ -67,6 +67,7 @@ def test_retention_rule_matches_the_oracle():
     (dict(window=-1), K.KVQ_ERR_INVALID_ARG),
     (dict(log_retain=2), K.KVQ_ERR_INVALID_ARG),
     (dict(max_context=0), K.KVQ_ERR_INVALID_ARG),
+    (dict(rot_keys=2), K.KVQ_ERR_INVALID_ARG),
 ])
 def test_invalid_configurations_are_rejected(bad, code):
     with pytest.raises(K.KVQError) as e:

@@ -319,3 +319,36 @@ def test_side_code_generic_kernel_shapes(shape):
 
 def test_full_size_headq_32k():
     sampled_full_size(W.WORKLOADS["headq32k"], rows=(0, 31))
+
+
+# ------------------------------------------------------ key-only rotation ----
+@pytest.mark.parametrize("kb,vb", [(4, 2), (2, 2), (8, 4)])
+def test_rotation_tensor_kernel(kb, vb):
+    """Rotated keys: codes, window and retained copies bit-exact across appends; outputs of
+    both kernels within the bound."""
+    w = W.WORKLOADS["rot32k"].with_(batch=2, context=1500, k_bits=kb, v_bits=vb, appends=70,
+                                    seed=171 + kb)
+    assert tensor_kernel_built(w)
+    run_small(w, num_splits=(0, 3), steps={0, 1, 57, 58, 69})
+
+
+def test_rotation_with_side_code():
+    w = W.WORKLOADS["headq32k"].with_(batch=2, context=1200, appends=66, rot_keys=1, rot_seed=5,
+                                      seed=181)
+    run_small(w, num_splits=(0, 2), steps={0, 63, 64, 65})
+
+
+@pytest.mark.parametrize("dk,dv", [(32, 128), (64, 64), (256, 128)])
+def test_rotation_head_dims(dk, dv):
+    w = W.WORKLOADS["rot32k"].with_(batch=1, n_q_heads=8, n_kv_heads=2, d_k=dk, d_v=dv, context=900,
+                                    group_k=32, group_v=32, window=64, appends=34, seed=191)
+    run_small(w, num_splits=(0, 2), steps={0, 33})
+
+
+def test_rotation_unquantized_cache():
+    w = W.WORKLOADS["rot32k"].with_(batch=2, context=700, k_bits=16, v_bits=16, appends=3, seed=201)
+    run_small(w, num_splits=(0, 3))
+
+
+def test_full_size_rot_32k():
+    sampled_full_size(W.WORKLOADS["rot32k"], rows=(0, 31))
