@@ -34,7 +34,9 @@ from mixed_precision_quantized_pack_b200 import workloads as W  # noqa: E402
 
 METRIC = "decode attn tokens/s and achieved HBM GB/s over packed KV (K4V2, ctx 32k)"
 UNIT = "tokens/s"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_long32k_ncu.md")
+def profile_summary(workload_key: str) -> str:
+    """The committed ncu summary of the decode kernel on a workload."""
+    return os.path.join(ROOT, "profiles", f"decode_{workload_key}_ncu.md")
 
 
 def peaks():
@@ -127,11 +129,11 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
 
 
-def profile_traffic():
-    """dram bytes per decode launch from the committed ncu summary, if it was taken on the
-    current kernel source (else None)."""
+def profile_traffic(workload_key: str):
+    """dram bytes per decode launch from the committed ncu summary of the workload, if it was
+    taken on the current kernel source (else None)."""
     try:
-        text = open(PROFILE_SUMMARY).read()
+        text = open(profile_summary(workload_key)).read()
     except OSError:
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
@@ -282,9 +284,11 @@ def main():
         cache.decode(inp.q[i], out=out)
         ends[i].record(stream)
         if timed:
-            launches += 2 + 2          # window writes (K, V) + decode + combine
-            if q1 != q0:
-                launches += 2 + (1 if cfg["log_retain"] else 0)
+            # append (one copy kernel for K and V; rotated keys take a second one), then the
+            # decode and the combine
+            launches += (2 if cfg.get("rot_keys") else 1) + 2
+            if q1 != q0:     # a window group was quantized: keys, values, side code, retained set
+                launches += 2 + (1 if cfg.get("side_rank") else 0) + (1 if cfg["log_retain"] else 0)
             bytes_read.append(decode_bytes(cfg, L))
 
     for i in range(warm):
@@ -317,43 +321,67 @@ def main():
     achieved = (sum(bytes_read) / len(bytes_read)) / (dec_avg / 1e3) / 1e9
     peak, peak_kind = peaks()
 
-    # end to end through the public API: pinned host inputs in, host output back, per step
+    # end to end through the public API: every step copies its inputs from pinned host memory
+    # and its output back to pinned host memory.  The copies run on two copy streams with
+    # double-buffered device tensors, so step i's input copy overlaps step i-1's decode and
+    # step i's output copy overlaps step i+1's; every copy still lies inside the timed region.
     h_q = [x.cpu().pin_memory() for x in inp.q[:steps]]
     h_k = [x.cpu().pin_memory() for x in inp.k_app[:steps]]
     h_v = [x.cpu().pin_memory() for x in inp.v_app[:steps]]
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    d_q = torch.empty_like(inp.q[0])
-    d_k = torch.empty_like(inp.k_app[0])
-    d_v = torch.empty_like(inp.v_app[0])
+    h_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    d_q = [torch.empty_like(inp.q[0]) for _ in range(2)]
+    d_k = [torch.empty_like(inp.k_app[0]) for _ in range(2)]
+    d_v = [torch.empty_like(inp.v_app[0]) for _ in range(2)]
+    d_out = [torch.empty_like(out) for _ in range(2)]
     inp2 = W.Inputs(wl.with_(appends=1), device=dev)
     e2e_cache = K.KVCache(cfg, device=dev, side_basis=inp2.side_basis)
     e2e_cache.prefill(inp2.k, inp2.v)
     del inp2
     torch.cuda.empty_cache()
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]       # inputs of the slot uploaded
+    ev_used = [torch.cuda.Event() for _ in range(2)]     # decode done with the slot
+    ev_down = [torch.cuda.Event() for _ in range(2)]     # output of the slot downloaded
+    for e in ev_used + ev_down:
+        e.record(stream)
+
+    def e2e_step(i):
+        j = i % 2
+        s_in.wait_event(ev_used[j])
+        with torch.cuda.stream(s_in):
+            d_q[j].copy_(h_q[i], non_blocking=True)
+            d_k[j].copy_(h_k[i], non_blocking=True)
+            d_v[j].copy_(h_v[i], non_blocking=True)
+        ev_in[j].record(s_in)
+        stream.wait_event(ev_in[j])
+        stream.wait_event(ev_down[j])
+        e2e_cache.append(d_k[j], d_v[j])
+        e2e_cache.decode(d_q[j], out=d_out[j])
+        ev_used[j].record(stream)
+        s_out.wait_event(ev_used[j])
+        with torch.cuda.stream(s_out):
+            h_out[j].copy_(d_out[j], non_blocking=True)
+        ev_down[j].record(s_out)
+
     for i in range(3):
-        d_q.copy_(h_q[i], non_blocking=True)
-        d_k.copy_(h_k[i], non_blocking=True)
-        d_v.copy_(h_v[i], non_blocking=True)
-        e2e_cache.append(d_k, d_v)
-        e2e_cache.decode(d_q, out=out)
-        h_out.copy_(out, non_blocking=True)
+        e2e_step(i)
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = min(steps, len(h_q)) - 3
     a.record(stream)
+    s_in.wait_event(a)
+    s_out.wait_event(a)
     for i in range(3, 3 + n_e2e):
-        d_q.copy_(h_q[i], non_blocking=True)
-        d_k.copy_(h_k[i], non_blocking=True)
-        d_v.copy_(h_v[i], non_blocking=True)
-        e2e_cache.append(d_k, d_v)
-        e2e_cache.decode(d_q, out=out)
-        h_out.copy_(out, non_blocking=True)
+        e2e_step(i)
+    for e in ev_down:
+        stream.wait_event(e)
     b.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = a.elapsed_time(b) / max(n_e2e, 1)
     (e2e_ms,) = max_over_ranks([e2e_ms], dist, dev)
+    d_q, d_k, d_v = d_q[0], d_k[0], d_v[0]
     h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
     d2h = out.numel() * 2
 
@@ -380,7 +408,8 @@ def main():
                        "step": "append 1 token + decode, per sequence",
                        "plan": plan},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": profile_traffic(),
+                         "frac": achieved / peak,
+                         "traffic": None if args.batch else profile_traffic(args.workload),
                          "peak_kind": f"{peak_kind} HBM copy bandwidth",
                          "kernel": "decode (split-K kernel + combine), CUDA events per launch",
                          "decode_ms": dec_avg, "bytes_per_launch": bytes_read[0]},
@@ -388,7 +417,9 @@ def main():
             "prefill_ms": prefill_ms,
             "cpu_baseline": cpu,
             "e2e": {"value": world * wl.batch / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "copies": "pinned host <-> device every step, on two copy streams that "
+                              "overlap the neighbouring steps' decodes"},
             "gpu_launches": launches,
             "clocks": clk,
             "device_status": status,
