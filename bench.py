@@ -21,7 +21,6 @@ import os
 import re
 import statistics
 import sys
-import threading
 import time
 
 import torch
@@ -64,69 +63,79 @@ def decode_bytes(cfg: dict, L: int) -> int:
     return B * H * (quant + fp16) + B * cfg["n_q_heads"] * dk * 2
 
 
-class ClockSampler:
-    """SM clock and clock-event (throttle) reasons polled through NVML every ~1 ms
-    during the timed region (read-only queries)."""
+CLOCK_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
-               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+def _clock_sampler_main(uuid, index, conn, stop):
+    """Child process: poll the SM clock and the clock-event reasons every 0.5 ms (read-only
+    NVML queries) until `stop` is set, then send [(monotonic time, MHz, reasons)] and the
+    maximum SM clock back through `conn`."""
+    samples, max_mhz = [], None
+    try:
+        import pynvml as nv
+        nv.nvmlInit()
+        try:
+            h = nv.nvmlDeviceGetHandleByUUID(uuid)
+        except Exception:
+            h = nv.nvmlDeviceGetHandleByIndex(index)
+        max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        conn.send("ready")
+        while not stop.is_set():
+            samples.append((time.monotonic(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                            get_reasons(h) if get_reasons else 0))
+            time.sleep(0.0005)
+    except Exception:
+        conn.send("ready")
+    conn.send((samples, max_mhz))
+
+
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons sampled by a separate process (so that it
+    never competes with the launching thread for the interpreter) every ~0.5 ms; the samples
+    kept are those taken between mark_start() and mark_end(), the host-side window in which
+    the GPU ran the timed steps."""
 
     def __init__(self, device_index: int):
-        self.dev = device_index
-        self.samples = []
-        self.stop_flag = threading.Event()
-        self.thread = None
-        self.max_mhz = None
-
-    def _handle(self, nv):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
         try:
-            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
-            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:
-            return nv.nvmlDeviceGetHandleByIndex(self.dev)
+            uuid = ""
+        self.conn, child = ctx.Pipe()
+        self.stop_evt = ctx.Event()
+        self.proc = ctx.Process(target=_clock_sampler_main,
+                                args=(uuid, device_index, child, self.stop_evt), daemon=True)
+        self.proc.start()
+        self.ready = self.conn.poll(60) and self.conn.recv() == "ready"
+        self.t_start = self.t_end = None
 
-    def start(self):
-        try:
-            import pynvml as nv
-            nv.nvmlInit()
-            h = self._handle(nv)
-            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
-                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
-        except Exception:
-            return
+    def mark_start(self):
+        self.t_start = time.monotonic()
 
-        def loop():
-            while not self.stop_flag.is_set():
-                try:
-                    self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
-                                         get_reasons(h) if get_reasons else 0))
-                except Exception:
-                    return
-                time.sleep(0.0005)
-
-        # the launching thread holds the GIL between its calls: switch often so the
-        # sampler gets to run during a short timed region
-        self.old_switch = sys.getswitchinterval()
-        sys.setswitchinterval(0.0002)
-        self.thread = threading.Thread(target=loop, daemon=True)
-        self.thread.start()
+    def mark_end(self):
+        self.t_end = time.monotonic()
 
     def stop(self):
-        if self.thread is None:
-            return None
-        self.stop_flag.set()
-        self.thread.join(timeout=2)
-        sys.setswitchinterval(self.old_switch)
-        if not self.samples:
+        self.stop_evt.set()
+        samples, max_mhz = self.conn.recv() if self.conn.poll(10) else ([], None)
+        self.proc.join(timeout=5)
+        if self.t_start is not None and self.t_end is not None:
+            samples = [x for x in samples if self.t_start <= x[0] <= self.t_end]
+        if not samples:
             return None
         reasons = set()
-        for _, r in self.samples:
-            for bit, name in self.REASONS.items():
+        for _, _, r in samples:
+            for bit, name in CLOCK_REASONS.items():
                 if r & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
+        return {"sm_mhz": statistics.median(m for _, m, _ in samples), "sm_max_mhz": max_mhz,
+                "reasons": sorted(reasons), "samples": len(samples),
+                "source": "nvml, separate process"}
 
 
 def profile_traffic(workload_key: str):
@@ -275,11 +284,17 @@ def main():
     launches = 0
     bytes_read = []
 
+    L0, _, _ = cache.state()
+    gk, R = cfg["group_k"], cfg["window"]
+
+    def q_of(L):          # quantized prefix after L tokens (the window rule of the cache)
+        return 0 if cfg["k_bits"] == 16 else max(L - R, 0) // gk * gk
+
     def step(i, timed):
         nonlocal launches
-        _, q0, _ = cache.state()
+        L = L0 + i + 1
+        q0, q1 = q_of(L - 1), q_of(L)
         cache.append(inp.k_app[i], inp.v_app[i])
-        L, q1, _ = cache.state()
         starts[i].record(stream)
         cache.decode(inp.q[i], out=out)
         ends[i].record(stream)
@@ -297,16 +312,15 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
+    clocks.mark_start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(warm, warm + steps):
         step(i, True)
     t1.record(stream)
-    # wait for the GPU without holding the interpreter lock, so that the clock sampler
-    # keeps polling while the timed steps run
     while not t1.query():
         time.sleep(0.0002)
+    clocks.mark_end()
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
