@@ -639,6 +639,19 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
             // value words: tokens 2qi, 2qi+1, 2qi+8, 2qi+9 of the tile, swapped for qi >= 2
             const int ta = 16 * mt + 2 * qi + (swap ? 1 : 0);
             const int tb = 16 * mt + 2 * qi + (swap ? 0 : 1);
+            // 16-bit runs (a value group's row is 16 bytes): ldmatrix.trans over the rows of
+            // tokens 0-7 and 8-15 of the tile hands lane (qr, qi) the pair (token 2qi, token
+            // 2qi+1) of 16-bit column qr, i.e. exactly its run of both tokens in one register
+            constexpr bool kLdm = G::RUN == 16 && GV * VB / 8 == 16 && G::NVG % 2 == 0;
+            uint32_t xv[G::NVG][2];
+            if constexpr (kLdm) {
+              const int j = lane >> 3, r = lane & 7;
+#pragma unroll
+              for (int g4 = 0; g4 < G::NVG; g4 += 2)
+                ptx::ldmatrix_x4_trans(ptx::smem_addr(svc) + (16 * mt + 8 * (j & 1) + r) * G::VBYTES_ROW +
+                                           (g4 + (j >> 1)) * 16,
+                                       xv[g4][0], xv[g4][1], xv[g4 + 1][0], xv[g4 + 1][1]);
+            }
 #pragma unroll
             for (int gg = 0; gg < G::NVG; ++gg) {
               const float2 f0 = __half22float2(ptx::u32_as_h2(vm0[gg]));
@@ -652,25 +665,31 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
               const int bit0 = (gg * GV + qr * G::CPG) * VB;
               const int wv = bit0 >> 5;
               const int ob = bit0 & 31;
-              const uint32_t wa0 = svc[ta * G::VW + wv], wb0 = svc[tb * G::VW + wv];
-              const uint32_t wa1 = svc[(ta + 8) * G::VW + wv], wb1 = svc[(tb + 8) * G::VW + wv];
               uint32_t ra[G::CPG], rb[G::CPG];   // codes of tokens (2qi, 2qi+1) and (2qi+8, 2qi+9)
-              if constexpr (G::RUN == 8) {
-                const uint32_t bsel = static_cast<uint32_t>(ob >> 3);
-                const uint32_t s8 = swap ? ((4 + bsel) | ((4 + bsel) << 4) | (bsel << 8) | (bsel << 12))
-                                         : (bsel | (bsel << 4) | ((4 + bsel) << 8) | ((4 + bsel) << 12));
-                unpack_value_piece8<VB>(ptx::prmt(wa0, wb0, s8), ra);
-                unpack_value_piece8<VB>(ptx::prmt(wa1, wb1, s8), rb);
-              } else if constexpr (G::RUN == 16) {
-                const uint32_t s16 = ob ? sel_hi : sel_lo;
-                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, s16), ra);
-                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, s16), rb);
+              if constexpr (kLdm) {
+                unpack_value_piece16<VB>(xv[gg][0], ra);
+                unpack_value_piece16<VB>(xv[gg][1], rb);
               } else {
-                constexpr int n16 = 16 / VB;
-                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_lo), ra);
-                unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_hi), ra + n16);
-                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_lo), rb);
-                unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_hi), rb + n16);
+                // other run widths: four word loads and a byte permute per pair of tokens
+                const uint32_t wa0 = svc[ta * G::VW + wv], wb0 = svc[tb * G::VW + wv];
+                const uint32_t wa1 = svc[(ta + 8) * G::VW + wv], wb1 = svc[(tb + 8) * G::VW + wv];
+                if constexpr (G::RUN == 8) {
+                  const uint32_t bsel = static_cast<uint32_t>(ob >> 3);
+                  const uint32_t s8 = swap ? ((4 + bsel) | ((4 + bsel) << 4) | (bsel << 8) | (bsel << 12))
+                                           : (bsel | (bsel << 4) | ((4 + bsel) << 8) | ((4 + bsel) << 12));
+                  unpack_value_piece8<VB>(ptx::prmt(wa0, wb0, s8), ra);
+                  unpack_value_piece8<VB>(ptx::prmt(wa1, wb1, s8), rb);
+                } else if constexpr (G::RUN == 16) {
+                  const uint32_t s16 = ob ? sel_hi : sel_lo;
+                  unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, s16), ra);
+                  unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, s16), rb);
+                } else {
+                  constexpr int n16 = 16 / VB;
+                  unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_lo), ra);
+                  unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_hi), ra + n16);
+                  unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_lo), rb);
+                  unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_hi), rb + n16);
+                }
               }
 #pragma unroll
               for (int ml = 0; ml < G::MPG; ++ml)
