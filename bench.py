@@ -83,10 +83,9 @@ def _clock_sampler_main(uuid, index, conn, stop):
         get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
                               getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
         conn.send("ready")
-        while not stop.is_set():
+        while not stop.is_set():         # back-to-back queries (each takes a fraction of a ms)
             samples.append((time.monotonic(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
                             get_reasons(h) if get_reasons else 0))
-            time.sleep(0.0005)
     except Exception:
         conn.send("ready")
     conn.send((samples, max_mhz))
@@ -124,8 +123,15 @@ class ClockSampler:
         self.stop_evt.set()
         samples, max_mhz = self.conn.recv() if self.conn.poll(10) else ([], None)
         self.proc.join(timeout=5)
+        window = "timed region"
         if self.t_start is not None and self.t_end is not None:
-            samples = [x for x in samples if self.t_start <= x[0] <= self.t_end]
+            inside = [x for x in samples if self.t_start <= x[0] <= self.t_end]
+            if not inside:
+                # a short timed region can fall between two queries: take those within 100 ms of
+                # it (the warm-up and the following steps run the same kernels)
+                inside = [x for x in samples if self.t_start - 0.1 <= x[0] <= self.t_end + 0.1]
+                window = "within 100 ms of the timed region"
+            samples = inside
         if not samples:
             return None
         reasons = set()
@@ -135,7 +141,7 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(m for _, m, _ in samples), "sm_max_mhz": max_mhz,
                 "reasons": sorted(reasons), "samples": len(samples),
-                "source": "nvml, separate process"}
+                "source": "nvml, separate process", "window": window}
 
 
 def profile_traffic(workload_key: str):

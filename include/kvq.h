@@ -168,6 +168,25 @@ int kvq_quantize_prefill(kvq_cache* cache, const void* k, const void* v, int L, 
  * Errors: STATE (no prefill yet), CAPACITY, INVALID_ARG, ALIGN, CUDA. */
 int kvq_append(kvq_cache* cache, const void* k_new, const void* v_new, void* stream);
 
+/* Sequences of different lengths (serving batches; no counterpart on the pages, whose
+ * rules apply to each sequence on its own: its window, quantized prefix and retained set
+ * follow from its own length).
+ *
+ * kvq_quantize_prefill_ragged: k fp16 [B][Hkv][L_max][d_k], v fp16 [B][Hkv][L_max][d_v];
+ * sequence b's first lengths[b] tokens are valid (lengths: host int[B], each in
+ * [1, L_max], L_max <= max_context).  With more than KVQ_MAX_SEQS sequences the lengths
+ * must be equal (UNSUPPORTED otherwise).
+ * kvq_append_ragged: kvq_append for the sequences with active[b] != 0 (host bytes [B];
+ * NULL = all); the rows of the others in k_new / v_new are ignored and their state is
+ * unchanged.  A partial mask needs B <= KVQ_MAX_SEQS (UNSUPPORTED otherwise).
+ * kvq_decode_attention then attends, for every sequence, over its own L_b tokens.
+ * Errors as for kvq_quantize_prefill / kvq_append. */
+#define KVQ_MAX_SEQS 256
+int kvq_quantize_prefill_ragged(kvq_cache* cache, const void* k, const void* v, int L_max,
+                                const int* lengths, void* stream);
+int kvq_append_ragged(kvq_cache* cache, const void* k_new, const void* v_new,
+                      const unsigned char* active, void* stream);
+
 /* Workspace bytes kvq_decode_attention needs at the cache's current length for
  * num_splits (0 = automatic).  Always <= kvq_sizes.workspace. */
 int kvq_decode_workspace_size(const kvq_cache* cache, int num_splits, size_t* bytes);
@@ -213,16 +232,22 @@ int kvq_set_decode_kernel(kvq_cache* cache, int kernel);
 int kvq_decode_attention_noalloc(kvq_cache* cache, const void* q, void* out, int num_splits,
                                  void* stream);
 
-/* The plan kvq_decode_attention would use now (host only, no launch). */
+/* The plan kvq_decode_attention would use now (host only, no launch); its counts are
+ * those of the longest sequence. */
 int kvq_get_plan(const kvq_cache* cache, int num_splits, kvq_plan* out);
 
 /* Pure host planner behind kvq_get_plan, for a configuration, length L, SM count
  * and split request.  Errors: INVALID_ARG, UNSUPPORTED. */
 int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, kvq_plan* out);
 
-/* Host-side cache state: length L, quantized prefix Q, retained count and the
- * ascending retained positions (retained_idx: host int[32], may be NULL). */
+/* Host-side state of sequence 0 (of every sequence when all have the same length):
+ * length L, quantized prefix Q, retained count and the ascending retained positions
+ * (retained_idx: host int[32], may be NULL). */
 int kvq_get_state(const kvq_cache* cache, int* L, int* Q, int* n_retained, int* retained_idx);
+
+/* The same for sequence b (0 <= b < batch, else INVALID_ARG). */
+int kvq_get_seq_state(const kvq_cache* cache, int b, int* L, int* Q, int* n_retained,
+                      int* retained_idx);
 
 /* The retention rule for a quantized prefix of Q tokens (host only): writes the
  * ascending positions into out[0..cap) and returns their count (>= 0), or

@@ -343,15 +343,16 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   const __half* qrow = qbase + (bvalid ? bhead : 0) * DK;
 
   // ---------------- work list of this warp ----------------
+  const SeqWork sw = seq_work(w, b, QUANT ? GK : 1, QUANT ? d.log_retain : 0);   // this sequence's lengths
   int unit_begin, unit_end;      // quantized: groups; fp16: tiles of 16 list entries
   int list_begin = 0, list_end = 0;
   if (quant) {
-    unit_begin = static_cast<int>(static_cast<long long>(split) * w.n_groups / w.splits_q);
-    unit_end = static_cast<int>(static_cast<long long>(split + 1) * w.n_groups / w.splits_q);
+    unit_begin = static_cast<int>(static_cast<long long>(split) * sw.n_groups / w.splits_q);
+    unit_end = static_cast<int>(static_cast<long long>(split + 1) * sw.n_groups / w.splits_q);
   } else {
     const int f = split - (QUANT ? w.splits_q : 0);
-    list_begin = static_cast<int>(static_cast<long long>(f) * w.n_fp16 / w.splits_f);
-    list_end = static_cast<int>(static_cast<long long>(f + 1) * w.n_fp16 / w.splits_f);
+    list_begin = static_cast<int>(static_cast<long long>(f) * sw.n_fp16 / w.splits_f);
+    list_end = static_cast<int>(static_cast<long long>(f + 1) * sw.n_fp16 / w.splits_f);
     unit_begin = 0;
     unit_end = (list_end - list_begin + 15) / 16;
   }
@@ -429,7 +430,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       __syncthreads();
 
       // retained positions, one per lane (ascending), for masking the quantized tiles
-      const int ret_pos = lane < w.ret.n ? w.ret.pos[lane] : -1;
+      const int ret_pos = lane < sw.n_ret ? retained_position(sw.Q, lane) : -1;
       const StageLayout L = quant_stage_layout(GK, DK, KB, VB, G::NVG, Z::ZB, SR);
       constexpr int gk = GK;
       constexpr int MT = GK / 16;     // 16-token m-tiles per key group
@@ -745,12 +746,12 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         size_t slot;
         const __half* base_k;
         const __half* base_v;
-        if (e < w.ret.n) {
+        if (e < sw.n_ret) {
           slot = static_cast<size_t>(bh) * kMaxRetained + e;
           base_k = cb.ret_k;
           base_v = cb.ret_v;
         } else {
-          const int pos = w.Q + (e - w.ret.n);
+          const int pos = sw.Q + (e - sw.n_ret);
           slot = static_cast<size_t>(bh) * d.cap + pos % d.cap;
           base_k = cb.win_k;
           base_v = cb.win_v;

@@ -78,15 +78,16 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
     __syncthreads();
   }
 
+  const SeqWork sw = seq_work(w, b, d.gk, d.log_retain);   // this sequence's lengths
   const bool quant = split < w.splits_q;
   int begin, end;
   if (quant) {
-    begin = static_cast<int>(static_cast<long long>(split) * w.n_groups / w.splits_q) * d.gk;
-    end = static_cast<int>(static_cast<long long>(split + 1) * w.n_groups / w.splits_q) * d.gk;
+    begin = static_cast<int>(static_cast<long long>(split) * sw.n_groups / w.splits_q) * d.gk;
+    end = static_cast<int>(static_cast<long long>(split + 1) * sw.n_groups / w.splits_q) * d.gk;
   } else {
     const int f = split - w.splits_q;
-    begin = static_cast<int>(static_cast<long long>(f) * w.n_fp16 / w.splits_f);
-    end = static_cast<int>(static_cast<long long>(f + 1) * w.n_fp16 / w.splits_f);
+    begin = static_cast<int>(static_cast<long long>(f) * sw.n_fp16 / w.splits_f);
+    end = static_cast<int>(static_cast<long long>(f + 1) * sw.n_fp16 / w.splits_f);
   }
   const int perk = d.kb == 16 ? 1 : 32 / d.kb, perv = d.vb == 16 ? 1 : 32 / d.vb;
   const uint32_t maskk = (1u << (d.kb & 15)) - 1u, maskv = (1u << (d.vb & 15)) - 1u;
@@ -97,9 +98,8 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
 #pragma unroll
     for (int j = 0; j < 8; ++j) zhat[j] = 0.0f;
     if (quant) {
-      bool retained = false;
-      for (int r = 0; r < w.ret.n; ++r) retained |= (w.ret.pos[r] == i);
-      if (retained) continue;                                   // read from the fp16 list
+      // retained ({p < Q : p mod 2^floor(log2(Q - p)) == 0}): read from the fp16 list
+      if (d.log_retain && (i & ((1 << (31 - __clz(sw.Q - i))) - 1)) == 0) continue;
       if (d.sr) {
         const uint8_t* zr = cb.zcode + (static_cast<size_t>(bh) * d.lcap + i) * d.zb;
         const uint32_t row = d.zb == 4 ? *reinterpret_cast<const uint32_t*>(zr)
@@ -140,12 +140,12 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
       }
     } else {
       const __half *kp, *vp;
-      if (i < w.ret.n) {
+      if (i < sw.n_ret) {
         const size_t s = static_cast<size_t>(bh) * kMaxRetained + i;
         kp = cb.ret_k + s * d.dk;
         vp = cb.ret_v + s * d.dv;
       } else {
-        const int pos = w.Q + (i - w.ret.n);
+        const int pos = sw.Q + (i - sw.n_ret);
         const size_t s = static_cast<size_t>(bh) * d.cap + pos % d.cap;
         kp = cb.win_k + s * d.dk;
         vp = cb.win_v + s * d.dv;

@@ -16,13 +16,17 @@
 struct kvq_cache {
   kvq::Dims d;
   kvq_buffers buf;
-  int L;
-  int Q;
-  std::vector<int> ret;   // ascending retained positions
+  std::vector<int> L;   // tokens of each sequence
+  std::vector<int> Q;   // quantized prefix of each sequence (its retained set follows from it)
   int sm_count;
   int kernel;     // KVQ_KERNEL_*
   bool prefilled;
   bool stall_next;  // test hook armed by kvq_debug_stall_next_decode
+  bool uniform() const {
+    for (size_t b = 1; b < L.size(); ++b)
+      if (L[b] != L[0]) return false;
+    return true;
+  }
 };
 
 namespace kvq {
@@ -148,15 +152,19 @@ int split_cap(const kvq::Dims& d) {
 // on the long-context workloads.
 int ctas_per_sm(bool fast) { return fast ? 3 : 4; }
 
-// Chooses the split counts: the number of CTAs per (b, kv head) over the quantized
-// groups and over the fp16 tokens, trading wave quantization against per-CTA cost.
-int plan_decode(const kvq::Dims& d, int L, int sm_count, int num_splits, bool fast,
-                kvq_plan* out) {
-  if (L < 1 || L > d.max_context || sm_count < 1 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
+// Quantized groups and fp16 entries of a sequence of L tokens.
+void seq_counts(const kvq::Dims& d, int L, int* nG, int* nF) {
   const int Q = quantized_prefix(d, L);
-  const int nret = d.log_retain ? static_cast<int>(retained_positions(Q).size()) : 0;
-  const int nG = Q / d.gk;
-  const int nF = nret + (L - Q);
+  *nG = Q / d.gk;
+  *nF = (d.log_retain ? kvq::retained_count(Q) : 0) + (L - Q);
+}
+
+// Chooses the split counts: the number of CTAs per (b, kv head) over the quantized
+// groups and over the fp16 tokens, trading wave quantization against per-CTA cost; nG and
+// nF are those of the longest sequence.
+int plan_counts(const kvq::Dims& d, int nG, int nF, int sm_count, int num_splits, bool fast,
+                kvq_plan* out) {
+  if (sm_count < 1 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
   const int rows = d.B * d.Hkv;
   const int cap = split_cap(d);
   const long long slots = static_cast<long long>(sm_count) * ctas_per_sm(fast);
@@ -203,10 +211,49 @@ int plan_decode(const kvq::Dims& d, int L, int sm_count, int num_splits, bool fa
   return KVQ_OK;
 }
 
+int plan_decode(const kvq::Dims& d, int L, int sm_count, int num_splits, bool fast, kvq_plan* out) {
+  if (L < 1 || L > d.max_context) return KVQ_ERR_INVALID_ARG;
+  int nG, nF;
+  seq_counts(d, L, &nG, &nF);
+  return plan_counts(d, nG, nF, sm_count, num_splits, fast, out);
+}
+
+// The plan of a cache: counts of its longest sequences.
+int plan_cache(const kvq_cache* c, int num_splits, bool fast, kvq_plan* out) {
+  int nG = 0, nF = 0;
+  for (size_t b = 0; b < c->L.size(); ++b) {
+    int g, f;
+    seq_counts(c->d, c->L[b], &g, &f);
+    nG = std::max(nG, g);
+    nF = std::max(nF, f);
+  }
+  return plan_counts(c->d, nG, nF, c->sm_count, num_splits, fast, out);
+}
+
 int check_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
 bool use_tensor_kernel(const kvq_cache* c) {
   return c->kernel != KVQ_KERNEL_GENERIC && kvq::decode_mma_supported(c->d);
+}
+
+// Dims and buffers of sequence b alone (a batch of one over the same memory).
+void sequence_view(const kvq_cache* c, int b, kvq::Dims* d1, kvq_buffers* b1) {
+  const kvq::Dims& d = c->d;
+  *d1 = d;
+  d1->B = 1;
+  const size_t bh = static_cast<size_t>(b) * d.Hkv;
+  auto at = [](void* p, size_t bytes) -> void* { return p ? static_cast<char*>(p) + bytes : nullptr; };
+  *b1 = c->buf;
+  b1->kcode = at(c->buf.kcode, bh * d.lcap * d.kw * 4);
+  b1->ksz = at(c->buf.ksz, bh * (d.lcap / d.gk) * d.dk * 4);
+  b1->vcode = at(c->buf.vcode, bh * d.lcap * d.vw * 4);
+  b1->vsz = at(c->buf.vsz, bh * d.lcap * d.nvg * 4);
+  b1->win_k = at(c->buf.win_k, bh * d.cap * d.dk * 2);
+  b1->win_v = at(c->buf.win_v, bh * d.cap * d.dv * 2);
+  b1->ret_k = at(c->buf.ret_k, bh * kvq::kMaxRetained * d.dk * 2);
+  b1->ret_v = at(c->buf.ret_v, bh * kvq::kMaxRetained * d.dv * 2);
+  b1->zcode = at(c->buf.zcode, bh * d.lcap * d.zb);
+  b1->zsz = at(c->buf.zsz, bh * (d.lcap / d.gk) * d.sr * 4);
 }
 
 kvq::CacheBufs cache_bufs(const kvq_cache* c) {
@@ -303,8 +350,8 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
   if (!c) return KVQ_ERR_INVALID_ARG;
   c->d = d;
   c->buf = *bufs;
-  c->L = 0;
-  c->Q = 0;
+  c->L.assign(d.B, 0);
+  c->Q.assign(d.B, 0);
   c->sm_count = sms;
   c->kernel = KVQ_KERNEL_AUTO;
   c->prefilled = false;
@@ -324,118 +371,207 @@ int kvq_retained_positions(int Q, int* out, int cap) {
   return static_cast<int>(r.size());
 }
 
+}  // extern "C"
+
+namespace {
+
+// Prefill of the sequences of (d, buf): k, v [d.B][Hkv][src_rows][d], the first L rows valid.
+int prefill_rows(const kvq::Dims& d, const kvq_buffers& buf, const __half* kh, const __half* vh,
+                 int src_rows, int L, cudaStream_t s) {
+  const int Q = quantized_prefix(d, L);
+  const int nbh = d.B * d.Hkv;
+  int rc = KVQ_OK;
+  if (Q > 0) {
+    rc = check_cuda(kvq::launch_quantize_keys(d, kh, src_rows, 0, Q / d.gk,
+                                              static_cast<uint32_t*>(buf.kcode),
+                                              static_cast<__half2*>(buf.ksz), d.rot != 0, s));
+    if (!rc)
+      rc = check_cuda(kvq::launch_quantize_side(
+          d, kh, src_rows, 0, Q / d.gk, static_cast<const uint32_t*>(buf.kcode),
+          static_cast<const __half2*>(buf.ksz), static_cast<const float*>(buf.side_u),
+          static_cast<uint8_t*>(buf.zcode), static_cast<__half2*>(buf.zsz), d.rot != 0, s));
+    if (!rc)
+      rc = check_cuda(kvq::launch_quantize_values(d, vh, src_rows, 0, Q,
+                                                  static_cast<uint32_t*>(buf.vcode),
+                                                  static_cast<__half2*>(buf.vsz), s));
+  }
+  if (!rc)
+    rc = check_cuda(d.rot ? kvq::launch_rotate_key_rows(d, kh, src_rows, Q, static_cast<__half*>(buf.win_k),
+                                                        d.cap, Q, L - Q, nullptr, s)
+                          : kvq::launch_copy_rows(kh, src_rows, Q, static_cast<__half*>(buf.win_k), d.cap,
+                                                  Q, L - Q, d.dk, nbh, s));
+  if (!rc)
+    rc = check_cuda(kvq::launch_copy_rows(vh, src_rows, Q, static_cast<__half*>(buf.win_v), d.cap, Q,
+                                          L - Q, d.dv, nbh, s));
+  if (!rc && d.log_retain && Q > 0) {
+    const std::vector<int> ret = retained_positions(Q);
+    kvq::RetList rl;
+    rl.n = static_cast<int>(ret.size());
+    for (int i = 0; i < rl.n; ++i) rl.pos[i] = ret[i];
+    rc = check_cuda(kvq::launch_copy_retained(d, d.rot ? nullptr : kh, vh, src_rows, rl,
+                                              static_cast<__half*>(buf.ret_k),
+                                              static_cast<__half*>(buf.ret_v), s));
+    if (!rc && d.rot)
+      rc = check_cuda(kvq::launch_rotate_key_rows(d, kh, src_rows, 0, static_cast<__half*>(buf.ret_k),
+                                                  kvq::kMaxRetained, 0, rl.n, &rl, s));
+  }
+  return rc;
+}
+
+// The oldest group_k window tokens of the sequences of (d, buf), whose quantized prefix is
+// Q, become one key group and group_k value rows; the retained set moves to that of Q + gk.
+// The window already holds the cached (rotated, if so configured) keys.
+int quantize_window_group(const kvq::Dims& d, const kvq_buffers& buf, int Q, cudaStream_t s) {
+  __half* wk = static_cast<__half*>(buf.win_k);
+  __half* wv = static_cast<__half*>(buf.win_v);
+  int rc = check_cuda(kvq::launch_quantize_keys(d, wk, d.cap, Q / d.gk, 1,
+                                                static_cast<uint32_t*>(buf.kcode),
+                                                static_cast<__half2*>(buf.ksz), false, s));
+  if (!rc)
+    rc = check_cuda(kvq::launch_quantize_side(
+        d, wk, d.cap, Q / d.gk, 1, static_cast<const uint32_t*>(buf.kcode),
+        static_cast<const __half2*>(buf.ksz), static_cast<const float*>(buf.side_u),
+        static_cast<uint8_t*>(buf.zcode), static_cast<__half2*>(buf.zsz), false, s));
+  if (!rc)
+    rc = check_cuda(kvq::launch_quantize_values(d, wv, d.cap, Q, d.gk, static_cast<uint32_t*>(buf.vcode),
+                                                static_cast<__half2*>(buf.vsz), s));
+  if (!rc && d.log_retain) {
+    const std::vector<int> old_ret = retained_positions(Q);
+    const std::vector<int> nr = retained_positions(Q + d.gk);
+    kvq::RetUpdate up;
+    up.n = static_cast<int>(nr.size());
+    for (int i = 0; i < up.n; ++i) {
+      const auto it = std::lower_bound(old_ret.begin(), old_ret.end(), nr[i]);
+      if (it != old_ret.end() && *it == nr[i]) {
+        up.from_window[i] = 0;
+        up.index[i] = static_cast<int>(it - old_ret.begin());
+      } else {
+        up.from_window[i] = 1;
+        up.index[i] = nr[i] % d.cap;
+      }
+    }
+    rc = check_cuda(kvq::launch_update_retained(d, up, wk, wv, static_cast<__half*>(buf.ret_k),
+                                                static_cast<__half*>(buf.ret_v), s));
+  }
+  return rc;
+}
+
+}  // namespace
+
+extern "C" {
+
 int kvq_quantize_prefill(kvq_cache* c, const void* k, const void* v, int L, void* stream) {
   if (!c || !k || !v) return KVQ_ERR_INVALID_ARG;
   const kvq::Dims& d = c->d;
   if (L < 1 || L > d.max_context) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const __half* kh = static_cast<const __half*>(k);
-  const __half* vh = static_cast<const __half*>(v);
-  const int Q = quantized_prefix(d, L);
-  const int nbh = d.B * d.Hkv;
-  int rc = KVQ_OK;
-  if (Q > 0) {
-    rc = check_cuda(kvq::launch_quantize_keys(d, kh, L, 0, Q / d.gk,
-                                              static_cast<uint32_t*>(c->buf.kcode),
-                                              static_cast<__half2*>(c->buf.ksz), d.rot != 0, s));
-    if (!rc)
-      rc = check_cuda(kvq::launch_quantize_side(
-          d, kh, L, 0, Q / d.gk, static_cast<const uint32_t*>(c->buf.kcode),
-          static_cast<const __half2*>(c->buf.ksz), static_cast<const float*>(c->buf.side_u),
-          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), d.rot != 0, s));
-    if (!rc)
-      rc = check_cuda(kvq::launch_quantize_values(d, vh, L, 0, Q,
-                                                  static_cast<uint32_t*>(c->buf.vcode),
-                                                  static_cast<__half2*>(c->buf.vsz), s));
-  }
-  if (!rc)
-    rc = check_cuda(d.rot ? kvq::launch_rotate_key_rows(d, kh, L, Q, static_cast<__half*>(c->buf.win_k),
-                                                        d.cap, Q, L - Q, nullptr, s)
-                          : kvq::launch_copy_rows(kh, L, Q, static_cast<__half*>(c->buf.win_k), d.cap,
-                                                  Q, L - Q, d.dk, nbh, s));
-  if (!rc)
-    rc = check_cuda(kvq::launch_copy_rows(vh, L, Q, static_cast<__half*>(c->buf.win_v), d.cap, Q,
-                                          L - Q, d.dv, nbh, s));
-  std::vector<int> ret;
-  if (d.log_retain) ret = retained_positions(Q);
-  if (!rc && !ret.empty()) {
-    kvq::RetList rl;
-    rl.n = static_cast<int>(ret.size());
-    for (int i = 0; i < rl.n; ++i) rl.pos[i] = ret[i];
-    rc = check_cuda(kvq::launch_copy_retained(d, d.rot ? nullptr : kh, vh, L, rl,
-                                              static_cast<__half*>(c->buf.ret_k),
-                                              static_cast<__half*>(c->buf.ret_v), s));
-    if (!rc && d.rot)
-      rc = check_cuda(kvq::launch_rotate_key_rows(d, kh, L, 0, static_cast<__half*>(c->buf.ret_k),
-                                                  kvq::kMaxRetained, 0, rl.n, &rl, s));
-  }
+  const int rc = prefill_rows(d, c->buf, static_cast<const __half*>(k), static_cast<const __half*>(v), L,
+                              L, static_cast<cudaStream_t>(stream));
   if (rc) return rc;
-  c->L = L;
-  c->Q = Q;
-  c->ret = ret;
+  c->L.assign(d.B, L);
+  c->Q.assign(d.B, quantized_prefix(d, L));
   c->prefilled = true;
   return KVQ_OK;
 }
 
-int kvq_append(kvq_cache* c, const void* k_new, const void* v_new, void* stream) {
+int kvq_quantize_prefill_ragged(kvq_cache* c, const void* k, const void* v, int L_max,
+                                const int* lengths, void* stream) {
+  if (!c || !k || !v || !lengths) return KVQ_ERR_INVALID_ARG;
+  const kvq::Dims& d = c->d;
+  if (L_max < 1 || L_max > d.max_context) return KVQ_ERR_INVALID_ARG;
+  for (int b = 0; b < d.B; ++b)
+    if (lengths[b] < 1 || lengths[b] > L_max) return KVQ_ERR_INVALID_ARG;
+  if (d.B > kvq::kMaxSeqs) {
+    for (int b = 1; b < d.B; ++b)
+      if (lengths[b] != lengths[0]) return KVQ_ERR_UNSUPPORTED;
+  }
+  if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __half* kh = static_cast<const __half*>(k);
+  const __half* vh = static_cast<const __half*>(v);
+  for (int b = 0; b < d.B; ++b) {
+    kvq::Dims d1;
+    kvq_buffers b1;
+    sequence_view(c, b, &d1, &b1);
+    const size_t off = static_cast<size_t>(b) * d.Hkv * L_max;
+    const int rc = prefill_rows(d1, b1, kh + off * d.dk, vh + off * d.dv, L_max, lengths[b], s);
+    if (rc) return rc;
+  }
+  for (int b = 0; b < d.B; ++b) {
+    c->L[b] = lengths[b];
+    c->Q[b] = quantized_prefix(d, lengths[b]);
+  }
+  c->prefilled = true;
+  return KVQ_OK;
+}
+
+int kvq_append_ragged(kvq_cache* c, const void* k_new, const void* v_new, const unsigned char* active,
+                      void* stream) {
   if (!c || !k_new || !v_new) return KVQ_ERR_INVALID_ARG;
   if (!c->prefilled) return KVQ_ERR_STATE;
   const kvq::Dims& d = c->d;
-  if (c->L + 1 > d.max_context) return KVQ_ERR_CAPACITY;
+  for (int b = 0; b < d.B; ++b)
+    if ((!active || active[b]) && c->L[b] + 1 > d.max_context) return KVQ_ERR_CAPACITY;
   if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_ALIGN;
+  bool all = true;
+  for (int b = 0; b < d.B && active; ++b) all = all && active[b];
+  if (!all && d.B > kvq::kMaxSeqs) return KVQ_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  __half* wk = static_cast<__half*>(c->buf.win_k);
-  __half* wv = static_cast<__half*>(c->buf.win_v);
-  const int slot = c->L % d.cap;
-  const __half* kn = static_cast<const __half*>(k_new);
-  int rc = check_cuda(kvq::launch_append_token(d, d.rot ? nullptr : kn,
-                                               static_cast<const __half*>(v_new), wk, wv, slot, s));
-  if (!rc && d.rot) rc = check_cuda(kvq::launch_rotate_key_rows(d, kn, 1, 0, wk, d.cap, slot, 1, nullptr, s));
-  if (rc) return rc;
-  const int L = c->L + 1;
-  int Q = c->Q;
-  std::vector<int> ret = c->ret;
-  if (d.quantized() && L - Q == d.R + d.gk) {
-    // the oldest group_k window tokens become one key group and group_k value rows
-    // the window already holds the cached (rotated, if so configured) keys
-    rc = check_cuda(kvq::launch_quantize_keys(d, wk, d.cap, Q / d.gk, 1,
-                                              static_cast<uint32_t*>(c->buf.kcode),
-                                              static_cast<__half2*>(c->buf.ksz), false, s));
-    if (!rc)
-      rc = check_cuda(kvq::launch_quantize_side(
-          d, wk, d.cap, Q / d.gk, 1, static_cast<const uint32_t*>(c->buf.kcode),
-          static_cast<const __half2*>(c->buf.ksz), static_cast<const float*>(c->buf.side_u),
-          static_cast<uint8_t*>(c->buf.zcode), static_cast<__half2*>(c->buf.zsz), false, s));
-    if (!rc)
-      rc = check_cuda(kvq::launch_quantize_values(d, wv, d.cap, Q, d.gk,
-                                                  static_cast<uint32_t*>(c->buf.vcode),
-                                                  static_cast<__half2*>(c->buf.vsz), s));
-    if (!rc && d.log_retain) {
-      const std::vector<int> nr = retained_positions(Q + d.gk);
-      kvq::RetUpdate up;
-      up.n = static_cast<int>(nr.size());
-      for (int i = 0; i < up.n; ++i) {
-        const auto it = std::lower_bound(c->ret.begin(), c->ret.end(), nr[i]);
-        if (it != c->ret.end() && *it == nr[i]) {
-          up.from_window[i] = 0;
-          up.index[i] = static_cast<int>(it - c->ret.begin());
-        } else {
-          up.from_window[i] = 1;
-          up.index[i] = nr[i] % d.cap;
-        }
-      }
-      rc = check_cuda(kvq::launch_update_retained(d, up, wk, wv, static_cast<__half*>(c->buf.ret_k),
-                                                  static_cast<__half*>(c->buf.ret_v), s));
-      ret = nr;
-    }
-    if (rc) return rc;
-    Q += d.gk;
+  const bool lockstep = all && c->uniform();
+  kvq::SlotMap slots;
+  if (lockstep) {
+    slots.slot[0] = c->L[0] % d.cap;
+    for (int b = 1; b < d.B && b < kvq::kMaxSeqs; ++b) slots.slot[b] = slots.slot[0];
+  } else {
+    for (int b = 0; b < d.B; ++b) slots.slot[b] = (!active || active[b]) ? c->L[b] % d.cap : -1;
   }
-  c->L = L;
-  c->Q = Q;
-  c->ret = ret;
+  int rc = KVQ_OK;
+  if (lockstep && d.B > kvq::kMaxSeqs) {
+    // more sequences than a slot map holds, all in the same slot: one launch per chunk
+    for (int b0 = 0; b0 < d.B && !rc; b0 += kvq::kMaxSeqs) {
+      kvq::Dims dc = d;
+      dc.B = std::min(kvq::kMaxSeqs, d.B - b0);
+      const size_t bh0 = static_cast<size_t>(b0) * d.Hkv;
+      rc = check_cuda(kvq::launch_append_token(
+          dc, static_cast<const __half*>(k_new) + bh0 * d.dk, static_cast<const __half*>(v_new) + bh0 * d.dv,
+          static_cast<__half*>(c->buf.win_k) + bh0 * d.cap * d.dk,
+          static_cast<__half*>(c->buf.win_v) + bh0 * d.cap * d.dv, slots, s));
+    }
+  } else {
+    rc = check_cuda(kvq::launch_append_token(d, static_cast<const __half*>(k_new),
+                                             static_cast<const __half*>(v_new),
+                                             static_cast<__half*>(c->buf.win_k),
+                                             static_cast<__half*>(c->buf.win_v), slots, s));
+  }
+  if (rc) return rc;
+  if (lockstep) {
+    // every sequence in step: one launch per kernel for the whole batch
+    const int L = c->L[0] + 1;
+    if (d.quantized() && L - c->Q[0] == d.R + d.gk) {
+      rc = quantize_window_group(d, c->buf, c->Q[0], s);
+      if (rc) return rc;
+      c->Q.assign(d.B, c->Q[0] + d.gk);
+    }
+    c->L.assign(d.B, L);
+    return KVQ_OK;
+  }
+  for (int b = 0; b < d.B; ++b) {
+    if (active && !active[b]) continue;
+    c->L[b] += 1;
+    if (d.quantized() && c->L[b] - c->Q[b] == d.R + d.gk) {
+      kvq::Dims d1;
+      kvq_buffers b1;
+      sequence_view(c, b, &d1, &b1);
+      rc = quantize_window_group(d1, b1, c->Q[b], s);
+      if (rc) return rc;
+      c->Q[b] += d.gk;
+    }
+  }
   return KVQ_OK;
+}
+
+int kvq_append(kvq_cache* c, const void* k_new, const void* v_new, void* stream) {
+  return kvq_append_ragged(c, k_new, v_new, nullptr, stream);
 }
 
 int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, kvq_plan* out) {
@@ -449,7 +585,7 @@ int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, 
 int kvq_get_plan(const kvq_cache* c, int num_splits, kvq_plan* out) {
   if (!c || !out) return KVQ_ERR_INVALID_ARG;
   if (!c->prefilled) return KVQ_ERR_STATE;
-  return plan_decode(c->d, c->L, c->sm_count, num_splits, use_tensor_kernel(c), out);
+  return plan_cache(c, num_splits, use_tensor_kernel(c), out);
 }
 
 int kvq_decode_workspace_size(const kvq_cache* c, int num_splits, size_t* bytes) {
@@ -468,19 +604,21 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
   const kvq::Dims& d = c->d;
   kvq_plan plan;
-  int rc = plan_decode(d, c->L, c->sm_count, num_splits, use_tensor_kernel(c), &plan);
+  int rc = plan_cache(c, num_splits, use_tensor_kernel(c), &plan);
   if (rc) return rc;
   kvq::DecodeWork w;
-  w.L = c->L;
-  w.Q = c->Q;
+  w.uniform = c->uniform() ? 1 : 0;
+  if (!w.uniform && d.B > kvq::kMaxSeqs) return KVQ_ERR_UNSUPPORTED;
+  for (int b = 0; b < (w.uniform ? 1 : d.B); ++b) {
+    w.L[b] = c->L[b];
+    w.Q[b] = c->Q[b];
+  }
   w.n_groups = plan.n_groups;
   w.n_fp16 = plan.n_fp16;
   w.splits_q = plan.splits_quant;
   w.splits_f = plan.splits_fp16;
   w.splits = plan.splits_quant + plan.splits_fp16;
   w.score_scale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.dk)));
-  w.ret.n = static_cast<int>(c->ret.size());
-  for (int i = 0; i < w.ret.n; ++i) w.ret.pos[i] = c->ret[i];
   w.stall = c->stall_next && plan.fast_path ? 1 : 0;
   c->stall_next = false;
   if (workspace_bytes < kvq::workspace_bytes(d, w.splits)) return KVQ_ERR_WORKSPACE;
@@ -509,14 +647,19 @@ int kvq_set_decode_kernel(kvq_cache* c, int kernel) {
   return KVQ_OK;
 }
 
-int kvq_get_state(const kvq_cache* c, int* L, int* Q, int* n_retained, int* retained_idx) {
-  if (!c) return KVQ_ERR_INVALID_ARG;
-  if (L) *L = c->L;
-  if (Q) *Q = c->Q;
-  if (n_retained) *n_retained = static_cast<int>(c->ret.size());
+int kvq_get_seq_state(const kvq_cache* c, int b, int* L, int* Q, int* n_retained, int* retained_idx) {
+  if (!c || b < 0 || b >= c->d.B) return KVQ_ERR_INVALID_ARG;
+  const std::vector<int> ret = c->d.log_retain ? retained_positions(c->Q[b]) : std::vector<int>();
+  if (L) *L = c->L[b];
+  if (Q) *Q = c->Q[b];
+  if (n_retained) *n_retained = static_cast<int>(ret.size());
   if (retained_idx)
-    for (size_t i = 0; i < c->ret.size(); ++i) retained_idx[i] = c->ret[i];
+    for (size_t i = 0; i < ret.size(); ++i) retained_idx[i] = ret[i];
   return KVQ_OK;
+}
+
+int kvq_get_state(const kvq_cache* c, int* L, int* Q, int* n_retained, int* retained_idx) {
+  return kvq_get_seq_state(c, 0, L, Q, n_retained, retained_idx);
 }
 
 int kvq_reset_status(void* workspace, void* stream) {

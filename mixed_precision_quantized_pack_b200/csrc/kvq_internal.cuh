@@ -8,6 +8,7 @@
 namespace kvq {
 
 constexpr int kMaxRetained = 32;
+constexpr int kMaxSeqs = 256;   // sequences of a cache whose lengths may differ (per-launch arrays)
 
 // Derived sizes of one cache (see include/kvq.h for the layouts).
 struct Dims {
@@ -73,17 +74,51 @@ struct RetUpdate {
   int index[kMaxRetained];         // the slot
 };
 
-// The tokens one decode call reads, and how they are split over CTAs.
+// Retained positions of a quantized prefix of Q tokens ({p < Q : p mod 2^floor(log2(Q-p)) == 0},
+// one per age octave): how many, and the i-th in ascending order (octave floor(log2 Q) - i).
+__host__ __device__ inline int retained_count(int Q) {
+  int n = 0;
+  while (n < 31 && (1 << n) <= Q) ++n;
+  return n;
+}
+__host__ __device__ inline int retained_position(int Q, int i) {
+  const int l = retained_count(Q) - 1 - i;
+  return ((Q - (1 << l)) >> l) << l;
+}
+
+// The tokens one decode call reads, and how they are split over CTAs.  Sequence b holds L[b]
+// tokens, Q[b] of them quantized (one entry for all sequences when `uniform`); its fp16 list
+// is its retained entries, then window positions Q[b]..L[b]-1.
 struct DecodeWork {
-  int L, Q;
-  int n_groups;      // Q / gk quantized groups
-  int n_fp16;        // fp16 list: retained entries, then window positions Q..L-1
+  int uniform;       // 1: every sequence has L[0], Q[0]
+  int L[kMaxSeqs], Q[kMaxSeqs];
+  int n_groups;      // quantized groups of the longest prefix (max over b of Q[b] / gk)
+  int n_fp16;        // longest fp16 list
   int splits_q;      // CTAs per (b, kv head) over the groups
   int splits_f;      // CTAs per (b, kv head) over the fp16 list
   int splits;        // splits_q + splits_f (partials per (b, query head))
   float score_scale; // log2(e) / sqrt(d_k)
   int stall;         // test hook: CTA (0, 0, 0) asks for 16 bytes more than its first copy delivers
-  RetList ret;
+};
+
+// Lengths of sequence b in a decode call: L, Q, quantized groups (Q / gk; Q is 0 for an
+// unquantized cache), retained entries and fp16 entries.
+struct SeqWork {
+  int L, Q, n_groups, n_ret, n_fp16;
+};
+__device__ __forceinline__ SeqWork seq_work(const DecodeWork& w, int b, int gk, int log_retain) {
+  SeqWork s;
+  s.L = w.uniform ? w.L[0] : w.L[b];
+  s.Q = w.uniform ? w.Q[0] : w.Q[b];
+  s.n_groups = s.Q / gk;
+  s.n_ret = log_retain ? retained_count(s.Q) : 0;
+  s.n_fp16 = s.n_ret + (s.L - s.Q);
+  return s;
+}
+
+// Window slot each sequence's new token goes to on an append (-1: the sequence does not append).
+struct SlotMap {
+  int slot[kMaxSeqs];
 };
 
 // Device views of the cache buffers.
@@ -133,9 +168,10 @@ cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __ha
 cudaError_t launch_rotate_key_rows(const Dims& d, const __half* src, int src_rows, int src_base,
                                    __half* dst, int dst_rows, int dst_base, int n,
                                    const RetList* list, cudaStream_t s);
-// k may be null: only the value row is copied
+// The new token of every sequence b with slots.slot[b] >= 0 into window slot slots.slot[b]:
+// the value row, and the key row (rotated when the cache rotates keys).
 cudaError_t launch_append_token(const Dims& d, const __half* k, const __half* v, __half* win_k,
-                                __half* win_v, int slot, cudaStream_t s);
+                                __half* win_v, const SlotMap& slots, cudaStream_t s);
 // k may be null: only the value rows are copied
 cudaError_t launch_copy_retained(const Dims& d, const __half* k, const __half* v, int L,
                                  const RetList& ret, __half* ret_k, __half* ret_v, cudaStream_t s);

@@ -292,15 +292,17 @@ __global__ void copy_rows_kernel(const __half* __restrict__ src, int src_rows, i
   }
 }
 
-// Append: the new token's key and value rows of every (b, kv head) into window slot `slot`
-// (one launch for both, 16 B per thread).
+// Append: the new token's key and value rows of every (b, kv head) into the window slot of
+// sequence b (none when it is -1), 16 B per thread; k null: values only.
 __global__ void append_token_kernel(const __half* __restrict__ k, const __half* __restrict__ v,
-                                    __half* __restrict__ win_k, __half* __restrict__ win_v, int slot,
-                                    int cap, int dk, int dv, int nbh) {
+                                    __half* __restrict__ win_k, __half* __restrict__ win_v,
+                                    SlotMap slots, int hkv, int cap, int dk, int dv, int nbh) {
   const int vk = dk / 8, vv = dv / 8;
   const int total = nbh * (vk + vv);
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
     const int bh = idx / (vk + vv), e = idx % (vk + vv);
+    const int slot = slots.slot[bh / hkv];
+    if (slot < 0) continue;
     if (e < vk) {
       if (k)
         reinterpret_cast<uint4*>(win_k + (static_cast<size_t>(bh) * cap + slot) * dk)[e] =
@@ -313,10 +315,12 @@ __global__ void append_token_kernel(const __half* __restrict__ k, const __half* 
 }
 
 // Rotated key rows, one warp per (b * kv head, row i < n): source row (src_base + i) %
-// src_rows, or list->pos[i], into destination row (dst_base + i) % dst_rows.
+// src_rows, or list->pos[i], into destination row (dst_base + i) % dst_rows, or, with
+// use_slots, into row slots.slot[b] (skipped when -1).
 __global__ void rotate_key_rows_kernel(const __half* __restrict__ src, int src_rows, int src_base,
                                        __half* __restrict__ dst, int dst_rows, int dst_base, int n,
-                                       int nbh, RetList list, int use_list, Dims d) {
+                                       int nbh, RetList list, int use_list, SlotMap slots,
+                                       int use_slots, Dims d) {
   const int lane = threadIdx.x & 31;
   const long long total = static_cast<long long>(nbh) * n;
   const int dk = d.dk;
@@ -325,7 +329,8 @@ __global__ void rotate_key_rows_kernel(const __half* __restrict__ src, int src_r
     const int i = static_cast<int>(r % n);
     const int bh = static_cast<int>(r / n);
     const int sr = use_list ? list.pos[i] : (src_base + i) % src_rows;
-    const int dr = (dst_base + i) % dst_rows;
+    const int dr = use_slots ? slots.slot[bh / d.Hkv] : (dst_base + i) % dst_rows;
+    if (dr < 0) continue;                                   // uniform per warp
     const __half* s = src + (static_cast<size_t>(bh) * src_rows + sr) * dk;
     __half* t = dst + (static_cast<size_t>(bh) * dst_rows + dr) * dk;
     float x[8];
@@ -429,8 +434,11 @@ cudaError_t launch_rotate_key_rows(const Dims& d, const __half* src, int src_row
   const long long warps = static_cast<long long>(nbh) * n;
   RetList empty;
   empty.n = 0;
+  SlotMap none;
+  none.slot[0] = -1;
   rotate_key_rows_kernel<<<grid_for(warps * 32, 256), 256, 0, s>>>(
-      src, src_rows, src_base, dst, dst_rows, dst_base, n, nbh, list ? *list : empty, list ? 1 : 0, d);
+      src, src_rows, src_base, dst, dst_rows, dst_base, n, nbh, list ? *list : empty, list ? 1 : 0,
+      none, 0, d);
   return cudaGetLastError();
 }
 
@@ -481,12 +489,19 @@ cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __ha
 }
 
 cudaError_t launch_append_token(const Dims& d, const __half* k, const __half* v, __half* win_k,
-                                __half* win_v, int slot, cudaStream_t s) {
+                                __half* win_v, const SlotMap& slots, cudaStream_t s) {
   const int nbh = d.B * d.Hkv;
   const int total = nbh * (d.dk + d.dv) / 8;
   const int block = 256;
-  append_token_kernel<<<(total + block - 1) / block, block, 0, s>>>(k, v, win_k, win_v, slot, d.cap, d.dk,
-                                                                  d.dv, nbh);
+  append_token_kernel<<<(total + block - 1) / block, block, 0, s>>>(
+      d.rot ? nullptr : k, v, win_k, win_v, slots, d.Hkv, d.cap, d.dk, d.dv, nbh);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !d.rot) return e;
+  // rotated keys: one warp per (b, kv head) row
+  RetList empty;
+  empty.n = 0;
+  rotate_key_rows_kernel<<<grid_for(static_cast<long long>(nbh) * 32, 256), 256, 0, s>>>(
+      k, 1, 0, win_k, d.cap, 0, 1, nbh, empty, 0, slots, 1, d);
   return cudaGetLastError();
 }
 

@@ -31,6 +31,7 @@ KVQ_KERNEL_GENERIC = 1
 KVQ_KERNEL_TENSOR = 2
 KVQ_STATUS_TIMEOUT = 1
 KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
+KVQ_MAX_SEQS = 256
 
 CONFIG_FIELDS = ("batch", "n_q_heads", "n_kv_heads", "d_k", "d_v", "k_bits", "v_bits", "group_k",
                  "group_v", "window", "log_retain", "max_context", "side_rank", "side_bits",
@@ -76,6 +77,10 @@ _SIGNATURES = {
     "kvq_cache_destroy": (None, [_P]),
     "kvq_quantize_prefill": (_I, [_P, _P, _P, _I, _P]),
     "kvq_append": (_I, [_P, _P, _P, _P]),
+    "kvq_quantize_prefill_ragged": (_I, [_P, _P, _P, _I, ctypes.POINTER(_I), _P]),
+    "kvq_append_ragged": (_I, [_P, _P, _P, ctypes.POINTER(ctypes.c_ubyte), _P]),
+    "kvq_get_seq_state": (_I, [_P, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
+                               ctypes.POINTER(_I)]),
     "kvq_decode_workspace_size": (_I, [_P, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "kvq_decode_attention": (_I, [_P, _P, _P, _P, ctypes.c_size_t, _I, _P]),
     "kvq_decode_attention_noalloc": (_I, [_P, _P, _P, _I, _P]),
@@ -171,6 +176,25 @@ def kvq_quantize_prefill(handle: int, k_ptr: int, v_ptr: int, L: int, stream: in
 
 def kvq_append(handle: int, k_ptr: int, v_ptr: int, stream: int) -> None:
     _check(lib().kvq_append(handle, k_ptr, v_ptr, stream), "kvq_append")
+
+
+def kvq_quantize_prefill_ragged(handle: int, k_ptr: int, v_ptr: int, L_max: int, lengths, stream: int) -> None:
+    arr = (_I * len(lengths))(*[int(x) for x in lengths])
+    _check(lib().kvq_quantize_prefill_ragged(handle, k_ptr, v_ptr, int(L_max), arr, stream),
+           "kvq_quantize_prefill_ragged")
+
+
+def kvq_append_ragged(handle: int, k_ptr: int, v_ptr: int, active, stream: int) -> None:
+    mask = None if active is None else (ctypes.c_ubyte * len(active))(*[1 if a else 0 for a in active])
+    _check(lib().kvq_append_ragged(handle, k_ptr, v_ptr, mask, stream), "kvq_append_ragged")
+
+
+def kvq_get_seq_state(handle: int, b: int) -> Tuple[int, int, List[int]]:
+    L, Q, n = _I(), _I(), _I()
+    idx = (ctypes.c_int * KVQ_MAX_RETAINED)()
+    _check(lib().kvq_get_seq_state(handle, int(b), ctypes.byref(L), ctypes.byref(Q), ctypes.byref(n), idx),
+           "kvq_get_seq_state")
+    return L.value, Q.value, [int(idx[i]) for i in range(n.value)]
 
 
 def kvq_decode_workspace_size(handle: int, num_splits: int = 0) -> int:
@@ -281,11 +305,31 @@ class KVCache:
         _fp16_cuda(v, (c["batch"], c["n_kv_heads"], L, c["d_v"]), "v")
         kvq_quantize_prefill(self.handle, k.data_ptr(), v.data_ptr(), L, _stream(stream))
 
-    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None) -> None:
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor, stream=None, active=None) -> None:
+        """One token per sequence; `active` (B bools) limits the append to some sequences."""
         c = self.cfg
         _fp16_cuda(k_new, (c["batch"], c["n_kv_heads"], c["d_k"]), "k_new")
         _fp16_cuda(v_new, (c["batch"], c["n_kv_heads"], c["d_v"]), "v_new")
-        kvq_append(self.handle, k_new.data_ptr(), v_new.data_ptr(), _stream(stream))
+        if active is None:
+            kvq_append(self.handle, k_new.data_ptr(), v_new.data_ptr(), _stream(stream))
+        else:
+            if len(active) != c["batch"]:
+                raise ValueError("active: one flag per sequence")
+            kvq_append_ragged(self.handle, k_new.data_ptr(), v_new.data_ptr(), list(active), _stream(stream))
+
+    def prefill_ragged(self, k: torch.Tensor, v: torch.Tensor, lengths, stream=None) -> None:
+        """k, v [B][Hkv][L_max][d]; sequence b's first lengths[b] tokens are its context."""
+        c = self.cfg
+        L_max = k.shape[2]
+        _fp16_cuda(k, (c["batch"], c["n_kv_heads"], L_max, c["d_k"]), "k")
+        _fp16_cuda(v, (c["batch"], c["n_kv_heads"], L_max, c["d_v"]), "v")
+        if len(lengths) != c["batch"]:
+            raise ValueError("lengths: one per sequence")
+        kvq_quantize_prefill_ragged(self.handle, k.data_ptr(), v.data_ptr(), L_max, list(lengths),
+                                    _stream(stream))
+
+    def seq_state(self, b: int) -> Tuple[int, int, List[int]]:
+        return kvq_get_seq_state(self.handle, b)
 
     def decode(self, q: torch.Tensor, out: Optional[torch.Tensor] = None, num_splits: int = 0,
                stream=None) -> torch.Tensor:

@@ -176,3 +176,10 @@ def test_side_code_buffers_are_required_and_aligned():
     with pytest.raises(K.KVQError) as e:
         K.kvq_cache_init(c, ptrs)
     assert e.value.code == K.KVQ_ERR_ALIGN
+
+
+def test_ragged_calls_check_their_arguments():
+    lib = K.lib()
+    assert lib.kvq_quantize_prefill_ragged(None, None, None, 1, None, None) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_append_ragged(None, None, None, None, None) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_get_seq_state(None, 0, None, None, None, None) == K.KVQ_ERR_INVALID_ARG

@@ -29,9 +29,10 @@ def np16(t):
     return t.detach().cpu().numpy()
 
 
-def compare_state(gc: K.KVCache, oc: O.OracleCache, b_rows=None, where=""):
-    """Bit-exact comparison of every valid byte of the cache, rows b in b_rows."""
-    L, Q, ret = gc.state()
+def compare_state(gc: K.KVCache, oc: O.OracleCache, b_rows=None, where="", seq=None):
+    """Bit-exact comparison of every valid byte of the cache, rows b in b_rows (the state of
+    sequence `seq` when the sequences' lengths differ)."""
+    L, Q, ret = gc.state() if seq is None else gc.seq_state(seq)
     assert (L, Q, ret) == (oc.L, oc.Q, oc.ret_idx), where
     rows = list(range(gc.B)) if b_rows is None else list(b_rows)
     c = gc.cfg
@@ -352,3 +353,75 @@ def test_rotation_unquantized_cache():
 
 def test_full_size_rot_32k():
     sampled_full_size(W.WORKLOADS["rot32k"], rows=(0, 31))
+
+
+# ------------------------------------------- sequences of different lengths ----
+def run_ragged(w: W.Workload, lengths, n_app, steps, seed, num_splits=(0, 2)):
+    """Ragged prefill, then appends where random sequences sit out: every sequence's cache
+    bytes and outputs match an oracle cache of that sequence alone."""
+    need_gpu()
+    L_max = max(lengths)
+    inp = W.Inputs(w.with_(context=L_max, appends=n_app), device="cpu")
+    cfg = w.kvq_config(max_context=L_max + n_app + 64)
+    gc = K.KVCache(cfg, side_basis=inp.side_basis)
+    gc.prefill_ragged(inp.k.cuda(), inp.v.cuda(), lengths)
+    U = None if inp.side_basis is None else inp.side_basis.numpy()
+    ocs = []
+    for b, Lb in enumerate(lengths):
+        oc = O.OracleCache(dict(cfg, batch=1), side_basis=U)
+        oc.prefill(np16(inp.k[b:b + 1, :, :Lb]), np16(inp.v[b:b + 1, :, :Lb]))
+        ocs.append(oc)
+    rng = np.random.default_rng(seed)
+    for i in range(n_app):
+        active = [True] * len(lengths) if i % 3 == 0 else [bool(x) for x in rng.integers(0, 2, len(lengths))]
+        gc.append(inp.k_app[i].cuda(), inp.v_app[i].cuda(), active=active)
+        for b, oc in enumerate(ocs):
+            if active[b]:
+                oc.append(np16(inp.k_app[i][b:b + 1]), np16(inp.v_app[i][b:b + 1]))
+        if i not in steps:
+            continue
+        for b, oc in enumerate(ocs):
+            assert gc.seq_state(b) == (oc.L, oc.Q, oc.ret_idx), (i, b)
+            compare_state(gc, oc, b_rows=[b], where=f"step {i} b={b}", seq=b)
+        for kern in KERNELS:
+            gc.set_kernel(kern)
+            for ns in num_splits:
+                out = gc.decode(inp.q[i].cuda(), num_splits=ns).float().cpu().numpy()
+                for b, oc in enumerate(ocs):
+                    err = O.max_rel_error(out[b:b + 1], oc.decode(np16(inp.q[i][b:b + 1])))
+                    assert err <= TOL, f"step {i} b={b} kernel {kern} splits {ns}: {err:.3e}"
+        gc.set_kernel(K.KVQ_KERNEL_AUTO)
+    assert gc.status() == 0
+
+
+def test_ragged_batch_tensor_kernel():
+    w = W.WORKLOADS["long32k"].with_(batch=5, seed=211)
+    run_ragged(w, [1500, 700, 64, 1111, 129], n_app=70, steps={0, 5, 40, 69}, seed=212)
+
+
+def test_ragged_batch_with_side_code_and_rotation():
+    w = W.WORKLOADS["headq32k"].with_(batch=3, rot_keys=1, rot_seed=9, seed=221)
+    run_ragged(w, [900, 333, 1280], n_app=66, steps={1, 64, 65}, seed=222)
+
+
+def test_ragged_batch_generic_shapes():
+    w = W.WORKLOADS["gqa4k"].with_(batch=3, n_q_heads=6, n_kv_heads=3, d_k=64, d_v=64, group_k=32,
+                                   group_v=32, window=48, log_retain=1, seed=231)
+    run_ragged(w, [400, 81, 257], n_app=40, steps={0, 17, 39}, seed=232)
+
+
+def test_uniform_lengths_through_the_ragged_calls_match_the_plain_ones():
+    need_gpu()
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=1000, appends=5, log_retain=1, seed=241)
+    inp = W.Inputs(w, device="cpu")
+    cfg = w.kvq_config()
+    a, b = K.KVCache(cfg), K.KVCache(cfg)
+    a.prefill(inp.k.cuda(), inp.v.cuda())
+    b.prefill_ragged(inp.k.cuda(), inp.v.cuda(), [1000, 1000])
+    for i in range(5):
+        a.append(inp.k_app[i].cuda(), inp.v_app[i].cuda())
+        b.append(inp.k_app[i].cuda(), inp.v_app[i].cuda(), active=[True, True])
+    assert a.state() == b.state() == b.seq_state(1)
+    for name in ("kcode", "ksz", "vcode", "vsz", "ret_k", "ret_v"):
+        assert torch.equal(a.buffers[name], b.buffers[name]), name
+    assert torch.equal(a.decode(inp.q[-1].cuda()), b.decode(inp.q[-1].cuda()))
