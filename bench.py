@@ -49,7 +49,8 @@ def peaks():
 
 def decode_bytes(cfg: dict, L: int) -> int:
     """Algorithmic bytes one decode reads: packed codes and (scale, zero) of the quantized
-    tokens (retained slots included), fp16 window and retained tokens, and q."""
+    tokens (retained slots included), fp16 window and retained tokens, q, and (paged caches)
+    the block-table entries of the quantized groups."""
     B, H, dk, dv = cfg["batch"], cfg["n_kv_heads"], cfg["d_k"], cfg["d_v"]
     kb, vb, gk, gv, R = cfg["k_bits"], cfg["v_bits"], cfg["group_k"], cfg["group_v"], cfg["window"]
     if kb == 16:
@@ -60,7 +61,8 @@ def decode_bytes(cfg: dict, L: int) -> int:
     per_tok = dk * kb // 8 + dv * vb // 8 + (dv // gv) * 4 + sr * sq // 8
     quant = Q * per_tok + (Q // gk) * (dk * 4 + sr * 4)
     fp16 = (L - Q + nret) * (dk + dv) * 2
-    return B * H * (quant + fp16) + B * cfg["n_q_heads"] * dk * 2
+    table = B * (Q // gk) * 4 if cfg.get("paged") else 0
+    return B * H * (quant + fp16) + B * cfg["n_q_heads"] * dk * 2 + table
 
 
 CLOCK_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
@@ -308,8 +310,10 @@ def main():
             # append (one copy kernel for K and V; rotated keys take a second one), then the
             # decode and the combine
             launches += (2 if cfg.get("rot_keys") else 1) + 2
-            if q1 != q0:     # a window group was quantized: keys, values, side code, retained set
+            if q1 != q0:     # a window group was quantized: keys, values, side code, retained set,
+                             # and (paged) the new page's block-table entries
                 launches += 2 + (1 if cfg.get("side_rank") else 0) + (1 if cfg["log_retain"] else 0)
+                launches += 1 if cfg.get("paged") else 0
             bytes_read.append(decode_bytes(cfg, L))
 
     for i in range(warm):

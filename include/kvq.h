@@ -70,6 +70,19 @@
  *               prefill, read by prefill, append and decode, never written here
  * with Lcap = max_context rounded up to a multiple of group_k.
  *
+ * Paged caches (paged = 1; serving shapes, no counterpart on the pages): the six
+ * quantized buffers hold a pool of n_pages pages instead of one Lcap-token region per
+ * (b, kv head): page p is one key group of one sequence for every kv head, laid out
+ *   kcode [n_pages][Hkv][group_k][d_k*k_bits/32]   ksz [n_pages][Hkv][2*d_k]
+ *   vcode [n_pages][Hkv][group_k][d_v*v_bits/32]   vsz [n_pages][Hkv][group_k][d_v/group_v][2]
+ *   zcode [n_pages][Hkv][group_k][r*side_bits/8]   zsz [n_pages][Hkv][r][2]
+ * (each page is the (b, h) layout above restricted to one group), and block_table
+ * int32 [B][Lcap/group_k] maps a sequence's group g to its page.  The library hands out
+ * pages (prefill, and an append that quantizes a window group) and takes them back
+ * (a new prefill of the sequence, kvq_release_sequence), and writes the table; the
+ * window and retained buffers stay per sequence.  Needs quantized keys and values;
+ * 1 <= n_pages, n_pages*Hkv*group_k < 2^30.
+ *
  * Conventions: every call is asynchronous on the caller's CUDA stream (passed as
  * void*, a cudaStream_t; NULL = legacy default stream); no call synchronizes or
  * copies device memory back to the host, except kvq_read_status.  The library
@@ -92,9 +105,9 @@ extern "C" {
 #define KVQ_ERR_INVALID_ARG   -1  /* null pointer, non-positive size, L > max_context */
 #define KVQ_ERR_UNSUPPORTED   -2  /* shape / bit width / group outside the built set */
 #define KVQ_ERR_ALIGN         -3  /* a device pointer is not 16-byte aligned */
-#define KVQ_ERR_CAPACITY      -4  /* an append past max_context */
+#define KVQ_ERR_CAPACITY      -4  /* an append past max_context; a page pool too small */
 #define KVQ_ERR_WORKSPACE     -5  /* workspace smaller than kvq_decode_workspace_size */
-#define KVQ_ERR_STATE         -6  /* decode or append before any prefill */
+#define KVQ_ERR_STATE         -6  /* decode or append on an empty sequence */
 #define KVQ_ERR_CUDA          -7  /* a CUDA runtime call or kernel launch failed */
 
 #define KVQ_MAX_RETAINED      32
@@ -103,7 +116,7 @@ extern "C" {
 #define KVQ_STATUS_TIMEOUT    1u  /* a bounded wait in the decode kernel gave up */
 
 typedef struct kvq_config {
-    int batch;          /* B, sequences sharing one length */
+    int batch;          /* B, sequences (slots) of the cache */
     int n_q_heads;      /* Hq */
     int n_kv_heads;     /* Hkv; Hq % Hkv == 0 */
     int d_k;            /* key/query head dim: 32, 64, 128 or 256 */
@@ -119,17 +132,21 @@ typedef struct kvq_config {
     int side_bits;      /* bits per side code: 4 or 8, with side_rank*side_bits 16 or 32 */
     int rot_keys;       /* 0/1: key-only rotation */
     unsigned int rot_signs[8];  /* rotation signs: bit c (word c/32, bit c%32) set -> -1 */
+    int paged;          /* 0/1: quantized groups live in a shared pool of pages (see below) */
+    int n_pages;        /* pages in the pool (paged caches); one page = one key group */
 } kvq_config;
 
 typedef struct kvq_sizes {
     size_t kcode, ksz, vcode, vsz, win_k, win_v, ret_k, ret_v;
     size_t workspace;   /* a decode workspace large enough for any length and split count */
     size_t zcode, zsz, side_u;   /* side code buffers (0 without a side code) */
+    size_t block_table; /* paged caches: int32 [B][max_context/group_k rounded up] */
 } kvq_sizes;
 
 typedef struct kvq_buffers {
     void *kcode, *ksz, *vcode, *vsz, *win_k, *win_v, *ret_k, *ret_v;
     void *zcode, *zsz, *side_u;  /* side code buffers (NULL without a side code) */
+    void *block_table;           /* paged caches (NULL otherwise); written by the library */
 } kvq_buffers;
 
 typedef struct kvq_cache kvq_cache;   /* opaque host-side handle */
@@ -159,7 +176,8 @@ void kvq_cache_destroy(kvq_cache* cache);
 /* Fill an empty cache with L >= 1 tokens: k fp16 [B][Hkv][L][d_k], v fp16
  * [B][Hkv][L][d_v], contiguous device memory.  Quantizes [0, Q), copies [Q, L)
  * into the window and the retained tokens into ret_k/ret_v.  Resets any earlier
- * content.  Errors: INVALID_ARG (L < 1 or L > max_context), ALIGN, CUDA. */
+ * content.  Errors: INVALID_ARG (L < 1 or L > max_context), CAPACITY (a paged
+ * pool with too few pages), ALIGN, CUDA. */
 int kvq_quantize_prefill(kvq_cache* cache, const void* k, const void* v, int L, void* stream);
 
 /* Append one token per sequence: k_new fp16 [B][Hkv][d_k], v_new fp16
@@ -184,8 +202,23 @@ int kvq_append(kvq_cache* cache, const void* k_new, const void* v_new, void* str
 #define KVQ_MAX_SEQS 256
 int kvq_quantize_prefill_ragged(kvq_cache* cache, const void* k, const void* v, int L_max,
                                 const int* lengths, void* stream);
+
 int kvq_append_ragged(kvq_cache* cache, const void* k_new, const void* v_new,
                       const unsigned char* active, void* stream);
+
+/* Slot management (serving; no counterpart on the pages).
+ * kvq_prefill_sequence: prefill sequence b alone with 1 <= L <= max_context tokens,
+ * k fp16 [Hkv][L][d_k], v fp16 [Hkv][L][d_v]; the other sequences are untouched.  A
+ * paged cache first takes back b's old pages.
+ * kvq_release_sequence: forget sequence b (a paged cache takes back its pages); its
+ * length becomes 0.  Decode fails with STATE while any sequence is empty, and so does
+ * an append that includes an empty sequence.
+ * kvq_free_pages: pages of the pool not in use (0 for caches that are not paged).
+ * Errors: INVALID_ARG (b or L out of range), CAPACITY (the pool has too few free pages;
+ * nothing changes), ALIGN, CUDA. */
+int kvq_prefill_sequence(kvq_cache* cache, int b, const void* k, const void* v, int L, void* stream);
+int kvq_release_sequence(kvq_cache* cache, int b);
+int kvq_free_pages(const kvq_cache* cache);
 
 /* Workspace bytes kvq_decode_attention needs at the cache's current length for
  * num_splits (0 = automatic).  Always <= kvq_sizes.workspace. */

@@ -234,7 +234,8 @@ struct Smem {
   static constexpr int kIssued = kBars + kMaxRing * 8;
   static constexpr int kTag = kIssued + kMaxRing * 4;
   static constexpr int kFail = kTag + kMaxRing * 4;
-  static constexpr int kQt = kFail + 16;                     // U_h^T q: fp32 [4 heads][SR]
+  static constexpr int kPage = kFail + 16;                   // per warp: the next unit's page
+  static constexpr int kQt = kPage + 16;                     // U_h^T q: fp32 [4 heads][SR]
   static constexpr int kStages = kBars + (SR ? 512 : 256);
   static_assert(kQt + 4 * SR * 4 <= kStages, "header overflow");
 };
@@ -283,7 +284,8 @@ struct Rings {
                                                                           : RING_F * STAGE_F);
 };
 
-template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4,
+          bool PAGED = false>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part) {
   using G = Quant<(QUANT ? KB : 4), (QUANT ? VB : 2), (QUANT ? DK : 128), (QUANT ? GV : 64)>;
@@ -440,9 +442,25 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       const uint32_t sel_hi = swap ? 0x3276u : 0x7632u;
 
       constexpr int RING = RG::RING_Q, STAGE = RG::STAGE_Q;
+      // Group index of unit k: its (scale, zero) block; its first token row is that times
+      // GK.  A paged cache takes the group's page from the block table: a refill reads the
+      // entry that its warp's lane 0 fetched (cp.async into the warp's slot) when the warp
+      // began the unit before it.
+      int* sm_page = reinterpret_cast<int*>(smem + SM::kPage);
+      auto table_entry = [&](int k) { return cb.table + (b * d.max_groups + unit_begin + k); };
+      auto group_of = [&](int k, bool fetched) -> size_t {
+        if constexpr (!PAGED) return static_cast<size_t>(bh) * d.max_groups + unit_begin + k;
+        int page;
+        if (fetched) {
+          ptx::cp_async_wait_all();
+          page = sm_page[warp];
+        } else {
+          page = __ldg(table_entry(k));
+        }
+        return static_cast<size_t>(page) * d.Hkv + h;
+      };
       // one lane copies unit k (a whole key group: 4 contiguous runs) into stage k % RING
-      auto issue = [&](int k) {
-        const int g = unit_begin + k;
+      auto issue = [&](int k, size_t gi) {
         const int st = k % RING;
         const uint32_t bar = bar0 + 8 * st;
         const uint32_t dst = stages_s + st * STAGE;
@@ -451,25 +469,26 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         // (test hook) one stage that never completes: its waits run into their bound
         const bool stall = w.stall && k == 0 && split == 0 && h == 0 && b == 0;
         ptx::mbar_arrive_expect_tx(bar, L.bytes + (stall ? 16u : 0u));
-        const size_t tok = static_cast<size_t>(bh) * d.lcap + static_cast<size_t>(g) * gk;
+        const size_t tok = gi * gk;
         ptx::bulk_g2s(dst + L.k_off, cb.kcode + tok * G::KW, gk * G::KBYTES_ROW, bar);
-        ptx::bulk_g2s(dst + L.kmeta_off, cb.ksz + (static_cast<size_t>(bh) * (d.lcap / gk) + g) * DK,
-                      DK * 4, bar);
+        ptx::bulk_g2s(dst + L.kmeta_off, cb.ksz + gi * DK, DK * 4, bar);
         ptx::bulk_g2s(dst + L.v_off, cb.vcode + tok * G::VW, gk * G::VBYTES_ROW, bar);
         ptx::bulk_g2s(dst + L.vmeta_off, cb.vsz + tok * G::NVG, gk * G::NVG * 4, bar);
         if constexpr (SR > 0) {
           ptx::bulk_g2s(dst + L.z_off, cb.zcode + tok * Z::ZB, gk * Z::ZB, bar);
-          ptx::bulk_g2s(dst + L.zmeta_off, cb.zsz + (static_cast<size_t>(bh) * (d.lcap / gk) + g) * SR,
-                        SR * 4, bar);
+          ptx::bulk_g2s(dst + L.zmeta_off, cb.zsz + gi * SR, SR * 4, bar);
         }
       };
 
       if (threadIdx.x == 0) {
         ptx::fence_proxy_async_smem();     // the rotated query rows were written to the stages
-        for (int k = 0; k < RING && k < n_units; ++k) issue(k);
+        for (int k = 0; k < RING && k < n_units; ++k) issue(k, group_of(k, false));
       }
 
       for (int k = warp; k < n_units; k += kWarps) {
+        // the page the stage is refilled with after this unit, fetched early
+        if (PAGED && lane == 0 && k + RING < n_units)
+          ptx::cp_async_4(ptx::smem_addr(sm_page + warp), table_entry(k + RING));
         const int g = unit_begin + k;
         const int st = k % RING;
         const bool ok = ptx::wait_equal_bounded(sm_tag + st, k, kWaitLimitNs) &&
@@ -704,7 +723,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
         __syncwarp();
         if (lane == 0 && k + RING < n_units) {
           ptx::fence_proxy_async_smem();
-          issue(k + RING);
+          issue(k + RING, group_of(k + RING, true));
         }
       }
     }
@@ -834,6 +853,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
     atomicOr(part.status, KVQ_STATUS_TIMEOUT);
     atomicOr(sm_fail, 1);
   }
+  if constexpr (PAGED) ptx::cp_async_wait_all();   // a page fetch of a unit given up on
   __syncthreads();
   if (*sm_fail) {
     if (threadIdx.x < ring && sm_issued[threadIdx.x] > 0)
@@ -905,14 +925,15 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   }
 }
 
-template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4>
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4,
+          bool PAGED = false>
 cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
                    const Partials& p, cudaStream_t s) {
   using RG = Rings<KB, VB, DK, GV, GK, QUANT, SR, SQ>;
   int smem = RG::BYTES;
   const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
   if (RG::HDR + merge > smem) smem = RG::HDR + merge;
-  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ>;
+  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ, PAGED>;
   static int configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

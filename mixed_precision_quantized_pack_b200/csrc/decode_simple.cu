@@ -100,24 +100,25 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
     if (quant) {
       // retained ({p < Q : p mod 2^floor(log2(Q - p)) == 0}): read from the fp16 list
       if (d.log_retain && (i & ((1 << (31 - __clz(sw.Q - i))) - 1)) == 0) continue;
+      const size_t row = group_row(d, cb.table, b, h, i / d.gk) + i % d.gk;
+      const size_t gidx = group_index(d, cb.table, b, h, i / d.gk);
       if (d.sr) {
-        const uint8_t* zr = cb.zcode + (static_cast<size_t>(bh) * d.lcap + i) * d.zb;
-        const uint32_t row = d.zb == 4 ? *reinterpret_cast<const uint32_t*>(zr)
-                                       : *reinterpret_cast<const uint16_t*>(zr);
-        const __half2* zs = cb.zsz + (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * d.sr;
+        const uint8_t* zr = cb.zcode + row * d.zb;
+        const uint32_t zrow = d.zb == 4 ? *reinterpret_cast<const uint32_t*>(zr)
+                                        : *reinterpret_cast<const uint16_t*>(zr);
+        const __half2* zs = cb.zsz + gidx * d.sr;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           if (j < d.sr) {
             const float2 sz = __half22float2(zs[j]);
-            const uint32_t code = (row >> (j * d.sq)) & ((1u << d.sq) - 1u);
+            const uint32_t code = (zrow >> (j * d.sq)) & ((1u << d.sq) - 1u);
             zhat[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
           }
       }
-      const uint32_t* kr = cb.kcode + (static_cast<size_t>(bh) * d.lcap + i) * d.kw;
-      const __half* ks = reinterpret_cast<const __half*>(cb.ksz) +
-                         (static_cast<size_t>(bh) * (d.lcap / d.gk) + i / d.gk) * 2 * d.dk;
-      const uint32_t* vr = cb.vcode + (static_cast<size_t>(bh) * d.lcap + i) * d.vw;
-      const __half2* vs = cb.vsz + (static_cast<size_t>(bh) * d.lcap + i) * d.nvg;
+      const uint32_t* kr = cb.kcode + row * d.kw;
+      const __half* ks = reinterpret_cast<const __half*>(cb.ksz) + gidx * 2 * d.dk;
+      const uint32_t* vr = cb.vcode + row * d.vw;
+      const __half2* vs = cb.vsz + row * d.nvg;
 #pragma unroll
       for (int j = 0; j < kMaxC; ++j) {
         kh[j] = 0.0f;

@@ -16,15 +16,22 @@
 struct kvq_cache {
   kvq::Dims d;
   kvq_buffers buf;
-  std::vector<int> L;   // tokens of each sequence
+  std::vector<int> L;   // tokens of each sequence (0: empty)
   std::vector<int> Q;   // quantized prefix of each sequence (its retained set follows from it)
+  std::vector<int> table;   // paged: host copy of the block table [B][max_groups]
+  std::vector<int> free_pages;   // paged: pages not in use, the next one handed out last
+  std::vector<int> held;         // paged: pages of each sequence, its table entries [0, held)
   int sm_count;
   int kernel;     // KVQ_KERNEL_*
-  bool prefilled;
   bool stall_next;  // test hook armed by kvq_debug_stall_next_decode
   bool uniform() const {
     for (size_t b = 1; b < L.size(); ++b)
       if (L[b] != L[0]) return false;
+    return true;
+  }
+  bool ready() const {   // every sequence holds at least one token
+    for (int x : L)
+      if (x < 1) return false;
     return true;
   }
 };
@@ -85,11 +92,21 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
     if (row_bits != 16 && row_bits != 32) return KVQ_ERR_UNSUPPORTED;
   }
   if (c->rot_keys != 0 && c->rot_keys != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->paged != 0 && c->paged != 1) return KVQ_ERR_INVALID_ARG;
+  if (c->paged) {
+    if (raw) return KVQ_ERR_UNSUPPORTED;
+    if (c->n_pages < 1) return KVQ_ERR_INVALID_ARG;
+    if (static_cast<long long>(c->n_pages) * c->n_kv_heads * c->group_k >= (1LL << 30))
+      return KVQ_ERR_UNSUPPORTED;
+  }
   // every element index must fit comfortably in 64 bits and every position in int
   const long long lcap = raw ? c->max_context
                              : (static_cast<long long>(c->max_context) + c->group_k - 1) /
                                    c->group_k * c->group_k;
   if (lcap > (1LL << 30)) return KVQ_ERR_UNSUPPORTED;
+  // group indices (b, h, g) of an unpaged cache fit in 31 bits
+  if (!raw && static_cast<long long>(c->batch) * c->n_kv_heads * (lcap / c->group_k) >= (1LL << 31))
+    return KVQ_ERR_UNSUPPORTED;
   kvq::Dims x;
   x.B = c->batch;
   x.Hq = c->n_q_heads;
@@ -105,6 +122,8 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
   x.log_retain = raw ? 0 : c->log_retain;
   x.max_context = c->max_context;
   x.lcap = static_cast<int>(lcap);
+  x.paged = c->paged;
+  x.max_groups = static_cast<int>(lcap / x.gk);
   x.cap = raw ? c->max_context : c->window + c->group_k;
   x.kw = raw ? 0 : c->d_k * c->k_bits / 32;
   x.vw = raw ? 0 : c->d_v * c->v_bits / 32;
@@ -244,17 +263,60 @@ void sequence_view(const kvq_cache* c, int b, kvq::Dims* d1, kvq_buffers* b1) {
   const size_t bh = static_cast<size_t>(b) * d.Hkv;
   auto at = [](void* p, size_t bytes) -> void* { return p ? static_cast<char*>(p) + bytes : nullptr; };
   *b1 = c->buf;
-  b1->kcode = at(c->buf.kcode, bh * d.lcap * d.kw * 4);
-  b1->ksz = at(c->buf.ksz, bh * (d.lcap / d.gk) * d.dk * 4);
-  b1->vcode = at(c->buf.vcode, bh * d.lcap * d.vw * 4);
-  b1->vsz = at(c->buf.vsz, bh * d.lcap * d.nvg * 4);
+  if (d.paged) {
+    // the pools are shared; the view's block table is row b
+    b1->block_table = at(c->buf.block_table, static_cast<size_t>(b) * d.max_groups * 4);
+  } else {
+    b1->kcode = at(c->buf.kcode, bh * d.lcap * d.kw * 4);
+    b1->ksz = at(c->buf.ksz, bh * (d.lcap / d.gk) * d.dk * 4);
+    b1->vcode = at(c->buf.vcode, bh * d.lcap * d.vw * 4);
+    b1->vsz = at(c->buf.vsz, bh * d.lcap * d.nvg * 4);
+    b1->zcode = at(c->buf.zcode, bh * d.lcap * d.zb);
+    b1->zsz = at(c->buf.zsz, bh * (d.lcap / d.gk) * d.sr * 4);
+  }
   b1->win_k = at(c->buf.win_k, bh * d.cap * d.dk * 2);
   b1->win_v = at(c->buf.win_v, bh * d.cap * d.dv * 2);
   b1->ret_k = at(c->buf.ret_k, bh * kvq::kMaxRetained * d.dk * 2);
   b1->ret_v = at(c->buf.ret_v, bh * kvq::kMaxRetained * d.dv * 2);
-  b1->zcode = at(c->buf.zcode, bh * d.lcap * d.zb);
-  b1->zsz = at(c->buf.zsz, bh * (d.lcap / d.gk) * d.sr * 4);
 }
+
+// ---- the page pool of a paged cache ----
+// Pages sequence b holds (those of its quantized groups, once their launches are queued).
+int pages_held(const kvq_cache* c, int b) { return c->d.paged ? c->held[b] : 0; }
+
+void release_pages(kvq_cache* c, int b) {
+  const int mg = c->d.max_groups;
+  for (int g = pages_held(c, b) - 1; g >= 0; --g) {
+    c->free_pages.push_back(c->table[b * mg + g]);
+    c->table[b * mg + g] = -1;
+  }
+  if (c->d.paged) c->held[b] = 0;
+}
+
+// Collects block-table writes and launches them in batches of a launch parameter's size.
+struct TableWriter {
+  kvq_cache* c;
+  cudaStream_t s;
+  kvq::TableWrites tw;
+  int rc = KVQ_OK;
+  TableWriter(kvq_cache* c_, cudaStream_t s_) : c(c_), s(s_) { tw.n = 0; }
+  int flush() {
+    if (tw.n > 0 && !rc)
+      rc = check_cuda(kvq::launch_table_writes(static_cast<int*>(c->buf.block_table), tw, s));
+    tw.n = 0;
+    return rc;
+  }
+  // hands sequence b the next free page for its next group (the caller checked there is one)
+  void assign(int b) {
+    const int page = c->free_pages.back();
+    c->free_pages.pop_back();
+    const int idx = b * c->d.max_groups + c->held[b]++;
+    c->table[idx] = page;
+    tw.idx[tw.n] = idx;
+    tw.page[tw.n] = page;
+    if (++tw.n == static_cast<int>(sizeof(tw.idx) / sizeof(tw.idx[0]))) flush();
+  }
+};
 
 kvq::CacheBufs cache_bufs(const kvq_cache* c) {
   kvq::CacheBufs b;
@@ -269,6 +331,7 @@ kvq::CacheBufs cache_bufs(const kvq_cache* c) {
   b.zcode = static_cast<const uint8_t*>(c->buf.zcode);
   b.zsz = static_cast<const __half2*>(c->buf.zsz);
   b.side_u = static_cast<const float*>(c->buf.side_u);
+  b.table = static_cast<const int*>(c->buf.block_table);
   return b;
 }
 
@@ -282,9 +345,9 @@ const char* kvq_strerror(int code) {
     case KVQ_ERR_INVALID_ARG: return "invalid argument";
     case KVQ_ERR_UNSUPPORTED: return "unsupported shape, bit width or group size";
     case KVQ_ERR_ALIGN: return "device pointer not 16-byte aligned";
-    case KVQ_ERR_CAPACITY: return "cache capacity (max_context) exceeded";
+    case KVQ_ERR_CAPACITY: return "cache capacity (max_context or page pool) exceeded";
     case KVQ_ERR_WORKSPACE: return "decode workspace too small";
-    case KVQ_ERR_STATE: return "cache not prefilled";
+    case KVQ_ERR_STATE: return "a sequence of the cache is empty";
     case KVQ_ERR_CUDA: return "CUDA runtime error";
     default: return "unknown error";
   }
@@ -299,17 +362,21 @@ int kvq_buffer_sizes(const kvq_config* cfg, kvq_sizes* out) {
   kvq_sizes s;
   memset(&s, 0, sizeof(s));
   if (d.quantized()) {
-    s.kcode = bh * d.lcap * d.kw * 4;
-    s.ksz = bh * (d.lcap / d.gk) * d.dk * 4;
-    s.vcode = bh * d.lcap * d.vw * 4;
-    s.vsz = bh * d.lcap * d.nvg * 4;
+    // token rows and groups of the quantized buffers: per (b, h) region, or per page
+    const size_t groups = d.paged ? static_cast<size_t>(cfg->n_pages) * d.Hkv : bh * d.max_groups;
+    const size_t rows = groups * d.gk;
+    s.kcode = rows * d.kw * 4;
+    s.ksz = groups * d.dk * 4;
+    s.vcode = rows * d.vw * 4;
+    s.vsz = rows * d.nvg * 4;
     s.ret_k = bh * kvq::kMaxRetained * d.dk * 2;
     s.ret_v = bh * kvq::kMaxRetained * d.dv * 2;
     if (d.sr) {
-      s.zcode = bh * d.lcap * d.zb;
-      s.zsz = bh * (d.lcap / d.gk) * d.sr * 4;
+      s.zcode = rows * d.zb;
+      s.zsz = groups * d.sr * 4;
       s.side_u = static_cast<size_t>(d.Hkv) * d.dk * d.sr * 4;
     }
+    if (d.paged) s.block_table = static_cast<size_t>(d.B) * d.max_groups * 4;
   }
   s.win_k = bh * d.cap * d.dk * 2;
   s.win_v = bh * d.cap * d.dv * 2;
@@ -336,8 +403,10 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
     for (const void* p : z)
       if (!p) return KVQ_ERR_INVALID_ARG;
   }
+  if (d.paged && !bufs->block_table) return KVQ_ERR_INVALID_ARG;
   const void* all[] = {bufs->kcode, bufs->ksz, bufs->vcode, bufs->vsz, bufs->win_k, bufs->win_v,
-                       bufs->ret_k, bufs->ret_v, bufs->zcode, bufs->zsz, bufs->side_u};
+                       bufs->ret_k, bufs->ret_v, bufs->zcode, bufs->zsz, bufs->side_u,
+                       bufs->block_table};
   for (const void* p : all)
     if (p && !aligned16(p)) return KVQ_ERR_ALIGN;
   int dev = 0, sms = 0;
@@ -350,11 +419,17 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
   if (!c) return KVQ_ERR_INVALID_ARG;
   c->d = d;
   c->buf = *bufs;
+  if (!d.paged) c->buf.block_table = nullptr;
   c->L.assign(d.B, 0);
   c->Q.assign(d.B, 0);
+  if (d.paged) {
+    c->table.assign(static_cast<size_t>(d.B) * d.max_groups, -1);
+    c->held.assign(d.B, 0);
+    // handed out from the back: a fresh pool gives pages 0, 1, 2, ... in order
+    for (int p = cfg->n_pages - 1; p >= 0; --p) c->free_pages.push_back(p);
+  }
   c->sm_count = sms;
   c->kernel = KVQ_KERNEL_AUTO;
-  c->prefilled = false;
   c->stall_next = false;
   *out = c;
   return KVQ_OK;
@@ -380,20 +455,21 @@ int prefill_rows(const kvq::Dims& d, const kvq_buffers& buf, const __half* kh, c
                  int src_rows, int L, cudaStream_t s) {
   const int Q = quantized_prefix(d, L);
   const int nbh = d.B * d.Hkv;
+  const int* table = static_cast<const int*>(buf.block_table);
   int rc = KVQ_OK;
   if (Q > 0) {
     rc = check_cuda(kvq::launch_quantize_keys(d, kh, src_rows, 0, Q / d.gk,
                                               static_cast<uint32_t*>(buf.kcode),
-                                              static_cast<__half2*>(buf.ksz), d.rot != 0, s));
+                                              static_cast<__half2*>(buf.ksz), table, d.rot != 0, s));
     if (!rc)
       rc = check_cuda(kvq::launch_quantize_side(
           d, kh, src_rows, 0, Q / d.gk, static_cast<const uint32_t*>(buf.kcode),
           static_cast<const __half2*>(buf.ksz), static_cast<const float*>(buf.side_u),
-          static_cast<uint8_t*>(buf.zcode), static_cast<__half2*>(buf.zsz), d.rot != 0, s));
+          static_cast<uint8_t*>(buf.zcode), static_cast<__half2*>(buf.zsz), table, d.rot != 0, s));
     if (!rc)
       rc = check_cuda(kvq::launch_quantize_values(d, vh, src_rows, 0, Q,
                                                   static_cast<uint32_t*>(buf.vcode),
-                                                  static_cast<__half2*>(buf.vsz), s));
+                                                  static_cast<__half2*>(buf.vsz), table, s));
   }
   if (!rc)
     rc = check_cuda(d.rot ? kvq::launch_rotate_key_rows(d, kh, src_rows, Q, static_cast<__half*>(buf.win_k),
@@ -424,17 +500,18 @@ int prefill_rows(const kvq::Dims& d, const kvq_buffers& buf, const __half* kh, c
 int quantize_window_group(const kvq::Dims& d, const kvq_buffers& buf, int Q, cudaStream_t s) {
   __half* wk = static_cast<__half*>(buf.win_k);
   __half* wv = static_cast<__half*>(buf.win_v);
+  const int* table = static_cast<const int*>(buf.block_table);
   int rc = check_cuda(kvq::launch_quantize_keys(d, wk, d.cap, Q / d.gk, 1,
                                                 static_cast<uint32_t*>(buf.kcode),
-                                                static_cast<__half2*>(buf.ksz), false, s));
+                                                static_cast<__half2*>(buf.ksz), table, false, s));
   if (!rc)
     rc = check_cuda(kvq::launch_quantize_side(
         d, wk, d.cap, Q / d.gk, 1, static_cast<const uint32_t*>(buf.kcode),
         static_cast<const __half2*>(buf.ksz), static_cast<const float*>(buf.side_u),
-        static_cast<uint8_t*>(buf.zcode), static_cast<__half2*>(buf.zsz), false, s));
+        static_cast<uint8_t*>(buf.zcode), static_cast<__half2*>(buf.zsz), table, false, s));
   if (!rc)
     rc = check_cuda(kvq::launch_quantize_values(d, wv, d.cap, Q, d.gk, static_cast<uint32_t*>(buf.vcode),
-                                                static_cast<__half2*>(buf.vsz), s));
+                                                static_cast<__half2*>(buf.vsz), table, s));
   if (!rc && d.log_retain) {
     const std::vector<int> old_ret = retained_positions(Q);
     const std::vector<int> nr = retained_positions(Q + d.gk);
@@ -456,22 +533,62 @@ int quantize_window_group(const kvq::Dims& d, const kvq_buffers& buf, int Q, cud
   return rc;
 }
 
+// Prefill of every sequence: k, v [B][Hkv][L_max][d], sequence b's first lengths[b] rows.
+// A paged cache takes back all pages first and hands out Q_b / gk to each sequence.
+int prefill_all(kvq_cache* c, const __half* kh, const __half* vh, int L_max, const int* lengths,
+                cudaStream_t s) {
+  const kvq::Dims& d = c->d;
+  if (d.paged) {
+    long long need = 0, avail = static_cast<long long>(c->free_pages.size());
+    for (int b = 0; b < d.B; ++b) {
+      need += quantized_prefix(d, lengths[b]) / d.gk;
+      avail += pages_held(c, b);
+    }
+    if (need > avail) return KVQ_ERR_CAPACITY;
+  }
+  for (int b = 0; b < d.B; ++b) {
+    release_pages(c, b);
+    c->L[b] = c->Q[b] = 0;
+  }
+  if (d.paged) {
+    TableWriter tw(c, s);
+    for (int b = 0; b < d.B; ++b)
+      for (int g = 0; g < quantized_prefix(d, lengths[b]) / d.gk; ++g) tw.assign(b);
+    if (tw.flush()) return tw.rc;
+  }
+  bool same = true;
+  for (int b = 1; b < d.B; ++b) same = same && lengths[b] == lengths[0];
+  if (same) {
+    const int rc = prefill_rows(d, c->buf, kh, vh, L_max, lengths[0], s);
+    if (rc) return rc;
+  } else {
+    for (int b = 0; b < d.B; ++b) {
+      kvq::Dims d1;
+      kvq_buffers b1;
+      sequence_view(c, b, &d1, &b1);
+      const size_t off = static_cast<size_t>(b) * d.Hkv * L_max;
+      const int rc = prefill_rows(d1, b1, kh + off * d.dk, vh + off * d.dv, L_max, lengths[b], s);
+      if (rc) return rc;
+    }
+  }
+  for (int b = 0; b < d.B; ++b) {
+    c->L[b] = lengths[b];
+    c->Q[b] = quantized_prefix(d, lengths[b]);
+  }
+  return KVQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
 
 int kvq_quantize_prefill(kvq_cache* c, const void* k, const void* v, int L, void* stream) {
   if (!c || !k || !v) return KVQ_ERR_INVALID_ARG;
-  const kvq::Dims& d = c->d;
-  if (L < 1 || L > d.max_context) return KVQ_ERR_INVALID_ARG;
+  if (L < 1 || L > c->d.max_context) return KVQ_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
-  const int rc = prefill_rows(d, c->buf, static_cast<const __half*>(k), static_cast<const __half*>(v), L,
-                              L, static_cast<cudaStream_t>(stream));
-  if (rc) return rc;
-  c->L.assign(d.B, L);
-  c->Q.assign(d.B, quantized_prefix(d, L));
-  c->prefilled = true;
-  return KVQ_OK;
+  const std::vector<int> lengths(c->d.B, L);
+  return prefill_all(c, static_cast<const __half*>(k), static_cast<const __half*>(v), L, lengths.data(),
+                     static_cast<cudaStream_t>(stream));
 }
 
 int kvq_quantize_prefill_ragged(kvq_cache* c, const void* k, const void* v, int L_max,
@@ -486,32 +603,60 @@ int kvq_quantize_prefill_ragged(kvq_cache* c, const void* k, const void* v, int 
       if (lengths[b] != lengths[0]) return KVQ_ERR_UNSUPPORTED;
   }
   if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
+  return prefill_all(c, static_cast<const __half*>(k), static_cast<const __half*>(v), L_max, lengths,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int kvq_prefill_sequence(kvq_cache* c, int b, const void* k, const void* v, int L, void* stream) {
+  if (!c || !k || !v) return KVQ_ERR_INVALID_ARG;
+  const kvq::Dims& d = c->d;
+  if (b < 0 || b >= d.B || L < 1 || L > d.max_context) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
+  const int Q = quantized_prefix(d, L);
+  if (d.paged && Q / d.gk > static_cast<int>(c->free_pages.size()) + pages_held(c, b))
+    return KVQ_ERR_CAPACITY;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const __half* kh = static_cast<const __half*>(k);
-  const __half* vh = static_cast<const __half*>(v);
-  for (int b = 0; b < d.B; ++b) {
-    kvq::Dims d1;
-    kvq_buffers b1;
-    sequence_view(c, b, &d1, &b1);
-    const size_t off = static_cast<size_t>(b) * d.Hkv * L_max;
-    const int rc = prefill_rows(d1, b1, kh + off * d.dk, vh + off * d.dv, L_max, lengths[b], s);
-    if (rc) return rc;
+  release_pages(c, b);
+  c->L[b] = c->Q[b] = 0;
+  if (d.paged) {
+    TableWriter tw(c, s);
+    for (int g = 0; g < Q / d.gk; ++g) tw.assign(b);
+    if (tw.flush()) return tw.rc;
   }
-  for (int b = 0; b < d.B; ++b) {
-    c->L[b] = lengths[b];
-    c->Q[b] = quantized_prefix(d, lengths[b]);
-  }
-  c->prefilled = true;
+  kvq::Dims d1;
+  kvq_buffers b1;
+  sequence_view(c, b, &d1, &b1);
+  const int rc = prefill_rows(d1, b1, static_cast<const __half*>(k), static_cast<const __half*>(v), L, L, s);
+  if (rc) return rc;
+  c->L[b] = L;
+  c->Q[b] = Q;
   return KVQ_OK;
+}
+
+int kvq_release_sequence(kvq_cache* c, int b) {
+  if (!c || b < 0 || b >= c->d.B) return KVQ_ERR_INVALID_ARG;
+  release_pages(c, b);
+  c->L[b] = c->Q[b] = 0;
+  return KVQ_OK;
+}
+
+int kvq_free_pages(const kvq_cache* c) {
+  if (!c) return KVQ_ERR_INVALID_ARG;
+  return static_cast<int>(c->free_pages.size());
 }
 
 int kvq_append_ragged(kvq_cache* c, const void* k_new, const void* v_new, const unsigned char* active,
                       void* stream) {
   if (!c || !k_new || !v_new) return KVQ_ERR_INVALID_ARG;
-  if (!c->prefilled) return KVQ_ERR_STATE;
   const kvq::Dims& d = c->d;
-  for (int b = 0; b < d.B; ++b)
-    if ((!active || active[b]) && c->L[b] + 1 > d.max_context) return KVQ_ERR_CAPACITY;
+  int crossing = 0;   // sequences whose window spills a group into the quantized prefix
+  for (int b = 0; b < d.B; ++b) {
+    if (active && !active[b]) continue;
+    if (c->L[b] < 1) return KVQ_ERR_STATE;
+    if (c->L[b] + 1 > d.max_context) return KVQ_ERR_CAPACITY;
+    crossing += d.quantized() && c->L[b] + 1 - c->Q[b] == d.R + d.gk;
+  }
+  if (d.paged && crossing > static_cast<int>(c->free_pages.size())) return KVQ_ERR_CAPACITY;
   if (!aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_ALIGN;
   bool all = true;
   for (int b = 0; b < d.B && active; ++b) all = all && active[b];
@@ -544,6 +689,13 @@ int kvq_append_ragged(kvq_cache* c, const void* k_new, const void* v_new, const 
                                              static_cast<__half*>(c->buf.win_v), slots, s));
   }
   if (rc) return rc;
+  // new pages for the groups that spill (paged caches), written before they are quantized
+  if (d.paged && crossing) {
+    TableWriter tw(c, s);
+    for (int b = 0; b < d.B; ++b)
+      if ((!active || active[b]) && c->L[b] + 1 - c->Q[b] == d.R + d.gk) tw.assign(b);
+    if (tw.flush()) return tw.rc;
+  }
   if (lockstep) {
     // every sequence in step: one launch per kernel for the whole batch
     const int L = c->L[0] + 1;
@@ -584,7 +736,7 @@ int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, 
 
 int kvq_get_plan(const kvq_cache* c, int num_splits, kvq_plan* out) {
   if (!c || !out) return KVQ_ERR_INVALID_ARG;
-  if (!c->prefilled) return KVQ_ERR_STATE;
+  if (!c->ready()) return KVQ_ERR_STATE;
   return plan_cache(c, num_splits, use_tensor_kernel(c), out);
 }
 
@@ -600,7 +752,7 @@ int kvq_decode_workspace_size(const kvq_cache* c, int num_splits, size_t* bytes)
 int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace,
                          size_t workspace_bytes, int num_splits, void* stream) {
   if (!c || !q || !out || !workspace || num_splits < 0) return KVQ_ERR_INVALID_ARG;
-  if (!c->prefilled) return KVQ_ERR_STATE;
+  if (!c->ready()) return KVQ_ERR_STATE;
   if (!aligned16(q) || !aligned16(out) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
   const kvq::Dims& d = c->d;
   kvq_plan plan;

@@ -24,8 +24,23 @@ struct Dims {
   int rot;    // key-only rotation on/off
   unsigned int rot_signs[8];   // bit c set: sigma_c = -1
   float rot_inv_ck, rot_inv_cq;   // 1/c_k (keys), 1/c_q (queries): powers of two
+  int paged;        // quantized groups in a pool of pages, located through a block table
+  int max_groups;   // groups per sequence: lcap / gk (block-table row length)
   bool quantized() const { return kb != 16; }
 };
+
+// Where key group g of (b, kv head h) lives in the quantized buffers: the token row of its
+// first token in the code arrays (rows of kw / vw words, of zb side bytes, of nvg value
+// (scale, zero) pairs) and its index in the per-group arrays (key and side (scale, zero)).
+// Unpaged: region (b, h) of lcap rows; paged: page table[b][g], laid out [page][h][gk].
+__host__ __device__ inline size_t group_row(const Dims& d, const int* table, int b, int h, int g) {
+  if (d.paged) return (static_cast<size_t>(table[b * d.max_groups + g]) * d.Hkv + h) * d.gk;
+  return static_cast<size_t>(b * d.Hkv + h) * d.lcap + static_cast<size_t>(g) * d.gk;
+}
+__host__ __device__ inline size_t group_index(const Dims& d, const int* table, int b, int h, int g) {
+  if (d.paged) return static_cast<size_t>(table[b * d.max_groups + g]) * d.Hkv + h;
+  return static_cast<size_t>(b * d.Hkv + h) * d.max_groups + g;
+}
 
 // The rotation of one key or query row of d = 32 * M channels by a warp, lane l holding
 // channels l + 32 m in x[m]: x <- FWHT(sigma * x) * inv_c in fp32, butterflies of span
@@ -134,6 +149,14 @@ struct CacheBufs {
   const uint8_t* zcode;   // side codes (null without a side code)
   const __half2* zsz;     // side (scale, zero) per key group and coordinate
   const float* side_u;    // basis U_h, fp32 [Hkv][dk][sr]
+  const int* table;       // block table of a paged cache, int32 [B][max_groups]
+};
+
+// Block-table entries to write (a launch parameter): table[idx[i]] = page[i].
+struct TableWrites {
+  int n;
+  int idx[480];
+  int page[480];
 };
 
 // Workspace layout: [status u32, padded to 256 B][(m, l) float2 per partial][o floats]
@@ -150,16 +173,19 @@ Partials workspace_views(const Dims& d, int splits, void* ws);
 // rotate: src holds unrotated keys that are rotated on the fly (prefill); otherwise src
 // already holds the cached (rotated or not) keys (the window, on append)
 cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
-                                 int n_groups, uint32_t* kcode, __half2* ksz, bool rotate,
-                                 cudaStream_t s);
+                                 int n_groups, uint32_t* kcode, __half2* ksz, const int* table,
+                                 bool rotate, cudaStream_t s);
+cudaError_t launch_table_writes(int* table, const TableWrites& tw, cudaStream_t s);
+
 // Side codes of key groups [g_begin, g_begin + n_groups) whose base codes and (scale, zero)
 // are already in kcode / ksz (same stream); keys read from src as for launch_quantize_keys.
 cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows, int g_begin,
                                  int n_groups, const uint32_t* kcode, const __half2* ksz,
-                                 const float* side_u, uint8_t* zcode, __half2* zsz, bool rotate,
-                                 cudaStream_t s);
+                                 const float* side_u, uint8_t* zcode, __half2* zsz, const int* table,
+                                 bool rotate, cudaStream_t s);
 cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_rows, int t_begin,
-                                   int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s);
+                                   int n_tokens, uint32_t* vcode, __half2* vsz, const int* table,
+                                   cudaStream_t s);
 cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,
                              int dst_rows, int dst_base, int n, int d, int nbh, cudaStream_t s);
 // Rotated key rows (one warp per row): dst[bh][dst row i] = rotate(src[bh][src row i]) for

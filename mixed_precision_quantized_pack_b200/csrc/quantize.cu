@@ -55,7 +55,7 @@ template <int BITS, bool ROT>
 __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_rows, int dk,
                                      int gk, int g_begin, int n_groups, int lcap,
                                      uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
-                                     Dims d) {
+                                     const int* __restrict__ table, Dims d) {
   extern __shared__ __half sm_rot[];
   const int c = threadIdx.x;
   const int gi = blockIdx.x * blockDim.y + threadIdx.y;
@@ -103,19 +103,20 @@ __global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_row
     const int wd = c / per_w, r = c % per_w;
     const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
     const int slot = pos * 2 * per_w + (r % half_w) * 2 + r / half_w;
-    __half* blk = reinterpret_cast<__half*>(ksz) + (static_cast<size_t>(bh) * (lcap / gk) + g) * 2 * dk;
+    __half* blk = reinterpret_cast<__half*>(ksz) + group_index(d, table, bh / d.Hkv, bh % d.Hkv, g) * 2 * dk;
     blk[slot] = __low2half(gp.sz);
     blk[slot + per_w] = __high2half(gp.sz);
   }
   constexpr int per = 32 / BITS;                    // channels per word
   const int words = dk / per;
+  const size_t row0 = group_row(d, table, bh / d.Hkv, bh % d.Hkv, g);
   for (int t = 0; t < gk; ++t) {
     const float x = key(t);
     uint32_t part = quant_code<BITS>(x, gp) << ((c % per) * BITS);
 #pragma unroll
     for (int off = 1; off < per; off <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, off);
     if (c % per == 0)
-      kcode[(static_cast<size_t>(bh) * lcap + g * gk + t) * words + c / per] = part;
+      kcode[(row0 + t) * words + c / per] = part;
   }
 }
 
@@ -135,7 +136,8 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
                                      const uint32_t* __restrict__ kcode,
                                      const __half2* __restrict__ ksz,
                                      const float* __restrict__ side_u,
-                                     uint8_t* __restrict__ zcode, __half2* __restrict__ zsz, Dims d) {
+                                     uint8_t* __restrict__ zcode, __half2* __restrict__ zsz,
+                                     const int* __restrict__ table, Dims d) {
   extern __shared__ float sm_side[];
   __shared__ float2 params[8];
   const int es = dk + 1;
@@ -148,8 +150,9 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
   const size_t base = static_cast<size_t>(bh) * src_rows;
   const int per = 32 / kb, half = per / 2, words = dk / per;
   const int quarter = words % 4 == 0 ? words / 4 : 0;
-  const __half* blk =
-      reinterpret_cast<const __half*>(ksz) + (static_cast<size_t>(bh) * (lcap / gk) + g) * 2 * dk;
+  const size_t row0 = group_row(d, table, bh / hkv, h, g);
+  const size_t gidx = group_index(d, table, bh / hkv, h, g);
+  const __half* blk = reinterpret_cast<const __half*>(ksz) + gidx * 2 * dk;
   // the cached key of token t, channel c: the source key, or its rotation (ROT: rotated
   // by warps into e, then read back from there)
   if constexpr (ROT) {
@@ -175,7 +178,7 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
       const int row = (g * gk + t) % src_rows;
       x = __half2float(src[(base + row) * dk + c]);
     }
-    const uint32_t w = kcode[(static_cast<size_t>(bh) * lcap + g * gk + t) * words + c / per];
+    const uint32_t w = kcode[(row0 + t) * words + c / per];
     const uint32_t code = (w >> ((c % per) * kb)) & ((1u << kb) - 1u);
     // the channel's (scale, zero) slots in the group's paired, quarter-interleaved block
     const int wd = c / per, r = c % per;
@@ -209,7 +212,7 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
     }
     if (lane == 0) {
       const GroupParams gp = group_params<SQ>(mn, mx);
-      zsz[(static_cast<size_t>(bh) * (lcap / gk) + g) * sr + i] = gp.sz;
+      zsz[gidx * sr + i] = gp.sz;
       params[i] = make_float2(gp.scale, gp.zero);
     }
   }
@@ -222,7 +225,7 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
       gp.zero = params[i].y;
       row |= quant_code<SQ>(y[t * sr + i], gp) << (i * SQ);
     }
-    uint8_t* dst = zcode + (static_cast<size_t>(bh) * lcap + g * gk + t) * zb;
+    uint8_t* dst = zcode + (row0 + t) * zb;
     if (zb == 4)
       *reinterpret_cast<uint32_t*>(dst) = row;
     else
@@ -234,7 +237,8 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
 template <int BITS>
 __global__ void quantize_values_kernel(const __half* __restrict__ src, int src_rows, int dv,
                                        int gv, int t_begin, int n_tokens, int nbh, int lcap,
-                                       uint32_t* __restrict__ vcode, __half2* __restrict__ vsz) {
+                                       uint32_t* __restrict__ vcode, __half2* __restrict__ vsz,
+                                       const int* __restrict__ table, Dims d) {
   const int nvg = dv / gv;
   const long long total = static_cast<long long>(nbh) * n_tokens * nvg;
   constexpr int per = 32 / BITS;
@@ -259,8 +263,9 @@ __global__ void quantize_values_kernel(const __half* __restrict__ src, int src_r
       }
     }
     const GroupParams gp = group_params<BITS>(mn, mx);
-    vsz[(static_cast<size_t>(bh) * lcap + t) * nvg + gidx] = gp.sz;
-    uint32_t* out = vcode + (static_cast<size_t>(bh) * lcap + t) * vw + gidx * (gv / per);
+    const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
+    vsz[vrow * nvg + gidx] = gp.sz;
+    uint32_t* out = vcode + vrow * vw + gidx * (gv / per);
     for (int w = 0; w < gv / per; ++w) {
       uint32_t word = 0;
       for (int k = 0; k < per; ++k) {
@@ -391,6 +396,11 @@ __global__ void update_retained_kernel(RetUpdate up, int cap, int dk, int dv,
   }
 }
 
+// Block-table entries of a paged cache: table[idx[i]] = page[i].
+__global__ void table_writes_kernel(int* __restrict__ table, TableWrites tw) {
+  for (int i = threadIdx.x; i < tw.n; i += blockDim.x) table[tw.idx[i]] = tw.page[i];
+}
+
 inline int grid_for(long long items, int block) {
   long long g = (items + block - 1) / block;
   if (g > 148LL * 32) g = 148LL * 32;
@@ -401,7 +411,8 @@ inline int grid_for(long long items, int block) {
 
 template <bool ROT>
 cudaError_t launch_quantize_keys_t(const Dims& d, const __half* src, int src_rows, int g_begin,
-                                   int n_groups, uint32_t* kcode, __half2* ksz, cudaStream_t s) {
+                                   int n_groups, uint32_t* kcode, __half2* ksz, const int* table,
+                                   cudaStream_t s) {
   const int gpb = d.dk >= 256 ? 1 : 256 / d.dk;
   dim3 block(d.dk, gpb);
   dim3 grid((n_groups + gpb - 1) / gpb, d.B * d.Hkv);
@@ -414,16 +425,22 @@ cudaError_t launch_quantize_keys_t(const Dims& d, const __half* src, int src_row
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, block, smem, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz, d);
+  kern<<<grid, block, smem, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz, table, d);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
-                                 int n_groups, uint32_t* kcode, __half2* ksz, bool rotate,
-                                 cudaStream_t s) {
+                                 int n_groups, uint32_t* kcode, __half2* ksz, const int* table,
+                                 bool rotate, cudaStream_t s) {
   if (n_groups <= 0) return cudaSuccess;
-  return rotate ? launch_quantize_keys_t<true>(d, src, src_rows, g_begin, n_groups, kcode, ksz, s)
-                : launch_quantize_keys_t<false>(d, src, src_rows, g_begin, n_groups, kcode, ksz, s);
+  return rotate ? launch_quantize_keys_t<true>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s)
+                : launch_quantize_keys_t<false>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
+}
+
+cudaError_t launch_table_writes(int* table, const TableWrites& tw, cudaStream_t s) {
+  if (tw.n <= 0) return cudaSuccess;
+  table_writes_kernel<<<1, 256, 0, s>>>(table, tw);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_rotate_key_rows(const Dims& d, const __half* src, int src_rows, int src_base,
@@ -444,8 +461,8 @@ cudaError_t launch_rotate_key_rows(const Dims& d, const __half* src, int src_row
 
 cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows, int g_begin,
                                  int n_groups, const uint32_t* kcode, const __half2* ksz,
-                                 const float* side_u, uint8_t* zcode, __half2* zsz, bool rotate,
-                                 cudaStream_t s) {
+                                 const float* side_u, uint8_t* zcode, __half2* zsz, const int* table,
+                                 bool rotate, cudaStream_t s) {
   if (n_groups <= 0 || d.sr == 0) return cudaSuccess;
   const size_t smem = (static_cast<size_t>(d.gk) * (d.dk + 1) + d.dk * d.sr + d.gk * d.sr) * 4;
   dim3 grid(n_groups, d.B * d.Hkv);
@@ -458,21 +475,22 @@ cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows,
     if (e != cudaSuccess) return e;
   }
   kern<<<grid, 256, smem, s>>>(src, src_rows, d.dk, d.kb, d.gk, g_begin, d.lcap, d.Hkv, d.sr, d.zb,
-                               kcode, ksz, side_u, zcode, zsz, d);
+                               kcode, ksz, side_u, zcode, zsz, table, d);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_rows, int t_begin,
-                                   int n_tokens, uint32_t* vcode, __half2* vsz, cudaStream_t s) {
+                                   int n_tokens, uint32_t* vcode, __half2* vsz, const int* table,
+                                   cudaStream_t s) {
   if (n_tokens <= 0) return cudaSuccess;
   const int nbh = d.B * d.Hkv;
   const long long items = static_cast<long long>(nbh) * n_tokens * d.nvg;
   const int block = 256;
   const int grid = grid_for(items, block);
   switch (d.vb) {
-    case 2: quantize_values_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
-    case 4: quantize_values_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
-    case 8: quantize_values_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz); break;
+    case 2: quantize_values_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz, table, d); break;
+    case 4: quantize_values_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz, table, d); break;
+    case 8: quantize_values_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz, table, d); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -37,13 +37,17 @@ CONFIG_FIELDS = ("batch", "n_q_heads", "n_kv_heads", "d_k", "d_v", "k_bits", "v_
                  "group_v", "window", "log_retain", "max_context", "side_rank", "side_bits",
                  "rot_keys")
 OPTIONAL_CONFIG = ("side_rank", "side_bits", "rot_keys")   # default 0: no side code, no rotation
+PAGE_CONFIG = ("paged", "n_pages")                          # default 0: one region per sequence
 BUFFER_FIELDS = ("kcode", "ksz", "vcode", "vsz", "win_k", "win_v", "ret_k", "ret_v")
 SIDE_FIELDS = ("zcode", "zsz", "side_u")
-SIZE_FIELDS = BUFFER_FIELDS + ("workspace",) + SIDE_FIELDS
+PAGE_FIELDS = ("block_table",)
+SIZE_FIELDS = BUFFER_FIELDS + ("workspace",) + SIDE_FIELDS + PAGE_FIELDS
+POINTER_FIELDS = BUFFER_FIELDS + SIDE_FIELDS + PAGE_FIELDS
 
 
 class kvq_config(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in CONFIG_FIELDS] + [("rot_signs", ctypes.c_uint * 8)]
+    _fields_ = ([(n, ctypes.c_int) for n in CONFIG_FIELDS] + [("rot_signs", ctypes.c_uint * 8)] +
+                [(n, ctypes.c_int) for n in PAGE_CONFIG])
 
 
 class kvq_sizes(ctypes.Structure):
@@ -51,7 +55,7 @@ class kvq_sizes(ctypes.Structure):
 
 
 class kvq_buffers(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_FIELDS + SIDE_FIELDS]
+    _fields_ = [(n, ctypes.c_void_p) for n in POINTER_FIELDS]
 
 
 class kvq_plan(ctypes.Structure):
@@ -94,6 +98,9 @@ _SIGNATURES = {
     "kvq_reset_status": (_I, [_P, _P]),
     "kvq_read_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint), _P]),
     "kvq_strerror": (ctypes.c_char_p, [_I]),
+    "kvq_prefill_sequence": (_I, [_P, _I, _P, _P, _I, _P]),
+    "kvq_release_sequence": (_I, [_P, _I]),
+    "kvq_free_pages": (_I, [_P]),
 }
 
 
@@ -130,6 +137,8 @@ def make_config(cfg: Dict[str, int]) -> kvq_config:
     c = kvq_config(*[int(cfg.get(n, 0) if n in OPTIONAL_CONFIG else cfg[n]) for n in CONFIG_FIELDS])
     for i, word in enumerate(list(cfg.get("rot_signs", ()))[:8]):
         c.rot_signs[i] = int(word) & 0xFFFFFFFF
+    for n in PAGE_CONFIG:
+        setattr(c, n, int(cfg.get(n, 0)))
     return c
 
 
@@ -159,7 +168,7 @@ def kvq_retained_positions(Q: int) -> List[int]:
 
 
 def kvq_cache_init(cfg: Dict[str, int], ptrs: Dict[str, int]) -> int:
-    bufs = kvq_buffers(*[ptrs.get(n) or None for n in BUFFER_FIELDS + SIDE_FIELDS])
+    bufs = kvq_buffers(*[ptrs.get(n) or None for n in POINTER_FIELDS])
     h = _P()
     _check(lib().kvq_cache_init(ctypes.byref(make_config(cfg)), ctypes.byref(bufs), ctypes.byref(h)),
            "kvq_cache_init")
@@ -187,6 +196,18 @@ def kvq_quantize_prefill_ragged(handle: int, k_ptr: int, v_ptr: int, L_max: int,
 def kvq_append_ragged(handle: int, k_ptr: int, v_ptr: int, active, stream: int) -> None:
     mask = None if active is None else (ctypes.c_ubyte * len(active))(*[1 if a else 0 for a in active])
     _check(lib().kvq_append_ragged(handle, k_ptr, v_ptr, mask, stream), "kvq_append_ragged")
+
+
+def kvq_prefill_sequence(handle: int, b: int, k_ptr: int, v_ptr: int, L: int, stream: int) -> None:
+    _check(lib().kvq_prefill_sequence(handle, int(b), k_ptr, v_ptr, int(L), stream), "kvq_prefill_sequence")
+
+
+def kvq_release_sequence(handle: int, b: int) -> None:
+    _check(lib().kvq_release_sequence(handle, int(b)), "kvq_release_sequence")
+
+
+def kvq_free_pages(handle: int) -> int:
+    return _check(lib().kvq_free_pages(handle), "kvq_free_pages")
 
 
 def kvq_get_seq_state(handle: int, b: int) -> Tuple[int, int, List[int]]:
@@ -261,14 +282,15 @@ class KVCache:
     """One attention layer's packed KV cache in device memory owned by PyTorch.
 
     With cfg["side_rank"] = r > 0 the cache keeps a side code and ``side_basis`` (fp32
-    [Hkv][d_k][r], any device) is copied into the cache's basis buffer."""
+    [Hkv][d_k][r], any device) is copied into the cache's basis buffer.  With cfg["paged"]
+    = 1 the quantized groups live in a pool of cfg["n_pages"] pages."""
 
     def __init__(self, cfg: Dict[str, int], device=None, side_basis: Optional[torch.Tensor] = None):
         self.cfg = dict(cfg)
         self.device = torch.device(device or "cuda")
         self.sizes = kvq_buffer_sizes(self.cfg)
         self.buffers: Dict[str, Optional[torch.Tensor]] = {}
-        for n in BUFFER_FIELDS + SIDE_FIELDS:
+        for n in POINTER_FIELDS:
             sz = self.sizes[n]
             self.buffers[n] = torch.zeros(sz, dtype=torch.uint8, device=self.device) if sz else None
         r = int(self.cfg.get("side_rank", 0))
@@ -328,6 +350,20 @@ class KVCache:
         kvq_quantize_prefill_ragged(self.handle, k.data_ptr(), v.data_ptr(), L_max, list(lengths),
                                     _stream(stream))
 
+    def prefill_sequence(self, b: int, k: torch.Tensor, v: torch.Tensor, stream=None) -> None:
+        """k, v [Hkv][L][d]: sequence b alone (re)starts with these L tokens."""
+        c = self.cfg
+        L = k.shape[1]
+        _fp16_cuda(k, (c["n_kv_heads"], L, c["d_k"]), "k")
+        _fp16_cuda(v, (c["n_kv_heads"], L, c["d_v"]), "v")
+        kvq_prefill_sequence(self.handle, b, k.data_ptr(), v.data_ptr(), L, _stream(stream))
+
+    def release(self, b: int) -> None:
+        kvq_release_sequence(self.handle, b)
+
+    def free_pages(self) -> int:
+        return kvq_free_pages(self.handle)
+
     def seq_state(self, b: int) -> Tuple[int, int, List[int]]:
         return kvq_get_seq_state(self.handle, b)
 
@@ -372,11 +408,16 @@ class KVCache:
         else:
             lcap = -(-c["max_context"] // gk) * gk
             cap = c["window"] + gk
+        # quantized buffers: [B][H][Lcap] regions, or a pool [n_pages][H][group_k]
+        paged = bool(c.get("paged", 0))
+        rows = (c["n_pages"], H, gk) if paged else (B, H, lcap)
+        groups = (c["n_pages"], H) if paged else (B, H, lcap // gk)
         shapes = {
-            "kcode": (torch.int32, (B, H, lcap, dk * kb // 32)),
-            "ksz": (torch.float16, (B, H, lcap // gk, 2 * dk)),
-            "vcode": (torch.int32, (B, H, lcap, dv * vb // 32)),
-            "vsz": (torch.float16, (B, H, lcap, dv // gv, 2)),
+            "kcode": (torch.int32, rows + (dk * kb // 32,)),
+            "ksz": (torch.float16, groups + (2 * dk,)),
+            "vcode": (torch.int32, rows + (dv * vb // 32,)),
+            "vsz": (torch.float16, rows + (dv // gv, 2)),
+            "block_table": (torch.int32, (B, lcap // gk)),
             "win_k": (torch.float16, (B, H, cap, dk)),
             "win_v": (torch.float16, (B, H, cap, dv)),
             "ret_k": (torch.float16, (B, H, KVQ_MAX_RETAINED, dk)),
@@ -385,9 +426,24 @@ class KVCache:
         r, sq = int(c.get("side_rank", 0)), int(c.get("side_bits", 0))
         if r:
             shapes.update({
-                "zcode": (torch.uint8, (B, H, lcap, r * sq // 8)),
-                "zsz": (torch.float16, (B, H, lcap // gk, r, 2)),
+                "zcode": (torch.uint8, rows + (r * sq // 8,)),
+                "zsz": (torch.float16, groups + (r, 2)),
                 "side_u": (torch.float32, (H, dk, r)),
             })
         dt, shape = shapes[name]
         return buf.view(dt).view(shape)
+
+    def sequence_view(self, name: str, b: int) -> torch.Tensor:
+        """Quantized buffer `name` of sequence b in the unpaged layout [H][Q_b/group_k...]:
+        for a paged cache, its pages gathered through the block table (a copy)."""
+        L, Q, _ = self.seq_state(b)
+        gk = self.cfg["group_k"]
+        t = self.view(name)
+        if not self.cfg.get("paged", 0):
+            return t[b, :, :Q] if name not in ("ksz", "zsz") else t[b, :, :Q // gk]
+        pages = self.view("block_table")[b, :Q // gk].long()
+        g = t[pages]                                   # [n_groups][H][...]
+        if name in ("ksz", "zsz"):
+            return g.transpose(0, 1).contiguous()
+        # [n][H][gk][...] -> [H][n*gk][...]
+        return g.transpose(0, 1).reshape((g.shape[1], -1) + tuple(g.shape[3:])).contiguous()

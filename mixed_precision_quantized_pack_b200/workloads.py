@@ -58,6 +58,7 @@ class Workload:
     q_in_basis: float = 0.0   # side workloads: fraction of query energy in span(U_h)
     rot_keys: int = 0     # key-only rotation, with signs drawn from rot_seed
     rot_seed: int = 0
+    paged: int = 0        # quantized groups in a page pool just large enough for max_context
 
     @property
     def n_rep(self) -> int:
@@ -71,13 +72,15 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
     def kvq_config(self, max_context: Optional[int] = None) -> dict:
+        mc = max_context if max_context is not None else self.max_context
         return dict(batch=self.batch, n_q_heads=self.n_q_heads, n_kv_heads=self.n_kv_heads,
                     d_k=self.d_k, d_v=self.d_v, k_bits=self.k_bits, v_bits=self.v_bits,
                     group_k=self.group_k, group_v=self.group_v, window=self.window,
-                    log_retain=self.log_retain,
-                    max_context=max_context if max_context is not None else self.max_context,
+                    log_retain=self.log_retain, max_context=mc,
                     side_rank=self.side_rank, side_bits=self.side_bits, rot_keys=self.rot_keys,
-                    rot_signs=rotation_signs(self.rot_seed) if self.rot_keys else [0] * 8)
+                    rot_signs=rotation_signs(self.rot_seed) if self.rot_keys else [0] * 8,
+                    paged=self.paged,
+                    n_pages=self.batch * -(-mc // self.group_k) if self.paged else 0)
 
 
 def rotation_signs(seed: int) -> List[int]:
@@ -117,6 +120,11 @@ WORKLOADS: Dict[str, Workload] = {
     "rot32k": _base(name="rot-b32-32/8-32k-k4v2-logretain", batch=32, n_q_heads=32, n_kv_heads=8,
                     d_k=128, d_v=128, context=32768, k_bits=4, v_bits=2, group_k=64, group_v=64,
                     window=128, log_retain=1, appends=0, seed=1006, rot_keys=1, rot_seed=77),
+    # the 32k case with its quantized groups in a page pool, found through a block table
+    "paged32k": _base(name="paged-b32-32/8-32k-k4v2-logretain", batch=32, n_q_heads=32,
+                      n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=4, v_bits=2,
+                      group_k=64, group_v=64, window=128, log_retain=1, appends=0, seed=1007,
+                      paged=1),
 }
 
 SWEEP_BATCHES = (1, 8, 32, 64)

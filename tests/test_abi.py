@@ -37,7 +37,7 @@ def cfg(**kw):
     return base
 
 
-@pytest.mark.parametrize("w", list(W.WORKLOADS.values()) +
+@pytest.mark.parametrize("w", [x for x in W.WORKLOADS.values() if not x.paged] +
                          [W.sweep_workload(b, kb, vb) for b in (1, 64) for kb, vb in W.SWEEP_BITS])
 def test_buffer_sizes_match_the_oracle_layout(w):
     c = w.kvq_config()
@@ -183,3 +183,63 @@ def test_ragged_calls_check_their_arguments():
     assert lib.kvq_quantize_prefill_ragged(None, None, None, 1, None, None) == K.KVQ_ERR_INVALID_ARG
     assert lib.kvq_append_ragged(None, None, None, None, None) == K.KVQ_ERR_INVALID_ARG
     assert lib.kvq_get_seq_state(None, 0, None, None, None, None) == K.KVQ_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------ paged layout ----
+@pytest.mark.parametrize("sr", [0, 4])
+def test_paged_pool_sizes_are_pages_of_the_unpaged_layout(sr):
+    """A pool of n_pages pages holds n_pages (b, group) blocks of the unpaged layout; the
+    block table is int32 [B][Lcap/group_k]."""
+    base = cfg(max_context=1000, side_rank=sr, side_bits=4 if sr else 0)
+    flat = K.kvq_buffer_sizes(base)
+    groups = base["batch"] * -(-1000 // base["group_k"])
+    for n_pages in (1, 7, groups, 3 * groups):
+        got = K.kvq_buffer_sizes(dict(base, paged=1, n_pages=n_pages))
+        for n in ("kcode", "ksz", "vcode", "vsz") + (("zcode", "zsz") if sr else ()):
+            assert got[n] * groups == flat[n] * n_pages, n
+        for n in ("win_k", "win_v", "ret_k", "ret_v", "workspace", "side_u"):
+            assert got[n] == flat[n], n
+        assert got["block_table"] == groups * 4
+    assert flat["block_table"] == 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(paged=2, n_pages=8), K.KVQ_ERR_INVALID_ARG),
+    (dict(paged=1, n_pages=0), K.KVQ_ERR_INVALID_ARG),
+    (dict(paged=1, n_pages=-3), K.KVQ_ERR_INVALID_ARG),
+    (dict(paged=1, n_pages=8, k_bits=16, v_bits=16), K.KVQ_ERR_UNSUPPORTED),
+    (dict(paged=1, n_pages=(1 << 30) // (2 * 64)), K.KVQ_ERR_UNSUPPORTED),   # 2^30 rows
+])
+def test_invalid_paged_configurations_are_rejected(bad, code):
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_buffer_sizes(cfg(**bad))
+    assert e.value.code == code
+
+
+def test_paged_caches_need_a_block_table():
+    c = cfg(paged=1, n_pages=16)
+    ptrs = {n: 4096 * (i + 1) for i, n in enumerate(K.POINTER_FIELDS)}
+    ptrs["block_table"] = 0
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_cache_init(c, ptrs)
+    assert e.value.code == K.KVQ_ERR_INVALID_ARG
+    ptrs = {n: 4096 * (i + 1) for i, n in enumerate(K.POINTER_FIELDS)}
+    ptrs["block_table"] += 4
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_cache_init(c, ptrs)
+    assert e.value.code == K.KVQ_ERR_ALIGN
+
+
+def test_sequence_calls_check_their_arguments():
+    lib = K.lib()
+    assert lib.kvq_prefill_sequence(None, 0, None, None, 1, None) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_release_sequence(None, 0) == K.KVQ_ERR_INVALID_ARG
+    assert lib.kvq_free_pages(None) == K.KVQ_ERR_INVALID_ARG
+
+
+def test_unpaged_group_indices_must_fit_31_bits():
+    # B * Hkv * Lcap / group_k >= 2^31 groups
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_buffer_sizes(cfg(batch=1 << 14, n_kv_heads=8, n_q_heads=8, group_k=16,
+                               max_context=1 << 18))
+    assert e.value.code == K.KVQ_ERR_UNSUPPORTED

@@ -43,7 +43,10 @@ def compare_state(gc: K.KVCache, oc: O.OracleCache, b_rows=None, where="", seq=N
         if c.get("side_rank", 0):
             pairs += [("zcode", slice(0, Q)), ("zsz", slice(0, Q // gk))]
         for name, sl in pairs:
-            g = gc.view(name)[rows][:, :, sl].cpu().numpy()
+            if c.get("paged"):     # the sequence's pages, gathered through the block table
+                g = np.stack([gc.sequence_view(name, b).cpu().numpy() for b in rows])
+            else:
+                g = gc.view(name)[rows][:, :, sl].cpu().numpy()
             o = getattr(oc, name)[:, :, sl]
             if b_rows is None:
                 o = o[rows]
@@ -425,3 +428,164 @@ def test_uniform_lengths_through_the_ragged_calls_match_the_plain_ones():
     for name in ("kcode", "ksz", "vcode", "vsz", "ret_k", "ret_v"):
         assert torch.equal(a.buffers[name], b.buffers[name]), name
     assert torch.equal(a.decode(inp.q[-1].cuda()), b.decode(inp.q[-1].cuda()))
+
+
+# ------------------------------------------------------------------ paged caches ----
+def paged_twins(w: W.Workload, max_context: int, n_pages: int, side_basis):
+    """A paged cache and an unpaged one of the same configuration."""
+    cfg = w.kvq_config(max_context=max_context)
+    paged = K.KVCache(dict(cfg, paged=1, n_pages=n_pages), side_basis=side_basis)
+    flat = K.KVCache(dict(cfg, paged=0, n_pages=0), side_basis=side_basis)
+    return cfg, paged, flat
+
+
+def run_paged(w: W.Workload, lengths, n_app, steps, seed, restart=None, num_splits=(0, 2)):
+    """Paged cache under ragged prefill, masked appends and (at step `restart`) a release and
+    a new prefill of sequence 1 with other tokens: every sequence's pages hold the oracle's
+    bytes, outputs match the oracle, and they equal the unpaged cache's outputs bit for bit."""
+    need_gpu()
+    L_max = max(lengths)
+    inp = W.Inputs(w.with_(context=L_max, appends=n_app), device="cpu")
+    mc = L_max + n_app + 64
+    gk = w.group_k
+    groups = len(lengths) * -(-mc // gk)
+    cfg, gp, gf = paged_twins(w, mc, groups + 3, inp.side_basis)
+    gp.prefill_ragged(inp.k.cuda(), inp.v.cuda(), lengths)
+    gf.prefill_ragged(inp.k.cuda(), inp.v.cuda(), lengths)
+    U = None if inp.side_basis is None else inp.side_basis.numpy()
+
+    def oracle_of(k, v):
+        oc = O.OracleCache(dict(cfg, batch=1), side_basis=U)
+        oc.prefill(np16(k), np16(v))
+        return oc
+
+    ocs = [oracle_of(inp.k[b:b + 1, :, :Lb], inp.v[b:b + 1, :, :Lb]) for b, Lb in enumerate(lengths)]
+    held = sum(oc.Q // gk for oc in ocs)
+    assert gp.free_pages() == groups + 3 - held
+    rng = np.random.default_rng(seed)
+    for i in range(n_app):
+        if i == restart:
+            # sequence 1 starts over with the first Lr tokens of sequence 0's prefill
+            Lr = lengths[0] - 3
+            k1 = inp.k[0, :, :Lr].contiguous()
+            v1 = inp.v[0, :, :Lr].contiguous()
+            before = gp.free_pages()
+            gp.release(1)
+            assert gp.free_pages() == before + ocs[1].Q // gk
+            gp.prefill_sequence(1, k1.cuda(), v1.cuda())
+            gf.prefill_sequence(1, k1.cuda(), v1.cuda())
+            ocs[1] = oracle_of(k1[None], v1[None])
+        active = [True] * len(lengths) if i % 3 == 0 else [bool(x) for x in rng.integers(0, 2, len(lengths))]
+        for c in (gp, gf):
+            c.append(inp.k_app[i].cuda(), inp.v_app[i].cuda(), active=active)
+        for b, oc in enumerate(ocs):
+            if active[b]:
+                oc.append(np16(inp.k_app[i][b:b + 1]), np16(inp.v_app[i][b:b + 1]))
+        assert gp.free_pages() == groups + 3 - sum(oc.Q // gk for oc in ocs)
+        if i not in steps:
+            continue
+        for b, oc in enumerate(ocs):
+            compare_state(gp, oc, b_rows=[b], where=f"paged step {i} b={b}", seq=b)
+        table = gp.view("block_table").cpu()
+        used = [int(p) for b, oc in enumerate(ocs) for p in table[b, :oc.Q // gk]]
+        assert len(set(used)) == len(used), "a page is held twice"
+        for kern in KERNELS:
+            gp.set_kernel(kern)
+            gf.set_kernel(kern)
+            # the same kernel on both layouts gives the same bits (the tensor-core kernel has
+            # no paged instances for side codes: there the paged cache runs the generic one)
+            same = gp.plan()["fast_path"] == gf.plan()["fast_path"]
+            for ns in num_splits:
+                out = gp.decode(inp.q[i].cuda(), num_splits=ns)
+                if same:
+                    assert torch.equal(out, gf.decode(inp.q[i].cuda(), num_splits=ns)), (i, kern, ns)
+                out = out.float().cpu().numpy()
+                for b, oc in enumerate(ocs):
+                    err = O.max_rel_error(out[b:b + 1], oc.decode(np16(inp.q[i][b:b + 1])))
+                    assert err <= TOL, f"paged step {i} b={b} kernel {kern} splits {ns}: {err:.3e}"
+        gp.set_kernel(K.KVQ_KERNEL_AUTO)
+        gf.set_kernel(K.KVQ_KERNEL_AUTO)
+    assert gp.status() == 0 and gf.status() == 0
+    return gp
+
+
+def test_paged_cache_tensor_kernel():
+    w = W.WORKLOADS["paged32k"].with_(batch=4, seed=251)
+    gp = run_paged(w, [1500, 700, 64, 1111], n_app=70, steps={0, 20, 21, 69}, seed=252, restart=20)
+    assert gp.plan()["fast_path"] == 1
+
+
+def test_paged_cache_with_side_code_and_rotation():
+    w = W.WORKLOADS["headq32k"].with_(batch=3, rot_keys=1, rot_seed=9, seed=261, paged=1)
+    run_paged(w, [900, 333, 1280], n_app=66, steps={1, 10, 64, 65}, seed=262, restart=10)
+
+
+def test_paged_cache_generic_shapes():
+    w = W.WORKLOADS["gqa4k"].with_(batch=3, n_q_heads=6, n_kv_heads=3, d_k=64, d_v=64, group_k=32,
+                                   group_v=32, window=48, log_retain=1, seed=271, paged=1)
+    run_paged(w, [400, 81, 257], n_app=40, steps={0, 5, 39}, seed=272, restart=5)
+
+
+@pytest.mark.parametrize("kb,vb", [(8, 4), (2, 2), (4, 4)])
+def test_paged_cache_bit_widths(kb, vb):
+    w = W.WORKLOADS["paged32k"].with_(batch=2, k_bits=kb, v_bits=vb, seed=281 + kb)
+    run_paged(w, [1000, 555], n_app=66, steps={0, 65}, seed=282)
+
+
+def test_full_size_paged_32k():
+    sampled_full_size(W.WORKLOADS["paged32k"], rows=(0, 31))
+
+
+def test_page_pool_exhaustion_changes_nothing():
+    need_gpu()
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=600, appends=80, seed=291, paged=1)
+    inp = W.Inputs(w, device="cpu")
+    gk, R = w.group_k, w.window
+    q600 = (600 - R) // gk          # groups of a 600-token prefill: 7
+    cfg = w.kvq_config(max_context=800)
+    c = K.KVCache(dict(cfg, n_pages=2 * q600), side_basis=None)
+    k, v = inp.k.cuda(), inp.v.cuda()
+    c.prefill(k, v)
+    assert c.free_pages() == 0
+    with pytest.raises(K.KVQError) as e:          # the pool is full: no room for a bigger prefill
+        c.prefill_sequence(0, torch.cat([k[0], k[1]], 1)[:, :700].contiguous(),
+                           torch.cat([v[0], v[1]], 1)[:, :700].contiguous())
+    assert e.value.code == K.KVQ_ERR_CAPACITY and c.seq_state(0)[:2] == (600, q600 * gk)
+    # appends until the window spills a group: that append needs a page and fails whole
+    n = 0
+    while True:
+        L = 600 + n
+        if L + 1 - q600 * gk == R + gk:
+            break
+        c.append(inp.k_app[n].cuda(), inp.v_app[n].cuda())
+        n += 1
+    s0, s1 = c.seq_state(0), c.seq_state(1)
+    with pytest.raises(K.KVQError) as e:
+        c.append(inp.k_app[n].cuda(), inp.v_app[n].cuda())
+    assert e.value.code == K.KVQ_ERR_CAPACITY
+    assert (c.seq_state(0), c.seq_state(1), c.free_pages()) == (s0, s1, 0)
+    # sequence 1 leaves: decode refuses an empty sequence, sequence 0 alone appends and
+    # takes one of the freed pages
+    c.release(1)
+    assert c.free_pages() == q600
+    with pytest.raises(K.KVQError) as e:
+        c.decode(inp.q[0].cuda())
+    assert e.value.code == K.KVQ_ERR_STATE
+    with pytest.raises(K.KVQError) as e:
+        c.append(inp.k_app[n].cuda(), inp.v_app[n].cuda())
+    assert e.value.code == K.KVQ_ERR_STATE
+    c.append(inp.k_app[n].cuda(), inp.v_app[n].cuda(), active=[True, False])
+    assert c.free_pages() == q600 - 1 and c.seq_state(0)[1] == (q600 + 1) * gk
+    # sequence 1 comes back and the cache decodes again, matching the oracle
+    c.prefill_sequence(1, k[1, :, :300].contiguous(), v[1, :, :300].contiguous())
+    oc0 = O.OracleCache(dict(cfg, batch=1))
+    oc0.prefill(np16(inp.k[0:1]), np16(inp.v[0:1]))
+    for i in range(n + 1):
+        oc0.append(np16(inp.k_app[i][0:1]), np16(inp.v_app[i][0:1]))
+    oc1 = O.OracleCache(dict(cfg, batch=1))
+    oc1.prefill(np16(inp.k[1:2, :, :300]), np16(inp.v[1:2, :, :300]))
+    compare_state(c, oc0, b_rows=[0], seq=0, where="after refill b=0")
+    compare_state(c, oc1, b_rows=[1], seq=1, where="after refill b=1")
+    out = c.decode(inp.q[1].cuda()).float().cpu().numpy()
+    for b, oc in enumerate((oc0, oc1)):
+        assert O.max_rel_error(out[b:b + 1], oc.decode(np16(inp.q[1][b:b + 1]))) <= TOL
