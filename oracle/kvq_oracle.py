@@ -71,6 +71,29 @@ What it computes, step by step in the order the pages give it:
    1, 2, 4, ..., d/2, each (x_i, x_{i+h}) -> (x_i + x_{i+h}, x_i - x_{i+h}).
    The rotated keys are then cached exactly as unrotated ones would be.
 
+9. Optional per-channel bit widths ("Attention-Aware Transform Coding (AATC)", §Méthodologie,
+   Allocation de Bits: reverse water-filling gives each transformed channel its own number
+   of bits, zero for the weakest, separately for keys and values).  Readings: the
+   decorrelating transform is the caller's (folded into the projections), so the cache
+   sees transformed keys and values; widths come from {0, 1, 2, 4, 8}; key channel c has
+   width kw_c, non-increasing in c (the transform orders channels by strength); the
+   channels of one value group share a width, non-increasing from group to group.  A
+   width-b channel (b >= 1) goes through the quantizer of step 3 with b bits (keys per
+   channel over G_k tokens, values per token over the group); a width-0 channel is
+   dropped: nothing is stored and it reads as 0.  A token row packs the codes channel
+   after channel, LSB-first: channel c at bit offset o_c = sum of the widths before it
+   (a power-of-two width never straddles a word because every width before it is a
+   multiple of it), in max(1, ceil(sum/32)) words.  Key (scale, zero) are stored plainly,
+   [group][d_k][2]; dropped channels and groups store (0, 0).
+   The allocation (allocate_bits) minimises sum_c w_c * 4^(-b_c) -- the high-rate
+   distortion of a b-bit uniform quantizer on a channel of weight w_c (its attention-
+   aware weight times its variance, from the caller's calibration), the whole w_c when
+   dropped -- under a budget of bits per row, as reverse water-filling does: lowering a
+   common slope ("water level"), every step of a channel's width (0->1->2->4->8) whose
+   distortion drop per bit lies above the level is taken.  Steps of equal slope are taken
+   together, zero-slope steps never, and the level stops at the first set of steps that
+   would exceed the budget (so the result is optimal for the bits it spends).
+
 Buffer formats mirror the CUDA library's so the tests can compare bytes:
   kcode u32 [B][Hkv][Lcap][d_k*kb/32]        ksz fp16 [B][Hkv][Lcap/Gk][2*d_k] (key_meta_order)
   vcode u32 [B][Hkv][Lcap][d_v*vb/32]        vsz fp16 [B][Hkv][Lcap][d_v/Gv][2]
@@ -79,6 +102,9 @@ Buffer formats mirror the CUDA library's so the tests can compare bytes:
   ret_k/v fp16 [B][Hkv][32][d] in ascending position order, ret_idx int32 list.
   zcode u8 [B][Hkv][Lcap][r*q/8]: the r side codes of a token, coordinate i at bit
         i*q of the little-endian row (pack_side); zsz fp16 [B][Hkv][Lcap/Gk][r][2].
+  Per-channel widths (k_bits = v_bits = 0, step 9): kcode u32 [B][Hkv][Lcap][Wk],
+        ksz fp16 [B][Hkv][Lcap/Gk][d_k][2], vcode u32 [B][Hkv][Lcap][Wv], vsz as above,
+        W = max(1, ceil(sum of the widths / 32)).
 """
 from __future__ import annotations
 
@@ -315,6 +341,115 @@ def unpack_codes(words: np.ndarray, bits: int) -> np.ndarray:
     return c.reshape(words.shape[:-1] + (words.shape[-1] * per,)).astype(np.uint32)
 
 
+# --------------------------------------------------- per-channel widths -----
+WIDTHS = (0, 1, 2, 4, 8)
+# distortion drop per bit of each width step of a channel of weight 1 (step 9):
+# (4^-b1 - 4^-b2) / (b2 - b1) for 0->1, 1->2, 2->4, 4->8 (exact binary fractions)
+STEP_SLOPES = ((0, 1, 0.75), (1, 2, 0.1875), (2, 4, 15.0 / 512.0), (4, 8, 255.0 / 262144.0))
+
+
+def allocation_distortion(weight, widths) -> float:
+    """sum_c w_c * 4^(-b_c), the objective of step 9's allocation."""
+    w = np.asarray(weight, np.float64)
+    b = np.asarray(widths, np.float64)
+    return float((w * np.power(4.0, -b)).sum())
+
+
+def allocate_bits(weight, budget: int, unit_bits: int = 1) -> np.ndarray:
+    """Step 9: widths in WIDTHS for units of weight w >= 0 (a key channel, or a value group
+    whose widening by one bit costs unit_bits = G_v bits) under `budget` bits per row, by
+    reverse water-filling: width steps in decreasing order of w * slope, equal slopes
+    together, until the next set does not fit; zero-slope steps are never taken."""
+    w = np.asarray(weight, np.float64)
+    steps = []
+    for c in range(w.shape[0]):
+        for b1, b2, f in STEP_SLOPES:
+            slope = float(w[c] * f)
+            if slope > 0.0:
+                steps.append((slope, c, b1, b2))
+    steps.sort(key=lambda e: -e[0])
+    widths = np.zeros(w.shape[0], np.int64)
+    used, i = 0, 0
+    while i < len(steps):
+        j = i
+        while j < len(steps) and steps[j][0] == steps[i][0]:
+            j += 1
+        cost = unit_bits * sum(b2 - b1 for _, _, b1, b2 in steps[i:j])
+        if used + cost > budget:
+            break
+        for _, c, b1, b2 in steps[i:j]:
+            assert widths[c] == b1
+            widths[c] = b2
+        used += cost
+        i = j
+    return widths
+
+
+def width_offsets(widths) -> np.ndarray:
+    """Bit offset of each channel in a packed row (step 9): the sum of the widths before it."""
+    w = np.asarray(widths, np.int64)
+    return np.concatenate([[0], np.cumsum(w)[:-1]]).astype(np.int64)
+
+
+def row_words(widths) -> int:
+    """Words of a packed row of per-channel widths: max(1, ceil(sum / 32))."""
+    return max(1, -(-int(np.sum(widths)) // 32))
+
+
+def pack_var(codes: np.ndarray, widths) -> np.ndarray:
+    """[..., d] codes -> [..., row_words] uint32, channel c at bit width_offsets[c] (step 9)."""
+    off = width_offsets(widths)
+    out = np.zeros(codes.shape[:-1] + (row_words(widths),), np.uint64)
+    for c, b in enumerate(widths):
+        if b:
+            out[..., off[c] // 32] |= codes[..., c].astype(np.uint64) << np.uint64(off[c] % 32)
+    return out.astype(np.uint32)
+
+
+def unpack_var(words: np.ndarray, widths) -> np.ndarray:
+    """Inverse of pack_var; dropped channels read code 0."""
+    off = width_offsets(widths)
+    out = np.zeros(words.shape[:-1] + (len(widths),), np.uint32)
+    for c, b in enumerate(widths):
+        if b:
+            w = words[..., off[c] // 32].astype(np.uint64)
+            out[..., c] = ((w >> np.uint64(off[c] % 32)) & np.uint64((1 << int(b)) - 1)).astype(np.uint32)
+    return out
+
+
+def quantize_keys_var(k: np.ndarray, group_k: int, widths):
+    """Keys [n][d] -> codes [n][d], sz fp16 [n/group_k][d][2]: channel c through step 3 with
+    widths[c] bits over each group of group_k tokens; dropped channels (0 bits) store 0."""
+    n, d = k.shape
+    assert n % group_k == 0
+    codes = np.zeros((n, d), np.uint32)
+    sz = np.zeros((n // group_k, d, 2), np.float16)
+    for c, b in enumerate(widths):
+        if b:
+            cc, s, z = minmax_quantize(k[:, c].reshape(n // group_k, group_k), int(b), axis=1)
+            codes[:, c] = cc.reshape(n)
+            sz[:, c, 0] = s[:, 0]
+            sz[:, c, 1] = z[:, 0]
+    return codes, sz
+
+
+def quantize_values_var(v: np.ndarray, group_v: int, widths):
+    """Values [n][d] -> codes [n][d], sz fp16 [n][d/group_v][2]: value group g through step 3
+    with the width of its channels; dropped groups store 0."""
+    n, d = v.shape
+    codes = np.zeros((n, d), np.uint32)
+    sz = np.zeros((n, d // group_v, 2), np.float16)
+    for g in range(d // group_v):
+        b = int(widths[g * group_v])
+        assert all(int(x) == b for x in widths[g * group_v:(g + 1) * group_v])
+        if b:
+            cc, s, z = minmax_quantize(v[:, g * group_v:(g + 1) * group_v], b, axis=1)
+            codes[:, g * group_v:(g + 1) * group_v] = cc
+            sz[:, g, 0] = s[:, 0]
+            sz[:, g, 1] = z[:, 0]
+    return codes, sz
+
+
 # -------------------------------------------------------------- attention -----
 def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
               extra: Optional[np.ndarray] = None) -> np.ndarray:
@@ -341,6 +476,13 @@ def buffer_bytes(cfg: dict) -> dict:
     lcap = -(-cfg["max_context"] // gk) * gk
     cap = R + gk
     sr, sq = cfg.get("side_rank", 0), cfg.get("side_bits", 0)
+    if kb == 0:      # per-channel widths (step 9)
+        wk, wv = row_words(cfg["k_widths"][:dk]), row_words(cfg["v_widths"][:dv])
+        return dict(kcode=B * H * lcap * wk * 4, ksz=B * H * (lcap // gk) * dk * 4,
+                    vcode=B * H * lcap * wv * 4, vsz=B * H * lcap * (dv // gv) * 4,
+                    win_k=B * H * cap * dk * 2, win_v=B * H * cap * dv * 2,
+                    ret_k=B * H * MAX_RETAINED * dk * 2, ret_v=B * H * MAX_RETAINED * dv * 2,
+                    zcode=0, zsz=0)
     return dict(kcode=B * H * lcap * dk * kb // 8, ksz=B * H * (lcap // gk) * dk * 4,
                 vcode=B * H * lcap * dv * vb // 8, vsz=B * H * lcap * (dv // gv) * 4,
                 win_k=B * H * cap * dk * 2, win_v=B * H * cap * dv * 2,
@@ -375,9 +517,23 @@ class OracleCache:
         self.gk, self.gv, self.R = cfg["group_k"], cfg["group_v"], cfg["window"]
         self.log_retain = bool(cfg["log_retain"]) and self.kb != 16
         self.max_context = cfg["max_context"]
+        self.var = self.kb == 0          # per-channel widths (step 9)
+        if self.var:
+            assert self.vb == 0 and not self.sr and not self.rot
+            self.kw = np.array(cfg["k_widths"][:self.dk], np.int64)
+            self.vw = np.array(cfg["v_widths"][:self.dv], np.int64)
         if self.kb == 16:
             self.lcap = self.max_context
             self.cap = self.lcap
+        elif self.var:
+            self.lcap = -(-self.max_context // self.gk) * self.gk
+            self.cap = self.R + self.gk
+            self.kcode = np.zeros((B, H, self.lcap, row_words(self.kw)), np.uint32)
+            self.ksz = np.zeros((B, H, self.lcap // self.gk, self.dk, 2), np.float16)
+            self.vcode = np.zeros((B, H, self.lcap, row_words(self.vw)), np.uint32)
+            self.vsz = np.zeros((B, H, self.lcap, self.dv // self.gv, 2), np.float16)
+            self.ret_k = np.zeros((B, H, MAX_RETAINED, self.dk), np.float16)
+            self.ret_v = np.zeros((B, H, MAX_RETAINED, self.dv), np.float16)
         else:
             self.lcap = -(-self.max_context // self.gk) * self.gk
             self.cap = self.R + self.gk
@@ -400,6 +556,14 @@ class OracleCache:
     def _quantize_rows(self, b: int, h: int, t0: int, k_rows: np.ndarray, v_rows: np.ndarray):
         """Quantize tokens [t0, t0+n) (n a multiple of G_k) and store their codes."""
         n = k_rows.shape[0]
+        if self.var:
+            kc, ksz = quantize_keys_var(k_rows, self.gk, self.kw)
+            vc, vsz = quantize_values_var(v_rows, self.gv, self.vw)
+            self.kcode[b, h, t0:t0 + n] = pack_var(kc, self.kw)
+            self.ksz[b, h, t0 // self.gk:(t0 + n) // self.gk] = ksz
+            self.vcode[b, h, t0:t0 + n] = pack_var(vc, self.vw)
+            self.vsz[b, h, t0:t0 + n] = vsz
+            return
         kc, ksz = quantize_keys(k_rows, self.gk, self.kb)
         vc, vsz = quantize_values(v_rows, self.gv, self.vb)
         self.kcode[b, h, t0:t0 + n] = pack_codes(kc, self.kb)
@@ -477,12 +641,19 @@ class OracleCache:
         kh = np.empty((L, self.dk), np.float64)
         vh = np.empty((L, self.dv), np.float64)
         if Q:
-            kc = unpack_codes(self.kcode[b, h, :Q], self.kb)                   # [Q][dk]
-            ksz = unpack_key_meta(self.ksz[b, h, :Q // self.gk], self.kb)       # [ng][dk][2]
+            if self.var:
+                kc = unpack_var(self.kcode[b, h, :Q], self.kw)
+                ksz = self.ksz[b, h, :Q // self.gk]
+            else:
+                kc = unpack_codes(self.kcode[b, h, :Q], self.kb)                   # [Q][dk]
+                ksz = unpack_key_meta(self.ksz[b, h, :Q // self.gk], self.kb)       # [ng][dk][2]
             ks = np.repeat(ksz[:, :, 0], self.gk, axis=0)
             kz = np.repeat(ksz[:, :, 1], self.gk, axis=0)
             kh[:Q] = dequantize(kc, ks, kz)
-            vc = unpack_codes(self.vcode[b, h, :Q], self.vb)                   # [Q][dv]
+            if self.var:
+                vc = unpack_var(self.vcode[b, h, :Q], self.vw)
+            else:
+                vc = unpack_codes(self.vcode[b, h, :Q], self.vb)                   # [Q][dv]
             vsz = self.vsz[b, h, :Q]                                            # [Q][ngv][2]
             vs = np.repeat(vsz[:, :, 0], self.gv, axis=1)
             vz = np.repeat(vsz[:, :, 1], self.gv, axis=1)

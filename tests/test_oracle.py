@@ -757,3 +757,198 @@ def test_rotated_appends_reach_the_same_state_as_one_prefill():
         assert np.array_equal(getattr(a, name).view(np.uint8), getattr(b, name).view(np.uint8)), name
     q = W.random_fp16((B, Hq, d), seed=163).numpy()
     assert np.array_equal(a.decode(q), b.decode(q))
+
+
+# ------------------------------------------------------- per-channel widths ----
+def test_golden_aatc_allocations_and_packing():
+    n_alloc = n_pack = 0
+    for row in read_golden("aatc_worked.txt"):
+        if row[0] == ["alloc"]:
+            w = [float(x) for x in row[1]]
+            got = O.allocate_bits(w, int(row[3][0]), int(row[2][0]))
+            assert [int(x) for x in got] == [int(x) for x in row[4]], row
+            n_alloc += 1
+        else:
+            widths = [int(x) for x in row[1]]
+            codes = np.array([[int(x) for x in row[2]]], np.uint32)
+            words = O.pack_var(codes, widths)
+            assert [int(x) for x in words[0]] == [int(x, 16) for x in row[3]], row
+            assert np.array_equal(O.unpack_var(words, widths), codes)
+            n_pack += 1
+    assert n_alloc >= 10 and n_pack >= 4
+
+
+def _all_allocations(n):
+    import itertools
+    return itertools.product(O.WIDTHS, repeat=n)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_allocation_is_optimal_for_the_bits_it_spends_brute_force(seed):
+    """No width vector that spends at most as many bits has a lower distortion (tiny n)."""
+    rng = np.random.default_rng(seed)
+    n = 3 if seed % 2 else 4
+    w = rng.lognormal(0.0, 1.5, size=n)
+    if seed == 5:
+        w[1] = w[2]                                     # a tie
+    for budget in range(0, 8 * n + 2):
+        got = O.allocate_bits(w, budget)
+        spent = int(got.sum())
+        assert spent <= budget
+        d = O.allocation_distortion(w, got)
+        for cand in _all_allocations(n):
+            if sum(cand) <= spent:
+                assert O.allocation_distortion(w, cand) >= d - 1e-12 * max(d, 1.0), (budget, cand, got)
+
+
+def test_allocation_is_monotone_and_permutation_equivariant():
+    rng = np.random.default_rng(7)
+    w = rng.lognormal(0.0, 2.0, size=64)
+    for budget in (0, 17, 64, 150, 256, 511, 512, 600):
+        got = O.allocate_bits(w, budget)
+        order = np.argsort(-w, kind="stable")
+        assert np.all(np.diff(got[order]) <= 0)                 # more weight, at least as many bits
+        perm = rng.permutation(64)
+        assert np.array_equal(O.allocate_bits(w[perm], budget), got[perm])
+        assert got.sum() <= budget
+    assert np.array_equal(O.allocate_bits(w, 10 ** 6), np.full(64, 8))
+    assert np.array_equal(O.allocate_bits(w, 0), np.zeros(64))
+
+
+def test_continuous_water_filling_is_bracketed():
+    """The allocation is a water level: every step whose drop per bit lies above the lowest
+    drop taken is taken, so a channel gets bits exactly when its first step (0 -> 1, drop
+    3w/4) lies above that level."""
+    rng = np.random.default_rng(11)
+    w = rng.lognormal(0.0, 2.0, size=128)
+    got = O.allocate_bits(w, 3 * 128)
+    # the level: the smallest drop per bit that was taken
+    taken = [w[c] * f for c in range(128) for b1, b2, f in O.STEP_SLOPES if got[c] >= b2]
+    lam = min(taken)
+    for c in range(128):
+        for b1, b2, f in O.STEP_SLOPES:
+            if w[c] * f > lam:
+                assert got[c] >= b2
+            elif w[c] * f < lam:
+                assert got[c] <= b1
+    assert np.all(got[w * 0.75 < lam] == 0)
+    assert np.all(got[w * 0.75 > lam] >= 1)
+
+
+def test_uniform_widths_reduce_to_the_fixed_width_quantizer():
+    """A map of one width b everywhere gives the fixed-width codes, (scale, zero) and packed
+    words of steps 3-4."""
+    rng = np.random.default_rng(3)
+    for b in (2, 4, 8):
+        k = (rng.standard_normal((128, 64)) * 3).astype(np.float16)
+        v = rng.standard_normal((128, 64)).astype(np.float16)
+        kc, ksz = O.quantize_keys_var(k, 32, [b] * 64)
+        kc0, ksz0 = O.quantize_keys(k, 32, b)
+        assert np.array_equal(kc, kc0) and np.array_equal(ksz.view(np.uint16), ksz0.view(np.uint16))
+        assert np.array_equal(O.pack_var(kc, [b] * 64), O.pack_codes(kc0, b))
+        vc, vsz = O.quantize_values_var(v, 16, [b] * 64)
+        vc0, vsz0 = O.quantize_values(v, 16, b)
+        assert np.array_equal(vc, vc0) and np.array_equal(vsz.view(np.uint16), vsz0.view(np.uint16))
+
+
+def test_packing_matches_big_integer_arithmetic():
+    """Each row, read as one little-endian integer, is sum_c code_c << offset_c."""
+    rng = np.random.default_rng(5)
+    for widths in ([8] * 3 + [4] * 5 + [2] * 7 + [1] * 9 + [0] * 8, [4] * 16 + [1] * 16, [1] * 32,
+                   [8, 8, 2, 2, 2, 2, 1, 1, 1, 1, 0, 0]):
+        codes = np.array([[rng.integers(0, 2 ** b) if b else 0 for b in widths] for _ in range(5)],
+                         np.uint32)
+        words = O.pack_var(codes, widths)
+        for r in range(5):
+            big = sum(int(codes[r, c]) << int(sum(widths[:c])) for c in range(len(widths)))
+            got = sum(int(words[r, j]) << (32 * j) for j in range(words.shape[1]))
+            assert got == big
+        assert words.shape[1] == max(1, -(-sum(widths) // 32))
+
+
+def var_cfg(B, Hq, Hkv, dk, dv, gk, gv, R, log_retain, max_context, kw, vw):
+    return dict(cfg_of(B, Hq, Hkv, dk, dv, 0, 0, gk, gv, R, log_retain, max_context),
+                k_widths=list(kw), v_widths=list(vw))
+
+
+def test_lossless_grid_cache_with_dropped_channels_equals_exact_attention():
+    """Inputs on each channel's (group's) grid quantize losslessly, and dropped channels read 0:
+    the decode must equal exact attention over keys and values with those channels zeroed."""
+    B, Hq, Hkv, dk, dv, gk, gv, R = 2, 4, 2, 64, 64, 32, 16, 16
+    kw = [8] * 8 + [4] * 24 + [2] * 16 + [1] * 8 + [0] * 8
+    vw = [4] * 16 + [2] * 16 + [1] * 16 + [0] * 16
+    L = 5 * gk + R + 3
+    rng = np.random.default_rng(21)
+    ng = -(-L // gk)
+    k = np.zeros((B, Hkv, ng * gk, dk))
+    for c, b in enumerate(kw):
+        kk, _ = grid_cache_inputs(B, Hkv, ng * gk, 32, 32, max(b, 1), 2, gk, 32, seed=100 + c)
+        k[:, :, :, c] = kk[:, :, :, 0]
+    k = k[:, :, :L].astype(np.float16)
+    v = np.zeros((B, Hkv, L, dv))
+    for g in range(dv // gv):
+        _, vv = grid_cache_inputs(B, Hkv, L, 32, gv, 2, max(vw[g * gv], 1), gk, gv, seed=200 + g)
+        v[:, :, :, g * gv:(g + 1) * gv] = vv
+    v = v.astype(np.float16)
+    q = W.random_fp16((B, Hq, dk), seed=42).numpy()
+    c = O.OracleCache(var_cfg(B, Hq, Hkv, dk, dv, gk, gv, R, 0, L + 8, kw, vw))
+    c.prefill(k, v)
+    assert c.Q > 0
+    kz, vz = k.astype(np.float64).copy(), v.astype(np.float64).copy()
+    kz[:, :, :c.Q, np.array(kw) == 0] = 0.0
+    vz[:, :, :c.Q, np.array(vw) == 0] = 0.0
+    assert np.allclose(c.decode(q), sdpa_fp64(q, kz, vz), rtol=1e-11, atol=1e-12)
+    # and without the zeroing the decode differs (the dropped channels carry signal)
+    assert not np.allclose(c.decode(q), sdpa_fp64(q, k, v), rtol=1e-6, atol=1e-6)
+
+
+def test_dropped_channels_do_not_influence_the_quantized_tokens():
+    B, Hq, Hkv, dk, dv, gk, gv, R = 1, 2, 1, 32, 32, 16, 8, 8
+    kw = [4] * 16 + [0] * 16
+    vw = [2] * 16 + [0] * 16
+    L = 4 * gk + R
+    k = W.random_fp16((B, Hkv, L, dk), seed=1).numpy()
+    v = W.random_fp16((B, Hkv, L, dv), seed=2).numpy()
+    q = W.random_fp16((B, Hq, dk), seed=3).numpy()
+    cfg = var_cfg(B, Hq, Hkv, dk, dv, gk, gv, R, 1, L + 8, kw, vw)
+    a, b2 = O.OracleCache(cfg), O.OracleCache(cfg)
+    a.prefill(k, v)
+    k2, v2 = k.copy(), v.copy()
+    Q = a.Q
+    keep = set(a.ret_idx)
+    rows = [p for p in range(Q) if p not in keep]
+    k2[:, :, rows, 16:] = 7.0                       # dropped key channels of non-retained quantized tokens
+    v2[:, :, rows, 16:] = -3.0
+    b2.prefill(k2, v2)
+    assert np.array_equal(a.decode(q), b2.decode(q))
+
+
+def test_variable_width_appends_reach_the_same_state_as_one_prefill():
+    B, Hq, Hkv, dk, dv, gk, gv, R = 2, 4, 2, 64, 32, 16, 8, 8
+    kw = [8] * 4 + [4] * 20 + [2] * 30 + [0] * 10
+    vw = [4] * 8 + [1] * 16 + [0] * 8
+    L0, n = 40, 45
+    k = W.random_fp16((B, Hkv, L0 + n, dk), seed=4).numpy()
+    v = W.random_fp16((B, Hkv, L0 + n, dv), seed=5).numpy()
+    cfg = var_cfg(B, Hq, Hkv, dk, dv, gk, gv, R, 1, L0 + n + 8, kw, vw)
+    a, b2 = O.OracleCache(cfg), O.OracleCache(cfg)
+    a.prefill(k[:, :, :L0], v[:, :, :L0])
+    for t in range(L0, L0 + n):
+        a.append(k[:, :, t], v[:, :, t])
+    b2.prefill(k, v)
+    assert (a.L, a.Q, a.ret_idx) == (b2.L, b2.Q, b2.ret_idx)
+    for name in ("kcode", "ksz", "vcode", "vsz"):
+        x, y = getattr(a, name)[:, :, :a.Q // (gk if name == "ksz" else 1)], \
+            getattr(b2, name)[:, :, :b2.Q // (gk if name == "ksz" else 1)]
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), name
+
+
+def test_variable_width_bytes_per_token():
+    """A K(8x16, 4x64, 2x32, 0x16) / V(4, 2 over two 64-channel groups) row is 14+12 words of
+    codes: 26 * 4 = 104 B per token vs 112 B for K4V2 (plus the (scale, zero))."""
+    kw = [8] * 16 + [4] * 64 + [2] * 32 + [0] * 16
+    vw = [4] * 64 + [2] * 64
+    cfg = var_cfg(1, 4, 1, 128, 128, 64, 64, 128, 0, 4096, kw, vw)
+    bb = O.buffer_bytes(cfg)
+    assert bb["kcode"] == 4096 * 4 * 14 and bb["vcode"] == 4096 * 4 * 12
+    assert bb["ksz"] == 64 * 128 * 4 and bb["vsz"] == 4096 * 2 * 4
