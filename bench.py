@@ -58,7 +58,12 @@ def decode_bytes(cfg: dict, L: int) -> int:
     Q = max(L - R, 0) // gk * gk
     nret = len(K.kvq_retained_positions(Q)) if cfg["log_retain"] else 0
     sr, sq = cfg.get("side_rank", 0), cfg.get("side_bits", 0)
-    per_tok = dk * kb // 8 + dv * vb // 8 + (dv // gv) * 4 + sr * sq // 8
+    if kb == 0:       # per-channel widths: rows of max(1, ceil(bits / 32)) words
+        kbytes = 4 * max(1, -(-sum(cfg["k_widths"][:dk]) // 32))
+        vbytes = 4 * max(1, -(-sum(cfg["v_widths"][:dv]) // 32))
+    else:
+        kbytes, vbytes = dk * kb // 8, dv * vb // 8
+    per_tok = kbytes + vbytes + (dv // gv) * 4 + sr * sq // 8
     quant = Q * per_tok + (Q // gk) * (dk * 4 + sr * 4)
     fp16 = (L - Q + nret) * (dk + dv) * 2
     table = B * (Q // gk) * 4 if cfg.get("paged") else 0
@@ -155,10 +160,11 @@ def profile_traffic(workload_key: str):
         return None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"decode_source_sha256:\s*([0-9a-f]+)", text)
+    f = re.search(r"decode_source:\s*([\w.]+)", text)
     if not m or not h:
         return None
     import hashlib
-    src = os.path.join(ROOT, "mixed_precision_quantized_pack_b200", "csrc", "decode_mma.cuh")
+    src = os.path.join(ROOT, "mixed_precision_quantized_pack_b200", "csrc", f.group(1) if f else "decode_mma.cuh")
     try:
         cur = hashlib.sha256(open(src, "rb").read()).hexdigest()
     except OSError:

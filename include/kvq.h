@@ -83,6 +83,18 @@
  * window and retained buffers stay per sequence.  Needs quantized keys and values;
  * 1 <= n_pages, n_pages*Hkv*group_k < 2^30.
  *
+ * Per-channel bit widths (k_bits = v_bits = 0; "Attention-Aware Transform Coding (AATC)",
+ * §Méthodologie, Allocation de Bits): key channel c has k_widths[c] bits and value channel c
+ * v_widths[c] bits, each in {0, 1, 2, 4, 8}, non-increasing over the channels (the
+ * caller's decorrelating transform, folded into its projections, orders them by
+ * strength); the channels of one value group share a width.  A channel of width 0 is
+ * dropped: nothing is stored and it reads as 0.  Rows pack the codes channel after
+ * channel, LSB-first, channel c at bit offset sum_{c'<c} width_c' (never straddling a
+ * word), in W = max(1, ceil(sum of the widths / 32)) words:
+ *   kcode u32 [B][Hkv][Lcap][Wk]    ksz f16 [B][Hkv][Lcap/group_k][d_k][2] (scale, zero)
+ *   vcode u32 [B][Hkv][Lcap][Wv]    vsz as above; dropped channels / groups store (0, 0).
+ * Not combined with side codes or rotation.  kvq_allocate_bits computes such a map.
+ *
  * Conventions: every call is asynchronous on the caller's CUDA stream (passed as
  * void*, a cudaStream_t; NULL = legacy default stream); no call synchronizes or
  * copies device memory back to the host, except kvq_read_status.  The library
@@ -121,8 +133,8 @@ typedef struct kvq_config {
     int n_kv_heads;     /* Hkv; Hq % Hkv == 0 */
     int d_k;            /* key/query head dim: 32, 64, 128 or 256 */
     int d_v;            /* value head dim: 32, 64, 128 or 256 */
-    int k_bits;         /* 2, 4, 8, or 16 (= unquantized; then v_bits must be 16) */
-    int v_bits;         /* 2, 4, 8, or 16 */
+    int k_bits;         /* 2, 4, 8, 16 (= unquantized; then v_bits must be 16), or 0 */
+    int v_bits;         /* 2, 4, 8, 16, or 0 (per-channel widths: both 0) */
     int group_k;        /* tokens per key group: 16, 32, 64 or 128 */
     int group_v;        /* channels per value group: divides d_v, >= 32/v_bits */
     int window;         /* R >= 0: fp16 recent tokens kept beside the quantized prefix */
@@ -134,6 +146,8 @@ typedef struct kvq_config {
     unsigned int rot_signs[8];  /* rotation signs: bit c (word c/32, bit c%32) set -> -1 */
     int paged;          /* 0/1: quantized groups live in a shared pool of pages (see below) */
     int n_pages;        /* pages in the pool (paged caches); one page = one key group */
+    unsigned char k_widths[256];  /* k_bits = v_bits = 0: bits of key channel c (see below) */
+    unsigned char v_widths[256];  /* k_bits = v_bits = 0: bits of value channel c */
 } kvq_config;
 
 typedef struct kvq_sizes {
@@ -219,6 +233,18 @@ int kvq_append_ragged(kvq_cache* cache, const void* k_new, const void* v_new,
 int kvq_prefill_sequence(kvq_cache* cache, int b, const void* k, const void* v, int L, void* stream);
 int kvq_release_sequence(kvq_cache* cache, int b);
 int kvq_free_pages(const kvq_cache* cache);
+
+/* Reverse water-filling ("Attention-Aware Transform Coding (AATC)", §Méthodologie,
+ * Allocation de Bits; host only): widths[i] in {0, 1, 2, 4, 8} for n units of weight
+ * weight[i] >= 0 (a key channel, or a value group whose width bit costs unit_bits = group_v
+ * bits), minimising sum_i weight[i] * 4^-widths[i] under `budget` bits per row.  Each
+ * step of a unit's width (0->1->2->4->8) lowers that sum by weight * (4^-b1 - 4^-b2) for
+ * (b2 - b1) * unit_bits bits; steps are taken in decreasing order of that drop per bit,
+ * equal drops together, until the next set would exceed the budget; a step that lowers
+ * nothing is never taken.  Units of larger weight get at least as many bits, so weights
+ * sorted in decreasing order give a map kvq_config accepts.  Returns the bits spent, or
+ * INVALID_ARG (n < 1, unit_bits < 1, budget < 0, a weight negative or not finite, null). */
+int kvq_allocate_bits(const double* weight, int n, int unit_bits, int budget, unsigned char* widths);
 
 /* Workspace bytes kvq_decode_attention needs at the cache's current length for
  * num_splits (0 = automatic).  Always <= kvq_sizes.workspace. */

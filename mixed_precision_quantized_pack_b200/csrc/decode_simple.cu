@@ -89,8 +89,27 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
     begin = static_cast<int>(static_cast<long long>(f) * sw.n_fp16 / w.splits_f);
     end = static_cast<int>(static_cast<long long>(f + 1) * sw.n_fp16 / w.splits_f);
   }
-  const int perk = d.kb == 16 ? 1 : 32 / d.kb, perv = d.vb == 16 ? 1 : 32 / d.vb;
+  const int perk = d.kb == 16 || d.var ? 1 : 32 / d.kb, perv = d.vb == 16 || d.var ? 1 : 32 / d.vb;
   const uint32_t maskk = (1u << (d.kb & 15)) - 1u, maskv = (1u << (d.vb & 15)) - 1u;
+  // per-channel widths: each lane's channels' (word, shift, width), keys and values; a
+  // dropped channel reads word 0 with an empty mask (its offset may be the row's end)
+  uint32_t kvw[kMaxC], vvw[kMaxC];     // word index << 16 | shift << 8 | width
+  auto pack_wsw = [](int wd, int off) -> uint32_t {
+    return wd ? static_cast<uint32_t>(off / 32) << 16 | static_cast<uint32_t>(off % 32) << 8 | wd : 0u;
+  };
+#pragma unroll
+  for (int j = 0; j < kMaxC; ++j) kvw[j] = vvw[j] = 0u;
+  if (d.var) {
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j) {
+      int wd = 0, off = 0;
+      if (j < ck) channel_width(d.kcnt, lane + 32 * j, &wd, &off);
+      kvw[j] = pack_wsw(wd, off);
+      wd = off = 0;
+      if (j < cv) channel_width(d.vcnt, lane + 32 * j, &wd, &off);
+      vvw[j] = pack_wsw(wd, off);
+    }
+  }
 
   for (int i = begin + warp; i < end; i += kWarps) {
     float kh[kMaxC], vh[kMaxC];
@@ -119,6 +138,25 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
       const __half* ks = reinterpret_cast<const __half*>(cb.ksz) + gidx * 2 * d.dk;
       const uint32_t* vr = cb.vcode + row * d.vw;
       const __half2* vs = cb.vsz + row * d.nvg;
+      if (d.var) {
+        // per-channel widths: plain (scale, zero) pairs; dropped channels read 0
+#pragma unroll
+        for (int j = 0; j < kMaxC; ++j) {
+          kh[j] = 0.0f;
+          vh[j] = 0.0f;
+          if (j < ck) {
+            const int ch = lane + 32 * j;
+            const uint32_t code = (kr[kvw[j] >> 16] >> ((kvw[j] >> 8) & 31u)) & ((1u << (kvw[j] & 15u)) - 1u);
+            kh[j] = fmaf(static_cast<float>(code), __half2float(ks[2 * ch]), __half2float(ks[2 * ch + 1]));
+          }
+          if (j < cv) {
+            const int ch = lane + 32 * j;
+            const uint32_t code = (vr[vvw[j] >> 16] >> ((vvw[j] >> 8) & 31u)) & ((1u << (vvw[j] & 15u)) - 1u);
+            const float2 sz = __half22float2(vs[ch / d.gv]);
+            vh[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
+          }
+        }
+      } else {
 #pragma unroll
       for (int j = 0; j < kMaxC; ++j) {
         kh[j] = 0.0f;
@@ -138,6 +176,7 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
           const float2 sz = __half22float2(vs[ch / d.gv]);
           vh[j] = fmaf(static_cast<float>(code), sz.x, sz.y);
         }
+      }
       }
     } else {
       const __half *kp, *vp;

@@ -73,7 +73,34 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
   if (n_rep > 8) return KVQ_ERR_UNSUPPORTED;
   if (!is_pow2_in(c->d_k, 32, 256) || !is_pow2_in(c->d_v, 32, 256)) return KVQ_ERR_UNSUPPORTED;
   const bool raw = c->k_bits == 16 || c->v_bits == 16;
-  if (raw) {
+  const bool var = c->k_bits == 0 || c->v_bits == 0;
+  int kcnt[4] = {0, 0, 0, 0}, vcnt[4] = {0, 0, 0, 0}, kbits = 0, vbits = 0;
+  if (var) {
+    // per-channel widths: both maps, each in {0, 1, 2, 4, 8} and non-increasing; a value
+    // group's channels share one width
+    if (c->k_bits != 0 || c->v_bits != 0) return KVQ_ERR_UNSUPPORTED;
+    if (!is_pow2_in(c->group_k, 16, 128)) return KVQ_ERR_UNSUPPORTED;
+    if (c->group_v < 8 || c->group_v > c->d_v || c->d_v % c->group_v != 0 || c->group_v % 8 != 0)
+      return KVQ_ERR_UNSUPPORTED;
+    auto class_of = [](int w) { return w == 8 ? 0 : w == 4 ? 1 : w == 2 ? 2 : w == 1 ? 3 : w == 0 ? 4 : -1; };
+    auto read_map = [&](const unsigned char* wmap, int n, int* cnt, int* bits) {
+      int prev = 0;
+      for (int i = 0; i < n; ++i) {
+        const int k = class_of(wmap[i]);
+        if (k < 0 || k < prev) return false;
+        prev = k;
+        if (k < 4) ++cnt[k];
+        *bits += wmap[i];
+      }
+      return true;
+    };
+    if (!read_map(c->k_widths, c->d_k, kcnt, &kbits) || !read_map(c->v_widths, c->d_v, vcnt, &vbits))
+      return KVQ_ERR_UNSUPPORTED;
+    for (int g = 0; g < c->d_v; g += c->group_v)
+      for (int i = 1; i < c->group_v; ++i)
+        if (c->v_widths[g + i] != c->v_widths[g]) return KVQ_ERR_UNSUPPORTED;
+    if (c->side_rank != 0 || c->rot_keys != 0) return KVQ_ERR_UNSUPPORTED;
+  } else if (raw) {
     if (c->k_bits != 16 || c->v_bits != 16) return KVQ_ERR_UNSUPPORTED;
   } else {
     auto okb = [](int b) { return b == 2 || b == 4 || b == 8; };
@@ -125,8 +152,13 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
   x.paged = c->paged;
   x.max_groups = static_cast<int>(lcap / x.gk);
   x.cap = raw ? c->max_context : c->window + c->group_k;
-  x.kw = raw ? 0 : c->d_k * c->k_bits / 32;
-  x.vw = raw ? 0 : c->d_v * c->v_bits / 32;
+  x.kw = raw ? 0 : var ? std::max(1, (kbits + 31) / 32) : c->d_k * c->k_bits / 32;
+  x.vw = raw ? 0 : var ? std::max(1, (vbits + 31) / 32) : c->d_v * c->v_bits / 32;
+  x.var = var ? 1 : 0;
+  for (int i = 0; i < 4; ++i) {
+    x.kcnt[i] = kcnt[i];
+    x.vcnt[i] = vcnt[i];
+  }
   x.nvg = raw ? 1 : c->d_v / c->group_v;
   x.sr = c->side_rank;
   x.sq = c->side_rank ? c->side_bits : 0;
@@ -251,8 +283,12 @@ int plan_cache(const kvq_cache* c, int num_splits, bool fast, kvq_plan* out) {
 
 int check_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
 
+bool tensor_kernel_built(const kvq::Dims& d) {
+  return d.var ? kvq::decode_var_supported(d) : kvq::decode_mma_supported(d);
+}
+
 bool use_tensor_kernel(const kvq_cache* c) {
-  return c->kernel != KVQ_KERNEL_GENERIC && kvq::decode_mma_supported(c->d);
+  return c->kernel != KVQ_KERNEL_GENERIC && tensor_kernel_built(c->d);
 }
 
 // Dims and buffers of sequence b alone (a batch of one over the same memory).
@@ -436,6 +472,44 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
 }
 
 void kvq_cache_destroy(kvq_cache* cache) { delete cache; }
+
+int kvq_allocate_bits(const double* weight, int n, int unit_bits, int budget, unsigned char* widths) {
+  if (!weight || !widths || n < 1 || unit_bits < 1 || budget < 0) return KVQ_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (!(weight[i] >= 0.0) || !isfinite(weight[i])) return KVQ_ERR_INVALID_ARG;
+  // the width steps 0->1->2->4->8 and their distortion drops per bit for weight 1:
+  // (4^-b1 - 4^-b2) / (b2 - b1), exact binary fractions
+  static const int kFrom[4] = {0, 1, 2, 4}, kTo[4] = {1, 2, 4, 8};
+  static const double kDrop[4] = {0.75, 0.1875, 15.0 / 512.0, 255.0 / 262144.0};
+  struct Step {
+    double drop;
+    int unit, from, to;
+  };
+  std::vector<Step> steps;
+  steps.reserve(static_cast<size_t>(n) * 4);
+  for (int i = 0; i < n; ++i)
+    for (int k = 0; k < 4; ++k) {
+      const double drop = weight[i] * kDrop[k];
+      if (drop > 0.0) steps.push_back({drop, i, kFrom[k], kTo[k]});
+    }
+  std::stable_sort(steps.begin(), steps.end(), [](const Step& a, const Step& b) { return a.drop > b.drop; });
+  std::vector<unsigned char> w(n, 0);
+  long long used = 0;
+  for (size_t i = 0; i < steps.size();) {
+    size_t j = i;
+    long long cost = 0;
+    while (j < steps.size() && steps[j].drop == steps[i].drop) {
+      cost += static_cast<long long>(steps[j].to - steps[j].from) * unit_bits;
+      ++j;
+    }
+    if (used + cost > budget) break;
+    for (size_t k = i; k < j; ++k) w[steps[k].unit] = static_cast<unsigned char>(steps[k].to);
+    used += cost;
+    i = j;
+  }
+  std::copy(w.begin(), w.end(), widths);
+  return static_cast<int>(used);
+}
 
 int kvq_retained_positions(int Q, int* out, int cap) {
   if (Q < 0) return KVQ_ERR_INVALID_ARG;
@@ -731,7 +805,7 @@ int kvq_plan_decode(const kvq_config* cfg, int L, int sm_count, int num_splits, 
   kvq::Dims d;
   const int rc = make_dims(cfg, &d);
   if (rc) return rc;
-  return plan_decode(d, L, sm_count, num_splits, kvq::decode_mma_supported(d), out);
+  return plan_decode(d, L, sm_count, num_splits, tensor_kernel_built(d), out);
 }
 
 int kvq_get_plan(const kvq_cache* c, int num_splits, kvq_plan* out) {
@@ -779,7 +853,8 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
   const __half* qh = static_cast<const __half*>(q);
   const kvq::CacheBufs cb = cache_bufs(c);
   if (plan.fast_path)
-    rc = check_cuda(kvq::launch_decode_mma(d, cb, w, qh, parts, s));
+    rc = check_cuda(d.var ? kvq::launch_decode_var(d, cb, w, qh, parts, s)
+                          : kvq::launch_decode_mma(d, cb, w, qh, parts, s));
   else
     rc = check_cuda(kvq::launch_decode_simple(d, cb, w, qh, parts, s));
   if (!rc) rc = check_cuda(kvq::launch_combine(d, w, parts, static_cast<__half*>(out), s));
@@ -794,7 +869,7 @@ int kvq_debug_stall_next_decode(kvq_cache* c) {
 
 int kvq_set_decode_kernel(kvq_cache* c, int kernel) {
   if (!c || kernel < KVQ_KERNEL_AUTO || kernel > KVQ_KERNEL_TENSOR) return KVQ_ERR_INVALID_ARG;
-  if (kernel == KVQ_KERNEL_TENSOR && !kvq::decode_mma_supported(c->d)) return KVQ_ERR_UNSUPPORTED;
+  if (kernel == KVQ_KERNEL_TENSOR && !tensor_kernel_built(c->d)) return KVQ_ERR_UNSUPPORTED;
   c->kernel = kernel;
   return KVQ_OK;
 }

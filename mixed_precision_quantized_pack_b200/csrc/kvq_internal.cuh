@@ -26,8 +26,32 @@ struct Dims {
   float rot_inv_ck, rot_inv_cq;   // 1/c_k (keys), 1/c_q (queries): powers of two
   int paged;        // quantized groups in a pool of pages, located through a block table
   int max_groups;   // groups per sequence: lcap / gk (block-table row length)
+  // per-channel widths (kb = vb = 0): widths are non-increasing over the channels, so a map
+  // is the number of channels of width 8, 4, 2 and 1 (the rest are dropped, width 0)
+  int var;
+  int kcnt[4], vcnt[4];
   bool quantized() const { return kb != 16; }
 };
+
+// Width and bit offset in its packed row of channel c of a per-channel width map given by
+// its class counts (channels of width 8, then 4, 2, 1, then 0): the offset is the sum of
+// the widths before c.
+__host__ __device__ inline void channel_width(const int* cnt, int c, int* width, int* offset) {
+  int off = 0, base = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int w = 8 >> i;
+    if (c < base + cnt[i]) {
+      *width = w;
+      *offset = off + (c - base) * w;
+      return;
+    }
+    off += cnt[i] * w;
+    base += cnt[i];
+  }
+  *width = 0;
+  *offset = off;
+}
 
 // Where key group g of (b, kv head h) lives in the quantized buffers: the token row of its
 // first token in the code arrays (rows of kw / vw words, of zb side bytes, of nvg value
@@ -205,6 +229,9 @@ cudaError_t launch_update_retained(const Dims& d, const RetUpdate& up, __half* w
                                    __half* win_v, __half* ret_k, __half* ret_v, cudaStream_t s);
 cudaError_t launch_decode_simple(const Dims& d, const CacheBufs& c, const DecodeWork& w,
                                  const __half* q, const Partials& p, cudaStream_t s);
+bool decode_var_supported(const Dims& d);
+cudaError_t launch_decode_var(const Dims& d, const CacheBufs& c, const DecodeWork& w,
+                              const __half* q, const Partials& p, cudaStream_t s);
 bool decode_mma_supported(const Dims& d);
 cudaError_t launch_decode_mma(const Dims& d, const CacheBufs& c, const DecodeWork& w,
                               const __half* q, const Partials& p, cudaStream_t s);

@@ -23,9 +23,8 @@ struct GroupParams {
   __half2 sz;    // (scale, zero) as stored
 };
 
-template <int BITS>
-__device__ __forceinline__ GroupParams group_params(float mn, float mx) {
-  const float levels = static_cast<float>((1 << BITS) - 1);
+__device__ __forceinline__ GroupParams group_params_b(float mn, float mx, int bits) {
+  const float levels = static_cast<float>((1 << bits) - 1);
   const float s32 = __fdiv_rn(__fsub_rn(mx, mn), levels);
   __half s16 = __float2half_rn(s32);
   if (__half2float(s16) == 0.0f) s16 = __ushort_as_half(0);          // canonical +0
@@ -37,14 +36,19 @@ __device__ __forceinline__ GroupParams group_params(float mn, float mx) {
   return g;
 }
 
-template <int BITS>
-__device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g) {
+__device__ __forceinline__ uint32_t quant_code_b(float x, const GroupParams& g, int bits) {
   if (g.scale == 0.0f) return 0u;
-  const float levels = static_cast<float>((1 << BITS) - 1);
+  const float levels = static_cast<float>((1 << bits) - 1);
   float c = rintf(__fdiv_rn(__fsub_rn(x, g.zero), g.scale));          // half-to-even
   c = fminf(fmaxf(c, 0.0f), levels);
   return static_cast<uint32_t>(c);
 }
+
+template <int BITS>
+__device__ __forceinline__ GroupParams group_params(float mn, float mx) { return group_params_b(mn, mx, BITS); }
+
+template <int BITS>
+__device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g) { return quant_code_b(x, g, BITS); }
 
 // One thread per (key group, channel); blockDim = (dk, groups per block).  The
 // 32/BITS lanes holding the channels of one packed word OR their codes together.
@@ -277,6 +281,106 @@ __global__ void quantize_values_kernel(const __half* __restrict__ src, int src_r
   }
 }
 
+// ---- per-channel widths ("Attention-Aware Transform Coding (AATC)", §Méthodologie,
+// Allocation de Bits): channel c has its own width (8, 4, 2, 1 or 0 = dropped), widths
+// non-increasing over the channels; the same quantizer with that many bits; a row packs
+// the codes channel after channel, channel c at the sum of the widths before it.
+
+// One CTA of dk threads per (key group, b * kv head): thread c quantizes channel c over the
+// group's gk tokens; the codes are ORed into the group's rows in shared memory
+// ([gk][kw] u32, at most 128 x 64 words), which are then written out whole.  The group's
+// (scale, zero) are stored plainly, [dk][2]; a dropped channel stores (0, 0).
+__global__ void quantize_keys_var_kernel(const __half* __restrict__ src, int src_rows, int g_begin,
+                                         uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
+                                         const int* __restrict__ table, Dims d) {
+  extern __shared__ uint32_t sm_rows[];
+  const int c = threadIdx.x, nt = blockDim.x;
+  const int g = g_begin + blockIdx.x, bh = blockIdx.y;
+  const int gk = d.gk, kw = d.kw;
+  for (int i = c; i < gk * kw; i += nt) sm_rows[i] = 0u;
+  __syncthreads();
+  int width, offset;
+  channel_width(d.kcnt, c, &width, &offset);
+  const size_t base = static_cast<size_t>(bh) * src_rows;
+  auto key = [&](int t) { return __half2float(src[(base + (g * gk + t) % src_rows) * d.dk + c]); };
+  const size_t gidx = group_index(d, table, bh / d.Hkv, bh % d.Hkv, g);
+  __half2 sz = __floats2half2_rn(0.0f, 0.0f);
+  if (width) {
+    float mn = INFINITY, mx = -INFINITY;
+    for (int t = 0; t < gk; ++t) {
+      const float x = key(t);
+      mn = fminf(mn, x);
+      mx = fmaxf(mx, x);
+    }
+    const GroupParams gp = group_params_b(mn, mx, width);
+    sz = gp.sz;
+    for (int t = 0; t < gk; ++t)
+      atomicOr(&sm_rows[t * kw + offset / 32], quant_code_b(key(t), gp, width) << (offset % 32));
+  }
+  ksz[gidx * d.dk + c] = sz;
+  __syncthreads();
+  const size_t row0 = group_row(d, table, bh / d.Hkv, bh % d.Hkv, g);
+  for (int i = c; i < gk * kw; i += nt) kcode[row0 * kw + i] = sm_rows[i];
+}
+
+// One CTA of dv threads per 16 consecutive (b * kv head, token) rows: thread c holds channel
+// c; a value group's min and max are reduced over its gv channels (shuffles within a warp,
+// then shared memory across warps when gv > 32), and the codes are ORed into the row in
+// shared memory ([kw] u32) before it is written out.
+__global__ void quantize_values_var_kernel(const __half* __restrict__ src, int src_rows, int t_begin,
+                                           int n_tokens, uint32_t* __restrict__ vcode,
+                                           __half2* __restrict__ vsz, const int* __restrict__ table,
+                                           Dims d) {
+  __shared__ uint32_t sm_row[64];
+  __shared__ float sm_mn[8], sm_mx[8];
+  const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
+  const int gv = d.gv, vw = d.vw;
+  int width, offset;
+  channel_width(d.vcnt, c, &width, &offset);
+  const long long rows = static_cast<long long>(d.B) * d.Hkv * n_tokens;
+  for (long long r = static_cast<long long>(blockIdx.x) * 16; r < rows; r += static_cast<long long>(gridDim.x) * 16) {
+    for (int rr = 0; rr < 16 && r + rr < rows; ++rr) {
+      const long long rowi = r + rr;
+      const int t = t_begin + static_cast<int>(rowi % n_tokens);
+      const int bh = static_cast<int>(rowi / n_tokens);
+      for (int i = c; i < vw; i += blockDim.x) sm_row[i] = 0u;
+      const float x = __half2float(src[(static_cast<size_t>(bh) * src_rows + t % src_rows) * d.dv + c]);
+      float mn = x, mx = x;
+      const int span = gv < 32 ? gv : 32;
+      for (int off = 1; off < span; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      }
+      if (gv > 32) {
+        if (lane == 0) {
+          sm_mn[warp] = mn;
+          sm_mx[warp] = mx;
+        }
+        __syncthreads();
+        const int w0 = (c / gv) * (gv / 32);
+        mn = sm_mn[w0];
+        mx = sm_mx[w0];
+        for (int k = 1; k < gv / 32; ++k) {
+          mn = fminf(mn, sm_mn[w0 + k]);
+          mx = fmaxf(mx, sm_mx[w0 + k]);
+        }
+      }
+      __syncthreads();        // the row is cleared; the warps' extremes are read
+      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
+      __half2 sz = __floats2half2_rn(0.0f, 0.0f);
+      if (width) {
+        const GroupParams gp = group_params_b(mn, mx, width);
+        sz = gp.sz;
+        atomicOr(&sm_row[offset / 32], quant_code_b(x, gp, width) << (offset % 32));
+      }
+      if (c % gv == 0) vsz[vrow * d.nvg + c / gv] = sz;
+      __syncthreads();
+      for (int i = c; i < vw; i += blockDim.x) vcode[vrow * vw + i] = sm_row[i];
+      __syncthreads();        // before the next row clears sm_row and sm_mn / sm_mx
+    }
+  }
+}
+
 // dst[bh][(dst_base + i) % dst_rows] = src[bh][(src_base + i) % src_rows], i < n, 16 B at a time.
 __global__ void copy_rows_kernel(const __half* __restrict__ src, int src_rows, int src_base,
                                  __half* __restrict__ dst, int dst_rows, int dst_base, int n,
@@ -433,6 +537,18 @@ cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows,
                                  int n_groups, uint32_t* kcode, __half2* ksz, const int* table,
                                  bool rotate, cudaStream_t s) {
   if (n_groups <= 0) return cudaSuccess;
+  if (d.var) {
+    if (rotate) return cudaErrorInvalidValue;
+    const int smem = d.gk * d.kw * 4;       // <= 128 x 64 words
+    if (smem > 48 * 1024) {
+      const cudaError_t e = cudaFuncSetAttribute(quantize_keys_var_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+    }
+    quantize_keys_var_kernel<<<dim3(n_groups, d.B * d.Hkv), d.dk, smem, s>>>(src, src_rows, g_begin,
+                                                                              kcode, ksz, table, d);
+    return cudaGetLastError();
+  }
   return rotate ? launch_quantize_keys_t<true>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s)
                 : launch_quantize_keys_t<false>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
 }
@@ -484,6 +600,13 @@ cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_row
                                    cudaStream_t s) {
   if (n_tokens <= 0) return cudaSuccess;
   const int nbh = d.B * d.Hkv;
+  if (d.var) {
+    const long long rows = static_cast<long long>(nbh) * n_tokens;
+    const long long blocks = (rows + 15) / 16;
+    const int grid = static_cast<int>(blocks < 148 * 16 ? blocks : 148 * 16);
+    quantize_values_var_kernel<<<grid, d.dv, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d);
+    return cudaGetLastError();
+  }
   const long long items = static_cast<long long>(nbh) * n_tokens * d.nvg;
   const int block = 256;
   const int grid = grid_for(items, block);

@@ -47,7 +47,8 @@ POINTER_FIELDS = BUFFER_FIELDS + SIDE_FIELDS + PAGE_FIELDS
 
 class kvq_config(ctypes.Structure):
     _fields_ = ([(n, ctypes.c_int) for n in CONFIG_FIELDS] + [("rot_signs", ctypes.c_uint * 8)] +
-                [(n, ctypes.c_int) for n in PAGE_CONFIG])
+                [(n, ctypes.c_int) for n in PAGE_CONFIG] +
+                [("k_widths", ctypes.c_ubyte * 256), ("v_widths", ctypes.c_ubyte * 256)])
 
 
 class kvq_sizes(ctypes.Structure):
@@ -101,6 +102,7 @@ _SIGNATURES = {
     "kvq_prefill_sequence": (_I, [_P, _I, _P, _P, _I, _P]),
     "kvq_release_sequence": (_I, [_P, _I]),
     "kvq_free_pages": (_I, [_P]),
+    "kvq_allocate_bits": (_I, [ctypes.POINTER(ctypes.c_double), _I, _I, _I, ctypes.POINTER(ctypes.c_ubyte)]),
 }
 
 
@@ -139,6 +141,9 @@ def make_config(cfg: Dict[str, int]) -> kvq_config:
         c.rot_signs[i] = int(word) & 0xFFFFFFFF
     for n in PAGE_CONFIG:
         setattr(c, n, int(cfg.get(n, 0)))
+    for n in ("k_widths", "v_widths"):
+        for i, w in enumerate(list(cfg.get(n, ()))[:256]):
+            getattr(c, n)[i] = int(w)
     return c
 
 
@@ -159,6 +164,15 @@ def kvq_plan_decode(cfg: Dict[str, int], L: int, sm_count: int, num_splits: int 
     _check(lib().kvq_plan_decode(ctypes.byref(make_config(cfg)), int(L), int(sm_count),
                                  int(num_splits), ctypes.byref(out)), "kvq_plan_decode")
     return {n: int(getattr(out, n)) for n, _ in kvq_plan._fields_}
+
+
+def kvq_allocate_bits(weight, budget: int, unit_bits: int = 1) -> Tuple[List[int], int]:
+    """Per-unit widths by reverse water-filling, and the bits they spend."""
+    n = len(weight)
+    w = (ctypes.c_double * n)(*[float(x) for x in weight])
+    out = (ctypes.c_ubyte * n)()
+    spent = _check(lib().kvq_allocate_bits(w, n, int(unit_bits), int(budget), out), "kvq_allocate_bits")
+    return [int(out[i]) for i in range(n)], spent
 
 
 def kvq_retained_positions(Q: int) -> List[int]:
@@ -412,10 +426,17 @@ class KVCache:
         paged = bool(c.get("paged", 0))
         rows = (c["n_pages"], H, gk) if paged else (B, H, lcap)
         groups = (c["n_pages"], H) if paged else (B, H, lcap // gk)
+        if kb == 0:        # per-channel widths: rows of max(1, ceil(sum / 32)) words
+            kwords = max(1, -(-sum(int(x) for x in c["k_widths"][:dk]) // 32))
+            vwords = max(1, -(-sum(int(x) for x in c["v_widths"][:dv]) // 32))
+            ksz_shape = groups + (dk, 2)
+        else:
+            kwords, vwords = dk * kb // 32, dv * vb // 32
+            ksz_shape = groups + (2 * dk,)
         shapes = {
-            "kcode": (torch.int32, rows + (dk * kb // 32,)),
-            "ksz": (torch.float16, groups + (2 * dk,)),
-            "vcode": (torch.int32, rows + (dv * vb // 32,)),
+            "kcode": (torch.int32, rows + (kwords,)),
+            "ksz": (torch.float16, ksz_shape),
+            "vcode": (torch.int32, rows + (vwords,)),
             "vsz": (torch.float16, rows + (dv // gv, 2)),
             "block_table": (torch.int32, (B, lcap // gk)),
             "win_k": (torch.float16, (B, H, cap, dk)),

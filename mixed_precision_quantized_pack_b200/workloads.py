@@ -59,6 +59,8 @@ class Workload:
     rot_keys: int = 0     # key-only rotation, with signs drawn from rot_seed
     rot_seed: int = 0
     paged: int = 0        # quantized groups in a page pool just large enough for max_context
+    k_widths: tuple = ()  # k_bits = v_bits = 0: per-channel key widths ...
+    v_widths: tuple = ()  # ... and value widths (data, given with the workload)
 
     @property
     def n_rep(self) -> int:
@@ -80,7 +82,8 @@ class Workload:
                     side_rank=self.side_rank, side_bits=self.side_bits, rot_keys=self.rot_keys,
                     rot_signs=rotation_signs(self.rot_seed) if self.rot_keys else [0] * 8,
                     paged=self.paged,
-                    n_pages=self.batch * -(-mc // self.group_k) if self.paged else 0)
+                    n_pages=self.batch * -(-mc // self.group_k) if self.paged else 0,
+                    k_widths=list(self.k_widths), v_widths=list(self.v_widths))
 
 
 def rotation_signs(seed: int) -> List[int]:
@@ -120,6 +123,14 @@ WORKLOADS: Dict[str, Workload] = {
     "rot32k": _base(name="rot-b32-32/8-32k-k4v2-logretain", batch=32, n_q_heads=32, n_kv_heads=8,
                     d_k=128, d_v=128, context=32768, k_bits=4, v_bits=2, group_k=64, group_v=64,
                     window=128, log_retain=1, appends=0, seed=1006, rot_keys=1, rot_seed=77),
+    # the 32k case with per-channel widths ("Attention-Aware Transform Coding", bit
+    # allocation): keys 16 x 8, 64 x 4, 32 x 2 bits and 16 dropped channels (448 bits per
+    # row, 3.5 on average); values in groups of 32 channels at 4, 2, 2 and 1 bits (288 bits)
+    "aatc32k": _base(name="aatc-b32-32/8-32k-kvar3.5-vvar2.25-logretain", batch=32, n_q_heads=32,
+                     n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=0, v_bits=0,
+                     group_k=64, group_v=32, window=128, log_retain=1, appends=0, seed=1008,
+                     k_widths=(8,) * 16 + (4,) * 64 + (2,) * 32 + (0,) * 16,
+                     v_widths=(4,) * 32 + (2,) * 64 + (1,) * 32),
     # the 32k case with its quantized groups in a page pool, found through a block table
     "paged32k": _base(name="paged-b32-32/8-32k-k4v2-logretain", batch=32, n_q_heads=32,
                       n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=4, v_bits=2,

@@ -243,3 +243,94 @@ def test_unpaged_group_indices_must_fit_31_bits():
         K.kvq_buffer_sizes(cfg(batch=1 << 14, n_kv_heads=8, n_q_heads=8, group_k=16,
                                max_context=1 << 18))
     assert e.value.code == K.KVQ_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------ per-channel widths ----
+def var(**kw):
+    base = cfg(k_bits=0, v_bits=0, group_v=32, k_widths=[8] * 16 + [4] * 64 + [2] * 32 + [0] * 16,
+               v_widths=[4] * 32 + [2] * 64 + [1] * 32)
+    base.update(kw)
+    return base
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_allocator_matches_the_oracle(seed):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 200))
+    w = rng.lognormal(0.0, 2.0, size=n)
+    if seed % 3 == 0:
+        w[rng.integers(0, n, size=n // 3)] = w[0]            # ties
+    if seed % 4 == 1:
+        w[rng.integers(0, n, size=n // 4)] = 0.0              # zero weights
+    if seed % 5 == 2:
+        w = np.round(w * 4) / 4                                # many exact ties
+    unit = int(rng.choice([1, 8, 16, 64]))
+    for budget in (0, 1, unit * n // 2, unit * 3 * n, unit * 8 * n, 10 ** 7):
+        got, spent = K.kvq_allocate_bits(list(w), budget, unit)
+        want = O.allocate_bits(w, budget, unit)
+        assert got == [int(x) for x in want], (seed, budget)
+        assert spent == unit * int(np.sum(want)) <= budget
+
+
+def test_allocator_rejects_bad_arguments():
+    for args in (([], 4, 1), ([1.0, -1.0], 4, 1), ([1.0, float("nan")], 4, 1), ([1.0, float("inf")], 4, 1),
+                 ([1.0], -1, 1), ([1.0], 4, 0)):
+        with pytest.raises(K.KVQError) as e:
+            K.kvq_allocate_bits(*args)
+        assert e.value.code == K.KVQ_ERR_INVALID_ARG
+    lib = K.lib()
+    assert lib.kvq_allocate_bits(None, 1, 1, 1, None) == K.KVQ_ERR_INVALID_ARG
+
+
+def test_allocation_of_sorted_weights_is_a_valid_width_map():
+    import numpy as np
+    rng = np.random.default_rng(9)
+    kw_ = sorted(rng.lognormal(0.0, 2.0, size=128), reverse=True)
+    vw_ = sorted(rng.lognormal(0.0, 1.0, size=4), reverse=True)
+    kmap, _ = K.kvq_allocate_bits(kw_, 3 * 128)
+    gmap, _ = K.kvq_allocate_bits(vw_, 2 * 128, unit_bits=32)
+    vmap = [w for w in gmap for _ in range(32)]
+    sizes = K.kvq_buffer_sizes(var(k_widths=kmap, v_widths=vmap))
+    c = var(k_widths=kmap, v_widths=vmap)
+    assert sizes["kcode"] == O.buffer_bytes(c)["kcode"]
+
+
+@pytest.mark.parametrize("kw_,vw_", [
+    ([4] * 64 + [8] * 64, [2] * 128),                        # keys increase
+    ([3] * 128, [2] * 128),                                  # width 3
+    ([4] * 128, [2] * 16 + [1] * 112),                       # a value group of 32 split 16/16
+    ([4] * 128, [1] * 32 + [2] * 96),                        # values increase
+    ([16] * 128, [2] * 128),                                 # width 16
+])
+def test_invalid_width_maps_are_rejected(kw_, vw_):
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_buffer_sizes(var(k_widths=kw_, v_widths=vw_))
+    assert e.value.code == K.KVQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("bad", [dict(v_bits=2), dict(k_bits=4), dict(side_rank=4, side_bits=4),
+                                 dict(rot_keys=1), dict(group_k=48), dict(group_v=12)])
+def test_width_maps_do_not_combine_with_other_modes(bad):
+    with pytest.raises(K.KVQError) as e:
+        K.kvq_buffer_sizes(var(**bad))
+    assert e.value.code == K.KVQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw_,vw_,gv,fast", [
+    ([8] * 16 + [4] * 64 + [2] * 32 + [0] * 16, [4] * 32 + [2] * 64 + [1] * 32, 32, 1),
+    ([0] * 128, [0] * 128, 64, 1),                           # everything dropped: 1-word rows
+    ([1] * 128, [8] * 8 + [1] * 120, 8, 0),                  # value groups below 16 channels
+    ([8] * 128, [4] * 128, 128, 1),
+    ([8] * 12 + [4] * 116, [2] * 128, 32, 0),                # 12 x 8 bits: a word mixes widths
+    ([4] * 128, [1] * 128, 16, 0),                           # 1-bit value groups of 16
+])
+def test_width_map_sizes_match_the_oracle_layout(kw_, vw_, gv, fast):
+    c = var(k_widths=kw_, v_widths=vw_, group_v=gv)
+    got, want = K.kvq_buffer_sizes(c), O.buffer_bytes(c)
+    for n in K.BUFFER_FIELDS:
+        assert got[n] == want[n], n
+    # the planner counts the packed rows; the tensor-core kernel takes the maps it is built for
+    p = K.kvq_plan_decode(c, 3000, 148, 0)
+    assert p["fast_path"] == fast and p["n_groups"] == (3000 - 128) // 64
+    assert K.kvq_plan_decode(dict(c, d_k=64), 3000, 148, 0)["fast_path"] == 0 if len(kw_) == 128 else True

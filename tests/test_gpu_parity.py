@@ -589,3 +589,50 @@ def test_page_pool_exhaustion_changes_nothing():
     out = c.decode(inp.q[1].cuda()).float().cpu().numpy()
     for b, oc in enumerate((oc0, oc1)):
         assert O.max_rel_error(out[b:b + 1], oc.decode(np16(inp.q[1][b:b + 1]))) <= TOL
+
+
+# ------------------------------------------------------------ per-channel widths ----
+AATC = W.WORKLOADS["aatc32k"]
+
+
+@pytest.mark.parametrize("shape", [
+    dict(),                                                                  # the bench map
+    dict(k_widths=(0,) * 128, v_widths=(0,) * 128, group_v=64),              # everything dropped
+    dict(k_widths=(1,) * 128, v_widths=(1,) * 128, group_v=8),
+    dict(d_k=64, d_v=256, group_k=16, group_v=128,
+         k_widths=(8,) * 8 + (4,) * 8 + (2,) * 16 + (1,) * 16 + (0,) * 16, v_widths=(8,) * 128 + (2,) * 128),
+    dict(d_k=32, d_v=32, group_k=128, group_v=8, window=5, k_widths=(4,) * 32,
+         v_widths=(8,) * 8 + (4,) * 8 + (0,) * 16),
+    dict(d_k=256, group_v=16, n_q_heads=8, n_kv_heads=8,
+         k_widths=(8,) * 32 + (4,) * 96 + (2,) * 64 + (1,) * 32 + (0,) * 32,
+         v_widths=(8,) * 16 + (4,) * 48 + (2,) * 32 + (1,) * 16 + (0,) * 16),
+    dict(k_widths=(8,) * 128, v_widths=(8,) * 128, group_v=128, log_retain=0),
+    dict(n_q_heads=8, n_kv_heads=8, group_k=16),                               # tensor cores, GQA 1
+    dict(group_k=128, group_v=16, v_widths=(8,) * 16 + (4,) * 32 + (2,) * 80),  # tensor cores
+])
+def test_width_maps(shape):
+    w = AATC.with_(batch=2, context=1500, appends=70, seed=301 + len(str(shape)), **shape)
+    run_small(w, num_splits=(0, 3), steps={0, 1, 57, 58, 69})
+
+
+def test_width_map_kernel_choice():
+    """The tensor-core kernel serves maps whose width classes fill whole words (d 128, value
+    groups >= 16); the others run on the generic kernel."""
+    assert tensor_kernel_built(AATC)
+    assert tensor_kernel_built(AATC.with_(n_q_heads=8, n_kv_heads=8))
+    assert not tensor_kernel_built(AATC.with_(d_k=64, k_widths=(4,) * 64))
+    assert not tensor_kernel_built(AATC.with_(group_v=8))
+    assert not tensor_kernel_built(AATC.with_(k_widths=(8,) * 12 + (4,) * 116))
+
+
+def test_width_maps_ragged_batch():
+    run_ragged(AATC.with_(batch=4, seed=311), [1300, 64, 777, 1029], n_app=66, steps={0, 33, 65}, seed=312)
+
+
+def test_width_maps_paged():
+    run_paged(AATC.with_(batch=3, seed=321, paged=1), [900, 333, 1280], n_app=66, steps={1, 10, 65},
+              seed=322, restart=10)
+
+
+def test_full_size_aatc_32k():
+    sampled_full_size(AATC, rows=(0, 31))
