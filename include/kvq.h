@@ -228,6 +228,7 @@ int kvq_append_ragged(kvq_cache* cache, const void* k_new, const void* v_new,
  * length becomes 0.  Decode fails with STATE while any sequence is empty, and so does
  * an append that includes an empty sequence.
  * kvq_free_pages: pages of the pool not in use (0 for caches that are not paged).
+ * With more than KVQ_MAX_SEQS sequences, decode needs their lengths equal (UNSUPPORTED).
  * Errors: INVALID_ARG (b or L out of range), CAPACITY (the pool has too few free pages;
  * nothing changes), ALIGN, CUDA. */
 int kvq_prefill_sequence(kvq_cache* cache, int b, const void* k, const void* v, int L, void* stream);
