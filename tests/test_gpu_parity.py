@@ -15,6 +15,7 @@ from mixed_precision_quantized_pack_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-3
+AATC = W.WORKLOADS["aatc32k"]
 # AUTO picks the tensor-core kernel wherever it is built for the shape; GENERIC is
 # the CUDA-core kernel.  Both are checked against the oracle.
 KERNELS = (K.KVQ_KERNEL_AUTO, K.KVQ_KERNEL_GENERIC)
@@ -184,19 +185,25 @@ def test_split_invariance():
         assert (o - outs[0]).abs().max().item() <= 2e-3 * outs[0].abs().max().item()
 
 
-def test_a_wait_that_runs_out_sets_the_timeout_status():
-    """The tensor-core kernel's waits are bounded: when one gives up (the test hook makes one
+@pytest.mark.parametrize("case", ["fixed", "paged", "widths"])
+def test_a_wait_that_runs_out_sets_the_timeout_status(case):
+    """The tensor-core kernels' waits are bounded: when one gives up (the test hook makes one
     copy stage ask for 16 bytes more than it receives) the call sets KVQ_STATUS_TIMEOUT
     within seconds, and the context and the cache stay usable for the next call."""
     need_gpu()
     import time
     w = W.WORKLOADS["gqa4k"].with_(batch=2, context=1024, appends=0, seed=91)
+    if case == "paged":
+        w = w.with_(paged=1)
+    elif case == "widths":
+        w = AATC.with_(batch=2, context=1024, appends=0, seed=92)
     inp = W.Inputs(w, device="cpu")
     cfg = w.kvq_config()
     gc = K.KVCache(cfg)
     oc = O.OracleCache(cfg)
     gc.prefill(inp.k.cuda(), inp.v.cuda())
     oc.prefill(np16(inp.k), np16(inp.v))
+    assert gc.plan()["fast_path"] == 1
     ref = oc.decode(np16(inp.q[0]))
     q = inp.q[0].cuda()
     assert O.max_rel_error(gc.decode(q).float().cpu().numpy(), ref) <= TOL
@@ -592,7 +599,6 @@ def test_page_pool_exhaustion_changes_nothing():
 
 
 # ------------------------------------------------------------ per-channel widths ----
-AATC = W.WORKLOADS["aatc32k"]
 
 
 @pytest.mark.parametrize("shape", [
