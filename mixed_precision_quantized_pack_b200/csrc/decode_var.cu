@@ -123,7 +123,87 @@ __device__ __forceinline__ void expand_row(const uint32_t* rowp, uint32_t* trow,
   expand_class<1>(rowp, trow, w3, w4, m3, ehalf);
 }
 
-template <int NREP>
+// A width map fixed at build time: channel counts of widths 8, 4, 2, 1 for keys (K*) and
+// values (V*), and the value group size.  K8 < 0 means "taken from the VarMap at run time".
+template <int K8_, int K4_, int K2_, int K1_, int V8_, int V4_, int V2_, int V1_, int GV_>
+struct MapSpec {
+  static constexpr bool kFixed = K8_ >= 0;
+  static constexpr int K8 = K8_, K4 = K4_, K2 = K2_, K1 = K1_;
+  static constexpr int V8 = V8_, V4 = V4_, V2 = V2_, V1 = V1_, GV = GV_;
+};
+using RuntimeMap = MapSpec<-1, 0, 0, 0, 0, 0, 0, 0, 0>;
+
+// Words [W0, W1) of width B at register M0, with every bound a compile-time constant: the
+// half-warp ehalf takes words W0 + ehalf, W0 + ehalf + 2, ...
+template <int B, int W0, int W1, int M0>
+__device__ __forceinline__ void expand_class_fixed(const uint32_t* rowp, uint32_t* trow, int ehalf) {
+  constexpr int R = 16 / B, N = W1 - W0;
+#pragma unroll
+  for (int i = 0; i < (N + 1) / 2; ++i) {
+    if (N % 2 == 0 || 2 * i + ehalf < N) {
+      uint32_t r[R];
+      expand_word<B>(rowp[W0 + 2 * i + ehalf], r);
+      uint2* dst = reinterpret_cast<uint2*>(trow + M0 + (2 * i + ehalf) * R);
+#pragma unroll
+      for (int k = 0; k < R; k += 2) dst[k / 2] = make_uint2(r[k], r[k + 1]);
+    }
+  }
+}
+
+template <int C8, int C4, int C2, int C1>
+__device__ __forceinline__ void expand_row_fixed(const uint32_t* rowp, uint32_t* trow, int ehalf) {
+  constexpr int N8 = C8 / 4, N4 = C4 / 8, N2 = C2 / 16, N1 = C1 / 32;      // words per class
+  expand_class_fixed<8, 0, N8, 0>(rowp, trow, ehalf);
+  expand_class_fixed<4, N8, N8 + N4, 2 * N8>(rowp, trow, ehalf);
+  expand_class_fixed<2, N8 + N4, N8 + N4 + N2, 2 * N8 + 4 * N4>(rowp, trow, ehalf);
+  expand_class_fixed<1, N8 + N4 + N2, N8 + N4 + N2 + N1, 2 * N8 + 4 * N4 + 8 * N2>(rowp, trow, ehalf);
+}
+
+// Channel of slot s of a fixed map (the order expand_word produces; -1 past the used slots).
+__host__ __device__ constexpr int fixed_slot_channel(int s, int c8, int c4, int c2, int c1) {
+  const int cnt[4] = {c8, c4, c2, c1};
+  int m = s / 2, hi = s % 2, c = 0, pairs = 0;
+  for (int i = 0; i < 4; ++i) {
+    const int b = 8 >> i, words = cnt[i] * b / 32, regs = 16 / b;
+    if (m < pairs + words * regs) {
+      const int k = (m - pairs) / regs, r = (m - pairs) % regs;
+      const int j = r / (8 / b), p = (r % (8 / b)) * b;
+      return c + k * (32 / b) + (8 * j + p + 16 * hi) / b;
+    }
+    pairs += words * regs;
+    c += cnt[i];
+  }
+  return -1;
+}
+
+// Value group of slot tile mv of a fixed map, and the first tile of that group (-1: unused).
+template <class M>
+__host__ __device__ constexpr int fixed_tile_group(int mv) {
+  const int ch = fixed_slot_channel(16 * mv, M::V8, M::V4, M::V2, M::V1);
+  return ch < 0 ? -1 : ch / M::GV;
+}
+template <class M>
+__host__ __device__ constexpr int fixed_tile_head(int mv) {
+  return fixed_tile_group<M>(mv) < 0 ? -1
+         : (mv > 0 && fixed_tile_group<M>(mv - 1) == fixed_tile_group<M>(mv)) ? fixed_tile_head<M>(mv - 1)
+                                                                              : mv;
+}
+
+// Value group and group-head tile of every slot tile of a fixed map, as one compile-time table.
+struct TileTable {
+  int group[8], head[8];
+};
+template <class M>
+__host__ __device__ constexpr TileTable fixed_tile_table() {
+  TileTable t{};
+  for (int mv = 0; mv < 8; ++mv) {
+    t.group[mv] = fixed_tile_group<M>(mv);
+    t.head[mv] = t.group[mv] < 0 ? -1 : (mv > 0 && t.group[mv - 1] == t.group[mv]) ? t.head[mv - 1] : mv;
+  }
+  return t;
+}
+
+template <int NREP, class M = RuntimeMap>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarMap vm, const __half* __restrict__ q,
                   Partials part) {
@@ -375,8 +455,11 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarMap vm, const __half* _
       if (quant) {
         // expand the 16 key rows of the tile: lane = (row, word parity)
         const uint32_t* rowp = reinterpret_cast<const uint32_t*>(S + L.k_off) + (16 * t + erow) * d.kw;
-        expand_row(rowp, reinterpret_cast<uint32_t*>(tile + erow * KST), vm.kwb[1], vm.kwb[2], vm.kwb[3],
-                   vm.kwb[4], vm.kmb[1], vm.kmb[2], vm.kmb[3], ehalf);
+        if constexpr (M::kFixed)
+          expand_row_fixed<M::K8, M::K4, M::K2, M::K1>(rowp, reinterpret_cast<uint32_t*>(tile + erow * KST), ehalf);
+        else
+          expand_row(rowp, reinterpret_cast<uint32_t*>(tile + erow * KST), vm.kwb[1], vm.kwb[2], vm.kwb[3],
+                     vm.kwb[4], vm.kmb[1], vm.kmb[2], vm.kmb[3], ehalf);
         __syncwarp();
         KT = tile_s;
       } else {
@@ -430,8 +513,11 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarMap vm, const __half* _
         // expand the 16 value rows into the same tile (the key slots are consumed)
         __syncwarp();
         const uint32_t* rowp = reinterpret_cast<const uint32_t*>(S + L.v_off) + (16 * t + erow) * d.vw;
-        expand_row(rowp, reinterpret_cast<uint32_t*>(tile + erow * VST), vm.vwb[1], vm.vwb[2], vm.vwb[3],
-                   vm.vwb[4], vm.vmb[1], vm.vmb[2], vm.vmb[3], ehalf);
+        if constexpr (M::kFixed)
+          expand_row_fixed<M::V8, M::V4, M::V2, M::V1>(rowp, reinterpret_cast<uint32_t*>(tile + erow * VST), ehalf);
+        else
+          expand_row(rowp, reinterpret_cast<uint32_t*>(tile + erow * VST), vm.vwb[1], vm.vwb[2], vm.vwb[3],
+                     vm.vwb[4], vm.vmb[1], vm.vmb[2], vm.vmb[3], ehalf);
         __syncwarp();
         VT = tile_s;
       } else {
@@ -440,24 +526,33 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarMap vm, const __half* _
       // p.V: A = V^T tiles of 16 slots via ldmatrix.trans, B = p (times the value group's
       // scale of each token), one (hi, lo) pair per token transposed by movmatrix
       const __half2* vmeta = quant ? reinterpret_cast<const __half2*>(S + L.vmeta_off) : nullptr;
-      const int vtiles = quant ? vm.vtiles : 8;
       uint32_t bp0 = 0u, bp1 = 0u;
 #pragma unroll
       for (int mv = 0; mv < 8; ++mv) {
-        if (mv >= vtiles) break;
-        if (quant ? vm.vhead[mv] == mv : mv == 0) {      // the first tile of a value group
+        int head, g;
+        if constexpr (M::kFixed) {
+          constexpr TileTable tt = fixed_tile_table<M>();
+          head = tt.head[mv];
+          g = tt.group[mv];
+        } else {
+          head = vm.vhead[mv];
+          g = vm.vgroup[mv];
+        }
+        if (quant && g < 0) break;
+        float zz = 0.0f;
+        if (quant ? head == mv : mv == 0) {      // the first tile of a value group
           float x0 = p0, x1 = p1;
           if (quant) {
-            const int g = vm.vgroup[mv];
             const float2 sz0 = __half22float2(vmeta[(16 * t + qr) * d.nvg + g]);
             const float2 sz1 = __half22float2(vmeta[(16 * t + qr + 8) * d.nvg + g]);
             x0 *= sz0.x;
             x1 *= sz1.x;
-            zsum[mv] += fmaf(p0, sz0.y, p1 * sz1.y);   // kept under the group's first tile
+            zz = fmaf(p0, sz0.y, p1 * sz1.y);
           }
           bp0 = ptx::movmatrix_trans(ptx::split_hi_lo_trunc(x0));
           bp1 = ptx::movmatrix_trans(ptx::split_hi_lo_trunc(x1));
         }
+        zsum[mv] += zz;          // a group's sum is kept under its first tile
         uint32_t a0, a1, a2, a3;
         ptx::ldmatrix_x4_trans(VT + vrow * VST + (16 * mv + (mi & 1) * 8) * 2, a0, a1, a2, a3);
         ptx::mma_16816(co[mv], a0, a1, a2, a3, bp0, bp1);
@@ -629,13 +724,44 @@ bool supported(const Dims& d) {
   return (kSmemPerCta - Smem::kStages) / stage >= 1 && kWarps * 4 * kDV * 4 + 256 <= kSmemPerCta - Smem::kStages;
 }
 
+namespace {
+
+// Maps with a build-time instance: keys 16 x 8, 64 x 4, 32 x 2 bits (+ 16 dropped), values in
+// groups of 32 channels at 4, 2, 2, 1 bits.
+using MapK3V2 = MapSpec<16, 64, 32, 0, 0, 32, 64, 32, 32>;
+
+// The instance's compile-time tables must be those of the run-time map.
+template <class M>
+bool fixed_map_matches(const Dims& d, const VarMap& vm) {
+  const int k[4] = {M::K8, M::K4, M::K2, M::K1}, v[4] = {M::V8, M::V4, M::V2, M::V1};
+  for (int i = 0; i < 4; ++i)
+    if (d.kcnt[i] != k[i] || d.vcnt[i] != v[i]) return false;
+  if (d.gv != M::GV) return false;
+  for (int sl = 0; sl < vm.kslots; ++sl)
+    if (fixed_slot_channel(sl, M::K8, M::K4, M::K2, M::K1) != vm.kch[sl]) return false;
+  for (int sl = 0; sl < vm.vslots; ++sl)
+    if (fixed_slot_channel(sl, M::V8, M::V4, M::V2, M::V1) != vm.vch[sl]) return false;
+  for (int mv = 0; mv < 8; ++mv)
+    if (fixed_tile_group<M>(mv) != vm.vgroup[mv] || fixed_tile_head<M>(mv) != vm.vhead[mv]) return false;
+  return true;
+}
+
+}  // namespace
+
 cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
                    const Partials& p, cudaStream_t s) {
   VarMap vm;
   if (!supported(d) || !make_map(d, &vm)) return cudaErrorNotSupported;
-  auto kern = d.n_rep == 4 ? decode_var_kernel<4> : decode_var_kernel<1>;
-  static bool configured[2] = {false, false};
-  const int which = d.n_rep == 4 ? 0 : 1;
+  void (*kern)(Dims, CacheBufs, DecodeWork, VarMap, const __half*, Partials);
+  int which;
+  if (fixed_map_matches<MapK3V2>(d, vm)) {
+    kern = d.n_rep == 4 ? decode_var_kernel<4, MapK3V2> : decode_var_kernel<1, MapK3V2>;
+    which = d.n_rep == 4 ? 2 : 3;
+  } else {
+    kern = d.n_rep == 4 ? decode_var_kernel<4> : decode_var_kernel<1>;
+    which = d.n_rep == 4 ? 0 : 1;
+  }
+  static bool configured[4] = {false, false, false, false};
   if (!configured[which]) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerCta);
     if (e != cudaSuccess) return e;
