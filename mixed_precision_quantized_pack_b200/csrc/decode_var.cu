@@ -18,7 +18,9 @@
 //
 // Shape limits of this kernel (others run on the generic kernel): d_k = d_v = 128, 1 or 4
 // query heads per kv head, value groups of >= 16 channels (>= 32 for 1-bit groups), and the
-// channels of each width filling whole 32-bit words.
+// channels of each width filling whole 32-bit words.  The map is read at run time from the
+// slot tables; a map listed at build time (MapSpec) gets an instance whose expansion loops
+// are unrolled and whose value-group tables are constants.
 #include <string.h>
 
 #include "../../include/kvq.h"
