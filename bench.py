@@ -245,18 +245,64 @@ def run_reference(args, w):
 
 
 # ------------------------------------------------------------------ GPU arm -------
+def step_plan(cfg: dict, L0: int, first: int, count: int):
+    """Per append+decode step i in [first, first+count): (algorithmic bytes of its decode,
+    launches of this library's kernels), computed on the host before anything is timed."""
+    gk, R = cfg["group_k"], cfg["window"]
+
+    def q_of(L):          # quantized prefix after L tokens (the window rule of the cache)
+        return 0 if cfg["k_bits"] == 16 else max(L - R, 0) // gk * gk
+
+    out = []
+    for i in range(first, first + count):
+        L = L0 + i + 1
+        # append (one copy kernel for K and V; rotated keys take a second one), decode, combine
+        n = (2 if cfg.get("rot_keys") else 1) + 2
+        if q_of(L) != q_of(L - 1):
+            # a window group was quantized: keys, values, side code, retained set, and (paged)
+            # the new page's block-table entries
+            n += 2 + (1 if cfg.get("side_rank") else 0) + (1 if cfg["log_retain"] else 0)
+            n += 1 if cfg.get("paged") else 0
+        out.append((decode_bytes(cfg, L), n))
+    return out
+
+
+def prefill_bytes(cfg: dict, L: int) -> int:
+    """Algorithmic bytes of a prefill of L tokens per sequence: every input key and value
+    read once; codes, (scale, zero), side codes, the fp16 window and the retained copies
+    written once (and, paged, the block-table entries)."""
+    B, H, dk, dv = cfg["batch"], cfg["n_kv_heads"], cfg["d_k"], cfg["d_v"]
+    kb, gk, gv, R = cfg["k_bits"], cfg["group_k"], cfg["group_v"], cfg["window"]
+    read = B * H * L * (dk + dv) * 2
+    if kb == 16:
+        return read + B * H * L * (dk + dv) * 2
+    Q = max(L - R, 0) // gk * gk
+    nret = len(K.kvq_retained_positions(Q)) if cfg["log_retain"] else 0
+    sr, sq = cfg.get("side_rank", 0), cfg.get("side_bits", 0)
+    if kb == 0:
+        kbytes = 4 * max(1, -(-sum(cfg["k_widths"][:dk]) // 32))
+        vbytes = 4 * max(1, -(-sum(cfg["v_widths"][:dv]) // 32))
+    else:
+        kbytes, vbytes = dk * kb // 8, dv * cfg["v_bits"] // 8
+    per_tok = kbytes + vbytes + (dv // gv) * 4 + sr * sq // 8
+    written = Q * per_tok + (Q // gk) * (dk * 4 + sr * 4) + (L - Q + nret) * (dk + dv) * 2
+    table = B * (Q // gk) * 4 if cfg.get("paged") else 0
+    return read + B * H * written + table
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
-    ap.add_argument("--workload", default="long32k", choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default="long32k", choices=W.ALL_KEYS)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     args = ap.parse_args()
-    w = W.WORKLOADS[args.workload]
+    w = W.by_key(args.workload)
     if args.batch:
         w = w.with_(batch=args.batch)
     if args.impl == "reference":
@@ -279,51 +325,52 @@ def main():
     inp = W.Inputs(wl, device=dev)
     cache = K.KVCache(cfg, device=dev, side_basis=inp.side_basis)
     stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = peaks()
 
-    # prefill (timed for information)
+    # prefill: three calls on the same inputs (each one resets the cache), median of the
+    # last two; the first is reported as well
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    cache.prefill(inp.k, inp.v)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    prefill_ms = e0.elapsed_time(e1)
+    pre_ms = []
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cache.prefill(inp.k, inp.v)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        pre_ms.append(e0.elapsed_time(e1))
+    pre_bytes = prefill_bytes(cfg, wl.context)
+    pre_med = statistics.median(pre_ms[1:])
     del inp.k, inp.v
     torch.cuda.empty_cache()
 
     out = torch.empty((wl.batch, wl.n_q_heads, wl.d_v), dtype=torch.float16, device=dev)
     n_ev = steps + warm
+    step_start = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    launches = 0
-    bytes_read = []
-
     L0, _, _ = cache.state()
-    gk, R = cfg["group_k"], cfg["window"]
+    plan_steps = step_plan(cfg, L0, warm, steps)
+    bytes_read = [b for b, _ in plan_steps]
+    launches = sum(n for _, n in plan_steps)
 
-    def q_of(L):          # quantized prefix after L tokens (the window rule of the cache)
-        return 0 if cfg["k_bits"] == 16 else max(L - R, 0) // gk * gk
+    # a decode whose bytes are not well above the L2 size would find part of them in L2 at
+    # the next step: then L2 is flushed (a write of twice its size) before every step,
+    # outside the step's events, and the step time is the mean of the steps' own events
+    l2 = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20))
+    flush = bytes_read[0] < 4 * l2
+    flush_buf = torch.empty(2 * l2, dtype=torch.uint8, device=dev) if flush else None
 
-    def step(i, timed):
-        nonlocal launches
-        L = L0 + i + 1
-        q0, q1 = q_of(L - 1), q_of(L)
+    def step(i):
+        if flush:
+            flush_buf.zero_()
+        step_start[i].record(stream)
         cache.append(inp.k_app[i], inp.v_app[i])
         starts[i].record(stream)
         cache.decode(inp.q[i], out=out)
         ends[i].record(stream)
-        if timed:
-            # append (one copy kernel for K and V; rotated keys take a second one), then the
-            # decode and the combine
-            launches += (2 if cfg.get("rot_keys") else 1) + 2
-            if q1 != q0:     # a window group was quantized: keys, values, side code, retained set,
-                             # and (paged) the new page's block-table entries
-                launches += 2 + (1 if cfg.get("side_rank") else 0) + (1 if cfg["log_retain"] else 0)
-                launches += 1 if cfg.get("paged") else 0
-            bytes_read.append(decode_bytes(cfg, L))
 
     for i in range(warm):
-        step(i, False)
+        step(i)
     clocks = ClockSampler(local)
     if dist:
         dist.barrier()
@@ -332,7 +379,7 @@ def main():
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(warm, warm + steps):
-        step(i, True)
+        step(i)
     t1.record(stream)
     while not t1.query():
         time.sleep(0.0002)
@@ -341,20 +388,79 @@ def main():
     if dist:
         dist.barrier()
     clk = clocks.stop()
-    total_ms = t0.elapsed_time(t1)
+    region_ms = t0.elapsed_time(t1)
+    step_ms = [step_start[i].elapsed_time(ends[i]) for i in range(warm, warm + steps)]
     dec_ms = [starts[i].elapsed_time(ends[i]) for i in range(warm, warm + steps)]
+    total_ms = sum(step_ms) if flush else region_ms
     dec_avg = sum(dec_ms) / len(dec_ms)
+    dec_med = statistics.median(dec_ms)
     status = cache.status()
-    total_ms, dec_avg = max_over_ranks([total_ms, dec_avg], dist, dev)
+    total_ms, dec_avg, dec_med = max_over_ranks([total_ms, dec_avg, dec_med], dist, dev)
     ms_step = total_ms / steps
     value = world * wl.batch / (ms_step / 1e3)
     achieved = (sum(bytes_read) / len(bytes_read)) / (dec_avg / 1e3) / 1e9
-    peak, peak_kind = peaks()
 
-    # end to end through the public API: every step copies its inputs from pinned host memory
-    # and its output back to pinned host memory.  The copies run on two copy streams with
-    # double-buffered device tensors, so step i's input copy overlaps step i-1's decode and
-    # step i's output copy overlaps step i+1's; every copy still lies inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_leg(wl, cfg, inp, out, steps, dev, stream, dist, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, spent, seqs, threads = oracle_decode_sample(w, args.cpu_budget, steps=8)
+        cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{seqs} append+decode steps of 1 of {w.batch} sequences "
+                         f"(all {w.n_kv_heads} kv heads, context {w.context}) in {spent:.1f} s"}
+
+    if rank == 0:
+        plan = cache.plan()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded; keys N(0,1)*sigma_c+mu_c with log-uniform sigma, values/q N(0,1))",
+            "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
+                       "n_kv_heads": wl.n_kv_heads, "d_k": wl.d_k, "d_v": wl.d_v,
+                       "context": wl.context, "k_bits": wl.k_bits, "v_bits": wl.v_bits,
+                       "group_k": wl.group_k, "group_v": wl.group_v, "window": wl.window,
+                       "log_retain": wl.log_retain, "parallelism": f"dp{world} (independent batches)",
+                       "l2": ("flushed before every step (write of %d MB, outside the step's events); "
+                              "each decode reads %.1f MB" % (2 * l2 >> 20, bytes_read[0] / 1e6)) if flush
+                             else "no flush: each decode reads %.0f MB > 4 x L2" % (bytes_read[0] / 1e6),
+                       "timing": "mean of the steps' own events" if flush
+                                 else "events around the whole timed region",
+                       "step": "append 1 token + decode, per sequence",
+                       "plan": plan},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak,
+                         "traffic": None if args.batch else profile_traffic(args.workload),
+                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                         "kernel": "decode (split-K kernel + combine), CUDA events per launch",
+                         "decode_ms": dec_avg, "decode_ms_median": dec_med,
+                         "bytes_per_launch": bytes_read[0]},
+            "decode_tokens_per_s": world * wl.batch / (dec_avg / 1e3),
+            "prefill": {"ms": pre_med, "ms_first_call": pre_ms[0], "tokens": wl.batch * wl.context,
+                        "bytes": pre_bytes, "achieved_gbs": pre_bytes / (pre_med / 1e3) / 1e9,
+                        "frac": pre_bytes / (pre_med / 1e3) / 1e9 / peak,
+                        "note": "algorithmic bytes: K and V read once, cache written once; "
+                                "median of calls 2 and 3"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    del cache
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_leg(wl, cfg, inp, out, steps, dev, stream, dist, world):
+    """End to end through the public API: every step copies its inputs from pinned host memory
+    and its output back to pinned host memory.  The copies run on two copy streams with
+    double-buffered device tensors, so step i's input copy overlaps step i-1's decode and step
+    i's output copy overlaps step i+1's; every copy still lies inside the timed region."""
     h_q = [x.cpu().pin_memory() for x in inp.q[:steps]]
     h_k = [x.cpu().pin_memory() for x in inp.k_app[:steps]]
     h_v = [x.cpu().pin_memory() for x in inp.v_app[:steps]]
@@ -411,54 +517,14 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = a.elapsed_time(b) / max(n_e2e, 1)
     (e2e_ms,) = max_over_ranks([e2e_ms], dist, dev)
-    d_q, d_k, d_v = d_q[0], d_k[0], d_v[0]
-    h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
+    h2d = (d_q[0].numel() + d_k[0].numel() + d_v[0].numel()) * 2
     d2h = out.numel() * 2
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v_cpu, spent, seqs, threads = oracle_decode_sample(w, args.cpu_budget, steps=8)
-        cpu = {"value": v_cpu, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"{seqs} append+decode steps of 1 of {w.batch} sequences "
-                         f"(all {w.n_kv_heads} kv heads, context {w.context}) in {spent:.1f} s"}
-
-    if rank == 0:
-        plan = cache.plan()
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
-            "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic (seeded; keys N(0,1)*sigma_c+mu_c with log-uniform sigma, values/q N(0,1))",
-            "config": {"workload": wl.name, "batch_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
-                       "n_kv_heads": wl.n_kv_heads, "d_k": wl.d_k, "d_v": wl.d_v,
-                       "context": wl.context, "k_bits": wl.k_bits, "v_bits": wl.v_bits,
-                       "group_k": wl.group_k, "group_v": wl.group_v, "window": wl.window,
-                       "log_retain": wl.log_retain, "parallelism": f"dp{world} (independent batches)",
-                       "l2": "no flush: each decode reads %.0f MB > 126 MB L2" % (bytes_read[0] / 1e6),
-                       "step": "append 1 token + decode, per sequence",
-                       "plan": plan},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak,
-                         "traffic": None if args.batch else profile_traffic(args.workload),
-                         "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                         "kernel": "decode (split-K kernel + combine), CUDA events per launch",
-                         "decode_ms": dec_avg, "bytes_per_launch": bytes_read[0]},
-            "decode_tokens_per_s": world * wl.batch / (dec_avg / 1e3),
-            "prefill_ms": prefill_ms,
-            "cpu_baseline": cpu,
-            "e2e": {"value": world * wl.batch / (e2e_ms / 1e3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "copies": "pinned host <-> device every step, on two copy streams that "
-                              "overlap the neighbouring steps' decodes"},
-            "gpu_launches": launches,
-            "clocks": clk,
-            "device_status": status,
-        }
-        print(json.dumps(line), flush=True)
-    del cache, e2e_cache
-    if dist:
-        dist.barrier()
-        dist.destroy_process_group()
+    del e2e_cache
+    torch.cuda.empty_cache()
+    return {"value": world * wl.batch / (e2e_ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "copies": "pinned host <-> device every step, on two copy streams that "
+                      "overlap the neighbouring steps' decodes"}
 
 
 if __name__ == "__main__":

@@ -281,9 +281,13 @@ int kvq_set_decode_kernel(kvq_cache* cache, int kernel);
  * process exits.  Nothing is allocated at call time.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress, with that
  * device current); make that first call before any stream capture.  The array
- * is shared by every call and keeps the last call's contents (this call clears
- * the status word it needs at zero); calls whose executions overlap on the GPU
- * race on it, so issue them on one stream or otherwise serialize them.
+ * is shared by every call and keeps the last call's contents; calls whose
+ * executions overlap on the GPU race on it, so issue them on one stream or
+ * otherwise serialize them.  Its first word is a status word like a workspace's:
+ * zero when the library is loaded, ORed with KVQ_STATUS_* bits by any call whose
+ * bounded waits gave up (that call's output is then undefined), never cleared by
+ * a decode; read it with kvq_noalloc_read_status, clear it with
+ * kvq_noalloc_reset_status (both for the current device).
  * num_splits: 0 = automatic, reduced if needed so that the partials fit in the
  * array; an explicit split count whose partials do not fit, or a cache so large
  * that even one split per (b, kv head) does not fit, returns KVQ_ERR_WORKSPACE.
@@ -291,6 +295,13 @@ int kvq_set_decode_kernel(kvq_cache* cache, int kernel);
 #define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 int kvq_decode_attention_noalloc(kvq_cache* cache, const void* q, void* out, int num_splits,
                                  void* stream);
+
+/* Status word of the current device's scratch array (see kvq_decode_attention_noalloc):
+ * kvq_noalloc_read_status waits for stream, then copies the word to *status (it
+ * synchronizes, like kvq_read_status); kvq_noalloc_reset_status zeroes it,
+ * asynchronously on stream.  Errors: INVALID_ARG (status NULL), CUDA. */
+int kvq_noalloc_read_status(unsigned int* status, void* stream);
+int kvq_noalloc_reset_status(void* stream);
 
 /* The plan kvq_decode_attention would use now (host only, no launch); its counts are
  * those of the longest sequence. */

@@ -13,7 +13,14 @@
 // exits.  In host code its name is only a host-side stand-in, not a device
 // address, so the real address is looked up once per device with
 // cudaGetSymbolAddress while that device is current, and passed on as the
-// workspace pointer.  That lookup happens inside the first call on each device.
+// workspace pointer.  That lookup happens inside the first call on each device
+// (of the decode or of the status calls below).
+//
+// Its first word is the status word the decode kernels OR KVQ_STATUS_* bits
+// into, exactly as in a caller's workspace: it starts at zero when the library
+// is loaded, is never cleared by a decode, and is read and cleared by
+// kvq_noalloc_read_status / kvq_noalloc_reset_status.
+#include <atomic>
 #include <mutex>
 
 #include "../../include/kvq.h"
@@ -27,25 +34,29 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
 std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
+std::atomic<void*> g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device (looked up once per device).
+// Device address of g_decode_scratch on the current device (looked up once per device;
+// later calls read the cached address without taking the lock).
 int scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     cudaGetLastError();
     return KVQ_ERR_CUDA;
   }
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return KVQ_ERR_CUDA;
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
+    if (!p) {
+      if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return KVQ_ERR_CUDA;
+      }
+      g_scratch_ptr[dev].store(p, std::memory_order_release);
     }
-    g_scratch_ptr[dev] = p;
   }
-  *out = g_scratch_ptr[dev];
+  *out = p;
   return KVQ_OK;
 }
 
@@ -79,11 +90,20 @@ extern "C" int kvq_decode_attention_noalloc(kvq_cache* cache, const void* q, voi
   void* scratch = nullptr;
   rc = scratch_for_current_device(&scratch);
   if (rc) return rc;
-  // the array keeps the previous call's contents: the status word must start at zero
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, sizeof(unsigned int), s) != cudaSuccess) {
-    cudaGetLastError();
-    return KVQ_ERR_CUDA;
-  }
   return kvq_decode_attention(cache, q, out, scratch, kNoAllocScratchBytes, splits, stream);
+}
+
+extern "C" int kvq_noalloc_read_status(unsigned int* status, void* stream) {
+  if (!status) return KVQ_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const int rc = scratch_for_current_device(&scratch);
+  if (rc) return rc;
+  return kvq_read_status(scratch, status, stream);
+}
+
+extern "C" int kvq_noalloc_reset_status(void* stream) {
+  void* scratch = nullptr;
+  const int rc = scratch_for_current_device(&scratch);
+  if (rc) return rc;
+  return kvq_reset_status(scratch, stream);
 }

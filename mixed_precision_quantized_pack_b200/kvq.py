@@ -89,6 +89,8 @@ _SIGNATURES = {
     "kvq_decode_workspace_size": (_I, [_P, _I, ctypes.POINTER(ctypes.c_size_t)]),
     "kvq_decode_attention": (_I, [_P, _P, _P, _P, ctypes.c_size_t, _I, _P]),
     "kvq_decode_attention_noalloc": (_I, [_P, _P, _P, _I, _P]),
+    "kvq_noalloc_read_status": (_I, [ctypes.POINTER(ctypes.c_uint), _P]),
+    "kvq_noalloc_reset_status": (_I, [_P]),
     "kvq_get_plan": (_I, [_P, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_set_decode_kernel": (_I, [_P, _I]),
     "kvq_debug_stall_next_decode": (_I, [_P]),
@@ -250,6 +252,17 @@ def kvq_decode_attention_noalloc(handle: int, q_ptr: int, out_ptr: int, num_spli
     """Decode without a workspace: the partials go to the library's own scratch array."""
     _check(lib().kvq_decode_attention_noalloc(handle, q_ptr, out_ptr, int(num_splits), stream),
            "kvq_decode_attention_noalloc")
+
+
+def kvq_noalloc_read_status(stream: int) -> int:
+    """Status word of the library's scratch array on the current device (waits for stream)."""
+    st = ctypes.c_uint()
+    _check(lib().kvq_noalloc_read_status(ctypes.byref(st), stream), "kvq_noalloc_read_status")
+    return int(st.value)
+
+
+def kvq_noalloc_reset_status(stream: int) -> None:
+    _check(lib().kvq_noalloc_reset_status(stream), "kvq_noalloc_reset_status")
 
 
 def kvq_get_plan(handle: int, num_splits: int = 0) -> Dict[str, int]:

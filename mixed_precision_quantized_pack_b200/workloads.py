@@ -24,7 +24,10 @@ values do not):
 Everything is drawn in fp32 from one ``torch.Generator`` seeded per workload and
 rounded once to fp16.  The generator lives on the device the tensors are made on,
 so a CPU and a CUDA draw of the same seed differ; each test or benchmark uses
-one of them and copies across as needed.
+one of them and copies across as needed.  Workloads with ``per_seq`` set (the
+131072-token sweep) draw each sequence's prefill keys and values from a
+generator of its own, seeded with (seed, b), so a batch of 64 such sequences
+is made one sequence at a time and any one sequence can be drawn alone.
 """
 from __future__ import annotations
 
@@ -61,6 +64,7 @@ class Workload:
     paged: int = 0        # quantized groups in a page pool just large enough for max_context
     k_widths: tuple = ()  # k_bits = v_bits = 0: per-channel key widths ...
     v_widths: tuple = ()  # ... and value widths (data, given with the workload)
+    per_seq: int = 0      # 1: prefill K/V drawn per sequence from generators seeded (seed, b)
 
     @property
     def n_rep(self) -> int:
@@ -147,7 +151,33 @@ def sweep_workload(batch: int, k_bits: int, v_bits: int, appends: int = 256) -> 
     return _base(name=f"sweep-b{batch}-k{k_bits}v{v_bits}-128k", batch=batch, n_q_heads=32,
                  n_kv_heads=8, d_k=128, d_v=128, context=131072, k_bits=k_bits, v_bits=v_bits,
                  group_k=64, group_v=64, window=128, log_retain=0, appends=appends,
-                 seed=1004)
+                 seed=1004, per_seq=1)
+
+
+def sweep_key(batch: int, k_bits: int, v_bits: int) -> str:
+    return f"sweep-b{batch}-k{k_bits}v{v_bits}"
+
+
+SWEEP_KEYS = [sweep_key(b, kb, vb) for b in SWEEP_BATCHES for kb, vb in SWEEP_BITS]
+ALL_KEYS = list(WORKLOADS) + SWEEP_KEYS
+
+
+def by_key(key: str) -> Workload:
+    """A named workload, or a sweep point "sweep-b<B>-k<kb>v<vb>"."""
+    if key in WORKLOADS:
+        return WORKLOADS[key]
+    for b in SWEEP_BATCHES:
+        for kb, vb in SWEEP_BITS:
+            if key == sweep_key(b, kb, vb):
+                return sweep_workload(b, kb, vb)
+    raise KeyError(f"unknown workload {key!r}; known: {', '.join(ALL_KEYS)}")
+
+
+def sequence_generator(w: Workload, b: int, device) -> torch.Generator:
+    """The generator of sequence b's prefill keys and values (per_seq workloads)."""
+    gen = torch.Generator(device=torch.device(device))
+    gen.manual_seed(w.seed * 1_000_003 + b)
+    return gen
 
 
 def _keys(gen: torch.Generator, device, batch: int, heads: int, tokens: int, d: int,
@@ -184,18 +214,28 @@ class Inputs:
                                dtype=torch.float32) / math.sqrt(w.thin_from)
         self.sigma, self.mu, self.proj = sigma, mu, proj
 
-        def keys(batch, tokens):
-            k = _keys(gen, dev, batch, w.n_kv_heads, tokens, d_src, sigma, mu)
+        def keys(batch, tokens, g=gen):
+            k = _keys(g, dev, batch, w.n_kv_heads, tokens, d_src, sigma, mu)
             if proj is not None:
                 k = k @ proj
             return k.to(torch.float16)
 
-        def normal(shape):
-            return torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).to(torch.float16)
+        def normal(shape, g=gen):
+            return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.float16)
 
         B = w.batch
-        self.k = keys(B, w.context)
-        self.v = normal((B, w.n_kv_heads, w.context, w.d_v))
+        rows = range(B) if batch_slice is None else range(B)[batch_slice]
+        if w.per_seq:
+            # sequence by sequence (only the sequences of batch_slice are drawn)
+            self.k = torch.empty((len(rows), w.n_kv_heads, w.context, w.d_k), dtype=torch.float16, device=dev)
+            self.v = torch.empty((len(rows), w.n_kv_heads, w.context, w.d_v), dtype=torch.float16, device=dev)
+            for i, b in enumerate(rows):
+                g = sequence_generator(w, b, dev)
+                self.k[i] = keys(1, w.context, g)[0]
+                self.v[i] = normal((w.n_kv_heads, w.context, w.d_v), g)
+        else:
+            self.k = keys(B, w.context)
+            self.v = normal((B, w.n_kv_heads, w.context, w.d_v))
         self.side_basis: Optional[torch.Tensor] = None
         if w.side_rank:
             g = torch.randn((w.n_kv_heads, w.d_k, w.side_rank), generator=gen, device=dev,
@@ -223,8 +263,9 @@ class Inputs:
                 self.k_app.append(keys(B, 1)[:, :, 0, :].contiguous())
                 self.v_app.append(normal((B, w.n_kv_heads, w.d_v)))
         if batch_slice is not None:
-            self.k = self.k[batch_slice].contiguous()
-            self.v = self.v[batch_slice].contiguous()
+            if not w.per_seq:
+                self.k = self.k[batch_slice].contiguous()
+                self.v = self.v[batch_slice].contiguous()
             self.q = [x[batch_slice].contiguous() for x in self.q]
             self.k_app = [x[batch_slice].contiguous() for x in self.k_app]
             self.v_app = [x[batch_slice].contiguous() for x in self.v_app]

@@ -65,3 +65,52 @@ def test_width_map_rows_are_counted_in_words():
     sizes = K.kvq_buffer_sizes(c)
     lcap = -(-c["max_context"] // 64) * 64
     assert sizes["kcode"] == 32 * 8 * lcap * 14 * 4 and sizes["vcode"] == 32 * 8 * lcap * 9 * 4
+
+
+@pytest.mark.parametrize("key", list(W.WORKLOADS) + ["sweep-b8-k8v4", "sweep-b1-k16v16"])
+def test_prefill_bytes_read_the_inputs_once_and_write_the_layout_once(key):
+    w = W.by_key(key)
+    c = w.kvq_config()
+    L = w.context
+    B, H, dk, dv = w.batch, w.n_kv_heads, w.d_k, w.d_v
+    got = bench.prefill_bytes(c, L)
+    read = B * H * L * (dk + dv) * 2
+    if w.k_bits == 16:
+        assert got == 2 * read
+        return
+    bb = O.buffer_bytes(dict(c, batch=1, n_kv_heads=1))
+    lcap = -(-c["max_context"] // w.group_k) * w.group_k
+    per_tok = (bb["kcode"] + bb["vcode"] + bb["vsz"] + bb["zcode"]) // lcap
+    per_group = (bb["ksz"] + bb["zsz"]) // (lcap // w.group_k)
+    Q = O.quantized_prefix(L, w.window, w.group_k, w.k_bits)
+    nret = len(O.retained_positions(Q)) if w.log_retain else 0
+    want = read + B * H * (Q * per_tok + (Q // w.group_k) * per_group + (L - Q + nret) * (dk + dv) * 2)
+    if w.paged:
+        want += B * (Q // w.group_k) * 4
+    assert got == want
+
+
+def test_every_sweep_point_has_a_key():
+    keys = set(W.SWEEP_KEYS)
+    assert len(keys) == 16
+    for b in W.SWEEP_BATCHES:
+        for kb, vb in W.SWEEP_BITS:
+            w = W.by_key(f"sweep-b{b}-k{kb}v{vb}")
+            assert (w.batch, w.k_bits, w.v_bits, w.context) == (b, kb, vb, 131072)
+            assert w.per_seq == 1
+    with pytest.raises(KeyError):
+        W.by_key("sweep-b3-k4v2")
+
+
+def test_step_plan_counts_the_group_quantize_launches():
+    """A step whose append makes the window R + G_k long also quantizes one group: keys, values
+    (and retained set, side code, table entries when the cache has them)."""
+    w = W.WORKLOADS["long32k"]
+    c = w.kvq_config(max_context=w.context + 200)
+    L0 = w.context
+    plan = bench.step_plan(c, L0, 0, 130)
+    crossing = [i for i in range(130) if (L0 + i + 1 - 128) // 64 != (L0 + i - 128) // 64]
+    assert crossing
+    for i, (nbytes, n) in enumerate(plan):
+        assert nbytes == bench.decode_bytes(c, L0 + i + 1)
+        assert n == 3 + (3 if i in crossing else 0)
