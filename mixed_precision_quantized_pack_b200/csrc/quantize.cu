@@ -17,6 +17,12 @@
 namespace kvq {
 namespace {
 
+// Shared-memory tables of the key quantizer: (zero, 1/scale, scale) per (group of a CTA,
+// channel) and the groups' (scale, zero) blocks; a CTA holds at most 2048 / gk * R channels'
+// parameters (512 for gk = 16 with 4 rows per thread).
+constexpr int kKeyPrm = 512;
+constexpr int kKeyBlk = 2 * kKeyPrm;
+
 struct GroupParams {
   float scale;   // fp32 value of the fp16 scale
   float zero;    // fp32 value of the fp16 zero
@@ -50,77 +56,203 @@ __device__ __forceinline__ GroupParams group_params(float mn, float mx) { return
 template <int BITS>
 __device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g) { return quant_code_b(x, g, BITS); }
 
-// One thread per (key group, channel); blockDim = (dk, groups per block).  The
-// 32/BITS lanes holding the channels of one packed word OR their codes together.
-// ROT: the source keys are unrotated; the block's warps first rotate the rows of its
-// groups into shared memory ([groups per block][gk][dk] fp16) and the quantizer reads
-// those.
-template <int BITS, bool ROT>
-__global__ void quantize_keys_kernel(const __half* __restrict__ src, int src_rows, int dk,
-                                     int gk, int g_begin, int n_groups, int lcap,
-                                     uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
-                                     const int* __restrict__ table, Dims d) {
-  extern __shared__ __half sm_rot[];
-  const int c = threadIdx.x;
-  const int gi = blockIdx.x * blockDim.y + threadIdx.y;
-  const int bh = blockIdx.y;
-  const size_t base = static_cast<size_t>(bh) * src_rows;
-  if constexpr (ROT) {
-    const int tid = threadIdx.y * blockDim.x + threadIdx.x;
-    const int lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x * blockDim.y / 32;
-    for (int rr = warp; rr < blockDim.y * gk; rr += nwarps) {
-      const int yy = rr / gk, t = rr % gk;
-      const int gg = blockIdx.x * blockDim.y + yy;
-      if (gg >= n_groups) continue;                  // uniform per warp
-      const int row = ((g_begin + gg) * gk + t) % src_rows;
-      float x[8];
+// The code of one element from the group's zero z and the reciprocal r = fl32(1/s) of its
+// scale, equal to the quantizer's rint(fl32(fl32(x - z) / s)) clamped to [0, 2^b - 1]
+// wherever `near` stays false:
+//   the quotient Q = d/s (d = fl32(x - z) >= 0) is below 512 (s is the fp16 rounding of
+//   (max - min)/(2^b - 1) with b <= 8, or a subnormal at most 1.5x smaller, or 0 and then r = 0
+//   and every code 0); q = fl32(d * r) = Q (1 + e1)(1 + e2) with |e1|, |e2| <= 2^-24, so
+//   |q - Q| <= 2^-14, and the IEEE quotient fl32(Q) is within half an ulp, 2^-16, of Q.  If q
+//   lies more than 2^-13 from every half-integer (|q - rint(q)| <= 1/2 - 2^-13; q - rint(q) is
+//   exact by Sterbenz), Q and fl32(Q) lie strictly inside q's rounding cell and round to the
+//   same integer.  Otherwise `near` is set and the caller takes the IEEE division.
+constexpr float kNearHalf = 0.5f - 1.0f / 8192.0f;
+
+__device__ __forceinline__ uint32_t code_fast_l(float x, float z, float r, float levels, bool& near) {
+  const float q = __fmul_rn(__fsub_rn(x, z), r);
+  const float c = rintf(q);
+  near |= fabsf(__fsub_rn(q, c)) > kNearHalf;
+  return static_cast<uint32_t>(fminf(c, levels));
+}
+
+// The quantizer's code with the IEEE division (the rare elements code_fast leaves undecided).
+__device__ __forceinline__ uint32_t code_exact_l(float x, float z, float s, float levels) {
+  if (s == 0.0f) return 0u;
+  float c = rintf(__fdiv_rn(__fsub_rn(x, z), s));
+  c = fminf(fmaxf(c, 0.0f), levels);
+  return static_cast<uint32_t>(c);
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t code_fast(float x, float z, float r, bool& near) {
+  return code_fast_l(x, z, r, static_cast<float>((1 << BITS) - 1), near);
+}
+
+template <int BITS>
+__device__ __forceinline__ uint32_t code_exact(float x, float z, float s) {
+  return code_exact_l(x, z, s, static_cast<float>((1 << BITS) - 1));
+}
+
+// Codes of 8 consecutive channels (one 16-byte chunk of fp16) packed LSB-first: 8 * BITS bits.
+// Channel j's group has zero z[j], reciprocal scale r[j] and scale sc[j] (keys: one group per
+// channel), or every channel the same (values: STRIDE 0 reads element 0 for all j).
+template <int BITS, int STRIDE>
+__device__ __forceinline__ uint64_t pack_chunk(const uint4& raw, const float* z, const float* r,
+                                               const float* sc) {
+  const __half2* hx = reinterpret_cast<const __half2*>(&raw);
+  float x[8];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) x[m] = m < dk / 32 ? __half2float(src[(base + row) * dk + lane + 32 * m]) : 0.0f;
-      rotate_row_warp<8>(x, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(hx[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
+  }
+  bool near = false;
+  uint64_t bits = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    bits |= static_cast<uint64_t>(code_fast<BITS>(x[j], z[j * STRIDE], r[j * STRIDE], near)) << (j * BITS);
+  if (near) {             // rare: a quotient within 2^-13 of a half-integer
+    bits = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      bits |= static_cast<uint64_t>(code_exact<BITS>(x[j], z[j * STRIDE], sc[j * STRIDE])) << (j * BITS);
+  }
+  return bits;
+}
+
+// Key quantize-pack of whole key groups.  A group (gk tokens x dk channels of fp16) is split
+// into 16-byte chunks of 8 channels; thread (slab rs, chunk cc) of the group's TPG = dk/8 *
+// gk/R threads holds rows rs, rs + gk/R, ... (R rows) of chunk cc, so a warp's loads and
+// stores are whole consecutive rows.  Each key is read once: the per-channel min and max are
+// taken in fp16 (exact) per thread, reduced across the group's slabs in shared memory, turned
+// into (scale, zero) there, and the codes are computed from the registers.  A CTA of 256
+// threads holds 256 / TPG groups.  ROT: the source keys are unrotated; warps first rotate the
+// CTA's rows into shared memory and the chunks are read from there.
+template <int BITS, int R, bool ROT>
+__global__ void __launch_bounds__(256) quantize_keys_kernel(
+    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
+    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
+  extern __shared__ __align__(16) unsigned char sm_dyn[];          // ROT: [gpc * gk][dk] fp16
+  __shared__ __align__(16) __half2 red[2][256][4];                  // per thread: min, max
+  __shared__ __align__(16) float prm[3][kKeyPrm];                   // zero, 1/scale, scale
+  __shared__ __align__(16) __half blk[kKeyBlk];                     // (scale, zero) blocks
+  const int dk = d.dk, gk = d.gk;
+  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int tid = threadIdx.x;
+  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt % tpg / cpr;
+  const int bh = blockIdx.y, b = bh / d.Hkv, h = bh % d.Hkv;
+  const int g_first = blockIdx.x * gpc;           // first group of the CTA, among the launch's
+  const bool active = g_first + gi < n_groups;
+  const int g = g_begin + g_first + gi;
+  const size_t base = static_cast<size_t>(bh) * src_rows;
+
+  uint4 x[R];
+  if constexpr (ROT) {
+    __half* rot = reinterpret_cast<__half*>(sm_dyn);
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int rr = warp; rr < gpc * gk; rr += 8) {
+      const int yy = rr / gk, t = rr % gk;
+      if (g_first + yy >= n_groups) continue;                     // uniform per warp
+      const int row = ((g_begin + g_first + yy) * gk + t) % src_rows;
+      float v[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) v[m] = m < dk / 32 ? __half2float(src[(base + row) * dk + lane + 32 * m]) : 0.0f;
+      rotate_row_warp<8>(v, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
 #pragma unroll
       for (int m = 0; m < 8; ++m)
-        if (m < dk / 32) sm_rot[(static_cast<size_t>(yy) * gk + t) * dk + lane + 32 * m] = __float2half_rn(x[m]);
+        if (m < dk / 32) rot[static_cast<size_t>(rr) * dk + lane + 32 * m] = __float2half_rn(v[m]);
     }
     __syncthreads();
-  }
-  if (gi >= n_groups) return;                       // uniform per warp: dk % 32 == 0
-  const int g = g_begin + gi;
-  // key t of the group, channel c
-  auto key = [&](int t) -> float {
-    if constexpr (ROT) return __half2float(sm_rot[(static_cast<size_t>(threadIdx.y) * gk + t) * dk + c]);
-    const int row = (g * gk + t) % src_rows;
-    return __half2float(src[(base + row) * dk + c]);
-  };
-  float mn = INFINITY, mx = -INFINITY;
-  for (int t = 0; t < gk; ++t) {
-    const float x = key(t);
-    mn = fminf(mn, x);
-    mx = fmaxf(mx, x);
-  }
-  const GroupParams gp = group_params<BITS>(mn, mx);
-  {
-    // the group's block of 2*dk fp16: per packed word w, the scales of channels
-    // (w*per + i, w*per + i + per/2) for i < per/2, then their zeros in the same order;
-    // the words' blocks quarter-interleaved when 4 divides the words per row
-    constexpr int per_w = 32 / BITS, half_w = 16 / BITS;
-    const int words = dk / per_w, quarter = words % 4 == 0 ? words / 4 : 0;
-    const int wd = c / per_w, r = c % per_w;
-    const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
-    const int slot = pos * 2 * per_w + (r % half_w) * 2 + r / half_w;
-    __half* blk = reinterpret_cast<__half*>(ksz) + group_index(d, table, bh / d.Hkv, bh % d.Hkv, g) * 2 * dk;
-    blk[slot] = __low2half(gp.sz);
-    blk[slot + per_w] = __high2half(gp.sz);
-  }
-  constexpr int per = 32 / BITS;                    // channels per word
-  const int words = dk / per;
-  const size_t row0 = group_row(d, table, bh / d.Hkv, bh % d.Hkv, g);
-  for (int t = 0; t < gk; ++t) {
-    const float x = key(t);
-    uint32_t part = quant_code<BITS>(x, gp) << ((c % per) * BITS);
 #pragma unroll
-    for (int off = 1; off < per; off <<= 1) part |= __shfl_xor_sync(0xffffffffu, part, off);
-    if (c % per == 0)
-      kcode[(row0 + t) * words + c / per] = part;
+    for (int i = 0; i < R; ++i)
+      x[i] = reinterpret_cast<const uint4*>(rot)[(gi * gk + rs + slabs * i) * cpr + cc];
+  } else {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int row = (g * gk + rs + slabs * i) % src_rows;
+      x[i] = active ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
+                    : make_uint4(0, 0, 0, 0);
+    }
+  }
+  {
+    const __half2* h0 = reinterpret_cast<const __half2*>(&x[0]);
+    __half2 mn[4], mx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mn[k] = mx[k] = h0[k];
+#pragma unroll
+    for (int i = 1; i < R; ++i) {
+      const __half2* hi = reinterpret_cast<const __half2*>(&x[i]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        mn[k] = __hmin2(mn[k], hi[k]);
+        mx[k] = __hmax2(mx[k], hi[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      red[0][tid][k] = mn[k];
+      red[1][tid][k] = mx[k];
+    }
+  }
+  __syncthreads();
+  // per (group of the CTA, channel pair): reduce over the slabs, then (scale, zero)
+  constexpr int per_w = 32 / BITS, half_w = 16 / BITS;
+  const int words = dk / per_w, quarter = words % 4 == 0 ? words / 4 : 0;
+  for (int p = tid; p < gpc * dk / 2; p += 256) {
+    const int g2 = p / (dk / 2), pp = p % (dk / 2), c2 = pp / 4, k = pp % 4;
+    const int t0 = g2 * tpg + c2;
+    __half2 mn = red[0][t0][k], mx = red[1][t0][k];
+    for (int sl = 1; sl < slabs; ++sl) {
+      mn = __hmin2(mn, red[0][t0 + sl * cpr][k]);
+      mx = __hmax2(mx, red[1][t0 + sl * cpr][k]);
+    }
+    const float2 fmn = __half22float2(mn), fmx = __half22float2(mx);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = 8 * c2 + 2 * k + e;
+      const GroupParams gp = group_params<BITS>(e ? fmn.y : fmn.x, e ? fmx.y : fmx.x);
+      prm[0][g2 * dk + c] = gp.zero;
+      prm[1][g2 * dk + c] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+      prm[2][g2 * dk + c] = gp.scale;
+      // the group's block of 2*dk fp16: per packed word w, the scales of channels
+      // (w*per + i, w*per + i + per/2) for i < per/2, then their zeros in the same order;
+      // the words' blocks quarter-interleaved when 4 divides the words per row
+      const int wd = c / per_w, r = c % per_w;
+      const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
+      const int slot = pos * 2 * per_w + (r % half_w) * 2 + r / half_w;
+      blk[g2 * 2 * dk + slot] = __low2half(gp.sz);
+      blk[g2 * 2 * dk + slot + per_w] = __high2half(gp.sz);
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < gpc * dk / 4; i += 256) {                 // 16 B of a block per thread
+    const int g2 = i / (dk / 4), j = i % (dk / 4);
+    if (g_first + g2 >= n_groups) continue;
+    const size_t gidx = group_index(d, table, b, h, g_begin + g_first + g2);
+    reinterpret_cast<uint4*>(reinterpret_cast<__half*>(ksz) + gidx * 2 * dk)[j] =
+        reinterpret_cast<const uint4*>(blk + g2 * 2 * dk)[j];
+  }
+  if (!active) return;
+  float z[8], r[8], sc[8];
+#pragma unroll
+  for (int j = 0; j < 8; j += 4) {
+    *reinterpret_cast<float4*>(z + j) = *reinterpret_cast<const float4*>(&prm[0][gi * dk + 8 * cc + j]);
+    *reinterpret_cast<float4*>(r + j) = *reinterpret_cast<const float4*>(&prm[1][gi * dk + 8 * cc + j]);
+    *reinterpret_cast<float4*>(sc + j) = *reinterpret_cast<const float4*>(&prm[2][gi * dk + 8 * cc + j]);
+  }
+  const size_t row0 = group_row(d, table, b, h, g);
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const uint64_t bits = pack_chunk<BITS, 1>(x[i], z, r, sc);
+    const size_t row = row0 + rs + slabs * i;
+    if constexpr (BITS == 2)
+      reinterpret_cast<uint16_t*>(kcode)[row * (dk / 8) + cc] = static_cast<uint16_t>(bits);
+    else if constexpr (BITS == 4)
+      kcode[row * (dk / 8) + cc] = static_cast<uint32_t>(bits);
+    else
+      reinterpret_cast<uint2*>(kcode)[row * (dk / 8) + cc] =
+          make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
   }
 }
 
@@ -237,46 +369,63 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
   }
 }
 
-// One thread per (kv row, token, value group).  gv is a multiple of 8 and of 32/BITS.
-template <int BITS>
-__global__ void quantize_values_kernel(const __half* __restrict__ src, int src_rows, int dv,
-                                       int gv, int t_begin, int n_tokens, int nbh, int lcap,
-                                       uint32_t* __restrict__ vcode, __half2* __restrict__ vsz,
-                                       const int* __restrict__ table, Dims d) {
-  const int nvg = dv / gv;
-  const long long total = static_cast<long long>(nbh) * n_tokens * nvg;
-  constexpr int per = 32 / BITS;
-  const int vw = dv / per;
-  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int gidx = static_cast<int>(idx % nvg);
-    const long long r = idx / nvg;
-    const int t = t_begin + static_cast<int>(r % n_tokens);
-    const int bh = static_cast<int>(r / n_tokens);
-    const int row = t % src_rows;
-    const __half* x = src + (static_cast<size_t>(bh) * src_rows + row) * dv + gidx * gv;
-    float mn = INFINITY, mx = -INFINITY;
-    for (int j = 0; j < gv; j += 8) {
-      const uint4 u = *reinterpret_cast<const uint4*>(x + j);
-      const __half2* h = reinterpret_cast<const __half2*>(&u);
+// Value quantize-pack, per token row over groups of gv channels.  A row is dv/8 16-byte chunks
+// of 8 channels, one chunk per lane, so a warp covers 32 / (dv/8) rows per load and each lane
+// R rows (rows rsub, rsub + 32/(dv/8), ... of the warp's block).  A value group is gv/8
+// consecutive lanes (gv is a multiple of 8): min and max in fp16 per lane, then by shuffles
+// across the group's lanes; every lane of a group derives the same (scale, zero).  Lane 0 of a
+// group writes its (scale, zero); each lane writes its chunk's 8 * BITS bits of codes.
+template <int BITS, int R>
+__global__ void __launch_bounds__(256) quantize_values_kernel(
+    const __half* __restrict__ src, int src_rows, int t_begin, int n_tokens,
+    uint32_t* __restrict__ vcode, __half2* __restrict__ vsz, const int* __restrict__ table, Dims d) {
+  const int dv = d.dv, cpr = dv / 8, rpw = 32 / cpr, gl = d.gv / 8;
+  const int lane = threadIdx.x & 31;
+  const int cc = lane % cpr, rsub = lane / cpr;
+  const long long rows = static_cast<long long>(d.B) * d.Hkv * n_tokens;
+  const long long block_rows = static_cast<long long>(rpw) * R;          // rows per warp block
+  const long long n_blocks = (rows + block_rows - 1) / block_rows;
+  for (long long wb = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; wb < n_blocks;
+       wb += static_cast<long long>(gridDim.x) * blockDim.x / 32) {
+    uint4 x[R];
+    long long ri[R];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h[e]);
-        mn = fminf(mn, fminf(f.x, f.y));
-        mx = fmaxf(mx, fmaxf(f.x, f.y));
+    for (int i = 0; i < R; ++i) {
+      ri[i] = wb * block_rows + rsub + static_cast<long long>(rpw) * i;
+      if (ri[i] < rows) {
+        const int bh = static_cast<int>(ri[i] / n_tokens);
+        const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
+        x[i] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + cc);
+      } else {
+        x[i] = make_uint4(0, 0, 0, 0);
       }
     }
-    const GroupParams gp = group_params<BITS>(mn, mx);
-    const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
-    vsz[vrow * nvg + gidx] = gp.sz;
-    uint32_t* out = vcode + vrow * vw + gidx * (gv / per);
-    for (int w = 0; w < gv / per; ++w) {
-      uint32_t word = 0;
-      for (int k = 0; k < per; ++k) {
-        const float xv = __half2float(x[w * per + k]);
-        word |= quant_code<BITS>(xv, gp) << (k * BITS);
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const __half2* hx = reinterpret_cast<const __half2*>(&x[i]);
+      __half2 mn2 = __hmin2(__hmin2(hx[0], hx[1]), __hmin2(hx[2], hx[3]));
+      __half2 mx2 = __hmax2(__hmax2(hx[0], hx[1]), __hmax2(hx[2], hx[3]));
+      float mn = fminf(__low2float(mn2), __high2float(mn2));
+      float mx = fmaxf(__low2float(mx2), __high2float(mx2));
+      for (int off = 1; off < gl; off <<= 1) {         // lanes of one group: aligned, consecutive
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       }
-      out[w] = word;
+      if (ri[i] >= rows) continue;
+      const GroupParams gp = group_params<BITS>(mn, mx);
+      const int bh = static_cast<int>(ri[i] / n_tokens);
+      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
+      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
+      if (cc % gl == 0) vsz[vrow * d.nvg + cc / gl] = gp.sz;
+      const float rcp = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+      const uint64_t bits = pack_chunk<BITS, 0>(x[i], &gp.zero, &rcp, &gp.scale);
+      if constexpr (BITS == 2)
+        reinterpret_cast<uint16_t*>(vcode)[vrow * cpr + cc] = static_cast<uint16_t>(bits);
+      else if constexpr (BITS == 4)
+        vcode[vrow * cpr + cc] = static_cast<uint32_t>(bits);
+      else
+        reinterpret_cast<uint2*>(vcode)[vrow * cpr + cc] =
+            make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
     }
   }
 }
@@ -286,98 +435,236 @@ __global__ void quantize_values_kernel(const __half* __restrict__ src, int src_r
 // non-increasing over the channels; the same quantizer with that many bits; a row packs
 // the codes channel after channel, channel c at the sum of the widths before it.
 
-// One CTA of dk threads per (key group, b * kv head): thread c quantizes channel c over the
-// group's gk tokens; the codes are ORed into the group's rows in shared memory
-// ([gk][kw] u32, at most 128 x 64 words), which are then written out whole.  The group's
-// (scale, zero) are stored plainly, [dk][2]; a dropped channel stores (0, 0).
-__global__ void quantize_keys_var_kernel(const __half* __restrict__ src, int src_rows, int g_begin,
-                                         uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
-                                         const int* __restrict__ table, Dims d) {
-  extern __shared__ uint32_t sm_rows[];
-  const int c = threadIdx.x, nt = blockDim.x;
-  const int g = g_begin + blockIdx.x, bh = blockIdx.y;
-  const int gk = d.gk, kw = d.kw;
-  for (int i = c; i < gk * kw; i += nt) sm_rows[i] = 0u;
-  __syncthreads();
-  int width, offset;
-  channel_width(d.kcnt, c, &width, &offset);
-  const size_t base = static_cast<size_t>(bh) * src_rows;
-  auto key = [&](int t) { return __half2float(src[(base + (g * gk + t) % src_rows) * d.dk + c]); };
-  const size_t gidx = group_index(d, table, bh / d.Hkv, bh % d.Hkv, g);
-  __half2 sz = __floats2half2_rn(0.0f, 0.0f);
-  if (width) {
-    float mn = INFINITY, mx = -INFINITY;
-    for (int t = 0; t < gk; ++t) {
-      const float x = key(t);
-      mn = fminf(mn, x);
-      mx = fmaxf(mx, x);
-    }
-    const GroupParams gp = group_params_b(mn, mx, width);
-    sz = gp.sz;
-    for (int t = 0; t < gk; ++t)
-      atomicOr(&sm_rows[t * kw + offset / 32], quant_code_b(key(t), gp, width) << (offset % 32));
+// Codes of a 16-byte chunk of 8 channels with per-channel widths w[j] (0 = dropped, no bits),
+// packed at bit offsets o[j] - o[0] (the offsets in the row are non-decreasing and a channel's
+// offset is a multiple of its width); 8 * w[0] bits at most.
+__device__ __forceinline__ uint64_t pack_chunk_var(const uint4& raw, const float* z, const float* r,
+                                                   const float* sc, const int* w, const int* o) {
+  const __half2* hx = reinterpret_cast<const __half2*>(&raw);
+  float x[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __half22float2(hx[e]);
+    x[2 * e] = f.x;
+    x[2 * e + 1] = f.y;
   }
-  ksz[gidx * d.dk + c] = sz;
-  __syncthreads();
-  const size_t row0 = group_row(d, table, bh / d.Hkv, bh % d.Hkv, g);
-  for (int i = c; i < gk * kw; i += nt) kcode[row0 * kw + i] = sm_rows[i];
+  bool near = false;
+  uint64_t bits = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (w[j]) bits |= static_cast<uint64_t>(code_fast_l(x[j], z[j], r[j], static_cast<float>((1 << w[j]) - 1), near)) << (o[j] - o[0]);
+  if (near) {
+    bits = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (w[j]) bits |= static_cast<uint64_t>(code_exact_l(x[j], z[j], sc[j], static_cast<float>((1 << w[j]) - 1))) << (o[j] - o[0]);
+  }
+  return bits;
 }
 
-// One CTA of dv threads per 16 consecutive (b * kv head, token) rows: thread c holds channel
-// c; a value group's min and max are reduced over its gv channels (shuffles within a warp,
-// then shared memory across warps when gv > 32), and the codes are ORed into the row in
-// shared memory ([kw] u32) before it is written out.
-__global__ void quantize_values_var_kernel(const __half* __restrict__ src, int src_rows, int t_begin,
-                                           int n_tokens, uint32_t* __restrict__ vcode,
-                                           __half2* __restrict__ vsz, const int* __restrict__ table,
-                                           Dims d) {
-  __shared__ uint32_t sm_row[64];
-  __shared__ float sm_mn[8], sm_mx[8];
-  const int c = threadIdx.x, lane = c & 31, warp = c >> 5;
-  const int gv = d.gv, vw = d.vw;
+// ORs a chunk's bits, which start at bit `off` of a row of 32-bit words, into that row.  A chunk
+// whose first channel has 8 bits starts on a 64-bit boundary (every channel before it has 8
+// bits); otherwise it spans at most 32 bits; so the bits fit in 64 bits after the shift.
+__device__ __forceinline__ void or_into_row(uint32_t* row, int off, uint64_t bits) {
+  const uint64_t v = bits << (off % 32);
+  if (static_cast<uint32_t>(v)) atomicOr(&row[off / 32], static_cast<uint32_t>(v));
+  if (v >> 32) atomicOr(&row[off / 32 + 1], static_cast<uint32_t>(v >> 32));
+}
+
+// Key quantize-pack with per-channel widths: the fixed-width kernel's tiling (16-byte chunks of
+// 8 channels, R rows per thread, each key read once, min/max reduced in shared memory), channel
+// c quantized with its own width; the codes are ORed into the CTA's rows in shared memory
+// ([gpc * gk][kw] words), which are then written out whole.  (scale, zero) are stored plainly,
+// [dk][2] per group; a dropped channel stores (0, 0).
+template <int R>
+__global__ void __launch_bounds__(256) quantize_keys_var_kernel(
+    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
+    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
+  extern __shared__ __align__(16) uint32_t sm_rows[];               // [gpc * gk][kw]
+  __shared__ __align__(16) __half2 red[2][256][4];
+  __shared__ __align__(16) float prm[3][kKeyPrm];
+  __shared__ __align__(16) __half2 blk[kKeyPrm];
+  const int dk = d.dk, gk = d.gk, kw = d.kw;
+  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int tid = threadIdx.x;
+  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt / cpr;
+  const int bh = blockIdx.y, b = bh / d.Hkv, h = bh % d.Hkv;
+  const int g_first = blockIdx.x * gpc;
+  const bool active = g_first + gi < n_groups;
+  const int g = g_begin + g_first + gi;
+  const size_t base = static_cast<size_t>(bh) * src_rows;
+  for (int i = tid; i < gpc * gk * kw; i += 256) sm_rows[i] = 0u;
+  uint4 x[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int row = (g * gk + rs + slabs * i) % src_rows;
+    x[i] = active ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
+                  : make_uint4(0, 0, 0, 0);
+  }
+  {
+    const __half2* h0 = reinterpret_cast<const __half2*>(&x[0]);
+    __half2 mn[4], mx[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mn[k] = mx[k] = h0[k];
+#pragma unroll
+    for (int i = 1; i < R; ++i) {
+      const __half2* hi = reinterpret_cast<const __half2*>(&x[i]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        mn[k] = __hmin2(mn[k], hi[k]);
+        mx[k] = __hmax2(mx[k], hi[k]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      red[0][tid][k] = mn[k];
+      red[1][tid][k] = mx[k];
+    }
+  }
+  __syncthreads();
+  for (int p = tid; p < gpc * dk / 2; p += 256) {
+    const int g2 = p / (dk / 2), pp = p % (dk / 2), c2 = pp / 4, k = pp % 4;
+    const int t0 = g2 * tpg + c2;
+    __half2 mn = red[0][t0][k], mx = red[1][t0][k];
+    for (int sl = 1; sl < slabs; ++sl) {
+      mn = __hmin2(mn, red[0][t0 + sl * cpr][k]);
+      mx = __hmax2(mx, red[1][t0 + sl * cpr][k]);
+    }
+    const float2 fmn = __half22float2(mn), fmx = __half22float2(mx);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int c = 8 * c2 + 2 * k + e;
+      int width, offset;
+      channel_width(d.kcnt, c, &width, &offset);
+      GroupParams gp;
+      gp.scale = gp.zero = 0.0f;
+      gp.sz = __floats2half2_rn(0.0f, 0.0f);
+      if (width) gp = group_params_b(e ? fmn.y : fmn.x, e ? fmx.y : fmx.x, width);
+      prm[0][g2 * dk + c] = gp.zero;
+      prm[1][g2 * dk + c] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+      prm[2][g2 * dk + c] = gp.scale;
+      blk[g2 * dk + c] = gp.sz;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < gpc * dk / 4; i += 256) {                 // 16 B of (scale, zero) per thread
+    const int g2 = i / (dk / 4), j = i % (dk / 4);
+    if (g_first + g2 >= n_groups) continue;
+    const size_t gidx = group_index(d, table, b, h, g_begin + g_first + g2);
+    reinterpret_cast<uint4*>(ksz + gidx * dk)[j] = reinterpret_cast<const uint4*>(blk + g2 * dk)[j];
+  }
+  if (active) {
+    float z[8], r[8], sc[8];
+    int w[8], o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      z[j] = prm[0][gi * dk + 8 * cc + j];
+      r[j] = prm[1][gi * dk + 8 * cc + j];
+      sc[j] = prm[2][gi * dk + 8 * cc + j];
+      channel_width(d.kcnt, 8 * cc + j, &w[j], &o[j]);
+    }
+    if (w[0]) {
+#pragma unroll
+      for (int i = 0; i < R; ++i)
+        or_into_row(sm_rows + (gi * gk + rs + slabs * i) * kw, o[0], pack_chunk_var(x[i], z, r, sc, w, o));
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < gpc * gk * kw; i += 256) {
+    const int g2 = i / (gk * kw);
+    if (g_first + g2 >= n_groups) continue;
+    kcode[group_row(d, table, b, h, g_begin + g_first + g2) * kw + i % (gk * kw)] = sm_rows[i];
+  }
+}
+
+// Value quantize-pack with per-group widths: the fixed-width value kernel's tiling (a lane per
+// 16-byte chunk of a row, R rows per lane, group extremes by shuffles); a chunk lies in one
+// value group, so its 8 channels share the group's width.  Each warp ORs its block's codes into
+// rows in shared memory, then writes the rows out whole.
+template <int R>
+__global__ void __launch_bounds__(256) quantize_values_var_kernel(
+    const __half* __restrict__ src, int src_rows, int t_begin, int n_tokens,
+    uint32_t* __restrict__ vcode, __half2* __restrict__ vsz, const int* __restrict__ table, Dims d) {
+  __shared__ uint32_t sm_rows[8][64 * R];           // per warp: 256 R / dv rows of <= dv / 4 words
+  const int dv = d.dv, cpr = dv / 8, rpw = 32 / cpr, gl = d.gv / 8, vw = d.vw;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int cc = lane % cpr, rsub = lane / cpr;
   int width, offset;
-  channel_width(d.vcnt, c, &width, &offset);
+  channel_width(d.vcnt, 8 * cc, &width, &offset);
+  const float levels = static_cast<float>((1 << width) - 1);
+  uint32_t* rows_sm = sm_rows[warp];
   const long long rows = static_cast<long long>(d.B) * d.Hkv * n_tokens;
-  for (long long r = static_cast<long long>(blockIdx.x) * 16; r < rows; r += static_cast<long long>(gridDim.x) * 16) {
-    for (int rr = 0; rr < 16 && r + rr < rows; ++rr) {
-      const long long rowi = r + rr;
-      const int t = t_begin + static_cast<int>(rowi % n_tokens);
-      const int bh = static_cast<int>(rowi / n_tokens);
-      for (int i = c; i < vw; i += blockDim.x) sm_row[i] = 0u;
-      const float x = __half2float(src[(static_cast<size_t>(bh) * src_rows + t % src_rows) * d.dv + c]);
-      float mn = x, mx = x;
-      const int span = gv < 32 ? gv : 32;
-      for (int off = 1; off < span; off <<= 1) {
+  const long long block_rows = static_cast<long long>(rpw) * R;
+  const long long n_blocks = (rows + block_rows - 1) / block_rows;
+  for (long long wb = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; wb < n_blocks;
+       wb += static_cast<long long>(gridDim.x) * blockDim.x / 32) {
+    for (int k = lane; k < block_rows * vw; k += 32) rows_sm[k] = 0u;
+    __syncwarp();
+    uint4 x[R];
+    long long ri[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      ri[i] = wb * block_rows + rsub + static_cast<long long>(rpw) * i;
+      if (ri[i] < rows) {
+        const int bh = static_cast<int>(ri[i] / n_tokens);
+        const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
+        x[i] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + cc);
+      } else {
+        x[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const __half2* hx = reinterpret_cast<const __half2*>(&x[i]);
+      __half2 mn2 = __hmin2(__hmin2(hx[0], hx[1]), __hmin2(hx[2], hx[3]));
+      __half2 mx2 = __hmax2(__hmax2(hx[0], hx[1]), __hmax2(hx[2], hx[3]));
+      float mn = fminf(__low2float(mn2), __high2float(mn2));
+      float mx = fmaxf(__low2float(mx2), __high2float(mx2));
+      for (int off = 1; off < gl; off <<= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       }
-      if (gv > 32) {
-        if (lane == 0) {
-          sm_mn[warp] = mn;
-          sm_mx[warp] = mx;
-        }
-        __syncthreads();
-        const int w0 = (c / gv) * (gv / 32);
-        mn = sm_mn[w0];
-        mx = sm_mx[w0];
-        for (int k = 1; k < gv / 32; ++k) {
-          mn = fminf(mn, sm_mn[w0 + k]);
-          mx = fmaxf(mx, sm_mx[w0 + k]);
-        }
-      }
-      __syncthreads();        // the row is cleared; the warps' extremes are read
+      if (ri[i] >= rows) continue;
+      GroupParams gp;
+      gp.scale = gp.zero = 0.0f;
+      gp.sz = __floats2half2_rn(0.0f, 0.0f);
+      if (width) gp = group_params_b(mn, mx, width);
+      const int bh = static_cast<int>(ri[i] / n_tokens);
+      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
       const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
-      __half2 sz = __floats2half2_rn(0.0f, 0.0f);
-      if (width) {
-        const GroupParams gp = group_params_b(mn, mx, width);
-        sz = gp.sz;
-        atomicOr(&sm_row[offset / 32], quant_code_b(x, gp, width) << (offset % 32));
+      if (cc % gl == 0) vsz[vrow * d.nvg + cc / gl] = gp.sz;
+      if (!width) continue;
+      const float rcp = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+      const __half2* h2 = reinterpret_cast<const __half2*>(&x[i]);
+      bool near = false;
+      uint64_t bits = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h2[e]);
+        bits |= static_cast<uint64_t>(code_fast_l(f.x, gp.zero, rcp, levels, near)) << (2 * e * width);
+        bits |= static_cast<uint64_t>(code_fast_l(f.y, gp.zero, rcp, levels, near)) << ((2 * e + 1) * width);
       }
-      if (c % gv == 0) vsz[vrow * d.nvg + c / gv] = sz;
-      __syncthreads();
-      for (int i = c; i < vw; i += blockDim.x) vcode[vrow * vw + i] = sm_row[i];
-      __syncthreads();        // before the next row clears sm_row and sm_mn / sm_mx
+      if (near) {
+        bits = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __half22float2(h2[e]);
+          bits |= static_cast<uint64_t>(code_exact_l(f.x, gp.zero, gp.scale, levels)) << (2 * e * width);
+          bits |= static_cast<uint64_t>(code_exact_l(f.y, gp.zero, gp.scale, levels)) << ((2 * e + 1) * width);
+        }
+      }
+      or_into_row(rows_sm + (rsub + rpw * i) * vw, offset, bits);
     }
+    __syncwarp();
+    for (int k = lane; k < block_rows * vw; k += 32) {
+      const long long rr = wb * block_rows + k / vw;
+      if (rr >= rows) continue;
+      const int bh = static_cast<int>(rr / n_tokens);
+      const int t = t_begin + static_cast<int>(rr % n_tokens);
+      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
+      vcode[vrow * vw + k % vw] = rows_sm[k];
+    }
+    __syncwarp();
   }
 }
 
@@ -513,24 +800,39 @@ inline int grid_for(long long items, int block) {
 
 }  // namespace
 
-template <bool ROT>
+template <int BITS, bool ROT>
 cudaError_t launch_quantize_keys_t(const Dims& d, const __half* src, int src_rows, int g_begin,
                                    int n_groups, uint32_t* kcode, __half2* ksz, const int* table,
                                    cudaStream_t s) {
-  const int gpb = d.dk >= 256 ? 1 : 256 / d.dk;
-  dim3 block(d.dk, gpb);
-  dim3 grid((n_groups + gpb - 1) / gpb, d.B * d.Hkv);
-  const size_t smem = ROT ? static_cast<size_t>(gpb) * d.gk * d.dk * 2 : 0;
-  auto kern = d.kb == 2 ? quantize_keys_kernel<2, ROT>
-            : d.kb == 4 ? quantize_keys_kernel<4, ROT> : quantize_keys_kernel<8, ROT>;
-  if (d.kb != 2 && d.kb != 4 && d.kb != 8) return cudaErrorInvalidValue;
+  // rows per thread: at least 4, and enough that one group needs at most 256 threads
+  const int cpr = d.dk / 8;
+  int rows = 4;
+  while (cpr * d.gk / rows > 256) rows *= 2;
+  const int tpg = cpr * d.gk / rows, gpc = 256 / tpg;
+  dim3 grid((n_groups + gpc - 1) / gpc, d.B * d.Hkv);
+  const size_t smem = ROT ? static_cast<size_t>(gpc) * d.gk * d.dk * 2 : 0;
+  auto kern = rows == 4 ? quantize_keys_kernel<BITS, 4, ROT>
+            : rows == 8 ? quantize_keys_kernel<BITS, 8, ROT> : quantize_keys_kernel<BITS, 16, ROT>;
+  if (rows > 16 || gpc * d.dk > kKeyPrm || gpc * 2 * d.dk > kKeyBlk) return cudaErrorInvalidValue;
   if (smem > 48 * 1024) {
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, block, smem, s>>>(src, src_rows, d.dk, d.gk, g_begin, n_groups, d.lcap, kcode, ksz, table, d);
+  kern<<<grid, 256, smem, s>>>(src, src_rows, g_begin, n_groups, kcode, ksz, table, d);
   return cudaGetLastError();
+}
+
+template <bool ROT>
+cudaError_t launch_quantize_keys_r(const Dims& d, const __half* src, int src_rows, int g_begin,
+                                   int n_groups, uint32_t* kcode, __half2* ksz, const int* table,
+                                   cudaStream_t s) {
+  switch (d.kb) {
+    case 2: return launch_quantize_keys_t<2, ROT>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
+    case 4: return launch_quantize_keys_t<4, ROT>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
+    case 8: return launch_quantize_keys_t<8, ROT>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
@@ -539,18 +841,24 @@ cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows,
   if (n_groups <= 0) return cudaSuccess;
   if (d.var) {
     if (rotate) return cudaErrorInvalidValue;
-    const int smem = d.gk * d.kw * 4;       // <= 128 x 64 words
+    const int cpr = d.dk / 8;
+    int rows = 4;
+    while (cpr * d.gk / rows > 256) rows *= 2;
+    const int tpg = cpr * d.gk / rows, gpc = 256 / tpg;
+    const int smem = gpc * d.gk * d.kw * 4;
+    auto kern = rows == 4 ? quantize_keys_var_kernel<4>
+              : rows == 8 ? quantize_keys_var_kernel<8> : quantize_keys_var_kernel<16>;
+    if (rows > 16 || gpc * d.dk > kKeyPrm) return cudaErrorInvalidValue;
     if (smem > 48 * 1024) {
-      const cudaError_t e = cudaFuncSetAttribute(quantize_keys_var_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
     }
-    quantize_keys_var_kernel<<<dim3(n_groups, d.B * d.Hkv), d.dk, smem, s>>>(src, src_rows, g_begin,
-                                                                              kcode, ksz, table, d);
+    kern<<<dim3((n_groups + gpc - 1) / gpc, d.B * d.Hkv), 256, smem, s>>>(src, src_rows, g_begin, n_groups,
+                                                                         kcode, ksz, table, d);
     return cudaGetLastError();
   }
-  return rotate ? launch_quantize_keys_t<true>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s)
-                : launch_quantize_keys_t<false>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
+  return rotate ? launch_quantize_keys_r<true>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s)
+                : launch_quantize_keys_r<false>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
 }
 
 cudaError_t launch_table_writes(int* table, const TableWrites& tw, cudaStream_t s) {
@@ -601,19 +909,23 @@ cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_row
   if (n_tokens <= 0) return cudaSuccess;
   const int nbh = d.B * d.Hkv;
   if (d.var) {
+    constexpr int kRows = 4;
     const long long rows = static_cast<long long>(nbh) * n_tokens;
-    const long long blocks = (rows + 15) / 16;
-    const int grid = static_cast<int>(blocks < 148 * 16 ? blocks : 148 * 16);
-    quantize_values_var_kernel<<<grid, d.dv, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d);
+    const long long per_cta = 8LL * (32 / (d.dv / 8)) * kRows;
+    const long long ctas = (rows + per_cta - 1) / per_cta;
+    const int grid = static_cast<int>(ctas < (1LL << 30) ? ctas : (1LL << 30));
+    quantize_values_var_kernel<kRows><<<grid, 256, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d);
     return cudaGetLastError();
   }
-  const long long items = static_cast<long long>(nbh) * n_tokens * d.nvg;
-  const int block = 256;
-  const int grid = grid_for(items, block);
+  constexpr int kRows = 4;
+  const long long rows = static_cast<long long>(nbh) * n_tokens;
+  const long long per_cta = 8LL * (32 / (d.dv / 8)) * kRows;   // 8 warps, each a block of rows
+  const long long ctas = (rows + per_cta - 1) / per_cta;
+  const int grid = static_cast<int>(ctas < (1LL << 30) ? ctas : (1LL << 30));
   switch (d.vb) {
-    case 2: quantize_values_kernel<2><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz, table, d); break;
-    case 4: quantize_values_kernel<4><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz, table, d); break;
-    case 8: quantize_values_kernel<8><<<grid, block, 0, s>>>(src, src_rows, d.dv, d.gv, t_begin, n_tokens, nbh, d.lcap, vcode, vsz, table, d); break;
+    case 2: quantize_values_kernel<2, kRows><<<grid, 256, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;
+    case 4: quantize_values_kernel<4, kRows><<<grid, 256, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;
+    case 8: quantize_values_kernel<8, kRows><<<grid, 256, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

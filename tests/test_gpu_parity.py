@@ -299,12 +299,6 @@ def test_full_size_thin_16k():
     sampled_full_size(W.WORKLOADS["thin16k"], rows=(0, 15))
 
 
-@pytest.mark.parametrize("kb,vb", [(4, 2), (16, 16)])
-def test_full_size_sweep_point_131k(kb, vb):
-    w = W.sweep_workload(8, kb, vb, appends=66)
-    sampled_full_size(w, rows=(5,), steps=(0, 63, 64, 65))
-
-
 # ------------------------------------------------------- HeadQ side code ----
 @pytest.mark.parametrize("kb", [4, 2])
 @pytest.mark.parametrize("sr,sq", [(4, 4), (4, 8), (8, 4)])
