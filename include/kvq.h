@@ -97,8 +97,11 @@
  *
  * Conventions: every call is asynchronous on the caller's CUDA stream (passed as
  * void*, a cudaStream_t; NULL = legacy default stream); no call synchronizes or
- * copies device memory back to the host, except kvq_read_status.  The library
- * allocates no device memory.  A cache handle must not be used from two host
+ * copies device memory back to the host, except the status and record readers
+ * (kvq_read_status, kvq_noalloc_read_status, kvq_debug_take_record).  The library
+ * allocates nothing at call time; the only device memory it holds is the static
+ * scratch array of kvq_decode_attention_noalloc (and, in a bounds-check build, its
+ * debug record), one per GPU that loads it.  A cache handle must not be used from two host
  * threads or two streams at once.  Inputs must be finite; NaN or Inf in K, V or
  * q gives undefined (but memory-safe) results.  GQA: query head hq reads kv
  * head hq / (n_q_heads / n_kv_heads).  Every function returns KVQ_OK (0) or one
@@ -343,6 +346,25 @@ int kvq_read_status(const void* workspace, unsigned int* status, void* stream);
 
 /* Static description of an error code. */
 const char* kvq_strerror(int code);
+
+/* Bounds-check build (a development aid; no counterpart on the pages).  The library built
+ * with -DKVQ_DEBUG (libkvq_debug.so beside libkvq.so) compares every global-memory index its
+ * kernels compute with the extent of the buffer it addresses; a failed check is counted in a
+ * record the library keeps on each device (the first failure's site, index and extent), and
+ * the access is skipped or redirected to the buffer's start.  Nothing traps.
+ * kvq_debug_build: 1 in a bounds-check build, else 0.
+ * kvq_debug_take_record: waits for stream, copies the current device's record to *out and
+ * clears it.  Errors: INVALID_ARG (out NULL), UNSUPPORTED (not a bounds-check build), CUDA.
+ * kvq_debug_site_name: static description of a record's site. */
+typedef struct kvq_debug_record {
+    unsigned int failures;   /* failed checks since the record was last taken */
+    unsigned int site;       /* where the first one failed (kvq_debug_site_name) */
+    long long index;         /* its index, in elements of the buffer's type */
+    long long extent;        /* the buffer's extent in the same elements */
+} kvq_debug_record;
+int kvq_debug_build(void);
+int kvq_debug_take_record(kvq_debug_record* out, void* stream);
+const char* kvq_debug_site_name(unsigned int site);
 
 #ifdef __cplusplus
 }

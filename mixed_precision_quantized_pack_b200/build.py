@@ -1,5 +1,6 @@
 """Builds libkvq.so (sm_100a) in place with nvcc: one object per .cu, compiled in
-parallel, then linked into a shared library beside this file."""
+parallel, then linked into a shared library beside this file.  build(debug=True) builds
+the bounds-check variant libkvq_debug.so from the same sources with -DKVQ_DEBUG."""
 from __future__ import annotations
 
 import concurrent.futures as cf
@@ -12,6 +13,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libkvq.so")
+DEBUG_LIB = os.path.join(HERE, "libkvq_debug.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -35,35 +37,38 @@ def _stale(obj, src, deps):
     return any(os.path.getmtime(p) > t for p in [src] + deps)
 
 
-def _compile(src, obj, verbose):
-    cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+def _compile(src, obj, verbose, debug=False):
+    cmd = [NVCC] + ARCH + FLAGS + (["-DKVQ_DEBUG"] if debug else []) + (["-Xptxas", "-v"] if verbose else []) + \
+        ["-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{r.stdout}\n{r.stderr}")
     return r.stderr if verbose else ""
 
 
-def build(verbose: bool = False, jobs: int | None = None) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose: bool = False, jobs: int | None = None, debug: bool = False) -> str:
+    bdir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = DEBUG_LIB if debug else LIB
+    os.makedirs(bdir, exist_ok=True)
     deps = _headers()
     objs, todo = [], []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(bdir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if verbose or _stale(obj, src, deps):
             todo.append((src, obj))
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs or os.cpu_count() or 4) as ex:
-            for log in ex.map(lambda so: _compile(so[0], so[1], verbose), todo):
+            for log in ex.map(lambda so: _compile(so[0], so[1], verbose, debug), todo):
                 if log:
                     print(log, file=sys.stderr)
-    if todo or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        cmd = [NVCC] + ARCH + ["-shared", "-o", LIB] + objs
+    if todo or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        cmd = [NVCC] + ARCH + ["-shared", "-o", lib] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -20,8 +20,13 @@ namespace mma {
   extern template cudaError_t launch<KB, VB, DK, NREP, GV, GK, true, 0, 4, true>(        \
       const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
       cudaStream_t);
+#define KVQ_DECL_T(KB, VB, DK, NREP, GV, GK, SR, SQ)                                       \
+  extern template cudaError_t launch<KB, VB, DK, NREP, GV, GK, true, SR, SQ, true>(        \
+      const Dims&, const CacheBufs&, const DecodeWork&, const __half*, const Partials&,     \
+      cudaStream_t);
 KVQ_MMA_QUANT_INSTANCES(KVQ_DECL_Q)
 KVQ_MMA_PAGED_INSTANCES(KVQ_DECL_P)
+KVQ_MMA_PAGED_SIDE_INSTANCES(KVQ_DECL_T)
 KVQ_MMA_SIDE_INSTANCES(KVQ_DECL_S)
 KVQ_MMA_FP16_INSTANCES(KVQ_DECL_F)
 }  // namespace mma
@@ -42,8 +47,11 @@ struct Entry {
 #define KVQ_ENTRY_F(DK, NREP) {16, 16, DK, NREP, 0, 0, 0, 0, 0, &mma::launch<4, 2, DK, NREP, 64, 64, false>},
 #define KVQ_ENTRY_P(KB, VB, DK, NREP, GV, GK) \
   {KB, VB, DK, NREP, GV, GK, 0, 0, 1, &mma::launch<KB, VB, DK, NREP, GV, GK, true, 0, 4, true>},
+#define KVQ_ENTRY_T(KB, VB, DK, NREP, GV, GK, SR, SQ) \
+  {KB, VB, DK, NREP, GV, GK, SR, SQ, 1, &mma::launch<KB, VB, DK, NREP, GV, GK, true, SR, SQ, true>},
 const Entry kTable[] = {KVQ_MMA_QUANT_INSTANCES(KVQ_ENTRY_Q) KVQ_MMA_SIDE_INSTANCES(KVQ_ENTRY_S)
-                            KVQ_MMA_FP16_INSTANCES(KVQ_ENTRY_F) KVQ_MMA_PAGED_INSTANCES(KVQ_ENTRY_P)};
+                            KVQ_MMA_FP16_INSTANCES(KVQ_ENTRY_F) KVQ_MMA_PAGED_INSTANCES(KVQ_ENTRY_P)
+                                KVQ_MMA_PAGED_SIDE_INSTANCES(KVQ_ENTRY_T)};
 
 LaunchFn find(const Dims& d) {
   if (d.dv != 128) return nullptr;

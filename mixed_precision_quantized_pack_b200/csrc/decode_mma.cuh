@@ -447,7 +447,10 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       // entry that its warp's lane 0 fetched (cp.async into the warp's slot) when the warp
       // began the unit before it.
       int* sm_page = reinterpret_cast<int*>(smem + SM::kPage);
-      auto table_entry = [&](int k) { return cb.table + (b * d.max_groups + unit_begin + k); };
+      auto table_entry = [&](int k) {
+        const int gg = unit_begin + k;
+        return cb.table + (b * d.max_groups + (KVQ_IN_BOUNDS(d, kSiteDecTable, gg, d.max_groups) ? gg : 0));
+      };
       auto group_of = [&](int k, bool fetched) -> size_t {
         if constexpr (!PAGED) return static_cast<size_t>(bh) * d.max_groups + unit_begin + k;
         int page;
@@ -461,6 +464,9 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       };
       // one lane copies unit k (a whole key group: 4 contiguous runs) into stage k % RING
       auto issue = [&](int k, size_t gi) {
+        // (bounds-check builds) a group outside the buffers is replaced by group 0, so that the
+        // stage's copies still complete
+        if (!KVQ_IN_BOUNDS(d, kSiteDecKCode, static_cast<long long>(gi), quant_groups(d))) gi = 0;
         const int st = k % RING;
         const uint32_t bar = bar0 + 8 * st;
         const uint32_t dst = stages_s + st * STAGE;
@@ -775,6 +781,9 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
           base_k = cb.win_k;
           base_v = cb.win_v;
         }
+        if (!KVQ_IN_BOUNDS(d, base_k == cb.ret_k ? kSiteDecRetK : kSiteDecWinK, static_cast<long long>(slot),
+                           base_k == cb.ret_k ? ret_rows(d) : win_rows(d)))
+          slot = 0;
         if (lane < 16)
           ptx::bulk_g2s(dst + row * R::KST, base_k + slot * DK, DK * 2, bar);
         else
@@ -920,6 +929,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
       lsum = fmaf(wt, sm_ml[(ww * NREP + r) * 2 + 1], lsum);
     }
     const size_t pi = (static_cast<size_t>(b) * d.Hq + h * NREP + r) * w.splits + split;
+    if (!KVQ_IN_BOUNDS(d, kSiteDecPartial, static_cast<long long>(pi), static_cast<long long>(d.B) * d.Hq * w.splits))
+      continue;
     part.o[pi * kDV + c] = acc;
     if (c == 0) part.ml[pi] = make_float2(M, lsum);
   }

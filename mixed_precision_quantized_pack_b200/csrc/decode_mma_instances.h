@@ -3,9 +3,11 @@
 //   S(KB, VB, DK, NREP, GV, GK, SR, SQ)  quantized caches with a rank-SR, SQ-bit side code
 //   F(DK, NREP)                          unquantized fp16 caches (value head dim 128)
 //   P(KB, VB, DK, NREP, GV, GK)          quantized paged caches (groups found through a block table)
+//   T(KB, VB, DK, NREP, GV, GK, SR, SQ)  paged caches with a side code
 // decode_mma.cu builds its dispatch table from the same lists; each
 // decode_mma_inst_k*.cu file instantiates the Q entries whose KB it owns,
-// decode_mma_inst_side.cu the S entries, decode_mma_inst_paged.cu the P entries.
+// decode_mma_inst_side.cu the S entries, decode_mma_inst_paged.cu the P entries and
+// decode_mma_inst_paged_side.cu the T entries.
 // Shapes not listed here run on the generic CUDA-core kernel.
 #pragma once
 
@@ -26,3 +28,7 @@
 #define KVQ_MMA_PAGED_INSTANCES(P)                                                              \
   P(4, 2, 128, 4, 64, 64) P(4, 2, 128, 1, 64, 64) P(4, 4, 128, 4, 64, 64) P(8, 4, 128, 4, 64, 64) \
   P(2, 2, 128, 4, 64, 64)
+
+#define KVQ_MMA_PAGED_SIDE_INSTANCES(T)                                                         \
+  T(4, 2, 128, 4, 64, 64, 4, 4) T(4, 2, 128, 4, 64, 64, 4, 8) T(4, 2, 128, 4, 64, 64, 8, 4)      \
+  T(2, 2, 128, 4, 64, 64, 4, 4) T(2, 2, 128, 4, 64, 64, 4, 8) T(2, 2, 128, 4, 64, 64, 8, 4)

@@ -119,8 +119,13 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
     if (quant) {
       // retained ({p < Q : p mod 2^floor(log2(Q - p)) == 0}): read from the fp16 list
       if (d.log_retain && (i & ((1 << (31 - __clz(sw.Q - i))) - 1)) == 0) continue;
-      const size_t row = group_row(d, cb.table, b, h, i / d.gk) + i % d.gk;
-      const size_t gidx = group_index(d, cb.table, b, h, i / d.gk);
+      const bool tab_ok = KVQ_IN_BOUNDS(d, kSiteDecTable, i / d.gk, d.max_groups);
+      size_t row = tab_ok ? group_row(d, cb.table, b, h, i / d.gk) + i % d.gk : 0;
+      size_t gidx = tab_ok ? group_index(d, cb.table, b, h, i / d.gk) : 0;
+      // (bounds-check builds) a token outside the buffers reads token 0 instead
+      if (!KVQ_IN_BOUNDS(d, kSiteDecKCode, static_cast<long long>(row), quant_rows(d)) ||
+          !KVQ_IN_BOUNDS(d, kSiteDecKMeta, static_cast<long long>(gidx), quant_groups(d)))
+        row = gidx = 0;
       if (d.sr) {
         const uint8_t* zr = cb.zcode + row * d.zb;
         const uint32_t zrow = d.zb == 4 ? *reinterpret_cast<const uint32_t*>(zr)
@@ -181,12 +186,14 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
     } else {
       const __half *kp, *vp;
       if (i < sw.n_ret) {
-        const size_t s = static_cast<size_t>(bh) * kMaxRetained + i;
+        size_t s = static_cast<size_t>(bh) * kMaxRetained + i;
+        if (!KVQ_IN_BOUNDS(d, kSiteDecRetK, static_cast<long long>(s), ret_rows(d))) s = 0;
         kp = cb.ret_k + s * d.dk;
         vp = cb.ret_v + s * d.dv;
       } else {
         const int pos = sw.Q + (i - sw.n_ret);
-        const size_t s = static_cast<size_t>(bh) * d.cap + pos % d.cap;
+        size_t s = static_cast<size_t>(bh) * d.cap + pos % d.cap;
+        if (!KVQ_IN_BOUNDS(d, kSiteDecWinK, static_cast<long long>(s), win_rows(d))) s = 0;
         kp = cb.win_k + s * d.dk;
         vp = cb.win_v + s * d.dv;
       }
@@ -237,6 +244,8 @@ decode_simple_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restric
     float M = -INFINITY;
     for (int k = 0; k < kWarps; ++k) M = fmaxf(M, sm_m[k][r]);
     const size_t part = (static_cast<size_t>(b) * d.Hq + h * nrep + r) * w.splits + split;
+    if (!KVQ_IN_BOUNDS(d, kSiteDecPartial, static_cast<long long>(part), static_cast<long long>(d.B) * d.Hq * w.splits))
+      continue;
     float wk[kWarps];
     float Lsum = 0.0f;
     for (int k = 0; k < kWarps; ++k) {

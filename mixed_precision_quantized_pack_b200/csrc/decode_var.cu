@@ -306,7 +306,10 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarMap vm, const __half* _
       sm_tag[st] = k;
       const bool stall = w.stall && k == 0 && split == 0 && h == 0 && b == 0;
       ptx::mbar_arrive_expect_tx(bar, L.bytes + (stall ? 16u : 0u));
-      const size_t gi = group_index(d, cb.table, b, h, g);
+      size_t gi = KVQ_IN_BOUNDS(d, kSiteDecTable, g, d.max_groups) ? group_index(d, cb.table, b, h, g) : 0;
+      // (bounds-check builds) a group outside the buffers is replaced by group 0, so that the
+      // stage's copies still complete
+      if (!KVQ_IN_BOUNDS(d, kSiteDecKCode, static_cast<long long>(gi), quant_groups(d))) gi = 0;
       const size_t tok = gi * gk;
       ptx::bulk_g2s(dst + L.k_off, cb.kcode + tok * d.kw, gk * d.kw * 4, bar);
       ptx::bulk_g2s(dst + L.kmeta_off, cb.ksz + gi * d.dk, d.dk * 4, bar);
@@ -338,6 +341,9 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarMap vm, const __half* _
           base_k = cb.win_k;
           base_v = cb.win_v;
         }
+        if (!KVQ_IN_BOUNDS(d, base_k == cb.ret_k ? kSiteDecRetK : kSiteDecWinK, static_cast<long long>(slot),
+                           base_k == cb.ret_k ? ret_rows(d) : win_rows(d)))
+          slot = 0;
         if (lane < 16)
           ptx::bulk_g2s(dst + row * KST, base_k + slot * kDK, kDK * 2, bar);
         else
@@ -655,6 +661,8 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarMap vm, const __half* _
       lsum = fmaf(wt, sm_ml[(ww * NREP + r) * 2 + 1], lsum);
     }
     const size_t pi = (static_cast<size_t>(b) * d.Hq + h * NREP + r) * w.splits + split;
+    if (!KVQ_IN_BOUNDS(d, kSiteDecPartial, static_cast<long long>(pi), static_cast<long long>(d.B) * d.Hq * w.splits))
+      continue;
     part.o[pi * kDV + c] = acc;
     if (c == 0) part.ml[pi] = make_float2(M, lsum);
   }

@@ -38,6 +38,12 @@ struct kvq_cache {
 
 namespace kvq {
 
+#ifdef KVQ_DEBUG
+// The bounds-check build's record of failed checks: one per device that loads the library
+// (zero at load), found by the kernels through Dims::dbg.
+static __device__ DebugRecord g_debug_record;
+#endif
+
 size_t workspace_bytes(const Dims& d, int splits) {
   const size_t rows = static_cast<size_t>(d.B) * d.Hq * splits;
   const size_t ml = (rows * sizeof(float2) + 255) / 256 * 256;
@@ -150,6 +156,8 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
   x.max_context = c->max_context;
   x.lcap = static_cast<int>(lcap);
   x.paged = c->paged;
+  x.n_pages = c->paged ? c->n_pages : 0;
+  x.dbg = nullptr;
   x.max_groups = static_cast<int>(lcap / x.gk);
   x.cap = raw ? c->max_context : c->window + c->group_k;
   x.kw = raw ? 0 : var ? std::max(1, (kbits + 31) / 32) : c->d_k * c->k_bits / 32;
@@ -338,7 +346,7 @@ struct TableWriter {
   TableWriter(kvq_cache* c_, cudaStream_t s_) : c(c_), s(s_) { tw.n = 0; }
   int flush() {
     if (tw.n > 0 && !rc)
-      rc = check_cuda(kvq::launch_table_writes(static_cast<int*>(c->buf.block_table), tw, s));
+      rc = check_cuda(kvq::launch_table_writes(c->d, static_cast<int*>(c->buf.block_table), tw, s));
     tw.n = 0;
     return rc;
   }
@@ -451,6 +459,12 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
     cudaGetLastError();
     return KVQ_ERR_CUDA;
   }
+#ifdef KVQ_DEBUG
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&d.dbg), kvq::g_debug_record) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+#endif
   kvq_cache* c = new (std::nothrow) kvq_cache;
   if (!c) return KVQ_ERR_INVALID_ARG;
   c->d = d;
@@ -548,10 +562,10 @@ int prefill_rows(const kvq::Dims& d, const kvq_buffers& buf, const __half* kh, c
   if (!rc)
     rc = check_cuda(d.rot ? kvq::launch_rotate_key_rows(d, kh, src_rows, Q, static_cast<__half*>(buf.win_k),
                                                         d.cap, Q, L - Q, nullptr, s)
-                          : kvq::launch_copy_rows(kh, src_rows, Q, static_cast<__half*>(buf.win_k), d.cap,
+                          : kvq::launch_copy_rows(d, kh, src_rows, Q, static_cast<__half*>(buf.win_k), d.cap,
                                                   Q, L - Q, d.dk, nbh, s));
   if (!rc)
-    rc = check_cuda(kvq::launch_copy_rows(vh, src_rows, Q, static_cast<__half*>(buf.win_v), d.cap, Q,
+    rc = check_cuda(kvq::launch_copy_rows(d, vh, src_rows, Q, static_cast<__half*>(buf.win_v), d.cap, Q,
                                           L - Q, d.dv, nbh, s));
   if (!rc && d.log_retain && Q > 0) {
     const std::vector<int> ret = retained_positions(Q);
@@ -887,6 +901,55 @@ int kvq_get_seq_state(const kvq_cache* c, int b, int* L, int* Q, int* n_retained
 
 int kvq_get_state(const kvq_cache* c, int* L, int* Q, int* n_retained, int* retained_idx) {
   return kvq_get_seq_state(c, 0, L, Q, n_retained, retained_idx);
+}
+
+int kvq_debug_build(void) {
+#ifdef KVQ_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int kvq_debug_take_record(kvq_debug_record* out, void* stream) {
+  if (!out) return KVQ_ERR_INVALID_ARG;
+#ifdef KVQ_DEBUG
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  kvq::DebugRecord r;
+  if (cudaStreamSynchronize(s) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&r, kvq::g_debug_record, sizeof(r)) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  const kvq::DebugRecord zero = {0u, 0u, 0, 0};
+  if (cudaMemcpyToSymbol(kvq::g_debug_record, &zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  out->failures = r.failures;
+  out->site = r.site;
+  out->index = r.index;
+  out->extent = r.extent;
+  return KVQ_OK;
+#else
+  (void)stream;
+  return KVQ_ERR_UNSUPPORTED;
+#endif
+}
+
+const char* kvq_debug_site_name(unsigned int site) {
+  static const char* const kNames[] = {
+      "none", "quantize keys: source", "quantize keys: codes", "quantize keys: (scale, zero)",
+      "quantize values: source", "quantize values: codes", "quantize values: (scale, zero)",
+      "side code: source", "side code: key codes", "side code: key (scale, zero)", "side code: basis",
+      "side code: codes", "side code: (scale, zero)", "row copy: source", "row copy: destination",
+      "append: window slot", "rotated rows: source", "rotated rows: destination",
+      "retained: source", "retained: destination", "retained update: source",
+      "block table: entry", "block table: page", "decode: block table entry",
+      "decode: quantized group", "decode: key (scale, zero) group", "decode: retained slot",
+      "decode: window slot", "decode: partial row"};
+  static_assert(sizeof(kNames) / sizeof(kNames[0]) == kvq::kSiteCount, "one name per site");
+  return site < kvq::kSiteCount ? kNames[site] : "unknown";
 }
 
 int kvq_reset_status(void* workspace, void* stream) {

@@ -8,6 +8,30 @@
 namespace kvq {
 
 constexpr int kMaxRetained = 32;
+
+// The first failed bounds check of a bounds-check build (see KVQ_IN_BOUNDS below).
+struct DebugRecord {
+  unsigned int failures;   // failed checks since the record was last taken
+  unsigned int site;       // DebugSite of the first one
+  long long index;         // its index (elements of the buffer's type)
+  long long extent;        // and the buffer's extent
+};
+
+// Where a bounds check sits: the data-dependent global-memory accesses of the kernels (rows
+// and groups found through the length rules or the block table, window and retained slots,
+// partial rows).  Accesses whose indices follow from the launch shape alone are not checked.
+enum DebugSite : unsigned int {
+  kSiteNone = 0,
+  kSiteQKeySrc, kSiteQKeyCode, kSiteQKeyMeta,                 // key quantizers
+  kSiteQValSrc, kSiteQValCode, kSiteQValMeta,                 // value quantizers
+  kSiteSideSrc, kSiteSideCode, kSiteSideMeta, kSiteSideU, kSiteSideZCode, kSiteSideZMeta,
+  kSiteCopySrc, kSiteCopyDst,                                 // window / retained copies
+  kSiteAppendWin, kSiteRotSrc, kSiteRotDst,
+  kSiteRetSrc, kSiteRetDst, kSiteRetUpd,
+  kSiteTableIdx, kSiteTablePage,
+  kSiteDecTable, kSiteDecKCode, kSiteDecKMeta, kSiteDecRetK, kSiteDecWinK, kSiteDecPartial,
+  kSiteCount
+};
 constexpr int kMaxSeqs = 256;   // sequences of a cache whose lengths may differ (per-launch arrays)
 
 // Derived sizes of one cache (see include/kvq.h for the layouts).
@@ -30,8 +54,47 @@ struct Dims {
   // is the number of channels of width 8, 4, 2 and 1 (the rest are dropped, width 0)
   int var;
   int kcnt[4], vcnt[4];
+  int n_pages;      // pages of a paged cache's pool (0 otherwise)
+  DebugRecord* dbg; // bounds-check builds: the library's debug record on this device (else null)
   bool quantized() const { return kb != 16; }
 };
+
+// Extents of the cache buffers in elements of their types (token rows of the quantized
+// buffers: a (b, kv head) region of lcap rows per sequence, or n_pages pages of Hkv * gk rows).
+__host__ __device__ inline long long quant_rows(const Dims& d) {
+  return d.paged ? static_cast<long long>(d.n_pages) * d.Hkv * d.gk
+                 : static_cast<long long>(d.B) * d.Hkv * d.lcap;
+}
+__host__ __device__ inline long long quant_groups(const Dims& d) {
+  return d.paged ? static_cast<long long>(d.n_pages) * d.Hkv
+                 : static_cast<long long>(d.B) * d.Hkv * d.max_groups;
+}
+__host__ __device__ inline long long win_rows(const Dims& d) { return static_cast<long long>(d.B) * d.Hkv * d.cap; }
+__host__ __device__ inline long long ret_rows(const Dims& d) { return static_cast<long long>(d.B) * d.Hkv * kMaxRetained; }
+
+// Bounds checks of a bounds-check build (compiled with -DKVQ_DEBUG): every global index a
+// kernel computes is compared with its buffer's extent; a failed check counts in the
+// library's debug record (the first failure's site, index and extent are kept) and the
+// caller skips the access or redirects it to the buffer's start.  No trap, no assert: the
+// kernel runs on.  In other builds the checks compile to `true`.
+#ifdef KVQ_DEBUG
+__device__ __forceinline__ bool debug_in_bounds(const Dims& d, unsigned int site, long long idx,
+                                                long long extent) {
+  if (idx >= 0 && idx < extent) return true;
+  if (d.dbg && atomicAdd(&d.dbg->failures, 1u) == 0u) {
+    d.dbg->site = site;
+    d.dbg->index = idx;
+    d.dbg->extent = extent;
+  }
+  return false;
+}
+#define KVQ_IN_BOUNDS(d, site, idx, extent) ::kvq::debug_in_bounds((d), (site), (idx), (extent))
+#else
+#define KVQ_IN_BOUNDS(d, site, idx, extent) true
+#endif
+// [idx, idx + len) inside [0, extent)
+#define KVQ_RANGE_IN_BOUNDS(d, site, idx, len, extent) \
+  (KVQ_IN_BOUNDS(d, site, idx, extent) && KVQ_IN_BOUNDS(d, site, (idx) + (len) - 1, extent))
 
 // Width and bit offset in its packed row of channel c of a per-channel width map given by
 // its class counts (channels of width 8, then 4, 2, 1, then 0): the offset is the sum of
@@ -199,7 +262,7 @@ Partials workspace_views(const Dims& d, int splits, void* ws);
 cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows, int g_begin,
                                  int n_groups, uint32_t* kcode, __half2* ksz, const int* table,
                                  bool rotate, cudaStream_t s);
-cudaError_t launch_table_writes(int* table, const TableWrites& tw, cudaStream_t s);
+cudaError_t launch_table_writes(const Dims& d, int* table, const TableWrites& tw, cudaStream_t s);
 
 // Side codes of key groups [g_begin, g_begin + n_groups) whose base codes and (scale, zero)
 // are already in kcode / ksz (same stream); keys read from src as for launch_quantize_keys.
@@ -210,8 +273,8 @@ cudaError_t launch_quantize_side(const Dims& d, const __half* src, int src_rows,
 cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_rows, int t_begin,
                                    int n_tokens, uint32_t* vcode, __half2* vsz, const int* table,
                                    cudaStream_t s);
-cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,
-                             int dst_rows, int dst_base, int n, int d, int nbh, cudaStream_t s);
+cudaError_t launch_copy_rows(const Dims& d, const __half* src, int src_rows, int src_base, __half* dst,
+                             int dst_rows, int dst_base, int n, int width, int nbh, cudaStream_t s);
 // Rotated key rows (one warp per row): dst[bh][dst row i] = rotate(src[bh][src row i]) for
 // i < n, rows (src_base + i) % src_rows -> (dst_base + i) % dst_rows, or, when `list` is
 // given, rows list->pos[i] -> i.

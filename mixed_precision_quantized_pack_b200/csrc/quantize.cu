@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
   const bool active = g_first + gi < n_groups;
   const int g = g_begin + g_first + gi;
   const size_t base = static_cast<size_t>(bh) * src_rows;
+  const long long src_ext = static_cast<long long>(d.B) * d.Hkv * src_rows * dk;
 
   uint4 x[R];
   if constexpr (ROT) {
@@ -157,7 +158,10 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
       const int row = ((g_begin + g_first + yy) * gk + t) % src_rows;
       float v[8];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) v[m] = m < dk / 32 ? __half2float(src[(base + row) * dk + lane + 32 * m]) : 0.0f;
+      for (int m = 0; m < 8; ++m) {
+        const long long si = static_cast<long long>((base + row) * dk) + lane + 32 * m;
+        v[m] = m < dk / 32 && KVQ_IN_BOUNDS(d, kSiteQKeySrc, si, src_ext) ? __half2float(src[si]) : 0.0f;
+      }
       rotate_row_warp<8>(v, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
 #pragma unroll
       for (int m = 0; m < 8; ++m)
@@ -171,8 +175,10 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       const int row = (g * gk + rs + slabs * i) % src_rows;
-      x[i] = active ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
-                    : make_uint4(0, 0, 0, 0);
+      const long long si = static_cast<long long>((base + row) * dk) + 8 * cc;
+      x[i] = active && KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, si, 8, src_ext)
+                 ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
+                 : make_uint4(0, 0, 0, 0);
     }
   }
   {
@@ -230,6 +236,9 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
     const int g2 = i / (dk / 4), j = i % (dk / 4);
     if (g_first + g2 >= n_groups) continue;
     const size_t gidx = group_index(d, table, b, h, g_begin + g_first + g2);
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeyMeta, static_cast<long long>(gidx * 2 * dk) + 8 * j, 8,
+                             quant_groups(d) * 2 * dk))
+      continue;
     reinterpret_cast<uint4*>(reinterpret_cast<__half*>(ksz) + gidx * 2 * dk)[j] =
         reinterpret_cast<const uint4*>(blk + g2 * 2 * dk)[j];
   }
@@ -246,6 +255,9 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
   for (int i = 0; i < R; ++i) {
     const uint64_t bits = pack_chunk<BITS, 1>(x[i], z, r, sc);
     const size_t row = row0 + rs + slabs * i;
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeyCode, static_cast<long long>(row * (dk * BITS / 8)) + cc * BITS, BITS,
+                             quant_rows(d) * d.kw * 4))
+      continue;
     if constexpr (BITS == 2)
       reinterpret_cast<uint16_t*>(kcode)[row * (dk / 8) + cc] = static_cast<uint16_t>(bits);
     else if constexpr (BITS == 4)
@@ -297,7 +309,11 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
       const int row = (g * gk + t) % src_rows;
       float x[8];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) x[m] = m < dk / 32 ? __half2float(src[(base + row) * dk + lane + 32 * m]) : 0.0f;
+      for (int m = 0; m < 8; ++m) {
+        const long long si = static_cast<long long>((base + row) * dk) + lane + 32 * m;
+        x[m] = m < dk / 32 && KVQ_IN_BOUNDS(d, kSiteSideSrc, si, static_cast<long long>(d.B) * hkv * src_rows * dk)
+                   ? __half2float(src[si]) : 0.0f;
+      }
       rotate_row_warp<8>(x, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
 #pragma unroll
       for (int m = 0; m < 8; ++m)
@@ -312,20 +328,27 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
       x = e[t * es + c];
     } else {
       const int row = (g * gk + t) % src_rows;
-      x = __half2float(src[(base + row) * dk + c]);
+      const long long si = static_cast<long long>((base + row) * dk) + c;
+      x = KVQ_IN_BOUNDS(d, kSiteSideSrc, si, static_cast<long long>(d.B) * hkv * src_rows * dk)
+              ? __half2float(src[si]) : 0.0f;
     }
-    const uint32_t w = kcode[(row0 + t) * words + c / per];
+    const long long ki = static_cast<long long>((row0 + t) * words) + c / per;
+    const uint32_t w = KVQ_IN_BOUNDS(d, kSiteSideCode, ki, quant_rows(d) * words) ? kcode[ki] : 0u;
     const uint32_t code = (w >> ((c % per) * kb)) & ((1u << kb) - 1u);
     // the channel's (scale, zero) slots in the group's paired, quarter-interleaved block
     const int wd = c / per, r = c % per;
     const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
     const int slot = pos * 2 * per + (r % half) * 2 + r / half;
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteSideMeta, static_cast<long long>(gidx * 2 * dk) + slot, per + 1,
+                             quant_groups(d) * 2 * dk))
+      continue;
     const float kh = __fadd_rn(__fmul_rn(static_cast<float>(code), __half2float(blk[slot])),
                                __half2float(blk[slot + per]));
     e[t * es + c] = __fsub_rn(x, kh);
   }
   for (int idx = threadIdx.x; idx < dk * sr; idx += blockDim.x)
-    u[idx] = side_u[static_cast<size_t>(h) * dk * sr + idx];
+    u[idx] = KVQ_IN_BOUNDS(d, kSiteSideU, static_cast<long long>(h) * dk * sr + idx, static_cast<long long>(hkv) * dk * sr)
+                 ? side_u[static_cast<size_t>(h) * dk * sr + idx] : 0.0f;
   __syncthreads();
   for (int idx = threadIdx.x; idx < gk * sr; idx += blockDim.x) {
     const int t = idx / sr, i = idx % sr;
@@ -348,7 +371,8 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
     }
     if (lane == 0) {
       const GroupParams gp = group_params<SQ>(mn, mx);
-      zsz[gidx * sr + i] = gp.sz;
+      if (KVQ_IN_BOUNDS(d, kSiteSideZMeta, static_cast<long long>(gidx * sr) + i, quant_groups(d) * sr))
+        zsz[gidx * sr + i] = gp.sz;
       params[i] = make_float2(gp.scale, gp.zero);
     }
   }
@@ -361,6 +385,8 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
       gp.zero = params[i].y;
       row |= quant_code<SQ>(y[t * sr + i], gp) << (i * SQ);
     }
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteSideZCode, static_cast<long long>((row0 + t) * zb), zb, quant_rows(d) * zb))
+      continue;
     uint8_t* dst = zcode + (row0 + t) * zb;
     if (zb == 4)
       *reinterpret_cast<uint32_t*>(dst) = row;
@@ -392,9 +418,10 @@ __global__ void __launch_bounds__(256) quantize_values_kernel(
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       ri[i] = wb * block_rows + rsub + static_cast<long long>(rpw) * i;
-      if (ri[i] < rows) {
-        const int bh = static_cast<int>(ri[i] / n_tokens);
-        const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
+      const int bh = static_cast<int>(ri[i] / n_tokens);
+      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
+      const long long si = static_cast<long long>((static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + 8 * cc;
+      if (ri[i] < rows && KVQ_RANGE_IN_BOUNDS(d, kSiteQValSrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dv)) {
         x[i] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + cc);
       } else {
         x[i] = make_uint4(0, 0, 0, 0);
@@ -416,9 +443,14 @@ __global__ void __launch_bounds__(256) quantize_values_kernel(
       const int bh = static_cast<int>(ri[i] / n_tokens);
       const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
       const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
-      if (cc % gl == 0) vsz[vrow * d.nvg + cc / gl] = gp.sz;
+      if (cc % gl == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow * d.nvg) + cc / gl,
+                                        quant_rows(d) * d.nvg))
+        vsz[vrow * d.nvg + cc / gl] = gp.sz;
       const float rcp = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
       const uint64_t bits = pack_chunk<BITS, 0>(x[i], &gp.zero, &rcp, &gp.scale);
+      if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQValCode, static_cast<long long>(vrow * (dv * BITS / 8)) + cc * BITS, BITS,
+                               quant_rows(d) * d.vw * 4))
+        continue;
       if constexpr (BITS == 2)
         reinterpret_cast<uint16_t*>(vcode)[vrow * cpr + cc] = static_cast<uint16_t>(bits);
       else if constexpr (BITS == 4)
@@ -498,8 +530,10 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
 #pragma unroll
   for (int i = 0; i < R; ++i) {
     const int row = (g * gk + rs + slabs * i) % src_rows;
-    x[i] = active ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
-                  : make_uint4(0, 0, 0, 0);
+    const long long si = static_cast<long long>((base + row) * dk) + 8 * cc;
+    x[i] = active && KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dk)
+               ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
+               : make_uint4(0, 0, 0, 0);
   }
   {
     const __half2* h0 = reinterpret_cast<const __half2*>(&x[0]);
@@ -551,6 +585,8 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
     const int g2 = i / (dk / 4), j = i % (dk / 4);
     if (g_first + g2 >= n_groups) continue;
     const size_t gidx = group_index(d, table, b, h, g_begin + g_first + g2);
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeyMeta, static_cast<long long>(gidx * dk) + 4 * j, 4, quant_groups(d) * dk))
+      continue;
     reinterpret_cast<uint4*>(ksz + gidx * dk)[j] = reinterpret_cast<const uint4*>(blk + g2 * dk)[j];
   }
   if (active) {
@@ -573,7 +609,8 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
   for (int i = tid; i < gpc * gk * kw; i += 256) {
     const int g2 = i / (gk * kw);
     if (g_first + g2 >= n_groups) continue;
-    kcode[group_row(d, table, b, h, g_begin + g_first + g2) * kw + i % (gk * kw)] = sm_rows[i];
+    const long long ki = static_cast<long long>(group_row(d, table, b, h, g_begin + g_first + g2) * kw) + i % (gk * kw);
+    if (KVQ_IN_BOUNDS(d, kSiteQKeyCode, ki, quant_rows(d) * kw)) kcode[ki] = sm_rows[i];
   }
 }
 
@@ -605,9 +642,10 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
 #pragma unroll
     for (int i = 0; i < R; ++i) {
       ri[i] = wb * block_rows + rsub + static_cast<long long>(rpw) * i;
-      if (ri[i] < rows) {
-        const int bh = static_cast<int>(ri[i] / n_tokens);
-        const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
+      const int bh = static_cast<int>(ri[i] / n_tokens);
+      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
+      const long long si = static_cast<long long>((static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + 8 * cc;
+      if (ri[i] < rows && KVQ_RANGE_IN_BOUNDS(d, kSiteQValSrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dv)) {
         x[i] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + cc);
       } else {
         x[i] = make_uint4(0, 0, 0, 0);
@@ -632,7 +670,9 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
       const int bh = static_cast<int>(ri[i] / n_tokens);
       const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
       const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
-      if (cc % gl == 0) vsz[vrow * d.nvg + cc / gl] = gp.sz;
+      if (cc % gl == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow * d.nvg) + cc / gl,
+                                        quant_rows(d) * d.nvg))
+        vsz[vrow * d.nvg + cc / gl] = gp.sz;
       if (!width) continue;
       const float rcp = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
       const __half2* h2 = reinterpret_cast<const __half2*>(&x[i]);
@@ -662,7 +702,8 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
       const int bh = static_cast<int>(rr / n_tokens);
       const int t = t_begin + static_cast<int>(rr % n_tokens);
       const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
-      vcode[vrow * vw + k % vw] = rows_sm[k];
+      const long long vi = static_cast<long long>(vrow * vw) + k % vw;
+      if (KVQ_IN_BOUNDS(d, kSiteQValCode, vi, quant_rows(d) * vw)) vcode[vi] = rows_sm[k];
     }
     __syncwarp();
   }
@@ -671,8 +712,8 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
 // dst[bh][(dst_base + i) % dst_rows] = src[bh][(src_base + i) % src_rows], i < n, 16 B at a time.
 __global__ void copy_rows_kernel(const __half* __restrict__ src, int src_rows, int src_base,
                                  __half* __restrict__ dst, int dst_rows, int dst_base, int n,
-                                 int d, int nbh) {
-  const int vec = d / 8;
+                                 int width, int nbh, Dims d) {
+  const int vec = width / 8;
   const long long total = static_cast<long long>(nbh) * n * vec;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -682,8 +723,13 @@ __global__ void copy_rows_kernel(const __half* __restrict__ src, int src_rows, i
     const int bh = static_cast<int>(r / n);
     const int sr = (src_base + i) % src_rows;
     const int dr = (dst_base + i) % dst_rows;
-    const uint4* s = reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + sr) * d);
-    uint4* t = reinterpret_cast<uint4*>(dst + (static_cast<size_t>(bh) * dst_rows + dr) * d);
+    const long long si = static_cast<long long>((static_cast<size_t>(bh) * src_rows + sr) * width) + 8 * e;
+    const long long di = static_cast<long long>((static_cast<size_t>(bh) * dst_rows + dr) * width) + 8 * e;
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteCopySrc, si, 8, static_cast<long long>(nbh) * src_rows * width) ||
+        !KVQ_RANGE_IN_BOUNDS(d, kSiteCopyDst, di, 8, static_cast<long long>(nbh) * dst_rows * width))
+      continue;
+    const uint4* s = reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + sr) * width);
+    uint4* t = reinterpret_cast<uint4*>(dst + (static_cast<size_t>(bh) * dst_rows + dr) * width);
     t[e] = s[e];
   }
 }
@@ -692,13 +738,14 @@ __global__ void copy_rows_kernel(const __half* __restrict__ src, int src_rows, i
 // sequence b (none when it is -1), 16 B per thread; k null: values only.
 __global__ void append_token_kernel(const __half* __restrict__ k, const __half* __restrict__ v,
                                     __half* __restrict__ win_k, __half* __restrict__ win_v,
-                                    SlotMap slots, int hkv, int cap, int dk, int dv, int nbh) {
+                                    SlotMap slots, int hkv, int cap, int dk, int dv, int nbh, Dims d) {
   const int vk = dk / 8, vv = dv / 8;
   const int total = nbh * (vk + vv);
   for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
     const int bh = idx / (vk + vv), e = idx % (vk + vv);
     const int slot = slots.slot[bh / hkv];
     if (slot < 0) continue;
+    if (!KVQ_IN_BOUNDS(d, kSiteAppendWin, slot, cap)) continue;
     if (e < vk) {
       if (k)
         reinterpret_cast<uint4*>(win_k + (static_cast<size_t>(bh) * cap + slot) * dk)[e] =
@@ -727,6 +774,7 @@ __global__ void rotate_key_rows_kernel(const __half* __restrict__ src, int src_r
     const int sr = use_list ? list.pos[i] : (src_base + i) % src_rows;
     const int dr = use_slots ? slots.slot[bh / d.Hkv] : (dst_base + i) % dst_rows;
     if (dr < 0) continue;                                   // uniform per warp
+    if (!KVQ_IN_BOUNDS(d, kSiteRotSrc, sr, src_rows) || !KVQ_IN_BOUNDS(d, kSiteRotDst, dr, dst_rows)) continue;
     const __half* s = src + (static_cast<size_t>(bh) * src_rows + sr) * dk;
     __half* t = dst + (static_cast<size_t>(bh) * dst_rows + dr) * dk;
     float x[8];
@@ -742,9 +790,10 @@ __global__ void rotate_key_rows_kernel(const __half* __restrict__ src, int src_r
 // Prefill: ret[bh][j] = K[bh][pos[j]] for the retained positions (keys and values).
 __global__ void copy_retained_kernel(const __half* __restrict__ k, const __half* __restrict__ v,
                                      int L, int dk, int dv, RetList ret,
-                                     __half* __restrict__ ret_k, __half* __restrict__ ret_v) {
+                                     __half* __restrict__ ret_k, __half* __restrict__ ret_v, Dims d) {
   const int bh = blockIdx.x;
   for (int j = 0; j < ret.n; ++j) {
+    if (!KVQ_IN_BOUNDS(d, kSiteRetSrc, ret.pos[j], L) || !KVQ_IN_BOUNDS(d, kSiteRetDst, j, kMaxRetained)) continue;
     const size_t src = static_cast<size_t>(bh) * L + ret.pos[j];
     const size_t dst = static_cast<size_t>(bh) * kMaxRetained + j;
     if (k)
@@ -761,9 +810,13 @@ __global__ void copy_retained_kernel(const __half* __restrict__ k, const __half*
 __global__ void update_retained_kernel(RetUpdate up, int cap, int dk, int dv,
                                        const __half* __restrict__ win_k,
                                        const __half* __restrict__ win_v, __half* ret_k,
-                                       __half* ret_v) {
+                                       __half* ret_v, Dims d) {
   const int bh = blockIdx.x;
   for (int i = 0; i < up.n; ++i) {
+    // uniform per CTA: the loop's barriers stay matched
+    if (!KVQ_IN_BOUNDS(d, kSiteRetUpd, up.index[i], up.from_window[i] ? cap : kMaxRetained) ||
+        !KVQ_IN_BOUNDS(d, kSiteRetDst, i, kMaxRetained))
+      continue;
     const size_t dst = static_cast<size_t>(bh) * kMaxRetained + i;
     const __half* sk;
     const __half* sv;
@@ -788,8 +841,11 @@ __global__ void update_retained_kernel(RetUpdate up, int cap, int dk, int dv,
 }
 
 // Block-table entries of a paged cache: table[idx[i]] = page[i].
-__global__ void table_writes_kernel(int* __restrict__ table, TableWrites tw) {
-  for (int i = threadIdx.x; i < tw.n; i += blockDim.x) table[tw.idx[i]] = tw.page[i];
+__global__ void table_writes_kernel(int* __restrict__ table, TableWrites tw, Dims d) {
+  for (int i = threadIdx.x; i < tw.n; i += blockDim.x)
+    if (KVQ_IN_BOUNDS(d, kSiteTableIdx, tw.idx[i], static_cast<long long>(d.B) * d.max_groups) &&
+        KVQ_IN_BOUNDS(d, kSiteTablePage, tw.page[i], d.n_pages))
+      table[tw.idx[i]] = tw.page[i];
 }
 
 inline int grid_for(long long items, int block) {
@@ -861,9 +917,9 @@ cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows,
                 : launch_quantize_keys_r<false>(d, src, src_rows, g_begin, n_groups, kcode, ksz, table, s);
 }
 
-cudaError_t launch_table_writes(int* table, const TableWrites& tw, cudaStream_t s) {
+cudaError_t launch_table_writes(const Dims& d, int* table, const TableWrites& tw, cudaStream_t s) {
   if (tw.n <= 0) return cudaSuccess;
-  table_writes_kernel<<<1, 256, 0, s>>>(table, tw);
+  table_writes_kernel<<<1, 256, 0, s>>>(table, tw, d);
   return cudaGetLastError();
 }
 
@@ -931,13 +987,13 @@ cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_row
   return cudaGetLastError();
 }
 
-cudaError_t launch_copy_rows(const __half* src, int src_rows, int src_base, __half* dst,
-                             int dst_rows, int dst_base, int n, int d, int nbh, cudaStream_t s) {
+cudaError_t launch_copy_rows(const Dims& d, const __half* src, int src_rows, int src_base, __half* dst,
+                             int dst_rows, int dst_base, int n, int width, int nbh, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  const long long items = static_cast<long long>(nbh) * n * (d / 8);
+  const long long items = static_cast<long long>(nbh) * n * (width / 8);
   const int block = 256;
   copy_rows_kernel<<<grid_for(items, block), block, 0, s>>>(src, src_rows, src_base, dst, dst_rows,
-                                                            dst_base, n, d, nbh);
+                                                            dst_base, n, width, nbh, d);
   return cudaGetLastError();
 }
 
@@ -947,7 +1003,7 @@ cudaError_t launch_append_token(const Dims& d, const __half* k, const __half* v,
   const int total = nbh * (d.dk + d.dv) / 8;
   const int block = 256;
   append_token_kernel<<<(total + block - 1) / block, block, 0, s>>>(
-      d.rot ? nullptr : k, v, win_k, win_v, slots, d.Hkv, d.cap, d.dk, d.dv, nbh);
+      d.rot ? nullptr : k, v, win_k, win_v, slots, d.Hkv, d.cap, d.dk, d.dv, nbh, d);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !d.rot) return e;
   // rotated keys: one warp per (b, kv head) row
@@ -961,7 +1017,7 @@ cudaError_t launch_append_token(const Dims& d, const __half* k, const __half* v,
 cudaError_t launch_copy_retained(const Dims& d, const __half* k, const __half* v, int L,
                                  const RetList& ret, __half* ret_k, __half* ret_v, cudaStream_t s) {
   if (ret.n <= 0) return cudaSuccess;
-  copy_retained_kernel<<<d.B * d.Hkv, 64, 0, s>>>(k, v, L, d.dk, d.dv, ret, ret_k, ret_v);
+  copy_retained_kernel<<<d.B * d.Hkv, 64, 0, s>>>(k, v, L, d.dk, d.dv, ret, ret_k, ret_v, d);
   return cudaGetLastError();
 }
 
@@ -970,7 +1026,7 @@ cudaError_t launch_update_retained(const Dims& d, const RetUpdate& up, __half* w
   if (up.n <= 0) return cudaSuccess;
   const int threads = ((d.dk > d.dv ? d.dk : d.dv) / 8 + 31) / 32 * 32;
   update_retained_kernel<<<d.B * d.Hkv, threads, 0, s>>>(up, d.cap, d.dk, d.dv, win_k, win_v,
-                                                          ret_k, ret_v);
+                                                          ret_k, ret_v, d);
   return cudaGetLastError();
 }
 

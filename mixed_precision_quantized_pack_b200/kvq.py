@@ -15,7 +15,9 @@ from typing import Dict, List, Optional, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkvq.so")
+# The library to load: the in-tree libkvq.so, or (KVQ_LIBRARY=debug) its bounds-check build
+# libkvq_debug.so, built from the same sources with -DKVQ_DEBUG.
+LIB_PATH = os.path.join(_HERE, "libkvq_debug.so" if os.environ.get("KVQ_LIBRARY") == "debug" else "libkvq.so")
 
 KVQ_OK = 0
 KVQ_ERR_INVALID_ARG = -1
@@ -55,6 +57,11 @@ class kvq_sizes(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in SIZE_FIELDS]
 
 
+class kvq_debug_record(ctypes.Structure):
+    _fields_ = [("failures", ctypes.c_uint), ("site", ctypes.c_uint), ("index", ctypes.c_longlong),
+                ("extent", ctypes.c_longlong)]
+
+
 class kvq_buffers(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in POINTER_FIELDS]
 
@@ -91,6 +98,9 @@ _SIGNATURES = {
     "kvq_decode_attention_noalloc": (_I, [_P, _P, _P, _I, _P]),
     "kvq_noalloc_read_status": (_I, [ctypes.POINTER(ctypes.c_uint), _P]),
     "kvq_noalloc_reset_status": (_I, [_P]),
+    "kvq_debug_build": (_I, []),
+    "kvq_debug_take_record": (_I, [ctypes.POINTER(kvq_debug_record), _P]),
+    "kvq_debug_site_name": (ctypes.c_char_p, [ctypes.c_uint]),
     "kvq_get_plan": (_I, [_P, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_set_decode_kernel": (_I, [_P, _I]),
     "kvq_debug_stall_next_decode": (_I, [_P]),
@@ -273,6 +283,19 @@ def kvq_get_plan(handle: int, num_splits: int = 0) -> Dict[str, int]:
 
 def kvq_set_decode_kernel(handle: int, kernel: int) -> None:
     _check(lib().kvq_set_decode_kernel(handle, int(kernel)), "kvq_set_decode_kernel")
+
+
+def kvq_debug_build() -> bool:
+    """True when the loaded library is the bounds-check build."""
+    return bool(lib().kvq_debug_build())
+
+
+def kvq_debug_take_record(stream: int) -> Dict[str, object]:
+    """The bounds-check build's record of failed checks on the current device (then cleared)."""
+    r = kvq_debug_record()
+    _check(lib().kvq_debug_take_record(ctypes.byref(r), stream), "kvq_debug_take_record")
+    return {"failures": int(r.failures), "site": lib().kvq_debug_site_name(r.site).decode(),
+            "index": int(r.index), "extent": int(r.extent)}
 
 
 def kvq_debug_stall_next_decode(handle: int) -> None:

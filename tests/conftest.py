@@ -23,3 +23,19 @@ def read_golden(name):
             if line:
                 rows.append([field.split() for field in line.split("|")])
     return rows
+
+
+@pytest.fixture(autouse=True)
+def _bounds_check_record(request):
+    """Under the bounds-check build (KVQ_LIBRARY=debug), every GPU test must leave the
+    library's record of failed bounds checks empty."""
+    yield
+    if os.environ.get("KVQ_LIBRARY") != "debug" or request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    from mixed_precision_quantized_pack_b200 import kvq as K
+    assert K.kvq_debug_build(), "KVQ_LIBRARY=debug but the loaded library has no bounds checks"
+    rec = K.kvq_debug_take_record(K._stream())
+    assert rec["failures"] == 0, f"a bounds check failed: {rec}"

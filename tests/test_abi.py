@@ -1,5 +1,8 @@
 """Host-side checks of the C ABI: no kernel launches, so these run without a GPU."""
+import ctypes
 import os
+import subprocess
+import sys
 import re
 
 import pytest
@@ -334,3 +337,28 @@ def test_width_map_sizes_match_the_oracle_layout(kw_, vw_, gv, fast):
     p = K.kvq_plan_decode(c, 3000, 148, 0)
     assert p["fast_path"] == fast and p["n_groups"] == (3000 - 128) // 64
     assert K.kvq_plan_decode(dict(c, d_k=64), 3000, 148, 0)["fast_path"] == 0 if len(kw_) == 128 else True
+
+
+def test_release_build_has_no_bounds_checks():
+    """The in-tree libkvq.so is the release build: kvq_debug_take_record is UNSUPPORTED there
+    (no device call is made), and every check site has a name."""
+    lib = K.lib()
+    assert lib.kvq_debug_build() == 0
+    rec = K.kvq_debug_record()
+    assert lib.kvq_debug_take_record(ctypes.byref(rec), None) == K.KVQ_ERR_UNSUPPORTED
+    assert lib.kvq_debug_take_record(None, None) == K.KVQ_ERR_INVALID_ARG
+    names = [lib.kvq_debug_site_name(i).decode() for i in range(64)]
+    assert names[0] == "none" and "unknown" in names
+    known = names[:names.index("unknown")]
+    assert len(set(known)) == len(known) > 20
+
+
+def test_bounds_check_build_reports_itself():
+    """libkvq_debug.so (built with -DKVQ_DEBUG from the same sources) says so."""
+    path = os.path.join(ROOT, "mixed_precision_quantized_pack_b200", "libkvq_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("bounds-check library not built")
+    code = ("import ctypes,sys; l=ctypes.CDLL(sys.argv[1]); l.kvq_debug_build.restype=ctypes.c_int; "
+            "print(l.kvq_debug_build())")
+    out = subprocess.run([sys.executable, "-c", code, path], capture_output=True, text=True, timeout=120)
+    assert out.stdout.strip() == "1", out.stderr

@@ -518,7 +518,18 @@ def test_paged_cache_tensor_kernel():
 
 def test_paged_cache_with_side_code_and_rotation():
     w = W.WORKLOADS["headq32k"].with_(batch=3, rot_keys=1, rot_seed=9, seed=261, paged=1)
+    assert tensor_kernel_built(w)
     run_paged(w, [900, 333, 1280], n_app=66, steps={1, 10, 64, 65}, seed=262, restart=10)
+
+
+@pytest.mark.parametrize("kb,sr,sq", [(2, 4, 4), (4, 8, 4), (4, 4, 8)])
+def test_paged_cache_with_side_code_tensor_kernel(kb, sr, sq):
+    """Paged caches with a side code run on the tensor-core kernel (the paged side-code
+    instances), against the oracle and bit for bit against their unpaged twins."""
+    w = W.WORKLOADS["headq32k"].with_(batch=2, k_bits=kb, side_rank=sr, side_bits=sq,
+                                      seed=263 + sr + sq, paged=1)
+    assert tensor_kernel_built(w)
+    run_paged(w, [1000, 555], n_app=66, steps={0, 65}, seed=264)
 
 
 def test_paged_cache_generic_shapes():
