@@ -175,6 +175,7 @@ typedef struct kvq_plan {
     int n_groups;       /* quantized groups, Q / group_k */
     int n_fp16;         /* fp16 tokens: retained + window */
     int fast_path;      /* 1: tensor-core kernel; 0: generic CUDA-core kernel */
+    int centered;       /* 1: the tensor-core kernel centres the value codes (see below) */
 } kvq_plan;
 
 /* Bytes of each buffer for a configuration (see the layout above).  Host only.
@@ -273,6 +274,19 @@ int kvq_decode_attention(kvq_cache* cache, const void* q, void* out, void* works
 #define KVQ_KERNEL_GENERIC  1
 #define KVQ_KERNEL_TENSOR   2
 int kvq_set_decode_kernel(kvq_cache* cache, int kernel);
+
+/* Value-code centring of the tensor-core kernel on fixed-width caches (a numerical choice of
+ * this library; no counterpart on the pages).  Its p.V products of unsigned value codes
+ * accumulate in fp32 inside the tensor core, which truncates; the accumulated magnitude grows
+ * with the tokens summed while the attention output shrinks, so the relative error grows with
+ * the context.  Centred codes (code - 2^(v_bits-1), the offset added back through the zero-point
+ * sum) keep the accumulators near zero, at about 7% more decode time.  KVQ_CENTER_AUTO (the
+ * default) centres when the longest sequence has at least 65536 quantized tokens; ON and OFF
+ * force it.  The plan's `centered` field reports the choice.  Errors: INVALID_ARG. */
+#define KVQ_CENTER_AUTO     0
+#define KVQ_CENTER_OFF      1
+#define KVQ_CENTER_ON       2
+int kvq_set_value_centering(kvq_cache* cache, int mode);
 
 /* kvq_decode_attention without a workspace argument, for callers that cannot
  * allocate device memory: an engine that has reserved the device's memory for

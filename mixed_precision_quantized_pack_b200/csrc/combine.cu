@@ -10,10 +10,12 @@
 namespace kvq {
 namespace {
 
-// One warp per row (b, hq): lane s < splits holds split s's (m, l); the warp reduces the
-// maximum and the weighted sum of l with shuffles, then every lane merges 4 channels
-// (dv / 4 <= 32 * 4) of all splits with independent 16-byte loads.
+// One warp per row (b, hq); lane l merges channels 4l .. 4l+3 of every 128-channel block.  The
+// merge is latency-bound (a few kilobytes per row, in L2), so each lane first issues the loads
+// of kChunk splits' 16-byte pieces at once, then reads the splits' (m, l) (the same address in
+// every lane) for the maximum and the denominator, then weights the pieces it already holds.
 constexpr int kRowsPerBlock = 4;
+constexpr int kChunk = 8;
 
 __global__ void __launch_bounds__(32 * kRowsPerBlock)
 combine_kernel(const float2* __restrict__ ml, const float* __restrict__ o, int rows, int splits, int dv,
@@ -26,40 +28,35 @@ combine_kernel(const float2* __restrict__ ml, const float* __restrict__ o, int r
   if (row >= rows) return;                                    // uniform per warp
   const float2* mlr = ml + static_cast<size_t>(row) * splits;
   const float* orow = o + static_cast<size_t>(row) * splits * dv;
-  float M = -INFINITY;
-  for (int s = lane; s < splits; s += 32) M = fmaxf(M, mlr[s].x);
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  float den = 0.0f;
-  for (int s = lane; s < splits; s += 32) {
-    const float2 v = mlr[s];
-    if (v.x != -INFINITY) den = fmaf(exp2f(v.x - M), v.y, den);
-  }
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-  // every lane runs every iteration (the shuffles need the whole warp); lanes past d_v
-  // only skip their loads and stores
+  float M = -INFINITY, den = 0.0f;
   for (int c0 = 0; c0 < dv; c0 += 128) {
     const int c = c0 + 4 * lane;
     const bool mine = c < dv;
     float4 num = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int s0 = 0; s0 < splits; s0 += 32) {
-      // weight of split s0 + j, held by lane j
-      const int sj = s0 + lane;
-      float wj = 0.0f;
-      if (sj < splits) {
-        const float mj = mlr[sj].x;
-        wj = mj == -INFINITY ? 0.0f : exp2f(mj - M);
+    for (int s0 = 0; s0 < splits; s0 += kChunk) {
+      float4 buf[kChunk];
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j)
+        buf[j] = mine && s0 + j < splits
+                     ? *reinterpret_cast<const float4*>(orow + static_cast<size_t>(s0 + j) * dv + c)
+                     : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (c0 == 0 && s0 == 0) {
+        // splits that saw no token carry m = -inf, l = 0 and are skipped
+        for (int s = 0; s < splits; ++s) M = fmaxf(M, mlr[s].x);
+        for (int s = 0; s < splits; ++s) {
+          const float2 v = mlr[s];
+          if (v.x != -INFINITY) den = fmaf(exp2f(v.x - M), v.y, den);
+        }
       }
-      const int n = min(32, splits - s0);
-      for (int j = 0; j < n; ++j) {
-        const float w = __shfl_sync(0xffffffffu, wj, j);
-        if (w == 0.0f || !mine) continue;
-        const float4 x = *reinterpret_cast<const float4*>(orow + static_cast<size_t>(s0 + j) * dv + c);
-        num.x = fmaf(w, x.x, num.x);
-        num.y = fmaf(w, x.y, num.y);
-        num.z = fmaf(w, x.z, num.z);
-        num.w = fmaf(w, x.w, num.w);
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) {
+        if (s0 + j >= splits) break;
+        const float mj = mlr[s0 + j].x;
+        const float wj = mj == -INFINITY ? 0.0f : exp2f(mj - M);
+        num.x = fmaf(wj, buf[j].x, num.x);
+        num.y = fmaf(wj, buf[j].y, num.y);
+        num.z = fmaf(wj, buf[j].z, num.z);
+        num.w = fmaf(wj, buf[j].w, num.w);
       }
     }
     if (mine) {

@@ -374,6 +374,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   bool failed = false;
 
   const float alpha = w.score_scale;                       // log2(e) / sqrt(d_k)
+  constexpr float kMid = static_cast<float>(1 << ((QUANT ? VB : 2) - 1));   // centre of the value codes
   const float alpha24 = w.score_scale * 16777216.0f;       // undoes the 2^-24 of subnormal codes
 
   if (quant) {
@@ -682,7 +683,10 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
             for (int gg = 0; gg < G::NVG; ++gg) {
               const float2 f0 = __half22float2(ptx::u32_as_h2(vm0[gg]));
               const float2 f1 = __half22float2(ptx::u32_as_h2(vm1[gg]));
-              zsum[gg] = fmaf(p0, f0.y, fmaf(p1, f1.y, zsum[gg]));
+              // with centred codes (c - mid) the zero-point sum takes z + mid * s instead of z
+              const float zc0 = w.center ? fmaf(kMid, f0.x, f0.y) : f0.y;
+              const float zc1 = w.center ? fmaf(kMid, f1.x, f1.y) : f1.y;
+              zsum[gg] = fmaf(p0, zc0, fmaf(p1, zc1, zsum[gg]));
               const uint32_t x0 = ptx::split_hi_lo_trunc(p0 * f0.x);
               const uint32_t x1 = ptx::split_hi_lo_trunc(p1 * f1.x);
               const uint32_t bp0 = ptx::movmatrix_trans(x0);
@@ -715,6 +719,16 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
                   unpack_value_piece16<VB>(ptx::prmt(wa0, wb0, sel_hi), ra + n16);
                   unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_lo), rb);
                   unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_hi), rb + n16);
+                }
+              }
+              if (w.center) {
+                // centred codes (c - mid) * 2^(p-24), mid = 2^(VB-1): an exact fp16 subnormal
+                // subtraction that keeps the accumulators near zero
+#pragma unroll
+                for (int e = 0; e < G::CPG; ++e) {
+                  const uint32_t mid = (1u << (VB - 1 + value_code_shift<VB, G::RUN>(e))) * 0x00010001u;
+                  ra[e] = ptx::h2_as_u32(__hsub2(ptx::u32_as_h2(ra[e]), ptx::u32_as_h2(mid)));
+                  rb[e] = ptx::h2_as_u32(__hsub2(ptx::u32_as_h2(rb[e]), ptx::u32_as_h2(mid)));
                 }
               }
 #pragma unroll

@@ -23,6 +23,7 @@ struct kvq_cache {
   std::vector<int> held;         // paged: pages of each sequence, its table entries [0, held)
   int sm_count;
   int kernel;     // KVQ_KERNEL_*
+  int centering;  // KVQ_CENTER_*
   bool stall_next;  // test hook armed by kvq_debug_stall_next_decode
   bool uniform() const {
     for (size_t b = 1; b < L.size(); ++b)
@@ -157,6 +158,7 @@ int make_dims(const kvq_config* c, kvq::Dims* d) {
   x.lcap = static_cast<int>(lcap);
   x.paged = c->paged;
   x.n_pages = c->paged ? c->n_pages : 0;
+  x.sm_count = 148;
   x.dbg = nullptr;
   x.max_groups = static_cast<int>(lcap / x.gk);
   x.cap = raw ? c->max_context : c->window + c->group_k;
@@ -221,8 +223,15 @@ void seq_counts(const kvq::Dims& d, int L, int* nG, int* nF) {
 // Chooses the split counts: the number of CTAs per (b, kv head) over the quantized
 // groups and over the fp16 tokens, trading wave quantization against per-CTA cost; nG and
 // nF are those of the longest sequence.
+// Value-code centring of the tensor-core kernel: on from this many quantized tokens (AUTO).  Its
+// p.V products of unsigned codes accumulate in fp32 inside the MMA, which truncates; the
+// accumulators grow with the tokens summed while the output (a softmax-weighted mean) shrinks,
+// so the relative error grows with the context.  Centred codes keep the accumulators near zero
+// at the cost of one fp16 subtraction per code register (measured: +7% decode time).
+constexpr int kCenterFromTokens = 65536;
+
 int plan_counts(const kvq::Dims& d, int nG, int nF, int sm_count, int num_splits, bool fast,
-                kvq_plan* out) {
+                kvq_plan* out, int centering = KVQ_CENTER_AUTO) {
   if (sm_count < 1 || num_splits < 0) return KVQ_ERR_INVALID_ARG;
   const int rows = d.B * d.Hkv;
   const int cap = split_cap(d);
@@ -267,6 +276,10 @@ int plan_counts(const kvq::Dims& d, int nG, int nF, int sm_count, int num_splits
   out->n_groups = nG;
   out->n_fp16 = nF;
   out->fast_path = fast ? 1 : 0;
+  out->centered = fast && d.quantized() && !d.var &&
+                  (centering == KVQ_CENTER_ON ||
+                   (centering == KVQ_CENTER_AUTO && static_cast<long long>(nG) * d.gk >= kCenterFromTokens))
+                      ? 1 : 0;
   return KVQ_OK;
 }
 
@@ -286,7 +299,7 @@ int plan_cache(const kvq_cache* c, int num_splits, bool fast, kvq_plan* out) {
     nG = std::max(nG, g);
     nF = std::max(nF, f);
   }
-  return plan_counts(c->d, nG, nF, c->sm_count, num_splits, fast, out);
+  return plan_counts(c->d, nG, nF, c->sm_count, num_splits, fast, out, c->centering);
 }
 
 int check_cuda(cudaError_t e) { return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA; }
@@ -468,6 +481,7 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
   kvq_cache* c = new (std::nothrow) kvq_cache;
   if (!c) return KVQ_ERR_INVALID_ARG;
   c->d = d;
+  c->d.sm_count = sms;
   c->buf = *bufs;
   if (!d.paged) c->buf.block_table = nullptr;
   c->L.assign(d.B, 0);
@@ -480,6 +494,7 @@ int kvq_cache_init(const kvq_config* cfg, const kvq_buffers* bufs, kvq_cache** o
   }
   c->sm_count = sms;
   c->kernel = KVQ_KERNEL_AUTO;
+  c->centering = KVQ_CENTER_AUTO;
   c->stall_next = false;
   *out = c;
   return KVQ_OK;
@@ -860,6 +875,7 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
   w.splits = plan.splits_quant + plan.splits_fp16;
   w.score_scale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(d.dk)));
   w.stall = c->stall_next && plan.fast_path ? 1 : 0;
+  w.center = plan.centered;
   c->stall_next = false;
   if (workspace_bytes < kvq::workspace_bytes(d, w.splits)) return KVQ_ERR_WORKSPACE;
   const kvq::Partials parts = kvq::workspace_views(d, w.splits, workspace);
@@ -878,6 +894,12 @@ int kvq_decode_attention(kvq_cache* c, const void* q, void* out, void* workspace
 int kvq_debug_stall_next_decode(kvq_cache* c) {
   if (!c) return KVQ_ERR_INVALID_ARG;
   c->stall_next = true;
+  return KVQ_OK;
+}
+
+int kvq_set_value_centering(kvq_cache* c, int mode) {
+  if (!c || mode < KVQ_CENTER_AUTO || mode > KVQ_CENTER_ON) return KVQ_ERR_INVALID_ARG;
+  c->centering = mode;
   return KVQ_OK;
 }
 

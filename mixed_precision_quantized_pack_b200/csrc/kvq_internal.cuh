@@ -55,6 +55,7 @@ struct Dims {
   int var;
   int kcnt[4], vcnt[4];
   int n_pages;      // pages of a paged cache's pool (0 otherwise)
+  int sm_count;     // SMs of the cache's device (persistent grids; set when the handle is made)
   DebugRecord* dbg; // bounds-check builds: the library's debug record on this device (else null)
   bool quantized() const { return kb != 16; }
 };
@@ -90,7 +91,7 @@ __device__ __forceinline__ bool debug_in_bounds(const Dims& d, unsigned int site
 }
 #define KVQ_IN_BOUNDS(d, site, idx, extent) ::kvq::debug_in_bounds((d), (site), (idx), (extent))
 #else
-#define KVQ_IN_BOUNDS(d, site, idx, extent) true
+#define KVQ_IN_BOUNDS(d, site, idx, extent) (static_cast<void>(idx), true)
 #endif
 // [idx, idx + len) inside [0, extent)
 #define KVQ_RANGE_IN_BOUNDS(d, site, idx, len, extent) \
@@ -201,6 +202,7 @@ struct DecodeWork {
   int splits;        // splits_q + splits_f (partials per (b, query head))
   float score_scale; // log2(e) / sqrt(d_k)
   int stall;         // test hook: CTA (0, 0, 0) asks for 16 bytes more than its first copy delivers
+  int center;        // 1: the tensor-core kernel centres the value codes (long contexts)
 };
 
 // Lengths of sequence b in a decode call: L, Q, quantized groups (Q / gk; Q is 0 for an

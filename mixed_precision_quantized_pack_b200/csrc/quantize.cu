@@ -13,6 +13,7 @@
 // (scale, zero) block is stored in the order the decode kernel pairs channels.
 // Values: one group per token over group_v consecutive channels.
 #include "kvq_internal.cuh"
+#include "ptx.cuh"
 
 namespace kvq {
 namespace {
@@ -57,40 +58,45 @@ template <int BITS>
 __device__ __forceinline__ uint32_t quant_code(float x, const GroupParams& g) { return quant_code_b(x, g, BITS); }
 
 // The code of one element from the group's zero z and the reciprocal r = fl32(1/s) of its
-// scale, equal to the quantizer's rint(fl32(fl32(x - z) / s)) clamped to [0, 2^b - 1]
-// wherever `near` stays false:
-//   the quotient Q = d/s (d = fl32(x - z) >= 0) is below 512 (s is the fp16 rounding of
-//   (max - min)/(2^b - 1) with b <= 8, or a subnormal at most 1.5x smaller, or 0 and then r = 0
-//   and every code 0); q = fl32(d * r) = Q (1 + e1)(1 + e2) with |e1|, |e2| <= 2^-24, so
-//   |q - Q| <= 2^-14, and the IEEE quotient fl32(Q) is within half an ulp, 2^-16, of Q.  If q
-//   lies more than 2^-13 from every half-integer (|q - rint(q)| <= 1/2 - 2^-13; q - rint(q) is
-//   exact by Sterbenz), Q and fl32(Q) lie strictly inside q's rounding cell and round to the
-//   same integer.  Otherwise `near` is set and the caller takes the IEEE division.
+// scale, equal to the quantizer's clamp(rint(fl32(fl32(x - z) / s)), 0, 2^b - 1) wherever
+// `near` stays false:
+//   with d = fl32(x - z) >= 0, the exact quotient Q = d/s is below 512 (s is the fp16 rounding
+//   of (max - min)/(2^b - 1) with b <= 8, or a subnormal at most 1.5x smaller; s = 0 gives
+//   r = 0 and code 0).  P = d * r = Q (1 + e), |e| <= 2^-24, so |P - Q| < 2^-15, and the IEEE
+//   quotient F = fl32(Q) is within half an ulp, 2^-16, of Q.  y = fma(d, r, 1.5 * 2^23) rounds
+//   the exact P to the nearest integer c (ties to even: spacing 1 at that magnitude, and the
+//   constant is even), c = y - 1.5 * 2^23 exactly, and t = fma(d, r, -c) is P - c up to 2^-25.
+//   If |t| <= 1/2 - 2^-13 then |F - c| < 1/2 - 2^-14, so rint(F) = c; otherwise `near` is set
+//   and the caller takes the IEEE division.  No float-to-integer conversion is needed: the
+//   integer c is the low bits of y.
 constexpr float kNearHalf = 0.5f - 1.0f / 8192.0f;
+constexpr float kRoundMagic = 12582912.0f;         // 1.5 * 2^23
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 
-__device__ __forceinline__ uint32_t code_fast_l(float x, float z, float r, float levels, bool& near) {
-  const float q = __fmul_rn(__fsub_rn(x, z), r);
-  const float c = rintf(q);
-  near |= fabsf(__fsub_rn(q, c)) > kNearHalf;
-  return static_cast<uint32_t>(fminf(c, levels));
+__device__ __forceinline__ uint32_t code_fast_l(float x, float z, float r, uint32_t levels, bool& near) {
+  const float d = __fsub_rn(x, z);
+  const float y = __fmaf_rn(d, r, kRoundMagic);
+  const float c = __fsub_rn(y, kRoundMagic);
+  near |= fabsf(__fmaf_rn(d, r, -c)) > kNearHalf;
+  return min(__float_as_uint(y) - kRoundMagicBits, levels);
 }
 
 // The quantizer's code with the IEEE division (the rare elements code_fast leaves undecided).
-__device__ __forceinline__ uint32_t code_exact_l(float x, float z, float s, float levels) {
+__device__ __forceinline__ uint32_t code_exact_l(float x, float z, float s, uint32_t levels) {
   if (s == 0.0f) return 0u;
   float c = rintf(__fdiv_rn(__fsub_rn(x, z), s));
-  c = fminf(fmaxf(c, 0.0f), levels);
+  c = fminf(fmaxf(c, 0.0f), static_cast<float>(levels));
   return static_cast<uint32_t>(c);
 }
 
 template <int BITS>
 __device__ __forceinline__ uint32_t code_fast(float x, float z, float r, bool& near) {
-  return code_fast_l(x, z, r, static_cast<float>((1 << BITS) - 1), near);
+  return code_fast_l(x, z, r, (1u << BITS) - 1u, near);
 }
 
 template <int BITS>
 __device__ __forceinline__ uint32_t code_exact(float x, float z, float s) {
-  return code_exact_l(x, z, s, static_cast<float>((1 << BITS) - 1));
+  return code_exact_l(x, z, s, (1u << BITS) - 1u);
 }
 
 // Codes of 8 consecutive channels (one 16-byte chunk of fp16) packed LSB-first: 8 * BITS bits.
@@ -129,58 +135,23 @@ __device__ __forceinline__ uint64_t pack_chunk(const uint4& raw, const float* z,
 // into (scale, zero) there, and the codes are computed from the registers.  A CTA of 256
 // threads holds 256 / TPG groups.  ROT: the source keys are unrotated; warps first rotate the
 // CTA's rows into shared memory and the chunks are read from there.
-template <int BITS, int R, bool ROT>
-__global__ void __launch_bounds__(256) quantize_keys_kernel(
-    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
-    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
-  extern __shared__ __align__(16) unsigned char sm_dyn[];          // ROT: [gpc * gk][dk] fp16
-  __shared__ __align__(16) __half2 red[2][256][4];                  // per thread: min, max
-  __shared__ __align__(16) float prm[3][kKeyPrm];                   // zero, 1/scale, scale
-  __shared__ __align__(16) __half blk[kKeyBlk];                     // (scale, zero) blocks
+// The part of the key quantizer after a tile's chunks are in registers: thread (group gi of the
+// CTA, slab rs, chunk cc) holds rows rs, rs + gk/R, ... of chunk cc of group g_begin + g_first + gi
+// (of the launch's n_groups) of (b, kv head) bh.  Per-channel min and max in fp16 (exact),
+// reduced over the slabs in shared memory; (scale, zero) per channel, written as the groups'
+// blocks; then the codes from the registers.  Called by every thread of the CTA (barriers).
+template <int BITS, int R>
+__device__ __forceinline__ void key_tile(const uint4 (&x)[R], int bh, int g_begin, int g_first, int n_groups,
+                                         uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
+                                         const int* __restrict__ table, const Dims& d,
+                                         __half2 (*red)[256][4], float (*prm)[kKeyPrm], __half* blk) {
   const int dk = d.dk, gk = d.gk;
   const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
   const int tid = threadIdx.x;
-  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt % tpg / cpr;
-  const int bh = blockIdx.y, b = bh / d.Hkv, h = bh % d.Hkv;
-  const int g_first = blockIdx.x * gpc;           // first group of the CTA, among the launch's
+  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt / cpr;
+  const int b = bh / d.Hkv, h = bh % d.Hkv;
   const bool active = g_first + gi < n_groups;
   const int g = g_begin + g_first + gi;
-  const size_t base = static_cast<size_t>(bh) * src_rows;
-  const long long src_ext = static_cast<long long>(d.B) * d.Hkv * src_rows * dk;
-
-  uint4 x[R];
-  if constexpr (ROT) {
-    __half* rot = reinterpret_cast<__half*>(sm_dyn);
-    const int lane = tid & 31, warp = tid >> 5;
-    for (int rr = warp; rr < gpc * gk; rr += 8) {
-      const int yy = rr / gk, t = rr % gk;
-      if (g_first + yy >= n_groups) continue;                     // uniform per warp
-      const int row = ((g_begin + g_first + yy) * gk + t) % src_rows;
-      float v[8];
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const long long si = static_cast<long long>((base + row) * dk) + lane + 32 * m;
-        v[m] = m < dk / 32 && KVQ_IN_BOUNDS(d, kSiteQKeySrc, si, src_ext) ? __half2float(src[si]) : 0.0f;
-      }
-      rotate_row_warp<8>(v, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
-#pragma unroll
-      for (int m = 0; m < 8; ++m)
-        if (m < dk / 32) rot[static_cast<size_t>(rr) * dk + lane + 32 * m] = __float2half_rn(v[m]);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-      x[i] = reinterpret_cast<const uint4*>(rot)[(gi * gk + rs + slabs * i) * cpr + cc];
-  } else {
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const int row = (g * gk + rs + slabs * i) % src_rows;
-      const long long si = static_cast<long long>((base + row) * dk) + 8 * cc;
-      x[i] = active && KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, si, 8, src_ext)
-                 ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
-                 : make_uint4(0, 0, 0, 0);
-    }
-  }
   {
     const __half2* h0 = reinterpret_cast<const __half2*>(&x[0]);
     __half2 mn[4], mx[4];
@@ -242,7 +213,7 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
     reinterpret_cast<uint4*>(reinterpret_cast<__half*>(ksz) + gidx * 2 * dk)[j] =
         reinterpret_cast<const uint4*>(blk + g2 * 2 * dk)[j];
   }
-  if (!active) return;
+  if (!active) return;   // (the caller's loop has no barrier after this call)
   float z[8], r[8], sc[8];
 #pragma unroll
   for (int j = 0; j < 8; j += 4) {
@@ -266,6 +237,62 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
       reinterpret_cast<uint2*>(kcode)[row * (dk / 8) + cc] =
           make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
   }
+}
+
+template <int BITS, int R, bool ROT>
+__global__ void __launch_bounds__(256) quantize_keys_kernel(
+    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
+    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
+  extern __shared__ __align__(16) unsigned char sm_dyn[];          // ROT: [gpc * gk][dk] fp16
+  __shared__ __align__(16) __half2 red[2][256][4];                  // per thread: min, max
+  __shared__ __align__(16) float prm[3][kKeyPrm];                   // zero, 1/scale, scale
+  __shared__ __align__(16) __half blk[kKeyBlk];                     // (scale, zero) blocks
+  const int dk = d.dk, gk = d.gk;
+  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int tid = threadIdx.x;
+  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt % tpg / cpr;
+  const int bh = blockIdx.y;
+  const int g_first = blockIdx.x * gpc;           // first group of the CTA, among the launch's
+  const bool active = g_first + gi < n_groups;
+  const int g = g_begin + g_first + gi;
+  const size_t base = static_cast<size_t>(bh) * src_rows;
+  [[maybe_unused]] const long long src_ext = static_cast<long long>(d.B) * d.Hkv * src_rows * dk;
+
+  uint4 x[R];
+  if constexpr (ROT) {
+    __half* rot = reinterpret_cast<__half*>(sm_dyn);
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int rr = warp; rr < gpc * gk; rr += 8) {
+      const int yy = rr / gk, t = rr % gk;
+      if (g_first + yy >= n_groups) continue;                     // uniform per warp
+      const int row = ((g_begin + g_first + yy) * gk + t) % src_rows;
+      float v[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const long long si = static_cast<long long>((base + row) * dk) + lane + 32 * m;
+        v[m] = m < dk / 32 && KVQ_IN_BOUNDS(d, kSiteQKeySrc, si, src_ext) ? __half2float(src[si]) : 0.0f;
+      }
+      rotate_row_warp<8>(v, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+        if (m < dk / 32) rot[static_cast<size_t>(rr) * dk + lane + 32 * m] = __float2half_rn(v[m]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      x[i] = reinterpret_cast<const uint4*>(rot)[(gi * gk + rs + slabs * i) * cpr + cc];
+  } else {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int tk = g * gk + rs + slabs * i;
+      const int row = tk < src_rows ? tk : tk % src_rows;            // the window is a ring
+      const long long si = static_cast<long long>((base + row) * dk) + 8 * cc;
+      x[i] = active && KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, si, 8, src_ext)
+                 ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
+                 : make_uint4(0, 0, 0, 0);
+    }
+  }
+  key_tile<BITS, R>(x, bh, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk);
 }
 
 // Side code of key groups ("HeadQ: Distortion visible par le modele et correction dans
@@ -395,59 +422,84 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
   }
 }
 
-// Value quantize-pack, per token row over groups of gv channels.  A row is dv/8 16-byte chunks
-// of 8 channels, one chunk per lane, so a warp covers 32 / (dv/8) rows per load and each lane
-// R rows (rows rsub, rsub + 32/(dv/8), ... of the warp's block).  A value group is gv/8
-// consecutive lanes (gv is a multiple of 8): min and max in fp16 per lane, then by shuffles
-// across the group's lanes; every lane of a group derives the same (scale, zero).  Lane 0 of a
-// group writes its (scale, zero); each lane writes its chunk's 8 * BITS bits of codes.
+__device__ __forceinline__ uint32_t ptx_h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 ptx_u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// Extremes of a value group over its gl lanes (each holding 8 channels of the row), as the half2
+// (min, -max): one min-reduction over both (fp16 min and max are exact).
+__device__ __forceinline__ __half2 group_extremes(const uint4& raw, int gl) {
+  const __half2* hx = reinterpret_cast<const __half2*>(&raw);
+  const __half2 mn2 = __hmin2(__hmin2(hx[0], hx[1]), __hmin2(hx[2], hx[3]));
+  const __half2 mx2 = __hmax2(__hmax2(hx[0], hx[1]), __hmax2(hx[2], hx[3]));
+  __half2 e = __halves2half2(__hmin(__low2half(mn2), __high2half(mn2)),
+                             __hneg(__hmax(__low2half(mx2), __high2half(mx2))));
+  for (int off = 1; off < gl; off <<= 1)
+    e = __hmin2(e, ptx_u32_as_h2(__shfl_xor_sync(0xffffffffu, ptx_h2_as_u32(e), off)));
+  return e;
+}
+
+// Value quantize-pack, per token row over groups of gv channels.  CTA (x, y) covers tokens of
+// (b, kv head) row y; a token row is dv/8 16-byte chunks of 8 channels, one chunk per lane, so a
+// warp covers 32 / (dv/8) rows per load and each lane R rows (rows rsub, rsub + 32/(dv/8), ...
+// of the warp's block).  A value group is gv/8 consecutive lanes (gv is a multiple of 8): min
+// and max in fp16 per lane, then by shuffles across the group's lanes; every lane of a group
+// derives the same (scale, zero).  Lane 0 of a group writes its (scale, zero); each lane writes
+// its chunk's 8 * BITS bits of codes.
+// The part of the value quantizer after a warp's rows are in registers: lane (rsub, cc) holds
+// chunk cc of tokens t_begin + ti[i] (valid when ti[i] < n_tokens) of (b, kv head) bh.  Group
+// extremes by shuffles; (scale, zero) and 1/scale per row and group; codes and (scale, zero)
+// stored.  Called by every lane of the warp (shuffles).
 template <int BITS, int R>
-__global__ void __launch_bounds__(256) quantize_values_kernel(
-    const __half* __restrict__ src, int src_rows, int t_begin, int n_tokens,
-    uint32_t* __restrict__ vcode, __half2* __restrict__ vsz, const int* __restrict__ table, Dims d) {
-  const int dv = d.dv, cpr = dv / 8, rpw = 32 / cpr, gl = d.gv / 8;
+__device__ __forceinline__ void value_rows(const uint4 (&x)[R], const int (&ti)[R], int bh, int t_begin,
+                                           int n_tokens, uint32_t* __restrict__ vcode,
+                                           __half2* __restrict__ vsz, const int* __restrict__ table,
+                                           const Dims& d) {
+  const int dv = d.dv, cpr = dv / 8, gl = d.gv / 8;
   const int lane = threadIdx.x & 31;
-  const int cc = lane % cpr, rsub = lane / cpr;
-  const long long rows = static_cast<long long>(d.B) * d.Hkv * n_tokens;
-  const long long block_rows = static_cast<long long>(rpw) * R;          // rows per warp block
-  const long long n_blocks = (rows + block_rows - 1) / block_rows;
-  for (long long wb = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; wb < n_blocks;
-       wb += static_cast<long long>(gridDim.x) * blockDim.x / 32) {
-    uint4 x[R];
-    long long ri[R];
+  const int cc = lane % cpr;
+  const int lg = __ffs(d.gk) - 1;
+  {
+    // each row's group extremes as one half2 (min, -max), reduced over the group's lanes
+    // (aligned and consecutive)
+    __half2 ext[R];
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      ri[i] = wb * block_rows + rsub + static_cast<long long>(rpw) * i;
-      const int bh = static_cast<int>(ri[i] / n_tokens);
-      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
-      const long long si = static_cast<long long>((static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + 8 * cc;
-      if (ri[i] < rows && KVQ_RANGE_IN_BOUNDS(d, kSiteQValSrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dv)) {
-        x[i] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + cc);
-      } else {
-        x[i] = make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < R; ++i) ext[i] = group_extremes(x[i], gl);
+    // (scale, zero) and 1/scale of the R rows: with groups of at least R lanes, lane j of a group
+    // derives row j's in one pass and the rows are broadcast; otherwise every lane derives its own
+    const int gsub = cc % gl, gbase = lane - gsub;
+    __half2 rsz[R];
+    float rrc[R];
+    if (gl >= R) {
+      __half2 e = ext[0];
+#pragma unroll
+      for (int i = 1; i < R; ++i)
+        if (gsub == i) e = ext[i];
+      const GroupParams gp = group_params<BITS>(__low2float(e), -__high2float(e));
+      const uint32_t sz = ptx_h2_as_u32(gp.sz);
+      const float rc = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        rsz[i] = ptx_u32_as_h2(__shfl_sync(0xffffffffu, sz, gbase + i));
+        rrc[i] = __shfl_sync(0xffffffffu, rc, gbase + i);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const GroupParams gp = group_params<BITS>(__low2float(ext[i]), -__high2float(ext[i]));
+        rsz[i] = gp.sz;
+        rrc[i] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
       }
     }
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      const __half2* hx = reinterpret_cast<const __half2*>(&x[i]);
-      __half2 mn2 = __hmin2(__hmin2(hx[0], hx[1]), __hmin2(hx[2], hx[3]));
-      __half2 mx2 = __hmax2(__hmax2(hx[0], hx[1]), __hmax2(hx[2], hx[3]));
-      float mn = fminf(__low2float(mn2), __high2float(mn2));
-      float mx = fmaxf(__low2float(mx2), __high2float(mx2));
-      for (int off = 1; off < gl; off <<= 1) {         // lanes of one group: aligned, consecutive
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      }
-      if (ri[i] >= rows) continue;
-      const GroupParams gp = group_params<BITS>(mn, mx);
-      const int bh = static_cast<int>(ri[i] / n_tokens);
-      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
-      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
-      if (cc % gl == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow * d.nvg) + cc / gl,
-                                        quant_rows(d) * d.nvg))
-        vsz[vrow * d.nvg + cc / gl] = gp.sz;
-      const float rcp = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
-      const uint64_t bits = pack_chunk<BITS, 0>(x[i], &gp.zero, &rcp, &gp.scale);
+      if (ti[i] >= n_tokens) continue;
+      const float2 szf = __half22float2(rsz[i]);             // (scale, zero), exact
+      const int t = t_begin + ti[i];
+      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t >> lg) + (t & (d.gk - 1));
+      if (gsub == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow * d.nvg) + cc / gl,
+                                     quant_rows(d) * d.nvg))
+        vsz[vrow * d.nvg + cc / gl] = rsz[i];
+      const uint64_t bits = pack_chunk<BITS, 0>(x[i], &szf.y, &rrc[i], &szf.x);
       if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQValCode, static_cast<long long>(vrow * (dv * BITS / 8)) + cc * BITS, BITS,
                                quant_rows(d) * d.vw * 4))
         continue;
@@ -460,6 +512,181 @@ __global__ void __launch_bounds__(256) quantize_values_kernel(
             make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
     }
   }
+}
+
+template <int BITS, int R>
+__global__ void __launch_bounds__(256) quantize_values_kernel(
+    const __half* __restrict__ src, int src_rows, int t_begin, int n_tokens,
+    uint32_t* __restrict__ vcode, __half2* __restrict__ vsz, const int* __restrict__ table, Dims d) {
+  const int dv = d.dv, cpr = dv / 8, rpw = 32 / cpr;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int cc = lane % cpr, rsub = lane / cpr;
+  const int bh = blockIdx.y;
+  const int t_first = (blockIdx.x * 8 + warp) * rpw * R;             // this warp's block of tokens
+  if (t_first >= n_tokens) return;                                    // uniform per warp
+  const size_t src_base = static_cast<size_t>(bh) * src_rows;
+  {
+    uint4 x[R];
+    int ti[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      ti[i] = t_first + rsub + rpw * i;
+      const int t = t_begin + ti[i];
+      const int row = t < src_rows ? t : t % src_rows;                // the window is a ring
+      const long long si = static_cast<long long>((src_base + row) * dv) + 8 * cc;
+      if (ti[i] < n_tokens && KVQ_RANGE_IN_BOUNDS(d, kSiteQValSrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dv)) {
+        x[i] = __ldg(reinterpret_cast<const uint4*>(src + (src_base + row) * dv) + cc);
+      } else {
+        x[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    value_rows<BITS, R>(x, ti, bh, t_begin, n_tokens, vcode, vsz, table, d);
+  }
+}
+
+// ---- prefill quantizers over a contiguous source, persistent and staged ----
+// CTA c takes tiles c, c + gridDim.x, ... of the launch (a key tile: the gpc consecutive groups
+// of one (b, kv head) that a CTA holds; a value tile: 1024 / (dv/8) consecutive token rows of one
+// (b, kv head), 16 KB), each brought into shared memory by one 1-D bulk copy (cp.async.bulk) two
+// tiles ahead (double buffer, one mbarrier per stage), so HBM reads overlap the quantizer's
+// arithmetic.  The rows of a tile must be contiguous in the source (a prefill input: row t of
+// (b, h) at (b * Hkv + h) * src_rows + t); waits are bounded and a CTA whose wait gives up stops.
+constexpr uint64_t kStageWaitNs = 1000000000ull;
+
+struct StageRing {
+  uint64_t bars[2];
+  int issued[2];
+};
+
+// Waits (bounded) for the copies still in flight into the two stages before a CTA exits.
+__device__ __forceinline__ void drain_stages(StageRing* ring) {
+  if (threadIdx.x == 0)
+    for (int s = 0; s < 2; ++s)
+      if (ring->issued[s] > 0)
+        ptx::mbar_wait_bounded(ptx::smem_addr(&ring->bars[s]), (ring->issued[s] - 1) & 1, kStageWaitNs);
+  __syncthreads();
+}
+
+template <int BITS, int R>
+__global__ void __launch_bounds__(256) quantize_keys_staged_kernel(
+    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
+    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
+  extern __shared__ __align__(128) unsigned char sm_stage[];        // 2 x [gpc * gk][dk] fp16
+  __shared__ __align__(16) __half2 red[2][256][4];
+  __shared__ __align__(16) float prm[3][kKeyPrm];
+  __shared__ __align__(16) __half blk[kKeyBlk];
+  __shared__ __align__(8) StageRing ring;
+  const int dk = d.dk, gk = d.gk;
+  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int tid = threadIdx.x;
+  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt / cpr;
+  const int tiles_per_row = (n_groups + gpc - 1) / gpc;
+  const long long n_tiles = static_cast<long long>(d.B) * d.Hkv * tiles_per_row;
+  const int stage_bytes = gpc * gk * dk * 2;
+  const uint32_t st0 = ptx::smem_addr(sm_stage);
+  [[maybe_unused]] const long long src_ext = static_cast<long long>(d.B) * d.Hkv * src_rows * dk;
+  // thread 0 copies tile `tile` (its groups' gk rows each) into stage st
+  auto issue = [&](long long tile, int st) {
+    const int bh = static_cast<int>(tile / tiles_per_row), g_first = static_cast<int>(tile % tiles_per_row) * gpc;
+    const int ng = min(gpc, n_groups - g_first);
+    long long first = (static_cast<long long>(bh) * src_rows + static_cast<long long>(g_begin + g_first) * gk) * dk;
+    const uint32_t bytes = static_cast<uint32_t>(ng) * gk * dk * 2;
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, first, static_cast<long long>(ng) * gk * dk, src_ext)) first = 0;
+    ring.issued[st] += 1;
+    ptx::mbar_arrive_expect_tx(ptx::smem_addr(&ring.bars[st]), bytes);
+    ptx::bulk_g2s(st0 + st * stage_bytes, src + first, bytes, ptx::smem_addr(&ring.bars[st]));
+  };
+  if (tid == 0) {
+    for (int st = 0; st < 2; ++st) {
+      ptx::mbar_init(ptx::smem_addr(&ring.bars[st]), 1);
+      ring.issued[st] = 0;
+    }
+    ptx::fence_barrier_init();
+    for (int k = 0; k < 2; ++k)
+      if (blockIdx.x + static_cast<long long>(k) * gridDim.x < n_tiles) issue(blockIdx.x + static_cast<long long>(k) * gridDim.x, k);
+  }
+  __syncthreads();
+  for (int it = 0;; ++it) {
+    const long long tile = blockIdx.x + static_cast<long long>(it) * gridDim.x;
+    if (tile >= n_tiles) break;
+    const int st = it & 1;
+    const bool ok = ptx::mbar_wait_bounded(ptx::smem_addr(&ring.bars[st]), (it >> 1) & 1, kStageWaitNs);
+    if (!__syncthreads_and(ok)) break;                                 // a wait gave up: stop
+    const uint4* stage = reinterpret_cast<const uint4*>(sm_stage + st * stage_bytes);
+    uint4 x[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) x[i] = stage[(gi * gk + rs + slabs * i) * cpr + cc];
+    __syncthreads();                                                   // the stage may be refilled
+    if (tid == 0 && tile + 2LL * gridDim.x < n_tiles) {
+      ptx::fence_proxy_async_smem();
+      issue(tile + 2LL * gridDim.x, st);
+    }
+    const int bh = static_cast<int>(tile / tiles_per_row), g_first = static_cast<int>(tile % tiles_per_row) * gpc;
+    key_tile<BITS, R>(x, bh, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk);
+    __syncthreads();                                                   // red, prm, blk are reused
+  }
+  drain_stages(&ring);
+}
+
+template <int BITS, int R>
+__global__ void __launch_bounds__(256) quantize_values_staged_kernel(
+    const __half* __restrict__ src, int src_rows, int t_begin, int n_tokens,
+    uint32_t* __restrict__ vcode, __half2* __restrict__ vsz, const int* __restrict__ table, Dims d) {
+  extern __shared__ __align__(128) unsigned char sm_stage[];        // 2 x [tile rows][dv] fp16
+  __shared__ __align__(8) StageRing ring;
+  const int dv = d.dv, cpr = dv / 8, rpw = 32 / cpr;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int cc = lane % cpr, rsub = lane / cpr;
+  const int tile_rows = 8 * rpw * R;                                  // 16 KB of fp16 rows
+  const int tiles_per_row = (n_tokens + tile_rows - 1) / tile_rows;
+  const long long n_tiles = static_cast<long long>(d.B) * d.Hkv * tiles_per_row;
+  const int stage_bytes = tile_rows * dv * 2;
+  const uint32_t st0 = ptx::smem_addr(sm_stage);
+  [[maybe_unused]] const long long src_ext = static_cast<long long>(d.B) * d.Hkv * src_rows * dv;
+  auto issue = [&](long long tile, int st) {
+    const int bh = static_cast<int>(tile / tiles_per_row), t0 = static_cast<int>(tile % tiles_per_row) * tile_rows;
+    const int nr = min(tile_rows, n_tokens - t0);
+    long long first = (static_cast<long long>(bh) * src_rows + t_begin + t0) * dv;
+    const uint32_t bytes = static_cast<uint32_t>(nr) * dv * 2;
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQValSrc, first, static_cast<long long>(nr) * dv, src_ext)) first = 0;
+    ring.issued[st] += 1;
+    ptx::mbar_arrive_expect_tx(ptx::smem_addr(&ring.bars[st]), bytes);
+    ptx::bulk_g2s(st0 + st * stage_bytes, src + first, bytes, ptx::smem_addr(&ring.bars[st]));
+  };
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < 2; ++st) {
+      ptx::mbar_init(ptx::smem_addr(&ring.bars[st]), 1);
+      ring.issued[st] = 0;
+    }
+    ptx::fence_barrier_init();
+    for (int k = 0; k < 2; ++k)
+      if (blockIdx.x + static_cast<long long>(k) * gridDim.x < n_tiles) issue(blockIdx.x + static_cast<long long>(k) * gridDim.x, k);
+  }
+  __syncthreads();
+  for (int it = 0;; ++it) {
+    const long long tile = blockIdx.x + static_cast<long long>(it) * gridDim.x;
+    if (tile >= n_tiles) break;
+    const int st = it & 1;
+    const bool ok = ptx::mbar_wait_bounded(ptx::smem_addr(&ring.bars[st]), (it >> 1) & 1, kStageWaitNs);
+    if (!__syncthreads_and(ok)) break;                                 // a wait gave up: stop
+    const int bh = static_cast<int>(tile / tiles_per_row), t0 = static_cast<int>(tile % tiles_per_row) * tile_rows;
+    const uint4* stage = reinterpret_cast<const uint4*>(sm_stage + st * stage_bytes);
+    uint4 x[R];
+    int ti[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const int r = warp * rpw * R + rsub + rpw * i;                  // row within the tile
+      ti[i] = t0 + r;
+      x[i] = ti[i] < n_tokens ? stage[r * cpr + cc] : make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();                                                   // the stage may be refilled
+    if (threadIdx.x == 0 && tile + 2LL * gridDim.x < n_tiles) {
+      ptx::fence_proxy_async_smem();
+      issue(tile + 2LL * gridDim.x, st);
+    }
+    value_rows<BITS, R>(x, ti, bh, t_begin, n_tokens, vcode, vsz, table, d);
+  }
+  drain_stages(&ring);
 }
 
 // ---- per-channel widths ("Attention-Aware Transform Coding (AATC)", §Méthodologie,
@@ -484,12 +711,12 @@ __device__ __forceinline__ uint64_t pack_chunk_var(const uint4& raw, const float
   uint64_t bits = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j)
-    if (w[j]) bits |= static_cast<uint64_t>(code_fast_l(x[j], z[j], r[j], static_cast<float>((1 << w[j]) - 1), near)) << (o[j] - o[0]);
+    if (w[j]) bits |= static_cast<uint64_t>(code_fast_l(x[j], z[j], r[j], (1u << w[j]) - 1u, near)) << (o[j] - o[0]);
   if (near) {
     bits = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      if (w[j]) bits |= static_cast<uint64_t>(code_exact_l(x[j], z[j], sc[j], static_cast<float>((1 << w[j]) - 1))) << (o[j] - o[0]);
+      if (w[j]) bits |= static_cast<uint64_t>(code_exact_l(x[j], z[j], sc[j], (1u << w[j]) - 1u)) << (o[j] - o[0]);
   }
   return bits;
 }
@@ -529,7 +756,8 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
   uint4 x[R];
 #pragma unroll
   for (int i = 0; i < R; ++i) {
-    const int row = (g * gk + rs + slabs * i) % src_rows;
+    const int tk = g * gk + rs + slabs * i;
+    const int row = tk < src_rows ? tk : tk % src_rows;              // the window is a ring
     const long long si = static_cast<long long>((base + row) * dk) + 8 * cc;
     x[i] = active && KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dk)
                ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
@@ -628,48 +856,41 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
   const int cc = lane % cpr, rsub = lane / cpr;
   int width, offset;
   channel_width(d.vcnt, 8 * cc, &width, &offset);
-  const float levels = static_cast<float>((1 << width) - 1);
+  const uint32_t levels = (1u << width) - 1u;
   uint32_t* rows_sm = sm_rows[warp];
-  const long long rows = static_cast<long long>(d.B) * d.Hkv * n_tokens;
-  const long long block_rows = static_cast<long long>(rpw) * R;
-  const long long n_blocks = (rows + block_rows - 1) / block_rows;
-  for (long long wb = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; wb < n_blocks;
-       wb += static_cast<long long>(gridDim.x) * blockDim.x / 32) {
+  const int bh = blockIdx.y, lg = __ffs(d.gk) - 1;
+  const int block_rows = rpw * R;
+  const int t_first = (blockIdx.x * 8 + warp) * block_rows;          // this warp's block of tokens
+  if (t_first >= n_tokens) return;                                    // uniform per warp
+  const size_t src_base = static_cast<size_t>(bh) * src_rows;
+  {
     for (int k = lane; k < block_rows * vw; k += 32) rows_sm[k] = 0u;
     __syncwarp();
     uint4 x[R];
-    long long ri[R];
+    int ti[R];
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      ri[i] = wb * block_rows + rsub + static_cast<long long>(rpw) * i;
-      const int bh = static_cast<int>(ri[i] / n_tokens);
-      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
-      const long long si = static_cast<long long>((static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + 8 * cc;
-      if (ri[i] < rows && KVQ_RANGE_IN_BOUNDS(d, kSiteQValSrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dv)) {
-        x[i] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<size_t>(bh) * src_rows + t % src_rows) * dv) + cc);
+      ti[i] = t_first + rsub + rpw * i;
+      const int t = t_begin + ti[i];
+      const int row = t < src_rows ? t : t % src_rows;                // the window is a ring
+      const long long si = static_cast<long long>((src_base + row) * dv) + 8 * cc;
+      if (ti[i] < n_tokens && KVQ_RANGE_IN_BOUNDS(d, kSiteQValSrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dv)) {
+        x[i] = __ldg(reinterpret_cast<const uint4*>(src + (src_base + row) * dv) + cc);
       } else {
         x[i] = make_uint4(0, 0, 0, 0);
       }
     }
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      const __half2* hx = reinterpret_cast<const __half2*>(&x[i]);
-      __half2 mn2 = __hmin2(__hmin2(hx[0], hx[1]), __hmin2(hx[2], hx[3]));
-      __half2 mx2 = __hmax2(__hmax2(hx[0], hx[1]), __hmax2(hx[2], hx[3]));
-      float mn = fminf(__low2float(mn2), __high2float(mn2));
-      float mx = fmaxf(__low2float(mx2), __high2float(mx2));
-      for (int off = 1; off < gl; off <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      }
-      if (ri[i] >= rows) continue;
+      const __half2 e = group_extremes(x[i], gl);
+      const float mn = __low2float(e), mx = -__high2float(e);
+      if (ti[i] >= n_tokens) continue;
       GroupParams gp;
       gp.scale = gp.zero = 0.0f;
       gp.sz = __floats2half2_rn(0.0f, 0.0f);
       if (width) gp = group_params_b(mn, mx, width);
-      const int bh = static_cast<int>(ri[i] / n_tokens);
-      const int t = t_begin + static_cast<int>(ri[i] % n_tokens);
-      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
+      const int t = t_begin + ti[i];
+      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t >> lg) + (t & (d.gk - 1));
       if (cc % gl == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow * d.nvg) + cc / gl,
                                         quant_rows(d) * d.nvg))
         vsz[vrow * d.nvg + cc / gl] = gp.sz;
@@ -697,11 +918,10 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
     }
     __syncwarp();
     for (int k = lane; k < block_rows * vw; k += 32) {
-      const long long rr = wb * block_rows + k / vw;
-      if (rr >= rows) continue;
-      const int bh = static_cast<int>(rr / n_tokens);
-      const int t = t_begin + static_cast<int>(rr % n_tokens);
-      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t / d.gk) + t % d.gk;
+      const int tl = t_first + k / vw;
+      if (tl >= n_tokens) continue;
+      const int t = t_begin + tl;
+      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t >> lg) + (t & (d.gk - 1));
       const long long vi = static_cast<long long>(vrow * vw) + k % vw;
       if (KVQ_IN_BOUNDS(d, kSiteQValCode, vi, quant_rows(d) * vw)) vcode[vi] = rows_sm[k];
     }
@@ -875,6 +1095,21 @@ cudaError_t launch_quantize_keys_t(const Dims& d, const __half* src, int src_row
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
+  if (!ROT && static_cast<long long>(g_begin + n_groups) * d.gk <= src_rows) {
+    // a contiguous source (prefill): the persistent staged kernel
+    auto staged = rows == 4 ? quantize_keys_staged_kernel<BITS, 4>
+                : rows == 8 ? quantize_keys_staged_kernel<BITS, 8> : quantize_keys_staged_kernel<BITS, 16>;
+    const int sbytes = 2 * gpc * d.gk * d.dk * 2;
+    // static + dynamic shared memory above 48 KB needs the opt-in (set on every launch: it is a
+    // property of the current device's context)
+    const cudaError_t e = cudaFuncSetAttribute(staged, cudaFuncAttributeMaxDynamicSharedMemorySize, sbytes);
+    if (e != cudaSuccess) return e;
+    const long long tiles = static_cast<long long>(d.B) * d.Hkv * ((n_groups + gpc - 1) / gpc);
+    const long long slots = static_cast<long long>(d.sm_count > 0 ? d.sm_count : 148) * 4;
+    staged<<<static_cast<int>(tiles < slots ? tiles : slots), 256, sbytes, s>>>(src, src_rows, g_begin, n_groups,
+                                                                               kcode, ksz, table, d);
+    return cudaGetLastError();
+  }
   kern<<<grid, 256, smem, s>>>(src, src_rows, g_begin, n_groups, kcode, ksz, table, d);
   return cudaGetLastError();
 }
@@ -964,20 +1199,29 @@ cudaError_t launch_quantize_values(const Dims& d, const __half* src, int src_row
                                    cudaStream_t s) {
   if (n_tokens <= 0) return cudaSuccess;
   const int nbh = d.B * d.Hkv;
+  // CTA (x, y): tokens [x * per_cta, (x + 1) * per_cta) of (b, kv head) row y; 8 warps, each
+  // a block of 32 / (dv / 8) * kRows tokens
+  constexpr int kRows = 4;
+  const int per_cta = 8 * (32 / (d.dv / 8)) * kRows;
+  const dim3 grid((n_tokens + per_cta - 1) / per_cta, nbh);
   if (d.var) {
-    constexpr int kRows = 4;
-    const long long rows = static_cast<long long>(nbh) * n_tokens;
-    const long long per_cta = 8LL * (32 / (d.dv / 8)) * kRows;
-    const long long ctas = (rows + per_cta - 1) / per_cta;
-    const int grid = static_cast<int>(ctas < (1LL << 30) ? ctas : (1LL << 30));
     quantize_values_var_kernel<kRows><<<grid, 256, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d);
     return cudaGetLastError();
   }
-  constexpr int kRows = 4;
-  const long long rows = static_cast<long long>(nbh) * n_tokens;
-  const long long per_cta = 8LL * (32 / (d.dv / 8)) * kRows;   // 8 warps, each a block of rows
-  const long long ctas = (rows + per_cta - 1) / per_cta;
-  const int grid = static_cast<int>(ctas < (1LL << 30) ? ctas : (1LL << 30));
+  if (t_begin + n_tokens <= src_rows) {
+    // a contiguous source (prefill): the persistent staged kernel (two 16 KB stages)
+    const long long tiles = static_cast<long long>(nbh) * ((n_tokens + per_cta - 1) / per_cta);
+    const long long slots = static_cast<long long>(d.sm_count > 0 ? d.sm_count : 148) * 4;
+    const dim3 pgrid(static_cast<unsigned>(tiles < slots ? tiles : slots));
+    const int sbytes = 2 * per_cta * d.dv * 2;         // 32 KB: below the 48 KB default
+    switch (d.vb) {
+      case 2: quantize_values_staged_kernel<2, kRows><<<pgrid, 256, sbytes, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;
+      case 4: quantize_values_staged_kernel<4, kRows><<<pgrid, 256, sbytes, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;
+      case 8: quantize_values_staged_kernel<8, kRows><<<pgrid, 256, sbytes, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;
+      default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+  }
   switch (d.vb) {
     case 2: quantize_values_kernel<2, kRows><<<grid, 256, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;
     case 4: quantize_values_kernel<4, kRows><<<grid, 256, 0, s>>>(src, src_rows, t_begin, n_tokens, vcode, vsz, table, d); break;

@@ -31,6 +31,9 @@ KVQ_MAX_RETAINED = 32
 KVQ_KERNEL_AUTO = 0
 KVQ_KERNEL_GENERIC = 1
 KVQ_KERNEL_TENSOR = 2
+KVQ_CENTER_AUTO = 0
+KVQ_CENTER_OFF = 1
+KVQ_CENTER_ON = 2
 KVQ_STATUS_TIMEOUT = 1
 KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 KVQ_MAX_SEQS = 256
@@ -68,7 +71,7 @@ class kvq_buffers(ctypes.Structure):
 
 class kvq_plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("splits_quant", "splits_fp16", "n_groups", "n_fp16",
-                                            "fast_path")]
+                                            "fast_path", "centered")]
 
 
 class KVQError(RuntimeError):
@@ -103,6 +106,7 @@ _SIGNATURES = {
     "kvq_debug_site_name": (ctypes.c_char_p, [ctypes.c_uint]),
     "kvq_get_plan": (_I, [_P, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_set_decode_kernel": (_I, [_P, _I]),
+    "kvq_set_value_centering": (_I, [_P, _I]),
     "kvq_debug_stall_next_decode": (_I, [_P]),
     "kvq_plan_decode": (_I, [ctypes.POINTER(kvq_config), _I, _I, _I, ctypes.POINTER(kvq_plan)]),
     "kvq_get_state": (_I, [_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I),
@@ -285,6 +289,10 @@ def kvq_set_decode_kernel(handle: int, kernel: int) -> None:
     _check(lib().kvq_set_decode_kernel(handle, int(kernel)), "kvq_set_decode_kernel")
 
 
+def kvq_set_value_centering(handle: int, mode: int) -> None:
+    _check(lib().kvq_set_value_centering(handle, int(mode)), "kvq_set_value_centering")
+
+
 def kvq_debug_build() -> bool:
     """True when the loaded library is the bounds-check build."""
     return bool(lib().kvq_debug_build())
@@ -440,6 +448,9 @@ class KVCache:
 
     def set_kernel(self, kernel: int) -> None:
         kvq_set_decode_kernel(self.handle, kernel)
+
+    def set_centering(self, mode: int) -> None:
+        kvq_set_value_centering(self.handle, mode)
 
     def plan(self, num_splits: int = 0) -> Dict[str, int]:
         return kvq_get_plan(self.handle, num_splits)

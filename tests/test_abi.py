@@ -362,3 +362,21 @@ def test_bounds_check_build_reports_itself():
             "print(l.kvq_debug_build())")
     out = subprocess.run([sys.executable, "-c", code, path], capture_output=True, text=True, timeout=120)
     assert out.stdout.strip() == "1", out.stderr
+
+
+def test_value_centering_policy():
+    """The tensor-core kernel centres value codes from 65536 quantized tokens (AUTO); the plan
+    reports it, and never for the generic kernel, unquantized or per-channel-width caches."""
+    w = W.sweep_workload(8, 4, 2)
+    cfg = w.kvq_config()
+    assert K.kvq_plan_decode(cfg, 131072, 148, 0)["centered"] == 1
+    assert K.kvq_plan_decode(cfg, 65536 + 128, 148, 0)["centered"] == 1       # Q = 65536
+    assert K.kvq_plan_decode(cfg, 65536 + 127, 148, 0)["centered"] == 0       # Q = 65472
+    assert K.kvq_plan_decode(W.WORKLOADS["long32k"].kvq_config(), 32768, 148, 0)["centered"] == 0
+    assert K.kvq_plan_decode(W.sweep_workload(8, 16, 16).kvq_config(), 131072, 148, 0)["centered"] == 0
+    assert K.kvq_plan_decode(W.WORKLOADS["aatc32k"].with_(context=131072).kvq_config(), 131072, 148, 0)["centered"] == 0
+    generic = W.WORKLOADS["gqa4k"].with_(n_q_heads=64, context=131072)
+    assert K.kvq_plan_decode(generic.kvq_config(), 131072, 148, 0) == dict(
+        K.kvq_plan_decode(generic.kvq_config(), 131072, 148, 0), fast_path=0, centered=0)
+    lib = K.lib()
+    assert lib.kvq_set_value_centering(None, K.KVQ_CENTER_ON) == K.KVQ_ERR_INVALID_ARG

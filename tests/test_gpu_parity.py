@@ -79,14 +79,18 @@ def make_caches(cfg, inp, batch=None):
     return gc, oc
 
 
-def run_small(w: W.Workload, num_splits=(0,), steps=None):
+def run_small(w: W.Workload, num_splits=(0,), steps=None, centering=None):
     """Prefill + (appends) + decodes of a workload small enough for the full oracle."""
     need_gpu()
     inp = W.Inputs(w, device="cpu")
     cfg = w.kvq_config()
     gc, oc = make_caches(cfg, inp)
+    if centering is not None:
+        gc.set_centering(centering)
     gc.prefill(inp.k.cuda(), inp.v.cuda())
     oc.prefill(np16(inp.k), np16(inp.v))
+    if centering == K.KVQ_CENTER_ON:
+        assert gc.plan()["centered"] == 1
     compare_state(gc, oc, where="prefill")
     worst = 0.0
     n_dec = len(inp.q)
@@ -139,6 +143,18 @@ def test_bit_widths(kb, vb):
     w = W.WORKLOADS["gqa4k"].with_(batch=2, context=1500, k_bits=kb, v_bits=vb, appends=70,
                                    log_retain=1, seed=77)
     run_small(w, num_splits=(0, 2), steps={0, 1, 57, 58, 69})
+
+
+@pytest.mark.parametrize("kb,vb,gv,gk", [(4, 2, 64, 64), (4, 2, 32, 32), (8, 4, 64, 64), (8, 4, 32, 32),
+                                         (2, 2, 64, 64), (4, 4, 64, 64)])
+def test_centred_value_codes(kb, vb, gv, gk):
+    """The tensor-core kernel with centred value codes (forced on at these short contexts; the
+    library turns it on by itself from 65536 quantized tokens) matches the oracle."""
+    w = W.WORKLOADS["gqa4k"].with_(batch=2, context=1500, k_bits=kb, v_bits=vb, group_v=gv, group_k=gk,
+                                   appends=66, log_retain=1, seed=71 + kb + gv)
+    assert tensor_kernel_built(w)
+    need_gpu()
+    run_small(w, num_splits=(0, 2), steps={0, 64, 65}, centering=K.KVQ_CENTER_ON)
 
 
 def test_unquantized_fp16_cache():
