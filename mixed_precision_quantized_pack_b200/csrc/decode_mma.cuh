@@ -285,7 +285,7 @@ struct Rings {
 };
 
 template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4,
-          bool PAGED = false>
+          bool PAGED = false, bool CENTER = false>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__ q, Partials part) {
   using G = Quant<(QUANT ? KB : 4), (QUANT ? VB : 2), (QUANT ? DK : 128), (QUANT ? GV : 64)>;
@@ -684,8 +684,8 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
               const float2 f0 = __half22float2(ptx::u32_as_h2(vm0[gg]));
               const float2 f1 = __half22float2(ptx::u32_as_h2(vm1[gg]));
               // with centred codes (c - mid) the zero-point sum takes z + mid * s instead of z
-              const float zc0 = w.center ? fmaf(kMid, f0.x, f0.y) : f0.y;
-              const float zc1 = w.center ? fmaf(kMid, f1.x, f1.y) : f1.y;
+              const float zc0 = CENTER ? fmaf(kMid, f0.x, f0.y) : f0.y;
+              const float zc1 = CENTER ? fmaf(kMid, f1.x, f1.y) : f1.y;
               zsum[gg] = fmaf(p0, zc0, fmaf(p1, zc1, zsum[gg]));
               const uint32_t x0 = ptx::split_hi_lo_trunc(p0 * f0.x);
               const uint32_t x1 = ptx::split_hi_lo_trunc(p1 * f1.x);
@@ -721,7 +721,7 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
                   unpack_value_piece16<VB>(ptx::prmt(wa1, wb1, sel_hi), rb + n16);
                 }
               }
-              if (w.center) {
+              if constexpr (CENTER) {
                 // centred codes (c - mid) * 2^(p-24), mid = 2^(VB-1): an exact fp16 subnormal
                 // subtraction that keeps the accumulators near zero
 #pragma unroll
@@ -950,15 +950,15 @@ decode_mma_kernel(Dims d, CacheBufs cb, DecodeWork w, const __half* __restrict__
   }
 }
 
-template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4,
-          bool PAGED = false>
-cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
-                   const Partials& p, cudaStream_t s) {
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR, int SQ, bool PAGED,
+          bool CENTER>
+cudaError_t launch_impl(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
+                        const Partials& p, cudaStream_t s) {
   using RG = Rings<KB, VB, DK, GV, GK, QUANT, SR, SQ>;
   int smem = RG::BYTES;
   const int merge = kWarps * NREP * kDV * 4 + kWarps * NREP * 8;
   if (RG::HDR + merge > smem) smem = RG::HDR + merge;
-  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ, PAGED>;
+  auto kern = decode_mma_kernel<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ, PAGED, CENTER>;
   static int configured = 0;
   if (configured < smem) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -968,6 +968,18 @@ cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const
   dim3 grid(w.splits, d.Hkv, d.B);
   kern<<<grid, kThreads, smem, s>>>(d, c, w, q, p);
   return cudaGetLastError();
+}
+
+// The kernel instance for a decode: quantized caches take the centred-code instance when the
+// plan asks for it (long contexts), so the uncentred instance carries no trace of it.
+template <int KB, int VB, int DK, int NREP, int GV, int GK, bool QUANT, int SR = 0, int SQ = 4,
+          bool PAGED = false>
+cudaError_t launch(const Dims& d, const CacheBufs& c, const DecodeWork& w, const __half* q,
+                   const Partials& p, cudaStream_t s) {
+  if constexpr (QUANT) {
+    if (w.center) return launch_impl<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ, PAGED, true>(d, c, w, q, p, s);
+  }
+  return launch_impl<KB, VB, DK, NREP, GV, GK, QUANT, SR, SQ, PAGED, false>(d, c, w, q, p, s);
 }
 
 }  // namespace mma

@@ -12,6 +12,8 @@
 // channel over group_k consecutive tokens (LogQuant §5, per-channel keys); a group's
 // (scale, zero) block is stored in the order the decode kernel pairs channels.
 // Values: one group per token over group_v consecutive channels.
+#include <type_traits>
+
 #include "kvq_internal.cuh"
 #include "ptx.cuh"
 
@@ -99,12 +101,17 @@ __device__ __forceinline__ uint32_t code_exact(float x, float z, float s) {
   return code_exact_l(x, z, s, (1u << BITS) - 1u);
 }
 
+// The packed codes of one 16-byte chunk: 8 * BITS bits (a 32-bit word below 8 bits).
+template <int BITS>
+using ChunkBits = typename std::conditional<(BITS == 8), uint64_t, uint32_t>::type;
+
 // Codes of 8 consecutive channels (one 16-byte chunk of fp16) packed LSB-first: 8 * BITS bits.
 // Channel j's group has zero z[j], reciprocal scale r[j] and scale sc[j] (keys: one group per
 // channel), or every channel the same (values: STRIDE 0 reads element 0 for all j).
 template <int BITS, int STRIDE>
-__device__ __forceinline__ uint64_t pack_chunk(const uint4& raw, const float* z, const float* r,
-                                               const float* sc) {
+__device__ __forceinline__ ChunkBits<BITS> pack_chunk(const uint4& raw, const float* z, const float* r,
+                                                      const float* sc) {
+  using W = ChunkBits<BITS>;
   const __half2* hx = reinterpret_cast<const __half2*>(&raw);
   float x[8];
 #pragma unroll
@@ -114,42 +121,48 @@ __device__ __forceinline__ uint64_t pack_chunk(const uint4& raw, const float* z,
     x[2 * e + 1] = f.y;
   }
   bool near = false;
-  uint64_t bits = 0;
+  W bits = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j)
-    bits |= static_cast<uint64_t>(code_fast<BITS>(x[j], z[j * STRIDE], r[j * STRIDE], near)) << (j * BITS);
+    bits |= static_cast<W>(code_fast<BITS>(x[j], z[j * STRIDE], r[j * STRIDE], near)) << (j * BITS);
   if (near) {             // rare: a quotient within 2^-13 of a half-integer
     bits = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j)
-      bits |= static_cast<uint64_t>(code_exact<BITS>(x[j], z[j * STRIDE], sc[j * STRIDE])) << (j * BITS);
+      bits |= static_cast<W>(code_exact<BITS>(x[j], z[j * STRIDE], sc[j * STRIDE])) << (j * BITS);
   }
   return bits;
 }
 
-// Key quantize-pack of whole key groups.  A group (gk tokens x dk channels of fp16) is split
-// into 16-byte chunks of 8 channels; thread (slab rs, chunk cc) of the group's TPG = dk/8 *
-// gk/R threads holds rows rs, rs + gk/R, ... (R rows) of chunk cc, so a warp's loads and
-// stores are whole consecutive rows.  Each key is read once: the per-channel min and max are
-// taken in fp16 (exact) per thread, reduced across the group's slabs in shared memory, turned
-// into (scale, zero) there, and the codes are computed from the registers.  A CTA of 256
-// threads holds 256 / TPG groups.  ROT: the source keys are unrotated; warps first rotate the
-// CTA's rows into shared memory and the chunks are read from there.
+// Stores a chunk's packed codes at chunk index `idx` of a row array of (8 * BITS)-bit units.
+template <int BITS>
+__device__ __forceinline__ void store_chunk(uint32_t* base, size_t idx, ChunkBits<BITS> bits) {
+  if constexpr (BITS == 2)
+    reinterpret_cast<uint16_t*>(base)[idx] = static_cast<uint16_t>(bits);
+  else if constexpr (BITS == 4)
+    base[idx] = static_cast<uint32_t>(bits);
+  else
+    reinterpret_cast<uint2*>(base)[idx] = make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
+}
+
+__host__ __device__ constexpr int ilog2c(int x) { return x <= 1 ? 0 : 1 + ilog2c(x / 2); }
+
 // The part of the key quantizer after a tile's chunks are in registers: thread (group gi of the
 // CTA, slab rs, chunk cc) holds rows rs, rs + gk/R, ... of chunk cc of group g_begin + g_first + gi
-// (of the launch's n_groups) of (b, kv head) bh.  Per-channel min and max in fp16 (exact),
+// (of the launch's n_groups) of sequence b, kv head h.  Per-channel min and max in fp16 (exact),
 // reduced over the slabs in shared memory; (scale, zero) per channel, written as the groups'
-// blocks; then the codes from the registers.  Called by every thread of the CTA (barriers).
+// blocks; then the codes from the registers.  Every size here is a power of two, so the index
+// arithmetic is shifts and masks.  Called by every thread of the CTA (barriers).
 template <int BITS, int R>
-__device__ __forceinline__ void key_tile(const uint4 (&x)[R], int bh, int g_begin, int g_first, int n_groups,
-                                         uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
+__device__ __forceinline__ void key_tile(const uint4 (&x)[R], int b, int h, int g_begin, int g_first,
+                                         int n_groups, uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
                                          const int* __restrict__ table, const Dims& d,
                                          __half2 (*red)[256][4], float (*prm)[kKeyPrm], __half* blk) {
-  const int dk = d.dk, gk = d.gk;
-  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int dk = d.dk;
+  const int ldk = __ffs(dk) - 1, lcpr = ldk - 3, lslabs = __ffs(d.gk) - 1 - ilog2c(R);
+  const int ltpg = lcpr + lslabs, slabs = 1 << lslabs, gpc = 256 >> ltpg;
   const int tid = threadIdx.x;
-  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt / cpr;
-  const int b = bh / d.Hkv, h = bh % d.Hkv;
+  const int gi = tid >> ltpg, lt = tid & ((1 << ltpg) - 1), cc = lt & ((1 << lcpr) - 1), rs = lt >> lcpr;
   const bool active = g_first + gi < n_groups;
   const int g = g_begin + g_first + gi;
   {
@@ -175,67 +188,62 @@ __device__ __forceinline__ void key_tile(const uint4 (&x)[R], int bh, int g_begi
   __syncthreads();
   // per (group of the CTA, channel pair): reduce over the slabs, then (scale, zero)
   constexpr int per_w = 32 / BITS, half_w = 16 / BITS;
-  const int words = dk / per_w, quarter = words % 4 == 0 ? words / 4 : 0;
-  for (int p = tid; p < gpc * dk / 2; p += 256) {
-    const int g2 = p / (dk / 2), pp = p % (dk / 2), c2 = pp / 4, k = pp % 4;
-    const int t0 = g2 * tpg + c2;
+  const int lwords = ldk - ilog2c(per_w);                  // words per key row, log2
+  const int lquarter = lwords >= 2 ? lwords - 2 : -1;      // quarter-interleaved when 4 | words
+  for (int p = tid; p < (gpc << (ldk - 1)); p += 256) {
+    const int g2 = p >> (ldk - 1), pp = p & ((dk >> 1) - 1), c2 = pp >> 2, k = pp & 3;
+    const int t0 = (g2 << ltpg) + c2;
     __half2 mn = red[0][t0][k], mx = red[1][t0][k];
     for (int sl = 1; sl < slabs; ++sl) {
-      mn = __hmin2(mn, red[0][t0 + sl * cpr][k]);
-      mx = __hmax2(mx, red[1][t0 + sl * cpr][k]);
+      mn = __hmin2(mn, red[0][t0 + (sl << lcpr)][k]);
+      mx = __hmax2(mx, red[1][t0 + (sl << lcpr)][k]);
     }
     const float2 fmn = __half22float2(mn), fmx = __half22float2(mx);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int c = 8 * c2 + 2 * k + e;
       const GroupParams gp = group_params<BITS>(e ? fmn.y : fmn.x, e ? fmx.y : fmx.x);
-      prm[0][g2 * dk + c] = gp.zero;
-      prm[1][g2 * dk + c] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
-      prm[2][g2 * dk + c] = gp.scale;
+      prm[0][(g2 << ldk) + c] = gp.zero;
+      prm[1][(g2 << ldk) + c] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+      prm[2][(g2 << ldk) + c] = gp.scale;
       // the group's block of 2*dk fp16: per packed word w, the scales of channels
       // (w*per + i, w*per + i + per/2) for i < per/2, then their zeros in the same order;
       // the words' blocks quarter-interleaved when 4 divides the words per row
       const int wd = c / per_w, r = c % per_w;
-      const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
+      const int pos = lquarter >= 0 ? ((wd & ((1 << lquarter) - 1)) << 2) + (wd >> lquarter) : wd;
       const int slot = pos * 2 * per_w + (r % half_w) * 2 + r / half_w;
-      blk[g2 * 2 * dk + slot] = __low2half(gp.sz);
-      blk[g2 * 2 * dk + slot + per_w] = __high2half(gp.sz);
+      blk[(g2 << (ldk + 1)) + slot] = __low2half(gp.sz);
+      blk[(g2 << (ldk + 1)) + slot + per_w] = __high2half(gp.sz);
     }
   }
   __syncthreads();
-  for (int i = tid; i < gpc * dk / 4; i += 256) {                 // 16 B of a block per thread
-    const int g2 = i / (dk / 4), j = i % (dk / 4);
+  for (int i = tid; i < (gpc << (ldk - 2)); i += 256) {     // 16 B of a block per thread
+    const int g2 = i >> (ldk - 2), j = i & ((dk >> 2) - 1);
     if (g_first + g2 >= n_groups) continue;
     const size_t gidx = group_index(d, table, b, h, g_begin + g_first + g2);
     if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeyMeta, static_cast<long long>(gidx * 2 * dk) + 8 * j, 8,
                              quant_groups(d) * 2 * dk))
       continue;
     reinterpret_cast<uint4*>(reinterpret_cast<__half*>(ksz) + gidx * 2 * dk)[j] =
-        reinterpret_cast<const uint4*>(blk + g2 * 2 * dk)[j];
+        reinterpret_cast<const uint4*>(blk + (g2 << (ldk + 1)))[j];
   }
   if (!active) return;   // (the caller's loop has no barrier after this call)
   float z[8], r[8], sc[8];
 #pragma unroll
   for (int j = 0; j < 8; j += 4) {
-    *reinterpret_cast<float4*>(z + j) = *reinterpret_cast<const float4*>(&prm[0][gi * dk + 8 * cc + j]);
-    *reinterpret_cast<float4*>(r + j) = *reinterpret_cast<const float4*>(&prm[1][gi * dk + 8 * cc + j]);
-    *reinterpret_cast<float4*>(sc + j) = *reinterpret_cast<const float4*>(&prm[2][gi * dk + 8 * cc + j]);
+    *reinterpret_cast<float4*>(z + j) = *reinterpret_cast<const float4*>(&prm[0][(gi << ldk) + 8 * cc + j]);
+    *reinterpret_cast<float4*>(r + j) = *reinterpret_cast<const float4*>(&prm[1][(gi << ldk) + 8 * cc + j]);
+    *reinterpret_cast<float4*>(sc + j) = *reinterpret_cast<const float4*>(&prm[2][(gi << ldk) + 8 * cc + j]);
   }
   const size_t row0 = group_row(d, table, b, h, g);
 #pragma unroll
   for (int i = 0; i < R; ++i) {
-    const uint64_t bits = pack_chunk<BITS, 1>(x[i], z, r, sc);
+    const ChunkBits<BITS> bits = pack_chunk<BITS, 1>(x[i], z, r, sc);
     const size_t row = row0 + rs + slabs * i;
     if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeyCode, static_cast<long long>(row * (dk * BITS / 8)) + cc * BITS, BITS,
                              quant_rows(d) * d.kw * 4))
       continue;
-    if constexpr (BITS == 2)
-      reinterpret_cast<uint16_t*>(kcode)[row * (dk / 8) + cc] = static_cast<uint16_t>(bits);
-    else if constexpr (BITS == 4)
-      kcode[row * (dk / 8) + cc] = static_cast<uint32_t>(bits);
-    else
-      reinterpret_cast<uint2*>(kcode)[row * (dk / 8) + cc] =
-          make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
+    store_chunk<BITS>(kcode, (row << lcpr) + cc, bits);
   }
 }
 
@@ -292,7 +300,7 @@ __global__ void __launch_bounds__(256) quantize_keys_kernel(
                  : make_uint4(0, 0, 0, 0);
     }
   }
-  key_tile<BITS, R>(x, bh, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk);
+  key_tile<BITS, R>(x, bh / d.Hkv, bh % d.Hkv, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk);
 }
 
 // Side code of key groups ("HeadQ: Distortion visible par le modele et correction dans
@@ -444,73 +452,65 @@ __device__ __forceinline__ __half2 group_extremes(const uint4& raw, int gl) {
 // of the warp's block).  A value group is gv/8 consecutive lanes (gv is a multiple of 8): min
 // and max in fp16 per lane, then by shuffles across the group's lanes; every lane of a group
 // derives the same (scale, zero).  Lane 0 of a group writes its (scale, zero); each lane writes
-// its chunk's 8 * BITS bits of codes.
 // The part of the value quantizer after a warp's rows are in registers: lane (rsub, cc) holds
-// chunk cc of tokens t_begin + ti[i] (valid when ti[i] < n_tokens) of (b, kv head) bh.  Group
-// extremes by shuffles; (scale, zero) and 1/scale per row and group; codes and (scale, zero)
-// stored.  Called by every lane of the warp (shuffles).
+// chunk cc of tokens t_begin + ti[i] (valid when ti[i] < n_tokens) of sequence b, kv head h.
+// Group extremes by shuffles; (scale, zero) and 1/scale per row and group; codes and (scale,
+// zero) stored.  Sizes are powers of two (shifts and masks).  Called by every lane of the warp.
 template <int BITS, int R>
-__device__ __forceinline__ void value_rows(const uint4 (&x)[R], const int (&ti)[R], int bh, int t_begin,
+__device__ __forceinline__ void value_rows(const uint4 (&x)[R], const int (&ti)[R], int b, int h, int t_begin,
                                            int n_tokens, uint32_t* __restrict__ vcode,
                                            __half2* __restrict__ vsz, const int* __restrict__ table,
                                            const Dims& d) {
-  const int dv = d.dv, cpr = dv / 8, gl = d.gv / 8;
+  const int lcpr = __ffs(d.dv) - 4, lgl = __ffs(d.gv) - 4, lnvg = lcpr - lgl;
+  const int gl = 1 << lgl;
   const int lane = threadIdx.x & 31;
-  const int cc = lane % cpr;
-  const int lg = __ffs(d.gk) - 1;
-  {
-    // each row's group extremes as one half2 (min, -max), reduced over the group's lanes
-    // (aligned and consecutive)
-    __half2 ext[R];
+  const int cc = lane & ((1 << lcpr) - 1);
+  const int lgk = __ffs(d.gk) - 1;
+  // each row's group extremes as one half2 (min, -max), reduced over the group's lanes
+  // (aligned and consecutive)
+  __half2 ext[R];
 #pragma unroll
-    for (int i = 0; i < R; ++i) ext[i] = group_extremes(x[i], gl);
-    // (scale, zero) and 1/scale of the R rows: with groups of at least R lanes, lane j of a group
-    // derives row j's in one pass and the rows are broadcast; otherwise every lane derives its own
-    const int gsub = cc % gl, gbase = lane - gsub;
-    __half2 rsz[R];
-    float rrc[R];
-    if (gl >= R) {
-      __half2 e = ext[0];
+  for (int i = 0; i < R; ++i) ext[i] = group_extremes(x[i], gl);
+  // (scale, zero) and 1/scale of the R rows: with groups of at least R lanes, lane j of a group
+  // derives row j's in one pass and the rows are broadcast; otherwise every lane derives its own
+  const int gsub = cc & (gl - 1), gbase = lane - gsub, vg = cc >> lgl;
+  __half2 rsz[R];
+  float rrc[R];
+  if (gl >= R) {
+    __half2 e = ext[0];
 #pragma unroll
-      for (int i = 1; i < R; ++i)
-        if (gsub == i) e = ext[i];
-      const GroupParams gp = group_params<BITS>(__low2float(e), -__high2float(e));
-      const uint32_t sz = ptx_h2_as_u32(gp.sz);
-      const float rc = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        rsz[i] = ptx_u32_as_h2(__shfl_sync(0xffffffffu, sz, gbase + i));
-        rrc[i] = __shfl_sync(0xffffffffu, rc, gbase + i);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        const GroupParams gp = group_params<BITS>(__low2float(ext[i]), -__high2float(ext[i]));
-        rsz[i] = gp.sz;
-        rrc[i] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
-      }
-    }
+    for (int i = 1; i < R; ++i)
+      if (gsub == i) e = ext[i];
+    const GroupParams gp = group_params<BITS>(__low2float(e), -__high2float(e));
+    const uint32_t sz = ptx_h2_as_u32(gp.sz);
+    const float rc = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
 #pragma unroll
     for (int i = 0; i < R; ++i) {
-      if (ti[i] >= n_tokens) continue;
-      const float2 szf = __half22float2(rsz[i]);             // (scale, zero), exact
-      const int t = t_begin + ti[i];
-      const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t >> lg) + (t & (d.gk - 1));
-      if (gsub == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow * d.nvg) + cc / gl,
-                                     quant_rows(d) * d.nvg))
-        vsz[vrow * d.nvg + cc / gl] = rsz[i];
-      const uint64_t bits = pack_chunk<BITS, 0>(x[i], &szf.y, &rrc[i], &szf.x);
-      if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQValCode, static_cast<long long>(vrow * (dv * BITS / 8)) + cc * BITS, BITS,
-                               quant_rows(d) * d.vw * 4))
-        continue;
-      if constexpr (BITS == 2)
-        reinterpret_cast<uint16_t*>(vcode)[vrow * cpr + cc] = static_cast<uint16_t>(bits);
-      else if constexpr (BITS == 4)
-        vcode[vrow * cpr + cc] = static_cast<uint32_t>(bits);
-      else
-        reinterpret_cast<uint2*>(vcode)[vrow * cpr + cc] =
-            make_uint2(static_cast<uint32_t>(bits), static_cast<uint32_t>(bits >> 32));
+      rsz[i] = ptx_u32_as_h2(__shfl_sync(0xffffffffu, sz, gbase + i));
+      rrc[i] = __shfl_sync(0xffffffffu, rc, gbase + i);
     }
+  } else {
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const GroupParams gp = group_params<BITS>(__low2float(ext[i]), -__high2float(ext[i]));
+      rsz[i] = gp.sz;
+      rrc[i] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    if (ti[i] >= n_tokens) continue;
+    const float2 szf = __half22float2(rsz[i]);             // (scale, zero), exact
+    const int t = t_begin + ti[i];
+    const size_t vrow = group_row(d, table, b, h, t >> lgk) + (t & (d.gk - 1));
+    if (gsub == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow << lnvg) + vg,
+                                   quant_rows(d) * d.nvg))
+      vsz[(vrow << lnvg) + vg] = rsz[i];
+    const ChunkBits<BITS> bits = pack_chunk<BITS, 0>(x[i], &szf.y, &rrc[i], &szf.x);
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQValCode, static_cast<long long>(vrow * (d.dv * BITS / 8)) + cc * BITS, BITS,
+                             quant_rows(d) * d.vw * 4))
+      continue;
+    store_chunk<BITS>(vcode, (vrow << lcpr) + cc, bits);
   }
 }
 
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(256) quantize_values_kernel(
         x[i] = make_uint4(0, 0, 0, 0);
       }
     }
-    value_rows<BITS, R>(x, ti, bh, t_begin, n_tokens, vcode, vsz, table, d);
+    value_rows<BITS, R>(x, ti, bh / d.Hkv, bh % d.Hkv, t_begin, n_tokens, vcode, vsz, table, d);
   }
 }
 
@@ -568,7 +568,7 @@ __device__ __forceinline__ void drain_stages(StageRing* ring) {
 }
 
 template <int BITS, int R>
-__global__ void __launch_bounds__(256) quantize_keys_staged_kernel(
+__global__ void __launch_bounds__(256, 16 / R) quantize_keys_staged_kernel(
     const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
     uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
   extern __shared__ __align__(128) unsigned char sm_stage[];        // 2 x [gpc * gk][dk] fp16
@@ -621,15 +621,15 @@ __global__ void __launch_bounds__(256) quantize_keys_staged_kernel(
       ptx::fence_proxy_async_smem();
       issue(tile + 2LL * gridDim.x, st);
     }
-    const int bh = static_cast<int>(tile / tiles_per_row), g_first = static_cast<int>(tile % tiles_per_row) * gpc;
-    key_tile<BITS, R>(x, bh, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk);
+    const int t32 = static_cast<int>(tile), bh = t32 / tiles_per_row, g_first = (t32 - bh * tiles_per_row) * gpc;
+    key_tile<BITS, R>(x, bh / d.Hkv, bh % d.Hkv, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk);
     __syncthreads();                                                   // red, prm, blk are reused
   }
   drain_stages(&ring);
 }
 
 template <int BITS, int R>
-__global__ void __launch_bounds__(256) quantize_values_staged_kernel(
+__global__ void __launch_bounds__(256, 4) quantize_values_staged_kernel(
     const __half* __restrict__ src, int src_rows, int t_begin, int n_tokens,
     uint32_t* __restrict__ vcode, __half2* __restrict__ vsz, const int* __restrict__ table, Dims d) {
   extern __shared__ __align__(128) unsigned char sm_stage[];        // 2 x [tile rows][dv] fp16
@@ -669,7 +669,7 @@ __global__ void __launch_bounds__(256) quantize_values_staged_kernel(
     const int st = it & 1;
     const bool ok = ptx::mbar_wait_bounded(ptx::smem_addr(&ring.bars[st]), (it >> 1) & 1, kStageWaitNs);
     if (!__syncthreads_and(ok)) break;                                 // a wait gave up: stop
-    const int bh = static_cast<int>(tile / tiles_per_row), t0 = static_cast<int>(tile % tiles_per_row) * tile_rows;
+    const int t32 = static_cast<int>(tile), bh = t32 / tiles_per_row, t0 = (t32 - bh * tiles_per_row) * tile_rows;
     const uint4* stage = reinterpret_cast<const uint4*>(sm_stage + st * stage_bytes);
     uint4 x[R];
     int ti[R];
@@ -684,7 +684,7 @@ __global__ void __launch_bounds__(256) quantize_values_staged_kernel(
       ptx::fence_proxy_async_smem();
       issue(tile + 2LL * gridDim.x, st);
     }
-    value_rows<BITS, R>(x, ti, bh, t_begin, n_tokens, vcode, vsz, table, d);
+    value_rows<BITS, R>(x, ti, bh / d.Hkv, bh % d.Hkv, t_begin, n_tokens, vcode, vsz, table, d);
   }
   drain_stages(&ring);
 }
