@@ -243,6 +243,11 @@ int plan_counts(const kvq::Dims& d, int nG, int nF, int sm_count, int num_splits
                         : 0.0;
   const double bf = 2.0 * (d.dk + d.dv);
   const double cta_cost = 16384.0;
+  // In a launch of a single wave a CTA's fixed work (query prologue, first copies, merge and
+  // partial rows, its share of the combine) is not hidden behind other CTAs' streaming, so there
+  // a split gets at least kMinSplitBytes of cache to read (measured on 4k-token caches: 3 splits
+  // of 21 groups beat 6 of 11 and 9 of 7; multi-wave launches are left to the wave model).
+  const double kMinSplitBytes = 112.0 * 1024.0;
   auto best_split = [&](int n_units, double unit_bytes, int forced) {
     if (n_units <= 0) return 0;
     const int hi = std::min(n_units, cap);
@@ -257,6 +262,10 @@ int plan_counts(const kvq::Dims& d, int nG, int nF, int sm_count, int num_splits
         best_t = t;
         best = s;
       }
+    }
+    if (static_cast<long long>(rows) * best <= slots) {
+      const int by_size = static_cast<int>(std::max(1.0, floor(n_units * unit_bytes / kMinSplitBytes)));
+      best = std::min(best, by_size);
     }
     return best;
   };

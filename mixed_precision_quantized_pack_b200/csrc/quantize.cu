@@ -356,38 +356,51 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
     }
     __syncthreads();
   }
-  for (int idx = threadIdx.x; idx < gk * dk; idx += blockDim.x) {
-    const int t = idx / dk, c = idx % dk;
-    float x;
-    if constexpr (ROT) {
-      x = e[t * es + c];
-    } else {
-      const int row = (g * gk + t) % src_rows;
-      const long long si = static_cast<long long>((base + row) * dk) + c;
-      x = KVQ_IN_BOUNDS(d, kSiteSideSrc, si, static_cast<long long>(d.B) * hkv * src_rows * dk)
-              ? __half2float(src[si]) : 0.0f;
+  // the residual e of every token, one channel per thread (dk, the words per row and the
+  // (scale, zero) block's quarters are powers of two): the channel's (scale, zero), word and
+  // field are fixed for the thread, its tokens step by blockDim / dk
+  {
+    const int ldk = __ffs(dk) - 1, lper = __ffs(per) - 1;
+    const int c = threadIdx.x & (dk - 1);
+    const int tstep = blockDim.x >> ldk;
+    const int wd = c >> lper, r = c & (per - 1);
+    const int pos = quarter ? (wd & (quarter - 1)) * 4 + (wd >> (__ffs(quarter) - 1)) : wd;
+    const int slot = pos * 2 * per + (r & (half - 1)) * 2 + (r >> (__ffs(half) - 1));
+    const bool meta_ok = KVQ_RANGE_IN_BOUNDS(d, kSiteSideMeta, static_cast<long long>(gidx * 2 * dk) + slot, per + 1,
+                                             quant_groups(d) * 2 * dk);
+    const float sc = meta_ok ? __half2float(blk[slot]) : 0.0f;
+    const float zc = meta_ok ? __half2float(blk[slot + per]) : 0.0f;
+    const int shift = r * kb;
+    const uint32_t mask = (1u << kb) - 1u;
+    int t = threadIdx.x >> ldk;
+    int row = static_cast<int>((static_cast<long long>(g) * gk + t) % src_rows);   // source row of token t
+    for (; t < gk; t += tstep) {
+      float x;
+      if constexpr (ROT) {
+        x = e[t * es + c];
+      } else {
+        const long long si = static_cast<long long>((base + row) * dk) + c;
+        x = KVQ_IN_BOUNDS(d, kSiteSideSrc, si, static_cast<long long>(d.B) * hkv * src_rows * dk)
+                ? __half2float(src[si]) : 0.0f;
+      }
+      const long long ki = static_cast<long long>((row0 + t) * words) + wd;
+      const uint32_t w = KVQ_IN_BOUNDS(d, kSiteSideCode, ki, quant_rows(d) * words) ? kcode[ki] : 0u;
+      const uint32_t code = (w >> shift) & mask;
+      const float kh = __fadd_rn(__fmul_rn(static_cast<float>(code), sc), zc);
+      e[t * es + c] = __fsub_rn(x, kh);
+      row += tstep;
+      while (row >= src_rows) row -= src_rows;
     }
-    const long long ki = static_cast<long long>((row0 + t) * words) + c / per;
-    const uint32_t w = KVQ_IN_BOUNDS(d, kSiteSideCode, ki, quant_rows(d) * words) ? kcode[ki] : 0u;
-    const uint32_t code = (w >> ((c % per) * kb)) & ((1u << kb) - 1u);
-    // the channel's (scale, zero) slots in the group's paired, quarter-interleaved block
-    const int wd = c / per, r = c % per;
-    const int pos = quarter ? (wd % quarter) * 4 + wd / quarter : wd;
-    const int slot = pos * 2 * per + (r % half) * 2 + r / half;
-    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteSideMeta, static_cast<long long>(gidx * 2 * dk) + slot, per + 1,
-                             quant_groups(d) * 2 * dk))
-      continue;
-    const float kh = __fadd_rn(__fmul_rn(static_cast<float>(code), __half2float(blk[slot])),
-                               __half2float(blk[slot + per]));
-    e[t * es + c] = __fsub_rn(x, kh);
   }
   for (int idx = threadIdx.x; idx < dk * sr; idx += blockDim.x)
     u[idx] = KVQ_IN_BOUNDS(d, kSiteSideU, static_cast<long long>(h) * dk * sr + idx, static_cast<long long>(hkv) * dk * sr)
                  ? side_u[static_cast<size_t>(h) * dk * sr + idx] : 0.0f;
   __syncthreads();
+  const int lsr = __ffs(sr) - 1;
   for (int idx = threadIdx.x; idx < gk * sr; idx += blockDim.x) {
-    const int t = idx / sr, i = idx % sr;
+    const int t = idx >> lsr, i = idx & (sr - 1);
     float acc = 0.0f;
+#pragma unroll 8
     for (int c = 0; c < dk; ++c) acc = __fadd_rn(acc, __fmul_rn(e[t * es + c], u[c * sr + i]));
     y[idx] = acc;
   }
@@ -567,7 +580,7 @@ __device__ __forceinline__ void drain_stages(StageRing* ring) {
   __syncthreads();
 }
 
-template <int BITS, int R>
+template <int BITS, int R, bool ROT>
 __global__ void __launch_bounds__(256, 16 / R) quantize_keys_staged_kernel(
     const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
     uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
@@ -612,6 +625,22 @@ __global__ void __launch_bounds__(256, 16 / R) quantize_keys_staged_kernel(
     const int st = it & 1;
     const bool ok = ptx::mbar_wait_bounded(ptx::smem_addr(&ring.bars[st]), (it >> 1) & 1, kStageWaitNs);
     if (!__syncthreads_and(ok)) break;                                 // a wait gave up: stop
+    if constexpr (ROT) {
+      // key-only rotation: each warp rotates rows of the stage in place (fp32 butterflies, one
+      // rounding to fp16), before any thread reads its chunks
+      __half* rows = reinterpret_cast<__half*>(sm_stage + st * stage_bytes);
+      const int lane = tid & 31, warp = tid >> 5;
+      for (int rr = warp; rr < gpc * gk; rr += 8) {
+        float v[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) v[m] = m < dk / 32 ? __half2float(rows[rr * dk + lane + 32 * m]) : 0.0f;
+        rotate_row_warp<8>(v, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          if (m < dk / 32) rows[rr * dk + lane + 32 * m] = __float2half_rn(v[m]);
+      }
+      __syncthreads();
+    }
     const uint4* stage = reinterpret_cast<const uint4*>(sm_stage + st * stage_bytes);
     uint4 x[R];
 #pragma unroll
@@ -1095,10 +1124,11 @@ cudaError_t launch_quantize_keys_t(const Dims& d, const __half* src, int src_row
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  if (!ROT && static_cast<long long>(g_begin + n_groups) * d.gk <= src_rows) {
-    // a contiguous source (prefill): the persistent staged kernel
-    auto staged = rows == 4 ? quantize_keys_staged_kernel<BITS, 4>
-                : rows == 8 ? quantize_keys_staged_kernel<BITS, 8> : quantize_keys_staged_kernel<BITS, 16>;
+  if (static_cast<long long>(g_begin + n_groups) * d.gk <= src_rows) {
+    // a contiguous source (prefill): the persistent staged kernel (rotating the staged rows in
+    // place when the keys are rotated)
+    auto staged = rows == 4 ? quantize_keys_staged_kernel<BITS, 4, ROT>
+                : rows == 8 ? quantize_keys_staged_kernel<BITS, 8, ROT> : quantize_keys_staged_kernel<BITS, 16, ROT>;
     const int sbytes = 2 * gpc * d.gk * d.dk * 2;
     // static + dynamic shared memory above 48 KB needs the opt-in (set on every launch: it is a
     // property of the current device's context)

@@ -140,6 +140,17 @@ WORKLOADS: Dict[str, Workload] = {
                       n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=4, v_bits=2,
                       group_k=64, group_v=64, window=128, log_retain=1, appends=0, seed=1007,
                       paged=1),
+    # a second width map at 32k: keys 32 x 8 and 96 x 2 bits (3.5 on average), values in
+    # groups of 64 channels at 4 and 2 bits (3)
+    "aatc32k-k8k2": _base(name="aatc-b32-32/8-32k-k8x32-k2x96-v4x64-v2x64-logretain", batch=32,
+                          n_q_heads=32, n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=0,
+                          v_bits=0, group_k=64, group_v=64, window=128, log_retain=1, appends=0,
+                          seed=1009, k_widths=(8,) * 32 + (2,) * 96, v_widths=(4,) * 64 + (2,) * 64),
+    # the HeadQ case on a paged cache
+    "headq-paged32k": _base(name="headq-paged-b32-32/8-32k-k2v2-r4q4-logretain", batch=32,
+                            n_q_heads=32, n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=2,
+                            v_bits=2, group_k=64, group_v=64, window=128, log_retain=1, appends=0,
+                            seed=1010, side_rank=4, side_bits=4, q_in_basis=0.9, paged=1),
 }
 
 SWEEP_BATCHES = (1, 8, 32, 64)

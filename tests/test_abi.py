@@ -325,8 +325,10 @@ def test_width_maps_do_not_combine_with_other_modes(bad):
     ([0] * 128, [0] * 128, 64, 1),                           # everything dropped: 1-word rows
     ([1] * 128, [8] * 8 + [1] * 120, 8, 0),                  # value groups below 16 channels
     ([8] * 128, [4] * 128, 128, 1),
-    ([8] * 12 + [4] * 116, [2] * 128, 32, 0),                # 12 x 8 bits: a word mixes widths
-    ([4] * 128, [1] * 128, 16, 0),                           # 1-bit value groups of 16
+    ([8] * 12 + [4] * 116, [2] * 128, 32, 0),                # 3 + 28 + 2 = 33 couples > 32
+    ([8] * 14 + [4] * 84 + [0] * 30, [2] * 128, 32, 1),      # word 3 mixes widths: 25 couples
+    ([4] * 128, [1] * 128, 16, 1),                           # 1-bit value groups of 16
+    ([4] * 128, [1] * 128, 8, 0),                            # value groups of 8
 ])
 def test_width_map_sizes_match_the_oracle_layout(kw_, vw_, gv, fast):
     c = var(k_widths=kw_, v_widths=vw_, group_v=gv)

@@ -564,6 +564,11 @@ def test_full_size_paged_32k():
     sampled_full_size(W.WORKLOADS["paged32k"], rows=(0, 31))
 
 
+def test_full_size_headq_paged_32k():
+    assert tensor_kernel_built(W.WORKLOADS["headq-paged32k"])
+    sampled_full_size(W.WORKLOADS["headq-paged32k"], rows=(0, 31))
+
+
 def test_page_pool_exhaustion_changes_nothing():
     need_gpu()
     w = W.WORKLOADS["gqa4k"].with_(batch=2, context=600, appends=80, seed=291, paged=1)
@@ -636,6 +641,9 @@ def test_page_pool_exhaustion_changes_nothing():
     dict(k_widths=(8,) * 128, v_widths=(8,) * 128, group_v=128, log_retain=0),
     dict(n_q_heads=8, n_kv_heads=8, group_k=16),                               # tensor cores, GQA 1
     dict(group_k=128, group_v=16, v_widths=(8,) * 16 + (4,) * 32 + (2,) * 80),  # tensor cores
+    # a key word holding 8- and 4-bit fields; 1-bit value groups of 16 (two-bit runs)
+    dict(group_v=16, k_widths=(8,) * 14 + (4,) * 84 + (0,) * 30, v_widths=(4,) * 16 + (2,) * 32 + (1,) * 80),
+    dict(group_v=64, k_widths=(8,) * 32 + (2,) * 96, v_widths=(4,) * 64 + (2,) * 64),
 ])
 def test_width_maps(shape):
     w = AATC.with_(batch=2, context=1500, appends=70, seed=301 + len(str(shape)), **shape)
@@ -643,13 +651,15 @@ def test_width_maps(shape):
 
 
 def test_width_map_kernel_choice():
-    """The tensor-core kernel serves maps whose width classes fill whole words (d 128, value
-    groups >= 16); the others run on the generic kernel."""
+    """The tensor-core kernel serves d 128 maps with value groups of 16-128 channels whose key
+    fields fit in 32 couples; the others run on the generic kernel."""
     assert tensor_kernel_built(AATC)
     assert tensor_kernel_built(AATC.with_(n_q_heads=8, n_kv_heads=8))
+    assert tensor_kernel_built(AATC.with_(group_v=16, k_widths=(8,) * 14 + (4,) * 84 + (0,) * 30,
+                                          v_widths=(4,) * 16 + (2,) * 32 + (1,) * 80))
     assert not tensor_kernel_built(AATC.with_(d_k=64, k_widths=(4,) * 64))
     assert not tensor_kernel_built(AATC.with_(group_v=8))
-    assert not tensor_kernel_built(AATC.with_(k_widths=(8,) * 12 + (4,) * 116))
+    assert not tensor_kernel_built(AATC.with_(k_widths=(8,) * 12 + (4,) * 116))   # 33 couples
 
 
 def test_width_maps_ragged_batch():
@@ -663,3 +673,8 @@ def test_width_maps_paged():
 
 def test_full_size_aatc_32k():
     sampled_full_size(AATC, rows=(0, 31))
+
+
+def test_full_size_aatc_32k_second_map():
+    assert tensor_kernel_built(W.WORKLOADS["aatc32k-k8k2"])
+    sampled_full_size(W.WORKLOADS["aatc32k-k8k2"], rows=(0, 31))
