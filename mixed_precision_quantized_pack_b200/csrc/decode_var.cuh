@@ -556,10 +556,12 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarPlan plan, const __half
             const uint32_t bp1 = ptx::movmatrix_trans(ptx::split_hi_lo_trunc(p1 * f1.x));
             const int bit0 = MAP::kFixed ? MAP::vbit0(gg, GV) : plan.vbit0[gg];
             float(*cg)[4] = co + gg * MPG;
-            if (vb == 8) value_group<8, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg);
-            else if (vb == 4) value_group<4, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg);
-            else if (vb == 2) value_group<2, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg);
-            else value_group<1, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg);
+            switch (vb) {
+              case 8: value_group<8, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg); break;
+              case 4: value_group<4, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg); break;
+              case 2: value_group<2, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg); break;
+              default: value_group<1, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, cg); break;
+            }
           }
         }
       }
