@@ -580,6 +580,31 @@ __device__ __forceinline__ void drain_stages(StageRing* ring) {
   __syncthreads();
 }
 
+// Rotates n rows of 32 * M fp16 channels in shared memory in place (a warp per row, two rows at
+// a time so that the butterfly chains of the two interleave), as rotate_row_warp then one
+// rounding to fp16.
+template <int M>
+__device__ __forceinline__ void rotate_stage_rows(__half* rows, int n, const Dims& d) {
+  constexpr int dk = 32 * M;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r0 = 2 * warp; r0 < n; r0 += 16) {
+    const bool two = r0 + 1 < n;
+    float a[M], b[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      a[m] = __half2float(rows[r0 * dk + lane + 32 * m]);
+      b[m] = two ? __half2float(rows[(r0 + 1) * dk + lane + 32 * m]) : 0.0f;
+    }
+    rotate_row_warp<M>(a, M, d.rot_signs, d.rot_inv_ck, lane);
+    rotate_row_warp<M>(b, M, d.rot_signs, d.rot_inv_ck, lane);
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      rows[r0 * dk + lane + 32 * m] = __float2half_rn(a[m]);
+      if (two) rows[(r0 + 1) * dk + lane + 32 * m] = __float2half_rn(b[m]);
+    }
+  }
+}
+
 template <int BITS, int R, bool ROT>
 __global__ void __launch_bounds__(256, 16 / R) quantize_keys_staged_kernel(
     const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
@@ -629,15 +654,11 @@ __global__ void __launch_bounds__(256, 16 / R) quantize_keys_staged_kernel(
       // key-only rotation: each warp rotates rows of the stage in place (fp32 butterflies, one
       // rounding to fp16), before any thread reads its chunks
       __half* rows = reinterpret_cast<__half*>(sm_stage + st * stage_bytes);
-      const int lane = tid & 31, warp = tid >> 5;
-      for (int rr = warp; rr < gpc * gk; rr += 8) {
-        float v[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) v[m] = m < dk / 32 ? __half2float(rows[rr * dk + lane + 32 * m]) : 0.0f;
-        rotate_row_warp<8>(v, dk / 32, d.rot_signs, d.rot_inv_ck, lane);
-#pragma unroll
-        for (int m = 0; m < 8; ++m)
-          if (m < dk / 32) rows[rr * dk + lane + 32 * m] = __float2half_rn(v[m]);
+      switch (dk) {
+        case 32: rotate_stage_rows<1>(rows, gpc * gk, d); break;
+        case 64: rotate_stage_rows<2>(rows, gpc * gk, d); break;
+        case 128: rotate_stage_rows<4>(rows, gpc * gk, d); break;
+        default: rotate_stage_rows<8>(rows, gpc * gk, d); break;
       }
       __syncthreads();
     }
@@ -764,34 +785,23 @@ __device__ __forceinline__ void or_into_row(uint32_t* row, int off, uint64_t bit
 // c quantized with its own width; the codes are ORed into the CTA's rows in shared memory
 // ([gpc * gk][kw] words), which are then written out whole.  (scale, zero) are stored plainly,
 // [dk][2] per group; a dropped channel stores (0, 0).
+// The part of the width-map key quantizer after a tile's chunks are in registers (the layout of
+// key_tile; sm_rows: [gpc * gk][kw] words of the CTA's rows, zeroed here).  Called by every thread
+// of the CTA (barriers).
 template <int R>
-__global__ void __launch_bounds__(256) quantize_keys_var_kernel(
-    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
-    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
-  extern __shared__ __align__(16) uint32_t sm_rows[];               // [gpc * gk][kw]
-  __shared__ __align__(16) __half2 red[2][256][4];
-  __shared__ __align__(16) float prm[3][kKeyPrm];
-  __shared__ __align__(16) __half2 blk[kKeyPrm];
+__device__ __forceinline__ void key_tile_var(const uint4 (&x)[R], int b, int h, int g_begin, int g_first,
+                                             int n_groups, uint32_t* __restrict__ kcode, __half2* __restrict__ ksz,
+                                             const int* __restrict__ table, const Dims& d,
+                                             __half2 (*red)[256][4], float (*prm)[kKeyPrm], __half2* blk,
+                                             uint32_t* sm_rows, const int (&w)[8], const int (&o)[8]) {
   const int dk = d.dk, gk = d.gk, kw = d.kw;
-  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int ldk = __ffs(dk) - 1, lcpr = ldk - 3, lslabs = __ffs(gk) - 1 - ilog2c(R);
+  const int ltpg = lcpr + lslabs, slabs = 1 << lslabs, tpg = 1 << ltpg, gpc = 256 >> ltpg;
+  const int cpr = 1 << lcpr;
   const int tid = threadIdx.x;
-  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt / cpr;
-  const int bh = blockIdx.y, b = bh / d.Hkv, h = bh % d.Hkv;
-  const int g_first = blockIdx.x * gpc;
+  const int gi = tid >> ltpg, lt = tid & (tpg - 1), cc = lt & (cpr - 1), rs = lt >> lcpr;
   const bool active = g_first + gi < n_groups;
-  const int g = g_begin + g_first + gi;
-  const size_t base = static_cast<size_t>(bh) * src_rows;
   for (int i = tid; i < gpc * gk * kw; i += 256) sm_rows[i] = 0u;
-  uint4 x[R];
-#pragma unroll
-  for (int i = 0; i < R; ++i) {
-    const int tk = g * gk + rs + slabs * i;
-    const int row = tk < src_rows ? tk : tk % src_rows;              // the window is a ring
-    const long long si = static_cast<long long>((base + row) * dk) + 8 * cc;
-    x[i] = active && KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dk)
-               ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
-               : make_uint4(0, 0, 0, 0);
-  }
   {
     const __half2* h0 = reinterpret_cast<const __half2*>(&x[0]);
     __half2 mn[4], mx[4];
@@ -813,13 +823,13 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
     }
   }
   __syncthreads();
-  for (int p = tid; p < gpc * dk / 2; p += 256) {
-    const int g2 = p / (dk / 2), pp = p % (dk / 2), c2 = pp / 4, k = pp % 4;
-    const int t0 = g2 * tpg + c2;
+  for (int p = tid; p < (gpc << (ldk - 1)); p += 256) {
+    const int g2 = p >> (ldk - 1), pp = p & ((dk >> 1) - 1), c2 = pp >> 2, k = pp & 3;
+    const int t0 = (g2 << ltpg) + c2;
     __half2 mn = red[0][t0][k], mx = red[1][t0][k];
     for (int sl = 1; sl < slabs; ++sl) {
-      mn = __hmin2(mn, red[0][t0 + sl * cpr][k]);
-      mx = __hmax2(mx, red[1][t0 + sl * cpr][k]);
+      mn = __hmin2(mn, red[0][t0 + (sl << lcpr)][k]);
+      mx = __hmax2(mx, red[1][t0 + (sl << lcpr)][k]);
     }
     const float2 fmn = __half22float2(mn), fmx = __half22float2(mx);
 #pragma unroll
@@ -831,15 +841,15 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
       gp.scale = gp.zero = 0.0f;
       gp.sz = __floats2half2_rn(0.0f, 0.0f);
       if (width) gp = group_params_b(e ? fmn.y : fmn.x, e ? fmx.y : fmx.x, width);
-      prm[0][g2 * dk + c] = gp.zero;
-      prm[1][g2 * dk + c] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
-      prm[2][g2 * dk + c] = gp.scale;
-      blk[g2 * dk + c] = gp.sz;
+      prm[0][(g2 << ldk) + c] = gp.zero;
+      prm[1][(g2 << ldk) + c] = gp.scale == 0.0f ? 0.0f : __frcp_rn(gp.scale);
+      prm[2][(g2 << ldk) + c] = gp.scale;
+      blk[(g2 << ldk) + c] = gp.sz;
     }
   }
   __syncthreads();
-  for (int i = tid; i < gpc * dk / 4; i += 256) {                 // 16 B of (scale, zero) per thread
-    const int g2 = i / (dk / 4), j = i % (dk / 4);
+  for (int i = tid; i < (gpc << (ldk - 2)); i += 256) {           // 16 B of (scale, zero) per thread
+    const int g2 = i >> (ldk - 2), j = i & ((dk >> 2) - 1);
     if (g_first + g2 >= n_groups) continue;
     const size_t gidx = group_index(d, table, b, h, g_begin + g_first + g2);
     if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeyMeta, static_cast<long long>(gidx * dk) + 4 * j, 4, quant_groups(d) * dk))
@@ -848,13 +858,11 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
   }
   if (active) {
     float z[8], r[8], sc[8];
-    int w[8], o[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      z[j] = prm[0][gi * dk + 8 * cc + j];
-      r[j] = prm[1][gi * dk + 8 * cc + j];
-      sc[j] = prm[2][gi * dk + 8 * cc + j];
-      channel_width(d.kcnt, 8 * cc + j, &w[j], &o[j]);
+      z[j] = prm[0][(gi << ldk) + 8 * cc + j];
+      r[j] = prm[1][(gi << ldk) + 8 * cc + j];
+      sc[j] = prm[2][(gi << ldk) + 8 * cc + j];
     }
     if (w[0]) {
 #pragma unroll
@@ -863,12 +871,120 @@ __global__ void __launch_bounds__(256) quantize_keys_var_kernel(
     }
   }
   __syncthreads();
-  for (int i = tid; i < gpc * gk * kw; i += 256) {
-    const int g2 = i / (gk * kw);
-    if (g_first + g2 >= n_groups) continue;
-    const long long ki = static_cast<long long>(group_row(d, table, b, h, g_begin + g_first + g2) * kw) + i % (gk * kw);
-    if (KVQ_IN_BOUNDS(d, kSiteQKeyCode, ki, quant_rows(d) * kw)) kcode[ki] = sm_rows[i];
+  // the packed rows out: a group's gk rows are contiguous in the cache
+  for (int g2 = 0; g2 < gpc && g_first + g2 < n_groups; ++g2) {
+    const long long k0 = static_cast<long long>(group_row(d, table, b, h, g_begin + g_first + g2) * kw);
+    const uint32_t* src_rows_sm = sm_rows + g2 * gk * kw;
+    for (int j = tid; j < gk * kw; j += 256)
+      if (KVQ_IN_BOUNDS(d, kSiteQKeyCode, k0 + j, quant_rows(d) * kw)) kcode[k0 + j] = src_rows_sm[j];
   }
+}
+
+// The widths and row bit offsets of the 8 channels of chunk cc (0 and the row's end for dropped
+// channels).
+__device__ __forceinline__ void chunk_widths(const Dims& d, int cc, int (&w)[8], int (&o)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) channel_width(d.kcnt, 8 * cc + j, &w[j], &o[j]);
+}
+
+template <int R>
+__global__ void __launch_bounds__(256) quantize_keys_var_kernel(
+    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
+    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
+  extern __shared__ __align__(16) uint32_t sm_rows[];               // [gpc * gk][kw]
+  __shared__ __align__(16) __half2 red[2][256][4];
+  __shared__ __align__(16) float prm[3][kKeyPrm];
+  __shared__ __align__(16) __half2 blk[kKeyPrm];
+  const int dk = d.dk, gk = d.gk;
+  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int tid = threadIdx.x;
+  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt / cpr;
+  const int bh = blockIdx.y;
+  const int g_first = blockIdx.x * gpc;
+  const bool active = g_first + gi < n_groups;
+  const int g = g_begin + g_first + gi;
+  const size_t base = static_cast<size_t>(bh) * src_rows;
+  uint4 x[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int tk = g * gk + rs + slabs * i;
+    const int row = tk < src_rows ? tk : tk % src_rows;              // the window is a ring
+    const long long si = static_cast<long long>((base + row) * dk) + 8 * cc;
+    x[i] = active && KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, si, 8, static_cast<long long>(d.B) * d.Hkv * src_rows * dk)
+               ? __ldg(reinterpret_cast<const uint4*>(src + (base + row) * dk) + cc)
+               : make_uint4(0, 0, 0, 0);
+  }
+  int w[8], o[8];
+  chunk_widths(d, cc, w, o);
+  key_tile_var<R>(x, bh / d.Hkv, bh % d.Hkv, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk, sm_rows,
+                  w, o);
+}
+
+// The width-map key quantizer for a contiguous source (prefill): the persistent staged form of
+// quantize_keys_var_kernel (two stages of raw rows by bulk copies, as quantize_keys_staged_kernel),
+// the CTA's packed rows after the stages in dynamic shared memory.
+template <int R>
+__global__ void __launch_bounds__(256, R == 4 ? 3 : 2) quantize_keys_var_staged_kernel(
+    const __half* __restrict__ src, int src_rows, int g_begin, int n_groups,
+    uint32_t* __restrict__ kcode, __half2* __restrict__ ksz, const int* __restrict__ table, Dims d) {
+  extern __shared__ __align__(128) unsigned char sm_stage[];        // 2 x [gpc * gk][dk] fp16, rows
+  __shared__ __align__(16) __half2 red[2][256][4];
+  __shared__ __align__(16) float prm[3][kKeyPrm];
+  __shared__ __align__(16) __half2 blk[kKeyPrm];
+  __shared__ __align__(8) StageRing ring;
+  const int dk = d.dk, gk = d.gk;
+  const int cpr = dk / 8, slabs = gk / R, tpg = cpr * slabs, gpc = 256 / tpg;
+  const int tid = threadIdx.x;
+  const int gi = tid / tpg, lt = tid % tpg, cc = lt % cpr, rs = lt / cpr;
+  const int tiles_per_row = (n_groups + gpc - 1) / gpc;
+  const long long n_tiles = static_cast<long long>(d.B) * d.Hkv * tiles_per_row;
+  const int stage_bytes = gpc * gk * dk * 2;
+  uint32_t* sm_rows = reinterpret_cast<uint32_t*>(sm_stage + 2 * stage_bytes);
+  const uint32_t st0 = ptx::smem_addr(sm_stage);
+  int w[8], o[8];
+  chunk_widths(d, cc, w, o);
+  [[maybe_unused]] const long long src_ext = static_cast<long long>(d.B) * d.Hkv * src_rows * dk;
+  auto issue = [&](long long tile, int st) {
+    const int bh = static_cast<int>(tile / tiles_per_row), g_first = static_cast<int>(tile % tiles_per_row) * gpc;
+    const int ng = min(gpc, n_groups - g_first);
+    long long first = (static_cast<long long>(bh) * src_rows + static_cast<long long>(g_begin + g_first) * gk) * dk;
+    const uint32_t bytes = static_cast<uint32_t>(ng) * gk * dk * 2;
+    if (!KVQ_RANGE_IN_BOUNDS(d, kSiteQKeySrc, first, static_cast<long long>(ng) * gk * dk, src_ext)) first = 0;
+    ring.issued[st] += 1;
+    ptx::mbar_arrive_expect_tx(ptx::smem_addr(&ring.bars[st]), bytes);
+    ptx::bulk_g2s(st0 + st * stage_bytes, src + first, bytes, ptx::smem_addr(&ring.bars[st]));
+  };
+  if (tid == 0) {
+    for (int st = 0; st < 2; ++st) {
+      ptx::mbar_init(ptx::smem_addr(&ring.bars[st]), 1);
+      ring.issued[st] = 0;
+    }
+    ptx::fence_barrier_init();
+    for (int k = 0; k < 2; ++k)
+      if (blockIdx.x + static_cast<long long>(k) * gridDim.x < n_tiles) issue(blockIdx.x + static_cast<long long>(k) * gridDim.x, k);
+  }
+  __syncthreads();
+  for (int it = 0;; ++it) {
+    const long long tile = blockIdx.x + static_cast<long long>(it) * gridDim.x;
+    if (tile >= n_tiles) break;
+    const int st = it & 1;
+    const bool ok = ptx::mbar_wait_bounded(ptx::smem_addr(&ring.bars[st]), (it >> 1) & 1, kStageWaitNs);
+    if (!__syncthreads_and(ok)) break;                                 // a wait gave up: stop
+    const uint4* stage = reinterpret_cast<const uint4*>(sm_stage + st * stage_bytes);
+    uint4 x[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) x[i] = stage[(gi * gk + rs + slabs * i) * cpr + cc];
+    __syncthreads();                                                   // the stage may be refilled
+    if (tid == 0 && tile + 2LL * gridDim.x < n_tiles) {
+      ptx::fence_proxy_async_smem();
+      issue(tile + 2LL * gridDim.x, st);
+    }
+    const int t32 = static_cast<int>(tile), bh = t32 / tiles_per_row, g_first = (t32 - bh * tiles_per_row) * gpc;
+    key_tile_var<R>(x, bh / d.Hkv, bh % d.Hkv, g_begin, g_first, n_groups, kcode, ksz, table, d, red, prm, blk,
+                    sm_rows, w, o);
+    __syncthreads();                                                   // red, prm, blk, rows are reused
+  }
+  drain_stages(&ring);
 }
 
 // Value quantize-pack with per-group widths: the fixed-width value kernel's tiling (a lane per
@@ -909,15 +1025,41 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
         x[i] = make_uint4(0, 0, 0, 0);
       }
     }
+    // (scale, zero) of the R rows: with groups of at least R lanes, lane j of a group derives row
+    // j's and the rows are broadcast; otherwise every lane derives its own
+    __half2 ext[R];
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const __half2 e = group_extremes(x[i], gl);
-      const float mn = __low2float(e), mx = -__high2float(e);
-      if (ti[i] >= n_tokens) continue;
+    for (int i = 0; i < R; ++i) ext[i] = group_extremes(x[i], gl);
+    const int gsub = cc % gl, gbase = lane - gsub;
+    GroupParams rgp[R];
+    if (gl >= R) {
+      __half2 e = ext[0];
+#pragma unroll
+      for (int i = 1; i < R; ++i)
+        if (gsub == i) e = ext[i];
       GroupParams gp;
       gp.scale = gp.zero = 0.0f;
       gp.sz = __floats2half2_rn(0.0f, 0.0f);
-      if (width) gp = group_params_b(mn, mx, width);
+      if (width) gp = group_params_b(__low2float(e), -__high2float(e), width);
+      const uint32_t sz = ptx_h2_as_u32(gp.sz);
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        rgp[i].sz = ptx_u32_as_h2(__shfl_sync(0xffffffffu, sz, gbase + i));
+        rgp[i].scale = __low2float(rgp[i].sz);
+        rgp[i].zero = __high2float(rgp[i].sz);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        rgp[i].scale = rgp[i].zero = 0.0f;
+        rgp[i].sz = __floats2half2_rn(0.0f, 0.0f);
+        if (width) rgp[i] = group_params_b(__low2float(ext[i]), -__high2float(ext[i]), width);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      if (ti[i] >= n_tokens) continue;
+      const GroupParams gp = rgp[i];
       const int t = t_begin + ti[i];
       const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t >> lg) + (t & (d.gk - 1));
       if (cc % gl == 0 && KVQ_IN_BOUNDS(d, kSiteQValMeta, static_cast<long long>(vrow * d.nvg) + cc / gl,
@@ -946,13 +1088,14 @@ __global__ void __launch_bounds__(256) quantize_values_var_kernel(
       or_into_row(rows_sm + (rsub + rpw * i) * vw, offset, bits);
     }
     __syncwarp();
-    for (int k = lane; k < block_rows * vw; k += 32) {
-      const int tl = t_first + k / vw;
-      if (tl >= n_tokens) continue;
-      const int t = t_begin + tl;
+    // the warp's rows out, row by row (a row's words are consecutive in the cache)
+    for (int rr = 0; rr < block_rows && t_first + rr < n_tokens; ++rr) {
+      const int t = t_begin + t_first + rr;
       const size_t vrow = group_row(d, table, bh / d.Hkv, bh % d.Hkv, t >> lg) + (t & (d.gk - 1));
-      const long long vi = static_cast<long long>(vrow * vw) + k % vw;
-      if (KVQ_IN_BOUNDS(d, kSiteQValCode, vi, quant_rows(d) * vw)) vcode[vi] = rows_sm[k];
+      for (int j = lane; j < vw; j += 32) {
+        const long long vi = static_cast<long long>(vrow * vw) + j;
+        if (KVQ_IN_BOUNDS(d, kSiteQValCode, vi, quant_rows(d) * vw)) vcode[vi] = rows_sm[rr * vw + j];
+      }
     }
     __syncwarp();
   }
@@ -1170,6 +1313,20 @@ cudaError_t launch_quantize_keys(const Dims& d, const __half* src, int src_rows,
     auto kern = rows == 4 ? quantize_keys_var_kernel<4>
               : rows == 8 ? quantize_keys_var_kernel<8> : quantize_keys_var_kernel<16>;
     if (rows > 16 || gpc * d.dk > kKeyPrm) return cudaErrorInvalidValue;
+    if (static_cast<long long>(g_begin + n_groups) * d.gk <= src_rows) {
+      // a contiguous source (prefill): the persistent staged kernel, three CTAs per SM (two when
+      // a thread holds more than four rows)
+      auto staged = rows == 4 ? quantize_keys_var_staged_kernel<4>
+                  : rows == 8 ? quantize_keys_var_staged_kernel<8> : quantize_keys_var_staged_kernel<16>;
+      const int sbytes = 2 * gpc * d.gk * d.dk * 2 + smem;
+      const cudaError_t e = cudaFuncSetAttribute(staged, cudaFuncAttributeMaxDynamicSharedMemorySize, sbytes);
+      if (e != cudaSuccess) return e;
+      const long long tiles = static_cast<long long>(d.B) * d.Hkv * ((n_groups + gpc - 1) / gpc);
+      const long long slots = static_cast<long long>(d.sm_count > 0 ? d.sm_count : 148) * (rows == 4 ? 3 : 2);
+      staged<<<static_cast<int>(tiles < slots ? tiles : slots), 256, sbytes, s>>>(src, src_rows, g_begin, n_groups,
+                                                                                 kcode, ksz, table, d);
+      return cudaGetLastError();
+    }
     if (smem > 48 * 1024) {
       const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
