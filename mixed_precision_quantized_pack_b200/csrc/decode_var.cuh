@@ -227,6 +227,27 @@ constexpr int ctas_per_sm() { return kCtasPerSm; }
 template <class MAP>
 constexpr int smem_per_cta() { return 233472 / ctas_per_sm<MAP>() - 1024; }
 
+// p.V of one value group of width B over the MT tiles of a key group: per tile the (scale, zero)
+// of the lane's two tokens, the B operand p_t s_{t,g} split (hi, lo) and transposed, and the
+// group's MMAs; zsum accumulates sum_t p_t z_{t,g}.
+template <int B, int GV, int MT, int NVG>
+__device__ __forceinline__ void value_group_tiles(const uint32_t* svc, const uint32_t* svm, int vw, int gg, int qi,
+                                                  int qr, bool swap, uint32_t sel_lo, uint32_t sel_hi, int bit0,
+                                                  const float (&pw)[MT][2], float& zsum, float (*c)[4]) {
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int t0 = 16 * mt + qr;
+    const float2 f0 = __half22float2(ptx::u32_as_h2(svm[t0 * NVG + gg]));
+    const float2 f1 = __half22float2(ptx::u32_as_h2(svm[(t0 + 8) * NVG + gg]));
+    zsum = fmaf(pw[mt][0], f0.y, fmaf(pw[mt][1], f1.y, zsum));
+    const uint32_t bp0 = ptx::movmatrix_trans(ptx::split_hi_lo_trunc(pw[mt][0] * f0.x));
+    const uint32_t bp1 = ptx::movmatrix_trans(ptx::split_hi_lo_trunc(pw[mt][1] * f1.x));
+    const int ta = 16 * mt + 2 * qi + (swap ? 1 : 0);
+    const int tb = 16 * mt + 2 * qi + (swap ? 0 : 1);
+    value_group<B, GV>(svc, vw, ta, tb, qr, swap, sel_lo, sel_hi, bit0, bp0, bp1, c);
+  }
+}
+
 template <int NREP, int GV, int GK, class MAP = RuntimeMap>
 __global__ void __launch_bounds__(kThreads, ctas_per_sm<MAP>())
 decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarPlan plan, const __half* __restrict__ q,
@@ -532,6 +553,29 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarPlan plan, const __half
       // ---- p.V over the group ----
       const uint32_t* svc = reinterpret_cast<const uint32_t*>(S + L.v_off);
       const uint32_t* svm = reinterpret_cast<const uint32_t*>(S + L.vmeta_off);
+      if constexpr (!MAP::kFixed) {
+        // a run-time map: one branch on each group's width per key group (not per tile), the
+        // group's tiles inside
+        float pw[MT][2];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          pw[mt][0] = ptx::ex2(sc[mt][0] - m_use);
+          pw[mt][1] = ptx::ex2(sc[mt][1] - m_use);
+          l_run += pw[mt][0] + pw[mt][1];
+        }
+#pragma unroll
+        for (int gg = 0; gg < NVG; ++gg) {
+          const int bit0 = plan.vbit0[gg];
+          float(*cg)[4] = co + gg * MPG;
+          switch (plan.vbits[gg]) {
+            case 8: value_group_tiles<8, GV, MT, NVG>(svc, svm, vw, gg, qi, qr, swap, sel_lo, sel_hi, bit0, pw, zsum[gg], cg); break;
+            case 4: value_group_tiles<4, GV, MT, NVG>(svc, svm, vw, gg, qi, qr, swap, sel_lo, sel_hi, bit0, pw, zsum[gg], cg); break;
+            case 2: value_group_tiles<2, GV, MT, NVG>(svc, svm, vw, gg, qi, qr, swap, sel_lo, sel_hi, bit0, pw, zsum[gg], cg); break;
+            case 1: value_group_tiles<1, GV, MT, NVG>(svc, svm, vw, gg, qi, qr, swap, sel_lo, sel_hi, bit0, pw, zsum[gg], cg); break;
+            default: break;                  // a dropped group: no codes, (scale, zero) = 0
+          }
+        }
+      } else {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         {
@@ -565,6 +609,7 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarPlan plan, const __half
             }
           }
         }
+      }
       }
 
       // ---- release the stage: refill it with unit k + ring ----
