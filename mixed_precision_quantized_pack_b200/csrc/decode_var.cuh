@@ -497,22 +497,42 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarPlan plan, const __half
         kmb[s] = dsc.z;
       }
       float sc[MT][2];
+      if constexpr (MAP::kFixed) {
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        {
+        for (int mt = 0; mt < MT; ++mt) {
           float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
           for (int s = 0; s < kKSteps; ++s) {
             if (s >= nks) break;
-            {
-              const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kp[s] + 16 * mt * kw4);
-              const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kp[s] + (16 * mt + 8) * kw4);
-              ptx::mma_16816(cs, w0 & kma[s], w1 & kma[s], (w0 >> 8) & kmb[s], (w1 >> 8) & kmb[s], bq[s][0],
-                             bq[s][1]);
-            }
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kp[s] + 16 * mt * kw4);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kp[s] + (16 * mt + 8) * kw4);
+            ptx::mma_16816(cs, w0 & kma[s], w1 & kma[s], (w0 >> 8) & kmb[s], (w1 >> 8) & kmb[s], bq[s][0],
+                           bq[s][1]);
           }
           sc[mt][0] = fmaf(cs[0] + cs[1], alpha24, beta);
           sc[mt][1] = fmaf(cs[2] + cs[3], alpha24, beta);
+        }
+      } else {
+        // a run-time k-step count: the k-steps outside, the tiles inside (one branch per k-step
+        // and key group)
+        float cs[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) cs[mt][0] = cs[mt][1] = cs[mt][2] = cs[mt][3] = 0.0f;
+#pragma unroll
+        for (int s = 0; s < kKSteps; ++s) {
+          if (s >= nks) break;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kp[s] + 16 * mt * kw4);
+            const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kp[s] + (16 * mt + 8) * kw4);
+            ptx::mma_16816(cs[mt], w0 & kma[s], w1 & kma[s], (w0 >> 8) & kmb[s], (w1 >> 8) & kmb[s], bq[s][0],
+                           bq[s][1]);
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          sc[mt][0] = fmaf(cs[mt][0] + cs[mt][1], alpha24, beta);
+          sc[mt][1] = fmaf(cs[mt][2] + cs[mt][3], alpha24, beta);
         }
       }
       // retained tokens of this group are read from the fp16 list: mask them here
