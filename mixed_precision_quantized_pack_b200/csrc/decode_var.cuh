@@ -47,6 +47,8 @@ constexpr int kCouples = 4 * kKSteps;
 constexpr int kMaxRing = 8;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kLazyRescale = 8.0f;
+// Three CTAs per SM (168 registers): the build-time map instances spill at four, and the run-time
+// ones, which fit four, measured 3-6% faster at three.
 constexpr int kCtasPerSm = 3;
 constexpr int kSmemPerCta = 233472 / kCtasPerSm - 1024;
 constexpr int KST = kDK * 2 + 16;          // padded fp16 row strides of an fp16 stage (bytes)
@@ -219,14 +221,6 @@ struct RuntimeMap {
 using MapK3V2 = FixedMap<16, 64, 32, 0, 0, 32, 64, 32>;
 using MapK8K2 = FixedMap<32, 0, 96, 0, 0, 64, 64, 0>;
 
-// CTAs per SM: three (168 registers).  The build-time maps' folded code keeps more values live
-// and spills at four; the run-time-map instances fit four (128 registers) but measured 3-6% faster
-// at three.
-template <class MAP>
-constexpr int ctas_per_sm() { return kCtasPerSm; }
-template <class MAP>
-constexpr int smem_per_cta() { return 233472 / ctas_per_sm<MAP>() - 1024; }
-
 // p.V of one value group of width B over the MT tiles of a key group: per tile the (scale, zero)
 // of the lane's two tokens, the B operand p_t s_{t,g} split (hi, lo) and transposed, and the
 // group's MMAs; zsum accumulates sum_t p_t z_{t,g}.
@@ -249,7 +243,7 @@ __device__ __forceinline__ void value_group_tiles(const uint32_t* svc, const uin
 }
 
 template <int NREP, int GV, int GK, class MAP = RuntimeMap>
-__global__ void __launch_bounds__(kThreads, ctas_per_sm<MAP>())
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarPlan plan, const __half* __restrict__ q,
                   Partials part) {
   constexpr int NVG = kDV / GV;          // value groups per row
@@ -279,7 +273,7 @@ decode_var_kernel(Dims d, CacheBufs cb, DecodeWork w, VarPlan plan, const __half
   const bool quant = split < w.splits_q;
   const StageLayout L = var_stage_layout(d);
   const int stage_bytes = quant ? round128(L.bytes) : kRawStage;
-  int ring = (smem_per_cta<MAP>() - Smem::kStages) / stage_bytes;
+  int ring = (kSmemPerCta - Smem::kStages) / stage_bytes;
   ring = ring > kMaxRing ? kMaxRing : ring;
 
   if (threadIdx.x == 0) {
@@ -796,7 +790,7 @@ template <int NREP, int GV, int GK, class M = RuntimeMap>
 cudaError_t launch_var(const Dims& d, const CacheBufs& c, const DecodeWork& w, const VarPlan& vp,
                        const __half* q, const Partials& p, cudaStream_t s) {
   auto kern = decode_var_kernel<NREP, GV, GK, M>;
-  constexpr int smem = smem_per_cta<M>();
+  constexpr int smem = kSmemPerCta;
   static bool configured = false;
   if (!configured) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
