@@ -23,12 +23,17 @@
 //         the two halves of one register (token 2qi low, 2qi + 1 high) and masks in place give
 //         one register per channel.  Channels on M, tokens on K, B = p_t s_{t,g} split (hi, lo)
 //         and transposed by movmatrix; o_c = C 2^(24-p) + sum_t p_t z_{t,g}.  A group's width
-//         is a run-time value (a warp-uniform branch); dropped groups are skipped.
+//         is a run-time value (one warp-uniform branch per group and key group); dropped groups
+//         are skipped.
 // fp16    Retained tokens and the window: rows loaded with ldmatrix as they are.
+//
+// A map known at build time (FixedMap) gets an instance in which the k-step count, the row
+// strides and the value groups' widths and first bits are compile-time constants.
 //
 // Shape limits (other maps run on the generic kernel): d_k = d_v = 128, 1 or 4 query heads per
 // kv head, value groups of 16, 32, 64 or 128 channels, and at most 32 couples in a key row
-// (eight k-steps; a row of coded channels only ever needs that many).
+// (eight k-steps: every map whose key words each hold one width fits; a map whose words mix
+// widths can need more).
 #pragma once
 #include <string.h>
 
