@@ -146,6 +146,12 @@ WORKLOADS: Dict[str, Workload] = {
                           n_q_heads=32, n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=0,
                           v_bits=0, group_k=64, group_v=64, window=128, log_retain=1, appends=0,
                           seed=1009, k_widths=(8,) * 32 + (2,) * 96, v_widths=(4,) * 64 + (2,) * 64),
+    # a third width map, not built in: it runs through the run-time plan of the map (keys 64 x 4
+    # and 64 x 2 bits, values in groups of 32 channels at 4, 4, 2 and 2 bits)
+    "aatc32k-k4k2": _base(name="aatc-b32-32/8-32k-k4x64-k2x64-v4x64-v2x64-logretain", batch=32,
+                          n_q_heads=32, n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=0,
+                          v_bits=0, group_k=64, group_v=32, window=128, log_retain=1, appends=0,
+                          seed=1011, k_widths=(4,) * 64 + (2,) * 64, v_widths=(4,) * 64 + (2,) * 64),
     # the HeadQ case on a paged cache
     "headq-paged32k": _base(name="headq-paged-b32-32/8-32k-k2v2-r4q4-logretain", batch=32,
                             n_q_heads=32, n_kv_heads=8, d_k=128, d_v=128, context=32768, k_bits=2,

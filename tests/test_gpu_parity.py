@@ -678,3 +678,9 @@ def test_full_size_aatc_32k():
 def test_full_size_aatc_32k_second_map():
     assert tensor_kernel_built(W.WORKLOADS["aatc32k-k8k2"])
     sampled_full_size(W.WORKLOADS["aatc32k-k8k2"], rows=(0, 31))
+
+
+def test_full_size_aatc_32k_run_time_map():
+    """A map with no build-time instance: the run-time plan at full size."""
+    assert tensor_kernel_built(W.WORKLOADS["aatc32k-k4k2"])
+    sampled_full_size(W.WORKLOADS["aatc32k-k4k2"], rows=(0, 31))
