@@ -372,7 +372,31 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
     const float zc = meta_ok ? __half2float(blk[slot + per]) : 0.0f;
     const int shift = r * kb;
     const uint32_t mask = (1u << kb) - 1u;
+    auto residual = [&](int t, float x) {
+      const long long ki = static_cast<long long>((row0 + t) * words) + wd;
+      const uint32_t w = KVQ_IN_BOUNDS(d, kSiteSideCode, ki, quant_rows(d) * words) ? kcode[ki] : 0u;
+      const uint32_t code = (w >> shift) & mask;
+      const float kh = __fadd_rn(__fmul_rn(static_cast<float>(code), sc), zc);
+      e[t * es + c] = __fsub_rn(x, kh);
+    };
     int t = threadIdx.x >> ldk;
+    if (ROT || static_cast<long long>(g + 1) * gk <= src_rows) {
+      // the group's rows are contiguous in the source (a prefill): independent iterations, so
+      // that the loads of several tokens are in flight together
+#pragma unroll 8
+      for (int tt = t; tt < gk; tt += tstep) {
+        float x;
+        if constexpr (ROT) {
+          x = e[tt * es + c];
+        } else {
+          const long long si = static_cast<long long>((base + static_cast<long long>(g) * gk + tt) * dk) + c;
+          x = KVQ_IN_BOUNDS(d, kSiteSideSrc, si, static_cast<long long>(d.B) * hkv * src_rows * dk)
+                  ? __half2float(src[si]) : 0.0f;
+        }
+        residual(tt, x);
+      }
+      t = gk;
+    }
     int row = static_cast<int>((static_cast<long long>(g) * gk + t) % src_rows);   // source row of token t
     for (; t < gk; t += tstep) {
       float x;
@@ -383,11 +407,7 @@ __global__ void quantize_side_kernel(const __half* __restrict__ src, int src_row
         x = KVQ_IN_BOUNDS(d, kSiteSideSrc, si, static_cast<long long>(d.B) * hkv * src_rows * dk)
                 ? __half2float(src[si]) : 0.0f;
       }
-      const long long ki = static_cast<long long>((row0 + t) * words) + wd;
-      const uint32_t w = KVQ_IN_BOUNDS(d, kSiteSideCode, ki, quant_rows(d) * words) ? kcode[ki] : 0u;
-      const uint32_t code = (w >> shift) & mask;
-      const float kh = __fadd_rn(__fmul_rn(static_cast<float>(code), sc), zc);
-      e[t * es + c] = __fsub_rn(x, kh);
+      residual(t, x);
       row += tstep;
       while (row >= src_rows) row -= src_rows;
     }
