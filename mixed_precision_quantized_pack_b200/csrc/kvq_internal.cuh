@@ -129,6 +129,15 @@ __host__ __device__ inline size_t group_index(const Dims& d, const int* table, i
   if (d.paged) return static_cast<size_t>(table[b * d.max_groups + g]) * d.Hkv + h;
   return static_cast<size_t>(b * d.Hkv + h) * d.max_groups + g;
 }
+// The same from the flat row bh = b * Hkv + h: a division only for a paged cache.
+__host__ __device__ inline size_t group_row_bh(const Dims& d, const int* table, int bh, int g) {
+  if (d.paged) return group_row(d, table, bh / d.Hkv, bh % d.Hkv, g);
+  return static_cast<size_t>(bh) * d.lcap + static_cast<size_t>(g) * d.gk;
+}
+__host__ __device__ inline size_t group_index_bh(const Dims& d, const int* table, int bh, int g) {
+  if (d.paged) return group_index(d, table, bh / d.Hkv, bh % d.Hkv, g);
+  return static_cast<size_t>(bh) * d.max_groups + g;
+}
 
 // The rotation of one key or query row of d = 32 * M channels by a warp, lane l holding
 // channels l + 32 m in x[m]: x <- FWHT(sigma * x) * inv_c in fp32, butterflies of span
