@@ -1326,6 +1326,7 @@ cudaError_t launch_quantize_keys_t(const Dims& d, const __half* src, int src_row
     // spread over more chunks (measured 2.91 against 2.96 ms on the 32k rotated-key prefill)
     const int rs8 = d.gk >= 64 && rows < 8 ? 8 : rows;
     const int gpc8 = 256 / (cpr * d.gk / rs8);
+    if (gpc8 * d.dk > kKeyPrm || gpc8 * 2 * d.dk > kKeyBlk) return cudaErrorInvalidValue;
     auto staged = rs8 == 4 ? quantize_keys_staged_kernel<BITS, 4, ROT>
                 : rs8 == 8 ? quantize_keys_staged_kernel<BITS, 8, ROT> : quantize_keys_staged_kernel<BITS, 16, ROT>;
     const int sbytes = 2 * gpc8 * d.gk * d.dk * 2;
